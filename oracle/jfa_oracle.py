@@ -1,0 +1,379 @@
+"""fp64 CPU oracle for approximate-then-correct low-bit KV decode attention.
+
+TEST INFRASTRUCTURE ONLY.  This module is a plain, slow, obviously correct
+statement of what the decode step computes.  Only ``tests/``,
+``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline / reference legs
+may import it.  The CUDA library (``bit_kv_cache_jfa_b200``) never imports it
+and shares no code with it; the only shared module is ``workloads`` (seeded
+random inputs, no method arithmetic).
+
+What is computed, and where the pages say so:
+
+* The method (JetFire README, introduction): keep a low-bit KV cache on the
+  GPU, score every cached token approximately from it, pick the top-k tokens
+  and correct them with a high-precision copy ("approximate-then-correct").
+* Low-bit formats K3V2 and K4V4 (JetFire README, benchmark section).
+* Partition-wise asymmetric quantization x ~ s * x' + m, with m the
+  partition minimum and s the scale (HACK review, Eq. (4) and its context);
+  group size 64 with an FP16 zero point and scale (TailorKV review, "free
+  parameters": quantization bit size and group size).
+* The most recent tokens stay high-precision so that appending never
+  requantizes (HACK review: last partial block of V kept in FP16, Figure 8;
+  Jet-QSparse abstract: at most two BF16 pages per sequence and layer).
+* A dense scan scores the full key history; selected tokens get
+  high-precision value aggregation with FP32 accumulation (Jet-QSparse
+  abstract).
+* Affine identity (HACK review, Eq. (4)): a product against affinely
+  quantized data is an integer product plus row/column correction terms.
+
+Readings taken where the pages are silent (each is also listed in the
+design notes): softmax scale is a parameter (default 1/sqrt(d)); the tail
+holds the last 1..64 tokens and is always exact; key groups are 64 tokens
+per channel, value groups 32 channels per token; the zero point is the fp16
+rounding *down* of the group minimum and the scale the fp16 rounding *up* of
+(max - zero) / (2^b - 1); codes round half to even on an fp64 quotient; the
+per-(sequence, KV head) selection score is the max over the group's query
+heads; top-k order is (score descending, index ascending); exact and
+approximate parts are merged in log-sum-exp form.
+
+Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
+(hand-derived fixtures in ``tests/golden/``, closed forms, invariants and
+brute force); none is "parity unpinned".
+"""
+from __future__ import annotations
+
+import dataclasses
+
+import numpy as np
+
+KEY_GROUP = 64    # tokens per key group (one scale/zero per channel)
+VAL_GROUP = 32    # channels per value group (one scale/zero per token)
+TAIL_MAX = 64     # most recent tokens kept exact (bf16)
+
+
+# ---------------------------------------------------------------------------
+# Tail split
+# ---------------------------------------------------------------------------
+def split_point(n_ctx: int) -> int:
+    """Number of quantized tokens N_q for a sequence of n_ctx tokens.
+
+    Reading of the HACK review (Figure 8: the last partial block stays
+    unquantized): tokens are appended to a bf16 tail; when a token arrives at
+    a full tail of 64, the 64 tail tokens are first quantized as one key
+    group.  Hence the tail always holds T = N - N_q in [1, 64] tokens.
+    """
+    if n_ctx <= 0:
+        return 0
+    return KEY_GROUP * ((n_ctx - 1) // KEY_GROUP)
+
+
+# ---------------------------------------------------------------------------
+# fp16 directed rounding (zero point rounds down, scale rounds up)
+# ---------------------------------------------------------------------------
+def fp16_round_down(x) -> np.ndarray:
+    """Largest fp16 value <= x (elementwise; x in fp64)."""
+    x = np.asarray(x, dtype=np.float64)
+    with np.errstate(over="ignore"):
+        h = x.astype(np.float16)
+    above = h.astype(np.float64) > x
+    return np.where(above, np.nextafter(h, np.float16(-np.inf)), h).astype(np.float16)
+
+
+def fp16_round_up(x) -> np.ndarray:
+    """Smallest fp16 value >= x (elementwise; x in fp64)."""
+    x = np.asarray(x, dtype=np.float64)
+    with np.errstate(over="ignore"):
+        h = x.astype(np.float16)
+    below = h.astype(np.float64) < x
+    return np.where(below, np.nextafter(h, np.float16(np.inf)), h).astype(np.float16)
+
+
+# ---------------------------------------------------------------------------
+# Group-wise asymmetric quantization (HACK review Eq. (4) context; TailorKV
+# review: group size 64, FP16 zero point and scale)
+# ---------------------------------------------------------------------------
+def quantize_last_axis(x, bits: int):
+    """Quantize every row of ``x`` (fp64 view of bf16 data) as one group.
+
+    zero  = fp16 round-down of min(row)
+    scale = fp16 round-up of (max(row) - zero) / (2^bits - 1)   [fp64 quotient]
+    code  = clip(rint((x - zero) / scale), 0, 2^bits - 1)       [fp64 quotient,
+                                                                 half to even]
+    A group with scale 0 (max == zero) gets code 0 everywhere.
+    Returns (codes uint8 like x, scale fp16 [rows], zero fp16 [rows]).
+    """
+    x = np.asarray(x, dtype=np.float64)
+    levels = (1 << bits) - 1
+    mn = x.min(axis=-1)
+    mx = x.max(axis=-1)
+    zero = fp16_round_down(mn)
+    scale = fp16_round_up((mx - zero.astype(np.float64)) / levels)
+    s = scale.astype(np.float64)[..., None]
+    z = zero.astype(np.float64)[..., None]
+    with np.errstate(divide="ignore", invalid="ignore"):
+        q = np.rint((x - z) / s)
+    q = np.where(s == 0.0, 0.0, q)
+    codes = np.clip(q, 0, levels).astype(np.uint8)
+    return codes, scale, zero
+
+
+def dequantize(codes, scale, zero) -> np.ndarray:
+    """x_hat = scale * code + zero (fp64); scale/zero broadcast over the group."""
+    return scale.astype(np.float64)[..., None] * codes.astype(np.float64) \
+        + zero.astype(np.float64)[..., None]
+
+
+def quantize_keys(k, bits: int):
+    """Keys [..., N_q, d]: one group per (64-token block, channel).
+
+    Returns codes uint8 [..., N_q, d], scale/zero fp16 [..., N_q/64, d].
+    """
+    k = np.asarray(k, dtype=np.float64)
+    *lead, nq, d = k.shape
+    assert nq % KEY_GROUP == 0
+    ng = nq // KEY_GROUP
+    blocks = k.reshape(*lead, ng, KEY_GROUP, d)
+    per_channel = np.swapaxes(blocks, -1, -2)          # [..., ng, d, 64]
+    codes, scale, zero = quantize_last_axis(per_channel, bits)
+    codes = np.swapaxes(codes, -1, -2).reshape(*lead, nq, d)
+    return codes, scale, zero
+
+
+def dequantize_keys(codes, scale, zero) -> np.ndarray:
+    *lead, nq, d = codes.shape
+    ng = nq // KEY_GROUP
+    c = np.swapaxes(codes.reshape(*lead, ng, KEY_GROUP, d), -1, -2)   # [..., ng, d, 64]
+    x = dequantize(c, scale, zero)
+    return np.swapaxes(x, -1, -2).reshape(*lead, nq, d)
+
+
+def quantize_values(v, bits: int):
+    """Values [..., N_q, d]: one group per (token, 32-channel block).
+
+    Returns codes uint8 [..., N_q, d], scale/zero fp16 [..., N_q, d/32].
+    """
+    v = np.asarray(v, dtype=np.float64)
+    *lead, nq, d = v.shape
+    groups = v.reshape(*lead, nq, d // VAL_GROUP, VAL_GROUP)
+    codes, scale, zero = quantize_last_axis(groups, bits)
+    return codes.reshape(*lead, nq, d), scale, zero
+
+
+def dequantize_values(codes, scale, zero) -> np.ndarray:
+    *lead, nq, d = codes.shape
+    c = codes.reshape(*lead, nq, d // VAL_GROUP, VAL_GROUP)
+    return dequantize(c, scale, zero).reshape(*lead, nq, d)
+
+
+@dataclasses.dataclass
+class PackedCache:
+    """Quantized state of a cache after n_ctx tokens (per sequence, uniform)."""
+    n_ctx: int
+    n_quant: int
+    key_bits: int
+    val_bits: int
+    k_codes: np.ndarray   # uint8 [B, H_kv, N_q, d]
+    k_scale: np.ndarray   # fp16  [B, H_kv, N_q/64, d]
+    k_zero: np.ndarray    # fp16  [B, H_kv, N_q/64, d]
+    v_codes: np.ndarray   # uint8 [B, H_kv, N_q, d]
+    v_scale: np.ndarray   # fp16  [B, H_kv, N_q, d/32]
+    v_zero: np.ndarray    # fp16  [B, H_kv, N_q, d/32]
+    tail_k: np.ndarray    # fp64 view of bf16 [B, H_kv, T, d]
+    tail_v: np.ndarray
+
+    def k_hat(self) -> np.ndarray:
+        return dequantize_keys(self.k_codes, self.k_scale, self.k_zero)
+
+    def v_hat(self) -> np.ndarray:
+        return dequantize_values(self.v_codes, self.v_scale, self.v_zero)
+
+
+def pack_cache(k, v, n_ctx: int, key_bits: int, val_bits: int) -> PackedCache:
+    """Quantize the first N_q tokens of K/V [B, H_kv, >=n_ctx, d]; keep the
+    rest as the exact tail.  Codes of a group depend only on that group's 64
+    tokens, so the state is a function of n_ctx alone: appending tokens never
+    changes codes already written (HACK review: no requantization)."""
+    k = np.asarray(k, dtype=np.float64)[:, :, :n_ctx]
+    v = np.asarray(v, dtype=np.float64)[:, :, :n_ctx]
+    nq = split_point(n_ctx)
+    kc, ks, kz = quantize_keys(k[:, :, :nq], key_bits)
+    vc, vs, vz = quantize_values(v[:, :, :nq], val_bits)
+    return PackedCache(n_ctx, nq, key_bits, val_bits, kc, ks, kz, vc, vs, vz,
+                       k[:, :, nq:].copy(), v[:, :, nq:].copy())
+
+
+# ---------------------------------------------------------------------------
+# Approximate scoring
+# ---------------------------------------------------------------------------
+def approx_logits(q, cache: PackedCache, scale: float) -> np.ndarray:
+    """s_hat[b, h, t] = scale * q[b, h] . x_hat_K[b, h // G, t] for t < N_q,
+    computed by dequantize-then-multiply in fp64.  Returns [B, H, N_q]."""
+    q = np.asarray(q, dtype=np.float64)
+    b, h, d = q.shape
+    hkv = cache.k_codes.shape[1]
+    g = h // hkv
+    kh = cache.k_hat()                                  # [B, H_kv, N_q, d]
+    qg = q.reshape(b, hkv, g, d)
+    s = np.einsum("bkgd,bktd->bkgt", qg, kh)
+    return scale * s.reshape(b, h, -1)
+
+
+def affine_logits(q, cache: PackedCache, scale: float) -> np.ndarray:
+    """The same logits through the affine identity (HACK review, Eq. (4)),
+    specialised to an unquantized query:  q . (s * k' + m)
+    = sum_c (q_c s_c) k'_c + sum_c q_c m_c, per key group."""
+    q = np.asarray(q, dtype=np.float64)
+    b, h, d = q.shape
+    hkv = cache.k_codes.shape[1]
+    g = h // hkv
+    ng = cache.n_quant // KEY_GROUP
+    qg = q.reshape(b, hkv, g, d)
+    s = cache.k_scale.astype(np.float64)                # [B, H_kv, ng, d]
+    m = cache.k_zero.astype(np.float64)
+    codes = cache.k_codes.astype(np.float64).reshape(b, hkv, ng, KEY_GROUP, d)
+    q_tilde = qg[:, :, None, :, :] * s[:, :, :, None, :]      # [B,H_kv,ng,G,d]
+    integer_part = np.einsum("bkngd,bkntd->bkngt", q_tilde, codes)
+    correction = np.einsum("bkgd,bknd->bkng", qg, m)[..., None]
+    out = (integer_part + correction)                         # [B,H_kv,ng,G,64]
+    out = np.moveaxis(out, 3, 2).reshape(b, hkv, g, ng * KEY_GROUP)
+    return scale * out.reshape(b, h, -1)
+
+
+def selection_scores(s_hat, kv_heads: int) -> np.ndarray:
+    """Per-(sequence, KV head) selection score: max over the G query heads
+    that share the KV head.  [B, H, N_q] -> [B, H_kv, N_q]."""
+    s_hat = np.asarray(s_hat)
+    b, h, n = s_hat.shape
+    return s_hat.reshape(b, kv_heads, h // kv_heads, n).max(axis=2)
+
+
+# ---------------------------------------------------------------------------
+# Top-k selection
+# ---------------------------------------------------------------------------
+def topk_indices(scores, k: int) -> np.ndarray:
+    """k largest scores per row, order (score descending, index ascending);
+    the chosen indices are returned sorted ascending, padded with -1 when
+    k > row length.  scores [..., N] -> int32 [..., k]."""
+    scores = np.asarray(scores)
+    *lead, n = scores.shape
+    flat = scores.reshape(-1, n)
+    out = np.full((flat.shape[0], k), -1, dtype=np.int32)
+    keff = min(k, n)
+    idx = np.arange(n)
+    for r in range(flat.shape[0]):
+        order = np.lexsort((idx, -flat[r]))       # primary: -score, then index
+        out[r, :keff] = np.sort(order[:keff])
+    return out.reshape(*lead, k)
+
+
+# ---------------------------------------------------------------------------
+# Softmax partials and log-sum-exp merge
+# ---------------------------------------------------------------------------
+@dataclasses.dataclass
+class Partial:
+    """Unnormalised softmax state over a token set: m = max logit,
+    l = sum exp(s - m), acc = sum exp(s - m) * v."""
+    m: float
+    l: float
+    acc: np.ndarray
+
+    @staticmethod
+    def empty(d: int) -> "Partial":
+        return Partial(-np.inf, 0.0, np.zeros(d))
+
+
+def softmax_partial(logits, values) -> Partial:
+    logits = np.asarray(logits, dtype=np.float64)
+    values = np.asarray(values, dtype=np.float64)
+    if logits.size == 0:
+        return Partial.empty(values.shape[-1])
+    m = logits.max()
+    w = np.exp(logits - m)
+    return Partial(float(m), float(w.sum()), w @ values)
+
+
+def merge(a: Partial, b: Partial) -> Partial:
+    """Log-sum-exp merge of two disjoint partials."""
+    m = max(a.m, b.m)
+    if m == -np.inf:
+        return Partial(m, 0.0, a.acc + b.acc)
+    wa = np.exp(a.m - m) if a.m > -np.inf else 0.0
+    wb = np.exp(b.m - m) if b.m > -np.inf else 0.0
+    return Partial(m, a.l * wa + b.l * wb, a.acc * wa + b.acc * wb)
+
+
+def finish(p: Partial) -> np.ndarray:
+    return p.acc / p.l
+
+
+# ---------------------------------------------------------------------------
+# The whole decode step
+# ---------------------------------------------------------------------------
+@dataclasses.dataclass
+class StepResult:
+    out: np.ndarray          # [B, H, d] fp64
+    s_hat: np.ndarray        # [B, H, N_q]
+    select: np.ndarray       # [B, H_kv, N_q]
+    idx: np.ndarray          # [B, H_kv, k] int32
+    approx_all: list         # [B][H] Partial over all N_q quantized tokens
+
+
+def decode_step(q, k_exact, v_exact, cache: PackedCache, k: int, scale: float,
+                idx=None) -> StepResult:
+    """One decode step for every sequence and query head.
+
+    1. approximate logits s_hat over the N_q quantized tokens;
+    2. selection score per (sequence, KV head) and its top-k (unless ``idx``
+       is given, in which case that index set is used as the exact set);
+    3. exact part: logits from the bf16 keys of the top-k tokens and the
+       tail, aggregated with bf16 values;
+    4. approximate remainder: the other quantized tokens with dequantized
+       keys and values;
+    5. log-sum-exp merge of the two, normalised.
+    ``k_exact``/``v_exact`` [B, H_kv, >=N, d] are the high-precision copies.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    b, h, d = q.shape
+    hkv = cache.k_codes.shape[1]
+    g = h // hkv
+    n, nq = cache.n_ctx, cache.n_quant
+    ke = np.asarray(k_exact, dtype=np.float64)
+    ve = np.asarray(v_exact, dtype=np.float64)
+    s_hat = approx_logits(q, cache, scale)
+    sel = selection_scores(s_hat, hkv)
+    if idx is None:
+        idx = topk_indices(sel, k)
+    idx = np.asarray(idx)
+    vh = cache.v_hat()
+    out = np.zeros((b, h, d))
+    approx_all = [[None] * h for _ in range(b)]
+    for bi in range(b):
+        for kv in range(hkv):
+            chosen = idx[bi, kv]
+            chosen = np.unique(chosen[chosen >= 0])
+            exact_set = np.concatenate([chosen, np.arange(nq, n)]).astype(np.int64)
+            rest = np.setdiff1d(np.arange(nq), chosen)
+            for j in range(g):
+                hq = kv * g + j
+                exact_logits = scale * (ke[bi, kv, exact_set] @ q[bi, hq])
+                pe = softmax_partial(exact_logits, ve[bi, kv, exact_set])
+                pa = softmax_partial(s_hat[bi, hq, rest], vh[bi, kv, rest])
+                out[bi, hq] = finish(merge(pe, pa))
+                approx_all[bi][hq] = softmax_partial(s_hat[bi, hq], vh[bi, kv])
+    return StepResult(out, s_hat, sel, idx, approx_all)
+
+
+def exact_attention(q, k_exact, v_exact, n_ctx: int, scale: float) -> np.ndarray:
+    """Plain softmax attention over all n_ctx bf16 tokens (GQA), fp64."""
+    q = np.asarray(q, dtype=np.float64)
+    b, h, d = q.shape
+    ke = np.asarray(k_exact, dtype=np.float64)[:, :, :n_ctx]
+    ve = np.asarray(v_exact, dtype=np.float64)[:, :, :n_ctx]
+    hkv = ke.shape[1]
+    g = h // hkv
+    out = np.zeros((b, h, d))
+    for bi in range(b):
+        for hq in range(h):
+            p = softmax_partial(scale * (ke[bi, hq // g] @ q[bi, hq]), ve[bi, hq // g])
+            out[bi, hq] = finish(p)
+    return out

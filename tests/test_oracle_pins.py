@@ -1,0 +1,322 @@
+"""Pins for the fp64 CPU oracle against facts fixed by the pages and by
+mathematics (not against the oracle itself): hand-derived fixtures, closed
+forms, invariants, library routines for special cases, and brute force."""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle.jfa_oracle as O
+import workloads as W
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _cases(fname):
+    cases, cur = [], None
+    with open(os.path.join(GOLDEN, fname)) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            key, _, val = line.partition(" ")
+            if key == "case":
+                cur = {"name": val}
+                cases.append(cur)
+            else:
+                cur[key] = val.split()
+    return cases
+
+
+def _bf16(x):
+    return torch.as_tensor(x, dtype=torch.float32).to(torch.bfloat16).double().numpy()
+
+
+# --------------------------------------------------------------------------
+# quantization
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("case", _cases("quantization_cases.txt"), ids=lambda c: c["name"])
+def test_quantization_golden(case):
+    bits = int(case["bits"][0])
+    x = np.array([float(v) for v in case["x"]])
+    codes, scale, zero = O.quantize_last_axis(x[None, :], bits)
+    assert codes[0].tolist() == [int(c) for c in case["codes"]]
+    assert int(zero.view(np.uint16)[0]) == int(case["zero_bits"][0], 16)
+    assert int(scale.view(np.uint16)[0]) == int(case["scale_bits"][0], 16)
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_quantization_error_bound(bits):
+    rng = np.random.default_rng(bits)
+    x = _bf16(rng.standard_normal((500, 64)) * rng.choice([0.01, 1, 10, 300], (500, 1)))
+    codes, scale, zero = O.quantize_last_axis(x, bits)
+    xh = O.dequantize(codes, scale, zero)
+    s = scale.astype(np.float64)[:, None]
+    assert codes.max() <= (1 << bits) - 1
+    # exact invariant of round-down zero / round-up scale / nearest code
+    assert np.all(np.abs(x - xh) <= s / 2 * (1 + 1e-12))
+    # the group minimum maps to code 0, the maximum to the top code
+    assert np.all(codes[np.arange(500), x.argmin(1)] == 0)
+    assert np.all(codes[np.arange(500), x.argmax(1)] == (1 << bits) - 1)
+    # zero <= min and zero + levels * scale >= max
+    assert np.all(zero.astype(np.float64) <= x.min(1))
+    assert np.all(zero.astype(np.float64) + ((1 << bits) - 1) * scale.astype(np.float64)
+                  >= x.max(1))
+
+
+def test_round_to_nearest_even_brute_force():
+    # build x = zero + (n + 1/2) * scale exactly: ties must go to even n
+    bits = 4
+    scale, zero = 0.5, -1.0
+    n = np.arange(15)
+    x = zero + (n + 0.5) * scale
+    x = np.concatenate([[zero, zero + 15 * scale], x])
+    codes, s, z = O.quantize_last_axis(x[None], bits)
+    assert float(s[0]) == scale and float(z[0]) == zero
+    expect = [0, 15] + [int(k) if k % 2 == 0 else int(k) + 1 for k in n]
+    assert codes[0].tolist() == expect
+
+
+def test_key_groups_run_along_tokens_per_channel():
+    # channel c is constant c + g/2 inside key group g: every key group has
+    # scale 0 and zero = that constant only if groups are (64 tokens, 1 channel)
+    ng, d = 3, 128
+    t = np.arange(64 * ng)[:, None]
+    c = np.arange(d)[None, :]
+    k = (c + 0.5 * (t // 64)).astype(np.float64)[None, None]
+    codes, scale, zero = O.quantize_keys(k, 3)
+    assert scale.shape == (1, 1, ng, d)
+    assert np.all(scale == 0) and np.all(codes == 0)
+    assert np.array_equal(zero[0, 0].astype(np.float64),
+                          np.arange(d)[None, :] + 0.5 * np.arange(ng)[:, None])
+
+
+def test_value_groups_run_along_channels_per_token():
+    n, d = 64, 128
+    t = np.arange(n)[:, None]
+    c = np.arange(d)[None, :]
+    v = (t + 0.25 * (c // 32)).astype(np.float64)[None, None]
+    codes, scale, zero = O.quantize_values(v, 2)
+    assert scale.shape == (1, 1, n, 4)
+    assert np.all(scale == 0) and np.all(codes == 0)
+    assert np.array_equal(zero[0, 0].astype(np.float64),
+                          np.arange(n)[:, None] + 0.25 * np.arange(4)[None, :])
+
+
+def test_grid_data_reconstructs_exactly():
+    rng = np.random.default_rng(7)
+    for bits in (2, 3, 4):
+        lv = (1 << bits) - 1
+        codes = rng.integers(0, lv + 1, (64, 128))
+        codes[0], codes[1] = 0, lv           # min and max present in every channel
+        k = -0.75 + 0.125 * codes.astype(np.float64)
+        kc, ks, kz = O.quantize_keys(k[None, None], bits)
+        assert np.array_equal(kc[0, 0], codes)
+        assert np.all(ks == np.float16(0.125)) and np.all(kz == np.float16(-0.75))
+        assert np.array_equal(O.dequantize_keys(kc, ks, kz)[0, 0], k)
+
+
+def test_split_point_closed_form():
+    assert [O.split_point(n) for n in (0, 1, 63, 64, 65, 128, 129, 4096)] == \
+        [0, 0, 0, 0, 64, 64, 128, 4032]
+    for n in range(1, 400):
+        t = n - O.split_point(n)
+        assert 1 <= t <= 64 and O.split_point(n) % 64 == 0
+
+
+# --------------------------------------------------------------------------
+# scoring: affine identity (HACK review, Eq. (4)) and selection
+# --------------------------------------------------------------------------
+def _small(ctx=300, heads=4, kv=2, kb=4, vb=4, planted=4, seed=11, lognormal=False):
+    w = W.Workload("t", batch=2, heads=heads, kv_heads=kv, ctx=ctx, key_bits=kb,
+                   val_bits=vb, topk=16, planted=planted, seed=seed,
+                   value_lognormal=lognormal)
+    q = W.gen_q(w)
+    k, v = W.gen_kv(w, q)
+    cache = O.pack_cache(k.double().numpy(), v.double().numpy(), ctx, kb, vb)
+    return w, q.double().numpy(), k.double().numpy(), v.double().numpy(), cache
+
+
+@pytest.mark.parametrize("kb,vb", [(3, 2), (4, 4)])
+def test_affine_identity_equals_dequantize_then_multiply(kb, vb):
+    w, q, k, v, cache = _small(kb=kb, vb=vb)
+    a = O.approx_logits(q, cache, 0.1)
+    b = O.affine_logits(q, cache, 0.1)
+    assert np.allclose(a, b, rtol=1e-12, atol=1e-12)
+
+
+def test_selection_is_max_over_group_heads():
+    w, q, k, v, cache = _small(heads=8, kv=2)
+    s = O.approx_logits(q, cache, 0.09)
+    sel = O.selection_scores(s, 2)
+    for b in range(2):
+        for h in range(2):
+            for t in (0, 5, 100, 255):
+                assert sel[b, h, t] == max(s[b, h * 4 + j, t] for j in range(4))
+
+
+# --------------------------------------------------------------------------
+# top-k
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("case", _cases("topk_cases.txt"), ids=lambda c: c["name"])
+def test_topk_golden(case):
+    s = np.array([float(x) for x in case["scores"]])
+    k = int(case["k"][0])
+    got = O.topk_indices(s[None], k)[0].tolist()
+    assert got == [int(x) for x in case.get("idx", [])]
+
+
+def test_topk_brute_force_with_ties():
+    rng = np.random.default_rng(3)
+    for trial in range(50):
+        n = int(rng.integers(1, 200))
+        k = int(rng.integers(0, 220))
+        s = rng.integers(-5, 5, n).astype(np.float64) * 0.5   # many ties
+        ref = sorted(range(n), key=lambda i: (-s[i], i))[:k]
+        ref = sorted(ref) + [-1] * max(0, k - n)
+        assert O.topk_indices(s[None], k)[0].tolist() == ref
+
+
+# --------------------------------------------------------------------------
+# softmax partials and merge
+# --------------------------------------------------------------------------
+def test_split_and_merge_equals_unsplit():
+    rng = np.random.default_rng(5)
+    s = rng.standard_normal(300) * 4
+    v = rng.standard_normal((300, 16))
+    full = O.softmax_partial(s, v)
+    perm = rng.permutation(300)
+    a = O.softmax_partial(s[perm[:77]], v[perm[:77]])
+    b = O.softmax_partial(s[perm[77:]], v[perm[77:]])
+    m = O.merge(a, b)
+    assert math.isclose(m.m, full.m)
+    assert np.allclose(O.finish(m), O.finish(full), rtol=1e-13, atol=1e-13)
+    # softmax(s) @ v by the library
+    ref = torch.softmax(torch.tensor(s), 0) @ torch.tensor(v)
+    assert np.allclose(O.finish(full), ref.numpy(), rtol=1e-12, atol=1e-12)
+    e = O.merge(O.Partial.empty(16), a)
+    assert np.allclose(O.finish(e), O.finish(a))
+
+
+# --------------------------------------------------------------------------
+# whole step: special cases that reduce to plain attention
+# --------------------------------------------------------------------------
+def _torch_attention(q, keys, vals, scale):
+    q, keys, vals = map(torch.tensor, (q, keys, vals))
+    return (torch.softmax(scale * keys @ q, dim=0) @ vals).numpy()
+
+
+@pytest.mark.parametrize("kb,vb", [(3, 2), (4, 4)])
+def test_k_at_least_nq_is_exact_attention(kb, vb):
+    w, q, k, v, cache = _small(kb=kb, vb=vb)
+    scale = 1 / math.sqrt(128)
+    res = O.decode_step(q, k, v, cache, cache.n_quant + 5, scale)
+    for b in range(2):
+        for h in range(4):
+            ref = _torch_attention(q[b, h], k[b, h // 2], v[b, h // 2], scale)
+            assert np.allclose(res.out[b, h], ref, rtol=1e-11, atol=1e-12)
+
+
+@pytest.mark.parametrize("kb,vb", [(3, 2), (4, 4)])
+def test_k_zero_is_attention_over_dequantized_plus_exact_tail(kb, vb):
+    w, q, k, v, cache = _small(kb=kb, vb=vb, lognormal=True)
+    scale = 0.07
+    res = O.decode_step(q, k, v, cache, 0, scale)
+    kh, vh = cache.k_hat(), cache.v_hat()
+    nq = cache.n_quant
+    for b in range(2):
+        for h in range(4):
+            keys = np.concatenate([kh[b, h // 2], k[b, h // 2, nq:]])
+            vals = np.concatenate([vh[b, h // 2], v[b, h // 2, nq:]])
+            ref = _torch_attention(q[b, h], keys, vals, scale)
+            assert np.allclose(res.out[b, h], ref, rtol=1e-11, atol=1e-12)
+
+
+def test_given_index_set_matches_hand_mixture():
+    # with idx given, token t in idx uses bf16 K/V, others use x_hat; check
+    # against a torch softmax over the mixed key/value matrix
+    w, q, k, v, cache = _small()
+    scale = 0.1
+    nq = cache.n_quant
+    rng = np.random.default_rng(1)
+    idx = np.full((2, 2, 16), -1, dtype=np.int32)
+    for b in range(2):
+        for h in range(2):
+            idx[b, h, :10] = np.sort(rng.choice(nq, 10, replace=False))
+    res = O.decode_step(q, k, v, cache, 16, scale, idx=idx)
+    kh, vh = cache.k_hat(), cache.v_hat()
+    for b in range(2):
+        for hq in range(4):
+            h = hq // 2
+            keys, vals = kh[b, h].copy(), vh[b, h].copy()
+            sel = idx[b, h][idx[b, h] >= 0]
+            keys[sel], vals[sel] = k[b, h, sel], v[b, h, sel]
+            keys = np.concatenate([keys, k[b, h, nq:]])
+            vals = np.concatenate([vals, v[b, h, nq:]])
+            ref = _torch_attention(q[b, hq], keys, vals, scale)
+            assert np.allclose(res.out[b, hq], ref, rtol=1e-11, atol=1e-12)
+
+
+def test_output_is_convex_combination_of_value_rows():
+    w, q, k, v, cache = _small(kb=3, vb=2)
+    res = O.decode_step(q, k, v, cache, 16, 1 / math.sqrt(128))
+    vh = cache.v_hat()
+    nq = cache.n_quant
+    for b in range(2):
+        for hq in range(4):
+            h = hq // 2
+            sel = res.idx[b, h][res.idx[b, h] >= 0]
+            rest = np.setdiff1d(np.arange(nq), sel)
+            rows = np.concatenate([v[b, h, sel], v[b, h, nq:], vh[b, h, rest]])
+            o = res.out[b, hq]
+            assert np.all(o <= rows.max(0) + 1e-12) and np.all(o >= rows.min(0) - 1e-12)
+
+
+def test_appending_never_changes_written_codes():
+    w, q, k, v, _ = _small(ctx=400, kb=3, vb=2)
+    prev = None
+    for n in (1, 64, 65, 130, 200, 256, 257, 400):
+        c = O.pack_cache(k, v, n, 3, 2)
+        assert c.tail_k.shape[2] == n - c.n_quant
+        assert np.array_equal(c.tail_k, k[:, :, c.n_quant:n])
+        if prev is not None:
+            nq = prev.n_quant
+            assert np.array_equal(c.k_codes[:, :, :nq], prev.k_codes)
+            assert np.array_equal(c.k_scale[:, :, :nq // 64], prev.k_scale)
+            assert np.array_equal(c.v_codes[:, :, :nq], prev.v_codes)
+            assert np.array_equal(c.v_zero[:, :, :nq], prev.v_zero)
+        prev = c
+
+
+def test_planted_tokens_are_selected_in_tiny_workload():
+    w = W.WORKLOADS["tiny_k4v4_4k"]
+    q = W.gen_q(w)
+    k, v = W.gen_kv(w, q)
+    cache = O.pack_cache(k.double().numpy(), v.double().numpy(), w.ctx, 4, 4)
+    res = O.decode_step(q.double().numpy(), k.double().numpy(), v.double().numpy(),
+                        cache, w.topk, W.default_scale(w))
+    pos = set(W.planted_positions(w, 0).tolist())
+    for h in range(w.kv_heads):
+        assert pos <= set(res.idx[0, h].tolist())
+
+
+# --------------------------------------------------------------------------
+# the pins above catch plausible oracle mistakes (planted on the CPU)
+# --------------------------------------------------------------------------
+def test_pins_reject_round_to_nearest_scale(monkeypatch):
+    monkeypatch.setattr(O, "fp16_round_up", lambda x: np.asarray(x).astype(np.float16))
+    case = [c for c in _cases("quantization_cases.txt") if c["name"] == "round_up_scale"][0]
+    with pytest.raises(AssertionError):
+        test_quantization_golden(case)
+
+
+def test_pins_reject_wrong_merge_sign(monkeypatch):
+    def bad_merge(a, b):
+        m = max(a.m, b.m)
+        wa, wb = np.exp(m - a.m), np.exp(m - b.m)
+        return O.Partial(m, a.l * wa + b.l * wb, a.acc * wa + b.acc * wb)
+    monkeypatch.setattr(O, "merge", bad_merge)
+    with pytest.raises(AssertionError):
+        test_k_zero_is_attention_over_dequantized_plus_exact_tail(4, 4)
