@@ -1,0 +1,115 @@
+"""B200-native approximate-then-correct low-bit KV decode attention.
+
+A thin Python layer over ``libjfa.so`` (C ABI in ``include/jfa.h``).  Torch
+provides device memory and streams; every step of the decode path runs in
+the library's sm_100a kernels:
+
+    cache = KVCache(batch, heads, kv_heads, capacity, key_bits=3, val_bits=2)
+    ws = Workspace(cache, max_topk=256)
+    cache.append(k_new, v_new, ws)              # jfa_pack_kv
+    out, idx = decode_step(cache, q, 256, k_exact, v_exact, ws)
+"""
+from __future__ import annotations
+
+import math
+
+from . import _lib
+from ._lib import (  # noqa: F401  (re-exported C ABI names)
+    Cache, CacheLayout, Geom, JfaError, WorkspaceLayout, check, jfa_cache_layout_get,
+    jfa_check_error, jfa_clear_error, jfa_correct_merge, jfa_decode_scores, jfa_decode_step,
+    jfa_decode_step_launches, jfa_pack_kv, jfa_topk, jfa_unpack_record,
+    jfa_workspace_layout_get, load)
+
+__all__ = ["KVCache", "Workspace", "decode_step", "JfaError", "load"]
+
+
+def _torch():
+    import torch
+    return torch
+
+
+class KVCache:
+    """One layer's quantized KV cache (device buffers owned by torch)."""
+
+    def __init__(self, batch: int, num_heads: int, num_kv_heads: int, capacity: int,
+                 key_bits: int = 3, val_bits: int = 2, device="cuda", head_dim: int = 128):
+        torch = _torch()
+        self.batch, self.num_heads, self.num_kv_heads = batch, num_heads, num_kv_heads
+        self.capacity, self.key_bits, self.val_bits = capacity, key_bits, val_bits
+        self.head_dim = head_dim
+        self.n_ctx = 0
+        self.layout = jfa_cache_layout_get(self.geom())
+        self.groups = torch.empty(self.layout.groups_bytes, dtype=torch.uint8, device=device)
+        shape = (batch, num_kv_heads, _lib.TAIL_MAX, head_dim)
+        self.tail_k = torch.zeros(shape, dtype=torch.bfloat16, device=device)
+        self.tail_v = torch.zeros(shape, dtype=torch.bfloat16, device=device)
+
+    def geom(self, n_ctx: int | None = None) -> Geom:
+        return Geom(self.batch, self.num_heads, self.num_kv_heads, self.head_dim, self.capacity,
+                    self.key_bits, self.val_bits, self.n_ctx if n_ctx is None else n_ctx)
+
+    def struct(self) -> Cache:
+        return Cache(self.groups.data_ptr(), self.tail_k.data_ptr(), self.tail_v.data_ptr())
+
+    @property
+    def n_quant(self) -> int:
+        return 0 if self.n_ctx <= 0 else 64 * ((self.n_ctx - 1) // 64)
+
+    def append(self, k_new, v_new, ws: "Workspace", stream=None) -> None:
+        """Append bf16 [B, H_kv, n, 128] keys/values (contiguous, on device)."""
+        n = k_new.shape[2]
+        check(jfa_pack_kv(self.geom(), self.struct(), k_new, v_new, n, ws.buf, stream),
+              "jfa_pack_kv")
+        self.n_ctx += n
+
+    def record(self, b: int, h: int, g: int):
+        """Host bytes of the packed record of (sequence b, KV head h, group g)."""
+        rb = self.layout.record_bytes
+        seg = b * self.num_kv_heads + h
+        off = (seg * (self.capacity // 64) + g) * rb
+        return self.groups[off:off + rb].cpu().numpy().tobytes()
+
+
+class Workspace:
+    """Scratch of the decode step for a cache geometry and a maximum k."""
+
+    def __init__(self, cache: KVCache, max_topk: int, device="cuda"):
+        torch = _torch()
+        self.layout = jfa_workspace_layout_get(cache.geom(), max_topk)
+        self.buf = torch.zeros(self.layout.total_bytes, dtype=torch.uint8, device=device)
+        self.max_topk = max_topk
+
+    def scores(self, cache: KVCache):
+        """View of the selection scores S: fp32 [B, H_kv, capacity]."""
+        torch = _torch()
+        n = cache.batch * cache.num_kv_heads * cache.capacity
+        v = self.buf[self.layout.off_scores:self.layout.off_scores + 4 * n].view(torch.float32)
+        return v.view(cache.batch, cache.num_kv_heads, cache.capacity)
+
+    def error_flag(self, cache: KVCache, stream=None) -> int:
+        return jfa_check_error(cache.geom(), self.buf, stream)[1]
+
+
+def default_scale(head_dim: int = 128) -> float:
+    return 1.0 / math.sqrt(head_dim)
+
+
+def decode_step(cache: KVCache, q, k: int, k_exact, v_exact, ws: Workspace, scale=None,
+                out=None, idx=None, exact_on_host: bool = False, stream=None):
+    """One decode step for every sequence and query head.
+
+    q: bf16 [B, H, 128]; k_exact/v_exact: bf16 [B, H_kv, capacity, 128]
+    (device, or pinned host with exact_on_host=True).  Returns (out fp32
+    [B, H, 128], idx int32 [B, H_kv, k])."""
+    torch = _torch()
+    if scale is None:
+        scale = default_scale(cache.head_dim)
+    dev = q.device
+    if out is None:
+        out = torch.empty(cache.batch, cache.num_heads, cache.head_dim, dtype=torch.float32,
+                          device=dev)
+    if idx is None:
+        idx = torch.empty(cache.batch, cache.num_kv_heads, k, dtype=torch.int32, device=dev)
+    check(jfa_decode_step(cache.geom(), cache.struct(), q, float(scale), k, idx, k_exact,
+                          v_exact, exact_on_host, ws.buf, out, stream), "jfa_decode_step")
+    return out, idx

@@ -1,0 +1,273 @@
+// api.cu — the C ABI declared in include/jfa.h: argument validation, buffer
+// layouts, launch plans and the host-side record decoder.
+#include <string.h>
+
+#include "jfa_internal.cuh"
+
+namespace jfa {
+
+static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+static bool geom_ok(const jfa_geom* g) {
+  if (!g) return false;
+  if (g->batch < 1 || g->num_heads < 1 || g->num_kv_heads < 1) return false;
+  if (g->num_heads % g->num_kv_heads != 0) return false;
+  const int G = g->num_heads / g->num_kv_heads;
+  if (G > kMaxG) return false;
+  if (g->head_dim != kD) return false;
+  if (g->capacity < kKG || g->capacity % kKG != 0) return false;
+  if (g->key_bits != 3 && g->key_bits != 4) return false;
+  if (g->val_bits != 2 && g->val_bits != 4) return false;
+  if (g->n_ctx < 0 || g->n_ctx > g->capacity) return false;
+  return true;
+}
+
+static bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int workspace_layout(const jfa_geom& g, int max_topk, jfa_workspace_layout* out) {
+  const size_t n_seg = (size_t)g.batch * g.num_kv_heads;
+  const size_t G = (size_t)(g.num_heads / g.num_kv_heads);
+  jfa_workspace_layout L;
+  memset(&L, 0, sizeof(L));
+  size_t off = 0;
+  L.off_flag = off;
+  off += 256;
+  L.off_scores = off;
+  off = align_up(off + n_seg * g.capacity * sizeof(float), 256);
+  L.partial_slots = (int32_t)(kMaxScanWarps + n_seg);
+  L.off_partials = off;
+  off = align_up(off + (size_t)L.partial_slots * G * kPartStride * sizeof(float), 256);
+  L.off_hist = off;
+  off += n_seg * kHistBins * sizeof(uint32_t);
+  L.off_counters = off;
+  off = align_up(off + n_seg * 4 * sizeof(uint32_t), 256);
+  L.cand_cap = g.capacity < 16384 ? g.capacity : 16384;
+  L.off_cand = off;
+  off = align_up(off + n_seg * (size_t)L.cand_cap * 2 * sizeof(uint32_t), 256);
+  L.max_topk = max_topk;
+  L.off_sel = off;
+  off = align_up(off + n_seg * (size_t)max_topk * sizeof(int32_t), 256);
+  L.merge_chunks = (max_topk + kTail + kMergeChunk - 1) / kMergeChunk;
+  L.off_merge = off;
+  off = align_up(off + n_seg * (size_t)L.merge_chunks * 2 * G * kPartStride * sizeof(float), 256);
+  L.total_bytes = off;
+  *out = L;
+  return JFA_OK;
+}
+
+int num_sms_current() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+ScanPlan scan_plan(const jfa_geom& g, int num_sms) {
+  ScanPlan p;
+  const long long n_seg = (long long)g.batch * g.num_kv_heads;
+  p.ng = split_point(g.n_ctx) / kKG;
+  p.total_groups = n_seg * p.ng;
+  long long w = (long long)num_sms * kScanWarps;
+  if (w > kMaxScanWarps) w = kMaxScanWarps;
+  if (w > p.total_groups) w = p.total_groups;
+  p.n_warps = (int)w;
+  p.n_ctas = (int)((w + kScanWarps - 1) / kScanWarps);
+  return p;
+}
+
+}  // namespace jfa
+
+using namespace jfa;
+
+extern "C" {
+
+const char* jfa_status_string(int status) {
+  switch (status) {
+    case JFA_OK: return "ok";
+    case JFA_ERR_INVALID_ARG: return "invalid argument";
+    case JFA_ERR_UNSUPPORTED: return "unsupported";
+    case JFA_ERR_CUDA: return "CUDA error";
+    case JFA_ERR_DEVICE: return "device error flag set";
+    default: return "unknown status";
+  }
+}
+
+int jfa_cache_layout_get(const jfa_geom* geom, jfa_cache_layout* out) {
+  if (!geom_ok(geom) || !out) return JFA_ERR_INVALID_ARG;
+  const size_t n_seg = (size_t)geom->batch * geom->num_kv_heads;
+  out->record_bytes = (size_t)record_bytes(geom->key_bits, geom->val_bits);
+  out->groups_bytes = n_seg * (geom->capacity / kKG) * out->record_bytes;
+  out->tail_bytes = n_seg * kTail * kD * sizeof(uint16_t);
+  out->off_key_scales = (size_t)off_ks();
+  out->off_key_codes = (size_t)off_kc();
+  out->off_val_scales = (size_t)off_vs(geom->key_bits);
+  out->off_val_codes = (size_t)off_vc(geom->key_bits);
+  return JFA_OK;
+}
+
+int jfa_workspace_layout_get(const jfa_geom* geom, int32_t max_topk, jfa_workspace_layout* out) {
+  if (!geom_ok(geom) || !out || max_topk < 1 || max_topk > JFA_MAX_TOPK)
+    return JFA_ERR_INVALID_ARG;
+  return workspace_layout(*geom, max_topk, out);
+}
+
+static bool cache_ok(const jfa_cache* c) {
+  return c && c->groups && c->tail_k && c->tail_v && aligned(c->groups, 16) &&
+         aligned(c->tail_k, 16) && aligned(c->tail_v, 16);
+}
+
+int jfa_pack_kv(const jfa_geom* geom, const jfa_cache* cache, const uint16_t* k_new,
+                const uint16_t* v_new, int32_t n_new, void* ws, void* stream) {
+  if (!geom_ok(geom) || !cache_ok(cache) || !ws || !aligned(ws, 256)) return JFA_ERR_INVALID_ARG;
+  if (n_new < 0 || (long long)geom->n_ctx + n_new > geom->capacity) return JFA_ERR_INVALID_ARG;
+  if (n_new == 0) return JFA_OK;
+  if (!k_new || !v_new || !aligned(k_new, 16) || !aligned(v_new, 16)) return JFA_ERR_INVALID_ARG;
+  jfa_workspace_layout L;
+  workspace_layout(*geom, 1, &L);
+  return launch_pack(*geom, *cache, k_new, v_new, n_new,
+                     reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + L.off_flag),
+                     static_cast<cudaStream_t>(stream));
+}
+
+int jfa_decode_scores(const jfa_geom* geom, const jfa_cache* cache, const uint16_t* q,
+                      float scale, void* ws, void* stream) {
+  if (!geom_ok(geom) || !cache_ok(cache) || !ws || !aligned(ws, 256)) return JFA_ERR_INVALID_ARG;
+  if (geom->n_ctx < 1 || !q || !aligned(q, 16) || !(scale > 0.f) || scale != scale)
+    return JFA_ERR_INVALID_ARG;
+  jfa_workspace_layout L;
+  workspace_layout(*geom, 1, &L);
+  return launch_scores(*geom, *cache, q, scale, static_cast<uint8_t*>(ws), L,
+                       static_cast<cudaStream_t>(stream));
+}
+
+int jfa_topk(const jfa_geom* geom, int32_t k, void* ws, int32_t* idx, void* stream) {
+  if (!geom_ok(geom) || !ws || !aligned(ws, 256) || !idx || !aligned(idx, 4))
+    return JFA_ERR_INVALID_ARG;
+  if (geom->n_ctx < 1 || k < 1 || k > JFA_MAX_TOPK) return JFA_ERR_INVALID_ARG;
+  jfa_workspace_layout L;
+  workspace_layout(*geom, k, &L);
+  return launch_topk(*geom, k, static_cast<uint8_t*>(ws), L, idx,
+                     static_cast<cudaStream_t>(stream));
+}
+
+int jfa_correct_merge(const jfa_geom* geom, const jfa_cache* cache, const uint16_t* q,
+                      float scale, const int32_t* idx, int32_t k, const uint16_t* k_exact,
+                      const uint16_t* v_exact, int32_t exact_on_host, void* ws, float* out,
+                      void* stream) {
+  if (!geom_ok(geom) || !cache_ok(cache) || !ws || !aligned(ws, 256)) return JFA_ERR_INVALID_ARG;
+  if (geom->n_ctx < 1 || !q || !aligned(q, 16) || !(scale > 0.f)) return JFA_ERR_INVALID_ARG;
+  if (k < 1 || k > JFA_MAX_TOPK || !idx || !out || !aligned(out, 16)) return JFA_ERR_INVALID_ARG;
+  if (!k_exact || !v_exact || !aligned(k_exact, 16) || !aligned(v_exact, 16))
+    return JFA_ERR_INVALID_ARG;
+  jfa_workspace_layout L;
+  workspace_layout(*geom, k, &L);
+  return launch_correct_merge(*geom, *cache, q, scale, idx, k, k_exact, v_exact, exact_on_host,
+                              static_cast<uint8_t*>(ws), L, out,
+                              static_cast<cudaStream_t>(stream));
+}
+
+int jfa_decode_step(const jfa_geom* geom, const jfa_cache* cache, const uint16_t* q, float scale,
+                    int32_t k, int32_t* idx, const uint16_t* k_exact, const uint16_t* v_exact,
+                    int32_t exact_on_host, void* ws, float* out, void* stream) {
+  // validate everything before the first launch
+  if (!geom_ok(geom) || !cache_ok(cache) || !ws || !aligned(ws, 256)) return JFA_ERR_INVALID_ARG;
+  if (geom->n_ctx < 1 || !q || !aligned(q, 16) || !(scale > 0.f)) return JFA_ERR_INVALID_ARG;
+  if (k < 1 || k > JFA_MAX_TOPK || !idx || !aligned(idx, 4) || !out || !aligned(out, 16))
+    return JFA_ERR_INVALID_ARG;
+  if (!k_exact || !v_exact || !aligned(k_exact, 16) || !aligned(v_exact, 16))
+    return JFA_ERR_INVALID_ARG;
+  int s = jfa_decode_scores(geom, cache, q, scale, ws, stream);
+  if (s != JFA_OK) return s;
+  s = jfa_topk(geom, k, ws, idx, stream);
+  if (s != JFA_OK) return s;
+  return jfa_correct_merge(geom, cache, q, scale, idx, k, k_exact, v_exact, exact_on_host, ws,
+                           out, stream);
+}
+
+int jfa_decode_step_launches(const jfa_geom* geom, int32_t k) {
+  if (!geom_ok(geom) || geom->n_ctx < 1 || k < 1 || k > JFA_MAX_TOPK) return 0;
+  const int scan = split_point(geom->n_ctx) > 0 ? 1 : 0;
+  return scan + count_topk_launches(*geom, k) + 2;
+}
+
+int jfa_clear_error(const jfa_geom* geom, void* ws, void* stream) {
+  if (!geom_ok(geom) || !ws) return JFA_ERR_INVALID_ARG;
+  jfa_workspace_layout L;
+  workspace_layout(*geom, 1, &L);
+  if (cudaMemsetAsync(static_cast<uint8_t*>(ws) + L.off_flag, 0, sizeof(uint32_t),
+                      static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return JFA_ERR_CUDA;
+  return JFA_OK;
+}
+
+int jfa_check_error(const jfa_geom* geom, void* ws, void* stream, uint32_t* flag_out) {
+  if (!geom_ok(geom) || !ws) return JFA_ERR_INVALID_ARG;
+  jfa_workspace_layout L;
+  workspace_layout(*geom, 1, &L);
+  uint32_t f = 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(&f, static_cast<uint8_t*>(ws) + L.off_flag, sizeof(f),
+                      cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return JFA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return JFA_ERR_CUDA;
+  if (flag_out) *flag_out = f;
+  return f ? JFA_ERR_DEVICE : JFA_OK;
+}
+
+int jfa_unpack_record(int32_t key_bits, int32_t val_bits, const void* record, uint8_t* k_codes,
+                      uint16_t* k_scale, uint16_t* k_zero, uint8_t* v_codes, uint16_t* v_scale,
+                      uint16_t* v_zero) {
+  if ((key_bits != 3 && key_bits != 4) || (val_bits != 2 && val_bits != 4) || !record)
+    return JFA_ERR_INVALID_ARG;
+  const uint8_t* r = static_cast<const uint8_t*>(record);
+  auto word = [&](int off) {
+    uint32_t w;
+    memcpy(&w, r + off, 4);
+    return w;
+  };
+  auto half = [&](int off) {
+    uint16_t h;
+    memcpy(&h, r + off, 2);
+    return h;
+  };
+  for (int c = 0; c < kD; ++c) {
+    if (k_scale) k_scale[c] = half(off_ks() + ks_scale_off(c));
+    if (k_zero) k_zero[c] = half(off_ks() + ks_zero_off(c));
+  }
+  const uint32_t km = (1u << key_bits) - 1u, vm = (1u << val_bits) - 1u;
+  if (k_codes) {
+    for (int t = 0; t < kKG; ++t)
+      for (int c = 0; c < kD; ++c) {
+        BitLoc L = kc_loc(key_bits, t, c);
+        uint32_t code;
+        if (key_bits == 3 && kc3_is_pair15(c)) {
+          code = 0;
+          for (int b = 0; b < 3; ++b) code |= ((word(off_kc() + L.byte + 4 * b) >> L.bit) & 1u) << b;
+        } else {
+          code = (word(off_kc() + L.byte) >> L.bit) & km;
+        }
+        k_codes[t * kD + c] = (uint8_t)code;
+      }
+  }
+  for (int t = 0; t < kKG; ++t)
+    for (int j = 0; j < kD / kVG; ++j) {
+      if (v_scale) v_scale[t * 4 + j] = half(off_vs(key_bits) + vs_scale_off(t, j));
+      if (v_zero) v_zero[t * 4 + j] = half(off_vs(key_bits) + vs_zero_off(t, j));
+    }
+  if (v_codes) {
+    for (int t = 0; t < kKG; ++t)
+      for (int c = 0; c < kD; ++c) {
+        BitLoc L = vc_loc(val_bits, t, c);
+        v_codes[t * kD + c] = (uint8_t)((word(off_vc(key_bits) + L.byte) >> L.bit) & vm);
+      }
+  }
+  return JFA_OK;
+}
+
+}  // extern "C"

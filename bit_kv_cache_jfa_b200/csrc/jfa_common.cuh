@@ -1,0 +1,335 @@
+// jfa_common.cuh — shared definitions of the sm_100a decode-attention kernels:
+// the packed group-record layout, fp16 directed rounding, code unpacking and
+// thin PTX wrappers (mma.sync, mbarrier, bulk copy).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "jfa.h"
+
+#define JFA_HD __host__ __device__ __forceinline__
+
+namespace jfa {
+
+constexpr int kD = JFA_HEAD_DIM;         // 128 channels
+constexpr int kKG = JFA_KEY_GROUP;       // 64 tokens per key group
+constexpr int kVG = JFA_VAL_GROUP;       // 32 channels per value group
+constexpr int kTail = JFA_TAIL_MAX;      // 64
+constexpr int kMaxG = JFA_MAX_GQA;       // 8
+constexpr int kPartStride = 132;         // floats per (slot, head): m, l, pad2, acc[128]
+constexpr int kScanWarps = 8;            // warps per scan CTA
+constexpr int kMaxScanWarps = 2048;      // cap on scan warps (partial slots)
+constexpr int kHistBins = 2048;          // top-k first-level histogram (11 key bits)
+constexpr int kMergeChunk = 32;          // tokens per correct/merge CTA
+
+// ---------------------------------------------------------------------------
+// Packed group record: 64 tokens of one (sequence, KV head).
+//   [KS: key scales+zeros 512 B][KC: key codes 64*128*kb/8 B]
+//   [VS: value scales+zeros 1024 B][VC: value codes 64*128*vb/8 B]
+// The code order follows the register fragments of mma.sync.m16n8k16 so the
+// scan kernel turns one 128-bit shared-memory load into ready B (keys) or A
+// (values) operands; see kc_loc / vc_loc for the exact bit positions.
+// ---------------------------------------------------------------------------
+JFA_HD int kc_bytes(int kb) { return kKG * kD * kb / 8; }
+JFA_HD int vc_bytes(int vb) { return kKG * kD * vb / 8; }
+JFA_HD int off_ks() { return 0; }
+JFA_HD int off_kc() { return 512; }
+JFA_HD int off_vs(int kb) { return 512 + kc_bytes(kb); }
+JFA_HD int off_vc(int kb) { return 512 + kc_bytes(kb) + 1024; }
+JFA_HD int record_bytes(int kb, int vb) { return off_vc(kb) + vc_bytes(vb); }
+
+struct BitLoc {
+  int byte;  // byte offset of the 32-bit word inside its section
+  int bit;   // bit of the code's least significant bit inside that word
+};
+
+// Fragment coordinates of key channel c for the QK product (B operand rows):
+// k-step ks = c/16; inside it the thread tig = (c%8)/2 holds channels
+// {2tig, 2tig+1} (half hf=0) and {2tig+8, 2tig+9} (hf=1); e picks the fp16
+// half of the register.  Pair index p = 2*ks + hf runs over 16 pairs.
+JFA_HD void key_channel_frag(int c, int& tig, int& pair, int& e) {
+  int ks = c >> 4, r = c & 15;
+  int hf = r >> 3;
+  tig = (r & 7) >> 1;
+  e = r & 1;
+  pair = 2 * ks + hf;
+}
+
+// Key code of (token t, channel c); for 3-bit keys pair 15 is split over the
+// spare top bit of each half of the thread's three words (bit-th code bit in
+// word bit_word); the function reports the word of code bit 0 and the caller
+// asks kc3_pair15 for the other bits.
+JFA_HD BitLoc kc_loc(int kb, int t, int c) {
+  int tig, p, e;
+  key_channel_frag(c, tig, p, e);
+  int nt = t >> 3, gid = t & 7;
+  int lane = gid * 4 + tig;
+  BitLoc L;
+  if (kb == 4) {
+    int w = p >> 2;
+    L.byte = nt * 512 + lane * 16 + w * 4;
+    L.bit = 4 * (p & 3) + 16 * e;
+  } else {  // 3-bit
+    int nt4 = nt >> 2, rr = nt & 3;
+    int base = nt4 * 1536 + lane * 48 + rr * 12;
+    if (p < 15) {
+      int w = p / 5;
+      L.byte = base + w * 4;
+      L.bit = 3 * (p % 5) + 16 * e;
+    } else {
+      L.byte = base;  // bit b of the code lives in word b at bit 15 + 16e
+      L.bit = 15 + 16 * e;
+    }
+  }
+  return L;
+}
+JFA_HD bool kc3_is_pair15(int c) {
+  int tig, p, e;
+  key_channel_frag(c, tig, p, e);
+  return p == 15;
+}
+
+// Key scale/zero of channel c: chunk i (16 B per tig) holds 4 pairs; chunks
+// 0..3 hold scales of pairs 4i..4i+3, chunks 4..7 the zeros.
+JFA_HD int ks_scale_off(int c) {
+  int tig, p, e;
+  key_channel_frag(c, tig, p, e);
+  return (p >> 2) * 64 + tig * 16 + (p & 3) * 4 + 2 * e;
+}
+JFA_HD int ks_zero_off(int c) {
+  int tig, p, e;
+  key_channel_frag(c, tig, p, e);
+  return (4 + (p >> 2)) * 64 + tig * 16 + (p & 3) * 4 + 2 * e;
+}
+
+// Value code of (token t, channel c) for the PV product (A operand: rows =
+// channels, columns = tokens).  k-step kk = t/16; thread tig holds tokens
+// {2tig, 2tig+1} (+8 for the second half); m-tile mt = c/16, row gid = c%8,
+// +8 rows for channels 8..15.  Register r = chi + 2*hi8 as in the A fragment.
+JFA_HD BitLoc vc_loc(int vb, int t, int c) {
+  int kk = t >> 4, rt = t & 15;
+  int hi8 = rt >> 3, tig = (rt & 7) >> 1, e = rt & 1;
+  int mt = c >> 4, rc = c & 15;
+  int gid = rc & 7, chi = rc >> 3;
+  int r = chi + 2 * hi8;
+  int lane = gid * 4 + tig;
+  BitLoc L;
+  if (vb == 4) {
+    int wi = kk * 8 + mt;
+    L.byte = (wi >> 2) * 512 + lane * 16 + (wi & 3) * 4;
+    L.bit = 4 * r + 16 * e;
+  } else {  // 2-bit
+    int mp = mt >> 1, em = mt & 1;
+    L.byte = kk * 512 + lane * 16 + mp * 4;
+    L.bit = 2 * (4 * em + r) + 16 * e;
+  }
+  return L;
+}
+
+// Value scale/zero of (token t, channel group j).
+JFA_HD int vs_scale_off(int t, int j) {
+  int kk = t >> 4, rt = t & 15;
+  int hi8 = rt >> 3, tig = (rt & 7) >> 1, e = rt & 1;
+  return kk * 128 + tig * 32 + j * 8 + hi8 * 4 + 2 * e;
+}
+JFA_HD int vs_zero_off(int t, int j) { return 512 + vs_scale_off(t, j); }
+
+// Quantized-token count for n tokens: the tail keeps N - N_q in [1, 64].
+JFA_HD int split_point(int n) { return n <= 0 ? 0 : kKG * ((n - 1) / kKG); }
+
+// ---------------------------------------------------------------------------
+// fp16 directed rounding of an fp64 value (largest fp16 <= x / smallest >= x)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint16_t fp16_bits_rd(double x) {
+  __half h = __double2half(x);  // round to nearest even
+  uint16_t b = __half_as_ushort(h);
+  double back = (double)__half2float(h);
+  if (back > x) {               // step one fp16 ulp toward -inf
+    if (b == 0x0000u) b = 0x8001u;
+    else if (b & 0x8000u) b = (uint16_t)(b + 1);
+    else b = (uint16_t)(b - 1);
+  }
+  return b;
+}
+__device__ __forceinline__ uint16_t fp16_bits_ru(double x) {
+  __half h = __double2half(x);
+  uint16_t b = __half_as_ushort(h);
+  double back = (double)__half2float(h);
+  if (back < x) {               // step one fp16 ulp toward +inf
+    if (b == 0x8000u) b = 0x0001u;
+    else if (b & 0x8000u) b = (uint16_t)(b - 1);
+    else b = (uint16_t)(b + 1);
+  }
+  return b;
+}
+
+// ---------------------------------------------------------------------------
+// Code unpacking: (x & mask) | 0x6400 in each fp16 half gives 1024 + code *
+// 2^pos exactly; one fp16x2 FMA by (2^-pos, -1024*2^-pos) leaves the code.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t lop_and_or(uint32_t a, uint32_t mask, uint32_t c) {
+  uint32_t r;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(a), "r"(mask), "r"(c));
+  return r;
+}
+__device__ __forceinline__ uint32_t h2_fma(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t r;
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
+  return r;
+}
+__device__ __forceinline__ uint32_t h2_sub(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+__device__ __forceinline__ uint32_t h2_mul(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+constexpr uint32_t kMagic = 0x64006400u;  // fp16x2 (1024, 1024)
+// fp16x2 constants (2^-pos, 2^-pos) and (-1024*2^-pos, ...)
+constexpr uint32_t kOneH2 = 0x3C003C00u;      // 1.0
+constexpr uint32_t kS4 = 0x34003400u;          // 1/4
+constexpr uint32_t kS8 = 0x30003000u;          // 1/8
+constexpr uint32_t kS16 = 0x2C002C00u;         // 1/16
+constexpr uint32_t kS64 = 0x24002400u;         // 1/64
+constexpr uint32_t kS256 = 0x1C001C00u;        // 1/256
+constexpr uint32_t kB0 = 0xE400E400u;          // -1024
+constexpr uint32_t kB2 = 0xDC00DC00u;          // -256
+constexpr uint32_t kB3 = 0xD800D800u;          // -128
+constexpr uint32_t kB4 = 0xD400D400u;          // -64
+constexpr uint32_t kB6 = 0xCC00CC00u;          // -16
+constexpr uint32_t kB8 = 0xC400C400u;          // -4
+
+// 4-bit word -> 4 fp16x2 code pairs (positions 0, 4, 8, 12)
+__device__ __forceinline__ void unpack4(uint32_t w, uint32_t* o) {
+  uint32_t w8 = w >> 8;
+  o[0] = h2_sub(lop_and_or(w, 0x000F000Fu, kMagic), kMagic);
+  o[1] = h2_fma(lop_and_or(w, 0x00F000F0u, kMagic), kS16, kB4);
+  o[2] = h2_sub(lop_and_or(w8, 0x000F000Fu, kMagic), kMagic);
+  o[3] = h2_fma(lop_and_or(w8, 0x00F000F0u, kMagic), kS16, kB4);
+}
+// 2-bit word -> 8 fp16x2 code pairs (positions 0, 2, ..., 14)
+__device__ __forceinline__ void unpack2(uint32_t w, uint32_t* o) {
+  uint32_t ws = w >> 10;
+  o[0] = h2_sub(lop_and_or(w, 0x00030003u, kMagic), kMagic);
+  o[1] = h2_fma(lop_and_or(w, 0x000C000Cu, kMagic), kS4, kB2);
+  o[2] = h2_fma(lop_and_or(w, 0x00300030u, kMagic), kS16, kB4);
+  o[3] = h2_fma(lop_and_or(w, 0x00C000C0u, kMagic), kS64, kB6);
+  o[4] = h2_fma(lop_and_or(w, 0x03000300u, kMagic), kS256, kB8);
+  o[5] = h2_sub(lop_and_or(ws, 0x00030003u, kMagic), kMagic);
+  o[6] = h2_fma(lop_and_or(ws, 0x000C000Cu, kMagic), kS4, kB2);
+  o[7] = h2_fma(lop_and_or(ws, 0x00300030u, kMagic), kS16, kB4);
+}
+// three 3-bit words -> 16 fp16x2 code pairs (five per word + one split pair)
+__device__ __forceinline__ void unpack3_word(uint32_t w, uint32_t* o) {
+  uint32_t ws = w >> 9;
+  o[0] = h2_sub(lop_and_or(w, 0x00070007u, kMagic), kMagic);
+  o[1] = h2_fma(lop_and_or(w, 0x00380038u, kMagic), kS8, kB3);
+  o[2] = h2_fma(lop_and_or(w, 0x01C001C0u, kMagic), kS64, kB6);
+  o[3] = h2_sub(lop_and_or(ws, 0x00070007u, kMagic), kMagic);
+  o[4] = h2_fma(lop_and_or(ws, 0x00380038u, kMagic), kS8, kB3);
+}
+__device__ __forceinline__ void unpack3(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t* o) {
+  unpack3_word(w0, o);
+  unpack3_word(w1, o + 5);
+  unpack3_word(w2, o + 10);
+  uint32_t t = lop_and_or(w0 >> 15, 0x00010001u, kMagic);
+  t = lop_and_or(w1 >> 14, 0x00020002u, t);
+  t = lop_and_or(w2 >> 13, 0x00040004u, t);
+  o[15] = h2_sub(t, kMagic);
+}
+
+// ---------------------------------------------------------------------------
+// mma.sync m16n8k16, fp16 inputs, fp32 accumulate (D += A * B)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void mma16816(float* d, uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
+  __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+__device__ __forceinline__ float2 unpack_h2(uint32_t v) {
+  return __half22float2(*reinterpret_cast<__half2*>(&v));
+}
+
+// ---------------------------------------------------------------------------
+// mbarrier + bulk copy (global -> shared), bounded waits
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes,
+                                         uint64_t* bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint "
+      "[%0], [%1], %2, [%3], %4;" ::"r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; "
+      "selp.u32 %0, 1, 0, p; }"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+// Wait for the phase with the given parity; gives up after ~1 s and returns
+// false (the caller records JFA_DEVERR_TIMEOUT).
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 0; it < (1u << 26); ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 255u) == 255u && globaltimer_ns() - t0 > 1000000000ull) break;
+  }
+  return false;
+}
+
+__device__ __forceinline__ void set_flag(uint32_t* flag, uint32_t bits) {
+  if (flag) atomicOr(flag, bits);
+}
+
+// Orderable 32-bit key of an fp32 score: larger float -> larger key.
+__device__ __forceinline__ uint32_t float_key(float f) {
+  uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+}  // namespace jfa

@@ -1,0 +1,44 @@
+// jfa_internal.cuh — declarations shared by the kernel files and the C ABI.
+#pragma once
+
+#include "jfa_common.cuh"
+
+namespace jfa {
+
+// Workspace layout for (geometry, max_topk); host and device agree on it.
+int workspace_layout(const jfa_geom& g, int max_topk, jfa_workspace_layout* out);
+
+// Scan decomposition: W warps each take a balanced contiguous range of the
+// flattened (segment, group) list; warp w writes one partial per segment it
+// touches into slot (w + segment).
+struct ScanPlan {
+  long long total_groups;  // n_seg * NG
+  int ng;                  // groups per segment in this call (N_q / 64)
+  int n_warps;             // warps with work
+  int n_ctas;
+};
+ScanPlan scan_plan(const jfa_geom& g, int num_sms);
+int num_sms_current();
+
+// First warp whose range contains flattened group x (W warps, T groups).
+__host__ __device__ __forceinline__ long long scan_warp_of(long long x, long long W, long long T) {
+  return ((x + 1) * W - 1) / T;
+}
+__host__ __device__ __forceinline__ long long scan_range_begin(long long w, long long W,
+                                                               long long T) {
+  return w * T / W;
+}
+
+int launch_pack(const jfa_geom& g, const jfa_cache& c, const uint16_t* k_new,
+                const uint16_t* v_new, int n_new, uint32_t* flag, cudaStream_t st);
+int launch_scores(const jfa_geom& g, const jfa_cache& c, const uint16_t* q, float scale,
+                  uint8_t* ws, const jfa_workspace_layout& L, cudaStream_t st);
+int launch_topk(const jfa_geom& g, int k, uint8_t* ws, const jfa_workspace_layout& L,
+                int32_t* idx, cudaStream_t st);
+int launch_correct_merge(const jfa_geom& g, const jfa_cache& c, const uint16_t* q, float scale,
+                         const int32_t* idx, int k, const uint16_t* k_exact,
+                         const uint16_t* v_exact, int exact_on_host, uint8_t* ws,
+                         const jfa_workspace_layout& L, float* out, cudaStream_t st);
+int count_topk_launches(const jfa_geom& g, int k);
+
+}  // namespace jfa

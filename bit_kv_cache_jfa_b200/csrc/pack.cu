@@ -1,0 +1,195 @@
+// pack.cu — jfa_pack_kv kernels: group-wise asymmetric quantization and
+// bit-packing of complete 64-token groups, and bf16 tail maintenance.
+//
+// Quantization rule (HACK review, Eq. (4) context: x ~ s * x' + m with m the
+// partition minimum; TailorKV review: FP16 zero point and scale per group):
+//   zero  = largest fp16 <= min,  scale = smallest fp16 >= (max - zero)/(2^b - 1)
+//   code  = round-half-even((x - zero) / scale), clipped; both quotients fp64.
+// Keys: one (scale, zero) per (64-token group, channel); values: one per
+// (token, 32-channel group).
+#include "jfa_internal.cuh"
+
+namespace jfa {
+
+struct PackParams {
+  uint8_t* groups;
+  uint16_t* tail_k;
+  uint16_t* tail_v;
+  const uint16_t* k_new;
+  const uint16_t* v_new;
+  uint32_t* flag;
+  int hkv, ng_cap, n_new;
+  int n0, nq0;      // tokens and quantized tokens before the append
+  int g_first;      // first group to flush (= nq0 / 64)
+  int key_bits, val_bits, rec_bytes;
+};
+
+// Source of token tau (absolute position) of segment seg: the old tail for
+// tau < n0, else the new tokens.
+__device__ __forceinline__ const uint16_t* token_row(const uint16_t* tail, const uint16_t* fresh,
+                                                     int seg, int tau, const PackParams& p) {
+  if (tau < p.n0) return tail + ((size_t)seg * kTail + (tau - p.nq0)) * kD;
+  return fresh + ((size_t)seg * p.n_new + (tau - p.n0)) * kD;
+}
+
+__device__ __forceinline__ void quant_params(double mn, double mx, int bits, uint16_t& zbits,
+                                             uint16_t& sbits, double& z, double& s) {
+  zbits = fp16_bits_rd(mn);
+  z = (double)__half2float(__ushort_as_half(zbits));
+  sbits = fp16_bits_ru((mx - z) / (double)((1 << bits) - 1));
+  s = (double)__half2float(__ushort_as_half(sbits));
+}
+
+__device__ __forceinline__ uint32_t quant_code(double x, double z, double s, int bits) {
+  if (s == 0.0) return 0u;
+  double c = rint((x - z) / s);
+  double lv = (double)((1 << bits) - 1);
+  c = c < 0.0 ? 0.0 : (c > lv ? lv : c);
+  return (uint32_t)c;
+}
+
+__device__ __forceinline__ bool finite_h(uint16_t b) { return (b & 0x7C00u) != 0x7C00u; }
+__device__ __forceinline__ float bf(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
+
+// One CTA (256 threads) quantizes one 64-token group of one segment.
+__global__ void __launch_bounds__(256) pack_groups_kernel(PackParams p) {
+  __shared__ uint16_t xk[kKG][kD + 2];  // bf16 bits
+  __shared__ uint16_t xv[kKG][kD + 2];
+  __shared__ __align__(16) uint32_t rec[9728 / 4];
+  const int seg = blockIdx.y;
+  const int g = p.g_first + blockIdx.x;
+  const int tid = threadIdx.x;
+
+  for (int i = tid; i < p.rec_bytes / 4; i += 256) rec[i] = 0u;
+  for (int i = tid; i < kKG * kD / 2; i += 256) {
+    int t = i / (kD / 2), c2 = (i % (kD / 2)) * 2;
+    int tau = g * kKG + t;
+    const uint32_t* rk = reinterpret_cast<const uint32_t*>(token_row(p.tail_k, p.k_new, seg, tau, p));
+    const uint32_t* rv = reinterpret_cast<const uint32_t*>(token_row(p.tail_v, p.v_new, seg, tau, p));
+    uint32_t wk = rk[c2 / 2], wv = rv[c2 / 2];
+    xk[t][c2] = (uint16_t)(wk & 0xFFFFu);
+    xk[t][c2 + 1] = (uint16_t)(wk >> 16);
+    xv[t][c2] = (uint16_t)(wv & 0xFFFFu);
+    xv[t][c2 + 1] = (uint16_t)(wv >> 16);
+  }
+  __syncthreads();
+
+  uint8_t* rb = reinterpret_cast<uint8_t*>(rec);
+  bool bad = false;
+  // keys: thread c < 128 owns channel c
+  if (tid < kD) {
+    const int c = tid;
+    float mn = bf(xk[0][c]), mx = mn;
+    for (int t = 1; t < kKG; ++t) {
+      mn = fminf(mn, bf(xk[t][c]));
+      mx = fmaxf(mx, bf(xk[t][c]));
+    }
+    uint16_t zb, sb;
+    double z, s;
+    quant_params((double)mn, (double)mx, p.key_bits, zb, sb, z, s);
+    bad |= !finite_h(zb) || !finite_h(sb);
+    *reinterpret_cast<uint16_t*>(rb + off_ks() + ks_scale_off(c)) = sb;
+    *reinterpret_cast<uint16_t*>(rb + off_ks() + ks_zero_off(c)) = zb;
+    const bool split15 = (p.key_bits == 3) && kc3_is_pair15(c);
+    for (int t = 0; t < kKG; ++t) {
+      uint32_t code = quant_code((double)bf(xk[t][c]), z, s, p.key_bits);
+      BitLoc L = kc_loc(p.key_bits, t, c);
+      uint32_t* base = reinterpret_cast<uint32_t*>(rb + off_kc() + L.byte);
+      if (!split15) {
+        if (code) atomicOr(base, code << L.bit);
+      } else {
+        for (int b = 0; b < 3; ++b)
+          if ((code >> b) & 1u) atomicOr(base + b, 1u << L.bit);
+      }
+    }
+  } else {
+    // values: threads 128..255 own (token, group) pairs 2 each
+    for (int u = tid - kD; u < kKG * (kD / kVG); u += 128) {
+      const int t = u >> 2, j = u & 3;
+      float mn = bf(xv[t][j * kVG]), mx = mn;
+      for (int c = 1; c < kVG; ++c) {
+        mn = fminf(mn, bf(xv[t][j * kVG + c]));
+        mx = fmaxf(mx, bf(xv[t][j * kVG + c]));
+      }
+      uint16_t zb, sb;
+      double z, s;
+      quant_params((double)mn, (double)mx, p.val_bits, zb, sb, z, s);
+      bad |= !finite_h(zb) || !finite_h(sb);
+      *reinterpret_cast<uint16_t*>(rb + off_vs(p.key_bits) + vs_scale_off(t, j)) = sb;
+      *reinterpret_cast<uint16_t*>(rb + off_vs(p.key_bits) + vs_zero_off(t, j)) = zb;
+      for (int cc = 0; cc < kVG; ++cc) {
+        const int c = j * kVG + cc;
+        uint32_t code = quant_code((double)bf(xv[t][c]), z, s, p.val_bits);
+        BitLoc L = vc_loc(p.val_bits, t, c);
+        if (code) atomicOr(reinterpret_cast<uint32_t*>(rb + off_vc(p.key_bits) + L.byte), code << L.bit);
+      }
+    }
+  }
+  if (bad) set_flag(p.flag, JFA_DEVERR_NONFINITE_QUANT);
+  __syncthreads();
+  uint4* dst = reinterpret_cast<uint4*>(p.groups + ((size_t)seg * p.ng_cap + g) * p.rec_bytes);
+  const uint4* src = reinterpret_cast<const uint4*>(rec);
+  for (int i = tid; i < p.rec_bytes / 16; i += 256) dst[i] = src[i];
+}
+
+// Tail update: copy new tokens [src0, n_new) to tail slots [dst0, ...).
+__global__ void pack_tail_kernel(uint16_t* tail_k, uint16_t* tail_v, const uint16_t* k_new,
+                                 const uint16_t* v_new, int n_new, int src0, int dst0, int count) {
+  const int seg = blockIdx.y;
+  const int nvec = count * (kD / 8);  // uint4 per row = 16
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < nvec; i += gridDim.x * blockDim.x) {
+    int t = i / (kD / 8), v = i % (kD / 8);
+    size_t s = ((size_t)seg * n_new + src0 + t) * (kD / 8) + v;
+    size_t d = ((size_t)seg * kTail + dst0 + t) * (kD / 8) + v;
+    reinterpret_cast<uint4*>(tail_k)[d] = reinterpret_cast<const uint4*>(k_new)[s];
+    reinterpret_cast<uint4*>(tail_v)[d] = reinterpret_cast<const uint4*>(v_new)[s];
+  }
+}
+
+int launch_pack(const jfa_geom& g, const jfa_cache& c, const uint16_t* k_new,
+                const uint16_t* v_new, int n_new, uint32_t* flag, cudaStream_t st) {
+  const int n_seg = g.batch * g.num_kv_heads;
+  const int n0 = g.n_ctx, n1 = g.n_ctx + n_new;
+  const int nq0 = split_point(n0), nq1 = split_point(n1);
+  const int flush = (nq1 - nq0) / kKG;
+  if (flush > 0) {
+    PackParams p;
+    p.groups = static_cast<uint8_t*>(c.groups);
+    p.tail_k = c.tail_k;
+    p.tail_v = c.tail_v;
+    p.k_new = k_new;
+    p.v_new = v_new;
+    p.flag = flag;
+    p.hkv = g.num_kv_heads;
+    p.ng_cap = g.capacity / kKG;
+    p.n_new = n_new;
+    p.n0 = n0;
+    p.nq0 = nq0;
+    p.g_first = nq0 / kKG;
+    p.key_bits = g.key_bits;
+    p.val_bits = g.val_bits;
+    p.rec_bytes = record_bytes(g.key_bits, g.val_bits);
+    pack_groups_kernel<<<dim3(flush, n_seg), 256, 0, st>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return JFA_ERR_CUDA;
+  }
+  // new tail = tokens [nq1, n1); the ones that are new come from k_new
+  int src0, dst0, count;
+  if (nq1 == nq0) {          // no flush: append after the current tail
+    src0 = 0;
+    dst0 = n0 - nq0;
+    count = n_new;
+  } else {                   // flushed: the tail restarts at nq1 (all new tokens)
+    src0 = nq1 - n0;
+    dst0 = 0;
+    count = n1 - nq1;
+  }
+  if (count > 0) {
+    int blocks = (count * (kD / 8) + 255) / 256;
+    pack_tail_kernel<<<dim3(blocks, n_seg), 256, 0, st>>>(c.tail_k, c.tail_v, k_new, v_new,
+                                                          n_new, src0, dst0, count);
+    if (cudaGetLastError() != cudaSuccess) return JFA_ERR_CUDA;
+  }
+  return JFA_OK;
+}
+
+}  // namespace jfa

@@ -1,0 +1,387 @@
+// scores.cu — jfa_decode_scores: the approximate scan over packed keys and
+// values (Jet-QSparse abstract: a dense scan scores the full key history).
+//
+// Per 64-token group g of a (sequence, KV head) and query head h:
+//   s_hat[h][t] = scale * ( sum_c (q[h][c]*s[g][c]) * k'[t][c] + sum_c q[h][c]*m[g][c] )
+// which is HACK's affine identity (HACK review, Eq. (4)) with an
+// unquantized query: integer codes times a scaled query, plus a per-group
+// bias.  The integer product runs on mma.sync.m16n8k16 (fp16 in, fp32 acc):
+// rows 0-7 of A hold fp16(q*s) ("hi") and rows 8-15 the rounding remainder
+// ("lo") of the G <= 8 query heads, so hi+lo carries q*s exactly; the codes
+// are exact small integers in fp16.  Columns are tokens.
+//
+// The same pass accumulates, per query head, the online-softmax partial over
+// the dequantized values v_hat = s_v * v' + m_v (v' codes exact in fp16):
+//   sum_t p_t v_hat[t][c] = sum_t (p_t s_v[t][j]) v'[t][c] + sum_t p_t m_v[t][j]
+// as an MMA with A = value codes (rows = channels, columns = tokens) and
+// B = fp16(p * s_v) (columns = heads), plus a small MMA whose A rows are the
+// value zeros of the four channel groups and a row of ones (giving sum p).
+//
+// Work split: W warps (8 per CTA, one CTA per SM) take balanced contiguous
+// ranges of the flattened (segment, group) list.  Each warp streams its
+// records through a private two-stage shared-memory ring filled by
+// cp.async.bulk (one bulk copy per 6.5-9.5 KB record, completion on an
+// mbarrier) and writes one softmax partial per segment it touched.
+#include "jfa_internal.cuh"
+
+namespace jfa {
+
+struct ScanParams {
+  const uint8_t* groups;
+  const uint16_t* q;
+  float* scores;
+  float* partials;
+  uint32_t* flag;
+  long long total;  // n_seg * ng
+  int ng, ng_cap, capacity;
+  int hkv, G, H;
+  int n_warps;
+  float kappa;      // scale * log2(e): logits are kept in log2 units
+};
+
+__device__ __forceinline__ uint4 lds128(const uint8_t* p) {
+  return *reinterpret_cast<const uint4*>(p);
+}
+__device__ __forceinline__ uint2 lds64(const uint8_t* p) {
+  return *reinterpret_cast<const uint2*>(p);
+}
+
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr unsigned kFull = 0xFFFFFFFFu;
+
+template <int KB, int VB>
+__global__ void __launch_bounds__(kScanWarps * 32, 1) scan_kernel(const ScanParams p) {
+  constexpr int REC = 512 + 1024 * KB + 1024 + 1024 * VB;
+  constexpr int OFF_KC = 512;
+  constexpr int OFF_VS = 512 + 1024 * KB;
+  constexpr int OFF_VC = OFF_VS + 1024;
+  extern __shared__ __align__(128) uint8_t smem[];
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gid = lane >> 2, tig = lane & 3;
+  const long long wg = (long long)blockIdx.x * kScanWarps + warp;
+  if (wg >= p.n_warps) return;
+  const long long W = p.n_warps, T = p.total;
+  const long long g0 = scan_range_begin(wg, W, T), g1 = scan_range_begin(wg + 1, W, T);
+  if (g0 >= g1) return;
+
+  uint8_t* ring = smem + (size_t)warp * 2 * REC;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + (size_t)kScanWarps * 2 * REC) + warp * 2;
+  const uint64_t pol = policy_evict_first();
+  if (lane == 0) {
+    mbar_init(&bar[0], 1);
+    mbar_init(&bar[1], 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+  auto rec_ptr = [&](long long gi) -> const uint8_t* {
+    long long seg = gi / p.ng, g = gi - seg * p.ng;
+    return p.groups + ((size_t)seg * p.ng_cap + (size_t)g) * REC;
+  };
+  if (lane == 0) {
+    for (int s = 0; s < 2; ++s) {
+      if (g0 + s < g1) {
+        mbar_expect_tx(&bar[s], REC);
+        bulk_g2s(ring + s * REC, rec_ptr(g0 + s), REC, &bar[s], pol);
+      }
+    }
+  }
+
+  const bool head_ok = gid < p.G;
+  float acc[8][4];
+  float dz[4];
+  float m_run = 0.f;
+  uint32_t q2[16];
+  float qf[32];
+  long long cur = -1;
+
+  auto reset = [&](long long seg) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+    dz[0] = dz[1] = dz[2] = dz[3] = 0.f;
+    m_run = head_ok ? -INFINITY : 0.f;
+    const int b = (int)(seg / p.hkv), h = (int)(seg % p.hkv);
+    const uint16_t* qrow = p.q + ((size_t)b * p.H + (size_t)h * p.G + (head_ok ? gid : 0)) * kD;
+#pragma unroll
+    for (int pp = 0; pp < 16; ++pp) {
+      const int c = 16 * (pp >> 1) + 2 * tig + 8 * (pp & 1);
+      uint32_t w = head_ok ? *reinterpret_cast<const uint32_t*>(qrow + c) : 0u;
+      float lo = __uint_as_float(w << 16), hi = __uint_as_float(w & 0xFFFF0000u);
+      qf[2 * pp] = lo;
+      qf[2 * pp + 1] = hi;
+      q2[pp] = pack_h2(lo, hi);
+    }
+  };
+
+  auto flush = [&](long long seg) {
+    float* base = p.partials + (size_t)(wg + seg) * p.G * kPartStride;
+    float zj[4][2];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      zj[j][0] = __shfl_sync(kFull, dz[0], j * 4 + tig);
+      zj[j][1] = __shfl_sync(kFull, dz[1], j * 4 + tig);
+    }
+    const float l0 = __shfl_sync(kFull, dz[0], 16 + tig);
+    const float l1 = __shfl_sync(kFull, dz[1], 16 + tig);
+    const float mh0 = __shfl_sync(kFull, m_run, (2 * tig) * 4);
+    const float mh1 = __shfl_sync(kFull, m_run, (2 * tig + 1) * 4);
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int h = 2 * tig + e;
+      if (h < p.G) {
+        float* row = base + h * kPartStride;
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+          row[4 + 16 * mt + gid] = acc[mt][e] + zj[mt >> 1][e];
+          row[4 + 16 * mt + gid + 8] = acc[mt][2 + e] + zj[mt >> 1][e];
+        }
+        if (gid == 0) {
+          row[0] = e ? mh1 : mh0;
+          row[1] = e ? l1 : l0;
+        }
+      }
+    }
+  };
+
+  for (long long gi = g0; gi < g1; ++gi) {
+    const long long seg = gi / p.ng;
+    const int g = (int)(gi - seg * p.ng);
+    if (seg != cur) {
+      if (cur >= 0) flush(cur);
+      reset(seg);
+      cur = seg;
+    }
+    const int it = (int)(gi - g0);
+    const int st = it & 1;
+    const uint32_t par = (uint32_t)(it >> 1) & 1u;
+    const bool ok = __all_sync(kFull, mbar_wait_bounded(&bar[st], par));
+    if (!ok) {
+      if (lane == 0) {
+        set_flag(p.flag, JFA_DEVERR_TIMEOUT);
+        // drain the copies still in flight before leaving (bounded)
+        mbar_wait_bounded(&bar[st], par);
+        if (gi + 1 < g1) mbar_wait_bounded(&bar[st ^ 1], (uint32_t)((it + 1) >> 1) & 1u);
+      }
+      __syncwarp();
+      return;
+    }
+    const uint8_t* r = ring + st * REC;
+
+    // ---- q * s (hi/lo) and the per-group bias sum_c q_c m_c ----
+    uint32_t ahi[16], alo[16];
+    float beta = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint4 sv = lds128(r + i * 64 + tig * 16);
+      const uint4 zv = lds128(r + (4 + i) * 64 + tig * 16);
+      const uint32_t s4[4] = {sv.x, sv.y, sv.z, sv.w};
+      const uint32_t z4[4] = {zv.x, zv.y, zv.z, zv.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int pp = 4 * i + k;
+        ahi[pp] = h2_mul(q2[pp], s4[k]);
+        alo[pp] = h2_fma(q2[pp], s4[k], ahi[pp] ^ 0x80008000u);
+        const float2 z = unpack_h2(z4[k]);
+        beta = fmaf(qf[2 * pp], z.x, beta);
+        beta = fmaf(qf[2 * pp + 1], z.y, beta);
+      }
+    }
+    beta += __shfl_xor_sync(kFull, beta, 1);
+    beta += __shfl_xor_sync(kFull, beta, 2);
+    const float bk = beta * p.kappa;
+
+    // ---- approximate logits (log2 units) for head gid, 64 tokens ----
+    float u[8][2];
+    auto qk_tile = [&](int nt, const uint32_t* b) {
+      float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks)
+        mma16816(d, ahi[2 * ks], alo[2 * ks], ahi[2 * ks + 1], alo[2 * ks + 1], b[2 * ks],
+                 b[2 * ks + 1]);
+      u[nt][0] = head_ok ? fmaf(d[0] + d[2], p.kappa, bk) : -INFINITY;
+      u[nt][1] = head_ok ? fmaf(d[1] + d[3], p.kappa, bk) : -INFINITY;
+    };
+    if constexpr (KB == 4) {
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) {
+        const uint4 cw = lds128(r + OFF_KC + nt * 512 + lane * 16);
+        uint32_t b[16];
+        unpack4(cw.x, b);
+        unpack4(cw.y, b + 4);
+        unpack4(cw.z, b + 8);
+        unpack4(cw.w, b + 12);
+        qk_tile(nt, b);
+      }
+    } else {
+#pragma unroll
+      for (int nt4 = 0; nt4 < 2; ++nt4) {
+        const uint8_t* cp = r + OFF_KC + nt4 * 1536 + lane * 48;
+        const uint4 c0 = lds128(cp), c1 = lds128(cp + 16), c2 = lds128(cp + 32);
+        const uint32_t w[12] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y,
+                                c1.z, c1.w, c2.x, c2.y, c2.z, c2.w};
+#pragma unroll
+        for (int rr = 0; rr < 4; ++rr) {
+          uint32_t b[16];
+          unpack3(w[3 * rr], w[3 * rr + 1], w[3 * rr + 2], b);
+          qk_tile(nt4 * 4 + rr, b);
+        }
+      }
+    }
+
+    // ---- online softmax bookkeeping for head gid ----
+    float mx = u[0][0];
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) mx = fmaxf(mx, fmaxf(u[nt][0], u[nt][1]));
+    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
+    const float m_new = fmaxf(m_run, mx);
+    if (__any_sync(kFull, m_new > m_run)) {
+      const float alpha = exp2f(m_run - m_new);
+      const float a0 = __shfl_sync(kFull, alpha, (2 * tig) * 4);
+      const float a1 = __shfl_sync(kFull, alpha, (2 * tig + 1) * 4);
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt) {
+        acc[mt][0] *= a0;
+        acc[mt][1] *= a1;
+        acc[mt][2] *= a0;
+        acc[mt][3] *= a1;
+      }
+      dz[0] *= a0;
+      dz[1] *= a1;
+      dz[2] *= a0;
+      dz[3] *= a1;
+      m_run = m_new;
+    }
+
+    // ---- selection score: max over the G heads (lanes differing in gid) ----
+    {
+      float v8[4][2], v4[2][2], s2[2];
+      const bool b2 = (gid & 4) != 0, b1 = (gid & 2) != 0, b0 = (gid & 1) != 0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const float keep = b2 ? u[i + 4][e] : u[i][e];
+          const float send = b2 ? u[i][e] : u[i + 4][e];
+          v8[i][e] = fmaxf(keep, __shfl_xor_sync(kFull, send, 16));
+        }
+#pragma unroll
+      for (int i = 0; i < 2; ++i)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const float keep = b1 ? v8[i + 2][e] : v8[i][e];
+          const float send = b1 ? v8[i][e] : v8[i + 2][e];
+          v4[i][e] = fmaxf(keep, __shfl_xor_sync(kFull, send, 8));
+        }
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const float keep = b0 ? v4[1][e] : v4[0][e];
+        const float send = b0 ? v4[0][e] : v4[1][e];
+        s2[e] = fmaxf(keep, __shfl_xor_sync(kFull, send, 4));
+      }
+      float2 o;
+      o.x = s2[0] * kLn2;
+      o.y = s2[1] * kLn2;
+      *reinterpret_cast<float2*>(p.scores + (size_t)seg * p.capacity + (size_t)g * kKG +
+                                 8 * gid + 2 * tig) = o;
+    }
+
+    // ---- probabilities (fp16 pairs of tokens 8nt+2tig, +1) ----
+    uint32_t ph[8];
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt)
+      ph[nt] = pack_h2(exp2f(u[nt][0] - m_run), exp2f(u[nt][1] - m_run));
+
+    // ---- value aggregate: acc^T[c][h] += sum_t v'[t][c] * (p[t][h] s_v[t][j]) ----
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      const uint4 s0 = lds128(r + OFF_VS + kk * 128 + tig * 32);
+      const uint4 s1 = lds128(r + OFF_VS + kk * 128 + tig * 32 + 16);
+      const uint32_t pa = ph[2 * kk], pb = ph[2 * kk + 1];
+      const uint32_t bj[4][2] = {{h2_mul(pa, s0.x), h2_mul(pb, s0.y)},
+                                 {h2_mul(pa, s0.z), h2_mul(pb, s0.w)},
+                                 {h2_mul(pa, s1.x), h2_mul(pb, s1.y)},
+                                 {h2_mul(pa, s1.z), h2_mul(pb, s1.w)}};
+      uint32_t za0 = 0u, za2 = 0u;
+      if (gid < 4) {
+        const uint2 zz = lds64(r + OFF_VS + 512 + kk * 128 + tig * 32 + gid * 8);
+        za0 = zz.x;
+        za2 = zz.y;
+      } else if (gid == 4) {
+        za0 = za2 = kOneH2;
+      }
+      mma16816(dz, za0, 0u, za2, 0u, pa, pb);
+      if constexpr (VB == 4) {
+        const uint4 v0 = lds128(r + OFF_VC + (2 * kk) * 512 + lane * 16);
+        const uint4 v1 = lds128(r + OFF_VC + (2 * kk + 1) * 512 + lane * 16);
+        const uint32_t vw[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+          uint32_t a[4];
+          unpack4(vw[mt], a);
+          mma16816(acc[mt], a[0], a[1], a[2], a[3], bj[mt >> 1][0], bj[mt >> 1][1]);
+        }
+      } else {
+        const uint4 v = lds128(r + OFF_VC + kk * 512 + lane * 16);
+        const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int mp = 0; mp < 4; ++mp) {
+          uint32_t a[8];
+          unpack2(vw[mp], a);
+          mma16816(acc[2 * mp], a[0], a[1], a[2], a[3], bj[mp][0], bj[mp][1]);
+          mma16816(acc[2 * mp + 1], a[4], a[5], a[6], a[7], bj[mp][0], bj[mp][1]);
+        }
+      }
+    }
+
+    __syncwarp();
+    if (lane == 0 && gi + 2 < g1) {
+      mbar_expect_tx(&bar[st], REC);
+      bulk_g2s(ring + st * REC, rec_ptr(gi + 2), REC, &bar[st], pol);
+    }
+  }
+  flush(cur);
+}
+
+template <int KB, int VB>
+static int launch_scan_t(const ScanParams& sp, int n_ctas, cudaStream_t st) {
+  constexpr int REC = 512 + 1024 * KB + 1024 + 1024 * VB;
+  const int smem = kScanWarps * 2 * REC + kScanWarps * 2 * 8;
+  static bool configured = false;
+  if (!configured) {
+    if (cudaFuncSetAttribute(scan_kernel<KB, VB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem) != cudaSuccess)
+      return JFA_ERR_CUDA;
+    configured = true;
+  }
+  scan_kernel<KB, VB><<<n_ctas, kScanWarps * 32, smem, st>>>(sp);
+  return cudaGetLastError() == cudaSuccess ? JFA_OK : JFA_ERR_CUDA;
+}
+
+int launch_scores(const jfa_geom& g, const jfa_cache& c, const uint16_t* q, float scale,
+                  uint8_t* ws, const jfa_workspace_layout& L, cudaStream_t st) {
+  ScanPlan plan = scan_plan(g, num_sms_current());
+  if (plan.total_groups == 0) return JFA_OK;
+  ScanParams sp;
+  sp.groups = static_cast<const uint8_t*>(c.groups);
+  sp.q = q;
+  sp.scores = reinterpret_cast<float*>(ws + L.off_scores);
+  sp.partials = reinterpret_cast<float*>(ws + L.off_partials);
+  sp.flag = reinterpret_cast<uint32_t*>(ws + L.off_flag);
+  sp.total = plan.total_groups;
+  sp.ng = plan.ng;
+  sp.ng_cap = g.capacity / kKG;
+  sp.capacity = g.capacity;
+  sp.hkv = g.num_kv_heads;
+  sp.G = g.num_heads / g.num_kv_heads;
+  sp.H = g.num_heads;
+  sp.n_warps = plan.n_warps;
+  sp.kappa = scale * 1.4426950408889634f;
+  if (g.key_bits == 3 && g.val_bits == 2) return launch_scan_t<3, 2>(sp, plan.n_ctas, st);
+  if (g.key_bits == 4 && g.val_bits == 4) return launch_scan_t<4, 4>(sp, plan.n_ctas, st);
+  if (g.key_bits == 3 && g.val_bits == 4) return launch_scan_t<3, 4>(sp, plan.n_ctas, st);
+  if (g.key_bits == 4 && g.val_bits == 2) return launch_scan_t<4, 2>(sp, plan.n_ctas, st);
+  return JFA_ERR_UNSUPPORTED;
+}
+
+}  // namespace jfa

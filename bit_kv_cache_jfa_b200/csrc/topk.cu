@@ -1,0 +1,335 @@
+// topk.cu — jfa_topk: per (sequence, KV head) the k tokens with the largest
+// selection score S (JetFire README, introduction: the top-k tokens are
+// corrected; Jet-QSparse abstract: selection per KV head).
+//
+// Order (S descending, index ascending); output indices sorted ascending.
+// Scores map to order-preserving 32-bit keys.  Three kernels:
+//   1. histogram of the top 11 key bits per segment (many CTAs per segment);
+//   2. every CTA finds the bin holding the k-th key, appends indices of keys
+//      in higher bins to the segment's selected list and (key, index) pairs in
+//      that bin to a candidate list;
+//   3. one CTA per segment refines the candidates by the next 11 and 10 key
+//      bits (radix select) to the exact k-th key, resolves ties by index,
+//      and sorts the k chosen indices (bitonic, in shared memory).
+// A candidate list that overflows its capacity falls back to reading S.
+#include "jfa_internal.cuh"
+
+namespace jfa {
+
+constexpr unsigned kFullMask = 0xFFFFFFFFu;
+
+// Block-wide exclusive sum over threads in DESCENDING thread order:
+// returns sum of v over threads with a larger index.  scratch: >= 32 uints.
+__device__ uint32_t block_suffix_excl(uint32_t v, uint32_t* scratch) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  // inclusive suffix within the warp
+  uint32_t x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    uint32_t y = __shfl_down_sync(kFullMask, x, o);
+    if (lane + o < 32) x += y;
+  }
+  if (lane == 0) scratch[warp] = x;  // warp total
+  __syncthreads();
+  uint32_t after = 0;
+  for (int w = warp + 1; w < nw; ++w) after += scratch[w];
+  __syncthreads();
+  return after + (x - v);
+}
+
+// Given per-bin counts in h[0..nbins), find the bin where the count taken
+// from the top reaches r.  Returns bin and count strictly above it.
+__device__ void find_from_top(const uint32_t* h, int nbins, uint32_t r, uint32_t* scratch,
+                              int* out_bin, uint32_t* out_above) {
+  const int per = nbins / blockDim.x;  // nbins is a multiple of blockDim
+  const int b0 = threadIdx.x * per;
+  uint32_t local = 0;
+  for (int i = 0; i < per; ++i) local += h[b0 + i];
+  uint32_t cum = block_suffix_excl(local, scratch);
+  for (int i = per - 1; i >= 0; --i) {
+    const uint32_t c = h[b0 + i];
+    if (cum < r && cum + c >= r) {
+      *out_bin = b0 + i;
+      *out_above = cum;
+    }
+    cum += c;
+  }
+  __syncthreads();
+}
+// Same from the bottom (smallest bins first): bin where the count reaches r.
+__device__ void find_from_bottom(const uint32_t* h, int nbins, uint32_t r, uint32_t* scratch,
+                                 int* out_bin, uint32_t* out_below) {
+  const int per = nbins / blockDim.x;
+  // reverse the bin order so the suffix helper gives "count below"
+  const int b0 = nbins - (threadIdx.x + 1) * per;
+  uint32_t local = 0;
+  for (int i = 0; i < per; ++i) local += h[b0 + i];
+  uint32_t cum = block_suffix_excl(local, scratch);
+  for (int i = 0; i < per; ++i) {
+    const uint32_t c = h[b0 + i];
+    if (cum < r && cum + c >= r) {
+      *out_bin = b0 + i;
+      *out_below = cum;
+    }
+    cum += c;
+  }
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(256) topk_hist_kernel(const float* scores, int capacity,
+                                                        int nq, uint32_t* hist) {
+  __shared__ uint32_t sh[kHistBins];
+  const int seg = blockIdx.y;
+  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) sh[i] = 0u;
+  __syncthreads();
+  const int per = ((nq + gridDim.x - 1) / gridDim.x + 3) & ~3;
+  const int lo = blockIdx.x * per, hi = min(nq, lo + per);
+  const float* s = scores + (size_t)seg * capacity;
+  for (int i = lo + 4 * threadIdx.x; i < hi; i += 4 * blockDim.x) {
+    const float4 v = *reinterpret_cast<const float4*>(s + i);  // nq is a multiple of 64
+    atomicAdd(&sh[float_key(v.x) >> 21], 1u);
+    atomicAdd(&sh[float_key(v.y) >> 21], 1u);
+    atomicAdd(&sh[float_key(v.z) >> 21], 1u);
+    atomicAdd(&sh[float_key(v.w) >> 21], 1u);
+  }
+  __syncthreads();
+  uint32_t* gh = hist + (size_t)seg * kHistBins;
+  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x)
+    if (sh[i]) atomicAdd(&gh[i], sh[i]);
+}
+
+struct TopkBufs {
+  const float* scores;
+  uint32_t* hist;      // [n_seg][2048]
+  uint32_t* counters;  // [n_seg][4]: n_sel, n_cand, bstar, above
+  uint2* cand;         // [n_seg][cand_cap] (key, index)
+  int32_t* sel;        // [n_seg][max_topk]
+  int capacity, nq, k, cand_cap, max_topk;
+};
+
+__global__ void __launch_bounds__(256) topk_collect_kernel(TopkBufs b) {
+  __shared__ uint32_t sh[kHistBins];
+  __shared__ uint32_t scratch[32];
+  __shared__ int s_bin;
+  __shared__ uint32_t s_above;
+  const int seg = blockIdx.y;
+  const uint32_t* gh = b.hist + (size_t)seg * kHistBins;
+  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) sh[i] = gh[i];
+  if (threadIdx.x == 0) {
+    s_bin = 0;
+    s_above = 0;
+  }
+  __syncthreads();
+  find_from_top(sh, kHistBins, (uint32_t)b.k, scratch, &s_bin, &s_above);
+  const uint32_t bstar = (uint32_t)s_bin;
+  uint32_t* ctr = b.counters + (size_t)seg * 4;
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    ctr[2] = bstar;
+    ctr[3] = s_above;
+  }
+  const int lane = threadIdx.x & 31;
+  const unsigned lt = (1u << lane) - 1u;
+  const int per = ((b.nq + gridDim.x - 1) / gridDim.x + 255) & ~255;
+  const int lo = blockIdx.x * per, hi = min(b.nq, lo + per);
+  const float* s = b.scores + (size_t)seg * b.capacity;
+  int32_t* sel = b.sel + (size_t)seg * b.max_topk;
+  uint2* cand = b.cand + (size_t)seg * b.cand_cap;
+  for (int base = lo; base < hi; base += blockDim.x) {
+    const int i = base + threadIdx.x;
+    const bool valid = i < hi;
+    const uint32_t key = valid ? float_key(s[i]) : 0u;
+    const uint32_t bin = key >> 21;
+    const bool is_sel = valid && bin > bstar;
+    const bool is_cand = valid && bin == bstar;
+    const unsigned ms = __ballot_sync(kFullMask, is_sel);
+    if (ms) {
+      uint32_t pos = 0;
+      if (lane == __ffs(ms) - 1) pos = atomicAdd(&ctr[0], (uint32_t)__popc(ms));
+      pos = __shfl_sync(kFullMask, pos, __ffs(ms) - 1);
+      if (is_sel) sel[pos + __popc(ms & lt)] = i;
+    }
+    const unsigned mc = __ballot_sync(kFullMask, is_cand);
+    if (mc) {
+      uint32_t pos = 0;
+      if (lane == __ffs(mc) - 1) pos = atomicAdd(&ctr[1], (uint32_t)__popc(mc));
+      pos = __shfl_sync(kFullMask, pos, __ffs(mc) - 1);
+      const uint32_t mine = pos + __popc(mc & lt);
+      if (is_cand && mine < (uint32_t)b.cand_cap) cand[mine] = make_uint2(key, (uint32_t)i);
+    }
+  }
+}
+
+// One CTA (1024 threads) per segment.
+__global__ void __launch_bounds__(1024) topk_final_kernel(TopkBufs b, int32_t* idx) {
+  __shared__ uint32_t h[kHistBins];
+  __shared__ int32_t out[JFA_MAX_TOPK];
+  __shared__ uint32_t scratch[32];
+  __shared__ int s_bin;
+  __shared__ uint32_t s_cnt, s_nout;
+  const int seg = blockIdx.x;
+  const int tid = threadIdx.x;
+  const uint32_t* ctr = b.counters + (size_t)seg * 4;
+  const uint32_t n_sel = ctr[0], n_cand = ctr[1], bstar = ctr[2];
+  const uint32_t r = (uint32_t)b.k - n_sel;  // >= 1
+  const int32_t* sel = b.sel + (size_t)seg * b.max_topk;
+  for (uint32_t i = tid; i < n_sel; i += blockDim.x) out[i] = sel[i];
+  const bool from_cand = n_cand <= (uint32_t)b.cand_cap;
+  const uint2* cand = b.cand + (size_t)seg * b.cand_cap;
+  const float* s = b.scores + (size_t)seg * b.capacity;
+  const uint32_t n_src = from_cand ? n_cand : (uint32_t)b.nq;
+  // element j of the source: (key, index, member of the threshold bin?)
+  auto src = [&](uint32_t j, uint32_t& key, int32_t& ix) -> bool {
+    if (from_cand) {
+      const uint2 c = cand[j];
+      key = c.x;
+      ix = (int32_t)c.y;
+      return true;
+    }
+    key = float_key(s[j]);
+    ix = (int32_t)j;
+    return (key >> 21) == bstar;
+  };
+
+  // refine bits 20..10
+  for (int i = tid; i < kHistBins; i += blockDim.x) h[i] = 0u;
+  if (tid == 0) s_nout = n_sel;
+  __syncthreads();
+  for (uint32_t j = tid; j < n_src; j += blockDim.x) {
+    uint32_t key;
+    int32_t ix;
+    if (src(j, key, ix)) atomicAdd(&h[(key >> 10) & 2047u], 1u);
+  }
+  __syncthreads();
+  int d2 = 0;
+  uint32_t above2 = 0;
+  find_from_top(h, 2048, r, scratch, &s_bin, &s_cnt);
+  d2 = s_bin;
+  above2 = s_cnt;
+  const uint32_t r2 = r - above2;
+  // refine bits 9..0
+  for (int i = tid; i < kHistBins; i += blockDim.x) h[i] = 0u;
+  __syncthreads();
+  for (uint32_t j = tid; j < n_src; j += blockDim.x) {
+    uint32_t key;
+    int32_t ix;
+    if (src(j, key, ix) && ((key >> 10) & 2047u) == (uint32_t)d2) atomicAdd(&h[key & 1023u], 1u);
+  }
+  __syncthreads();
+  find_from_top(h, 1024, r2, scratch, &s_bin, &s_cnt);
+  const int d3 = s_bin;
+  const uint32_t r3 = r2 - s_cnt;        // ties to take at the exact k-th key
+  const uint32_t n_eq = h[d3];
+  const uint32_t kstar = (bstar << 21) | ((uint32_t)d2 << 10) | (uint32_t)d3;
+  __syncthreads();
+
+  // smallest r3 indices among keys == kstar: index threshold istar
+  int32_t istar = 0x7FFFFFFF;
+  if (r3 < n_eq) {
+    uint32_t need = r3;
+    uint32_t prefix = 0;  // high index bits fixed so far
+    for (int pass = 0; pass < 3; ++pass) {
+      const int shift = 22 - 11 * pass;   // bits 32..22, 21..11, 10..0
+      const uint32_t nb = 2048;
+      for (int i = tid; i < kHistBins; i += blockDim.x) h[i] = 0u;
+      __syncthreads();
+      for (uint32_t j = tid; j < n_src; j += blockDim.x) {
+        uint32_t key;
+        int32_t ix;
+        if (src(j, key, ix) && key == kstar) {
+          const uint32_t ux = (uint32_t)ix;
+          const bool match = pass == 0 || (ux >> (shift + 11)) == prefix;
+          if (match) atomicAdd(&h[(ux >> shift) & (nb - 1)], 1u);
+        }
+      }
+      __syncthreads();
+      find_from_bottom(h, 2048, need, scratch, &s_bin, &s_cnt);
+      need -= s_cnt;
+      prefix = (prefix << 11) | (uint32_t)s_bin;
+      __syncthreads();
+    }
+    istar = (int32_t)prefix;
+  }
+
+  // collect the rest of the selection from the source
+  for (uint32_t j = tid; j < n_src; j += blockDim.x) {
+    uint32_t key;
+    int32_t ix;
+    if (!src(j, key, ix)) continue;
+    if (key > kstar || (key == kstar && ix <= istar)) {
+      const uint32_t pos = atomicAdd(&s_nout, 1u);
+      if (pos < (uint32_t)b.k) out[pos] = ix;
+    }
+  }
+  __syncthreads();
+  // bitonic sort out[0..npow) ascending
+  int npow = 1;
+  while (npow < b.k) npow <<= 1;
+  for (int i = b.k + tid; i < npow; i += blockDim.x) out[i] = 0x7FFFFFFF;
+  __syncthreads();
+  for (int size = 2; size <= npow; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int i = tid; i < npow / 2; i += blockDim.x) {
+        const int lo = 2 * i - (i & (stride - 1));
+        const int hi = lo + stride;
+        const bool up = (lo & size) == 0;
+        const int32_t a = out[lo], c = out[hi];
+        if ((a > c) == up) {
+          out[lo] = c;
+          out[hi] = a;
+        }
+      }
+      __syncthreads();
+    }
+  }
+  int32_t* o = idx + (size_t)seg * b.k;
+  for (int i = tid; i < b.k; i += blockDim.x) o[i] = out[i];
+}
+
+__global__ void topk_fill_kernel(int32_t* idx, int k, int nq) {
+  const int seg = blockIdx.y;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < k; i += gridDim.x * blockDim.x)
+    idx[(size_t)seg * k + i] = i < nq ? i : -1;
+}
+
+static int topk_chunks(int nq, int n_seg) {
+  int by_size = (nq + 4095) / 4096;
+  int by_sm = (2 * num_sms_current() + n_seg - 1) / n_seg;
+  int c = by_size < by_sm ? by_size : by_sm;
+  return c < 1 ? 1 : c;
+}
+
+int count_topk_launches(const jfa_geom& g, int k) {
+  const int nq = split_point(g.n_ctx);
+  return k >= nq ? 1 : 4;  // fill | memset + hist + collect + final
+}
+
+int launch_topk(const jfa_geom& g, int k, uint8_t* ws, const jfa_workspace_layout& L,
+                int32_t* idx, cudaStream_t st) {
+  const int n_seg = g.batch * g.num_kv_heads;
+  const int nq = split_point(g.n_ctx);
+  if (k >= nq) {
+    topk_fill_kernel<<<dim3((k + 255) / 256, n_seg), 256, 0, st>>>(idx, k, nq);
+    return cudaGetLastError() == cudaSuccess ? JFA_OK : JFA_ERR_CUDA;
+  }
+  TopkBufs b;
+  b.scores = reinterpret_cast<const float*>(ws + L.off_scores);
+  b.hist = reinterpret_cast<uint32_t*>(ws + L.off_hist);
+  b.counters = reinterpret_cast<uint32_t*>(ws + L.off_counters);
+  b.cand = reinterpret_cast<uint2*>(ws + L.off_cand);
+  b.sel = reinterpret_cast<int32_t*>(ws + L.off_sel);
+  b.capacity = g.capacity;
+  b.nq = nq;
+  b.k = k;
+  b.cand_cap = L.cand_cap;
+  b.max_topk = L.max_topk;
+  // histograms and counters are contiguous: clear both at once
+  if (cudaMemsetAsync(ws + L.off_hist, 0, L.off_cand - L.off_hist, st) != cudaSuccess)
+    return JFA_ERR_CUDA;
+  const int chunks = topk_chunks(nq, n_seg);
+  topk_hist_kernel<<<dim3(chunks, n_seg), 256, 0, st>>>(b.scores, g.capacity, nq, b.hist);
+  topk_collect_kernel<<<dim3(chunks, n_seg), 256, 0, st>>>(b);
+  topk_final_kernel<<<n_seg, 1024, 0, st>>>(b, idx);
+  return cudaGetLastError() == cudaSuccess ? JFA_OK : JFA_ERR_CUDA;
+}
+
+}  // namespace jfa

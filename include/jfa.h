@@ -1,0 +1,233 @@
+/*
+ * jfa.h — C ABI of the approximate-then-correct low-bit KV decode-attention
+ * library (sm_100a).
+ *
+ * The method (JetFire README, introduction): the KV cache lives on the GPU at
+ * low bit width (K3V2: 3-bit keys / 2-bit values, or K4V4; README, benchmark
+ * section), every cached token is scored approximately from it, the top-k
+ * tokens are re-scored and re-aggregated from a high-precision BF16 copy
+ * (held in GPU memory or in pinned host memory), and the exact and
+ * approximate parts are merged.
+ *
+ * One decode step for all sequences of a batch and all heads of one layer is
+ *     jfa_decode_scores -> jfa_topk -> jfa_correct_merge
+ * and new tokens enter the cache through jfa_pack_kv.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - All tensor pointers are DEVICE pointers (or, where stated, pointers to
+ *    pinned host memory that the device can address), caller-owned; the
+ *    library never allocates, frees or synchronises (except
+ *    jfa_check_error).  Work is ordered on the given stream.
+ *  - bf16 tensors are raw 16-bit patterns (`uint16_t`), row-major.
+ *  - Every call returns a jfa_status; on an argument error nothing is
+ *    launched.  No exception or abort crosses the ABI.
+ *  - Device-side problems (non-finite scale/zero while packing, an
+ *    out-of-range index handed to jfa_correct_merge, an exhausted bounded
+ *    wait) set a flag word in the workspace; jfa_check_error reads it.
+ *  - head_dim is 128; query heads per KV head G = H / H_kv must be 1..8.
+ *  - All sequences of a batch hold the same number of tokens (n_ctx).
+ */
+#ifndef JFA_H_
+#define JFA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Fixed quantization geometry.
+ * Keys: one fp16 (scale, zero) per (64-token group, channel); values: one
+ * per (token, 32-channel group).  Group size 64 with an FP16 zero point and
+ * scale follows the TailorKV review ("free parameters": quantization bit
+ * size and group size) and HACK's default partition size 64 (HACK review,
+ * "free parameters").  The newest 1..64 tokens stay exact in a bf16 tail so
+ * appends never requantize (HACK review, Figure 8: last block of V kept in
+ * FP16; Jet-QSparse abstract: at most two BF16 pages per sequence). */
+#define JFA_HEAD_DIM 128
+#define JFA_KEY_GROUP 64
+#define JFA_VAL_GROUP 32
+#define JFA_TAIL_MAX 64
+#define JFA_MAX_GQA 8
+#define JFA_MAX_TOPK 4096
+
+typedef enum jfa_status {
+  JFA_OK = 0,
+  JFA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size or geometry */
+  JFA_ERR_UNSUPPORTED = 2, /* valid request this build does not implement   */
+  JFA_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed          */
+  JFA_ERR_DEVICE = 4       /* the device error flag is set (jfa_check_error)*/
+} jfa_status;
+
+/* Device error flag bits (OR-ed into the workspace flag word). */
+#define JFA_DEVERR_NONFINITE_QUANT 0x1u /* a packed scale/zero is inf/nan   */
+#define JFA_DEVERR_BAD_INDEX 0x2u       /* top-k index outside [0, N_q)     */
+#define JFA_DEVERR_TIMEOUT 0x4u         /* a bounded wait gave up           */
+
+typedef struct jfa_geom {
+  int32_t batch;        /* B: sequences                                   */
+  int32_t num_heads;    /* H: query heads                                 */
+  int32_t num_kv_heads; /* H_kv: KV heads; H % H_kv == 0, H/H_kv <= 8      */
+  int32_t head_dim;     /* must be 128                                    */
+  int32_t capacity;     /* max tokens per sequence; multiple of 64, >= 64 */
+  int32_t key_bits;     /* 3 or 4                                         */
+  int32_t val_bits;     /* 2 or 4                                         */
+  int32_t n_ctx;        /* tokens currently cached per sequence           */
+} jfa_geom;
+
+/* Device buffers of one layer's quantized cache (caller-allocated with the
+ * sizes jfa_cache_layout reports; every pointer 256-byte aligned).
+ *   groups : packed group records, [B][H_kv][capacity/64][record_bytes].
+ *            A record holds the codes and fp16 scales/zeros of the keys and
+ *            values of 64 consecutive tokens, in a layout private to this
+ *            library (decode it with jfa_unpack_record).
+ *   tail_k, tail_v : bf16 [B][H_kv][64][128], the newest 1..64 tokens. */
+typedef struct jfa_cache {
+  void* groups;
+  uint16_t* tail_k;
+  uint16_t* tail_v;
+} jfa_cache;
+
+typedef struct jfa_cache_layout {
+  size_t record_bytes; /* bytes per (sequence, KV head, 64-token group)   */
+  size_t groups_bytes; /* size of jfa_cache.groups                        */
+  size_t tail_bytes;   /* size of each of tail_k and tail_v               */
+  /* byte offsets of the record sections */
+  size_t off_key_scales, off_key_codes, off_val_scales, off_val_codes;
+} jfa_cache_layout;
+
+/* Workspace layout: scratch of the decode step (selection scores, split
+ * softmax partials, top-k histograms/candidates, merge partials, the error
+ * flag).  Sized by jfa_workspace_bytes for a geometry and a maximum k. */
+typedef struct jfa_workspace_layout {
+  size_t total_bytes;
+  size_t off_flag;       /* uint32 device error flag                          */
+  size_t off_scores;     /* fp32 [B][H_kv][capacity]: selection score S_t     */
+  size_t off_partials;   /* fp32 split partials of the approximate scan       */
+  size_t off_hist;       /* top-k histograms                                  */
+  size_t off_counters;   /* top-k counters                                    */
+  size_t off_cand;       /* top-k candidate (key, index) pairs                */
+  size_t off_sel;        /* top-k selected-index lists                        */
+  size_t off_merge;      /* fp32 per-chunk exact / removal partials           */
+  int32_t max_topk;
+  int32_t partial_slots; /* slots of off_partials                             */
+  int32_t cand_cap;      /* candidates per segment                            */
+  int32_t merge_chunks;  /* chunks of off_merge per segment                   */
+} jfa_workspace_layout;
+
+/* Human-readable name of a status code (static string). */
+const char* jfa_status_string(int status);
+
+/* Sizes and section offsets of the cache buffers for a geometry.
+ * Pure host function; JFA_ERR_INVALID_ARG on a bad geometry. */
+int jfa_cache_layout_get(const jfa_geom* geom, jfa_cache_layout* out);
+
+/* Sizes and offsets of the decode workspace for a geometry and a maximum k
+ * (1..JFA_MAX_TOPK).  Pure host function.  The workspace needs no
+ * initialisation: each call clears what it accumulates into. */
+int jfa_workspace_layout_get(const jfa_geom* geom, int32_t max_topk,
+                             jfa_workspace_layout* out);
+
+/* jfa_pack_kv — append n_new tokens to every sequence.
+ * Definition: partition-wise asymmetric quantization x ~ s*x' + m with m the
+ * partition minimum (HACK review, Eq. (4) and context), FP16 zero point and
+ * scale per group of 64 (TailorKV review).  This library takes
+ *   zero  = largest fp16 <= min, scale = smallest fp16 >= (max-zero)/(2^b-1),
+ *   code  = round-half-even((x-zero)/scale) clipped to [0, 2^b-1],
+ * both quotients in fp64; keys per (64-token group, channel), values per
+ * (token, 32-channel group).  Tokens enter the bf16 tail; a token arriving
+ * at a full tail (64) first flushes the tail as one group, so the tail holds
+ * N - N_q in [1, 64] tokens with N_q = 64*floor((N-1)/64), and codes once
+ * written never change.
+ *   geom->n_ctx : tokens already cached (before this call); the caller adds
+ *                 n_new to its own counter after the call.
+ *   k_new, v_new: bf16 [B][H_kv][n_new][128] device pointers, 16-B aligned.
+ *   ws          : workspace (only the error flag is used).
+ * Requires n_ctx + n_new <= capacity.  The high-precision copy of K/V used
+ * by jfa_correct_merge is the caller's (written by the caller). */
+int jfa_pack_kv(const jfa_geom* geom, const jfa_cache* cache,
+                const uint16_t* k_new, const uint16_t* v_new, int32_t n_new,
+                void* ws, void* stream);
+
+/* jfa_decode_scores — approximate scan over the N_q quantized tokens.
+ * Definition (Jet-QSparse abstract: a dense scan scores the full key
+ * history; HACK review, Eq. (4): the product with affinely quantized keys is
+ * an integer product plus correction terms):
+ *   s_hat[h][t] = scale * sum_c q[h][c] * (s[g][c]*k'[t][c] + m[g][c])
+ * for every query head h and quantized token t (g = t/64), and the selection
+ * score S[t] = max over the G query heads sharing the KV head.  In the same
+ * pass it accumulates, per split of the token range, the softmax partial
+ * (max, sum exp, sum exp * v_hat) of every query head over the dequantized
+ * values, which jfa_correct_merge turns into the approximate remainder.
+ *   q     : bf16 [B][H][128] device pointer, 16-B aligned.
+ *   scale : softmax scale (e.g. 1/sqrt(128)).
+ *   ws    : workspace for at least this geometry.
+ * Writes S (workspace off_scores) and the split partials. */
+int jfa_decode_scores(const jfa_geom* geom, const jfa_cache* cache,
+                      const uint16_t* q, float scale, void* ws, void* stream);
+
+/* jfa_topk — per (sequence, KV head) the k tokens with the largest S
+ * (JetFire README: correct the top-k tokens; Jet-QSparse abstract: selection
+ * per KV head).  Order is (S descending, index ascending); the k_eff =
+ * min(k, N_q) chosen indices are written sorted ascending to
+ * idx[B][H_kv][k] (int32 device pointer), the remaining k - k_eff entries
+ * set to -1.  1 <= k <= max_topk of the workspace. */
+int jfa_topk(const jfa_geom* geom, int32_t k, void* ws, int32_t* idx,
+             void* stream);
+
+/* jfa_correct_merge — exact correction and log-sum-exp merge.
+ * For every query head: exact logits scale*q.K_t from the bf16 copy for the
+ * top-k tokens and the tail, aggregated with bf16 values in fp32 (Jet-QSparse
+ * abstract: sparse high-precision value aggregation with FP32 accumulation;
+ * JetFire README: high-precision correction of the top-k tokens); the
+ * approximate remainder over the other quantized tokens (the scan partials
+ * minus the top-k tokens' approximate terms); merged as
+ *   m = max(m_e, m_a), out = (acc_e e^(m_e-m) + acc_a e^(m_a-m)) /
+ *                            (l_e e^(m_e-m) + l_a e^(m_a-m)).
+ *   idx          : int32 [B][H_kv][k] from jfa_topk (entries -1 ignored).
+ *   k_exact,
+ *   v_exact      : bf16 [B][H_kv][capacity][128], every cached token; device
+ *                  memory, or pinned host memory the device can address
+ *                  (exact_on_host = 1: rows are read by zero-copy loads).
+ *   out          : fp32 [B][H][128] device pointer.
+ * Must follow jfa_decode_scores with the same geometry, q and scale. */
+int jfa_correct_merge(const jfa_geom* geom, const jfa_cache* cache,
+                      const uint16_t* q, float scale, const int32_t* idx,
+                      int32_t k, const uint16_t* k_exact,
+                      const uint16_t* v_exact, int32_t exact_on_host,
+                      void* ws, float* out, void* stream);
+
+/* The whole decode step (scores, top-k, correct+merge) in one call;
+ * equivalent to the three calls in order.  idx is written as by jfa_topk. */
+int jfa_decode_step(const jfa_geom* geom, const jfa_cache* cache,
+                    const uint16_t* q, float scale, int32_t k, int32_t* idx,
+                    const uint16_t* k_exact, const uint16_t* v_exact,
+                    int32_t exact_on_host, void* ws, float* out, void* stream);
+
+/* Clear the workspace error flag (stream-ordered). */
+int jfa_clear_error(const jfa_geom* geom, void* ws, void* stream);
+
+/* Synchronise the stream and read the device error flag into *flag_out
+ * (0 = no error).  Returns JFA_ERR_DEVICE if the flag is non-zero. */
+int jfa_check_error(const jfa_geom* geom, void* ws, void* stream,
+                    uint32_t* flag_out);
+
+/* Host-side decoder of one packed group record (record_bytes from
+ * jfa_cache_layout_get), for inspection and tests.  Outputs:
+ *   k_codes [64][128] (token-major), k_scale/k_zero [128] fp16 bits,
+ *   v_codes [64][128], v_scale/v_zero [64][4] fp16 bits.  Any output may be
+ *   NULL to skip it. */
+int jfa_unpack_record(int32_t key_bits, int32_t val_bits, const void* record,
+                      uint8_t* k_codes, uint16_t* k_scale, uint16_t* k_zero,
+                      uint8_t* v_codes, uint16_t* v_scale, uint16_t* v_zero);
+
+/* Number of kernel launches one jfa_decode_step issues for a geometry
+ * (for launch accounting); 0 on a bad geometry. */
+int jfa_decode_step_launches(const jfa_geom* geom, int32_t k);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* JFA_H_ */

@@ -1,0 +1,142 @@
+"""CPU-side checks of the C ABI: the library loads, exports every symbol the
+header declares, reports layouts, rejects bad arguments before any CUDA
+work, and its record decoder is a bijection on the packed bits."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from bit_kv_cache_jfa_b200 import build
+    build.build()
+    from bit_kv_cache_jfa_b200 import _lib
+    return _lib
+
+
+def header_symbols():
+    text = open(os.path.join(ROOT, "include", "jfa.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(jfa_[a-z_]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(lib):
+    syms = header_symbols()
+    assert len(syms) >= 12
+    so = ctypes.CDLL(lib.LIB_PATH)
+    for s in syms:
+        assert hasattr(so, s), s
+        assert s in lib.SIGNATURES, s
+    assert sorted(lib.SIGNATURES) == syms
+
+
+def G(**kw):
+    from bit_kv_cache_jfa_b200 import Geom
+    d = dict(batch=2, num_heads=8, num_kv_heads=2, head_dim=128, capacity=4096, key_bits=3,
+             val_bits=2, n_ctx=100)
+    d.update(kw)
+    return Geom(**d)
+
+
+@pytest.mark.parametrize("kb,vb,rec", [(3, 2, 6656), (4, 4, 9728), (3, 4, 8704), (4, 2, 7680)])
+def test_cache_layout(lib, kb, vb, rec):
+    L = lib.jfa_cache_layout_get(G(key_bits=kb, val_bits=vb))
+    assert L.record_bytes == rec
+    # bytes per token per KV head: codes + scales (104 for K3V2, 152 for K4V4)
+    assert L.record_bytes == 64 * (128 * kb // 8 + 8 + 128 * vb // 8 + 16)
+    assert L.groups_bytes == 2 * 2 * (4096 // 64) * rec
+    assert L.tail_bytes == 2 * 2 * 64 * 128 * 2
+    assert (L.off_key_scales, L.off_key_codes) == (0, 512)
+    assert L.off_val_scales == 512 + 1024 * kb and L.off_val_codes == L.off_val_scales + 1024
+    for off in (L.off_key_codes, L.off_val_scales, L.off_val_codes):
+        assert off % 16 == 0
+
+
+def test_workspace_layout(lib):
+    a = lib.jfa_workspace_layout_get(G(), 64)
+    b = lib.jfa_workspace_layout_get(G(), 4096)
+    assert b.total_bytes > a.total_bytes
+    for L in (a, b):
+        offs = [L.off_flag, L.off_scores, L.off_partials, L.off_hist, L.off_cand, L.off_sel,
+                L.off_merge]
+        assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
+        assert L.off_counters == L.off_hist + 4 * 4 * 2048
+        assert L.off_scores + 4 * 4 * 4096 <= L.off_partials
+
+
+@pytest.mark.parametrize("bad", [dict(head_dim=64), dict(num_heads=12, num_kv_heads=1),
+                                 dict(num_heads=9), dict(capacity=100), dict(key_bits=2),
+                                 dict(val_bits=3), dict(n_ctx=5000), dict(batch=0)])
+def test_bad_geometry_rejected(lib, bad):
+    g = G(**bad)
+    assert lib.load().jfa_cache_layout_get(ctypes.byref(g), ctypes.byref(lib.CacheLayout())) == 1
+    c = lib.Cache(256, 512, 1024)
+    assert lib.jfa_pack_kv(g, c, 256, 256, 1, 256) == lib.JFA_ERR_INVALID_ARG
+    assert lib.jfa_decode_scores(g, c, 256, 0.1, 256) == lib.JFA_ERR_INVALID_ARG
+    assert lib.jfa_topk(g, 8, 256, 256) == lib.JFA_ERR_INVALID_ARG
+    assert lib.jfa_decode_step_launches(g, 8) == 0
+
+
+def test_bad_arguments_rejected_before_launch(lib):
+    g, c = G(), lib.Cache(256, 512, 1024)
+    inv = lib.JFA_ERR_INVALID_ARG
+    assert lib.jfa_pack_kv(g, lib.Cache(0, 512, 1024), 256, 256, 1, 256) == inv
+    assert lib.jfa_pack_kv(g, lib.Cache(257, 512, 1024), 256, 256, 1, 256) == inv  # misaligned
+    assert lib.jfa_pack_kv(g, c, 256, 256, 4000, 256) == inv                       # > capacity
+    assert lib.jfa_pack_kv(g, c, None, 256, 1, 256) == inv
+    assert lib.jfa_pack_kv(g, c, 256, 256, -1, 256) == inv
+    assert lib.jfa_decode_scores(g, c, 256, -1.0, 256) == inv
+    assert lib.jfa_decode_scores(G(n_ctx=0), c, 256, 0.1, 256) == inv
+    assert lib.jfa_topk(g, 0, 256, 256) == inv
+    assert lib.jfa_topk(g, 4097, 256, 256) == inv
+    assert lib.jfa_correct_merge(g, c, 256, 0.1, 256, 8, 256, 256, 0, 256, None) == inv
+    assert lib.jfa_correct_merge(g, c, 256, 0.1, None, 8, 256, 256, 0, 256, 256) == inv
+    assert lib.jfa_correct_merge(g, c, 256, 0.1, 256, 8, 258, 256, 0, 256, 256) == inv
+    assert lib.jfa_decode_step(g, c, 256, 0.1, 0, 256, 256, 256, 0, 256, 256) == inv
+    with pytest.raises(ctypes.ArgumentError):
+        lib.jfa_topk(g, 1.5, 256, 256)
+
+
+def test_launch_accounting(lib):
+    # scan + (memset, hist, collect, final) + (correct, merge)
+    assert lib.jfa_decode_step_launches(G(n_ctx=4096), 64) == 7
+    # k >= N_q: the top-k is a fill kernel
+    assert lib.jfa_decode_step_launches(G(n_ctx=100), 64) == 4
+    # N_q = 0: no scan
+    assert lib.jfa_decode_step_launches(G(n_ctx=64), 8) == 3
+
+
+def test_status_strings(lib):
+    assert lib.status_string(0) == "ok"
+    assert lib.status_string(4) == "device error flag set"
+
+
+@pytest.mark.parametrize("kb,vb", [(3, 2), (4, 4)])
+def test_record_decoder_is_a_bijection_on_bits(lib, kb, vb):
+    L = lib.jfa_cache_layout_get(G(key_bits=kb, val_bits=vb))
+    n = L.record_bytes
+    zero = bytes(n)
+    base = [a.copy() for a in lib.jfa_unpack_record(kb, vb, zero)]
+    assert all(int(a.max()) == 0 for a in base)
+    rng = np.random.default_rng(0)
+    seen = {}
+    # every bit of every section decodes into exactly one output element
+    bits = list(range(n * 8))
+    rng.shuffle(bits)
+    for bit in bits[:3000]:
+        rec = bytearray(n)
+        rec[bit // 8] = 1 << (bit % 8)
+        outs = lib.jfa_unpack_record(kb, vb, bytes(rec))
+        hits = [(i, tuple(np.argwhere(a != 0)[0])) for i, a in enumerate(outs) if a.any()]
+        assert len(hits) == 1 and sum(int(np.count_nonzero(a)) for a in outs) == 1, bit
+        i, pos = hits[0]
+        val = int(outs[i][pos])
+        assert val & (val - 1) == 0  # a single bit of one code / half
+        key = (i, pos, val)
+        assert key not in seen, (bit, seen.get(key))
+        seen[key] = bit

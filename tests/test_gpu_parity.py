@@ -1,0 +1,256 @@
+"""GPU parity: every C-ABI call against the fp64 oracle on the same seeded
+inputs (bit-exact for codes, scales, zeros, tails and top-k sets; fp
+outputs within max-abs 2e-3 and rel-L2 1e-3)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle.jfa_oracle as O
+import workloads as W
+from bit_kv_cache_jfa_b200 import _lib
+
+from jfa_testutil import (GpuRun, SCORE_ABS, assert_out_close, assert_topk_valid)
+
+pytestmark = pytest.mark.gpu
+
+TINY = W.WORKLOADS["tiny_k4v4_4k"]
+
+
+def small(kb=4, vb=4, heads=8, kv=2, ctx=4096, batch=1, topk=64, planted=16, seed=0,
+          lognormal=False):
+    return W.Workload(f"small_k{kb}v{vb}_g{heads // kv}", batch=batch, heads=heads, kv_heads=kv,
+                      ctx=ctx, key_bits=kb, val_bits=vb, topk=topk, planted=planted, seed=seed,
+                      value_lognormal=lognormal)
+
+
+def check_pack(run: GpuRun):
+    oc = run.oracle_cache()
+    torch.cuda.synchronize()
+    w = run.w
+    for b in range(w.batch):
+        for h in range(w.kv_heads):
+            for g in range(oc.n_quant // 64):
+                kc, ks, kz, vc, vs, vz = _lib.jfa_unpack_record(w.key_bits, w.val_bits,
+                                                               run.cache.record(b, h, g))
+                sl = slice(64 * g, 64 * g + 64)
+                assert np.array_equal(kc, oc.k_codes[b, h, sl]), (b, h, g, "key codes")
+                assert np.array_equal(ks, oc.k_scale[b, h, g].view(np.uint16)), (b, h, g)
+                assert np.array_equal(kz, oc.k_zero[b, h, g].view(np.uint16)), (b, h, g)
+                assert np.array_equal(vc, oc.v_codes[b, h, sl]), (b, h, g, "value codes")
+                assert np.array_equal(vs, oc.v_scale[b, h, sl].view(np.uint16)), (b, h, g)
+                assert np.array_equal(vz, oc.v_zero[b, h, sl].view(np.uint16)), (b, h, g)
+    t = run.ctx - oc.n_quant
+    tk = run.cache.tail_k[:, :, :t].cpu()
+    tv = run.cache.tail_v[:, :, :t].cpu()
+    assert torch.equal(tk, run.k_cpu[:, :, oc.n_quant:run.ctx])
+    assert torch.equal(tv, run.v_cpu[:, :, oc.n_quant:run.ctx])
+
+
+# ---------------------------------------------------------------- pack
+@pytest.mark.parametrize("kb,vb", [(4, 4), (3, 2), (3, 4), (4, 2)])
+def test_pack_bulk_bit_exact(kb, vb):
+    w = small(kb, vb, ctx=1000, batch=2, lognormal=True)
+    check_pack(GpuRun(w))
+
+
+def test_pack_appends_equal_bulk():
+    # ragged appends crossing group and tail boundaries, including 1-token steps
+    w = small(3, 2, ctx=777, batch=2)
+    chunks = [1, 63, 1, 64, 65, 2, 1, 200, 127, 129, 64, 60]
+    assert sum(chunks) == 777
+    check_pack(GpuRun(w, chunks=chunks))
+
+
+def test_pack_single_token_appends():
+    w = small(4, 4, ctx=200)
+    check_pack(GpuRun(w, chunks=[1] * 200))
+
+
+# ---------------------------------------------------------------- scores
+def scan_partials(run: GpuRun):
+    """Merge the scan's split partials on the host (log2 units)."""
+    g = run.cache.geom()
+    w = run.w
+    nq = run.cache.n_quant
+    ng = nq // 64
+    n_seg = w.batch * w.kv_heads
+    T = n_seg * ng
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    Wn = min(T, sms * 8, 2048)
+    L = run.ws.layout
+    G = w.group
+    part = run.ws.buf[L.off_partials:L.off_partials + 4 * L.partial_slots * G * 132]
+    part = part.view(torch.float32).view(L.partial_slots, G, 132).cpu().double().numpy()
+    res = {}
+    for seg in range(n_seg):
+        x0, x1 = seg * ng, seg * ng + ng - 1
+        w0, w1 = ((x0 + 1) * Wn - 1) // T, ((x1 + 1) * Wn - 1) // T
+        for j in range(G):
+            m, l, acc = -np.inf, 0.0, np.zeros(128)
+            for wi in range(w0, w1 + 1):
+                row = part[wi + seg, j]
+                mn = max(m, row[0])
+                l = l * 2.0 ** (m - mn) + row[1] * 2.0 ** (row[0] - mn)
+                acc = acc * 2.0 ** (m - mn) + row[4:] * 2.0 ** (row[0] - mn)
+                m = mn
+            res[(seg // w.kv_heads, (seg % w.kv_heads) * G + j)] = (m, l, acc)
+    return res
+
+
+@pytest.mark.parametrize("kb,vb,heads,kv", [(4, 4, 8, 2), (3, 2, 8, 2), (3, 2, 32, 8),
+                                            (4, 4, 32, 4), (3, 4, 8, 8), (4, 2, 4, 2)])
+def test_scores_and_scan_partials(kb, vb, heads, kv):
+    w = small(kb, vb, heads=heads, kv=kv, ctx=2100, batch=2, lognormal=True)
+    run = GpuRun(w)
+    run.scores()
+    s_gpu = run.selection_scores()
+    ref = run.oracle_step()
+    err = np.abs(s_gpu - ref.select).max()
+    assert err <= SCORE_ABS, err
+    parts = scan_partials(run)
+    for (b, hq), (m, l, acc) in parts.items():
+        pa = ref.approx_all[b][hq]
+        # same normalised aggregate and consistent mass
+        assert np.allclose(acc / l, O.finish(pa), rtol=1e-4, atol=1e-4)
+        assert abs(m / np.log2(np.e) - pa.m) < 1e-4
+        assert abs(l * 2.0 ** (m - pa.m * np.log2(np.e)) / pa.l - 1) < 1e-4
+
+
+# ---------------------------------------------------------------- top-k
+def write_scores(run: GpuRun, s: np.ndarray):
+    v = run.ws.scores(run.cache)
+    v[:, :, :s.shape[2]] = torch.from_numpy(s.astype(np.float32)).cuda()
+
+
+@pytest.mark.parametrize("nq_ctx,k,mode", [(4096, 64, "normal"), (4096, 1, "normal"),
+                                           (32768, 256, "normal"), (32768, 4096, "normal"),
+                                           (131072, 512, "normal"), (8192, 300, "ties"),
+                                           (40000, 100, "constant"), (70000, 2000, "few_values"),
+                                           (4096, 4031, "normal")])
+def test_topk_bit_exact_on_synthetic_scores(nq_ctx, k, mode):
+    w = small(4, 4, ctx=nq_ctx, batch=2, heads=8, kv=4)
+    run = GpuRun(w, k=k, chunks=[nq_ctx], kv=(torch.zeros(2, 4, nq_ctx, 128, dtype=torch.bfloat16),
+                                              torch.zeros(2, 4, nq_ctx, 128, dtype=torch.bfloat16)))
+    nq = run.cache.n_quant
+    rng = np.random.default_rng(nq_ctx + k)
+    if mode == "normal":
+        s = rng.standard_normal((2, 4, nq)) * 2
+    elif mode == "ties":
+        s = np.round(rng.standard_normal((2, 4, nq)) * 4) / 4
+    elif mode == "constant":     # every score equal: the lowest indices win; candidates overflow
+        s = np.full((2, 4, nq), 1.5)
+    else:                        # few distinct values, heavy ties at the threshold
+        s = rng.integers(0, 5, (2, 4, nq)).astype(np.float64) - 2.0
+    s = s.astype(np.float32)
+    write_scores(run, s)
+    run.topk()
+    got = run.idx.cpu().numpy()
+    ref = O.topk_indices(s.astype(np.float64), k)
+    assert np.array_equal(got, ref)
+
+
+def test_topk_k_at_least_nq_fills():
+    w = small(4, 4, ctx=300)
+    run = GpuRun(w, k=300)
+    run.topk()
+    got = run.idx.cpu().numpy()
+    nq = run.cache.n_quant
+    assert np.array_equal(got[0, 0], np.r_[np.arange(nq), -np.ones(300 - nq)])
+
+
+# ---------------------------------------------------------------- correct + merge
+@pytest.mark.parametrize("kb,vb,heads,kv,ctx,k", [(4, 4, 8, 2, 4096, 64), (3, 2, 32, 8, 3000, 128),
+                                                  (3, 2, 32, 4, 2048, 256), (4, 4, 8, 8, 1000, 7),
+                                                  (4, 2, 4, 1, 777, 33)])
+def test_correct_merge_with_oracle_index_set(kb, vb, heads, kv, ctx, k):
+    w = small(kb, vb, heads=heads, kv=kv, ctx=ctx, batch=2, topk=k, lognormal=True)
+    run = GpuRun(w)
+    ref = run.oracle_step()
+    run.scores()
+    oidx = torch.from_numpy(ref.idx.astype(np.int32)).cuda()
+    run.correct_merge(oidx)
+    torch.cuda.synchronize()
+    assert_out_close(run.out.cpu().numpy(), ref.out)
+
+
+@pytest.mark.parametrize("wl", ["tiny_k4v4_4k"])
+def test_end_to_end_tiny_workload(wl):
+    w = W.WORKLOADS[wl]
+    run = GpuRun(w)
+    out, idx = run.step()
+    ref = run.oracle_step()
+    assert_topk_valid(idx, ref.select, w.topk)
+    assert_out_close(out, run.oracle_step(idx=idx).out)
+    assert_out_close(out, ref.out)
+    # planted tokens are found
+    pos = set(W.planted_positions(w, 0).tolist())
+    for h in range(w.kv_heads):
+        assert pos <= set(idx[0, h].tolist())
+
+
+@pytest.mark.parametrize("kb,vb,heads,kv,ctx,k,batch", [(3, 2, 32, 8, 5000, 256, 2),
+                                                        (4, 4, 32, 4, 4500, 96, 3),
+                                                        (3, 2, 64, 8, 3333, 256, 1)])
+def test_end_to_end_no_planted(kb, vb, heads, kv, ctx, k, batch):
+    # without planted tokens the bulk of the distribution carries the output
+    w = small(kb, vb, heads=heads, kv=kv, ctx=ctx, batch=batch, topk=k, planted=0, seed=5)
+    run = GpuRun(w)
+    out, idx = run.step()
+    ref = run.oracle_step()
+    assert_topk_valid(idx, ref.select, k)
+    assert_out_close(out, run.oracle_step(idx=idx).out)
+    assert_out_close(out, ref.out)
+
+
+def test_host_resident_rows_match_device_rows():
+    w = small(4, 4, heads=32, kv=8, ctx=3000, batch=2, topk=128)
+    a = GpuRun(w)
+    b = GpuRun(w, exact_on_host=True)
+    oa, ia = a.step()
+    ob, ib = b.step()
+    assert np.array_equal(ia, ib)
+    assert np.array_equal(oa, ob)
+
+
+# ---------------------------------------------------------------- edge cases
+@pytest.mark.parametrize("ctx", [1, 37, 64, 65, 127, 128, 129, 191])
+def test_short_contexts(ctx):
+    w = small(3, 2, heads=8, kv=2, ctx=ctx, batch=2, topk=16, planted=0)
+    run = GpuRun(w)
+    out, idx = run.step()
+    ref = run.oracle_step()
+    assert np.array_equal(idx, ref.idx)
+    assert_out_close(out, ref.out)
+
+
+def test_k_at_least_nq_is_exact_attention():
+    w = small(4, 4, heads=8, kv=2, ctx=700, batch=1, topk=700)
+    run = GpuRun(w)
+    out, idx = run.step()
+    ref = O.exact_attention(run.q_cpu.double().numpy(), run.k_cpu.double().numpy(),
+                            run.v_cpu.double().numpy(), 700, run.scale)
+    assert_out_close(out, ref)
+
+
+def test_bad_index_sets_device_flag_without_fault():
+    w = small(4, 4, ctx=600, topk=8)
+    run = GpuRun(w)
+    run.scores()
+    bad = torch.full((1, 2, 8), -1, dtype=torch.int32, device="cuda")
+    bad[0, 0, 0] = 10_000_000
+    bad[0, 1, 0] = 5
+    run.correct_merge(bad)
+    st, flag = _lib.jfa_check_error(run.cache.geom(), run.ws.buf)
+    assert st == _lib.JFA_ERR_DEVICE and flag & _lib.DEVERR_BAD_INDEX
+    _lib.check(_lib.jfa_clear_error(run.cache.geom(), run.ws.buf), "clear")
+    st, flag = _lib.jfa_check_error(run.cache.geom(), run.ws.buf)
+    assert st == 0 and flag == 0
+
+
+def test_capacity_larger_than_context():
+    w = small(3, 2, heads=32, kv=8, ctx=1500, batch=2, topk=100)
+    run = GpuRun(w, capacity=4096)
+    out, idx = run.step()
+    ref = run.oracle_step()
+    assert_topk_valid(idx, ref.select, 100)
+    assert_out_close(out, run.oracle_step(idx=idx).out)

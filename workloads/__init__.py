@@ -194,3 +194,37 @@ def sample_segments(w: Workload, n: int, seed: int = 0) -> list[tuple[int, int]]
 
 def default_scale(w: Workload) -> float:
     return 1.0 / math.sqrt(w.head_dim)
+
+
+def gen_kv_device(w: Workload, device, q: torch.Tensor | None = None,
+                  ctx: int | None = None) -> tuple[torch.Tensor, torch.Tensor]:
+    """Same recipe as gen_kv, drawn with the device's generator (fast for large
+    workloads).  Values differ from the CPU stream but are deterministic for
+    a given seed; parity checks copy the sampled segments back to the host."""
+    n = w.ctx if ctx is None else ctx
+    d = w.head_dim
+    if q is None:
+        q = gen_q(w)
+    qd = q.to(device)
+    k = torch.empty(w.batch, w.kv_heads, n, d, dtype=torch.bfloat16, device=device)
+    v = torch.empty_like(k)
+    outl = outlier_channels(w).to(device)
+    g = torch.Generator(device=device)
+    for b in range(w.batch):
+        pos = planted_positions(w, b)
+        pos = pos[pos < n].to(device)
+        for h in range(w.kv_heads):
+            g.manual_seed(_mix(w.seed, 6, b, h) & 0x7FFF_FFFF_FFFF_FFFF)
+            kk = torch.randn(n, d, generator=g, device=device)
+            kk[:, outl] *= 10.0
+            if pos.numel():
+                j = torch.arange(pos.numel(), device=device)
+                src = qd[b, h * w.group + (j % w.group)].float()
+                kk[pos] = 3.0 * src + 0.5 * torch.randn(pos.numel(), d, generator=g,
+                                                        device=device)
+            vv = torch.randn(n, d, generator=g, device=device)
+            if w.value_lognormal:
+                vv *= torch.exp(0.5 * torch.randn(n, 1, generator=g, device=device))
+            k[b, h] = kk.to(torch.bfloat16)
+            v[b, h] = vv.to(torch.bfloat16)
+    return k, v
