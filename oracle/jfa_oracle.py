@@ -256,8 +256,9 @@ def topk_indices(scores, k: int) -> np.ndarray:
     k > row length.  scores [..., N] -> int32 [..., k]."""
     scores = np.asarray(scores)
     *lead, n = scores.shape
-    flat = scores.reshape(-1, n)
-    out = np.full((flat.shape[0], k), -1, dtype=np.int32)
+    rows = int(np.prod(lead)) if lead else 1
+    flat = scores.reshape(rows, n)
+    out = np.full((rows, k), -1, dtype=np.int32)
     keff = min(k, n)
     idx = np.arange(n)
     for r in range(flat.shape[0]):

@@ -320,3 +320,9 @@ def test_pins_reject_wrong_merge_sign(monkeypatch):
     monkeypatch.setattr(O, "merge", bad_merge)
     with pytest.raises(AssertionError):
         test_k_zero_is_attention_over_dequantized_plus_exact_tail(4, 4)
+
+
+def test_topk_empty_rows_pad_with_minus_one():
+    # N_q = 0 (context within the tail): no quantized token can be chosen
+    out = O.topk_indices(np.zeros((2, 3, 0)), 4)
+    assert out.shape == (2, 3, 4) and np.all(out == -1)
