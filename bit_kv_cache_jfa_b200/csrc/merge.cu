@@ -44,10 +44,9 @@ struct MergeParams {
 
 __device__ __forceinline__ float bf16f(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
 
-__device__ __forceinline__ float quant_dequant(float x, const uint8_t* rec, int soff, int zoff,
-                                               int bits) {
-  const float s = __half2float(__ushort_as_half(*reinterpret_cast<const uint16_t*>(rec + soff)));
-  const float z = __half2float(__ushort_as_half(*reinterpret_cast<const uint16_t*>(rec + zoff)));
+__device__ __forceinline__ float quant_dequant_bits(float x, uint16_t sb, uint16_t zb, int bits) {
+  const float s = __half2float(__ushort_as_half(sb));
+  const float z = __half2float(__ushort_as_half(zb));
   double c = 0.0;
   if (s != 0.f) {
     c = rint(((double)x - (double)z) / (double)s);
@@ -89,86 +88,93 @@ struct OnlineState {
   }
 };
 
-// merge partial (mb, lb, ab[4]) into (m, l, a[4])
-__device__ __forceinline__ void merge_into(float& m, float& l, float* a, float mb, float lb,
-                                           const float* ab) {
-  if (mb == -INFINITY || lb == 0.f) return;
-  if (m == -INFINITY || l == 0.f) {
-    m = mb;
-    l = lb;
-    a[0] = ab[0];
-    a[1] = ab[1];
-    a[2] = ab[2];
-    a[3] = ab[3];
-    return;
-  }
-  const float mn = fmaxf(m, mb);
-  const float sa = exp2f(m - mn), sb = exp2f(mb - mn);
-  l = l * sa + lb * sb;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) a[i] = a[i] * sa + ab[i] * sb;
-  m = mn;
-}
-
-// grid (n_chunks, n_seg), 4 warps; warp w handles tokens chunk*32 + w*8 + i
+// grid (n_chunks, n_seg), 4 warps; warp w handles tokens chunk*32 + w*8 + i,
+// in two batches of four whose loads are all issued before any use.
+template <int G>
 __global__ void __launch_bounds__(128) correct_chunk_kernel(const MergeParams p) {
-  __shared__ float red[4][2][kMaxG][kPartStride];
+  __shared__ float red[4][2][G][kPartStride];
   const int seg = blockIdx.y, chunk = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = seg / p.hkv, h = seg % p.hkv;
   const int c0 = 4 * lane;
-  const int G = p.G;
+  const int jv = lane >> 3;  // channels 4*lane.. lie in value group lane/8
 
-  float q[kMaxG][4];
+  float q[G][4];
 #pragma unroll
-  for (int j = 0; j < kMaxG; ++j) {
-    if (j < G) {
-      const uint2 w = *reinterpret_cast<const uint2*>(p.q + ((size_t)b * p.H + h * G + j) * kD + c0);
-      q[j][0] = __uint_as_float(w.x << 16);
-      q[j][1] = __uint_as_float(w.x & 0xFFFF0000u);
-      q[j][2] = __uint_as_float(w.y << 16);
-      q[j][3] = __uint_as_float(w.y & 0xFFFF0000u);
-    } else {
-      q[j][0] = q[j][1] = q[j][2] = q[j][3] = 0.f;
-    }
+  for (int j = 0; j < G; ++j) {
+    const uint2 w = *reinterpret_cast<const uint2*>(p.q + ((size_t)b * p.H + h * G + j) * kD + c0);
+    q[j][0] = __uint_as_float(w.x << 16);
+    q[j][1] = __uint_as_float(w.x & 0xFFFF0000u);
+    q[j][2] = __uint_as_float(w.y << 16);
+    q[j][3] = __uint_as_float(w.y & 0xFFFF0000u);
   }
-  OnlineState ex[kMaxG], rm[kMaxG];
+  OnlineState ex[G], rm[G];
 #pragma unroll
-  for (int j = 0; j < kMaxG; ++j) {
+  for (int j = 0; j < G; ++j) {
     ex[j].init();
     rm[j].init();
   }
+  const int ks_s0 = off_ks() + ks_scale_off(c0), ks_s1 = off_ks() + ks_scale_off(c0 + 2);
+  const int ks_z0 = off_ks() + ks_zero_off(c0), ks_z1 = off_ks() + ks_zero_off(c0 + 2);
 
-  for (int i = 0; i < kMergeChunk / 4; ++i) {
-    const int e = chunk * kMergeChunk + warp * (kMergeChunk / 4) + i;
-    int t = -1;
-    bool quant = false;
-    const uint16_t *kr = nullptr, *vr = nullptr;
+  const int e_base = chunk * kMergeChunk + warp * (kMergeChunk / 4);
+  // token ids of this warp's 8 entries (lane i < 8 resolves entry i)
+  int my_t = -1;
+  if (lane < 8) {
+    const int e = e_base + lane;
     if (e < p.k) {
-      t = p.idx[(size_t)seg * p.k + e];
-      if (t >= p.nq) {
-        if (lane == 0) set_flag(p.flag, JFA_DEVERR_BAD_INDEX);
-        t = -1;
-      }
-      if (t >= 0) {
-        quant = true;
-        kr = p.k_exact + ((size_t)seg * p.capacity + t) * kD;
-        vr = p.v_exact + ((size_t)seg * p.capacity + t) * kD;
+      my_t = p.idx[(size_t)seg * p.k + e];
+      if (my_t >= p.nq) {
+        set_flag(p.flag, JFA_DEVERR_BAD_INDEX);
+        my_t = -1;
       }
     } else if (e - p.k < p.tail) {
-      const int tt = e - p.k;
-      t = p.nq + tt;
-      kr = p.tail_k + ((size_t)seg * kTail + tt) * kD;
-      vr = p.tail_v + ((size_t)seg * kTail + tt) * kD;
+      my_t = (1 << 30) | (e - p.k);  // tail slot
     }
-    if (kr == nullptr) continue;  // warp-uniform
-    const uint2 kw = *reinterpret_cast<const uint2*>(kr + c0);
-    const uint2 vw = *reinterpret_cast<const uint2*>(vr + c0);
-    float kx[4] = {bf16f(kw.x & 0xFFFFu), bf16f(kw.x >> 16), bf16f(kw.y & 0xFFFFu), bf16f(kw.y >> 16)};
-    float vx[4] = {bf16f(vw.x & 0xFFFFu), bf16f(vw.x >> 16), bf16f(vw.y & 0xFFFFu), bf16f(vw.y >> 16)};
+  }
 #pragma unroll
-    for (int j = 0; j < kMaxG; ++j) {
-      if (j < G) {
+  for (int half = 0; half < 2; ++half) {
+    int tk[4];
+    uint2 kw[4], vw[4];
+    uint32_t s01[4], s23[4], z01[4], z23[4];
+    uint16_t vsb[4], vzb[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      tk[i] = __shfl_sync(kAll, my_t, half * 4 + i);
+      kw[i] = vw[i] = make_uint2(0u, 0u);
+      s01[i] = s23[i] = z01[i] = z23[i] = 0u;
+      vsb[i] = vzb[i] = 0;
+      if (tk[i] < 0) continue;
+      const uint16_t *kr, *vr;
+      if (tk[i] & (1 << 30)) {
+        const int tt = tk[i] & ~(1 << 30);
+        kr = p.tail_k + ((size_t)seg * kTail + tt) * kD;
+        vr = p.tail_v + ((size_t)seg * kTail + tt) * kD;
+      } else {
+        const int t = tk[i];
+        kr = p.k_exact + ((size_t)seg * p.capacity + t) * kD;
+        vr = p.v_exact + ((size_t)seg * p.capacity + t) * kD;
+        const uint8_t* rec = p.groups + ((size_t)seg * p.ng_cap + t / kKG) * p.rec_bytes;
+        s01[i] = *reinterpret_cast<const uint32_t*>(rec + ks_s0);
+        s23[i] = *reinterpret_cast<const uint32_t*>(rec + ks_s1);
+        z01[i] = *reinterpret_cast<const uint32_t*>(rec + ks_z0);
+        z23[i] = *reinterpret_cast<const uint32_t*>(rec + ks_z1);
+        const int vb = off_vs(p.key_bits);
+        vsb[i] = *reinterpret_cast<const uint16_t*>(rec + vb + vs_scale_off(t % kKG, jv));
+        vzb[i] = *reinterpret_cast<const uint16_t*>(rec + vb + vs_zero_off(t % kKG, jv));
+      }
+      kw[i] = *reinterpret_cast<const uint2*>(kr + c0);
+      vw[i] = *reinterpret_cast<const uint2*>(vr + c0);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      if (tk[i] < 0) continue;  // warp-uniform
+      const float kx[4] = {bf16f(kw[i].x & 0xFFFFu), bf16f(kw[i].x >> 16), bf16f(kw[i].y & 0xFFFFu),
+                           bf16f(kw[i].y >> 16)};
+      const float vx[4] = {bf16f(vw[i].x & 0xFFFFu), bf16f(vw[i].x >> 16), bf16f(vw[i].y & 0xFFFFu),
+                           bf16f(vw[i].y >> 16)};
+#pragma unroll
+      for (int j = 0; j < G; ++j) {
         float d = q[j][0] * kx[0];
         d = fmaf(q[j][1], kx[1], d);
         d = fmaf(q[j][2], kx[2], d);
@@ -176,23 +182,19 @@ __global__ void __launch_bounds__(128) correct_chunk_kernel(const MergeParams p)
         d = warp_sum(d);
         ex[j].add(d * p.kappa, vx);
       }
-    }
-    if (quant) {
-      const int g = t / kKG, tl = t % kKG;
-      const uint8_t* rec = p.groups + ((size_t)seg * p.ng_cap + g) * p.rec_bytes;
-      float kh[4], vh[4];
-      const int jv = lane >> 3;  // channels 4*lane.. lie in value group lane/8
-      const int vso = off_vs(p.key_bits) + vs_scale_off(tl, jv);
-      const int vzo = off_vs(p.key_bits) + vs_zero_off(tl, jv);
+      if (!(tk[i] & (1 << 30))) {
+        const uint16_t ksb[4] = {(uint16_t)(s01[i] & 0xFFFFu), (uint16_t)(s01[i] >> 16),
+                                 (uint16_t)(s23[i] & 0xFFFFu), (uint16_t)(s23[i] >> 16)};
+        const uint16_t kzb[4] = {(uint16_t)(z01[i] & 0xFFFFu), (uint16_t)(z01[i] >> 16),
+                                 (uint16_t)(z23[i] & 0xFFFFu), (uint16_t)(z23[i] >> 16)};
+        float kh[4], vh[4];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        kh[c] = quant_dequant(kx[c], rec, off_ks() + ks_scale_off(c0 + c),
-                              off_ks() + ks_zero_off(c0 + c), p.key_bits);
-        vh[c] = quant_dequant(vx[c], rec, vso, vzo, p.val_bits);
-      }
+        for (int c = 0; c < 4; ++c) {
+          kh[c] = quant_dequant_bits(kx[c], ksb[c], kzb[c], p.key_bits);
+          vh[c] = quant_dequant_bits(vx[c], vsb[i], vzb[i], p.val_bits);
+        }
 #pragma unroll
-      for (int j = 0; j < kMaxG; ++j) {
-        if (j < G) {
+        for (int j = 0; j < G; ++j) {
           float d = q[j][0] * kh[0];
           d = fmaf(q[j][1], kh[1], d);
           d = fmaf(q[j][2], kh[2], d);
@@ -205,43 +207,41 @@ __global__ void __launch_bounds__(128) correct_chunk_kernel(const MergeParams p)
   }
   // combine the 4 warps
 #pragma unroll
-  for (int j = 0; j < kMaxG; ++j) {
-    if (j < G) {
-      float* re = red[warp][0][j];
-      float* rr = red[warp][1][j];
-      if (lane == 0) {
-        re[0] = ex[j].m;
-        re[1] = ex[j].l;
-        rr[0] = rm[j].m;
-        rr[1] = rm[j].l;
-      }
+  for (int j = 0; j < G; ++j) {
+    float* re = red[warp][0][j];
+    float* rr = red[warp][1][j];
+    if (lane == 0) {
+      re[0] = ex[j].m;
+      re[1] = ex[j].l;
+      rr[0] = rm[j].m;
+      rr[1] = rm[j].l;
+    }
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        re[4 + c0 + c] = ex[j].a[c];
-        rr[4 + c0 + c] = rm[j].a[c];
-      }
+    for (int c = 0; c < 4; ++c) {
+      re[4 + c0 + c] = ex[j].a[c];
+      rr[4 + c0 + c] = rm[j].a[c];
     }
   }
   __syncthreads();
-  // thread tid: channel tid; loop over (part, head)
-  const int c = threadIdx.x;
+  const int c = threadIdx.x;  // channel
+#pragma unroll
   for (int part = 0; part < 2; ++part) {
+#pragma unroll
     for (int j = 0; j < G; ++j) {
-      float m = -INFINITY, l = 0.f, a = 0.f;
-      for (int w = 0; w < 4; ++w) {
-        const float mb = red[w][part][j][0], lb = red[w][part][j][1];
-        if (mb == -INFINITY || lb == 0.f) continue;
-        const float ab = red[w][part][j][4 + c];
-        if (m == -INFINITY) {
-          m = mb;
-          l = lb;
-          a = ab;
-        } else {
-          const float mn = fmaxf(m, mb);
-          const float sa = exp2f(m - mn), sb = exp2f(mb - mn);
-          l = l * sa + lb * sb;
-          a = a * sa + ab * sb;
-          m = mn;
+      float m = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < 4; ++w)
+        if (red[w][part][j][1] > 0.f) m = fmaxf(m, red[w][part][j][0]);
+      float l = 0.f, a = 0.f;
+      if (m > -INFINITY) {
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          const float lb = red[w][part][j][1];
+          if (lb > 0.f) {
+            const float sc = exp2f(red[w][part][j][0] - m);
+            l = fmaf(lb, sc, l);
+            a = fmaf(red[w][part][j][4 + c], sc, a);
+          }
         }
       }
       float* dst = p.chunk_part +
@@ -255,37 +255,72 @@ __global__ void __launch_bounds__(128) correct_chunk_kernel(const MergeParams p)
   }
 }
 
-// grid n_seg, one warp per query head of the segment
-__global__ void __launch_bounds__(256) merge_final_kernel(const MergeParams p) {
+// Merge all partials of (segment, head): max first, then independent sums,
+// so every partial's loads are in flight together.
+template <int G>
+__global__ void __launch_bounds__(32 * G) merge_final_kernel(const MergeParams p) {
   const int seg = blockIdx.x;
   const int j = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (j >= p.G) return;
   const int c0 = 4 * lane;
-  // approximate total over the scan slots of this segment
-  float ma = -INFINITY, la = 0.f, aa[4] = {0.f, 0.f, 0.f, 0.f};
+  long long w0 = 0, w1 = -1;
   if (p.ng > 0) {
     const long long T = p.scan_total, W = p.scan_warps;
     const long long x0 = (long long)seg * p.ng, x1 = x0 + p.ng - 1;
-    const long long w0 = scan_warp_of(x0, W, T), w1 = scan_warp_of(x1, W, T);
-    for (long long w = w0; w <= w1; ++w) {
-      const float* row = p.scan_part + ((size_t)(w + seg) * p.G + j) * kPartStride;
-      const float4 av = *reinterpret_cast<const float4*>(row + 4 + c0);
-      const float ab[4] = {av.x, av.y, av.z, av.w};
-      merge_into(ma, la, aa, row[0], row[1], ab);
-    }
+    w0 = scan_warp_of(x0, W, T);
+    w1 = scan_warp_of(x1, W, T);
   }
-  // exact and removal totals over the chunks
-  float me = -INFINITY, le = 0.f, ae[4] = {0.f, 0.f, 0.f, 0.f};
-  float mr = -INFINITY, lr = 0.f, ar[4] = {0.f, 0.f, 0.f, 0.f};
+  const int ns = (int)(w1 - w0 + 1);
+  auto srow = [&](int i) { return p.scan_part + ((size_t)(w0 + i + seg) * G + j) * kPartStride; };
+  auto crow = [&](int ch, int part) {
+    return p.chunk_part + ((((size_t)seg * p.n_chunks + ch) * 2 + part) * G + j) * kPartStride;
+  };
+  // pass 1: maxima
+  float ma = -INFINITY, me = -INFINITY, mr = -INFINITY;
+  for (int i = 0; i < ns; ++i) {
+    const float2 ml = *reinterpret_cast<const float2*>(srow(i));
+    if (ml.y > 0.f) ma = fmaxf(ma, ml.x);
+  }
   for (int ch = 0; ch < p.n_chunks; ++ch) {
-    const float* pe = p.chunk_part + ((((size_t)seg * p.n_chunks + ch) * 2 + 0) * p.G + j) * kPartStride;
-    const float* pr = p.chunk_part + ((((size_t)seg * p.n_chunks + ch) * 2 + 1) * p.G + j) * kPartStride;
-    const float4 ev = *reinterpret_cast<const float4*>(pe + 4 + c0);
-    const float4 rv = *reinterpret_cast<const float4*>(pr + 4 + c0);
-    const float eb[4] = {ev.x, ev.y, ev.z, ev.w};
-    const float rb[4] = {rv.x, rv.y, rv.z, rv.w};
-    merge_into(me, le, ae, pe[0], pe[1], eb);
-    merge_into(mr, lr, ar, pr[0], pr[1], rb);
+    const float2 e = *reinterpret_cast<const float2*>(crow(ch, 0));
+    const float2 r = *reinterpret_cast<const float2*>(crow(ch, 1));
+    if (e.y > 0.f) me = fmaxf(me, e.x);
+    if (r.y > 0.f) mr = fmaxf(mr, r.x);
+  }
+  // pass 2: sums in the frames of those maxima
+  float la = 0.f, le = 0.f, lr = 0.f;
+  float aa[4] = {0.f, 0.f, 0.f, 0.f}, ae[4] = {0.f, 0.f, 0.f, 0.f}, ar[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+  for (int i = 0; i < ns; ++i) {
+    const float* row = srow(i);
+    const float2 ml = *reinterpret_cast<const float2*>(row);
+    const float4 v = *reinterpret_cast<const float4*>(row + 4 + c0);
+    const float sc = ml.y > 0.f ? exp2f(ml.x - ma) : 0.f;
+    la = fmaf(ml.y, sc, la);
+    aa[0] = fmaf(v.x, sc, aa[0]);
+    aa[1] = fmaf(v.y, sc, aa[1]);
+    aa[2] = fmaf(v.z, sc, aa[2]);
+    aa[3] = fmaf(v.w, sc, aa[3]);
+  }
+#pragma unroll 4
+  for (int ch = 0; ch < p.n_chunks; ++ch) {
+    const float* re = crow(ch, 0);
+    const float* rr = crow(ch, 1);
+    const float2 e = *reinterpret_cast<const float2*>(re);
+    const float2 r = *reinterpret_cast<const float2*>(rr);
+    const float4 ev = *reinterpret_cast<const float4*>(re + 4 + c0);
+    const float4 rv = *reinterpret_cast<const float4*>(rr + 4 + c0);
+    const float se = e.y > 0.f ? exp2f(e.x - me) : 0.f;
+    const float sr = r.y > 0.f ? exp2f(r.x - mr) : 0.f;
+    le = fmaf(e.y, se, le);
+    lr = fmaf(r.y, sr, lr);
+    ae[0] = fmaf(ev.x, se, ae[0]);
+    ae[1] = fmaf(ev.y, se, ae[1]);
+    ae[2] = fmaf(ev.z, se, ae[2]);
+    ae[3] = fmaf(ev.w, se, ae[3]);
+    ar[0] = fmaf(rv.x, sr, ar[0]);
+    ar[1] = fmaf(rv.y, sr, ar[1]);
+    ar[2] = fmaf(rv.z, sr, ar[2]);
+    ar[3] = fmaf(rv.w, sr, ar[3]);
   }
   // remainder = approximate total minus the removed top-k terms (m_a frame)
   float lrest = la, arest[4] = {aa[0], aa[1], aa[2], aa[3]};
@@ -302,15 +337,20 @@ __global__ void __launch_bounds__(256) merge_final_kernel(const MergeParams p) {
     wl = exp2f(me - m);
     wa = exp2f(ma - m);
   }
-  const float den = le * wl + lrest * wa;
-  const float inv = 1.f / den;
+  const float inv = 1.f / (le * wl + lrest * wa);
   float4 o;
   o.x = (ae[0] * wl + arest[0] * wa) * inv;
   o.y = (ae[1] * wl + arest[1] * wa) * inv;
   o.z = (ae[2] * wl + arest[2] * wa) * inv;
   o.w = (ae[3] * wl + arest[3] * wa) * inv;
   const int b = seg / p.hkv, h = seg % p.hkv;
-  *reinterpret_cast<float4*>(p.out + ((size_t)b * p.H + h * p.G + j) * kD + c0) = o;
+  *reinterpret_cast<float4*>(p.out + ((size_t)b * p.H + h * G + j) * kD + c0) = o;
+}
+
+template <int G>
+static void launch_cm_t(const MergeParams& p, int n_seg, cudaStream_t st) {
+  correct_chunk_kernel<G><<<dim3(p.n_chunks, n_seg), 128, 0, st>>>(p);
+  merge_final_kernel<G><<<n_seg, 32 * G, 0, st>>>(p);
 }
 
 int launch_correct_merge(const jfa_geom& g, const jfa_cache& c, const uint16_t* q, float scale,
@@ -349,8 +389,16 @@ int launch_correct_merge(const jfa_geom& g, const jfa_cache& c, const uint16_t* 
   p.scan_warps = plan.n_warps;
   p.ng = plan.ng;
   p.kappa = scale * 1.4426950408889634f;
-  correct_chunk_kernel<<<dim3(p.n_chunks, n_seg), 128, 0, st>>>(p);
-  merge_final_kernel<<<n_seg, 32 * p.G, 0, st>>>(p);
+  switch (p.G) {
+    case 1: launch_cm_t<1>(p, n_seg, st); break;
+    case 2: launch_cm_t<2>(p, n_seg, st); break;
+    case 3: launch_cm_t<3>(p, n_seg, st); break;
+    case 4: launch_cm_t<4>(p, n_seg, st); break;
+    case 5: launch_cm_t<5>(p, n_seg, st); break;
+    case 6: launch_cm_t<6>(p, n_seg, st); break;
+    case 7: launch_cm_t<7>(p, n_seg, st); break;
+    default: launch_cm_t<8>(p, n_seg, st); break;
+  }
   return cudaGetLastError() == cudaSuccess ? JFA_OK : JFA_ERR_CUDA;
 }
 

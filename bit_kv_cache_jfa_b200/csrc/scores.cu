@@ -14,12 +14,16 @@
 // the dequantized values v_hat = s_v * v' + m_v (v' codes exact in fp16):
 //   sum_t p_t v_hat[t][c] = sum_t (p_t s_v[t][j]) v'[t][c] + sum_t p_t m_v[t][j]
 // as an MMA with A = value codes (rows = channels, columns = tokens) and
-// B = fp16(p * s_v) (columns = heads), plus a small MMA whose A rows are the
-// value zeros of the four channel groups and a row of ones (giving sum p).
+// B = p * s_v (columns = heads), plus a small MMA whose A rows are the value
+// zeros of the four channel groups and a row of ones (giving sum p).  Both
+// B operands enter as an fp16 pair (rounded value, rounding remainder) in two
+// MMAs, so each token's weight carries ~22 bits: the correction step later
+// subtracts the top-k tokens' terms, and a plain fp16 weight would leave a
+// 2^-12 residue of the largest weights in the output.
 //
 // Work split: W warps (8 per CTA, one CTA per SM) take balanced contiguous
 // ranges of the flattened (segment, group) list.  Each warp streams its
-// records through a private two-stage shared-memory ring filled by
+// records through a private two- or three-stage shared-memory ring filled by
 // cp.async.bulk (one bulk copy per 6.5-9.5 KB record, completion on an
 // mbarrier) and writes one softmax partial per segment it touched.
 #include "jfa_internal.cuh"
@@ -50,8 +54,17 @@ constexpr float kLn2 = 0.6931471805599453f;
 constexpr unsigned kFull = 0xFFFFFFFFu;
 
 template <int KB, int VB>
+struct ScanCfg {
+  static constexpr int REC = 512 + 1024 * KB + 1024 + 1024 * VB;
+  // three ring stages per warp when they fit in shared memory, else two
+  static constexpr int STAGES = (kScanWarps * 3 * REC + 1024 <= 227 * 1024) ? 3 : 2;
+  static constexpr int SMEM = kScanWarps * STAGES * REC + kScanWarps * STAGES * 8;
+};
+
+template <int KB, int VB>
 __global__ void __launch_bounds__(kScanWarps * 32, 1) scan_kernel(const ScanParams p) {
-  constexpr int REC = 512 + 1024 * KB + 1024 + 1024 * VB;
+  constexpr int REC = ScanCfg<KB, VB>::REC;
+  constexpr int S = ScanCfg<KB, VB>::STAGES;
   constexpr int OFF_KC = 512;
   constexpr int OFF_VS = 512 + 1024 * KB;
   constexpr int OFF_VC = OFF_VS + 1024;
@@ -65,26 +78,31 @@ __global__ void __launch_bounds__(kScanWarps * 32, 1) scan_kernel(const ScanPara
   const long long g0 = scan_range_begin(wg, W, T), g1 = scan_range_begin(wg + 1, W, T);
   if (g0 >= g1) return;
 
-  uint8_t* ring = smem + (size_t)warp * 2 * REC;
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + (size_t)kScanWarps * 2 * REC) + warp * 2;
+  uint8_t* ring = smem + (size_t)warp * S * REC;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + (size_t)kScanWarps * S * REC) + warp * S;
   const uint64_t pol = policy_evict_first();
   if (lane == 0) {
-    mbar_init(&bar[0], 1);
-    mbar_init(&bar[1], 1);
+#pragma unroll
+    for (int i = 0; i < S; ++i) mbar_init(&bar[i], 1);
     fence_mbar_init();
   }
   __syncwarp();
-  auto rec_ptr = [&](long long gi) -> const uint8_t* {
-    long long seg = gi / p.ng, g = gi - seg * p.ng;
-    return p.groups + ((size_t)seg * p.ng_cap + (size_t)g) * REC;
+  // prefetch cursor (segment, group) of the next record to request
+  long long pf_seg = g0 / p.ng;
+  int pf_g = (int)(g0 - pf_seg * p.ng);
+  auto issue_next = [&](int stage) {
+    mbar_expect_tx(&bar[stage], REC);
+    bulk_g2s(ring + stage * REC, p.groups + ((size_t)pf_seg * p.ng_cap + (size_t)pf_g) * REC,
+             REC, &bar[stage], pol);
+    if (++pf_g == p.ng) {
+      pf_g = 0;
+      ++pf_seg;
+    }
   };
   if (lane == 0) {
-    for (int s = 0; s < 2; ++s) {
-      if (g0 + s < g1) {
-        mbar_expect_tx(&bar[s], REC);
-        bulk_g2s(ring + s * REC, rec_ptr(g0 + s), REC, &bar[s], pol);
-      }
-    }
+#pragma unroll
+    for (int i = 0; i < S; ++i)
+      if (g0 + i < g1) issue_next(i);
   }
 
   const bool head_ok = gid < p.G;
@@ -143,24 +161,28 @@ __global__ void __launch_bounds__(kScanWarps * 32, 1) scan_kernel(const ScanPara
     }
   };
 
+  long long seg = g0 / p.ng;
+  int g = (int)(g0 - seg * p.ng);
+  int st = 0;
+  uint32_t par = 0;
   for (long long gi = g0; gi < g1; ++gi) {
-    const long long seg = gi / p.ng;
-    const int g = (int)(gi - seg * p.ng);
     if (seg != cur) {
       if (cur >= 0) flush(cur);
       reset(seg);
       cur = seg;
     }
-    const int it = (int)(gi - g0);
-    const int st = it & 1;
-    const uint32_t par = (uint32_t)(it >> 1) & 1u;
     const bool ok = __all_sync(kFull, mbar_wait_bounded(&bar[st], par));
     if (!ok) {
       if (lane == 0) {
         set_flag(p.flag, JFA_DEVERR_TIMEOUT);
         // drain the copies still in flight before leaving (bounded)
-        mbar_wait_bounded(&bar[st], par);
-        if (gi + 1 < g1) mbar_wait_bounded(&bar[st ^ 1], (uint32_t)((it + 1) >> 1) & 1u);
+        for (int i = 0; i < S; ++i) {
+          const long long gj = gi + i;
+          if (gj >= g1) break;
+          const int sj = (st + i) % S;
+          const uint32_t pj = par ^ (uint32_t)((st + i) / S);
+          mbar_wait_bounded(&bar[sj], pj & 1u);
+        }
       }
       __syncwarp();
       return;
@@ -191,26 +213,37 @@ __global__ void __launch_bounds__(kScanWarps * 32, 1) scan_kernel(const ScanPara
     const float bk = beta * p.kappa;
 
     // ---- approximate logits (log2 units) for head gid, 64 tokens ----
+    // two n-tiles at a time so two independent MMA chains interleave
     float u[8][2];
-    auto qk_tile = [&](int nt, const uint32_t* b) {
-      float d[4] = {0.f, 0.f, 0.f, 0.f};
+    auto qk_pair = [&](int nt, const uint32_t* b0, const uint32_t* b1) {
+      float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int ks = 0; ks < 8; ++ks)
-        mma16816(d, ahi[2 * ks], alo[2 * ks], ahi[2 * ks + 1], alo[2 * ks + 1], b[2 * ks],
-                 b[2 * ks + 1]);
-      u[nt][0] = head_ok ? fmaf(d[0] + d[2], p.kappa, bk) : -INFINITY;
-      u[nt][1] = head_ok ? fmaf(d[1] + d[3], p.kappa, bk) : -INFINITY;
+      for (int ks = 0; ks < 8; ++ks) {
+        mma16816(d0, ahi[2 * ks], alo[2 * ks], ahi[2 * ks + 1], alo[2 * ks + 1], b0[2 * ks],
+                 b0[2 * ks + 1]);
+        mma16816(d1, ahi[2 * ks], alo[2 * ks], ahi[2 * ks + 1], alo[2 * ks + 1], b1[2 * ks],
+                 b1[2 * ks + 1]);
+      }
+      u[nt][0] = head_ok ? fmaf(d0[0] + d0[2], p.kappa, bk) : -INFINITY;
+      u[nt][1] = head_ok ? fmaf(d0[1] + d0[3], p.kappa, bk) : -INFINITY;
+      u[nt + 1][0] = head_ok ? fmaf(d1[0] + d1[2], p.kappa, bk) : -INFINITY;
+      u[nt + 1][1] = head_ok ? fmaf(d1[1] + d1[3], p.kappa, bk) : -INFINITY;
     };
     if constexpr (KB == 4) {
 #pragma unroll
-      for (int nt = 0; nt < 8; ++nt) {
-        const uint4 cw = lds128(r + OFF_KC + nt * 512 + lane * 16);
-        uint32_t b[16];
-        unpack4(cw.x, b);
-        unpack4(cw.y, b + 4);
-        unpack4(cw.z, b + 8);
-        unpack4(cw.w, b + 12);
-        qk_tile(nt, b);
+      for (int nt = 0; nt < 8; nt += 2) {
+        const uint4 ca = lds128(r + OFF_KC + nt * 512 + lane * 16);
+        const uint4 cb = lds128(r + OFF_KC + (nt + 1) * 512 + lane * 16);
+        uint32_t b0[16], b1[16];
+        unpack4(ca.x, b0);
+        unpack4(ca.y, b0 + 4);
+        unpack4(ca.z, b0 + 8);
+        unpack4(ca.w, b0 + 12);
+        unpack4(cb.x, b1);
+        unpack4(cb.y, b1 + 4);
+        unpack4(cb.z, b1 + 8);
+        unpack4(cb.w, b1 + 12);
+        qk_pair(nt, b0, b1);
       }
     } else {
 #pragma unroll
@@ -220,10 +253,11 @@ __global__ void __launch_bounds__(kScanWarps * 32, 1) scan_kernel(const ScanPara
         const uint32_t w[12] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y,
                                 c1.z, c1.w, c2.x, c2.y, c2.z, c2.w};
 #pragma unroll
-        for (int rr = 0; rr < 4; ++rr) {
-          uint32_t b[16];
-          unpack3(w[3 * rr], w[3 * rr + 1], w[3 * rr + 2], b);
-          qk_tile(nt4 * 4 + rr, b);
+        for (int rr = 0; rr < 4; rr += 2) {
+          uint32_t b0[16], b1[16];
+          unpack3(w[3 * rr], w[3 * rr + 1], w[3 * rr + 2], b0);
+          unpack3(w[3 * rr + 3], w[3 * rr + 4], w[3 * rr + 5], b1);
+          qk_pair(nt4 * 4 + rr, b0, b1);
         }
       }
     }
@@ -286,22 +320,33 @@ __global__ void __launch_bounds__(kScanWarps * 32, 1) scan_kernel(const ScanPara
                                  8 * gid + 2 * tig) = o;
     }
 
-    // ---- probabilities (fp16 pairs of tokens 8nt+2tig, +1) ----
-    uint32_t ph[8];
+    // ---- probabilities: fp16 pairs (tokens 8nt+2tig, +1) and their rounding
+    // remainders, so p and p*s_v enter the MMAs with ~22-bit precision ----
+    uint32_t ph[8], pl[8];
 #pragma unroll
-    for (int nt = 0; nt < 8; ++nt)
-      ph[nt] = pack_h2(exp2f(u[nt][0] - m_run), exp2f(u[nt][1] - m_run));
+    for (int nt = 0; nt < 8; ++nt) {
+      const float p0 = exp2f(u[nt][0] - m_run), p1 = exp2f(u[nt][1] - m_run);
+      ph[nt] = pack_h2(p0, p1);
+      const float2 hf = unpack_h2(ph[nt]);
+      pl[nt] = pack_h2(p0 - hf.x, p1 - hf.y);
+    }
 
     // ---- value aggregate: acc^T[c][h] += sum_t v'[t][c] * (p[t][h] s_v[t][j]) ----
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk) {
       const uint4 s0 = lds128(r + OFF_VS + kk * 128 + tig * 32);
       const uint4 s1 = lds128(r + OFF_VS + kk * 128 + tig * 32 + 16);
+      const uint32_t sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
       const uint32_t pa = ph[2 * kk], pb = ph[2 * kk + 1];
-      const uint32_t bj[4][2] = {{h2_mul(pa, s0.x), h2_mul(pb, s0.y)},
-                                 {h2_mul(pa, s0.z), h2_mul(pb, s0.w)},
-                                 {h2_mul(pa, s1.x), h2_mul(pb, s1.y)},
-                                 {h2_mul(pa, s1.z), h2_mul(pb, s1.w)}};
+      const uint32_t la = pl[2 * kk], lb = pl[2 * kk + 1];
+      uint32_t bh[4][2], bl[4][2];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        bh[j][0] = h2_mul(pa, sv[2 * j]);
+        bh[j][1] = h2_mul(pb, sv[2 * j + 1]);
+        bl[j][0] = h2_fma(la, sv[2 * j], h2_fma(pa, sv[2 * j], bh[j][0] ^ 0x80008000u));
+        bl[j][1] = h2_fma(lb, sv[2 * j + 1], h2_fma(pb, sv[2 * j + 1], bh[j][1] ^ 0x80008000u));
+      }
       uint32_t za0 = 0u, za2 = 0u;
       if (gid < 4) {
         const uint2 zz = lds64(r + OFF_VS + 512 + kk * 128 + tig * 32 + gid * 8);
@@ -311,6 +356,7 @@ __global__ void __launch_bounds__(kScanWarps * 32, 1) scan_kernel(const ScanPara
         za0 = za2 = kOneH2;
       }
       mma16816(dz, za0, 0u, za2, 0u, pa, pb);
+      mma16816(dz, za0, 0u, za2, 0u, la, lb);
       if constexpr (VB == 4) {
         const uint4 v0 = lds128(r + OFF_VC + (2 * kk) * 512 + lane * 16);
         const uint4 v1 = lds128(r + OFF_VC + (2 * kk + 1) * 512 + lane * 16);
@@ -319,7 +365,8 @@ __global__ void __launch_bounds__(kScanWarps * 32, 1) scan_kernel(const ScanPara
         for (int mt = 0; mt < 8; ++mt) {
           uint32_t a[4];
           unpack4(vw[mt], a);
-          mma16816(acc[mt], a[0], a[1], a[2], a[3], bj[mt >> 1][0], bj[mt >> 1][1]);
+          mma16816(acc[mt], a[0], a[1], a[2], a[3], bh[mt >> 1][0], bh[mt >> 1][1]);
+          mma16816(acc[mt], a[0], a[1], a[2], a[3], bl[mt >> 1][0], bl[mt >> 1][1]);
         }
       } else {
         const uint4 v = lds128(r + OFF_VC + kk * 512 + lane * 16);
@@ -328,16 +375,23 @@ __global__ void __launch_bounds__(kScanWarps * 32, 1) scan_kernel(const ScanPara
         for (int mp = 0; mp < 4; ++mp) {
           uint32_t a[8];
           unpack2(vw[mp], a);
-          mma16816(acc[2 * mp], a[0], a[1], a[2], a[3], bj[mp][0], bj[mp][1]);
-          mma16816(acc[2 * mp + 1], a[4], a[5], a[6], a[7], bj[mp][0], bj[mp][1]);
+          mma16816(acc[2 * mp], a[0], a[1], a[2], a[3], bh[mp][0], bh[mp][1]);
+          mma16816(acc[2 * mp + 1], a[4], a[5], a[6], a[7], bh[mp][0], bh[mp][1]);
+          mma16816(acc[2 * mp], a[0], a[1], a[2], a[3], bl[mp][0], bl[mp][1]);
+          mma16816(acc[2 * mp + 1], a[4], a[5], a[6], a[7], bl[mp][0], bl[mp][1]);
         }
       }
     }
 
     __syncwarp();
-    if (lane == 0 && gi + 2 < g1) {
-      mbar_expect_tx(&bar[st], REC);
-      bulk_g2s(ring + st * REC, rec_ptr(gi + 2), REC, &bar[st], pol);
+    if (lane == 0 && gi + S < g1) issue_next(st);
+    if (++st == S) {
+      st = 0;
+      par ^= 1u;
+    }
+    if (++g == p.ng) {
+      g = 0;
+      ++seg;
     }
   }
   flush(cur);
@@ -345,8 +399,7 @@ __global__ void __launch_bounds__(kScanWarps * 32, 1) scan_kernel(const ScanPara
 
 template <int KB, int VB>
 static int launch_scan_t(const ScanParams& sp, int n_ctas, cudaStream_t st) {
-  constexpr int REC = 512 + 1024 * KB + 1024 + 1024 * VB;
-  const int smem = kScanWarps * 2 * REC + kScanWarps * 2 * 8;
+  const int smem = ScanCfg<KB, VB>::SMEM;
   static bool configured = false;
   if (!configured) {
     if (cudaFuncSetAttribute(scan_kernel<KB, VB>, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -76,21 +76,30 @@ __device__ void find_from_bottom(const uint32_t* h, int nbins, uint32_t r, uint3
   __syncthreads();
 }
 
+constexpr int kTopkChunk = 4096;  // scores per CTA of the histogram / collect kernels
+
 __global__ void __launch_bounds__(256) topk_hist_kernel(const float* scores, int capacity,
                                                         int nq, uint32_t* hist) {
   __shared__ uint32_t sh[kHistBins];
   const int seg = blockIdx.y;
   for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) sh[i] = 0u;
-  __syncthreads();
-  const int per = ((nq + gridDim.x - 1) / gridDim.x + 3) & ~3;
-  const int lo = blockIdx.x * per, hi = min(nq, lo + per);
+  const int lo = blockIdx.x * kTopkChunk;
   const float* s = scores + (size_t)seg * capacity;
-  for (int i = lo + 4 * threadIdx.x; i < hi; i += 4 * blockDim.x) {
-    const float4 v = *reinterpret_cast<const float4*>(s + i);  // nq is a multiple of 64
-    atomicAdd(&sh[float_key(v.x) >> 21], 1u);
-    atomicAdd(&sh[float_key(v.y) >> 21], 1u);
-    atomicAdd(&sh[float_key(v.z) >> 21], 1u);
-    atomicAdd(&sh[float_key(v.w) >> 21], 1u);
+  float4 v[4];
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {  // nq is a multiple of 64: a float4 is all in or all out
+    const int i = lo + 4 * (threadIdx.x + 256 * r);
+    v[r] = i < nq ? *reinterpret_cast<const float4*>(s + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  __syncthreads();
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    if (lo + 4 * (threadIdx.x + 256 * r) < nq) {
+      atomicAdd(&sh[float_key(v[r].x) >> 21], 1u);
+      atomicAdd(&sh[float_key(v[r].y) >> 21], 1u);
+      atomicAdd(&sh[float_key(v[r].z) >> 21], 1u);
+      atomicAdd(&sh[float_key(v[r].w) >> 21], 1u);
+    }
   }
   __syncthreads();
   uint32_t* gh = hist + (size_t)seg * kHistBins;
@@ -113,6 +122,15 @@ __global__ void __launch_bounds__(256) topk_collect_kernel(TopkBufs b) {
   __shared__ int s_bin;
   __shared__ uint32_t s_above;
   const int seg = blockIdx.y;
+  // this CTA's scores are loaded first so they arrive while the histogram is scanned
+  const int lo = blockIdx.x * kTopkChunk;
+  const float* s = b.scores + (size_t)seg * b.capacity;
+  float4 v[4];
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const int i = lo + 4 * (threadIdx.x + 256 * r);
+    v[r] = i < b.nq ? *reinterpret_cast<const float4*>(s + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
   const uint32_t* gh = b.hist + (size_t)seg * kHistBins;
   for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) sh[i] = gh[i];
   if (threadIdx.x == 0) {
@@ -129,32 +147,35 @@ __global__ void __launch_bounds__(256) topk_collect_kernel(TopkBufs b) {
   }
   const int lane = threadIdx.x & 31;
   const unsigned lt = (1u << lane) - 1u;
-  const int per = ((b.nq + gridDim.x - 1) / gridDim.x + 255) & ~255;
-  const int lo = blockIdx.x * per, hi = min(b.nq, lo + per);
-  const float* s = b.scores + (size_t)seg * b.capacity;
   int32_t* sel = b.sel + (size_t)seg * b.max_topk;
   uint2* cand = b.cand + (size_t)seg * b.cand_cap;
-  for (int base = lo; base < hi; base += blockDim.x) {
-    const int i = base + threadIdx.x;
-    const bool valid = i < hi;
-    const uint32_t key = valid ? float_key(s[i]) : 0u;
-    const uint32_t bin = key >> 21;
-    const bool is_sel = valid && bin > bstar;
-    const bool is_cand = valid && bin == bstar;
-    const unsigned ms = __ballot_sync(kFullMask, is_sel);
-    if (ms) {
-      uint32_t pos = 0;
-      if (lane == __ffs(ms) - 1) pos = atomicAdd(&ctr[0], (uint32_t)__popc(ms));
-      pos = __shfl_sync(kFullMask, pos, __ffs(ms) - 1);
-      if (is_sel) sel[pos + __popc(ms & lt)] = i;
-    }
-    const unsigned mc = __ballot_sync(kFullMask, is_cand);
-    if (mc) {
-      uint32_t pos = 0;
-      if (lane == __ffs(mc) - 1) pos = atomicAdd(&ctr[1], (uint32_t)__popc(mc));
-      pos = __shfl_sync(kFullMask, pos, __ffs(mc) - 1);
-      const uint32_t mine = pos + __popc(mc & lt);
-      if (is_cand && mine < (uint32_t)b.cand_cap) cand[mine] = make_uint2(key, (uint32_t)i);
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const int i0 = lo + 4 * (threadIdx.x + 256 * r);
+    const float vals[4] = {v[r].x, v[r].y, v[r].z, v[r].w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int i = i0 + e;
+      const bool valid = i0 < b.nq;
+      const uint32_t key = float_key(vals[e]);
+      const uint32_t bin = key >> 21;
+      const bool is_sel = valid && bin > bstar;
+      const bool is_cand = valid && bin == bstar;
+      const unsigned ms = __ballot_sync(kFullMask, is_sel);
+      if (ms) {
+        uint32_t pos = 0;
+        if (lane == __ffs(ms) - 1) pos = atomicAdd(&ctr[0], (uint32_t)__popc(ms));
+        pos = __shfl_sync(kFullMask, pos, __ffs(ms) - 1);
+        if (is_sel) sel[pos + __popc(ms & lt)] = i;
+      }
+      const unsigned mc = __ballot_sync(kFullMask, is_cand);
+      if (mc) {
+        uint32_t pos = 0;
+        if (lane == __ffs(mc) - 1) pos = atomicAdd(&ctr[1], (uint32_t)__popc(mc));
+        pos = __shfl_sync(kFullMask, pos, __ffs(mc) - 1);
+        const uint32_t mine = pos + __popc(mc & lt);
+        if (is_cand && mine < (uint32_t)b.cand_cap) cand[mine] = make_uint2(key, (uint32_t)i);
+      }
     }
   }
 }
@@ -266,21 +287,46 @@ __global__ void __launch_bounds__(1024) topk_final_kernel(TopkBufs b, int32_t* i
   while (npow < b.k) npow <<= 1;
   for (int i = b.k + tid; i < npow; i += blockDim.x) out[i] = 0x7FFFFFFF;
   __syncthreads();
-  for (int size = 2; size <= npow; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int i = tid; i < npow / 2; i += blockDim.x) {
-        const int lo = 2 * i - (i & (stride - 1));
-        const int hi = lo + stride;
-        const bool up = (lo & size) == 0;
-        const int32_t a = out[lo], c = out[hi];
-        if ((a > c) == up) {
-          out[lo] = c;
-          out[hi] = a;
+  if (npow <= (int)blockDim.x) {
+    // one element per thread; strides below 32 exchange through shuffles
+    int32_t x = tid < npow ? out[tid] : 0x7FFFFFFF;
+    for (int size = 2; size <= npow; size <<= 1) {
+      for (int stride = size >> 1; stride > 0; stride >>= 1) {
+        int32_t y;
+        if (stride >= 32) {
+          __syncthreads();
+          if (tid < npow) out[tid] = x;
+          __syncthreads();
+          y = tid < npow ? out[tid ^ stride] : 0x7FFFFFFF;
+        } else {
+          y = __shfl_xor_sync(kFullMask, x, stride);
         }
+        const bool up = (tid & size) == 0;
+        const bool lower = (tid & stride) == 0;
+        // the lower element of a pair keeps the min when sorting up
+        x = (lower == up) ? min(x, y) : max(x, y);
       }
-      __syncthreads();
+    }
+    __syncthreads();
+    if (tid < npow) out[tid] = x;
+  } else {
+    for (int size = 2; size <= npow; size <<= 1) {
+      for (int stride = size >> 1; stride > 0; stride >>= 1) {
+        for (int i = tid; i < npow / 2; i += blockDim.x) {
+          const int lo = 2 * i - (i & (stride - 1));
+          const int hi = lo + stride;
+          const bool up = (lo & size) == 0;
+          const int32_t a = out[lo], c = out[hi];
+          if ((a > c) == up) {
+            out[lo] = c;
+            out[hi] = a;
+          }
+        }
+        __syncthreads();
+      }
     }
   }
+  __syncthreads();
   int32_t* o = idx + (size_t)seg * b.k;
   for (int i = tid; i < b.k; i += blockDim.x) o[i] = out[i];
 }
@@ -292,10 +338,8 @@ __global__ void topk_fill_kernel(int32_t* idx, int k, int nq) {
 }
 
 static int topk_chunks(int nq, int n_seg) {
-  int by_size = (nq + 4095) / 4096;
-  int by_sm = (2 * num_sms_current() + n_seg - 1) / n_seg;
-  int c = by_size < by_sm ? by_size : by_sm;
-  return c < 1 ? 1 : c;
+  (void)n_seg;
+  return (nq + kTopkChunk - 1) / kTopkChunk;
 }
 
 int count_topk_launches(const jfa_geom& g, int k) {
