@@ -40,7 +40,7 @@ int workspace_layout(const jfa_geom& g, int max_topk, jfa_workspace_layout* out)
   L.off_hist = off;
   off += n_seg * kHistBins * sizeof(uint32_t);
   L.off_counters = off;
-  off = align_up(off + n_seg * 4 * sizeof(uint32_t), 256);
+  off = align_up(off + n_seg * 8 * sizeof(uint32_t), 256);
   L.cand_cap = g.capacity < 16384 ? g.capacity : 16384;
   L.off_cand = off;
   off = align_up(off + n_seg * (size_t)L.cand_cap * 2 * sizeof(uint32_t), 256);

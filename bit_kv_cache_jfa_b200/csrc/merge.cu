@@ -7,9 +7,8 @@
 // top-k token and every tail token, aggregated with bf16 values in fp32.
 //
 // Approximate remainder: the scan accumulated every quantized token; here
-// the top-k tokens' approximate terms are recomputed (codes re-derived from
-// the bf16 row with the packing rule and the stored scale/zero, which gives
-// the stored codes exactly) and removed:
+// the top-k tokens' approximate terms are recomputed from their stored codes
+// and scales/zeros (exactly what the scan used) and removed:
 //   (m_a, l_a, acc_a) - (m_r, l_r, acc_r)  in the m_a frame, l clamped >= 0.
 // The removed mass is replaced by the exact part, so the cancellation error
 // is relative to that part's weight.
@@ -44,224 +43,240 @@ struct MergeParams {
 
 __device__ __forceinline__ float bf16f(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
 
-__device__ __forceinline__ float quant_dequant_bits(float x, uint16_t sb, uint16_t zb, int bits) {
-  const float s = __half2float(__ushort_as_half(sb));
-  const float z = __half2float(__ushort_as_half(zb));
-  double c = 0.0;
-  if (s != 0.f) {
-    c = rint(((double)x - (double)z) / (double)s);
-    const double lv = (double)((1 << bits) - 1);
-    c = c < 0.0 ? 0.0 : (c > lv ? lv : c);
-  }
-  return fmaf(s, (float)c, z);
-}
-
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kAll, v, o);
   return v;
 }
 
-struct OnlineState {
-  float m, l, a[4];
-  __device__ void init() {
-    m = -INFINITY;
-    l = 0.f;
-    a[0] = a[1] = a[2] = a[3] = 0.f;
+// Stored code of (token tt of its group, channel c) read from the packed
+// record (the codes the scan used), dequantized as scale * code + zero.
+__device__ __forceinline__ uint32_t key_code(const uint8_t* rec, int kb, int tt, int c) {
+  const BitLoc L = kc_loc(kb, tt, c);
+  const uint8_t* w = rec + off_kc() + L.byte;
+  if (kb == 3 && kc3_is_pair15(c)) {
+    uint32_t v = 0;
+#pragma unroll
+    for (int b = 0; b < 3; ++b) v |= ((*reinterpret_cast<const uint32_t*>(w + 4 * b) >> L.bit) & 1u) << b;
+    return v;
   }
-  __device__ void add(float u, const float* v) {
-    if (u > m) {
-      const float sc = exp2f(m - u);  // 0 when m = -inf
-      l *= sc;
-      a[0] *= sc;
-      a[1] *= sc;
-      a[2] *= sc;
-      a[3] *= sc;
-      m = u;
-    }
-    const float w = exp2f(u - m);
-    l += w;
-    a[0] = fmaf(w, v[0], a[0]);
-    a[1] = fmaf(w, v[1], a[1]);
-    a[2] = fmaf(w, v[2], a[2]);
-    a[3] = fmaf(w, v[3], a[3]);
-  }
-};
+  return (*reinterpret_cast<const uint32_t*>(w) >> L.bit) & ((1u << kb) - 1u);
+}
+__device__ __forceinline__ uint32_t val_code(const uint8_t* rec, int kb, int vb, int tt, int c) {
+  const BitLoc L = vc_loc(vb, tt, c);
+  return (*reinterpret_cast<const uint32_t*>(rec + off_vc(kb) + L.byte) >> L.bit) &
+         ((1u << vb) - 1u);
+}
+__device__ __forceinline__ float h2f(const uint8_t* p) {
+  return __half2float(__ushort_as_half(*reinterpret_cast<const uint16_t*>(p)));
+}
 
-// grid (n_chunks, n_seg), 4 warps; warp w handles tokens chunk*32 + w*8 + i,
-// in two batches of four whose loads are all issued before any use.
+constexpr int kRow = kD + 4;  // padded fp32 row in shared memory
+
+// grid (n_chunks, n_seg), 256 threads.  Chunk = 32 entries of (top-k list,
+// then tail).  Phase A: thread (token slot, 16-channel part) stages the exact
+// bf16 rows and the dequantized rows of its token in shared memory (all its
+// loads issued together).  Phase B: thread (token, head) computes the exact
+// and approximate logits.  Phase C: one warp per head turns them into
+// weights.  Phase D: thread (channel, exact|removal) accumulates the weighted
+// rows.  Writes one (m, l, acc) partial per (part, head).
 template <int G>
-__global__ void __launch_bounds__(128) correct_chunk_kernel(const MergeParams p) {
-  __shared__ float red[4][2][G][kPartStride];
+__global__ void __launch_bounds__(256) correct_chunk_kernel(const MergeParams p) {
+  extern __shared__ __align__(16) float sm[];
+  float* kx = sm;                      // [32][kRow] exact keys
+  float* vx = kx + kMergeChunk * kRow; // [32][kRow] exact values
+  float* kh = vx + kMergeChunk * kRow; // [32][kRow] dequantized keys
+  float* vh = kh + kMergeChunk * kRow; // [32][kRow] dequantized values
+  float* qs = vh + kMergeChunk * kRow; // [G][kRow]
+  float* ue = qs + G * kRow;           // [32][G] exact logits, then weights
+  float* ur = ue + kMergeChunk * G;    // [32][G] approximate logits, then weights
+  float* ml = ur + kMergeChunk * G;    // [2][G][2] (m, l)
+  __shared__ int s_tok[kMergeChunk];
+
   const int seg = blockIdx.y, chunk = blockIdx.x;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tid = threadIdx.x;
   const int b = seg / p.hkv, h = seg % p.hkv;
-  const int c0 = 4 * lane;
-  const int jv = lane >> 3;  // channels 4*lane.. lie in value group lane/8
 
-  float q[G][4];
-#pragma unroll
-  for (int j = 0; j < G; ++j) {
-    const uint2 w = *reinterpret_cast<const uint2*>(p.q + ((size_t)b * p.H + h * G + j) * kD + c0);
-    q[j][0] = __uint_as_float(w.x << 16);
-    q[j][1] = __uint_as_float(w.x & 0xFFFF0000u);
-    q[j][2] = __uint_as_float(w.y << 16);
-    q[j][3] = __uint_as_float(w.y & 0xFFFF0000u);
-  }
-  OnlineState ex[G], rm[G];
-#pragma unroll
-  for (int j = 0; j < G; ++j) {
-    ex[j].init();
-    rm[j].init();
-  }
-  const int ks_s0 = off_ks() + ks_scale_off(c0), ks_s1 = off_ks() + ks_scale_off(c0 + 2);
-  const int ks_z0 = off_ks() + ks_zero_off(c0), ks_z1 = off_ks() + ks_zero_off(c0 + 2);
-
-  const int e_base = chunk * kMergeChunk + warp * (kMergeChunk / 4);
-  // token ids of this warp's 8 entries (lane i < 8 resolves entry i)
-  int my_t = -1;
-  if (lane < 8) {
-    const int e = e_base + lane;
+  if (tid < kMergeChunk) {
+    const int e = chunk * kMergeChunk + tid;
+    int t = -1;
     if (e < p.k) {
-      my_t = p.idx[(size_t)seg * p.k + e];
-      if (my_t >= p.nq) {
+      t = p.idx[(size_t)seg * p.k + e];
+      if (t >= p.nq) {
         set_flag(p.flag, JFA_DEVERR_BAD_INDEX);
-        my_t = -1;
+        t = -1;
       }
     } else if (e - p.k < p.tail) {
-      my_t = (1 << 30) | (e - p.k);  // tail slot
+      t = (1 << 30) | (e - p.k);  // tail slot
     }
+    s_tok[tid] = t;
   }
+  for (int i = tid; i < G * kD; i += 256) {
+    const int j = i / kD, c = i % kD;
+    qs[j * kRow + c] = bf16f(p.q[((size_t)b * p.H + h * G + j) * kD + c]);
+  }
+  __syncthreads();
+
+  // ---- phase A ----
+  {
+    const int tl = tid >> 3, part = tid & 7, c0 = 16 * part;
+    const int t = s_tok[tl];
+    float* krow = kx + tl * kRow + c0;
+    float* vrow = vx + tl * kRow + c0;
+    if (t < 0) {
 #pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    int tk[4];
-    uint2 kw[4], vw[4];
-    uint32_t s01[4], s23[4], z01[4], z23[4];
-    uint16_t vsb[4], vzb[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      tk[i] = __shfl_sync(kAll, my_t, half * 4 + i);
-      kw[i] = vw[i] = make_uint2(0u, 0u);
-      s01[i] = s23[i] = z01[i] = z23[i] = 0u;
-      vsb[i] = vzb[i] = 0;
-      if (tk[i] < 0) continue;
+      for (int i = 0; i < 16; ++i) krow[i] = vrow[i] = 0.f;
+    } else {
+      const bool tail = (t & (1 << 30)) != 0;
       const uint16_t *kr, *vr;
-      if (tk[i] & (1 << 30)) {
-        const int tt = tk[i] & ~(1 << 30);
+      if (tail) {
+        const int tt = t & ~(1 << 30);
         kr = p.tail_k + ((size_t)seg * kTail + tt) * kD;
         vr = p.tail_v + ((size_t)seg * kTail + tt) * kD;
       } else {
-        const int t = tk[i];
         kr = p.k_exact + ((size_t)seg * p.capacity + t) * kD;
         vr = p.v_exact + ((size_t)seg * p.capacity + t) * kD;
+      }
+      const uint4 ka = *reinterpret_cast<const uint4*>(kr + c0);
+      const uint4 kb = *reinterpret_cast<const uint4*>(kr + c0 + 8);
+      const uint4 va = *reinterpret_cast<const uint4*>(vr + c0);
+      const uint4 vb = *reinterpret_cast<const uint4*>(vr + c0 + 8);
+      float khq[16], vhq[16];
+      if (!tail) {
+        const int tt = t % kKG;
         const uint8_t* rec = p.groups + ((size_t)seg * p.ng_cap + t / kKG) * p.rec_bytes;
-        s01[i] = *reinterpret_cast<const uint32_t*>(rec + ks_s0);
-        s23[i] = *reinterpret_cast<const uint32_t*>(rec + ks_s1);
-        z01[i] = *reinterpret_cast<const uint32_t*>(rec + ks_z0);
-        z23[i] = *reinterpret_cast<const uint32_t*>(rec + ks_z1);
-        const int vb = off_vs(p.key_bits);
-        vsb[i] = *reinterpret_cast<const uint16_t*>(rec + vb + vs_scale_off(t % kKG, jv));
-        vzb[i] = *reinterpret_cast<const uint16_t*>(rec + vb + vs_zero_off(t % kKG, jv));
-      }
-      kw[i] = *reinterpret_cast<const uint2*>(kr + c0);
-      vw[i] = *reinterpret_cast<const uint2*>(vr + c0);
-    }
+        const float vs = h2f(rec + off_vs(p.key_bits) + vs_scale_off(tt, part >> 1));
+        const float vz = h2f(rec + off_vs(p.key_bits) + vs_zero_off(tt, part >> 1));
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      if (tk[i] < 0) continue;  // warp-uniform
-      const float kx[4] = {bf16f(kw[i].x & 0xFFFFu), bf16f(kw[i].x >> 16), bf16f(kw[i].y & 0xFFFFu),
-                           bf16f(kw[i].y >> 16)};
-      const float vx[4] = {bf16f(vw[i].x & 0xFFFFu), bf16f(vw[i].x >> 16), bf16f(vw[i].y & 0xFFFFu),
-                           bf16f(vw[i].y >> 16)};
-#pragma unroll
-      for (int j = 0; j < G; ++j) {
-        float d = q[j][0] * kx[0];
-        d = fmaf(q[j][1], kx[1], d);
-        d = fmaf(q[j][2], kx[2], d);
-        d = fmaf(q[j][3], kx[3], d);
-        d = warp_sum(d);
-        ex[j].add(d * p.kappa, vx);
-      }
-      if (!(tk[i] & (1 << 30))) {
-        const uint16_t ksb[4] = {(uint16_t)(s01[i] & 0xFFFFu), (uint16_t)(s01[i] >> 16),
-                                 (uint16_t)(s23[i] & 0xFFFFu), (uint16_t)(s23[i] >> 16)};
-        const uint16_t kzb[4] = {(uint16_t)(z01[i] & 0xFFFFu), (uint16_t)(z01[i] >> 16),
-                                 (uint16_t)(z23[i] & 0xFFFFu), (uint16_t)(z23[i] >> 16)};
-        float kh[4], vh[4];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          kh[c] = quant_dequant_bits(kx[c], ksb[c], kzb[c], p.key_bits);
-          vh[c] = quant_dequant_bits(vx[c], vsb[i], vzb[i], p.val_bits);
-        }
-#pragma unroll
-        for (int j = 0; j < G; ++j) {
-          float d = q[j][0] * kh[0];
-          d = fmaf(q[j][1], kh[1], d);
-          d = fmaf(q[j][2], kh[2], d);
-          d = fmaf(q[j][3], kh[3], d);
-          d = warp_sum(d);
-          rm[j].add(d * p.kappa, vh);
+        for (int i = 0; i < 16; ++i) {
+          const int c = c0 + i;
+          const float s = h2f(rec + off_ks() + ks_scale_off(c));
+          const float z = h2f(rec + off_ks() + ks_zero_off(c));
+          khq[i] = fmaf(s, (float)key_code(rec, p.key_bits, tt, c), z);
+          vhq[i] = fmaf(vs, (float)val_code(rec, p.key_bits, p.val_bits, tt, c), vz);
         }
       }
-    }
-  }
-  // combine the 4 warps
+      const uint32_t kw[8] = {ka.x, ka.y, ka.z, ka.w, kb.x, kb.y, kb.z, kb.w};
+      const uint32_t vw[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
 #pragma unroll
-  for (int j = 0; j < G; ++j) {
-    float* re = red[warp][0][j];
-    float* rr = red[warp][1][j];
-    if (lane == 0) {
-      re[0] = ex[j].m;
-      re[1] = ex[j].l;
-      rr[0] = rm[j].m;
-      rr[1] = rm[j].l;
-    }
+      for (int i = 0; i < 8; ++i) {
+        krow[2 * i] = __uint_as_float(kw[i] << 16);
+        krow[2 * i + 1] = __uint_as_float(kw[i] & 0xFFFF0000u);
+        vrow[2 * i] = __uint_as_float(vw[i] << 16);
+        vrow[2 * i + 1] = __uint_as_float(vw[i] & 0xFFFF0000u);
+      }
+      if (!tail) {
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      re[4 + c0 + c] = ex[j].a[c];
-      rr[4 + c0 + c] = rm[j].a[c];
+        for (int i = 0; i < 16; ++i) {
+          kh[tl * kRow + c0 + i] = khq[i];
+          vh[tl * kRow + c0 + i] = vhq[i];
+        }
+      }
     }
   }
   __syncthreads();
-  const int c = threadIdx.x;  // channel
+
+  // ---- phase B: logits (log2 units) ----
+  for (int i = tid; i < kMergeChunk * G; i += 256) {
+    const int tl = i / G, j = i % G;
+    const int t = s_tok[tl];
+    float de = -INFINITY, dr = -INFINITY;
+    if (t >= 0) {
+      const float4* qr = reinterpret_cast<const float4*>(qs + j * kRow);
+      const float4* kr4 = reinterpret_cast<const float4*>(kx + tl * kRow);
+      float a0 = 0.f, a1 = 0.f;
+#pragma unroll 8
+      for (int c = 0; c < kD / 4; ++c) {
+        const float4 qv = qr[c], kv = kr4[c];
+        a0 = fmaf(qv.x, kv.x, a0);
+        a1 = fmaf(qv.y, kv.y, a1);
+        a0 = fmaf(qv.z, kv.z, a0);
+        a1 = fmaf(qv.w, kv.w, a1);
+      }
+      de = (a0 + a1) * p.kappa;
+      if (!(t & (1 << 30))) {
+        const float4* hr4 = reinterpret_cast<const float4*>(kh + tl * kRow);
+        float b0 = 0.f, b1 = 0.f;
+#pragma unroll 8
+        for (int c = 0; c < kD / 4; ++c) {
+          const float4 qv = qr[c], kv = hr4[c];
+          b0 = fmaf(qv.x, kv.x, b0);
+          b1 = fmaf(qv.y, kv.y, b1);
+          b0 = fmaf(qv.z, kv.z, b0);
+          b1 = fmaf(qv.w, kv.w, b1);
+        }
+        dr = (b0 + b1) * p.kappa;
+      }
+    }
+    ue[tl * G + j] = de;
+    ur[tl * G + j] = dr;
+  }
+  __syncthreads();
+
+  // ---- phase C: weights, one warp per head ----
+  {
+    const int warp = tid >> 5, lane = tid & 31;
+    for (int j = warp; j < G; j += 8) {
 #pragma unroll
-  for (int part = 0; part < 2; ++part) {
+      for (int part = 0; part < 2; ++part) {
+        float* u = part ? ur : ue;
+        const float x = u[lane * G + j];
+        float m = x;
 #pragma unroll
-    for (int j = 0; j < G; ++j) {
-      float m = -INFINITY;
-#pragma unroll
-      for (int w = 0; w < 4; ++w)
-        if (red[w][part][j][1] > 0.f) m = fmaxf(m, red[w][part][j][0]);
-      float l = 0.f, a = 0.f;
-      if (m > -INFINITY) {
-#pragma unroll
-        for (int w = 0; w < 4; ++w) {
-          const float lb = red[w][part][j][1];
-          if (lb > 0.f) {
-            const float sc = exp2f(red[w][part][j][0] - m);
-            l = fmaf(lb, sc, l);
-            a = fmaf(red[w][part][j][4 + c], sc, a);
-          }
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kAll, m, o));
+        const float w = m == -INFINITY ? 0.f : exp2f(x - m);
+        const float l = warp_sum(w);
+        u[lane * G + j] = w;
+        if (lane == 0) {
+          ml[(part * G + j) * 2] = m;
+          ml[(part * G + j) * 2 + 1] = l;
         }
       }
+    }
+  }
+  __syncthreads();
+
+  // ---- phase D: weighted rows ----
+  {
+    const int c = tid & (kD - 1), part = tid >> 7;
+    const float* rows = part ? vh : vx;
+    const float* w = part ? ur : ue;
+    float acc[G];
+#pragma unroll
+    for (int j = 0; j < G; ++j) acc[j] = 0.f;
+    for (int tl = 0; tl < kMergeChunk; ++tl) {
+      const float v = rows[tl * kRow + c];
+#pragma unroll
+      for (int j = 0; j < G; ++j) acc[j] = fmaf(w[tl * G + j], v, acc[j]);
+    }
+#pragma unroll
+    for (int j = 0; j < G; ++j) {
       float* dst = p.chunk_part +
                    ((((size_t)seg * p.n_chunks + chunk) * 2 + part) * G + j) * kPartStride;
+      dst[4 + c] = acc[j];
       if (c == 0) {
-        dst[0] = m;
-        dst[1] = l;
+        dst[0] = ml[(part * G + j) * 2];
+        dst[1] = ml[(part * G + j) * 2 + 1];
       }
-      dst[4 + c] = a;
     }
   }
 }
 
-// Merge all partials of (segment, head): max first, then independent sums,
-// so every partial's loads are in flight together.
 template <int G>
-__global__ void __launch_bounds__(32 * G) merge_final_kernel(const MergeParams p) {
-  const int seg = blockIdx.x;
-  const int j = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int c0 = 4 * lane;
+constexpr int correct_smem_bytes() {
+  return (4 * kMergeChunk * kRow + G * kRow + 2 * kMergeChunk * G + 4 * G) * 4;
+}
+
+// grid (n_seg, G), 256 threads: one (segment, head).  All partial rows of the
+// head (scan slots, exact chunks, removal chunks) are staged in shared memory
+// in tiles of kTileRows with every load of a tile in flight together, then
+// reduced max-first per tile into a running state.
+constexpr int kTileRows = 48;
+template <int G>
+__global__ void __launch_bounds__(256) merge_final_kernel(const MergeParams p) {
+  __shared__ __align__(16) float tile[kTileRows][kPartStride];
+  const int seg = blockIdx.x, j = blockIdx.y;
+  const int tid = threadIdx.x;
   long long w0 = 0, w1 = -1;
   if (p.ng > 0) {
     const long long T = p.scan_total, W = p.scan_warps;
@@ -270,87 +285,102 @@ __global__ void __launch_bounds__(32 * G) merge_final_kernel(const MergeParams p
     w1 = scan_warp_of(x1, W, T);
   }
   const int ns = (int)(w1 - w0 + 1);
-  auto srow = [&](int i) { return p.scan_part + ((size_t)(w0 + i + seg) * G + j) * kPartStride; };
-  auto crow = [&](int ch, int part) {
+  const int nrows = ns + 2 * p.n_chunks;  // kind of row r: 0 scan, 1 exact, 2 removal
+  auto row_ptr = [&](int r) -> const float* {
+    if (r < ns) return p.scan_part + ((size_t)(w0 + r + seg) * G + j) * kPartStride;
+    r -= ns;
+    const int ch = r >> 1, part = r & 1;
     return p.chunk_part + ((((size_t)seg * p.n_chunks + ch) * 2 + part) * G + j) * kPartStride;
   };
-  // pass 1: maxima
-  float ma = -INFINITY, me = -INFINITY, mr = -INFINITY;
-  for (int i = 0; i < ns; ++i) {
-    const float2 ml = *reinterpret_cast<const float2*>(srow(i));
-    if (ml.y > 0.f) ma = fmaxf(ma, ml.x);
+  auto kind_of = [&](int r) { return r < ns ? 0 : 1 + ((r - ns) & 1); };
+  const int c = tid & (kD - 1);
+  const bool worker = tid < kD;
+  float m[3] = {-INFINITY, -INFINITY, -INFINITY}, l[3] = {0.f, 0.f, 0.f}, a[3] = {0.f, 0.f, 0.f};
+  for (int r0 = 0; r0 < nrows; r0 += kTileRows) {
+    const int nr = min(kTileRows, nrows - r0);
+    __syncthreads();
+    for (int i = tid; i < nr * (kPartStride / 4); i += 256) {
+      const int r = i / (kPartStride / 4), v = i % (kPartStride / 4);
+      reinterpret_cast<float4*>(tile[r])[v] = reinterpret_cast<const float4*>(row_ptr(r0 + r))[v];
+    }
+    __syncthreads();
+    if (worker) {
+      // kinds: 0 scan slots (rows [0, ns)), then exact / removal alternating
+      float tm0 = m[0], tm1 = m[1], tm2 = m[2];
+      for (int r = 0; r < nr; ++r) {
+        if (tile[r][1] > 0.f) {
+          const int k = kind_of(r0 + r);
+          const float x = tile[r][0];
+          if (k == 0) tm0 = fmaxf(tm0, x);
+          else if (k == 1) tm1 = fmaxf(tm1, x);
+          else tm2 = fmaxf(tm2, x);
+        }
+      }
+      const float tmv[3] = {tm0, tm1, tm2};
+#pragma unroll
+      for (int k = 0; k < 3; ++k) {
+        if (tmv[k] > m[k] && m[k] > -INFINITY) {
+          const float sc = exp2f(m[k] - tmv[k]);
+          l[k] *= sc;
+          a[k] *= sc;
+        }
+        m[k] = tmv[k];
+      }
+      for (int r = 0; r < nr; ++r) {
+        const float lb = tile[r][1];
+        if (lb > 0.f) {
+          const int k = kind_of(r0 + r);
+          const float mk = k == 0 ? m[0] : (k == 1 ? m[1] : m[2]);
+          const float sc = exp2f(tile[r][0] - mk);
+          const float lv = lb * sc, av = tile[r][4 + c] * sc;
+          if (k == 0) {
+            l[0] += lv;
+            a[0] += av;
+          } else if (k == 1) {
+            l[1] += lv;
+            a[1] += av;
+          } else {
+            l[2] += lv;
+            a[2] += av;
+          }
+        }
+      }
+    }
   }
-  for (int ch = 0; ch < p.n_chunks; ++ch) {
-    const float2 e = *reinterpret_cast<const float2*>(crow(ch, 0));
-    const float2 r = *reinterpret_cast<const float2*>(crow(ch, 1));
-    if (e.y > 0.f) me = fmaxf(me, e.x);
-    if (r.y > 0.f) mr = fmaxf(mr, r.x);
-  }
-  // pass 2: sums in the frames of those maxima
-  float la = 0.f, le = 0.f, lr = 0.f;
-  float aa[4] = {0.f, 0.f, 0.f, 0.f}, ae[4] = {0.f, 0.f, 0.f, 0.f}, ar[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
-  for (int i = 0; i < ns; ++i) {
-    const float* row = srow(i);
-    const float2 ml = *reinterpret_cast<const float2*>(row);
-    const float4 v = *reinterpret_cast<const float4*>(row + 4 + c0);
-    const float sc = ml.y > 0.f ? exp2f(ml.x - ma) : 0.f;
-    la = fmaf(ml.y, sc, la);
-    aa[0] = fmaf(v.x, sc, aa[0]);
-    aa[1] = fmaf(v.y, sc, aa[1]);
-    aa[2] = fmaf(v.z, sc, aa[2]);
-    aa[3] = fmaf(v.w, sc, aa[3]);
-  }
-#pragma unroll 4
-  for (int ch = 0; ch < p.n_chunks; ++ch) {
-    const float* re = crow(ch, 0);
-    const float* rr = crow(ch, 1);
-    const float2 e = *reinterpret_cast<const float2*>(re);
-    const float2 r = *reinterpret_cast<const float2*>(rr);
-    const float4 ev = *reinterpret_cast<const float4*>(re + 4 + c0);
-    const float4 rv = *reinterpret_cast<const float4*>(rr + 4 + c0);
-    const float se = e.y > 0.f ? exp2f(e.x - me) : 0.f;
-    const float sr = r.y > 0.f ? exp2f(r.x - mr) : 0.f;
-    le = fmaf(e.y, se, le);
-    lr = fmaf(r.y, sr, lr);
-    ae[0] = fmaf(ev.x, se, ae[0]);
-    ae[1] = fmaf(ev.y, se, ae[1]);
-    ae[2] = fmaf(ev.z, se, ae[2]);
-    ae[3] = fmaf(ev.w, se, ae[3]);
-    ar[0] = fmaf(rv.x, sr, ar[0]);
-    ar[1] = fmaf(rv.y, sr, ar[1]);
-    ar[2] = fmaf(rv.z, sr, ar[2]);
-    ar[3] = fmaf(rv.w, sr, ar[3]);
-  }
+  if (!worker) return;
   // remainder = approximate total minus the removed top-k terms (m_a frame)
-  float lrest = la, arest[4] = {aa[0], aa[1], aa[2], aa[3]};
+  const float ma = m[0], la = l[0], me = m[1], le = l[1], mr = m[2], lr = l[2];
+  float lrest = la, arest = a[0];
   if (la > 0.f && lr > 0.f) {
     const float f = exp2f(mr - ma);
     lrest = la - lr * f;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) arest[i] = aa[i] - ar[i] * f;
+    arest = a[0] - a[2] * f;
     if (lrest < 0.f) lrest = 0.f;
   }
-  float m = me, wl = 1.f, wa = 0.f;
+  float mm = me, wl = 1.f, wa = 0.f;
   if (la > 0.f) {
-    m = fmaxf(me, ma);
-    wl = exp2f(me - m);
-    wa = exp2f(ma - m);
+    mm = fmaxf(me, ma);
+    wl = exp2f(me - mm);
+    wa = exp2f(ma - mm);
   }
-  const float inv = 1.f / (le * wl + lrest * wa);
-  float4 o;
-  o.x = (ae[0] * wl + arest[0] * wa) * inv;
-  o.y = (ae[1] * wl + arest[1] * wa) * inv;
-  o.z = (ae[2] * wl + arest[2] * wa) * inv;
-  o.w = (ae[3] * wl + arest[3] * wa) * inv;
+  const float o = (a[1] * wl + arest * wa) / (le * wl + lrest * wa);
   const int b = seg / p.hkv, h = seg % p.hkv;
-  *reinterpret_cast<float4*>(p.out + ((size_t)b * p.H + h * G + j) * kD + c0) = o;
+  p.out[((size_t)b * p.H + h * G + j) * kD + c] = o;
 }
 
 template <int G>
 static void launch_cm_t(const MergeParams& p, int n_seg, cudaStream_t st) {
-  correct_chunk_kernel<G><<<dim3(p.n_chunks, n_seg), 128, 0, st>>>(p);
-  merge_final_kernel<G><<<n_seg, 32 * G, 0, st>>>(p);
+  constexpr int smem = correct_smem_bytes<G>();
+  static bool configured[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !configured[dev]) {
+    cudaFuncSetAttribute(correct_chunk_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         smem);
+    configured[dev] = true;
+  }
+  correct_chunk_kernel<G><<<dim3(p.n_chunks, n_seg), 256, smem, st>>>(p);
+  merge_final_kernel<G><<<dim3(n_seg, G), 256, 0, st>>>(p);
 }
 
 int launch_correct_merge(const jfa_geom& g, const jfa_cache& c, const uint16_t* q, float scale,

@@ -17,6 +17,7 @@
 namespace jfa {
 
 constexpr unsigned kFullMask = 0xFFFFFFFFu;
+constexpr uint32_t kRankCap = 1024;  // candidates handled by the counting-rank path
 
 // Block-wide exclusive sum over threads in DESCENDING thread order:
 // returns sum of v over threads with a larger index.  scratch: >= 32 uints.
@@ -77,9 +78,11 @@ __device__ void find_from_bottom(const uint32_t* h, int nbins, uint32_t r, uint3
 }
 
 constexpr int kTopkChunk = 4096;  // scores per CTA of the histogram / collect kernels
+constexpr int kCtrStride = 8;     // counters per segment: n_sel, n_cand, bstar, above, done
 
 __global__ void __launch_bounds__(256) topk_hist_kernel(const float* scores, int capacity,
-                                                        int nq, uint32_t* hist) {
+                                                        int nq, int k, uint32_t* hist,
+                                                        uint32_t* counters) {
   __shared__ uint32_t sh[kHistBins];
   const int seg = blockIdx.y;
   for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) sh[i] = 0u;
@@ -105,24 +108,42 @@ __global__ void __launch_bounds__(256) topk_hist_kernel(const float* scores, int
   uint32_t* gh = hist + (size_t)seg * kHistBins;
   for (int i = threadIdx.x; i < kHistBins; i += blockDim.x)
     if (sh[i]) atomicAdd(&gh[i], sh[i]);
+  // the last CTA of the segment finds the bin holding the k-th key
+  __shared__ bool s_last;
+  __shared__ uint32_t scratch[32];
+  __shared__ int s_bin;
+  __shared__ uint32_t s_above;
+  uint32_t* ctr = counters + (size_t)seg * kCtrStride;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    s_last = atomicAdd(&ctr[4], 1u) == gridDim.x - 1;
+    s_bin = 0;
+    s_above = 0;
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) sh[i] = __ldcg(&gh[i]);
+  __syncthreads();
+  find_from_top(sh, kHistBins, (uint32_t)k, scratch, &s_bin, &s_above);
+  if (threadIdx.x == 0) {
+    ctr[2] = (uint32_t)s_bin;
+    ctr[3] = s_above;
+  }
 }
 
 struct TopkBufs {
   const float* scores;
   uint32_t* hist;      // [n_seg][2048]
-  uint32_t* counters;  // [n_seg][4]: n_sel, n_cand, bstar, above
+  uint32_t* counters;  // [n_seg][8]: n_sel, n_cand, bstar, above, hist CTAs done
   uint2* cand;         // [n_seg][cand_cap] (key, index)
   int32_t* sel;        // [n_seg][max_topk]
   int capacity, nq, k, cand_cap, max_topk;
 };
 
 __global__ void __launch_bounds__(256) topk_collect_kernel(TopkBufs b) {
-  __shared__ uint32_t sh[kHistBins];
-  __shared__ uint32_t scratch[32];
-  __shared__ int s_bin;
-  __shared__ uint32_t s_above;
   const int seg = blockIdx.y;
-  // this CTA's scores are loaded first so they arrive while the histogram is scanned
   const int lo = blockIdx.x * kTopkChunk;
   const float* s = b.scores + (size_t)seg * b.capacity;
   float4 v[4];
@@ -131,20 +152,8 @@ __global__ void __launch_bounds__(256) topk_collect_kernel(TopkBufs b) {
     const int i = lo + 4 * (threadIdx.x + 256 * r);
     v[r] = i < b.nq ? *reinterpret_cast<const float4*>(s + i) : make_float4(0.f, 0.f, 0.f, 0.f);
   }
-  const uint32_t* gh = b.hist + (size_t)seg * kHistBins;
-  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) sh[i] = gh[i];
-  if (threadIdx.x == 0) {
-    s_bin = 0;
-    s_above = 0;
-  }
-  __syncthreads();
-  find_from_top(sh, kHistBins, (uint32_t)b.k, scratch, &s_bin, &s_above);
-  const uint32_t bstar = (uint32_t)s_bin;
-  uint32_t* ctr = b.counters + (size_t)seg * 4;
-  if (blockIdx.x == 0 && threadIdx.x == 0) {
-    ctr[2] = bstar;
-    ctr[3] = s_above;
-  }
+  uint32_t* ctr = b.counters + (size_t)seg * kCtrStride;
+  const uint32_t bstar = ctr[2];
   const int lane = threadIdx.x & 31;
   const unsigned lt = (1u << lane) - 1u;
   int32_t* sel = b.sel + (size_t)seg * b.max_topk;
@@ -189,12 +198,48 @@ __global__ void __launch_bounds__(1024) topk_final_kernel(TopkBufs b, int32_t* i
   __shared__ uint32_t s_cnt, s_nout;
   const int seg = blockIdx.x;
   const int tid = threadIdx.x;
-  const uint32_t* ctr = b.counters + (size_t)seg * 4;
+  const uint32_t* ctr = b.counters + (size_t)seg * kCtrStride;
   const uint32_t n_sel = ctr[0], n_cand = ctr[1], bstar = ctr[2];
   const uint32_t r = (uint32_t)b.k - n_sel;  // >= 1
   const int32_t* sel = b.sel + (size_t)seg * b.max_topk;
   for (uint32_t i = tid; i < n_sel; i += blockDim.x) out[i] = sel[i];
   const bool from_cand = n_cand <= (uint32_t)b.cand_cap;
+  if (from_cand && n_cand <= kRankCap && b.k <= (int)blockDim.x) {
+    // small case: rank every candidate by counting (no refinement passes),
+    // then rank the k chosen indices by counting to sort them
+    uint32_t* ck = h;                                  // keys   [<= 1024]
+    int32_t* cx = reinterpret_cast<int32_t*>(h) + kRankCap;  // indices
+    const uint2* cand = b.cand + (size_t)seg * b.cand_cap;
+    for (uint32_t i = tid; i < n_cand; i += blockDim.x) {
+      const uint2 c = cand[i];
+      ck[i] = c.x;
+      cx[i] = (int32_t)c.y;
+    }
+    __syncthreads();
+    if (tid < n_cand) {
+      const uint32_t key = ck[tid];
+      const int32_t ix = cx[tid];
+      uint32_t rank = 0;
+      for (uint32_t j = 0; j < n_cand; ++j) {
+        const uint32_t kj = ck[j];
+        rank += (kj > key) || (kj == key && cx[j] < ix);
+      }
+      if (rank < r) out[n_sel + rank] = ix;
+    }
+    __syncthreads();
+    int32_t mine = 0;
+    uint32_t pos = 0;
+    if (tid < b.k) {
+      mine = out[tid];
+      for (int j = 0; j < b.k; ++j) pos += out[j] < mine;
+    }
+    __syncthreads();
+    if (tid < b.k) out[pos] = mine;
+    __syncthreads();
+    int32_t* o = idx + (size_t)seg * b.k;
+    if (tid < b.k) o[tid] = out[tid];
+    return;
+  }
   const uint2* cand = b.cand + (size_t)seg * b.cand_cap;
   const float* s = b.scores + (size_t)seg * b.capacity;
   const uint32_t n_src = from_cand ? n_cand : (uint32_t)b.nq;
@@ -370,7 +415,8 @@ int launch_topk(const jfa_geom& g, int k, uint8_t* ws, const jfa_workspace_layou
   if (cudaMemsetAsync(ws + L.off_hist, 0, L.off_cand - L.off_hist, st) != cudaSuccess)
     return JFA_ERR_CUDA;
   const int chunks = topk_chunks(nq, n_seg);
-  topk_hist_kernel<<<dim3(chunks, n_seg), 256, 0, st>>>(b.scores, g.capacity, nq, b.hist);
+  topk_hist_kernel<<<dim3(chunks, n_seg), 256, 0, st>>>(b.scores, g.capacity, nq, k, b.hist,
+                                                       b.counters);
   topk_collect_kernel<<<dim3(chunks, n_seg), 256, 0, st>>>(b);
   topk_final_kernel<<<n_seg, 1024, 0, st>>>(b, idx);
   return cudaGetLastError() == cudaSuccess ? JFA_OK : JFA_ERR_CUDA;
