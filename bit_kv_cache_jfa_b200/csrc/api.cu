@@ -41,12 +41,14 @@ int workspace_layout(const jfa_geom& g, int max_topk, jfa_workspace_layout* out)
   off += n_seg * kHistBins * sizeof(uint32_t);
   L.off_counters = off;
   off = align_up(off + n_seg * 8 * sizeof(uint32_t), 256);
-  L.cand_cap = g.capacity < 16384 ? g.capacity : 16384;
+  // top-k lists: per 4096-score chunk, up to 4096 (key, index) pairs; then counts
+  const size_t n_chunks_cap = ((size_t)g.capacity + 4095) / 4096;
+  L.cand_cap = (int32_t)(n_chunks_cap * 4096);
   L.off_cand = off;
   off = align_up(off + n_seg * (size_t)L.cand_cap * 2 * sizeof(uint32_t), 256);
   L.max_topk = max_topk;
   L.off_sel = off;
-  off = align_up(off + n_seg * (size_t)max_topk * sizeof(int32_t), 256);
+  off = align_up(off + n_seg * n_chunks_cap * sizeof(uint32_t), 256);
   L.merge_chunks = (max_topk + kTail + kMergeChunk - 1) / kMergeChunk;
   L.off_merge = off;
   off = align_up(off + n_seg * (size_t)L.merge_chunks * 2 * G * kPartStride * sizeof(float), 256);

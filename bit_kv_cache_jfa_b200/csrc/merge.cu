@@ -49,28 +49,8 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-// Stored code of (token tt of its group, channel c) read from the packed
-// record (the codes the scan used), dequantized as scale * code + zero.
-__device__ __forceinline__ uint32_t key_code(const uint8_t* rec, int kb, int tt, int c) {
-  const BitLoc L = kc_loc(kb, tt, c);
-  const uint8_t* w = rec + off_kc() + L.byte;
-  if (kb == 3 && kc3_is_pair15(c)) {
-    uint32_t v = 0;
-#pragma unroll
-    for (int b = 0; b < 3; ++b) v |= ((*reinterpret_cast<const uint32_t*>(w + 4 * b) >> L.bit) & 1u) << b;
-    return v;
-  }
-  return (*reinterpret_cast<const uint32_t*>(w) >> L.bit) & ((1u << kb) - 1u);
-}
-__device__ __forceinline__ uint32_t val_code(const uint8_t* rec, int kb, int vb, int tt, int c) {
-  const BitLoc L = vc_loc(vb, tt, c);
-  return (*reinterpret_cast<const uint32_t*>(rec + off_vc(kb) + L.byte) >> L.bit) &
-         ((1u << vb) - 1u);
-}
-__device__ __forceinline__ float h2f(const uint8_t* p) {
-  return __half2float(__ushort_as_half(*reinterpret_cast<const uint16_t*>(p)));
-}
-
+// The correction kernel reads the stored codes (exactly what the scan used)
+// and the stored scales/zeros straight from the packed records.
 constexpr int kRow = kD + 4;  // padded fp32 row in shared memory
 
 // grid (n_chunks, n_seg), 256 threads.  Chunk = 32 entries of (top-k list,
@@ -123,55 +103,119 @@ __global__ void __launch_bounds__(256) correct_chunk_kernel(const MergeParams p)
     const int t = s_tok[tl];
     float* krow = kx + tl * kRow + c0;
     float* vrow = vx + tl * kRow + c0;
-    if (t < 0) {
+    float* khrow = kh + tl * kRow + c0;
+    float* vhrow = vh + tl * kRow + c0;
+    const bool valid = t >= 0;
+    const bool tail = valid && (t & (1 << 30)) != 0;
+    const bool quant = valid && !tail;
+    const uint16_t *kr = nullptr, *vr = nullptr;
+    if (tail) {
+      const int tt = t & ~(1 << 30);
+      kr = p.tail_k + ((size_t)seg * kTail + tt) * kD;
+      vr = p.tail_v + ((size_t)seg * kTail + tt) * kD;
+    } else if (quant) {
+      kr = p.k_exact + ((size_t)seg * p.capacity + t) * kD;
+      vr = p.v_exact + ((size_t)seg * p.capacity + t) * kD;
+    }
+    // every load of this thread is issued before any is used
+    uint4 ka = make_uint4(0u, 0u, 0u, 0u), kb4 = ka, va = ka, vb4 = ka;
+    if (valid) {
+      ka = *reinterpret_cast<const uint4*>(kr + c0);
+      kb4 = *reinterpret_cast<const uint4*>(kr + c0 + 8);
+      va = *reinterpret_cast<const uint4*>(vr + c0);
+      vb4 = *reinterpret_cast<const uint4*>(vr + c0 + 8);
+    }
+    // key scales/zeros of channels c0..c0+15: pairs 2*part, 2*part+1 of each tig
+    uint2 ksw[4], kzw[4];
+    uint32_t kcw[4][3], vcw[8];
+    uint16_t vsb = 0, vzb = 0;
+    const int tt = quant ? t % kKG : 0;
+    if (quant) {
+      const uint8_t* rec = p.groups + ((size_t)seg * p.ng_cap + t / kKG) * p.rec_bytes;
+      const int ksrow = (part >> 1) * 64 + ((2 * part) & 3) * 4;
 #pragma unroll
-      for (int i = 0; i < 16; ++i) krow[i] = vrow[i] = 0.f;
-    } else {
-      const bool tail = (t & (1 << 30)) != 0;
-      const uint16_t *kr, *vr;
-      if (tail) {
-        const int tt = t & ~(1 << 30);
-        kr = p.tail_k + ((size_t)seg * kTail + tt) * kD;
-        vr = p.tail_v + ((size_t)seg * kTail + tt) * kD;
+      for (int tg = 0; tg < 4; ++tg) {
+        ksw[tg] = *reinterpret_cast<const uint2*>(rec + off_ks() + ksrow + tg * 16);
+        kzw[tg] = *reinterpret_cast<const uint2*>(rec + off_ks() + 256 + ksrow + tg * 16);
+      }
+      const int nt = tt >> 3, gd = tt & 7;
+      if (p.key_bits == 4) {
+#pragma unroll
+        for (int tg = 0; tg < 4; ++tg) {
+          kcw[tg][0] = *reinterpret_cast<const uint32_t*>(
+              rec + off_kc() + nt * 512 + (gd * 4 + tg) * 16 + (part >> 1) * 4);
+          kcw[tg][1] = kcw[tg][2] = 0u;
+        }
       } else {
-        kr = p.k_exact + ((size_t)seg * p.capacity + t) * kD;
-        vr = p.v_exact + ((size_t)seg * p.capacity + t) * kD;
-      }
-      const uint4 ka = *reinterpret_cast<const uint4*>(kr + c0);
-      const uint4 kb = *reinterpret_cast<const uint4*>(kr + c0 + 8);
-      const uint4 va = *reinterpret_cast<const uint4*>(vr + c0);
-      const uint4 vb = *reinterpret_cast<const uint4*>(vr + c0 + 8);
-      float khq[16], vhq[16];
-      if (!tail) {
-        const int tt = t % kKG;
-        const uint8_t* rec = p.groups + ((size_t)seg * p.ng_cap + t / kKG) * p.rec_bytes;
-        const float vs = h2f(rec + off_vs(p.key_bits) + vs_scale_off(tt, part >> 1));
-        const float vz = h2f(rec + off_vs(p.key_bits) + vs_zero_off(tt, part >> 1));
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int c = c0 + i;
-          const float s = h2f(rec + off_ks() + ks_scale_off(c));
-          const float z = h2f(rec + off_ks() + ks_zero_off(c));
-          khq[i] = fmaf(s, (float)key_code(rec, p.key_bits, tt, c), z);
-          vhq[i] = fmaf(vs, (float)val_code(rec, p.key_bits, p.val_bits, tt, c), vz);
+        for (int tg = 0; tg < 4; ++tg)
+#pragma unroll
+          for (int wd = 0; wd < 3; ++wd)
+            kcw[tg][wd] = *reinterpret_cast<const uint32_t*>(
+                rec + off_kc() + (nt >> 2) * 1536 + (gd * 4 + tg) * 48 + (nt & 3) * 12 + wd * 4);
+      }
+      // value codes: one word per channel row gid (0..7) of m-tile `part`
+      const int kk = tt >> 4, rt = tt & 15, tgt = (rt & 7) >> 1;
+      const int vco = off_vc(p.key_bits);
+#pragma unroll
+      for (int gd2 = 0; gd2 < 8; ++gd2) {
+        const int lanev = gd2 * 4 + tgt;
+        int off;
+        if (p.val_bits == 4) {
+          const int wi = kk * 8 + part;
+          off = (wi >> 2) * 512 + lanev * 16 + (wi & 3) * 4;
+        } else {
+          off = kk * 512 + lanev * 16 + (part >> 1) * 4;
         }
+        vcw[gd2] = *reinterpret_cast<const uint32_t*>(rec + vco + off);
       }
-      const uint32_t kw[8] = {ka.x, ka.y, ka.z, ka.w, kb.x, kb.y, kb.z, kb.w};
-      const uint32_t vw[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
+      vsb = *reinterpret_cast<const uint16_t*>(rec + off_vs(p.key_bits) + vs_scale_off(tt, part >> 1));
+      vzb = *reinterpret_cast<const uint16_t*>(rec + off_vs(p.key_bits) + vs_zero_off(tt, part >> 1));
+    }
+    const uint32_t kw[8] = {ka.x, ka.y, ka.z, ka.w, kb4.x, kb4.y, kb4.z, kb4.w};
+    const uint32_t vw[8] = {va.x, va.y, va.z, va.w, vb4.x, vb4.y, vb4.z, vb4.w};
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        krow[2 * i] = __uint_as_float(kw[i] << 16);
-        krow[2 * i + 1] = __uint_as_float(kw[i] & 0xFFFF0000u);
-        vrow[2 * i] = __uint_as_float(vw[i] << 16);
-        vrow[2 * i + 1] = __uint_as_float(vw[i] & 0xFFFF0000u);
-      }
-      if (!tail) {
+    for (int i = 0; i < 8; ++i) {
+      krow[2 * i] = __uint_as_float(kw[i] << 16);
+      krow[2 * i + 1] = __uint_as_float(kw[i] & 0xFFFF0000u);
+      vrow[2 * i] = __uint_as_float(vw[i] << 16);
+      vrow[2 * i + 1] = __uint_as_float(vw[i] & 0xFFFF0000u);
+    }
+    if (quant) {
+      const float vs = __half2float(__ushort_as_half(vsb));
+      const float vz = __half2float(__ushort_as_half(vzb));
+      const int rt = tt & 15, hi8 = rt >> 3, e = rt & 1;
+      // channel c0 + i, i = 2*tig + 8*hf + ec  (pair 2*part + hf of thread tig)
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          kh[tl * kRow + c0 + i] = khq[i];
-          vh[tl * kRow + c0 + i] = vhq[i];
+      for (int i = 0; i < 16; ++i) {
+        const int tg = (i & 7) >> 1, hf = i >> 3, ec = i & 1;
+        const uint32_t sw = hf ? ksw[tg].y : ksw[tg].x;
+        const uint32_t zw = hf ? kzw[tg].y : kzw[tg].x;
+        const float s = __half2float(__ushort_as_half((uint16_t)(ec ? sw >> 16 : sw & 0xFFFFu)));
+        const float z = __half2float(__ushort_as_half((uint16_t)(ec ? zw >> 16 : zw & 0xFFFFu)));
+        const int pr = 2 * part + hf;
+        uint32_t code;
+        if (p.key_bits == 4) {
+          code = (kcw[tg][0] >> (4 * (pr & 3) + 16 * ec)) & 15u;
+        } else if (pr < 15) {
+          const int wd = pr / 5;
+          const uint32_t wsel = wd == 0 ? kcw[tg][0] : (wd == 1 ? kcw[tg][1] : kcw[tg][2]);
+          code = (wsel >> (3 * (pr % 5) + 16 * ec)) & 7u;
+        } else {
+          code = ((kcw[tg][0] >> (15 + 16 * ec)) & 1u) | (((kcw[tg][1] >> (15 + 16 * ec)) & 1u) << 1) |
+                 (((kcw[tg][2] >> (15 + 16 * ec)) & 1u) << 2);
         }
+        khrow[i] = fmaf(s, (float)code, z);
+        // value channel c0 + i: row gid = i & 7, chi = i >> 3 of m-tile `part`
+        const int gd2 = i & 7, chi = i >> 3;
+        const int r = chi + 2 * hi8;
+        const uint32_t vcode = p.val_bits == 4 ? (vcw[gd2] >> (4 * r + 16 * e)) & 15u
+                                               : (vcw[gd2] >> (2 * (4 * (part & 1) + r) + 16 * e)) & 3u;
+        vhrow[i] = fmaf(vs, (float)vcode, vz);
       }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) khrow[i] = vhrow[i] = 0.f;
     }
   }
   __syncthreads();
@@ -299,9 +343,18 @@ __global__ void __launch_bounds__(256) merge_final_kernel(const MergeParams p) {
   for (int r0 = 0; r0 < nrows; r0 += kTileRows) {
     const int nr = min(kTileRows, nrows - r0);
     __syncthreads();
-    for (int i = tid; i < nr * (kPartStride / 4); i += 256) {
-      const int r = i / (kPartStride / 4), v = i % (kPartStride / 4);
-      reinterpret_cast<float4*>(tile[r])[v] = reinterpret_cast<const float4*>(row_ptr(r0 + r))[v];
+    constexpr int kVec = kPartStride / 4;  // float4 per row
+    float4 buf[(kTileRows * kVec + 255) / 256];
+#pragma unroll
+    for (int u = 0; u < (kTileRows * kVec + 255) / 256; ++u) {
+      const int i = tid + 256 * u;
+      if (i < nr * kVec)
+        buf[u] = reinterpret_cast<const float4*>(row_ptr(r0 + i / kVec))[i % kVec];
+    }
+#pragma unroll
+    for (int u = 0; u < (kTileRows * kVec + 255) / 256; ++u) {
+      const int i = tid + 256 * u;
+      if (i < nr * kVec) reinterpret_cast<float4*>(tile[i / kVec])[i % kVec] = buf[u];
     }
     __syncthreads();
     if (worker) {

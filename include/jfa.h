@@ -108,12 +108,12 @@ typedef struct jfa_workspace_layout {
   size_t off_partials;   /* fp32 split partials of the approximate scan       */
   size_t off_hist;       /* top-k histograms                                  */
   size_t off_counters;   /* top-k counters                                    */
-  size_t off_cand;       /* top-k candidate (key, index) pairs                */
-  size_t off_sel;        /* top-k selected-index lists                        */
+  size_t off_cand;       /* top-k per-chunk (key, index) lists                */
+  size_t off_sel;        /* top-k per-chunk list lengths                      */
   size_t off_merge;      /* fp32 per-chunk exact / removal partials           */
   int32_t max_topk;
   int32_t partial_slots; /* slots of off_partials                             */
-  int32_t cand_cap;      /* candidates per segment                            */
+  int32_t cand_cap;      /* list entries per segment                          */
   int32_t merge_chunks;  /* chunks of off_merge per segment                   */
 } jfa_workspace_layout;
 
