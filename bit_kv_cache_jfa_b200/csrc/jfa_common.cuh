@@ -23,6 +23,7 @@ constexpr int kPartStride = 132;         // floats per (slot, head): m, l, pad2,
 constexpr int kScanWarps = 8;            // warps per scan CTA
 constexpr int kMaxScanWarps = 2048;      // cap on scan warps (partial slots)
 constexpr int kHistBins = 2048;          // top-k first-level histogram (11 key bits)
+constexpr int kCtrStride = 8;            // top-k counters per segment: [0] scan warps done, [2] b*, [3] keys above b*
 constexpr int kMergeChunk = 32;          // tokens per correct/merge CTA
 
 // ---------------------------------------------------------------------------

@@ -4,23 +4,24 @@
 //
 // Order (S descending, index ascending); the chosen indices are written in
 // ascending index order.  Scores map to order-preserving 32-bit keys.
-//   1. histogram kernel: many CTAs per segment build a histogram of the top
-//      11 key bits; the last CTA of a segment finds the bin b* holding the
-//      k-th key and the count of keys above it.
-//   2. collect kernel: every 4096-score chunk writes the (key, index) of each
-//      score with bin >= b* to its own list, in index order (ordered
+//   0. the scan kernel (jfa_decode_scores) already left, per segment, the
+//      suffix counts of a histogram of the top 11 key bits (keys with bin >= b);
+//   1. collect kernel: every CTA finds the bin b* holding the k-th key from
+//      those counts, and every 4096-score chunk writes the (key, index) of
+//      each score with bin >= b* to its own list, in index order (ordered
 //      compaction with a block scan).
-//   3. final kernel, one CTA per segment: two radix refinements (next 11,
-//      then 10 key bits) over the short lists give the exact k-th key K*;
-//      ties at K* go to the lowest indices, which come first in list order;
-//      one ordered pass writes the chosen indices, already ascending.
+//   2. final kernel, one CTA per segment: the short lists are staged in shared
+//      memory; two radix refinements (next 11, then 10 key bits) give the
+//      exact k-th key K*; ties at K* go to the lowest indices, which come
+//      first in list order; one ordered pass writes the chosen indices,
+//      already ascending.
 #include "jfa_internal.cuh"
 
 namespace jfa {
 
 constexpr unsigned kFullMask = 0xFFFFFFFFu;
 constexpr int kTopkChunk = 4096;  // scores per CTA of the histogram / collect kernels
-constexpr int kCtrStride = 8;     // per segment: [2] b*, [3] count above b*, [4] hist CTAs done
+constexpr int kStageCap = 4096;   // list entries the final kernel stages in shared memory
 
 // Block-wide exclusive sum over threads in DESCENDING thread order:
 // returns the sum of v over threads with a larger index.
@@ -84,63 +85,12 @@ __device__ void find_from_top(const uint32_t* h, int nbins, uint32_t r, uint32_t
 
 struct TopkBufs {
   const float* scores;
-  uint32_t* hist;      // [n_seg][2048]
+  const uint32_t* hist;  // [n_seg][2048] suffix counts: keys with bin >= b
   uint32_t* counters;  // [n_seg][kCtrStride]
   uint2* lists;        // [n_seg][n_chunks_cap][kTopkChunk] (key, index)
   uint32_t* counts;    // [n_seg][n_chunks_cap]
   int capacity, nq, k, n_chunks, n_chunks_cap;
 };
-
-__global__ void __launch_bounds__(256) topk_hist_kernel(TopkBufs b) {
-  __shared__ uint32_t sh[kHistBins];
-  __shared__ uint32_t scratch[32];
-  __shared__ bool s_last;
-  __shared__ int s_bin;
-  __shared__ uint32_t s_above;
-  const int seg = blockIdx.y;
-  const int lo = blockIdx.x * kTopkChunk;
-  const float* s = b.scores + (size_t)seg * b.capacity;
-  float4 v[4];
-#pragma unroll
-  for (int r = 0; r < 4; ++r) {  // nq is a multiple of 64: a float4 is all in or all out
-    const int i = lo + 4 * (threadIdx.x + 256 * r);
-    v[r] = i < b.nq ? *reinterpret_cast<const float4*>(s + i) : make_float4(0.f, 0.f, 0.f, 0.f);
-  }
-  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) sh[i] = 0u;
-  __syncthreads();
-#pragma unroll
-  for (int r = 0; r < 4; ++r) {
-    if (lo + 4 * (threadIdx.x + 256 * r) < b.nq) {
-      atomicAdd(&sh[float_key(v[r].x) >> 21], 1u);
-      atomicAdd(&sh[float_key(v[r].y) >> 21], 1u);
-      atomicAdd(&sh[float_key(v[r].z) >> 21], 1u);
-      atomicAdd(&sh[float_key(v[r].w) >> 21], 1u);
-    }
-  }
-  __syncthreads();
-  uint32_t* gh = b.hist + (size_t)seg * kHistBins;
-  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x)
-    if (sh[i]) atomicAdd(&gh[i], sh[i]);
-  // the last CTA of the segment finds the bin holding the k-th key
-  uint32_t* ctr = b.counters + (size_t)seg * kCtrStride;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    __threadfence();
-    s_last = atomicAdd(&ctr[4], 1u) == gridDim.x - 1;
-    s_bin = 0;
-    s_above = 0;
-  }
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) sh[i] = __ldcg(&gh[i]);
-  __syncthreads();
-  find_from_top(sh, kHistBins, (uint32_t)b.k, scratch, &s_bin, &s_above);
-  if (threadIdx.x == 0) {
-    ctr[2] = (uint32_t)s_bin;
-    ctr[3] = s_above;
-  }
-}
 
 // Thread t owns the 16 consecutive scores lo + 16t .. lo + 16t + 15, so a
 // block prefix sum of per-thread counts gives index-ordered positions.
@@ -155,7 +105,29 @@ __global__ void __launch_bounds__(256) topk_collect_kernel(TopkBufs b) {
   for (int r = 0; r < 4; ++r)
     v[r] = base + 4 * r < b.nq ? *reinterpret_cast<const float4*>(s + base + 4 * r)
                                : make_float4(0.f, 0.f, 0.f, 0.f);
-  const uint32_t bstar = b.counters[(size_t)seg * kCtrStride + 2];
+  // b* = the largest bin whose suffix count reaches k (counts fall with b)
+  const uint32_t* suf = b.hist + (size_t)seg * kHistBins;
+  uint32_t sv[kHistBins / 256];
+#pragma unroll
+  for (int i = 0; i < kHistBins / 256; ++i) sv[i] = suf[(kHistBins / 256) * threadIdx.x + i];
+  int best = -1;
+#pragma unroll
+  for (int i = 0; i < kHistBins / 256; ++i)
+    if (sv[i] >= (uint32_t)b.k) best = (kHistBins / 256) * threadIdx.x + i;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) best = max(best, __shfl_xor_sync(kFullMask, best, o));
+  __shared__ int s_best[8];
+  if ((threadIdx.x & 31) == 0) s_best[threadIdx.x >> 5] = best;
+  __syncthreads();
+  best = s_best[0];
+#pragma unroll
+  for (int w = 1; w < 8; ++w) best = max(best, s_best[w]);
+  const uint32_t bstar = (uint32_t)max(best, 0);
+  if (chunk == 0 && threadIdx.x == 0) {
+    uint32_t* ctr = b.counters + (size_t)seg * kCtrStride;
+    ctr[2] = bstar;
+    ctr[3] = bstar + 1 < (uint32_t)kHistBins ? suf[bstar + 1] : 0u;
+  }
   uint32_t keys[16];
   uint32_t mask = 0, n = 0;
 #pragma unroll
@@ -182,8 +154,9 @@ __global__ void __launch_bounds__(256) topk_collect_kernel(TopkBufs b) {
 // One CTA (256 threads) per segment.
 __global__ void __launch_bounds__(256) topk_final_kernel(TopkBufs b, int32_t* idx) {
   __shared__ uint32_t h[kHistBins];
+  __shared__ uint2 st[kStageCap];
   __shared__ uint32_t scratch[32];
-  __shared__ uint32_t cnt[64];
+  __shared__ uint32_t off[65];
   __shared__ int s_bin;
   __shared__ uint32_t s_above;
   const int seg = blockIdx.x;
@@ -193,17 +166,99 @@ __global__ void __launch_bounds__(256) topk_final_kernel(TopkBufs b, int32_t* id
   const uint32_t r = (uint32_t)b.k - ctr[3];  // keys to take from bin b* (>= 1)
   const uint2* lists = b.lists + (size_t)seg * b.n_chunks_cap * kTopkChunk;
   const uint32_t* counts = b.counts + (size_t)seg * b.n_chunks_cap;
-  const bool small = b.n_chunks <= 64;
-  if (small && tid < b.n_chunks) cnt[tid] = counts[tid];
-  __syncthreads();
-  auto count_of = [&](int c) -> uint32_t { return small ? cnt[c] : counts[c]; };
-
-  // refinement 1: bits 20..10 of keys in bin b*
-  for (int i = tid; i < kHistBins; i += blockDim.x) h[i] = 0u;
+  // chunk offsets in the concatenated (index-ordered) list
+  if (tid < 32) {
+    uint32_t run = 0;
+    for (int c0 = 0; c0 < b.n_chunks; c0 += 32) {
+      const int c = c0 + tid;
+      const uint32_t v = c < b.n_chunks ? counts[c] : 0u;
+      uint32_t x = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(kFullMask, x, o);
+        if (tid >= o) x += y;
+      }
+      if (c < b.n_chunks && c < 64) off[c] = run + x - v;
+      run += __shfl_sync(kFullMask, x, 31);
+    }
+    if (tid == 0) off[min(b.n_chunks, 64)] = run;
+  }
   if (tid == 0) {
     s_bin = 0;
     s_above = 0;
   }
+  __syncthreads();
+  const uint32_t total = off[min(b.n_chunks, 64)];
+  const bool staged = b.n_chunks <= 64 && total <= (uint32_t)kStageCap;
+  int32_t* o = idx + (size_t)seg * b.k;
+
+  if (staged) {
+    // stage every list entry (loads independent of the shared-memory stores)
+#pragma unroll 4
+    for (uint32_t j = tid; j < total; j += 256) {
+      int lo = 0, hi = b.n_chunks;  // last chunk with off[c] <= j
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (off[mid] <= j) lo = mid;
+        else hi = mid;
+      }
+      st[j] = lists[(size_t)lo * kTopkChunk + (j - off[lo])];
+    }
+    for (int i = tid; i < kHistBins; i += blockDim.x) h[i] = 0u;
+    __syncthreads();
+    // refinement 1: bits 20..10 of keys in bin b*
+    for (uint32_t i = tid; i < total; i += blockDim.x) {
+      const uint32_t key = st[i].x;
+      if ((key >> 21) == bstar) atomicAdd(&h[(key >> 10) & 2047u], 1u);
+    }
+    __syncthreads();
+    find_from_top(h, 2048, r, scratch, &s_bin, &s_above);
+    const uint32_t d2 = (uint32_t)s_bin;
+    const uint32_t r2 = r - s_above;
+    const uint32_t pre = (bstar << 11) | d2;
+    for (int i = tid; i < kHistBins; i += blockDim.x) h[i] = 0u;
+    __syncthreads();
+    // refinement 2: bits 9..0 of keys with prefix (b*, d2)
+    for (uint32_t i = tid; i < total; i += blockDim.x) {
+      const uint32_t key = st[i].x;
+      if ((key >> 10) == pre) atomicAdd(&h[key & 1023u], 1u);
+    }
+    __syncthreads();
+    find_from_top(h, 1024, r2, scratch, &s_bin, &s_above);
+    const uint32_t kstar = (pre << 10) | (uint32_t)s_bin;
+    const uint32_t r3 = r2 - s_above;
+    // ordered pass; thread t owns entries [t*per, (t+1)*per) so one block scan
+    // per counter orders the whole list
+    const uint32_t per = (total + 255) / 256;
+    const uint32_t i0 = tid * per, i1 = min(total, i0 + per);
+    uint32_t n_eq = 0;
+    for (uint32_t i = i0; i < i1; ++i) n_eq += st[i].x == kstar;
+    uint32_t tot;
+    uint32_t eq_rank = block_prefix_excl(n_eq, scratch, &tot);
+    uint32_t n_ch = 0;
+    for (uint32_t i = i0; i < i1; ++i) {
+      const uint32_t key = st[i].x;
+      const bool eq = key == kstar;
+      n_ch += (key > kstar || (eq && eq_rank < r3)) ? 1u : 0u;
+      eq_rank += eq;
+    }
+    uint32_t pos = block_prefix_excl(n_ch, scratch, &tot);
+    eq_rank -= n_eq;  // back to this thread's first entry
+    for (uint32_t i = i0; i < i1; ++i) {
+      const uint2 e = st[i];
+      const bool eq = e.x == kstar;
+      if (e.x > kstar || (eq && eq_rank < r3)) {
+        if (pos < (uint32_t)b.k) o[pos] = (int32_t)e.y;
+        ++pos;
+      }
+      eq_rank += eq;
+    }
+    return;
+  }
+
+  // general path (long lists): the same steps reading the lists in place
+  auto count_of = [&](int c) -> uint32_t { return counts[c]; };
+  for (int i = tid; i < kHistBins; i += blockDim.x) h[i] = 0u;
   __syncthreads();
   for (int c = 0; c < b.n_chunks; ++c) {
     const uint32_t n = count_of(c);
@@ -217,7 +272,6 @@ __global__ void __launch_bounds__(256) topk_final_kernel(TopkBufs b, int32_t* id
   find_from_top(h, 2048, r, scratch, &s_bin, &s_above);
   const uint32_t d2 = (uint32_t)s_bin;
   const uint32_t r2 = r - s_above;
-  // refinement 2: bits 9..0 of keys with prefix (b*, d2)
   const uint32_t pre = (bstar << 11) | d2;
   for (int i = tid; i < kHistBins; i += blockDim.x) h[i] = 0u;
   __syncthreads();
@@ -232,11 +286,8 @@ __global__ void __launch_bounds__(256) topk_final_kernel(TopkBufs b, int32_t* id
   __syncthreads();
   find_from_top(h, 1024, r2, scratch, &s_bin, &s_above);
   const uint32_t kstar = (pre << 10) | (uint32_t)s_bin;
-  const uint32_t r3 = r2 - s_above;  // keys equal to K* to take, lowest indices first
-
-  // ordered pass: chosen = key > K*, or key == K* among the first r3 such
+  const uint32_t r3 = r2 - s_above;
   uint32_t out_base = 0, eq_base = 0;
-  int32_t* o = idx + (size_t)seg * b.k;
   for (int c = 0; c < b.n_chunks; ++c) {
     const uint32_t n = count_of(c);
     const uint2* L = lists + (size_t)c * kTopkChunk;
@@ -257,6 +308,75 @@ __global__ void __launch_bounds__(256) topk_final_kernel(TopkBufs b, int32_t* id
   }
 }
 
+// Histogram of the selection-score keys of caller-provided scores, turned
+// into per-segment suffix counts by the last CTA of each segment (the scan
+// kernel builds the same counts on the fly).
+__global__ void __launch_bounds__(256) score_hist_kernel(const float* scores, int capacity, int nq,
+                                                         uint32_t* hist, uint32_t* counters) {
+  __shared__ uint32_t sh[kHistBins];
+  __shared__ bool s_last;
+  const int seg = blockIdx.y;
+  const int lo = blockIdx.x * kTopkChunk;
+  const float* s = scores + (size_t)seg * capacity;
+  float4 v[4];
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const int i = lo + 4 * (threadIdx.x + 256 * r);
+    v[r] = i < nq ? *reinterpret_cast<const float4*>(s + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) sh[i] = 0u;
+  __syncthreads();
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    if (lo + 4 * (threadIdx.x + 256 * r) < nq) {
+      atomicAdd(&sh[float_key(v[r].x) >> 21], 1u);
+      atomicAdd(&sh[float_key(v[r].y) >> 21], 1u);
+      atomicAdd(&sh[float_key(v[r].z) >> 21], 1u);
+      atomicAdd(&sh[float_key(v[r].w) >> 21], 1u);
+    }
+  }
+  __syncthreads();
+  uint32_t* gh = hist + (size_t)seg * kHistBins;
+  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x)
+    if (sh[i]) atomicAdd(&gh[i], sh[i]);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    s_last = atomicAdd(&counters[(size_t)seg * kCtrStride], 1u) == gridDim.x - 1;
+  }
+  __syncthreads();
+  if (!s_last || threadIdx.x >= 32) return;
+  __threadfence();
+  const int lane = threadIdx.x;
+  uint32_t local = 0;
+  for (int i = 0; i < 64; ++i) local += __ldcg(&gh[64 * lane + i]);
+  uint32_t suf = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_down_sync(kFullMask, suf, o);
+    if (lane + o < 32) suf += y;
+  }
+  uint32_t run = suf - local;
+  for (int i = 63; i >= 0; --i) {
+    run += __ldcg(&gh[64 * lane + i]);
+    gh[64 * lane + i] = run;
+  }
+}
+
+int launch_score_histogram(const jfa_geom& g, uint8_t* ws, const jfa_workspace_layout& L,
+                           cudaStream_t st) {
+  const int n_seg = g.batch * g.num_kv_heads;
+  const int nq = split_point(g.n_ctx);
+  if (cudaMemsetAsync(ws + L.off_hist, 0, L.off_cand - L.off_hist, st) != cudaSuccess)
+    return JFA_ERR_CUDA;
+  if (nq == 0) return JFA_OK;
+  const int chunks = (nq + kTopkChunk - 1) / kTopkChunk;
+  score_hist_kernel<<<dim3(chunks, n_seg), 256, 0, st>>>(
+      reinterpret_cast<const float*>(ws + L.off_scores), g.capacity, nq,
+      reinterpret_cast<uint32_t*>(ws + L.off_hist), reinterpret_cast<uint32_t*>(ws + L.off_counters));
+  return cudaGetLastError() == cudaSuccess ? JFA_OK : JFA_ERR_CUDA;
+}
+
 __global__ void topk_fill_kernel(int32_t* idx, int k, int nq) {
   const int seg = blockIdx.y;
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < k; i += gridDim.x * blockDim.x)
@@ -265,7 +385,7 @@ __global__ void topk_fill_kernel(int32_t* idx, int k, int nq) {
 
 int count_topk_launches(const jfa_geom& g, int k) {
   const int nq = split_point(g.n_ctx);
-  return k >= nq ? 1 : 3;  // fill | hist + collect + final (plus one memset)
+  return k >= nq ? 1 : 2;  // fill | collect + final
 }
 
 int launch_topk(const jfa_geom& g, int k, uint8_t* ws, const jfa_workspace_layout& L,
@@ -287,10 +407,6 @@ int launch_topk(const jfa_geom& g, int k, uint8_t* ws, const jfa_workspace_layou
   b.k = k;
   b.n_chunks = (nq + kTopkChunk - 1) / kTopkChunk;
   b.n_chunks_cap = (g.capacity + kTopkChunk - 1) / kTopkChunk;
-  // histograms and counters are contiguous: clear both at once
-  if (cudaMemsetAsync(ws + L.off_hist, 0, L.off_cand - L.off_hist, st) != cudaSuccess)
-    return JFA_ERR_CUDA;
-  topk_hist_kernel<<<dim3(b.n_chunks, n_seg), 256, 0, st>>>(b);
   topk_collect_kernel<<<dim3(b.n_chunks, n_seg), 256, 0, st>>>(b);
   topk_final_kernel<<<n_seg, 256, 0, st>>>(b, idx);
   return cudaGetLastError() == cudaSuccess ? JFA_OK : JFA_ERR_CUDA;

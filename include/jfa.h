@@ -78,7 +78,7 @@ typedef struct jfa_geom {
 } jfa_geom;
 
 /* Device buffers of one layer's quantized cache (caller-allocated with the
- * sizes jfa_cache_layout reports; every pointer 256-byte aligned).
+ * sizes jfa_cache_layout_get reports; every pointer 16-byte aligned).
  *   groups : packed group records, [B][H_kv][capacity/64][record_bytes].
  *            A record holds the codes and fp16 scales/zeros of the keys and
  *            values of 64 consecutive tokens, in a layout private to this
@@ -100,7 +100,7 @@ typedef struct jfa_cache_layout {
 
 /* Workspace layout: scratch of the decode step (selection scores, split
  * softmax partials, top-k histograms/candidates, merge partials, the error
- * flag).  Sized by jfa_workspace_bytes for a geometry and a maximum k. */
+ * flag).  Sized by jfa_workspace_layout_get for a geometry and a maximum k. */
 typedef struct jfa_workspace_layout {
   size_t total_bytes;
   size_t off_flag;       /* uint32 device error flag                          */
@@ -173,9 +173,17 @@ int jfa_decode_scores(const jfa_geom* geom, const jfa_cache* cache,
  * per KV head).  Order is (S descending, index ascending); the k_eff =
  * min(k, N_q) chosen indices are written sorted ascending to
  * idx[B][H_kv][k] (int32 device pointer), the remaining k - k_eff entries
- * set to -1.  1 <= k <= max_topk of the workspace. */
+ * set to -1.  1 <= k <= max_topk of the workspace.
+ * Reads the selection scores and their key histogram that jfa_decode_scores
+ * leaves in the workspace (or that jfa_score_histogram rebuilds). */
 int jfa_topk(const jfa_geom* geom, int32_t k, void* ws, int32_t* idx,
              void* stream);
+
+/* jfa_score_histogram — rebuild the selection-score key histogram that
+ * jfa_topk reads, from the scores currently in the workspace (off_scores).
+ * jfa_decode_scores builds it on the fly; call this only after writing the
+ * scores yourself. */
+int jfa_score_histogram(const jfa_geom* geom, void* ws, void* stream);
 
 /* jfa_correct_merge — exact correction and log-sum-exp merge.
  * For every query head: exact logits scale*q.K_t from the bf16 copy for the
