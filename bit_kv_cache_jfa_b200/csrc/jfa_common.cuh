@@ -323,6 +323,14 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   return false;
 }
 
+// Programmatic dependent launch: wait for the preceding kernel of the stream
+// (its writes visible) / let the next kernel of the stream start launching.
+// Both are no-ops for a kernel launched without the PDL attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ void set_flag(uint32_t* flag, uint32_t bits) {
   if (flag) atomicOr(flag, bits);
 }

@@ -3,7 +3,28 @@
 
 #include "jfa_common.cuh"
 
+#include <utility>
+
 namespace jfa {
+
+// Launch with programmatic stream serialization, so the kernel may be
+// scheduled while the previous kernel of the stream drains; the kernel calls
+// pdl_wait() before touching anything the previous kernel writes.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // Workspace layout for (geometry, max_topk); host and device agree on it.
 int workspace_layout(const jfa_geom& g, int max_topk, jfa_workspace_layout* out);

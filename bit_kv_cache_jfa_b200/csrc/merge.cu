@@ -53,6 +53,13 @@ __device__ __forceinline__ float warp_sum(float v) {
 // and the stored scales/zeros straight from the packed records.
 constexpr int kRow = kD + 4;  // padded fp32 row in shared memory
 
+// a[i] for a runtime i without spilling the array to local memory
+__device__ __forceinline__ uint32_t pick8(const uint32_t (&a)[8], int i) {
+  const uint32_t lo = (i & 2) ? ((i & 1) ? a[3] : a[2]) : ((i & 1) ? a[1] : a[0]);
+  const uint32_t hi = (i & 2) ? ((i & 1) ? a[7] : a[6]) : ((i & 1) ? a[5] : a[4]);
+  return (i & 4) ? hi : lo;
+}
+
 // grid (n_chunks, n_seg), 256 threads.  Chunk = 32 entries of (top-k list,
 // then tail).  Phase A: thread (token slot, 16-channel part) stages the exact
 // bf16 rows and the dequantized rows of its token in shared memory (all its
@@ -76,6 +83,8 @@ __global__ void __launch_bounds__(256) correct_chunk_kernel(const MergeParams p)
   const int seg = blockIdx.y, chunk = blockIdx.x;
   const int tid = threadIdx.x;
   const int b = seg / p.hkv, h = seg % p.hkv;
+  pdl_wait();
+  pdl_launch_dependents();
 
   if (tid < kMergeChunk) {
     const int e = chunk * kMergeChunk + tid;
@@ -97,125 +106,149 @@ __global__ void __launch_bounds__(256) correct_chunk_kernel(const MergeParams p)
   }
   __syncthreads();
 
-  // ---- phase A ----
+  // ---- phase A: stage the chunk's rows in shared memory.  Jobs move 16-byte
+  // vectors; every load of a thread is issued before any is used.
+  //   rows : 32 tokens x (K, V) x 16 pieces of 8 bf16  (4 jobs per thread)
+  //   keys : 32 tokens x 4 fragment threads tig: 32 codes + their scales/zeros
+  //   vals : 32 tokens x (8 or 16) fragment slots: codes of 4 or 8 m-tiles
   {
-    const int tl = tid >> 3, part = tid & 7, c0 = 16 * part;
-    const int t = s_tok[tl];
-    float* krow = kx + tl * kRow + c0;
-    float* vrow = vx + tl * kRow + c0;
-    float* khrow = kh + tl * kRow + c0;
-    float* vhrow = vh + tl * kRow + c0;
-    const bool valid = t >= 0;
-    const bool tail = valid && (t & (1 << 30)) != 0;
-    const bool quant = valid && !tail;
-    const uint16_t *kr = nullptr, *vr = nullptr;
-    if (tail) {
-      const int tt = t & ~(1 << 30);
-      kr = p.tail_k + ((size_t)seg * kTail + tt) * kD;
-      vr = p.tail_v + ((size_t)seg * kTail + tt) * kD;
-    } else if (quant) {
-      kr = p.k_exact + ((size_t)seg * p.capacity + t) * kD;
-      vr = p.v_exact + ((size_t)seg * p.capacity + t) * kD;
-    }
-    // every load of this thread is issued before any is used
-    uint4 ka = make_uint4(0u, 0u, 0u, 0u), kb4 = ka, va = ka, vb4 = ka;
-    if (valid) {
-      ka = *reinterpret_cast<const uint4*>(kr + c0);
-      kb4 = *reinterpret_cast<const uint4*>(kr + c0 + 8);
-      va = *reinterpret_cast<const uint4*>(vr + c0);
-      vb4 = *reinterpret_cast<const uint4*>(vr + c0 + 8);
-    }
-    // key scales/zeros of channels c0..c0+15: pairs 2*part, 2*part+1 of each tig
-    uint2 ksw[4], kzw[4];
-    uint32_t kcw[4][3], vcw[8];
-    uint16_t vsb = 0, vzb = 0;
-    const int tt = quant ? t % kKG : 0;
-    if (quant) {
-      const uint8_t* rec = p.groups + ((size_t)seg * p.ng_cap + t / kKG) * p.rec_bytes;
-      const int ksrow = (part >> 1) * 64 + ((2 * part) & 3) * 4;
+    // rows
 #pragma unroll
-      for (int tg = 0; tg < 4; ++tg) {
-        ksw[tg] = *reinterpret_cast<const uint2*>(rec + off_ks() + ksrow + tg * 16);
-        kzw[tg] = *reinterpret_cast<const uint2*>(rec + off_ks() + 256 + ksrow + tg * 16);
+    for (int u = 0; u < 4; ++u) {
+      const int j = tid + 256 * u;
+      const int tl = j >> 5, part = j & 31, isv = part >> 4, piece = part & 15;
+      const int t = s_tok[tl];
+      uint4 w = make_uint4(0u, 0u, 0u, 0u);
+      if (t >= 0) {
+        const uint16_t* row;
+        if (t & (1 << 30)) {
+          const int tt = t & ~(1 << 30);
+          row = (isv ? p.tail_v : p.tail_k) + ((size_t)seg * kTail + tt) * kD;
+        } else {
+          row = (isv ? p.v_exact : p.k_exact) + ((size_t)seg * p.capacity + t) * kD;
+        }
+        w = *reinterpret_cast<const uint4*>(row + 8 * piece);
       }
-      const int nt = tt >> 3, gd = tt & 7;
-      if (p.key_bits == 4) {
+      float* dst = (isv ? vx : kx) + tl * kRow + 8 * piece;
+      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-        for (int tg = 0; tg < 4; ++tg) {
-          kcw[tg][0] = *reinterpret_cast<const uint32_t*>(
-              rec + off_kc() + nt * 512 + (gd * 4 + tg) * 16 + (part >> 1) * 4);
-          kcw[tg][1] = kcw[tg][2] = 0u;
+      for (int i = 0; i < 4; ++i) {
+        dst[2 * i] = __uint_as_float(ww[i] << 16);
+        dst[2 * i + 1] = __uint_as_float(ww[i] & 0xFFFF0000u);
+      }
+    }
+    // keys: thread tid < 128 -> (token tid/4, fragment thread tig = tid%4)
+    if (tid < 4 * kMergeChunk) {
+      const int tl = tid >> 2, tg = tid & 3;
+      const int t = s_tok[tl];
+      float* dst = kh + tl * kRow;
+      if (t >= 0 && !(t & (1 << 30))) {
+        const int tt = t % kKG, nt = tt >> 3, gd = tt & 7;
+        const uint8_t* rec = p.groups + ((size_t)seg * p.ng_cap + t / kKG) * p.rec_bytes;
+        uint4 sz[8];  // chunks 0..3: scale pairs 0..15, chunks 4..7: zero pairs
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          sz[i] = *reinterpret_cast<const uint4*>(rec + off_ks() + i * 64 + tg * 16);
+        uint32_t cw[3];
+        if (p.key_bits == 4) {
+          const uint4 c4 = *reinterpret_cast<const uint4*>(rec + off_kc() + nt * 512 +
+                                                           (gd * 4 + tg) * 16);
+          cw[0] = c4.x;
+          cw[1] = c4.y;
+          cw[2] = c4.z;
+          const uint32_t c3 = c4.w;
+#pragma unroll
+          for (int pr = 0; pr < 16; ++pr) {
+            const uint32_t word = pr < 4 ? cw[0] : (pr < 8 ? cw[1] : (pr < 12 ? cw[2] : c3));
+            const uint4 sq = sz[pr >> 2], zq = sz[4 + (pr >> 2)];
+            const uint32_t sw = (pr & 3) == 0 ? sq.x : ((pr & 3) == 1 ? sq.y : ((pr & 3) == 2 ? sq.z : sq.w));
+            const uint32_t zw = (pr & 3) == 0 ? zq.x : ((pr & 3) == 1 ? zq.y : ((pr & 3) == 2 ? zq.z : zq.w));
+            const float2 s2 = unpack_h2(sw), z2 = unpack_h2(zw);
+            const int c = 16 * (pr >> 1) + 2 * tg + 8 * (pr & 1);
+            const int pos = 4 * (pr & 3);
+            dst[c] = fmaf(s2.x, (float)((word >> pos) & 15u), z2.x);
+            dst[c + 1] = fmaf(s2.y, (float)((word >> (pos + 16)) & 15u), z2.y);
+          }
+        } else {
+          const uint8_t* cp = rec + off_kc() + (nt >> 2) * 1536 + (gd * 4 + tg) * 48 + (nt & 3) * 12;
+          cw[0] = *reinterpret_cast<const uint32_t*>(cp);
+          cw[1] = *reinterpret_cast<const uint32_t*>(cp + 4);
+          cw[2] = *reinterpret_cast<const uint32_t*>(cp + 8);
+#pragma unroll
+          for (int pr = 0; pr < 16; ++pr) {
+            const uint4 sq = sz[pr >> 2], zq = sz[4 + (pr >> 2)];
+            const uint32_t sw = (pr & 3) == 0 ? sq.x : ((pr & 3) == 1 ? sq.y : ((pr & 3) == 2 ? sq.z : sq.w));
+            const uint32_t zw = (pr & 3) == 0 ? zq.x : ((pr & 3) == 1 ? zq.y : ((pr & 3) == 2 ? zq.z : zq.w));
+            const float2 s2 = unpack_h2(sw), z2 = unpack_h2(zw);
+            uint32_t c0v, c1v;
+            if (pr < 15) {
+              const uint32_t word = cw[pr / 5];
+              const int pos = 3 * (pr % 5);
+              c0v = (word >> pos) & 7u;
+              c1v = (word >> (pos + 16)) & 7u;
+            } else {
+              c0v = ((cw[0] >> 15) & 1u) | (((cw[1] >> 15) & 1u) << 1) | (((cw[2] >> 15) & 1u) << 2);
+              c1v = ((cw[0] >> 31) & 1u) | (((cw[1] >> 31) & 1u) << 1) | (((cw[2] >> 31) & 1u) << 2);
+            }
+            const int c = 16 * (pr >> 1) + 2 * tg + 8 * (pr & 1);
+            dst[c] = fmaf(s2.x, (float)c0v, z2.x);
+            dst[c + 1] = fmaf(s2.y, (float)c1v, z2.y);
+          }
         }
       } else {
 #pragma unroll
-        for (int tg = 0; tg < 4; ++tg)
-#pragma unroll
-          for (int wd = 0; wd < 3; ++wd)
-            kcw[tg][wd] = *reinterpret_cast<const uint32_t*>(
-                rec + off_kc() + (nt >> 2) * 1536 + (gd * 4 + tg) * 48 + (nt & 3) * 12 + wd * 4);
-      }
-      // value codes: one word per channel row gid (0..7) of m-tile `part`
-      const int kk = tt >> 4, rt = tt & 15, tgt = (rt & 7) >> 1;
-      const int vco = off_vc(p.key_bits);
-#pragma unroll
-      for (int gd2 = 0; gd2 < 8; ++gd2) {
-        const int lanev = gd2 * 4 + tgt;
-        int off;
-        if (p.val_bits == 4) {
-          const int wi = kk * 8 + part;
-          off = (wi >> 2) * 512 + lanev * 16 + (wi & 3) * 4;
-        } else {
-          off = kk * 512 + lanev * 16 + (part >> 1) * 4;
+        for (int pr = 0; pr < 16; ++pr) {
+          const int c = 16 * (pr >> 1) + 2 * tg + 8 * (pr & 1);
+          dst[c] = dst[c + 1] = 0.f;
         }
-        vcw[gd2] = *reinterpret_cast<const uint32_t*>(rec + vco + off);
       }
-      vsb = *reinterpret_cast<const uint16_t*>(rec + off_vs(p.key_bits) + vs_scale_off(tt, part >> 1));
-      vzb = *reinterpret_cast<const uint16_t*>(rec + off_vs(p.key_bits) + vs_zero_off(tt, part >> 1));
     }
-    const uint32_t kw[8] = {ka.x, ka.y, ka.z, ka.w, kb4.x, kb4.y, kb4.z, kb4.w};
-    const uint32_t vw[8] = {va.x, va.y, va.z, va.w, vb4.x, vb4.y, vb4.z, vb4.w};
+    // values: (token, slot); a slot is one fragment lane's 16 bytes of codes
+    const int slots = p.val_bits == 4 ? 16 : 8;
+    for (int j = tid; j < kMergeChunk * slots; j += 256) {
+      const int tl = j / slots, slot = j % slots;
+      const int t = s_tok[tl];
+      float* dst = vh + tl * kRow;
+      const int gd = slot & 7;
+      if (t >= 0 && !(t & (1 << 30))) {
+        const int tt = t % kKG, kk = tt >> 4, rt = tt & 15;
+        const int hi8 = rt >> 3, tgt = (rt & 7) >> 1, e = rt & 1;
+        const uint8_t* rec = p.groups + ((size_t)seg * p.ng_cap + t / kKG) * p.rec_bytes;
+        const uint8_t* vs = rec + off_vs(p.key_bits) + kk * 128 + tgt * 32;
+        const uint4 sa = *reinterpret_cast<const uint4*>(vs), sb = *reinterpret_cast<const uint4*>(vs + 16);
+        const uint4 za = *reinterpret_cast<const uint4*>(vs + 512);
+        const uint4 zb = *reinterpret_cast<const uint4*>(vs + 528);
+        const uint32_t sws[8] = {sa.x, sa.y, sa.z, sa.w, sb.x, sb.y, sb.z, sb.w};
+        const uint32_t zws[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
+        const int chunk = p.val_bits == 4 ? 2 * kk + (slot >> 3) : kk;
+        const uint4 cv = *reinterpret_cast<const uint4*>(rec + off_vc(p.key_bits) + chunk * 512 +
+                                                         (gd * 4 + tgt) * 16);
+        const uint32_t cws[4] = {cv.x, cv.y, cv.z, cv.w};
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      krow[2 * i] = __uint_as_float(kw[i] << 16);
-      krow[2 * i + 1] = __uint_as_float(kw[i] & 0xFFFF0000u);
-      vrow[2 * i] = __uint_as_float(vw[i] << 16);
-      vrow[2 * i + 1] = __uint_as_float(vw[i] & 0xFFFF0000u);
-    }
-    if (quant) {
-      const float vs = __half2float(__ushort_as_half(vsb));
-      const float vz = __half2float(__ushort_as_half(vzb));
-      const int rt = tt & 15, hi8 = rt >> 3, e = rt & 1;
-      // channel c0 + i, i = 2*tig + 8*hf + ec  (pair 2*part + hf of thread tig)
+        for (int wd = 0; wd < 4; ++wd) {
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int tg = (i & 7) >> 1, hf = i >> 3, ec = i & 1;
-        const uint32_t sw = hf ? ksw[tg].y : ksw[tg].x;
-        const uint32_t zw = hf ? kzw[tg].y : kzw[tg].x;
-        const float s = __half2float(__ushort_as_half((uint16_t)(ec ? sw >> 16 : sw & 0xFFFFu)));
-        const float z = __half2float(__ushort_as_half((uint16_t)(ec ? zw >> 16 : zw & 0xFFFFu)));
-        const int pr = 2 * part + hf;
-        uint32_t code;
-        if (p.key_bits == 4) {
-          code = (kcw[tg][0] >> (4 * (pr & 3) + 16 * ec)) & 15u;
-        } else if (pr < 15) {
-          const int wd = pr / 5;
-          const uint32_t wsel = wd == 0 ? kcw[tg][0] : (wd == 1 ? kcw[tg][1] : kcw[tg][2]);
-          code = (wsel >> (3 * (pr % 5) + 16 * ec)) & 7u;
-        } else {
-          code = ((kcw[tg][0] >> (15 + 16 * ec)) & 1u) | (((kcw[tg][1] >> (15 + 16 * ec)) & 1u) << 1) |
-                 (((kcw[tg][2] >> (15 + 16 * ec)) & 1u) << 2);
+          for (int em = 0; em < 2; ++em) {
+            if (p.val_bits == 4 && em == 1) continue;
+            const int mt = p.val_bits == 4 ? 4 * (slot >> 3) + wd : 2 * wd + em;
+            const int jg = mt >> 1;  // value group of channels 16mt..16mt+15
+            const uint32_t sw = pick8(sws, 2 * jg + hi8), zw = pick8(zws, 2 * jg + hi8);
+            const float sv = __half2float(__ushort_as_half((uint16_t)(e ? sw >> 16 : sw & 0xFFFFu)));
+            const float zv = __half2float(__ushort_as_half((uint16_t)(e ? zw >> 16 : zw & 0xFFFFu)));
+#pragma unroll
+            for (int chi = 0; chi < 2; ++chi) {
+              const int r = chi + 2 * hi8;
+              const uint32_t code = p.val_bits == 4 ? (cws[wd] >> (4 * r + 16 * e)) & 15u
+                                                    : (cws[wd] >> (2 * (4 * em + r) + 16 * e)) & 3u;
+              dst[16 * mt + gd + 8 * chi] = fmaf(sv, (float)code, zv);
+            }
+          }
         }
-        khrow[i] = fmaf(s, (float)code, z);
-        // value channel c0 + i: row gid = i & 7, chi = i >> 3 of m-tile `part`
-        const int gd2 = i & 7, chi = i >> 3;
-        const int r = chi + 2 * hi8;
-        const uint32_t vcode = p.val_bits == 4 ? (vcw[gd2] >> (4 * r + 16 * e)) & 15u
-                                               : (vcw[gd2] >> (2 * (4 * (part & 1) + r) + 16 * e)) & 3u;
-        vhrow[i] = fmaf(vs, (float)vcode, vz);
+      } else {
+        for (int mt = 0; mt < 8; ++mt) {
+          if (p.val_bits == 4 && (mt >> 2) != (slot >> 3)) continue;
+          dst[16 * mt + gd] = dst[16 * mt + gd + 8] = 0.f;
+        }
       }
-    } else {
-#pragma unroll
-      for (int i = 0; i < 16; ++i) khrow[i] = vhrow[i] = 0.f;
     }
   }
   __syncthreads();
@@ -321,6 +354,8 @@ __global__ void __launch_bounds__(256) merge_final_kernel(const MergeParams p) {
   __shared__ __align__(16) float tile[kTileRows][kPartStride];
   const int seg = blockIdx.x, j = blockIdx.y;
   const int tid = threadIdx.x;
+  pdl_wait();
+  pdl_launch_dependents();
   long long w0 = 0, w1 = -1;
   if (p.ng > 0) {
     const long long T = p.scan_total, W = p.scan_warps;
@@ -432,8 +467,8 @@ static void launch_cm_t(const MergeParams& p, int n_seg, cudaStream_t st) {
                          smem);
     configured[dev] = true;
   }
-  correct_chunk_kernel<G><<<dim3(p.n_chunks, n_seg), 256, smem, st>>>(p);
-  merge_final_kernel<G><<<dim3(n_seg, G), 256, 0, st>>>(p);
+  launch_pdl(correct_chunk_kernel<G>, dim3(p.n_chunks, n_seg), dim3(256), (size_t)smem, st, p);
+  launch_pdl(merge_final_kernel<G>, dim3(n_seg, G), dim3(256), 0, st, p);
 }
 
 int launch_correct_merge(const jfa_geom& g, const jfa_cache& c, const uint16_t* q, float scale,

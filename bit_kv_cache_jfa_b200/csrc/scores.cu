@@ -35,8 +35,6 @@ struct ScanParams {
   const uint16_t* q;
   float* scores;
   float* partials;
-  uint32_t* hist;   // [n_seg][2048] selection-score key histogram -> suffix counts
-  uint32_t* done;   // [n_seg][kCtrStride], word 0: warps finished with the segment
   uint32_t* flag;
   long long total;  // n_seg * ng
   int ng, ng_cap, capacity;
@@ -59,9 +57,8 @@ template <int KB, int VB>
 struct ScanCfg {
   static constexpr int REC = 512 + 1024 * KB + 1024 + 1024 * VB;
   // three ring stages per warp when they fit in shared memory, else two
-  static constexpr int HIST = kScanWarps * kHistBins * 4;  // one key histogram per warp
-  static constexpr int STAGES = (kScanWarps * 3 * REC + HIST + 1024 <= 227 * 1024) ? 3 : 2;
-  static constexpr int SMEM = kScanWarps * STAGES * REC + HIST + kScanWarps * STAGES * 8;
+  static constexpr int STAGES = (kScanWarps * 3 * REC + 1024 <= 227 * 1024) ? 3 : 2;
+  static constexpr int SMEM = kScanWarps * STAGES * REC + kScanWarps * STAGES * 8;
 };
 
 template <int KB, int VB>
@@ -75,6 +72,8 @@ __global__ void __launch_bounds__(kScanWarps * 32, 1) scan_kernel(const ScanPara
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gid = lane >> 2, tig = lane & 3;
+  pdl_wait();
+  pdl_launch_dependents();
   const long long wg = (long long)blockIdx.x * kScanWarps + warp;
   if (wg >= p.n_warps) return;
   const long long W = p.n_warps, T = p.total;
@@ -82,11 +81,7 @@ __global__ void __launch_bounds__(kScanWarps * 32, 1) scan_kernel(const ScanPara
   if (g0 >= g1) return;
 
   uint8_t* ring = smem + (size_t)warp * S * REC;
-  uint32_t* hist = reinterpret_cast<uint32_t*>(smem + (size_t)kScanWarps * S * REC) +
-                   warp * kHistBins;
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + (size_t)kScanWarps * S * REC +
-                                              ScanCfg<KB, VB>::HIST) + warp * S;
-  for (int i = lane; i < kHistBins; i += 32) hist[i] = 0u;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + (size_t)kScanWarps * S * REC) + warp * S;
   const uint64_t pol = policy_evict_first();
   if (lane == 0) {
 #pragma unroll
@@ -138,46 +133,7 @@ __global__ void __launch_bounds__(kScanWarps * 32, 1) scan_kernel(const ScanPara
     }
   };
 
-  // Add this warp's key histogram of segment seg to the global one; the last
-  // warp to finish the segment turns it into suffix counts (keys with bin >= b).
-  auto flush_hist = [&](long long seg) {
-    uint32_t* gh = p.hist + (size_t)seg * kHistBins;
-    for (int i = lane; i < kHistBins; i += 32) {
-      const uint32_t v = hist[i];
-      if (v) {
-        atomicAdd(&gh[i], v);
-        hist[i] = 0u;
-      }
-    }
-    __syncwarp();
-    const long long x0 = seg * p.ng, x1 = x0 + p.ng - 1;
-    const uint32_t n_contrib = (uint32_t)(scan_warp_of(x1, W, T) - scan_warp_of(x0, W, T) + 1);
-    uint32_t last = 0;
-    if (lane == 0) {
-      __threadfence();
-      last = atomicAdd(&p.done[seg * kCtrStride], 1u) == n_contrib - 1 ? 1u : 0u;
-    }
-    last = __shfl_sync(kFull, last, 0);
-    if (!last) return;
-    __threadfence();
-    // lane l owns bins [64l, 64l + 64)
-    uint32_t local = 0;
-    for (int i = 0; i < 64; ++i) local += __ldcg(&gh[64 * lane + i]);
-    uint32_t suf = local;  // inclusive suffix over lanes >= l
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t y = __shfl_down_sync(kFull, suf, o);
-      if (lane + o < 32) suf += y;
-    }
-    uint32_t run = suf - local;  // keys in bins above this lane's range
-    for (int i = 63; i >= 0; --i) {
-      run += __ldcg(&gh[64 * lane + i]);
-      gh[64 * lane + i] = run;
-    }
-  };
-
   auto flush = [&](long long seg) {
-    flush_hist(seg);
     float* base = p.partials + (size_t)(wg + seg) * p.G * kPartStride;
     float zj[4][2];
 #pragma unroll
@@ -364,8 +320,6 @@ __global__ void __launch_bounds__(kScanWarps * 32, 1) scan_kernel(const ScanPara
       o.y = s2[1] * kLn2;
       *reinterpret_cast<float2*>(p.scores + (size_t)seg * p.capacity + (size_t)g * kKG +
                                  8 * gid + 2 * tig) = o;
-      atomicAdd(&hist[float_key(o.x) >> 21], 1u);
-      atomicAdd(&hist[float_key(o.y) >> 21], 1u);
     }
 
     // ---- probabilities: fp16 pairs (tokens 8nt+2tig, +1) and their rounding
@@ -455,24 +409,21 @@ static int launch_scan_t(const ScanParams& sp, int n_ctas, cudaStream_t st) {
       return JFA_ERR_CUDA;
     configured = true;
   }
-  scan_kernel<KB, VB><<<n_ctas, kScanWarps * 32, smem, st>>>(sp);
-  return cudaGetLastError() == cudaSuccess ? JFA_OK : JFA_ERR_CUDA;
+  return launch_pdl(scan_kernel<KB, VB>, dim3(n_ctas), dim3(kScanWarps * 32), (size_t)smem, st,
+                    sp) == cudaSuccess
+             ? JFA_OK
+             : JFA_ERR_CUDA;
 }
 
 int launch_scores(const jfa_geom& g, const jfa_cache& c, const uint16_t* q, float scale,
                   uint8_t* ws, const jfa_workspace_layout& L, cudaStream_t st) {
   ScanPlan plan = scan_plan(g, num_sms_current());
   if (plan.total_groups == 0) return JFA_OK;
-  // key histograms and per-segment completion counters are contiguous
-  if (cudaMemsetAsync(ws + L.off_hist, 0, L.off_cand - L.off_hist, st) != cudaSuccess)
-    return JFA_ERR_CUDA;
   ScanParams sp;
   sp.groups = static_cast<const uint8_t*>(c.groups);
   sp.q = q;
   sp.scores = reinterpret_cast<float*>(ws + L.off_scores);
   sp.partials = reinterpret_cast<float*>(ws + L.off_partials);
-  sp.hist = reinterpret_cast<uint32_t*>(ws + L.off_hist);
-  sp.done = reinterpret_cast<uint32_t*>(ws + L.off_counters);
   sp.flag = reinterpret_cast<uint32_t*>(ws + L.off_flag);
   sp.total = plan.total_groups;
   sp.ng = plan.ng;

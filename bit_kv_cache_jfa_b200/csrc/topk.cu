@@ -4,8 +4,9 @@
 //
 // Order (S descending, index ascending); the chosen indices are written in
 // ascending index order.  Scores map to order-preserving 32-bit keys.
-//   0. the scan kernel (jfa_decode_scores) already left, per segment, the
-//      suffix counts of a histogram of the top 11 key bits (keys with bin >= b);
+//   0. histogram kernel: many CTAs per segment count the top 11 key bits; the
+//      last CTA of a segment turns the counts into suffix counts (keys with
+//      bin >= b);
 //   1. collect kernel: every CTA finds the bin b* holding the k-th key from
 //      those counts, and every 4096-score chunk writes the (key, index) of
 //      each score with bin >= b* to its own list, in index order (ordered
@@ -14,7 +15,8 @@
 //      memory; two radix refinements (next 11, then 10 key bits) give the
 //      exact k-th key K*; ties at K* go to the lowest indices, which come
 //      first in list order; one ordered pass writes the chosen indices,
-//      already ascending.
+//      already ascending; it then clears the segment's histogram and counters
+//      for the next call (the workspace starts zero-filled).
 #include "jfa_internal.cuh"
 
 namespace jfa {
@@ -96,6 +98,8 @@ struct TopkBufs {
 // block prefix sum of per-thread counts gives index-ordered positions.
 __global__ void __launch_bounds__(256) topk_collect_kernel(TopkBufs b) {
   __shared__ uint32_t scratch[32];
+  pdl_wait();
+  pdl_launch_dependents();
   const int seg = blockIdx.y, chunk = blockIdx.x;
   const int lo = chunk * kTopkChunk;
   const int base = lo + 16 * threadIdx.x;
@@ -151,9 +155,19 @@ __global__ void __launch_bounds__(256) topk_collect_kernel(TopkBufs b) {
   if (threadIdx.x == 0) b.counts[(size_t)seg * b.n_chunks_cap + chunk] = total;
 }
 
+// Zero a segment's histogram and counters (all their readers are done).
+__device__ __forceinline__ void clear_segment(uint32_t* hist, uint32_t* counters, int seg) {
+  __syncthreads();
+  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) hist[(size_t)seg * kHistBins + i] = 0u;
+  if (threadIdx.x < kCtrStride) counters[(size_t)seg * kCtrStride + threadIdx.x] = 0u;
+}
+
 // One CTA (256 threads) per segment.
-__global__ void __launch_bounds__(256) topk_final_kernel(TopkBufs b, int32_t* idx) {
+__global__ void __launch_bounds__(256) topk_final_kernel(TopkBufs b, int32_t* idx,
+                                                         uint32_t* hist_clear) {
   __shared__ uint32_t h[kHistBins];
+  pdl_wait();
+  pdl_launch_dependents();
   __shared__ uint2 st[kStageCap];
   __shared__ uint32_t scratch[32];
   __shared__ uint32_t off[65];
@@ -253,6 +267,7 @@ __global__ void __launch_bounds__(256) topk_final_kernel(TopkBufs b, int32_t* id
       }
       eq_rank += eq;
     }
+    clear_segment(hist_clear, b.counters, seg);
     return;
   }
 
@@ -306,6 +321,7 @@ __global__ void __launch_bounds__(256) topk_final_kernel(TopkBufs b, int32_t* id
       eq_base += eq_tot;
     }
   }
+  clear_segment(hist_clear, b.counters, seg);
 }
 
 // Histogram of the selection-score keys of caller-provided scores, turned
@@ -315,6 +331,8 @@ __global__ void __launch_bounds__(256) score_hist_kernel(const float* scores, in
                                                          uint32_t* hist, uint32_t* counters) {
   __shared__ uint32_t sh[kHistBins];
   __shared__ bool s_last;
+  pdl_wait();
+  pdl_launch_dependents();
   const int seg = blockIdx.y;
   const int lo = blockIdx.x * kTopkChunk;
   const float* s = scores + (size_t)seg * capacity;
@@ -379,13 +397,15 @@ int launch_score_histogram(const jfa_geom& g, uint8_t* ws, const jfa_workspace_l
 
 __global__ void topk_fill_kernel(int32_t* idx, int k, int nq) {
   const int seg = blockIdx.y;
+  pdl_wait();
+  pdl_launch_dependents();
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < k; i += gridDim.x * blockDim.x)
     idx[(size_t)seg * k + i] = i < nq ? i : -1;
 }
 
 int count_topk_launches(const jfa_geom& g, int k) {
   const int nq = split_point(g.n_ctx);
-  return k >= nq ? 1 : 2;  // fill | collect + final
+  return k >= nq ? 1 : 3;  // fill | histogram + collect + final
 }
 
 int launch_topk(const jfa_geom& g, int k, uint8_t* ws, const jfa_workspace_layout& L,
@@ -393,12 +413,14 @@ int launch_topk(const jfa_geom& g, int k, uint8_t* ws, const jfa_workspace_layou
   const int n_seg = g.batch * g.num_kv_heads;
   const int nq = split_point(g.n_ctx);
   if (k >= nq) {
-    topk_fill_kernel<<<dim3((k + 255) / 256, n_seg), 256, 0, st>>>(idx, k, nq);
-    return cudaGetLastError() == cudaSuccess ? JFA_OK : JFA_ERR_CUDA;
+    return launch_pdl(topk_fill_kernel, dim3((k + 255) / 256, n_seg), dim3(256), 0, st, idx, k,
+                      nq) == cudaSuccess
+               ? JFA_OK
+               : JFA_ERR_CUDA;
   }
   TopkBufs b;
   b.scores = reinterpret_cast<const float*>(ws + L.off_scores);
-  b.hist = reinterpret_cast<uint32_t*>(ws + L.off_hist);
+  b.hist = reinterpret_cast<const uint32_t*>(ws + L.off_hist);
   b.counters = reinterpret_cast<uint32_t*>(ws + L.off_counters);
   b.lists = reinterpret_cast<uint2*>(ws + L.off_cand);
   b.counts = reinterpret_cast<uint32_t*>(ws + L.off_sel);
@@ -407,9 +429,16 @@ int launch_topk(const jfa_geom& g, int k, uint8_t* ws, const jfa_workspace_layou
   b.k = k;
   b.n_chunks = (nq + kTopkChunk - 1) / kTopkChunk;
   b.n_chunks_cap = (g.capacity + kTopkChunk - 1) / kTopkChunk;
-  topk_collect_kernel<<<dim3(b.n_chunks, n_seg), 256, 0, st>>>(b);
-  topk_final_kernel<<<n_seg, 256, 0, st>>>(b, idx);
-  return cudaGetLastError() == cudaSuccess ? JFA_OK : JFA_ERR_CUDA;
+  uint32_t* hist = reinterpret_cast<uint32_t*>(ws + L.off_hist);
+  // the histogram and counters start zero: the workspace is zero-filled at
+  // allocation and every final kernel clears its segment when done
+  cudaError_t e = launch_pdl(score_hist_kernel, dim3(b.n_chunks, n_seg), dim3(256), 0, st,
+                             b.scores, g.capacity, nq, hist, b.counters);
+  if (e == cudaSuccess)
+    e = launch_pdl(topk_collect_kernel, dim3(b.n_chunks, n_seg), dim3(256), 0, st, b);
+  if (e == cudaSuccess)
+    e = launch_pdl(topk_final_kernel, dim3(n_seg), dim3(256), 0, st, b, idx, hist);
+  return e == cudaSuccess ? JFA_OK : JFA_ERR_CUDA;
 }
 
 }  // namespace jfa

@@ -125,8 +125,9 @@ const char* jfa_status_string(int status);
 int jfa_cache_layout_get(const jfa_geom* geom, jfa_cache_layout* out);
 
 /* Sizes and offsets of the decode workspace for a geometry and a maximum k
- * (1..JFA_MAX_TOPK).  Pure host function.  The workspace needs no
- * initialisation: each call clears what it accumulates into. */
+ * (1..JFA_MAX_TOPK).  Pure host function.  Zero-fill the workspace once
+ * after allocating it: the top-k counters and histograms it holds start at
+ * zero and every completed jfa_topk call leaves them at zero again. */
 int jfa_workspace_layout_get(const jfa_geom* geom, int32_t max_topk,
                              jfa_workspace_layout* out);
 

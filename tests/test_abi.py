@@ -103,8 +103,8 @@ def test_bad_arguments_rejected_before_launch(lib):
 
 
 def test_launch_accounting(lib):
-    # scan (with the score histogram) + (collect, final) + (correct, merge)
-    assert lib.jfa_decode_step_launches(G(n_ctx=4096), 64) == 5
+    # scan + (histogram, collect, final) + (correct, merge)
+    assert lib.jfa_decode_step_launches(G(n_ctx=4096), 64) == 6
     # k >= N_q: the top-k is a fill kernel
     assert lib.jfa_decode_step_launches(G(n_ctx=100), 64) == 4
     # N_q = 0: no scan
