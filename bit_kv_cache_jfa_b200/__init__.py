@@ -17,7 +17,7 @@ from . import _lib
 from ._lib import (  # noqa: F401  (re-exported C ABI names)
     Cache, CacheLayout, Geom, JfaError, WorkspaceLayout, check, jfa_cache_layout_get,
     jfa_check_error, jfa_clear_error, jfa_correct_merge, jfa_decode_scores, jfa_decode_step,
-    jfa_decode_step_launches, jfa_pack_kv, jfa_score_histogram, jfa_topk, jfa_unpack_record,
+    jfa_decode_step_launches, jfa_pack_kv, jfa_topk, jfa_unpack_record,
     jfa_workspace_layout_get, load)
 
 __all__ = ["KVCache", "Workspace", "decode_step", "JfaError", "load"]

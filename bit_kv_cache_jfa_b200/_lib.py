@@ -69,7 +69,6 @@ SIGNATURES = {
     "jfa_decode_scores": (c_int32, [POINTER(Geom), POINTER(Cache), c_void_p, c_float, c_void_p,
                                     c_void_p]),
     "jfa_topk": (c_int32, [POINTER(Geom), c_int32, c_void_p, c_void_p, c_void_p]),
-    "jfa_score_histogram": (c_int32, [POINTER(Geom), c_void_p, c_void_p]),
     "jfa_correct_merge": (c_int32, [POINTER(Geom), POINTER(Cache), c_void_p, c_float, c_void_p,
                                     c_int32, c_void_p, c_void_p, c_int32, c_void_p, c_void_p,
                                     c_void_p]),
@@ -160,10 +159,6 @@ def jfa_decode_scores(geom, cache, q, scale, ws, stream=None) -> int:
 
 def jfa_topk(geom, k, ws, idx, stream=None) -> int:
     return load().jfa_topk(ctypes.byref(geom), k, _ptr(ws), _ptr(idx), _stream(stream))
-
-
-def jfa_score_histogram(geom, ws, stream=None) -> int:
-    return load().jfa_score_histogram(ctypes.byref(geom), _ptr(ws), _stream(stream))
 
 
 def jfa_correct_merge(geom, cache, q, scale, idx, k, k_exact, v_exact, exact_on_host, ws, out,

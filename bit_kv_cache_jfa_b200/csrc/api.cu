@@ -158,14 +158,6 @@ int jfa_topk(const jfa_geom* geom, int32_t k, void* ws, int32_t* idx, void* stre
                      static_cast<cudaStream_t>(stream));
 }
 
-int jfa_score_histogram(const jfa_geom* geom, void* ws, void* stream) {
-  if (!geom_ok(geom) || !ws || !aligned(ws, 256) || geom->n_ctx < 1) return JFA_ERR_INVALID_ARG;
-  jfa_workspace_layout L;
-  workspace_layout(*geom, 1, &L);
-  return launch_score_histogram(*geom, static_cast<uint8_t*>(ws), L,
-                                static_cast<cudaStream_t>(stream));
-}
-
 int jfa_correct_merge(const jfa_geom* geom, const jfa_cache* cache, const uint16_t* q,
                       float scale, const int32_t* idx, int32_t k, const uint16_t* k_exact,
                       const uint16_t* v_exact, int32_t exact_on_host, void* ws, float* out,

@@ -61,7 +61,5 @@ int launch_correct_merge(const jfa_geom& g, const jfa_cache& c, const uint16_t* 
                          const uint16_t* v_exact, int exact_on_host, uint8_t* ws,
                          const jfa_workspace_layout& L, float* out, cudaStream_t st);
 int count_topk_launches(const jfa_geom& g, int k);
-int launch_score_histogram(const jfa_geom& g, uint8_t* ws, const jfa_workspace_layout& L,
-                           cudaStream_t st);
 
 }  // namespace jfa

@@ -324,9 +324,8 @@ __global__ void __launch_bounds__(256) topk_final_kernel(TopkBufs b, int32_t* id
   clear_segment(hist_clear, b.counters, seg);
 }
 
-// Histogram of the selection-score keys of caller-provided scores, turned
-// into per-segment suffix counts by the last CTA of each segment (the scan
-// kernel builds the same counts on the fly).
+// Histogram of the selection-score keys, turned into per-segment suffix
+// counts (keys with bin >= b) by the last CTA of each segment.
 __global__ void __launch_bounds__(256) score_hist_kernel(const float* scores, int capacity, int nq,
                                                          uint32_t* hist, uint32_t* counters) {
   __shared__ uint32_t sh[kHistBins];
@@ -363,36 +362,23 @@ __global__ void __launch_bounds__(256) score_hist_kernel(const float* scores, in
     s_last = atomicAdd(&counters[(size_t)seg * kCtrStride], 1u) == gridDim.x - 1;
   }
   __syncthreads();
-  if (!s_last || threadIdx.x >= 32) return;
+  if (!s_last) return;
   __threadfence();
-  const int lane = threadIdx.x;
-  uint32_t local = 0;
-  for (int i = 0; i < 64; ++i) local += __ldcg(&gh[64 * lane + i]);
-  uint32_t suf = local;
+  // thread t owns bins [8t, 8t + 8): all loads first, one block suffix scan
+  constexpr int kPer = kHistBins / 256;
+  uint32_t hv[kPer];
 #pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t y = __shfl_down_sync(kFullMask, suf, o);
-    if (lane + o < 32) suf += y;
+  for (int i = 0; i < kPer; ++i) hv[i] = __ldcg(&gh[kPer * threadIdx.x + i]);
+  uint32_t local = 0;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) local += hv[i];
+  __shared__ uint32_t scratch[32];
+  uint32_t run = block_suffix_excl(local, scratch);  // keys in bins above this range
+#pragma unroll
+  for (int i = kPer - 1; i >= 0; --i) {
+    run += hv[i];
+    gh[kPer * threadIdx.x + i] = run;
   }
-  uint32_t run = suf - local;
-  for (int i = 63; i >= 0; --i) {
-    run += __ldcg(&gh[64 * lane + i]);
-    gh[64 * lane + i] = run;
-  }
-}
-
-int launch_score_histogram(const jfa_geom& g, uint8_t* ws, const jfa_workspace_layout& L,
-                           cudaStream_t st) {
-  const int n_seg = g.batch * g.num_kv_heads;
-  const int nq = split_point(g.n_ctx);
-  if (cudaMemsetAsync(ws + L.off_hist, 0, L.off_cand - L.off_hist, st) != cudaSuccess)
-    return JFA_ERR_CUDA;
-  if (nq == 0) return JFA_OK;
-  const int chunks = (nq + kTopkChunk - 1) / kTopkChunk;
-  score_hist_kernel<<<dim3(chunks, n_seg), 256, 0, st>>>(
-      reinterpret_cast<const float*>(ws + L.off_scores), g.capacity, nq,
-      reinterpret_cast<uint32_t*>(ws + L.off_hist), reinterpret_cast<uint32_t*>(ws + L.off_counters));
-  return cudaGetLastError() == cudaSuccess ? JFA_OK : JFA_ERR_CUDA;
 }
 
 __global__ void topk_fill_kernel(int32_t* idx, int k, int nq) {

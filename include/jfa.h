@@ -175,16 +175,10 @@ int jfa_decode_scores(const jfa_geom* geom, const jfa_cache* cache,
  * min(k, N_q) chosen indices are written sorted ascending to
  * idx[B][H_kv][k] (int32 device pointer), the remaining k - k_eff entries
  * set to -1.  1 <= k <= max_topk of the workspace.
- * Reads the selection scores and their key histogram that jfa_decode_scores
- * leaves in the workspace (or that jfa_score_histogram rebuilds). */
+ * Reads the selection scores jfa_decode_scores leaves in the workspace
+ * (off_scores); a caller may also write its own scores there first. */
 int jfa_topk(const jfa_geom* geom, int32_t k, void* ws, int32_t* idx,
              void* stream);
-
-/* jfa_score_histogram — rebuild the selection-score key histogram that
- * jfa_topk reads, from the scores currently in the workspace (off_scores).
- * jfa_decode_scores builds it on the fly; call this only after writing the
- * scores yourself. */
-int jfa_score_histogram(const jfa_geom* geom, void* ws, void* stream);
 
 /* jfa_correct_merge — exact correction and log-sum-exp merge.
  * For every query head: exact logits scale*q.K_t from the bf16 copy for the
