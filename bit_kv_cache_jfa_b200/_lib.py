@@ -69,6 +69,8 @@ SIGNATURES = {
     "jfa_decode_scores": (c_int32, [POINTER(Geom), POINTER(Cache), c_void_p, c_float, c_void_p,
                                     c_void_p]),
     "jfa_topk": (c_int32, [POINTER(Geom), c_int32, c_void_p, c_void_p, c_void_p]),
+    "jfa_topk_noalloc": (c_int32, [c_void_p, c_int32, c_int32, c_int32, c_int32, c_void_p,
+                                   c_void_p]),
     "jfa_correct_merge": (c_int32, [POINTER(Geom), POINTER(Cache), c_void_p, c_float, c_void_p,
                                     c_int32, c_void_p, c_void_p, c_int32, c_void_p, c_void_p,
                                     c_void_p]),
@@ -159,6 +161,13 @@ def jfa_decode_scores(geom, cache, q, scale, ws, stream=None) -> int:
 
 def jfa_topk(geom, k, ws, idx, stream=None) -> int:
     return load().jfa_topk(ctypes.byref(geom), k, _ptr(ws), _ptr(idx), _stream(stream))
+
+
+def jfa_topk_noalloc(scores, n_seg, stride, n_scores, k, idx, stream=None) -> int:
+    """Top-k without any device allocation (scratch is a fixed array in the
+    library); scores is an int device address or a tensor."""
+    return load().jfa_topk_noalloc(_ptr(scores), n_seg, stride, n_scores, k, _ptr(idx),
+                                   _stream(stream))
 
 
 def jfa_correct_merge(geom, cache, q, scale, idx, k, k_exact, v_exact, exact_on_host, ws, out,

@@ -428,3 +428,79 @@ int launch_topk(const jfa_geom& g, int k, uint8_t* ws, const jfa_workspace_layou
 }
 
 }  // namespace jfa
+
+// ---------------------------------------------------------------------------
+// Allocation-free top-k (jfa_topk_noalloc): the same three kernels, with their
+// histogram, counters and lists in a fixed file-scope device array instead of
+// a caller-allocated workspace.
+// ---------------------------------------------------------------------------
+namespace {
+constexpr int kNoAllocMaxSeg = 64;     // segments per call
+constexpr int kNoAllocMaxChunks = 64;  // segments x ceil(scores / 4096) per call
+constexpr size_t kNoAllocHistWords = (size_t)kNoAllocMaxSeg * jfa::kHistBins;
+constexpr size_t kNoAllocCtrWords = (size_t)kNoAllocMaxSeg * jfa::kCtrStride;
+constexpr size_t kNoAllocCountOff = kNoAllocHistWords + kNoAllocCtrWords;
+constexpr size_t kNoAllocListOff = (kNoAllocCountOff + kNoAllocMaxChunks + 63) / 64 * 64;
+constexpr size_t kNoAllocWords = kNoAllocListOff + (size_t)kNoAllocMaxChunks * 4096 * 2;
+}  // namespace
+
+// About 2.5 MB; every device that loads the library holds it until exit.
+static __device__ __align__(256) uint32_t g_topk_scratch[kNoAllocWords];
+
+namespace jfa {
+
+// Device address of g_topk_scratch on the current device (resolved once per
+// device; the host-side name is only a stand-in, never a device address).
+static uint32_t* noalloc_scratch() {
+  static uint32_t* addr[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_topk_scratch) != cudaSuccess || p == nullptr) return nullptr;
+    addr[dev] = static_cast<uint32_t*>(p);
+  }
+  return addr[dev];
+}
+
+}  // namespace jfa
+
+extern "C" int jfa_topk_noalloc(const float* scores, int32_t n_seg, int32_t stride,
+                                int32_t n_scores, int32_t k, int32_t* idx, void* stream) {
+  using namespace jfa;
+  if (!scores || !idx || (reinterpret_cast<uintptr_t>(scores) & 15u) != 0 ||
+      (reinterpret_cast<uintptr_t>(idx) & 3u) != 0)
+    return JFA_ERR_INVALID_ARG;
+  if (n_seg < 1 || n_scores < 1 || n_scores % 4 != 0 || stride < n_scores || stride % 4 != 0 ||
+      k < 1 || k > JFA_MAX_TOPK)
+    return JFA_ERR_INVALID_ARG;
+  const int n_chunks = (n_scores + kTopkChunk - 1) / kTopkChunk;
+  if (n_seg > kNoAllocMaxSeg || (long long)n_seg * n_chunks > kNoAllocMaxChunks)
+    return JFA_ERR_UNSUPPORTED;  // beyond the fixed scratch
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (k >= n_scores) {
+    topk_fill_kernel<<<dim3((k + 255) / 256, n_seg), 256, 0, st>>>(idx, k, n_scores);
+    return cudaGetLastError() == cudaSuccess ? JFA_OK : JFA_ERR_CUDA;
+  }
+  uint32_t* scratch = noalloc_scratch();
+  if (scratch == nullptr) return JFA_ERR_CUDA;
+  // histogram and counters must start at zero; the previous call's contents remain
+  if (cudaMemsetAsync(scratch, 0, kNoAllocCountOff * sizeof(uint32_t), st) != cudaSuccess)
+    return JFA_ERR_CUDA;
+  TopkBufs b;
+  b.scores = scores;
+  b.hist = scratch;
+  b.counters = scratch + kNoAllocHistWords;
+  b.counts = scratch + kNoAllocCountOff;
+  b.lists = reinterpret_cast<uint2*>(scratch + kNoAllocListOff);
+  b.capacity = stride;
+  b.nq = n_scores;
+  b.k = k;
+  b.n_chunks = n_chunks;
+  b.n_chunks_cap = n_chunks;
+  score_hist_kernel<<<dim3(n_chunks, n_seg), 256, 0, st>>>(scores, stride, n_scores, scratch,
+                                                          b.counters);
+  topk_collect_kernel<<<dim3(n_chunks, n_seg), 256, 0, st>>>(b);
+  topk_final_kernel<<<n_seg, 256, 0, st>>>(b, idx, scratch);
+  return cudaGetLastError() == cudaSuccess ? JFA_OK : JFA_ERR_CUDA;
+}

@@ -180,6 +180,29 @@ int jfa_decode_scores(const jfa_geom* geom, const jfa_cache* cache,
 int jfa_topk(const jfa_geom* geom, int32_t k, void* ws, int32_t* idx,
              void* stream);
 
+/* jfa_topk_noalloc — the selection of jfa_topk for callers that cannot
+ * allocate device memory: an inference-engine plugin whose execute callback
+ * must not allocate, code between cudaStreamBeginCapture and EndCapture
+ * (where cudaMalloc is not a stream operation and cannot be recorded), or a
+ * latency-bound loop where an allocation would stall the device.  The pages
+ * have no counterpart; it is a deployment convenience.
+ *   scores   : fp32 [n_seg][stride] device pointer, 16-B aligned; the first
+ *              n_scores entries of each row are scored (n_scores % 4 == 0,
+ *              stride % 4 == 0, stride >= n_scores).
+ *   idx      : int32 [n_seg][k] output, as jfa_topk writes it.
+ * Scratch lives in one fixed ~2.5 MB device array inside the library (held by
+ * every device that loads it until exit): n_seg <= 64 and
+ * n_seg * ceil(n_scores / 4096) <= 64 (e.g. 8 rows of 32768 scores, 2 of
+ * 131072); larger requests return JFA_ERR_UNSUPPORTED before any work.
+ * The call allocates nothing.  Its first call on a device looks up the
+ * array's device address (cudaGetSymbolAddress); make that first call
+ * before any stream capture.  Every call clears the parts of the array that
+ * must start at zero and otherwise reuses the previous call's contents, so
+ * calls that overlap on the GPU (other streams, other threads) race: keep
+ * them on one stream. */
+int jfa_topk_noalloc(const float* scores, int32_t n_seg, int32_t stride,
+                     int32_t n_scores, int32_t k, int32_t* idx, void* stream);
+
 /* jfa_correct_merge — exact correction and log-sum-exp merge.
  * For every query head: exact logits scale*q.K_t from the bf16 copy for the
  * top-k tokens and the tail, aggregated with bf16 values in fp32 (Jet-QSparse
