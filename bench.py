@@ -1,8 +1,8 @@
 #!/usr/bin/env python
 """Throughput of the approximate-then-correct low-bit KV decode-attention step.
 
-One step = jfa_decode_scores + jfa_topk + jfa_correct_merge over every
-sequence and head of one decode layer (the Llama-3.1-8B-shaped K3V2 layer by
+One step = jfa_decode_scores + jfa_decode_finish (top-k, correction and merge
+in one cluster kernel) over every sequence and head of one decode layer (the Llama-3.1-8B-shaped K3V2 layer by
 default: batch 4, 32 query / 8 KV heads, 32768 cached tokens, top-k 256).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
@@ -310,9 +310,8 @@ def run_jfa(args, w):
 
     def step():
         _lib.check(_lib.jfa_decode_scores(geom, cst, q, scale, ws.buf, sp), "scores")
-        _lib.check(_lib.jfa_topk(geom, w.topk, ws.buf, idx, sp), "topk")
-        _lib.check(_lib.jfa_correct_merge(geom, cst, q, scale, idx, w.topk, k_exact, v_exact,
-                                          host, ws.buf, out, sp), "correct_merge")
+        _lib.check(_lib.jfa_decode_finish(geom, cst, q, scale, w.topk, idx, k_exact, v_exact,
+                                          host, ws.buf, out, sp), "finish")
 
     for _ in range(max(3, args.warmup)):
         flush.zero_()
@@ -332,9 +331,8 @@ def run_jfa(args, w):
         ev[i][0].record(stream)
         _lib.check(_lib.jfa_decode_scores(geom, cst, q, scale, ws.buf, sp), "scores")
         ev[i][1].record(stream)
-        _lib.check(_lib.jfa_topk(geom, w.topk, ws.buf, idx, sp), "topk")
-        _lib.check(_lib.jfa_correct_merge(geom, cst, q, scale, idx, w.topk, k_exact, v_exact,
-                                          host, ws.buf, out, sp), "correct_merge")
+        _lib.check(_lib.jfa_decode_finish(geom, cst, q, scale, w.topk, idx, k_exact, v_exact,
+                                          host, ws.buf, out, sp), "finish")
         ev[i][2].record(stream)
     torch.cuda.synchronize()
     barrier(world)

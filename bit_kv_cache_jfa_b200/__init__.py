@@ -16,7 +16,8 @@ import math
 from . import _lib
 from ._lib import (  # noqa: F401  (re-exported C ABI names)
     Cache, CacheLayout, Geom, JfaError, WorkspaceLayout, check, jfa_cache_layout_get,
-    jfa_check_error, jfa_clear_error, jfa_correct_merge, jfa_decode_scores, jfa_decode_step,
+    jfa_check_error, jfa_clear_error, jfa_correct_merge, jfa_decode_finish, jfa_decode_scores,
+    jfa_decode_step,
     jfa_decode_step_launches, jfa_pack_kv, jfa_topk, jfa_unpack_record,
     jfa_workspace_layout_get, load)
 

@@ -77,6 +77,9 @@ SIGNATURES = {
     "jfa_decode_step": (c_int32, [POINTER(Geom), POINTER(Cache), c_void_p, c_float, c_int32,
                                   c_void_p, c_void_p, c_void_p, c_int32, c_void_p, c_void_p,
                                   c_void_p]),
+    "jfa_decode_finish": (c_int32, [POINTER(Geom), POINTER(Cache), c_void_p, c_float, c_int32,
+                                    c_void_p, c_void_p, c_void_p, c_int32, c_void_p, c_void_p,
+                                    c_void_p]),
     "jfa_clear_error": (c_int32, [POINTER(Geom), c_void_p, c_void_p]),
     "jfa_check_error": (c_int32, [POINTER(Geom), c_void_p, c_void_p, POINTER(c_uint32)]),
     "jfa_unpack_record": (c_int32, [c_int32, c_int32, c_void_p, POINTER(c_uint8),
@@ -182,6 +185,13 @@ def jfa_decode_step(geom, cache, q, scale, k, idx, k_exact, v_exact, exact_on_ho
     return load().jfa_decode_step(ctypes.byref(geom), ctypes.byref(cache), _ptr(q), scale, k,
                                   _ptr(idx), _ptr(k_exact), _ptr(v_exact), int(exact_on_host),
                                   _ptr(ws), _ptr(out), _stream(stream))
+
+
+def jfa_decode_finish(geom, cache, q, scale, k, idx, k_exact, v_exact, exact_on_host, ws, out,
+                      stream=None) -> int:
+    return load().jfa_decode_finish(ctypes.byref(geom), ctypes.byref(cache), _ptr(q), scale, k,
+                                    _ptr(idx), _ptr(k_exact), _ptr(v_exact), int(exact_on_host),
+                                    _ptr(ws), _ptr(out), _stream(stream))
 
 
 def jfa_clear_error(geom, ws, stream=None) -> int:

@@ -42,8 +42,10 @@ int workspace_layout(const jfa_geom& g, int max_topk, jfa_workspace_layout* out)
   L.off_counters = off;
   off = align_up(off + n_seg * 8 * sizeof(uint32_t), 256);
   // top-k lists: per 4096-score chunk, up to 4096 (key, index) pairs; then counts
+  // (also holds the per-CTA lists of the fused finishing kernel: <= capacity + 512)
   const size_t n_chunks_cap = ((size_t)g.capacity + 4095) / 4096;
-  L.cand_cap = (int32_t)(n_chunks_cap * 4096);
+  const size_t cap_fused = (size_t)g.capacity + 512;
+  L.cand_cap = (int32_t)(n_chunks_cap * 4096 > cap_fused ? n_chunks_cap * 4096 : cap_fused);
   L.off_cand = off;
   off = align_up(off + n_seg * (size_t)L.cand_cap * 2 * sizeof(uint32_t), 256);
   L.max_topk = max_topk;
@@ -184,18 +186,32 @@ int jfa_decode_step(const jfa_geom* geom, const jfa_cache* cache, const uint16_t
     return JFA_ERR_INVALID_ARG;
   if (!k_exact || !v_exact || !aligned(k_exact, 16) || !aligned(v_exact, 16))
     return JFA_ERR_INVALID_ARG;
-  int s = jfa_decode_scores(geom, cache, q, scale, ws, stream);
+  const int s = jfa_decode_scores(geom, cache, q, scale, ws, stream);
   if (s != JFA_OK) return s;
-  s = jfa_topk(geom, k, ws, idx, stream);
-  if (s != JFA_OK) return s;
-  return jfa_correct_merge(geom, cache, q, scale, idx, k, k_exact, v_exact, exact_on_host, ws,
+  return jfa_decode_finish(geom, cache, q, scale, k, idx, k_exact, v_exact, exact_on_host, ws,
                            out, stream);
+}
+
+int jfa_decode_finish(const jfa_geom* geom, const jfa_cache* cache, const uint16_t* q, float scale,
+                      int32_t k, int32_t* idx, const uint16_t* k_exact, const uint16_t* v_exact,
+                      int32_t exact_on_host, void* ws, float* out, void* stream) {
+  if (!geom_ok(geom) || !cache_ok(cache) || !ws || !aligned(ws, 256)) return JFA_ERR_INVALID_ARG;
+  if (geom->n_ctx < 1 || !q || !aligned(q, 16) || !(scale > 0.f)) return JFA_ERR_INVALID_ARG;
+  if (k < 1 || k > JFA_MAX_TOPK || !idx || !aligned(idx, 4) || !out || !aligned(out, 16))
+    return JFA_ERR_INVALID_ARG;
+  if (!k_exact || !v_exact || !aligned(k_exact, 16) || !aligned(v_exact, 16))
+    return JFA_ERR_INVALID_ARG;
+  (void)exact_on_host;  // same loads either way; the rows are device-addressable
+  jfa_workspace_layout L;
+  workspace_layout(*geom, k, &L);
+  return launch_finish(*geom, *cache, q, scale, k, idx, k_exact, v_exact,
+                       static_cast<uint8_t*>(ws), L, out, static_cast<cudaStream_t>(stream));
 }
 
 int jfa_decode_step_launches(const jfa_geom* geom, int32_t k) {
   if (!geom_ok(geom) || geom->n_ctx < 1 || k < 1 || k > JFA_MAX_TOPK) return 0;
   const int scan = split_point(geom->n_ctx) > 0 ? 1 : 0;
-  return scan + count_topk_launches(*geom, k) + 2;
+  return scan + 1;  // scan + fused finishing kernel
 }
 
 int jfa_clear_error(const jfa_geom* geom, void* ws, void* stream) {

@@ -61,5 +61,8 @@ int launch_correct_merge(const jfa_geom& g, const jfa_cache& c, const uint16_t* 
                          const uint16_t* v_exact, int exact_on_host, uint8_t* ws,
                          const jfa_workspace_layout& L, float* out, cudaStream_t st);
 int count_topk_launches(const jfa_geom& g, int k);
+int launch_finish(const jfa_geom& g, const jfa_cache& c, const uint16_t* q, float scale, int k,
+                  int32_t* idx, const uint16_t* k_exact, const uint16_t* v_exact, uint8_t* ws,
+                  const jfa_workspace_layout& L, float* out, cudaStream_t st);
 
 }  // namespace jfa

@@ -225,12 +225,23 @@ int jfa_correct_merge(const jfa_geom* geom, const jfa_cache* cache,
                       const uint16_t* v_exact, int32_t exact_on_host,
                       void* ws, float* out, void* stream);
 
-/* The whole decode step (scores, top-k, correct+merge) in one call;
- * equivalent to the three calls in order.  idx is written as by jfa_topk. */
+/* The whole decode step (scores, top-k, correct+merge) in one call, with the
+ * same results as the three calls in order (idx identical, out to rounding):
+ * the scan, then one kernel in which a thread-block cluster per (sequence,
+ * KV head) selects, corrects and merges.  idx is written as by jfa_topk. */
 int jfa_decode_step(const jfa_geom* geom, const jfa_cache* cache,
                     const uint16_t* q, float scale, int32_t k, int32_t* idx,
                     const uint16_t* k_exact, const uint16_t* v_exact,
                     int32_t exact_on_host, void* ws, float* out, void* stream);
+
+/* jfa_decode_finish — the rest of the step after jfa_decode_scores: top-k
+ * selection, exact correction and merge in one kernel (a thread-block
+ * cluster per (sequence, KV head)); results as jfa_topk followed by
+ * jfa_correct_merge.  Arguments as jfa_decode_step. */
+int jfa_decode_finish(const jfa_geom* geom, const jfa_cache* cache,
+                      const uint16_t* q, float scale, int32_t k, int32_t* idx,
+                      const uint16_t* k_exact, const uint16_t* v_exact,
+                      int32_t exact_on_host, void* ws, float* out, void* stream);
 
 /* Clear the workspace error flag (stream-ordered). */
 int jfa_clear_error(const jfa_geom* geom, void* ws, void* stream);

@@ -86,6 +86,18 @@ class GpuRun:
         assert flag == 0, f"device error flag {flag:#x}"
         return self.out.cpu().double().numpy(), self.idx.cpu().numpy()
 
+    def fused_step(self):
+        """jfa_decode_step (scan + fused finishing kernel) into fresh outputs."""
+        out = torch.empty_like(self.out)
+        idx = torch.empty_like(self.idx)
+        _lib.check(_lib.jfa_decode_step(self.cache.geom(), self.cache.struct(), self.q, self.scale,
+                                        self.k, idx, self.k_exact, self.v_exact,
+                                        self.exact_on_host, self.ws.buf, out), "decode_step")
+        torch.cuda.synchronize()
+        st, flag = _lib.jfa_check_error(self.cache.geom(), self.ws.buf)
+        assert flag == 0, f"device error flag {flag:#x}"
+        return out.cpu().double().numpy(), idx.cpu().numpy()
+
     def selection_scores(self):
         torch.cuda.synchronize()
         nq = self.cache.n_quant

@@ -103,12 +103,11 @@ def test_bad_arguments_rejected_before_launch(lib):
 
 
 def test_launch_accounting(lib):
-    # scan + (histogram, collect, final) + (correct, merge)
-    assert lib.jfa_decode_step_launches(G(n_ctx=4096), 64) == 6
-    # k >= N_q: the top-k is a fill kernel
-    assert lib.jfa_decode_step_launches(G(n_ctx=100), 64) == 4
+    # scan + the fused finishing kernel
+    assert lib.jfa_decode_step_launches(G(n_ctx=4096), 64) == 2
+    assert lib.jfa_decode_step_launches(G(n_ctx=100), 64) == 2
     # N_q = 0: no scan
-    assert lib.jfa_decode_step_launches(G(n_ctx=64), 8) == 3
+    assert lib.jfa_decode_step_launches(G(n_ctx=64), 8) == 1
 
 
 def test_status_strings(lib):

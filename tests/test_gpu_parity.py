@@ -254,3 +254,28 @@ def test_capacity_larger_than_context():
     ref = run.oracle_step()
     assert_topk_valid(idx, ref.select, 100)
     assert_out_close(out, run.oracle_step(idx=idx).out)
+
+
+# ---------------------------------------------------------------- fused step
+@pytest.mark.parametrize("kb,vb,heads,kv,ctx,k,batch", [
+    (4, 4, 8, 2, 4096, 64, 1), (3, 2, 32, 8, 5000, 256, 2), (4, 4, 32, 4, 9000, 512, 1),
+    (3, 2, 8, 8, 2100, 33, 3), (4, 2, 64, 8, 3333, 256, 2), (3, 4, 4, 1, 700, 700, 2),
+    (3, 2, 32, 8, 100, 16, 2), (4, 4, 8, 2, 64, 8, 1), (3, 2, 32, 8, 40000, 4096, 1)])
+def test_fused_step_matches_separate_calls(kb, vb, heads, kv, ctx, k, batch):
+    w = small(kb, vb, heads=heads, kv=kv, ctx=ctx, batch=batch, topk=k, lognormal=True)
+    run = GpuRun(w)
+    out3, idx3 = run.step()
+    out1, idx1 = run.fused_step()
+    assert np.array_equal(idx1, idx3)
+    assert np.allclose(out1, out3, rtol=1e-5, atol=1e-6)
+    if ctx <= 9000:
+        assert_out_close(out1, run.oracle_step(idx=idx1).out)
+
+
+def test_fused_step_tiny_workload_against_oracle():
+    w = W.WORKLOADS["tiny_k4v4_4k"]
+    run = GpuRun(w)
+    out, idx = run.fused_step()
+    ref = run.oracle_step()
+    assert_topk_valid(idx, ref.select, w.topk)
+    assert_out_close(out, ref.out)
