@@ -109,7 +109,7 @@ __device__ void select_ordered(Get get, uint32_t total, uint32_t bstar, uint32_t
 }
 
 template <int G>
-__global__ void __launch_bounds__(kFinThreads) finish_kernel(const FinishParams fp) {
+__global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishParams fp) {
   extern __shared__ __align__(16) uint8_t fsm[];
   const MergeParams& p = fp.m;
   cg::cluster_group cl = cg::this_cluster();
@@ -164,20 +164,34 @@ __global__ void __launch_bounds__(kFinThreads) finish_kernel(const FinishParams 
   }
   cl.sync();
 
-  // ---- P1b: CTA 0 sums the histograms and finds b*
+  // ---- P1b: CTA 0 sums the histograms (all remote loads issued first) and finds b*
   if (select && r == 0) {
-    constexpr int kPer = kHistBins / kFinThreads;
-    uint32_t tot[kPer];
+    uint4 hv[kFinMaxC][2];
 #pragma unroll
-    for (int i = 0; i < kPer; ++i) tot[i] = 0u;
-    for (int q = 0; q < C; ++q) {
-      const uint32_t* ph = cl.map_shared_rank(hist, q);
+    for (int q = 0; q < kFinMaxC; ++q) {
+      if (q < C) {
+        const uint4* ph = reinterpret_cast<const uint4*>(cl.map_shared_rank(hist, q)) + 2 * tid;
+        hv[q][0] = ph[0];
+        hv[q][1] = ph[1];
+      }
+    }
+    uint32_t tot[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
 #pragma unroll
-      for (int i = 0; i < kPer; ++i) tot[i] += ph[kPer * tid + i];
+    for (int q = 0; q < kFinMaxC; ++q) {
+      if (q < C) {
+        tot[0] += hv[q][0].x;
+        tot[1] += hv[q][0].y;
+        tot[2] += hv[q][0].z;
+        tot[3] += hv[q][0].w;
+        tot[4] += hv[q][1].x;
+        tot[5] += hv[q][1].y;
+        tot[6] += hv[q][1].z;
+        tot[7] += hv[q][1].w;
+      }
     }
     __syncthreads();
-#pragma unroll
-    for (int i = 0; i < kPer; ++i) hist[kPer * tid + i] = tot[i];
+    reinterpret_cast<uint4*>(hist)[2 * tid] = make_uint4(tot[0], tot[1], tot[2], tot[3]);
+    reinterpret_cast<uint4*>(hist)[2 * tid + 1] = make_uint4(tot[4], tot[5], tot[6], tot[7]);
     if (tid == 0) {
       s_bin = 0;
       s_above = 0;
@@ -321,51 +335,118 @@ __global__ void __launch_bounds__(kFinThreads) finish_kernel(const FinishParams 
   }
   cl.sync();
 
-  // ---- P5: merge per query head (CTA r owns heads j = r, r + C, ...)
+  // ---- P5a: each CTA merges its share of the scan slots for every head into
+  // sp[G][kPartStride] (one tiled pass with all loads of a tile in flight)
+  float* sp = bat;  // the batch buffer is free now: [G][kPartStride] (first half)
+  {
+    long long w0 = 0, w1 = -1;
+    if (p.ng > 0) {
+      const long long T = p.scan_total, W = p.scan_warps;
+      const long long x0 = (long long)seg * p.ng, x1 = x0 + p.ng - 1;
+      w0 = scan_warp_of(x0, W, T);
+      w1 = scan_warp_of(x1, W, T);
+    }
+    const int ns = (int)(w1 - w0 + 1);
+    const int s0 = (int)((long long)ns * r / C), s1 = (int)((long long)ns * (r + 1) / C);
+    float* tile = reinterpret_cast<float*>(U);
+    constexpr int kTile = (int)(((size_t)correct_smem_floats<G>()) / kPartStride);  // rows per tile
+    const int c = tid & (kD - 1);
+    float mrun[G], lrun[G], arun[G];
+#pragma unroll
+    for (int j = 0; j < G; ++j) {
+      mrun[j] = -INFINITY;
+      lrun[j] = 0.f;
+      arun[j] = 0.f;
+    }
+    for (int t0 = s0 * G; t0 < s1 * G; t0 += kTile) {
+      const int nr = min(kTile, s1 * G - t0);
+      __syncthreads();
+      for (int i = tid; i < nr * (kPartStride / 4); i += kFinThreads) {
+        const int row = i / (kPartStride / 4), v = i % (kPartStride / 4);
+        const int gr = t0 + row;  // row = slot * G + head
+        reinterpret_cast<float4*>(tile + row * kPartStride)[v] = reinterpret_cast<const float4*>(
+            p.scan_part + ((size_t)(w0 + gr / G + seg) * G + gr % G) * kPartStride)[v];
+      }
+      __syncthreads();
+      if (tid < kD) {
+#pragma unroll
+        for (int j = 0; j < G; ++j) {
+          float tm = mrun[j];
+          for (int row = (j - t0 % G + G) % G; row < nr; row += G)
+            if (tile[row * kPartStride + 1] > 0.f) tm = fmaxf(tm, tile[row * kPartStride]);
+          const float sc0 = (lrun[j] > 0.f) ? exp2f(mrun[j] - tm) : 0.f;
+          float l = lrun[j] * sc0, a = arun[j] * sc0;
+          for (int row = (j - t0 % G + G) % G; row < nr; row += G) {
+            const float lb = tile[row * kPartStride + 1];
+            if (lb > 0.f) {
+              const float sc = exp2f(tile[row * kPartStride] - tm);
+              l = fmaf(lb, sc, l);
+              a = fmaf(tile[row * kPartStride + 4 + c], sc, a);
+            }
+          }
+          mrun[j] = tm;
+          lrun[j] = l;
+          arun[j] = a;
+        }
+      }
+    }
+    if (tid < kD) {
+#pragma unroll
+      for (int j = 0; j < G; ++j) {
+        sp[j * kPartStride + 4 + c] = arun[j];
+        if (c == 0) {
+          sp[j * kPartStride] = lrun[j] > 0.f ? mrun[j] : -INFINITY;
+          sp[j * kPartStride + 1] = lrun[j];
+        }
+      }
+    }
+  }
+  cl.sync();
+
+  // ---- P5b: CTA r owns heads j = r, r + C, ...: merge the C scan, exact and
+  // removal partials (remote loads issued together) and write the output row
   for (int j = r; j < G; j += C) {
     const int c = tid;
     if (c < kD) {
-      long long w0 = 0, w1 = -1;
-      if (p.ng > 0) {
-        const long long T = p.scan_total, W = p.scan_warps;
-        const long long x0 = (long long)seg * p.ng, x1 = x0 + p.ng - 1;
-        w0 = scan_warp_of(x0, W, T);
-        w1 = scan_warp_of(x1, W, T);
+      float2 hd[kFinMaxC][3];  // (m, l) of scan / exact / removal parts
+      float av[kFinMaxC][3];   // channel c of each
+#pragma unroll
+      for (int q = 0; q < kFinMaxC; ++q) {
+        if (q < C) {
+          const float* spq = cl.map_shared_rank(sp, q) + j * kPartStride;
+          const float* rq = cl.map_shared_rank(run, q);
+          const float* re = rq + (0 * G + j) * kPartStride;
+          const float* rm = rq + (1 * G + j) * kPartStride;
+          hd[q][0] = *reinterpret_cast<const float2*>(spq);
+          hd[q][1] = *reinterpret_cast<const float2*>(re);
+          hd[q][2] = *reinterpret_cast<const float2*>(rm);
+          av[q][0] = spq[4 + c];
+          av[q][1] = re[4 + c];
+          av[q][2] = rm[4 + c];
+        }
       }
-      const int ns = (int)(w1 - w0 + 1);
-      auto srow = [&](int i) { return p.scan_part + ((size_t)(w0 + i + seg) * G + j) * kPartStride; };
-      float ma = -INFINITY, me = -INFINITY, mr = -INFINITY;
-      for (int i = 0; i < ns; ++i) {
-        const float2 ml = *reinterpret_cast<const float2*>(srow(i));
-        if (ml.y > 0.f) ma = fmaxf(ma, ml.x);
-      }
-      for (int q = 0; q < C; ++q) {
-        const float* rq = cl.map_shared_rank(run, q);
-        const float* re = rq + (0 * G + j) * kPartStride;
-        const float* rm = rq + (1 * G + j) * kPartStride;
-        if (re[1] > 0.f) me = fmaxf(me, re[0]);
-        if (rm[1] > 0.f) mr = fmaxf(mr, rm[0]);
-      }
-      float la = 0.f, aa = 0.f, le = 0.f, ae = 0.f, lr = 0.f, ar = 0.f;
-#pragma unroll 4
-      for (int i = 0; i < ns; ++i) {
-        const float* row = srow(i);
-        const float2 ml = *reinterpret_cast<const float2*>(row);
-        const float sc = ml.y > 0.f ? exp2f(ml.x - ma) : 0.f;
-        la = fmaf(ml.y, sc, la);
-        aa = fmaf(row[4 + c], sc, aa);
-      }
-      for (int q = 0; q < C; ++q) {
-        const float* rq = cl.map_shared_rank(run, q);
-        const float* re = rq + (0 * G + j) * kPartStride;
-        const float* rm = rq + (1 * G + j) * kPartStride;
-        const float se = re[1] > 0.f ? exp2f(re[0] - me) : 0.f;
-        const float sr = rm[1] > 0.f ? exp2f(rm[0] - mr) : 0.f;
-        le = fmaf(re[1], se, le);
-        ae = fmaf(re[4 + c], se, ae);
-        lr = fmaf(rm[1], sr, lr);
-        ar = fmaf(rm[4 + c], sr, ar);
-      }
+      float mk[3] = {-INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int q = 0; q < kFinMaxC; ++q)
+        if (q < C) {
+#pragma unroll
+          for (int t = 0; t < 3; ++t)
+            if (hd[q][t].y > 0.f) mk[t] = fmaxf(mk[t], hd[q][t].x);
+        }
+      float lk[3] = {0.f, 0.f, 0.f}, ak[3] = {0.f, 0.f, 0.f};
+#pragma unroll
+      for (int q = 0; q < kFinMaxC; ++q)
+        if (q < C) {
+#pragma unroll
+          for (int t = 0; t < 3; ++t) {
+            const float sc = hd[q][t].y > 0.f ? exp2f(hd[q][t].x - mk[t]) : 0.f;
+            lk[t] = fmaf(hd[q][t].y, sc, lk[t]);
+            ak[t] = fmaf(av[q][t], sc, ak[t]);
+          }
+        }
+      const float ma = mk[0], la = lk[0], aa = ak[0];
+      const float me = mk[1], le = lk[1], ae = ak[1];
+      const float mr = mk[2], lr = lk[2], ar = ak[2];
       // remainder = approximate total minus the removed top-k terms (m_a frame)
       float lrest = la, arest = aa;
       if (la > 0.f && lr > 0.f) {
@@ -388,16 +469,41 @@ __global__ void __launch_bounds__(kFinThreads) finish_kernel(const FinishParams 
   cl.sync();
 }
 
+// Largest cluster size (<= 8) whose clusters all fit on the device at once
+// (so the whole grid runs in one wave), using up to about two CTAs per SM.
+template <int G>
 static int pick_cluster(int n_seg, int num_sms) {
-  int c = 1;
-  while (c < kFinMaxC && n_seg * c * 2 <= 2 * num_sms) c *= 2;
-  return c;
+  constexpr size_t smem = finish_smem_bytes<G>();
+  int best = 1;
+  for (int c = 2; c <= kFinMaxC; c *= 2) {
+    if ((long long)n_seg * c > 2LL * num_sms) break;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(n_seg * c);
+    cfg.blockDim = dim3(kFinThreads);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = c;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    int n_active = 0;
+    if (cudaOccupancyMaxActiveClusters(&n_active, finish_kernel<G>, &cfg) != cudaSuccess) {
+      cudaGetLastError();
+      break;
+    }
+    if (n_active >= n_seg) best = c;
+    else break;
+  }
+  return best;
 }
 
 template <int G>
-static int launch_finish_t(const FinishParams& fp, int n_seg, int C, cudaStream_t st) {
+static int launch_finish_t(FinishParams fp, int n_seg, cudaStream_t st) {
   constexpr size_t smem = finish_smem_bytes<G>();
   static bool configured[64] = {false};
+  static int memo_seg[64][8] = {{0}}, memo_c[64][8] = {{0}};  // cluster size per (device, n_seg)
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !configured[dev]) {
@@ -406,6 +512,24 @@ static int launch_finish_t(const FinishParams& fp, int n_seg, int C, cudaStream_
       return JFA_ERR_CUDA;
     configured[dev] = true;
   }
+  int C = 0;
+  if (dev >= 0 && dev < 64) {
+    for (int i = 0; i < 8; ++i)
+      if (memo_seg[dev][i] == n_seg) C = memo_c[dev][i];
+  }
+  if (C == 0) {
+    C = pick_cluster<G>(n_seg, num_sms_current());
+    if (dev >= 0 && dev < 64) {
+      for (int i = 0; i < 8; ++i)
+        if (memo_seg[dev][i] == 0) {
+          memo_seg[dev][i] = n_seg;
+          memo_c[dev][i] = C;
+          break;
+        }
+    }
+  }
+  const int nq = fp.m.nq;
+  fp.slice = nq > 0 ? ((nq + C - 1) / C + 63) / 64 * 64 : 64;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(n_seg * C);
   cfg.blockDim = dim3(kFinThreads);
@@ -461,17 +585,15 @@ int launch_finish(const jfa_geom& g, const jfa_cache& c, const uint16_t* q, floa
   fp.scores = reinterpret_cast<const float*>(ws + L.off_scores);
   fp.idx_out = idx;
   fp.lists = reinterpret_cast<uint2*>(ws + L.off_cand);
-  const int C = pick_cluster(n_seg, num_sms_current());
-  fp.slice = nq > 0 ? ((nq + C - 1) / C + 63) / 64 * 64 : 64;
   switch (p.G) {
-    case 1: return launch_finish_t<1>(fp, n_seg, C, st);
-    case 2: return launch_finish_t<2>(fp, n_seg, C, st);
-    case 3: return launch_finish_t<3>(fp, n_seg, C, st);
-    case 4: return launch_finish_t<4>(fp, n_seg, C, st);
-    case 5: return launch_finish_t<5>(fp, n_seg, C, st);
-    case 6: return launch_finish_t<6>(fp, n_seg, C, st);
-    case 7: return launch_finish_t<7>(fp, n_seg, C, st);
-    default: return launch_finish_t<8>(fp, n_seg, C, st);
+    case 1: return launch_finish_t<1>(fp, n_seg, st);
+    case 2: return launch_finish_t<2>(fp, n_seg, st);
+    case 3: return launch_finish_t<3>(fp, n_seg, st);
+    case 4: return launch_finish_t<4>(fp, n_seg, st);
+    case 5: return launch_finish_t<5>(fp, n_seg, st);
+    case 6: return launch_finish_t<6>(fp, n_seg, st);
+    case 7: return launch_finish_t<7>(fp, n_seg, st);
+    default: return launch_finish_t<8>(fp, n_seg, st);
   }
 }
 
