@@ -108,6 +108,41 @@ __device__ void select_ordered(Get get, uint32_t total, uint32_t bstar, uint32_t
   }
 }
 
+// L2 prefetch of what the correction of token t reads (t: token index, or
+// (1 << 30) | tail slot): bf16 K/V rows and, for quantized tokens, the key
+// scales/zeros, key codes and value scales/codes of its record.  part picks
+// one of kPrefParts 128-byte pieces, so consecutive threads split the work.
+constexpr int kPrefParts = 12;
+__device__ __forceinline__ void prefetch_token(const MergeParams& p, int seg, int t, int part) {
+  if (t < 0) return;
+  if (t & (1 << 30)) {
+    const int tt = t & ~(1 << 30);
+    if (part < 4) {
+      const uint16_t* row = ((part & 2) ? p.tail_v : p.tail_k) + ((size_t)seg * kTail + tt) * kD;
+      prefetch_l2(row + 64 * (part & 1));
+    }
+    return;
+  }
+  const uint8_t* rec = p.groups + ((size_t)seg * p.ng_cap + t / kKG) * p.rec_bytes;
+  const int tt = t % kKG;
+  if (part < 4) {
+    const uint16_t* row = ((part & 2) ? p.v_exact : p.k_exact) + ((size_t)seg * p.capacity + t) * kD;
+    prefetch_l2(row + 64 * (part & 1));
+  } else if (part < 8) {
+    prefetch_l2(rec + off_ks() + 128 * (part - 4));  // key scales/zeros (512 B)
+  } else if (part == 8) {
+    const int nt = tt >> 3, gd = tt & 7;
+    prefetch_l2(rec + off_kc() +
+                (p.key_bits == 4 ? nt * 512 + gd * 64 : (nt >> 2) * 1536 + gd * 192));
+  } else if (part == 9) {
+    prefetch_l2(rec + off_vs(p.key_bits) + (tt >> 4) * 128);
+  } else {
+    const int kk = tt >> 4;
+    const int chunk = p.val_bits == 4 ? 2 * kk + (part - 10) : kk;
+    prefetch_l2(rec + off_vc(p.key_bits) + chunk * 512 + 256 * (p.val_bits == 4 ? 0 : (part - 10)));
+  }
+}
+
 template <int G>
 __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishParams fp) {
   extern __shared__ __align__(16) uint8_t fsm[];
@@ -139,6 +174,30 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
   const int lo = r * fp.slice, hi = min(nq, lo + fp.slice);
   const float* S = fp.scores + (size_t)seg * p.capacity;
   uint2* lists = fp.lists + (size_t)seg * C * fp.slice;
+  // exact-set share of this CTA (P4) and scan slots it merges (P5a)
+  const int nE = keff + p.tail;
+  const int e_per = (nE + C - 1) / C;
+  const int e0 = r * e_per, e1 = min(nE, e0 + e_per);
+  long long w0 = 0, w1 = -1;
+  if (p.ng > 0) {
+    const long long T = p.scan_total, W = p.scan_warps;
+    const long long x0 = (long long)seg * p.ng, x1 = x0 + p.ng - 1;
+    w0 = scan_warp_of(x0, W, T);
+    w1 = scan_warp_of(x1, W, T);
+  }
+  const int ns = (int)(w1 - w0 + 1);
+  const int s0 = (int)((long long)ns * r / C), s1 = (int)((long long)ns * (r + 1) / C);
+  // known from the start: the tail tokens among this CTA's share, and its
+  // scan-slot rows -- start pulling them into L2 now
+  for (int i = tid; i < (e1 - e0) * kPrefParts; i += kFinThreads) {
+    const int e = e0 + i / kPrefParts;
+    if (e >= keff) prefetch_token(p, seg, (1 << 30) | (e - keff), i % kPrefParts);
+  }
+  for (int i = tid; i < (s1 - s0) * G * 5; i += kFinThreads) {
+    const int row = s0 * G + i / 5;
+    prefetch_l2(p.scan_part + ((size_t)(w0 + row / G + seg) * G + row % G) * kPartStride +
+                32 * (i % 5));
+  }
 
   // ---- P1: histogram of this CTA's slice
   if (select) {
@@ -288,10 +347,11 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
 
   // ---- P4: correction of this CTA's share of the exact set
   {
-    const int nE = keff + p.tail;
-    const int per = (nE + C - 1) / C;
-    const int e0 = r * per, e1 = min(nE, e0 + per);
     const int32_t* chosen0 = cl.map_shared_rank(chosen, 0);
+    // every chosen token of the share is known now: pull its rows and record
+    // pieces into L2 before the batches read them
+    for (int i = tid; i < (min(e1, keff) - e0) * kPrefParts; i += kFinThreads)
+      prefetch_token(p, seg, chosen0[e0 + i / kPrefParts], i % kPrefParts);
     const CorrectSmem CS = correct_smem_carve(reinterpret_cast<float*>(U), G);
     correct_load_q<G>(p, seg, CS.qs);
     for (int i = tid; i < 2 * G * kPartStride; i += kFinThreads) run[i] = 0.f;
@@ -339,15 +399,6 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
   // sp[G][kPartStride] (one tiled pass with all loads of a tile in flight)
   float* sp = bat;  // the batch buffer is free now: [G][kPartStride] (first half)
   {
-    long long w0 = 0, w1 = -1;
-    if (p.ng > 0) {
-      const long long T = p.scan_total, W = p.scan_warps;
-      const long long x0 = (long long)seg * p.ng, x1 = x0 + p.ng - 1;
-      w0 = scan_warp_of(x0, W, T);
-      w1 = scan_warp_of(x1, W, T);
-    }
-    const int ns = (int)(w1 - w0 + 1);
-    const int s0 = (int)((long long)ns * r / C), s1 = (int)((long long)ns * (r + 1) / C);
     float* tile = reinterpret_cast<float*>(U);
     constexpr int kTile = (int)(((size_t)correct_smem_floats<G>()) / kPartStride);  // rows per tile
     const int c = tid & (kD - 1);

@@ -73,7 +73,6 @@ __global__ void __launch_bounds__(kScanWarps * 32, 1) scan_kernel(const ScanPara
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gid = lane >> 2, tig = lane & 3;
   pdl_wait();
-  pdl_launch_dependents();
   const long long wg = (long long)blockIdx.x * kScanWarps + warp;
   if (wg >= p.n_warps) return;
   const long long W = p.n_warps, T = p.total;
@@ -397,6 +396,9 @@ __global__ void __launch_bounds__(kScanWarps * 32, 1) scan_kernel(const ScanPara
     }
   }
   flush(cur);
+  // the next kernel may be scheduled once every scan CTA got here: launching it
+  // earlier would let its CTAs hold SMs the scan still needs
+  pdl_launch_dependents();
 }
 
 template <int KB, int VB>
