@@ -37,6 +37,10 @@ int workspace_layout(const jfa_geom& g, int max_topk, jfa_workspace_layout* out)
   L.partial_slots = (int32_t)(kMaxScanWarps + n_seg);
   L.off_partials = off;
   off = align_up(off + (size_t)L.partial_slots * G * kPartStride * sizeof(float), 256);
+  L.off_mused = off;
+  off = align_up(off + n_seg * (size_t)(g.capacity / kKG) * kMaxG * sizeof(float), 256);
+  L.off_scan_hist = off;
+  off = align_up(off + n_seg * kScanHistBins * sizeof(uint32_t), 256);
   L.off_hist = off;
   off += n_seg * kHistBins * sizeof(uint32_t);
   L.off_counters = off;
@@ -51,9 +55,6 @@ int workspace_layout(const jfa_geom& g, int max_topk, jfa_workspace_layout* out)
   L.max_topk = max_topk;
   L.off_sel = off;
   off = align_up(off + n_seg * n_chunks_cap * sizeof(uint32_t), 256);
-  L.merge_chunks = (max_topk + kTail + kMergeChunk - 1) / kMergeChunk;
-  L.off_merge = off;
-  off = align_up(off + n_seg * (size_t)L.merge_chunks * 2 * G * kPartStride * sizeof(float), 256);
   L.total_bytes = off;
   *out = L;
   return JFA_OK;
@@ -77,11 +78,12 @@ ScanPlan scan_plan(const jfa_geom& g, int num_sms) {
   const long long n_seg = (long long)g.batch * g.num_kv_heads;
   p.ng = split_point(g.n_ctx) / kKG;
   p.total_groups = n_seg * p.ng;
-  long long w = (long long)num_sms * kScanWarps;
+  const int nw = scan_cta_warps(g.key_bits, g.val_bits);
+  long long w = (long long)num_sms * nw;
   if (w > kMaxScanWarps) w = kMaxScanWarps;
   if (w > p.total_groups) w = p.total_groups;
   p.n_warps = (int)w;
-  p.n_ctas = (int)((w + kScanWarps - 1) / kScanWarps);
+  p.n_ctas = (int)((w + nw - 1) / nw);
   return p;
 }
 
@@ -171,9 +173,9 @@ int jfa_correct_merge(const jfa_geom* geom, const jfa_cache* cache, const uint16
     return JFA_ERR_INVALID_ARG;
   jfa_workspace_layout L;
   workspace_layout(*geom, k, &L);
-  return launch_correct_merge(*geom, *cache, q, scale, idx, k, k_exact, v_exact, exact_on_host,
-                              static_cast<uint8_t*>(ws), L, out,
-                              static_cast<cudaStream_t>(stream));
+  (void)exact_on_host;  // same loads either way; the rows are device-addressable
+  return launch_finish(*geom, *cache, q, scale, k, nullptr, idx, k_exact, v_exact,
+                       static_cast<uint8_t*>(ws), L, out, static_cast<cudaStream_t>(stream));
 }
 
 int jfa_decode_step(const jfa_geom* geom, const jfa_cache* cache, const uint16_t* q, float scale,
@@ -204,7 +206,7 @@ int jfa_decode_finish(const jfa_geom* geom, const jfa_cache* cache, const uint16
   (void)exact_on_host;  // same loads either way; the rows are device-addressable
   jfa_workspace_layout L;
   workspace_layout(*geom, k, &L);
-  return launch_finish(*geom, *cache, q, scale, k, idx, k_exact, v_exact,
+  return launch_finish(*geom, *cache, q, scale, k, idx, nullptr, k_exact, v_exact,
                        static_cast<uint8_t*>(ws), L, out, static_cast<cudaStream_t>(stream));
 }
 

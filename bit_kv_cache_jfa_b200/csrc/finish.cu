@@ -1,22 +1,26 @@
-// finish.cu — everything after the scan in one kernel: a thread-block cluster
-// of C CTAs (C <= 8) per (sequence, KV head) runs
-//   P1  histogram of the top 11 selection-key bits of each CTA's score slice,
-//   P1b CTA 0 sums the C histograms through distributed shared memory and
-//       finds the bin b* holding the k-th key,
-//   P2  each CTA writes its slice's keys with bin >= b* to an index-ordered
-//       list (block-scan compaction),
-//   P3  CTA 0 refines the k-th key over those lists (two more radix levels),
-//       resolves ties by index and writes the chosen indices in one ordered
-//       pass (to idx and to its shared memory),
-//   P4  each CTA corrects its share of the exact set (chosen tokens + tail):
-//       exact bf16 logits/values and the approximate terms to remove,
-//   P5  the CTAs owning a query head merge the scan partials and the exact
-//       and removal partials of all C CTAs (read through distributed shared
-//       memory) in log-sum-exp form and write the output row.
-// Cluster barriers replace the kernel boundaries of the separate
-// jfa_topk / jfa_correct_merge path; the arithmetic is the same.
+// finish.cu — everything after the scan in one kernel.  A thread-block
+// cluster of C CTAs (C <= 8) per (sequence, KV head):
+//   T   (before waiting for the scan) corrects its share of the bf16 tail;
+//   P1  reads the scan's 8192-bin histogram of the selection keys and finds
+//       the bin b* holding the k-th largest key (every CTA, redundantly);
+//   P2  lists its slice's keys above b* ("sure") and in b* ("ties"), in
+//       index order, in its shared memory;
+//   P3  after a cluster barrier, gathers every CTA's ties and resolves the
+//       k-th key inside b* by two more radix levels (ties to lower indices),
+//       writes its own chosen indices to idx in ascending order and takes
+//       an even share of the chosen set for the correction;
+//   P4  corrects that share: exact bf16 logits and values, and the scan's
+//       approximate terms of each chosen token recomputed bit for bit
+//       (jfa_approx.cuh, with the stored running maxima) for removal;
+//   P5  merges a share of the scan's split partials, then the CTAs owning a
+//       query head combine scan, exact and removal partials of all C CTAs
+//       (distributed shared memory) in log-sum-exp form.
+// With a given index set (jfa_correct_merge) P1-P3 are skipped.  If the
+// histogram is stale or the candidates overflow shared memory, every CTA
+// selects over the whole segment instead (slower, same result).
 #include <cooperative_groups.h>
 
+#include "jfa_approx.cuh"
 #include "jfa_blocks.cuh"
 
 namespace cg = cooperative_groups;
@@ -24,507 +28,910 @@ namespace cg = cooperative_groups;
 namespace jfa {
 
 constexpr int kFinThreads = 256;
-constexpr int kFinStage = 4096;  // list entries CTA 0 stages in shared memory
 constexpr int kFinMaxC = 8;
+constexpr int kLCap = 1024;   // sure / tie list entries per CTA
+constexpr int kTCap = 1024;   // gathered tie entries
+constexpr int kRefBins = 2048;
+constexpr int kWD = 3;        // cp.async stages per warp (tokens in flight)
+constexpr int kFinWarps = kFinThreads / 32;
 
 struct FinishParams {
-  MergeParams m;          // correction / merge inputs (m.idx unused)
-  const float* scores;    // [n_seg][capacity] selection scores from the scan
-  int32_t* idx_out;       // [n_seg][k]
-  uint2* lists;           // [n_seg * C][slice] per-CTA ordered (key, index) lists
-  int slice;              // scores per CTA, multiple of 64
+  const uint8_t* groups;
+  const uint16_t* tail_k;
+  const uint16_t* tail_v;
+  const uint16_t* k_exact;
+  const uint16_t* v_exact;
+  const uint16_t* q;
+  const float* scores;     // [n_seg][capacity]
+  const float* scan_part;  // per scan warp and segment: [slot][G][kPartStride]
+  const float* m_used;     // [n_seg][ng_cap][8]
+  uint32_t* hist;          // [n_seg][kScanHistBins], zeroed here after use
+  uint32_t* glists;        // [n_seg][C][slice] chosen lists of the fallback
+  const int32_t* idx_in;   // given index sets (no selection), [n_seg][k]
+  int32_t* idx_out;        // [n_seg][k] (selection)
+  float* out;
+  uint32_t* flag;
+  int k, nq, tail, capacity, ng_cap, hkv, H, key_bits, val_bits, rec_bytes, ng, slice;
+  long long scan_total;
+  int scan_warps;
+  float kappa;
 };
 
+// Shared memory.  The persistent part is read by other CTAs of the cluster
+// (lists, counts, partials) and lives until the last barrier; the union part
+// is private and reused: selection buffers, then the correction's token list
+// and per-warp staging rings.
+struct FinPersist {
+  uint32_t sure[kLCap];               // chosen-for-sure indices of the slice, ascending
+  uint32_t tkey[kLCap], tidx[kLCap];  // ties of the slice (key, index), ascending index
+  uint32_t chtie[kTCap];              // chosen ties of the whole segment, ascending
+  uint32_t n_sure, n_tie, overflow, n_gl;
+};
+// A correction partial (m, l, pad, pad, acc[128]) per query head; in the
+// combined form the top-k tokens' approximate terms enter with a minus sign,
+// so l may be negative.
 template <int G>
-constexpr size_t finish_smem_bytes() {
-  constexpr size_t sel = kHistBins * 4 + kFinStage * 8;
-  constexpr size_t cor = (size_t)correct_smem_floats<G>() * 4;
-  return JFA_MAX_TOPK * 4 + 2 * (2 * G * kPartStride * 4) + (sel > cor ? sel : cor);
+struct FinParts {
+  float qs[G][kD];
+  float run[G][kPartStride];   // this CTA's exact-minus-removed partial
+  float sp[G][kPartStride];    // this CTA's share of the scan partials
+  float wp[kFinWarps][G][kPartStride];  // per-warp partials
+};
+// Shared-memory histograms store bin b at hpad(b) = b + b/32, so threads
+// that each read a contiguous run of bins hit distinct banks.
+__device__ __forceinline__ int hpad(int b) { return b + (b >> 5); }
+struct FinSelect {
+  uint32_t hist[kRefBins + kRefBins / 32];
+  uint32_t akey[kTCap], aidx[kTCap];
+};
+// Record pieces of one quantized token, staged by cp.async.
+struct WStage {
+  uint8_t ksz[512];    // key scales / zeros of its group
+  uint8_t kcode[512];  // key codes of its 8-token tile, in lane order
+  uint8_t vp[256];     // value-code pieces holding its column (8 or 16 x 16 B)
+  uint8_t vsz[64];     // its value scales (32 B block) and zeros (32 B block)
+  float mu[kMaxG];     // the scan's running maxima of its group
+};
+constexpr int kTokCap = 1024;  // tokens listed per correction round
+struct FinCorr {
+  WStage st[kFinWarps][kWD];
+  int32_t tok[kTokCap];
+};
+template <int G>
+constexpr size_t fin_smem_bytes() {
+  return sizeof(FinPersist) + sizeof(FinParts<G>) +
+         (sizeof(FinSelect) > sizeof(FinCorr) ? sizeof(FinSelect) : sizeof(FinCorr));
 }
 
-// Selection over an index-ordered list given by get(i), i < total: the k-th
-// key K* below bin b* (r = keys still to take from bin b*), ties to the lowest
-// indices, chosen indices written ascending to out[] and chosen[].
-template <typename Get>
-__device__ void select_ordered(Get get, uint32_t total, uint32_t bstar, uint32_t r, int k,
-                               int32_t* out, int32_t* chosen, uint32_t* h, uint32_t* scratch,
-                               int* s_bin, uint32_t* s_above) {
+// Block-wide maximum of a float (all threads get it).
+__device__ __forceinline__ float block_max(float v, float* scratch) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(kAll, v, o));
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  __syncthreads();
+  if (lane == 0) scratch[warp] = v;
+  __syncthreads();
+  float m = scratch[0];
+  for (int w = 1; w < (int)(blockDim.x >> 5); ++w) m = fmaxf(m, scratch[w]);
+  __syncthreads();
+  return m;
+}
+
+// From bin counts h[hpad(0..nbins)) (nbins a multiple of blockDim) find the
+// bin where the count taken from the top reaches r (1 <= r); *bin = -1 if
+// the total < r.
+__device__ __noinline__ void find_bin_from_top(const uint32_t* h, int nbins, uint32_t r, uint32_t* scratch,
+                                  int* bin, uint32_t* above, uint32_t* total) {
+  const int per = nbins / blockDim.x;
+  const int b0 = threadIdx.x * per;
+  uint32_t local = 0;
+  for (int i = 0; i < per; ++i) local += h[hpad(b0 + i)];
+  uint32_t tot;
+  block_prefix_excl(local, scratch, &tot);
+  uint32_t cum = block_suffix_excl(local, scratch);
+  if (threadIdx.x == 0) *bin = -1;
+  __syncthreads();
+  for (int i = per - 1; i >= 0; --i) {
+    const uint32_t c = h[hpad(b0 + i)];
+    if (cum < r && cum + c >= r) {
+      *bin = b0 + i;
+      *above = cum;
+    }
+    cum += c;
+  }
+  if (threadIdx.x == 0) *total = tot;
+  __syncthreads();
+}
+
+// Selection inside the histogram bin b* (keys share their top 13 bits):
+// the r largest of the T ties akey/aidx (index order), larger key first and
+// equal keys to the lower index, two radix levels (11 + 8 bits) and one
+// ordered pass.  Writes the chosen indices ascending to chosen[] (r of them).
+__device__ __noinline__ void refine_ties(const uint32_t* akey, const uint32_t* aidx, uint32_t T, uint32_t r,
+                            uint32_t* h, uint32_t* chosen, uint32_t* scratch, int* s_bin,
+                            uint32_t* s_above, uint32_t* s_tot) {
   const int tid = threadIdx.x;
-  for (int i = tid; i < kHistBins; i += blockDim.x) h[i] = 0u;
-  if (tid == 0) {
-    *s_bin = 0;
-    *s_above = 0;
-  }
+  // level 2: key bits 18..8
+  for (int i = tid; i < hpad(kRefBins); i += blockDim.x) h[i] = 0u;
   __syncthreads();
-  for (uint32_t i = tid; i < total; i += blockDim.x) {
-    const uint32_t key = get(i).x;
-    if ((key >> 21) == bstar) atomicAdd(&h[(key >> 10) & 2047u], 1u);
-  }
+  for (uint32_t i = tid; i < T; i += blockDim.x) atomicAdd(&h[hpad((akey[i] >> 8) & 2047u)], 1u);
   __syncthreads();
-  find_from_top(h, 2048, r, scratch, s_bin, s_above);
+  find_bin_from_top(h, kRefBins, r, scratch, s_bin, s_above, s_tot);
   const uint32_t d2 = (uint32_t)*s_bin;
   const uint32_t r2 = r - *s_above;
-  const uint32_t pre = (bstar << 11) | d2;
   __syncthreads();
-  for (int i = tid; i < kHistBins; i += blockDim.x) h[i] = 0u;
+  // level 3: key bits 7..0 among keys whose bits 18..8 are d2
+  for (int i = tid; i < hpad(256); i += blockDim.x) h[i] = 0u;
   __syncthreads();
-  for (uint32_t i = tid; i < total; i += blockDim.x) {
-    const uint32_t key = get(i).x;
-    if ((key >> 10) == pre) atomicAdd(&h[key & 1023u], 1u);
-  }
+  for (uint32_t i = tid; i < T; i += blockDim.x)
+    if (((akey[i] >> 8) & 2047u) == d2) atomicAdd(&h[hpad(akey[i] & 255u)], 1u);
   __syncthreads();
-  find_from_top(h, 1024, r2, scratch, s_bin, s_above);
-  const uint32_t kstar = (pre << 10) | (uint32_t)*s_bin;
+  find_bin_from_top(h, 256, r2, scratch, s_bin, s_above, s_tot);
+  const uint32_t low = (akey[0] >> 19) << 19;  // the shared top bits
+  const uint32_t kstar = low | (d2 << 8) | (uint32_t)*s_bin;
   const uint32_t r3 = r2 - *s_above;
-  // thread t owns entries [t*per, (t+1)*per), so block scans order the list
-  const uint32_t per = (total + blockDim.x - 1) / blockDim.x;
-  const uint32_t i0 = tid * per, i1 = min(total, i0 + per);
+  __syncthreads();
+  // ordered pass: thread t owns entries [t*per, (t+1)*per)
+  const uint32_t per = (T + blockDim.x - 1) / blockDim.x;
+  const uint32_t i0 = min(T, tid * per), i1 = min(T, i0 + per);
   uint32_t n_eq = 0;
-  for (uint32_t i = i0; i < i1; ++i) n_eq += get(i).x == kstar;
+  for (uint32_t i = i0; i < i1; ++i) n_eq += akey[i] == kstar;
   uint32_t tot;
-  uint32_t eq_rank = block_prefix_excl(n_eq, scratch, &tot);
+  uint32_t er = block_prefix_excl(n_eq, scratch, &tot);
   uint32_t n_ch = 0;
   {
-    uint32_t er = eq_rank;
+    uint32_t e2 = er;
     for (uint32_t i = i0; i < i1; ++i) {
-      const uint32_t key = get(i).x;
-      const bool eq = key == kstar;
-      n_ch += (key > kstar || (eq && er < r3)) ? 1u : 0u;
-      er += eq;
+      const bool eq = akey[i] == kstar;
+      n_ch += (akey[i] > kstar || (eq && e2 < r3)) ? 1u : 0u;
+      e2 += eq;
     }
   }
   uint32_t pos = block_prefix_excl(n_ch, scratch, &tot);
   for (uint32_t i = i0; i < i1; ++i) {
-    const uint2 e = get(i);
-    const bool eq = e.x == kstar;
-    if (e.x > kstar || (eq && eq_rank < r3)) {
-      if (pos < (uint32_t)k) {
-        out[pos] = (int32_t)e.y;
-        chosen[pos] = (int32_t)e.y;
-      }
-      ++pos;
-    }
-    eq_rank += eq;
+    const bool eq = akey[i] == kstar;
+    if (akey[i] > kstar || (eq && er < r3)) chosen[pos++] = aidx[i];
+    er += eq;
   }
+  __syncthreads();
 }
 
-// L2 prefetch of what the correction of token t reads (t: token index, or
-// (1 << 30) | tail slot): bf16 K/V rows and, for quantized tokens, the key
-// scales/zeros, key codes and value scales/codes of its record.  part picks
-// one of kPrefParts 128-byte pieces, so consecutive threads split the work.
-constexpr int kPrefParts = 12;
-__device__ __forceinline__ void prefetch_token(const MergeParams& p, int seg, int t, int part) {
-  if (t < 0) return;
-  if (t & (1 << 30)) {
-    const int tt = t & ~(1 << 30);
-    if (part < 4) {
-      const uint16_t* row = ((part & 2) ? p.tail_v : p.tail_k) + ((size_t)seg * kTail + tt) * kD;
-      prefetch_l2(row + 64 * (part & 1));
+// Fallback selection over the whole segment (stale histogram or too many
+// candidates): three radix levels (11 + 11 + 10 bits) over all nq scores, then this CTA's slice
+// [lo, hi) of chosen indices, ascending, into out[]; returns their count.
+__device__ __noinline__ uint32_t select_full(const float* S, int nq, int k, int lo, int hi, uint32_t* h,
+                                uint32_t* out, uint32_t* scratch, int* s_bin, uint32_t* s_above,
+                                uint32_t* s_tot) {
+  const int tid = threadIdx.x;
+  uint32_t prefix = 0, r = (uint32_t)k;
+  const int shifts[3] = {21, 10, 0};
+  const int bits[3] = {11, 11, 10};
+#pragma unroll 1
+  for (int lv = 0; lv < 3; ++lv) {
+    const int nb = 1 << bits[lv];
+    for (int i = tid; i < hpad(nb); i += blockDim.x) h[i] = 0u;
+    __syncthreads();
+    const int hs = lv == 0 ? 32 : shifts[lv - 1];
+    for (int i = tid; i < nq; i += blockDim.x) {
+      const uint32_t key = float_key(S[i]);
+      if (lv == 0 || (key >> hs) == prefix) atomicAdd(&h[hpad((key >> shifts[lv]) & (nb - 1))], 1u);
     }
-    return;
+    __syncthreads();
+    find_bin_from_top(h, nb, r, scratch, s_bin, s_above, s_tot);
+    prefix = (prefix << bits[lv]) | (uint32_t)*s_bin;
+    r -= *s_above;
+    __syncthreads();
   }
-  const uint8_t* rec = p.groups + ((size_t)seg * p.ng_cap + t / kKG) * p.rec_bytes;
-  const int tt = t % kKG;
-  if (part < 4) {
-    const uint16_t* row = ((part & 2) ? p.v_exact : p.k_exact) + ((size_t)seg * p.capacity + t) * kD;
-    prefetch_l2(row + 64 * (part & 1));
-  } else if (part < 8) {
-    prefetch_l2(rec + off_ks() + 128 * (part - 4));  // key scales/zeros (512 B)
-  } else if (part == 8) {
-    const int nt = tt >> 3, gd = tt & 7;
-    prefetch_l2(rec + off_kc() +
-                (p.key_bits == 4 ? nt * 512 + gd * 64 : (nt >> 2) * 1536 + gd * 192));
-  } else if (part == 9) {
-    prefetch_l2(rec + off_vs(p.key_bits) + (tt >> 4) * 128);
-  } else {
-    const int kk = tt >> 4;
-    const int chunk = p.val_bits == 4 ? 2 * kk + (part - 10) : kk;
-    prefetch_l2(rec + off_vc(p.key_bits) + chunk * 512 + 256 * (p.val_bits == 4 ? 0 : (part - 10)));
+  const uint32_t kstar = prefix;
+  // equal keys before the slice
+  uint32_t n_eq = 0;
+  for (int i = tid; i < lo; i += blockDim.x) n_eq += float_key(S[i]) == kstar;
+  uint32_t tot;
+  block_prefix_excl(n_eq, scratch, &tot);
+  const uint32_t eq_before = tot;
+  const uint32_t len = (uint32_t)(hi - lo);
+  const uint32_t per = (len + blockDim.x - 1) / blockDim.x;
+  const uint32_t i0 = min(len, tid * per), i1 = min(len, i0 + per);
+  uint32_t ne = 0;
+  for (uint32_t i = i0; i < i1; ++i) ne += float_key(S[lo + i]) == kstar;
+  uint32_t er = eq_before + block_prefix_excl(ne, scratch, &tot);
+  uint32_t nc = 0;
+  {
+    uint32_t e2 = er;
+    for (uint32_t i = i0; i < i1; ++i) {
+      const uint32_t key = float_key(S[lo + i]);
+      const bool eq = key == kstar;
+      nc += (key > kstar || (eq && e2 < r)) ? 1u : 0u;
+      e2 += eq;
+    }
   }
+  uint32_t pos = block_prefix_excl(nc, scratch, &tot);
+  for (uint32_t i = i0; i < i1; ++i) {
+    const uint32_t key = float_key(S[lo + i]);
+    const bool eq = key == kstar;
+    if (key > kstar || (eq && er < r)) out[pos++] = (uint32_t)(lo + i);
+    er += eq;
+  }
+  __syncthreads();
+  return tot;
 }
 
+// Number of entries of the ascending list a[0..n) below v.
+__device__ __forceinline__ uint32_t lower_bound_u32(const uint32_t* a, uint32_t n, uint32_t v) {
+  uint32_t lo = 0, hi = n;
+  while (lo < hi) {
+    const uint32_t mid = (lo + hi) >> 1;
+    if (a[mid] < v) lo = mid + 1;
+    else hi = mid;
+  }
+  return lo;
+}
+
+// ---------------------------------------------------------------------------
+// Correction, a warp per token.  Token encoding: t in [0, nq) a quantized
+// token, (1 << 30) | s the tail slot s.  Lane l owns channels 4l..4l+3 of
+// every head.  The quantized token's record pieces are staged by cp.async
+// kWD tokens ahead; its exact bf16 row is loaded one token ahead.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ bool tok_quant(int t) { return t >= 0 && !(t & (1 << 30)); }
+
+template <typename T4>
+__device__ __forceinline__ T4 ld16(const void* p) {
+  return *reinterpret_cast<const T4*>(p);
+}
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Stage the record pieces of token t (one commit group per lane, possibly empty).
+__device__ __forceinline__ void stage_issue(const FinishParams& p, int seg, int t, WStage& S,
+                                            int lane) {
+  if (tok_quant(t)) {
+    const uint8_t* rec = p.groups + ((size_t)seg * p.ng_cap + (size_t)(t / kKG)) * p.rec_bytes;
+    const int tt = t % kKG, nt = tt >> 3, kk = tt >> 4, tgt = (tt & 7) >> 1;
+    cp_async16(S.ksz + lane * 16, rec + lane * 16);
+    if (p.key_bits == 4) {
+      cp_async16(S.kcode + lane * 16, rec + off_kc() + nt * 512 + lane * 16);
+    } else {
+      const uint8_t* src = rec + off_kc() + (nt >> 2) * 1536 + lane * 48 + (nt & 3) * 12;
+      cp_async4(S.kcode + lane * 12, src);
+      cp_async4(S.kcode + lane * 12 + 4, src + 4);
+      cp_async4(S.kcode + lane * 12 + 8, src + 8);
+    }
+    const int vslots = p.val_bits == 4 ? 16 : 8;
+    if (lane < vslots) {
+      const int chunk = p.val_bits == 4 ? 2 * kk + (lane >> 3) : kk;
+      cp_async16(S.vp + lane * 16, rec + off_vc(p.key_bits) + chunk * 512 + ((lane & 7) * 4 + tgt) * 16);
+    }
+    if (lane < 4)
+      cp_async16(S.vsz + lane * 16,
+                 rec + off_vs(p.key_bits) + kk * 128 + tgt * 32 + (lane & 1) * 16 + (lane >> 1) * 512);
+    if (lane < 2)
+      cp_async16(reinterpret_cast<uint8_t*>(S.mu) + lane * 16,
+                 p.m_used + ((size_t)seg * p.ng_cap + (size_t)(t / kKG)) * kMaxG + lane * 4);
+  }
+  cp_async_commit();
+}
+
+// Exact bf16 row pieces of token t for lane l: channels 4l..4l+3 of K and V.
+__device__ __forceinline__ void row_load(const FinishParams& p, int seg, int t, int lane, uint2& kr,
+                                         uint2& vr) {
+  const size_t off = (t & (1 << 30)) ? ((size_t)seg * kTail + (t & 0xFFFF)) * kD
+                                     : ((size_t)seg * p.capacity + t) * kD;
+  const uint16_t* kb = (t & (1 << 30)) ? p.tail_k : p.k_exact;
+  const uint16_t* vb = (t & (1 << 30)) ? p.tail_v : p.v_exact;
+  kr = *reinterpret_cast<const uint2*>(kb + off + 4 * lane);
+  vr = *reinterpret_cast<const uint2*>(vb + off + 4 * lane);
+}
+
+// The scan's fp16 weights of quantized token t for every head, recomputed
+// from its staged group pieces with the scan's own arithmetic (q_frag,
+// key_sz/q_tilde, qk_chain, approx_logit, approx_weight, in the same order,
+// here fused per k-step); ph[j] = fp16 bits of head j's weight, on all lanes.
 template <int G>
-__global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishParams fp) {
+__device__ __forceinline__ void replay_weights(const FinishParams& p, int t, const WStage& S,
+                                               const uint32_t q2[16], int lane, uint32_t ph[G]) {
+  const int gid = lane >> 2, tig = lane & 3;
+  const int tt = t % kKG, tq = (tt & 7) >> 1, e = tt & 1;
+  uint32_t b[16];
+  if (p.key_bits == 4) {
+    const uint4 c = ld16<uint4>(S.kcode + lane * 16);
+    unpack4(c.x, b);
+    unpack4(c.y, b + 4);
+    unpack4(c.z, b + 8);
+    unpack4(c.w, b + 12);
+  } else {
+    const uint32_t* w = reinterpret_cast<const uint32_t*>(S.kcode + lane * 12);
+    unpack3(w[0], w[1], w[2], b);
+  }
+  float d[4] = {0.f, 0.f, 0.f, 0.f}, db[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int ks = 0; ks < 8; ++ks) {
+    const int p0 = 2 * ks, p1 = 2 * ks + 1;
+    const uint32_t s0 = *reinterpret_cast<const uint32_t*>(S.ksz + (p0 >> 2) * 64 + tig * 16 + (p0 & 3) * 4);
+    const uint32_t s1 = *reinterpret_cast<const uint32_t*>(S.ksz + (p1 >> 2) * 64 + tig * 16 + (p1 & 3) * 4);
+    const uint32_t z0 = *reinterpret_cast<const uint32_t*>(S.ksz + (4 + (p0 >> 2)) * 64 + tig * 16 + (p0 & 3) * 4);
+    const uint32_t z1 = *reinterpret_cast<const uint32_t*>(S.ksz + (4 + (p1 >> 2)) * 64 + tig * 16 + (p1 & 3) * 4);
+    const uint32_t h0 = h2_mul(q2[p0], s0), h1 = h2_mul(q2[p1], s1);
+    const uint32_t l0 = h2_fma(q2[p0], s0, h0 ^ 0x80008000u);
+    const uint32_t l1 = h2_fma(q2[p1], s1, h1 ^ 0x80008000u);
+    mma16816(db, q2[p0], 0u, q2[p1], 0u, z0, z1);
+    mma16816(d, h0, l0, h1, l1, b[p0], b[p1]);
+  }
+  const float bk = __fmul_rn(db[0], p.kappa);
+  uint32_t mine = 0u;
+  if (gid < G && tig == tq) mine = f2h_rn(approx_weight(approx_logit(d, e, p.kappa, bk), S.mu[gid]));
+#pragma unroll
+  for (int j = 0; j < G; ++j) ph[j] = __shfl_sync(kAll, mine, j * 4 + tq);
+}
+
+// One token into the warp's combined partial (m, l, a): + its exact term,
+// and, for a quantized token, - the approximate term the scan added for it.
+template <int G>
+__device__ __forceinline__ void warp_token(const FinishParams& p, int t, const WStage& S, uint2 kr,
+                                           uint2 vr, const FinParts<G>& P, const uint32_t q2[16],
+                                           int lane, float (&m)[G], float (&l)[G],
+                                           float (&a)[G][4]) {
+  const float kf[4] = {__uint_as_float(kr.x << 16), __uint_as_float(kr.x & 0xFFFF0000u),
+                       __uint_as_float(kr.y << 16), __uint_as_float(kr.y & 0xFFFF0000u)};
+  const float vf[4] = {__uint_as_float(vr.x << 16), __uint_as_float(vr.x & 0xFFFF0000u),
+                       __uint_as_float(vr.y << 16), __uint_as_float(vr.y & 0xFFFF0000u)};
+  float se[G];
+#pragma unroll
+  for (int j = 0; j < G; ++j) {
+    const float4 qv = *reinterpret_cast<const float4*>(&P.qs[j][4 * lane]);
+    se[j] = warp_sum(fmaf(qv.x, kf[0], fmaf(qv.y, kf[1], fmaf(qv.z, kf[2], qv.w * kf[3])))) * p.kappa;
+  }
+  const bool qt = tok_quant(t);
+  uint32_t ph[G];
+  float code[4] = {0.f, 0.f, 0.f, 0.f};
+  uint16_t svb = 0;
+  float zv = 0.f;
+  if (qt) {
+    replay_weights<G>(p, t, S, q2, lane, ph);
+    const int tt = t % kKG, rt = tt & 15, hi8 = rt >> 3, e = rt & 1, jg = lane >> 3;
+    svb = *reinterpret_cast<const uint16_t*>(S.vsz + jg * 8 + hi8 * 4 + 2 * e);
+    zv = h2f(*reinterpret_cast<const uint16_t*>(S.vsz + 32 + jg * 8 + hi8 * 4 + 2 * e));
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int c = 4 * lane + i, mt = c >> 4, rc = c & 15, gd = rc & 7, r = (rc >> 3) + 2 * hi8;
+      if (p.val_bits == 4) {
+        const uint32_t w = *reinterpret_cast<const uint32_t*>(S.vp + ((mt >> 2) * 8 + gd) * 16 + (mt & 3) * 4);
+        code[i] = (float)((w >> (4 * r + 16 * e)) & 15u);
+      } else {
+        const uint32_t w = *reinterpret_cast<const uint32_t*>(S.vp + gd * 16 + (mt >> 1) * 4);
+        code[i] = (float)((w >> (2 * (4 * (mt & 1) + r) + 16 * e)) & 3u);
+      }
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < G; ++j) {
+    const float mu = qt ? S.mu[j] : -INFINITY;
+    const float mn = fmaxf(fmaxf(m[j], se[j]), mu);
+    const float al = exp2f(m[j] - mn);  // 0 while the partial is empty (m = -inf)
+    const float pe = exp2f(se[j] - mn);
+    l[j] = fmaf(l[j], al, pe);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) a[j][i] = fmaf(a[j][i], al, pe * vf[i]);
+    if (qt) {
+      const float f = exp2f(mu - mn);
+      const uint16_t phj = (uint16_t)ph[j];
+      const float pf = h2f(phj), w = h2f(h_mul_rn(phj, svb));
+      l[j] -= pf * f;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[j][i] -= f * fmaf(w, code[i], pf * zv);
+    }
+    m[j] = mn;
+  }
+}
+
+// The warp's tokens tok_at(0..n) into its partial P.wp[warp] (loaded,
+// updated, stored back).
+template <int G, typename TokAt>
+__device__ __forceinline__ void warp_correct(const FinishParams& p, int seg, TokAt tok_at, int n,
+                                             WStage* ring, FinParts<G>& P, const uint32_t q2[16],
+                                             int warp, int lane) {
+  float m[G], l[G], a[G][4];
+#pragma unroll
+  for (int j = 0; j < G; ++j) {
+    m[j] = P.wp[warp][j][0];
+    l[j] = P.wp[warp][j][1];
+    const float4 v = *reinterpret_cast<const float4*>(&P.wp[warp][j][4 + 4 * lane]);
+    a[j][0] = v.x;
+    a[j][1] = v.y;
+    a[j][2] = v.z;
+    a[j][3] = v.w;
+  }
+#pragma unroll
+  for (int i = 0; i < kWD - 1; ++i) stage_issue(p, seg, i < n ? tok_at(i) : -1, ring[i], lane);
+  uint2 kr = make_uint2(0u, 0u), vr = kr;
+  if (n > 0) row_load(p, seg, tok_at(0), lane, kr, vr);
+#pragma unroll 1
+  for (int i = 0; i < n; ++i) {
+    const int t = tok_at(i);
+    stage_issue(p, seg, i + kWD - 1 < n ? tok_at(i + kWD - 1) : -1, ring[(i + kWD - 1) % kWD], lane);
+    uint2 kn = kr, vn = vr;
+    if (i + 1 < n) row_load(p, seg, tok_at(i + 1), lane, kn, vn);
+    cp_async_wait<kWD - 1>();
+    __syncwarp();
+    warp_token<G>(p, t, ring[i % kWD], kr, vr, P, q2, lane, m, l, a);
+    __syncwarp();
+    kr = kn;
+    vr = vn;
+  }
+  cp_async_wait<0>();
+  __syncwarp();
+#pragma unroll
+  for (int j = 0; j < G; ++j) {
+    if (lane == 0) {
+      P.wp[warp][j][0] = m[j];
+      P.wp[warp][j][1] = l[j];
+    }
+    *reinterpret_cast<float4*>(&P.wp[warp][j][4 + 4 * lane]) = make_float4(a[j][0], a[j][1], a[j][2], a[j][3]);
+  }
+  __syncwarp();
+}
+
+template <int G, bool SELECT>
+__global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishParams p) {
   extern __shared__ __align__(16) uint8_t fsm[];
-  const MergeParams& p = fp.m;
+  FinPersist& PS = *reinterpret_cast<FinPersist*>(fsm);
+  FinParts<G>& P = *reinterpret_cast<FinParts<G>*>(fsm + sizeof(FinPersist));
+  uint8_t* U = fsm + sizeof(FinPersist) + sizeof(FinParts<G>);
+  FinSelect& SS = *reinterpret_cast<FinSelect*>(U);
+  FinCorr& FC = *reinterpret_cast<FinCorr*>(U);
+  __shared__ uint32_t scratch[32];
+  __shared__ int s_bin;
+  __shared__ uint32_t s_above, s_tot;
+  __shared__ uint32_t s_cnt[kFinMaxC], s_pre[kFinMaxC + 1], s_tpre[kFinMaxC + 1];
+  __shared__ uint32_t s_chq[kFinMaxC + 1];  // chosen ties before slice q
+  __shared__ int s_mode;                     // 0 lists in shared memory, 1 fallback lists
+
   cg::cluster_group cl = cg::this_cluster();
   const int C = (int)cl.num_blocks();
   const int r = (int)cl.block_rank();
   const int seg = blockIdx.x / C;
-  const int tid = threadIdx.x;
-  int32_t* chosen = reinterpret_cast<int32_t*>(fsm);
-  float* run = reinterpret_cast<float*>(fsm + JFA_MAX_TOPK * 4);  // [2][G][kPartStride]
-  float* bat = run + 2 * G * kPartStride;                          // [2][G][kPartStride]
-  uint8_t* U = reinterpret_cast<uint8_t*>(bat + 2 * G * kPartStride);
-  uint32_t* hist = reinterpret_cast<uint32_t*>(U);
-  uint2* stage = reinterpret_cast<uint2*>(U + kHistBins * 4);
-  __shared__ uint32_t scratch[32];
-  __shared__ int s_bin;
-  __shared__ uint32_t s_above;
-  __shared__ uint32_t s_bstar, s_babove, s_count;
-  __shared__ uint32_t s_off[kFinMaxC + 1];
-  __shared__ int s_tok[kMergeChunk];
+  const int tid = threadIdx.x, lane = tid & 31, gid = lane >> 2, tig = lane & 3;
+  const int nq = p.nq, k = p.k;
+  const int bb = seg / p.hkv, hh = seg % p.hkv;
+
+  // ---- set-up: nothing here is written by the scan
+  for (int i = tid; i < G * kD; i += kFinThreads)
+    P.qs[i / kD][i % kD] = bf16f(p.q[((size_t)bb * p.H + hh * G + i / kD) * kD + i % kD]);
+  for (int i = tid; i < kFinWarps * G * kPartStride; i += kFinThreads)
+    (&P.wp[0][0][0])[i] = (i % kPartStride) == 0 ? -INFINITY : 0.f;
+  uint32_t q2[16];
+  q_frag(p.q + ((size_t)bb * p.H + (size_t)hh * G + (gid < G ? gid : 0)) * kD, gid < G, tig, q2);
+  __syncthreads();
+  const int warp = tid >> 5;
+
+  // ---- T: this CTA's tail slots r, r + C, ... (exact rows only), warp w
+  // taking every kFinWarps-th of them
+  {
+    const int n_mine = p.tail > r ? (p.tail - r + C - 1) / C : 0;
+    const int n_w = n_mine > warp ? (n_mine - warp + kFinWarps - 1) / kFinWarps : 0;
+    auto tail_at = [&](int i) { return (1 << 30) | (r + C * (warp + kFinWarps * i)); };
+    warp_correct<G>(p, seg, tail_at, n_w, FC.st[warp], P, q2, warp, lane);
+  }
 
   pdl_wait();
   pdl_launch_dependents();
 
-  const int nq = p.nq, k = p.k;
-  const int keff = min(k, nq);
-  const bool select = k < nq;
-  const int lo = r * fp.slice, hi = min(nq, lo + fp.slice);
-  const float* S = fp.scores + (size_t)seg * p.capacity;
-  uint2* lists = fp.lists + (size_t)seg * C * fp.slice;
-  // exact-set share of this CTA (P4) and scan slots it merges (P5a)
-  const int nE = keff + p.tail;
-  const int e_per = (nE + C - 1) / C;
-  const int e0 = r * e_per, e1 = min(nE, e0 + e_per);
-  long long w0 = 0, w1 = -1;
-  if (p.ng > 0) {
-    const long long T = p.scan_total, W = p.scan_warps;
-    const long long x0 = (long long)seg * p.ng, x1 = x0 + p.ng - 1;
-    w0 = scan_warp_of(x0, W, T);
-    w1 = scan_warp_of(x1, W, T);
-  }
-  const int ns = (int)(w1 - w0 + 1);
-  const int s0 = (int)((long long)ns * r / C), s1 = (int)((long long)ns * (r + 1) / C);
-  // known from the start: the tail tokens among this CTA's share, and its
-  // scan-slot rows -- start pulling them into L2 now
-  for (int i = tid; i < (e1 - e0) * kPrefParts; i += kFinThreads) {
-    const int e = e0 + i / kPrefParts;
-    if (e >= keff) prefetch_token(p, seg, (1 << 30) | (e - keff), i % kPrefParts);
-  }
-  for (int i = tid; i < (s1 - s0) * G * 5; i += kFinThreads) {
-    const int row = s0 * G + i / 5;
-    prefetch_l2(p.scan_part + ((size_t)(w0 + row / G + seg) * G + row % G) * kPartStride +
-                32 * (i % 5));
-  }
-
-  // ---- P1: histogram of this CTA's slice
+  const bool select = SELECT && k < nq;
+  const int lo = min(nq, r * p.slice), hi = min(nq, lo + p.slice);
+  bool hist_ok = false;
+  // ---- P1 + P2: bin b* from the scan's histogram, then this slice's lists
   if (select) {
-    for (int i = tid; i < kHistBins; i += kFinThreads) hist[i] = 0u;
+    // thread t owns bins [32t, 32t + 32): loaded straight into registers
+    const uint32_t* hg = p.hist + (size_t)seg * kScanHistBins + 32 * tid;
+    uint32_t hb[32];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const uint4 v = ld16<uint4>(hg + 4 * u);
+      hb[4 * u] = v.x;
+      hb[4 * u + 1] = v.y;
+      hb[4 * u + 2] = v.z;
+      hb[4 * u + 3] = v.w;
+    }
+    uint32_t local = 0;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) local += hb[i];
+    uint32_t tot_all;
+    block_prefix_excl(local, scratch, &tot_all);
+    uint32_t cum = block_suffix_excl(local, scratch);  // keys in bins above this thread's
+    if (tid == 0) {
+      s_bin = -1;
+      s_tot = tot_all;
+    }
     __syncthreads();
-    for (int t0 = lo; t0 < hi; t0 += 16 * kFinThreads) {
-      const int b0 = t0 + 16 * tid;
-      float4 v[4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
-        v[u] = b0 + 4 * u < hi ? *reinterpret_cast<const float4*>(S + b0 + 4 * u)
-                               : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int i = 31; i >= 0; --i) {
+      if (cum < (uint32_t)k && cum + hb[i] >= (uint32_t)k) {
+        s_bin = 32 * tid + i;
+        s_above = cum;
+      }
+      cum += hb[i];
+    }
+    __syncthreads();
+    hist_ok = s_tot == (uint32_t)nq && s_bin >= 0;
+    const uint32_t bstar = (uint32_t)s_bin;
+    uint32_t base_s = 0, base_t = 0;
+    if (hist_ok) {
+      const float* S = p.scores + (size_t)seg * p.capacity;
+      for (int t0 = lo; t0 < hi; t0 += 16 * kFinThreads) {
+        const int b0 = t0 + 16 * tid;
+        float4 v[4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        if (b0 + 4 * u < hi) {
-          atomicAdd(&hist[float_key(v[u].x) >> 21], 1u);
-          atomicAdd(&hist[float_key(v[u].y) >> 21], 1u);
-          atomicAdd(&hist[float_key(v[u].z) >> 21], 1u);
-          atomicAdd(&hist[float_key(v[u].w) >> 21], 1u);
+        for (int u = 0; u < 4; ++u)
+          v[u] = b0 + 4 * u < hi ? ld16<float4>(S + b0 + 4 * u) : make_float4(0.f, 0.f, 0.f, 0.f);
+        uint32_t keys[16];
+        uint32_t ms = 0, mt = 0, ns = 0, nt = 0;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float vals[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int i = 4 * u + e;
+            keys[i] = float_key(vals[e]);
+            const bool in = b0 + i < hi;
+            const uint32_t bin = keys[i] >> (32 - kScanHistBits);
+            const bool su = in && bin > bstar, ti = in && bin == bstar;
+            ms |= (su ? 1u : 0u) << i;
+            mt |= (ti ? 1u : 0u) << i;
+            ns += su;
+            nt += ti;
+          }
+        }
+        uint32_t tot;
+        const uint32_t pos = block_prefix_excl((ns << 16) | nt, scratch, &tot);
+        uint32_t ps = base_s + (pos >> 16), pt = base_t + (pos & 0xFFFFu);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          if (ms & (1u << i)) {
+            if (ps < (uint32_t)kLCap) PS.sure[ps] = (uint32_t)(b0 + i);
+            ++ps;
+          }
+          if (mt & (1u << i)) {
+            if (pt < (uint32_t)kLCap) {
+              PS.tkey[pt] = keys[i];
+              PS.tidx[pt] = (uint32_t)(b0 + i);
+            }
+            ++pt;
+          }
+        }
+        base_s += tot >> 16;
+        base_t += tot & 0xFFFFu;
+      }
+    }
+    if (tid == 0) {
+      PS.n_sure = base_s;
+      PS.n_tie = base_t;
+      PS.overflow = (base_s > (uint32_t)kLCap || base_t > (uint32_t)kLCap) ? 1u : 0u;
+    }
+  }
+  cl.sync();
+
+  // ---- P3: resolve the selection; every CTA knows the whole chosen set:
+  // list q (CTA q's sure list, or its fallback list) and the chosen ties.
+  uint32_t n_ch = 0;  // chosen ties (ascending in PS.chtie)
+  const uint32_t* glist_base = p.glists + (size_t)seg * C * p.slice;
+  if (select) {
+    if (r == 0) {  // the scan's histogram is consumed: clear it for the next scan
+      uint32_t* hg = p.hist + (size_t)seg * kScanHistBins;
+      for (int i = 4 * tid; i < kScanHistBins; i += 4 * kFinThreads)
+        *reinterpret_cast<uint4*>(hg + i) = make_uint4(0u, 0u, 0u, 0u);
+    }
+    __shared__ uint32_t s_tie[kFinMaxC], s_ovf[kFinMaxC];
+    if (tid < C) {
+      const FinPersist* o = cl.map_shared_rank(&PS, tid);
+      s_cnt[tid] = o->n_sure;
+      s_tie[tid] = o->n_tie;
+      s_ovf[tid] = o->overflow;
+    }
+    __syncthreads();
+    if (tid == 0) {
+      uint32_t ps = 0, pt = 0, ovf = 0;
+      for (int q = 0; q < C; ++q) {
+        s_pre[q] = ps;
+        s_tpre[q] = pt;
+        ps += s_cnt[q];
+        pt += s_tie[q];
+        ovf |= s_ovf[q];
+      }
+      s_pre[C] = ps;
+      s_tpre[C] = pt;
+      // the ties must hold the k-th key: 1 <= k - (keys above b*) <= ties
+      const bool consistent = ps < (uint32_t)k && (uint32_t)k - ps <= pt;
+      s_mode = (!hist_ok || ovf || pt > (uint32_t)kTCap || !consistent) ? 1 : 0;
+    }
+    __syncthreads();
+    if (s_mode == 0) {
+      for (int q = 0; q < C; ++q) {
+        const FinPersist* o = cl.map_shared_rank(&PS, q);
+        const uint32_t n = s_tpre[q + 1] - s_tpre[q];
+        for (uint32_t i = tid; i < n; i += kFinThreads) {
+          SS.akey[s_tpre[q] + i] = o->tkey[i];
+          SS.aidx[s_tpre[q] + i] = o->tidx[i];
         }
       }
-    }
-  }
-  cl.sync();
-
-  // ---- P1b: CTA 0 sums the histograms (all remote loads issued first) and finds b*
-  if (select && r == 0) {
-    uint4 hv[kFinMaxC][2];
-#pragma unroll
-    for (int q = 0; q < kFinMaxC; ++q) {
-      if (q < C) {
-        const uint4* ph = reinterpret_cast<const uint4*>(cl.map_shared_rank(hist, q)) + 2 * tid;
-        hv[q][0] = ph[0];
-        hv[q][1] = ph[1];
-      }
-    }
-    uint32_t tot[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-#pragma unroll
-    for (int q = 0; q < kFinMaxC; ++q) {
-      if (q < C) {
-        tot[0] += hv[q][0].x;
-        tot[1] += hv[q][0].y;
-        tot[2] += hv[q][0].z;
-        tot[3] += hv[q][0].w;
-        tot[4] += hv[q][1].x;
-        tot[5] += hv[q][1].y;
-        tot[6] += hv[q][1].z;
-        tot[7] += hv[q][1].w;
-      }
-    }
-    __syncthreads();
-    reinterpret_cast<uint4*>(hist)[2 * tid] = make_uint4(tot[0], tot[1], tot[2], tot[3]);
-    reinterpret_cast<uint4*>(hist)[2 * tid + 1] = make_uint4(tot[4], tot[5], tot[6], tot[7]);
-    if (tid == 0) {
-      s_bin = 0;
-      s_above = 0;
-    }
-    __syncthreads();
-    find_from_top(hist, kHistBins, (uint32_t)k, scratch, &s_bin, &s_above);
-    if (tid == 0) {
-      s_bstar = (uint32_t)s_bin;
-      s_babove = s_above;
-    }
-  }
-  cl.sync();
-
-  // ---- P2: index-ordered list of this slice's keys with bin >= b*
-  if (select) {
-    const uint32_t bstar = *cl.map_shared_rank(&s_bstar, 0);
-    uint2* lst = lists + (size_t)r * fp.slice;
-    uint32_t base_out = 0;
-    for (int t0 = lo; t0 < hi; t0 += 16 * kFinThreads) {
-      const int b0 = t0 + 16 * tid;
-      float4 v[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-        v[u] = b0 + 4 * u < hi ? *reinterpret_cast<const float4*>(S + b0 + 4 * u)
-                               : make_float4(0.f, 0.f, 0.f, 0.f);
-      uint32_t keys[16];
-      uint32_t mask = 0, n = 0;
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const float vals[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int i = 4 * u + e;
-          keys[i] = float_key(vals[e]);
-          const bool in = (b0 + i < hi) && (keys[i] >> 21) >= bstar;
-          mask |= (in ? 1u : 0u) << i;
-          n += in ? 1u : 0u;
+      __syncthreads();
+      n_ch = (uint32_t)k - s_pre[C];
+      const uint32_t T = s_tpre[C];
+      if (T <= (uint32_t)kFinThreads) {
+        // direct ranking: entry i is chosen iff fewer than n_ch entries come
+        // before it in (key descending, index ascending) order
+        uint32_t chosen = 0, my_idx = 0;
+        if ((uint32_t)tid < T) {
+          const uint32_t key = SS.akey[tid];
+          my_idx = SS.aidx[tid];
+          uint32_t rank = 0;
+#pragma unroll 4
+          for (uint32_t j = 0; j < T; ++j) {
+            const uint32_t k2 = SS.akey[j];
+            rank += (k2 > key || (k2 == key && SS.aidx[j] < my_idx)) ? 1u : 0u;
+          }
+          chosen = rank < n_ch ? 1u : 0u;
         }
-      }
-      uint32_t total;
-      uint32_t pos = base_out + block_prefix_excl(n, scratch, &total);
-#pragma unroll
-      for (int i = 0; i < 16; ++i)
-        if (mask & (1u << i)) lst[pos++] = make_uint2(keys[i], (uint32_t)(b0 + i));
-      base_out += total;
-    }
-    if (tid == 0) s_count = base_out;
-  }
-  cl.sync();
-
-  // ---- P3: CTA 0 selects the k tokens
-  if (r == 0) {
-    int32_t* out = fp.idx_out + (size_t)seg * k;
-    if (!select) {
-      for (int i = tid; i < k; i += kFinThreads) {
-        out[i] = i < nq ? i : -1;
-        if (i < keff) chosen[i] = i;
+        uint32_t tot;
+        const uint32_t pos = block_prefix_excl(chosen, scratch, &tot);
+        if (chosen) PS.chtie[pos] = my_idx;  // entries are in index order
+        __syncthreads();
+      } else {
+        refine_ties(SS.akey, SS.aidx, T, n_ch, SS.hist, PS.chtie, scratch, &s_bin, &s_above,
+                    &s_tot);
       }
     } else {
-      if (tid < 32) {
-        const uint32_t cnt = tid < C ? *cl.map_shared_rank(&s_count, tid) : 0u;
-        uint32_t x = cnt;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const uint32_t y = __shfl_up_sync(kAll, x, o);
-          if (tid >= o) x += y;
-        }
-        if (tid < C) s_off[tid] = x - cnt;
-        if (tid == C - 1) s_off[C] = x;
-      }
-      __syncthreads();
-      const uint32_t total = s_off[C];
-      const uint32_t bstar = s_bstar;
-      const uint32_t rr = (uint32_t)k - s_babove;  // keys still to take from bin b*
-      const int slice = fp.slice;
-      const int nC = C;
-      auto in_place = [&](uint32_t j) -> uint2 {
-        int q = 0;
-        while (q + 1 < nC && s_off[q + 1] <= j) ++q;
-        return lists[(size_t)q * slice + (j - s_off[q])];
-      };
-      if (total <= (uint32_t)kFinStage) {
-        for (uint32_t j = tid; j < total; j += kFinThreads) stage[j] = in_place(j);
-        __syncthreads();
-        auto staged = [&](uint32_t j) -> uint2 { return stage[j]; };
-        select_ordered(staged, total, bstar, rr, k, out, chosen, hist, scratch, &s_bin, &s_above);
-      } else {
-        select_ordered(in_place, total, bstar, rr, k, out, chosen, hist, scratch, &s_bin,
-                       &s_above);
-      }
+      const uint32_t n =
+          select_full(p.scores + (size_t)seg * p.capacity, nq, k, lo, hi, SS.hist,
+                      const_cast<uint32_t*>(glist_base) + (size_t)r * p.slice, scratch, &s_bin,
+                      &s_above, &s_tot);
+      if (tid == 0) PS.n_gl = n;
+      __threadfence();
     }
   }
-  cl.sync();
-
-  // ---- P4: correction of this CTA's share of the exact set
-  {
-    const int32_t* chosen0 = cl.map_shared_rank(chosen, 0);
-    // every chosen token of the share is known now: pull its rows and record
-    // pieces into L2 before the batches read them
-    for (int i = tid; i < (min(e1, keff) - e0) * kPrefParts; i += kFinThreads)
-      prefetch_token(p, seg, chosen0[e0 + i / kPrefParts], i % kPrefParts);
-    const CorrectSmem CS = correct_smem_carve(reinterpret_cast<float*>(U), G);
-    correct_load_q<G>(p, seg, CS.qs);
-    for (int i = tid; i < 2 * G * kPartStride; i += kFinThreads) run[i] = 0.f;
+  const int mode = select ? s_mode : 0;
+  if (select && mode == 1) {
+    cl.sync();  // the fallback lists and counts are complete
+    if (tid < C) s_cnt[tid] = cl.map_shared_rank(&PS, tid)->n_gl;
     __syncthreads();
-    if (tid < 2 * G) run[tid * kPartStride] = -INFINITY;
-    for (int eb = e0; eb < e1; eb += kMergeChunk) {
-      __syncthreads();
-      if (tid < kMergeChunk) {
-        const int e = eb + tid;
-        int t = -1;
-        if (e < e1) t = e < keff ? chosen0[e] : ((1 << 30) | (e - keff));
-        s_tok[tid] = t;
+    if (tid == 0) {
+      uint32_t ps = 0;
+      for (int q = 0; q < C; ++q) {
+        s_pre[q] = ps;
+        ps += s_cnt[q];
       }
-      __syncthreads();
-      correct_batch<G>(p, seg, s_tok, CS, bat);
-      __syncthreads();
-      // fold the batch partial into the running one
-      const int c = tid & (kD - 1), part = tid >> 7;
-      float mv[G], lv[G];
-#pragma unroll
-      for (int j = 0; j < G; ++j) {
-        const float* ro = run + (part * G + j) * kPartStride;
-        const float* bo = bat + (part * G + j) * kPartStride;
-        const float m1 = ro[0], l1 = ro[1], m2 = bo[0], l2 = bo[1];
-        const float mn = fmaxf(m1, m2);
-        const float s1 = l1 > 0.f ? exp2f(m1 - mn) : 0.f;
-        const float s2 = l2 > 0.f ? exp2f(m2 - mn) : 0.f;
-        mv[j] = (l1 > 0.f || l2 > 0.f) ? mn : -INFINITY;
-        lv[j] = l1 * s1 + l2 * s2;
-        run[(part * G + j) * kPartStride + 4 + c] = ro[4 + c] * s1 + bo[4 + c] * s2;
-      }
-      __syncthreads();
-      if (c == 0) {
-#pragma unroll
-        for (int j = 0; j < G; ++j) {
-          run[(part * G + j) * kPartStride] = mv[j];
-          run[(part * G + j) * kPartStride + 1] = lv[j];
-        }
-      }
+      s_pre[C] = ps;
     }
+    __syncthreads();
   }
-  cl.sync();
+  auto list_of = [&](int q) -> const uint32_t* {
+    return mode == 1 ? glist_base + (size_t)q * p.slice : cl.map_shared_rank(PS.sure, q);
+  };
 
-  // ---- P5a: each CTA merges its share of the scan slots for every head into
-  // sp[G][kPartStride] (one tiled pass with all loads of a tile in flight)
-  float* sp = bat;  // the batch buffer is free now: [G][kPartStride] (first half)
+  // ---- idx output: this CTA's chosen indices, ascending, at its offset
+  if (select) {
+    if (tid <= C) {
+      const uint32_t b0 = (uint32_t)min(nq, tid * p.slice);
+      s_chq[tid] = lower_bound_u32(PS.chtie, n_ch, b0);
+    }
+    __syncthreads();
+    const uint32_t c0 = s_chq[r], c1 = s_chq[r + 1];
+    const uint32_t off = s_pre[r] + c0;  // earlier slices: their lists and chosen ties
+    const uint32_t* Lr = list_of(r);
+    const uint32_t nr = s_cnt[r];
+    int32_t* out = p.idx_out + (size_t)seg * k;
+    for (uint32_t i = tid; i < nr; i += kFinThreads) {
+      const uint32_t v = Lr[i];
+      const uint32_t pos = off + i + lower_bound_u32(PS.chtie + c0, c1 - c0, v);
+      if (pos < (uint32_t)k) out[pos] = (int32_t)v;
+    }
+    for (uint32_t j = c0 + tid; j < c1; j += kFinThreads) {
+      const uint32_t v = PS.chtie[j];
+      const uint32_t pos = off + (j - c0) + lower_bound_u32(Lr, nr, v);
+      if (pos < (uint32_t)k) out[pos] = (int32_t)v;
+    }
+  } else if (SELECT && r == 0) {
+    int32_t* out = p.idx_out + (size_t)seg * k;
+    for (int i = tid; i < k; i += kFinThreads) out[i] = i < nq ? i : -1;
+  }
+  if (!SELECT && r == 0) {  // nothing reads the scan's histogram here: clear it
+    uint32_t* hg = p.hist + (size_t)seg * kScanHistBins;
+    for (int i = 4 * tid; i < kScanHistBins; i += 4 * kFinThreads)
+      *reinterpret_cast<uint4*>(hg + i) = make_uint4(0u, 0u, 0u, 0u);
+  }
+
+  // ---- P4: correction of an even share of the chosen set: the token list
+  // first (compacted, in shared memory), then a warp per token
   {
-    float* tile = reinterpret_cast<float*>(U);
-    constexpr int kTile = (int)(((size_t)correct_smem_floats<G>()) / kPartStride);  // rows per tile
-    const int c = tid & (kD - 1);
-    float mrun[G], lrun[G], arun[G];
-#pragma unroll
-    for (int j = 0; j < G; ++j) {
-      mrun[j] = -INFINITY;
-      lrun[j] = 0.f;
-      arun[j] = 0.f;
-    }
-    for (int t0 = s0 * G; t0 < s1 * G; t0 += kTile) {
-      const int nr = min(kTile, s1 * G - t0);
-      __syncthreads();
-      for (int i = tid; i < nr * (kPartStride / 4); i += kFinThreads) {
-        const int row = i / (kPartStride / 4), v = i % (kPartStride / 4);
-        const int gr = t0 + row;  // row = slot * G + head
-        reinterpret_cast<float4*>(tile + row * kPartStride)[v] = reinterpret_cast<const float4*>(
-            p.scan_part + ((size_t)(w0 + gr / G + seg) * G + gr % G) * kPartStride)[v];
-      }
-      __syncthreads();
-      if (tid < kD) {
-#pragma unroll
-        for (int j = 0; j < G; ++j) {
-          float tm = mrun[j];
-          for (int row = (j - t0 % G + G) % G; row < nr; row += G)
-            if (tile[row * kPartStride + 1] > 0.f) tm = fmaxf(tm, tile[row * kPartStride]);
-          const float sc0 = (lrun[j] > 0.f) ? exp2f(mrun[j] - tm) : 0.f;
-          float l = lrun[j] * sc0, a = arun[j] * sc0;
-          for (int row = (j - t0 % G + G) % G; row < nr; row += G) {
-            const float lb = tile[row * kPartStride + 1];
-            if (lb > 0.f) {
-              const float sc = exp2f(tile[row * kPartStride] - tm);
-              l = fmaf(lb, sc, l);
-              a = fmaf(tile[row * kPartStride + 4 + c], sc, a);
-            }
+    const int n_x = select ? k : (SELECT ? nq : k);  // positions of the chosen sequence
+    const int per = (n_x + C - 1) / C;
+    const int x0 = min(n_x, r * per), x1 = min(n_x, x0 + per);
+#pragma unroll 1
+    for (int xr = x0; xr < x1; xr += kTokCap) {
+    const int xe = min(x1, xr + kTokCap);
+    uint32_t base = 0;
+#pragma unroll 1
+    for (int xb = xr; xb < xe; xb += kFinThreads) {
+      const int j = xb + tid;
+      int t = -1;
+      if (j < xe) {
+        if (select) {
+          if ((uint32_t)j < s_pre[C]) {
+            int q = 0;
+            while (q + 1 < C && s_pre[q + 1] <= (uint32_t)j) ++q;
+            t = (int)list_of(q)[j - s_pre[q]];
+          } else {
+            t = (int)PS.chtie[j - s_pre[C]];
           }
-          mrun[j] = tm;
-          lrun[j] = l;
-          arun[j] = a;
+        } else if (SELECT) {
+          t = j;
+        } else {
+          t = p.idx_in[(size_t)seg * k + j];
+          if (t < -1 || t >= nq) {
+            set_flag(p.flag, JFA_DEVERR_BAD_INDEX);
+            t = -1;
+          }
         }
       }
+      uint32_t tot;
+      const uint32_t pos = base + block_prefix_excl(t >= 0 ? 1u : 0u, scratch, &tot);
+      if (t >= 0) FC.tok[pos] = t;
+      base += tot;
     }
-    if (tid < kD) {
+    __syncthreads();
+    const int n = (int)base;
+    const int n_w = n > warp ? (n - warp + kFinWarps - 1) / kFinWarps : 0;
+    const int32_t* tl = FC.tok;
+    auto chosen_at = [&](int i) { return tl[warp + kFinWarps * i]; };
+    warp_correct<G>(p, seg, chosen_at, n_w, FC.st[warp], P, q2, warp, lane);
+    __syncthreads();
+    }
+    // combine the warps' partials into P.run: thread (channel, half) merges
+    // heads half, half + 2, ...
+    const int c = tid & (kD - 1), half = tid >> 7;
+    for (int j = half; j < G; j += 2) {
+      float mx = -INFINITY;
 #pragma unroll
-      for (int j = 0; j < G; ++j) {
-        sp[j * kPartStride + 4 + c] = arun[j];
+      for (int w = 0; w < kFinWarps; ++w) mx = fmaxf(mx, P.wp[w][j][0]);
+      float l = 0.f, acc = 0.f;
+#pragma unroll
+      for (int w = 0; w < kFinWarps; ++w) {
+        const float mw = P.wp[w][j][0];
+        const float f = mw == -INFINITY ? 0.f : exp2f(mw - mx);  // empty partials add nothing
+        l = fmaf(P.wp[w][j][1], f, l);
+        acc = fmaf(P.wp[w][j][4 + c], f, acc);
+      }
+      P.run[j][4 + c] = acc;
+      if (c == 0) {
+        P.run[j][0] = mx;
+        P.run[j][1] = l;
+      }
+    }
+  }
+
+  // ---- P5a: this CTA's share of the scan's split partials, every head
+  {
+    long long w0 = 0, w1 = -1;
+    if (p.ng > 0) {
+      const long long T = p.scan_total, W = p.scan_warps;
+      const long long x0 = (long long)seg * p.ng, x1 = x0 + p.ng - 1;
+      w0 = scan_warp_of(x0, W, T);
+      w1 = scan_warp_of(x1, W, T);
+    }
+    const int ns = (int)(w1 - w0 + 1);
+    const int s0 = (int)((long long)ns * r / C), s1 = (int)((long long)ns * (r + 1) / C);
+    // rows (slot, head) staged in shared memory a tile at a time, every load
+    // of a tile in flight together; thread (channel, half) merges the heads
+    // j = half, half + 2, ... online
+    const int c = tid & (kD - 1), half = tid >> 7;
+    constexpr int kH2 = (G + 1) / 2;
+    float mrun[kH2], lrun[kH2], arun[kH2];
+#pragma unroll
+    for (int i = 0; i < kH2; ++i) {
+      mrun[i] = -INFINITY;
+      lrun[i] = 0.f;
+      arun[i] = 0.f;
+    }
+    float* tile = reinterpret_cast<float*>(U);
+    constexpr int kTR = (int)(sizeof(FinCorr) / (kPartStride * sizeof(float)));
+    constexpr int kV = kPartStride / 4;  // float4 per row
+    const int nrows = (s1 - s0) * G;
+    for (int r0 = 0; r0 < nrows; r0 += kTR) {
+      const int nr = min(kTR, nrows - r0);
+#pragma unroll 4
+      for (int i = tid; i < nr * kV; i += kFinThreads) {
+        const int row = i / kV, v = i % kV;
+        const int gr = r0 + row;
+        const float* src = p.scan_part + ((size_t)(w0 + s0 + gr / G + seg) * G + gr % G) * kPartStride;
+        reinterpret_cast<float4*>(tile + row * kPartStride)[v] = ld16<float4>(src + 4 * v);
+      }
+      __syncthreads();
+#pragma unroll 1
+      for (int row = 0; row < nr; ++row) {
+        const int j = (r0 + row) % G;
+        if ((j & 1) != half) continue;
+        const float* tr = tile + row * kPartStride;
+        const float rl = tr[1];
+        if (rl > 0.f) {
+          const int i = j >> 1;
+          const float mn = fmaxf(mrun[i], tr[0]);
+          const float s0f = lrun[i] > 0.f ? exp2f(mrun[i] - mn) : 0.f;
+          const float s1f = exp2f(tr[0] - mn);
+          lrun[i] = lrun[i] * s0f + rl * s1f;
+          arun[i] = arun[i] * s0f + tr[4 + c] * s1f;
+          mrun[i] = mn;
+        }
+      }
+      __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < kH2; ++i) {
+      const int j = half + 2 * i;
+      if (j < G) {
+        P.sp[j][4 + c] = arun[i];
         if (c == 0) {
-          sp[j * kPartStride] = lrun[j] > 0.f ? mrun[j] : -INFINITY;
-          sp[j * kPartStride + 1] = lrun[j];
+          P.sp[j][0] = lrun[i] > 0.f ? mrun[i] : -INFINITY;
+          P.sp[j][1] = lrun[i];
         }
       }
     }
   }
   cl.sync();
 
-  // ---- P5b: CTA r owns heads j = r, r + C, ...: merge the C scan, exact and
-  // removal partials (remote loads issued together) and write the output row
+  // ---- P5b: CTA r owns heads j = r, r + C, ...: merge the C CTAs' scan
+  // partials (m_a, l_a, a_a) and exact-minus-removed partials (m_c, l_c, a_c),
+  // remote loads issued together, and write
+  //   out = (a_c 2^(m_c-m) + a_a 2^(m_a-m)) / (l_c 2^(m_c-m) + l_a 2^(m_a-m))
   for (int j = r; j < G; j += C) {
     const int c = tid;
     if (c < kD) {
-      float2 hd[kFinMaxC][3];  // (m, l) of scan / exact / removal parts
-      float av[kFinMaxC][3];   // channel c of each
+      float2 hd[kFinMaxC][2];
+      float av[kFinMaxC][2];
 #pragma unroll
       for (int q = 0; q < kFinMaxC; ++q) {
         if (q < C) {
-          const float* spq = cl.map_shared_rank(sp, q) + j * kPartStride;
-          const float* rq = cl.map_shared_rank(run, q);
-          const float* re = rq + (0 * G + j) * kPartStride;
-          const float* rm = rq + (1 * G + j) * kPartStride;
-          hd[q][0] = *reinterpret_cast<const float2*>(spq);
-          hd[q][1] = *reinterpret_cast<const float2*>(re);
-          hd[q][2] = *reinterpret_cast<const float2*>(rm);
-          av[q][0] = spq[4 + c];
-          av[q][1] = re[4 + c];
-          av[q][2] = rm[4 + c];
+          FinParts<G>* o = cl.map_shared_rank(&P, q);
+          hd[q][0] = *reinterpret_cast<const float2*>(&o->sp[j][0]);
+          hd[q][1] = *reinterpret_cast<const float2*>(&o->run[j][0]);
+          av[q][0] = o->sp[j][4 + c];
+          av[q][1] = o->run[j][4 + c];
         }
       }
-      float mk[3] = {-INFINITY, -INFINITY, -INFINITY};
+      float ma = -INFINITY, mc = -INFINITY;
 #pragma unroll
       for (int q = 0; q < kFinMaxC; ++q)
         if (q < C) {
-#pragma unroll
-          for (int t = 0; t < 3; ++t)
-            if (hd[q][t].y > 0.f) mk[t] = fmaxf(mk[t], hd[q][t].x);
+          if (hd[q][0].y > 0.f) ma = fmaxf(ma, hd[q][0].x);
+          mc = fmaxf(mc, hd[q][1].x);
         }
-      float lk[3] = {0.f, 0.f, 0.f}, ak[3] = {0.f, 0.f, 0.f};
+      const float m = fmaxf(ma, mc);
+      float l = 0.f, acc = 0.f;
 #pragma unroll
       for (int q = 0; q < kFinMaxC; ++q)
         if (q < C) {
-#pragma unroll
-          for (int t = 0; t < 3; ++t) {
-            const float sc = hd[q][t].y > 0.f ? exp2f(hd[q][t].x - mk[t]) : 0.f;
-            lk[t] = fmaf(hd[q][t].y, sc, lk[t]);
-            ak[t] = fmaf(av[q][t], sc, ak[t]);
-          }
+          const float fa = hd[q][0].y > 0.f ? exp2f(hd[q][0].x - m) : 0.f;
+          const float fc = hd[q][1].x == -INFINITY ? 0.f : exp2f(hd[q][1].x - m);
+          l = fmaf(hd[q][0].y, fa, fmaf(hd[q][1].y, fc, l));
+          acc = fmaf(av[q][0], fa, fmaf(av[q][1], fc, acc));
         }
-      const float ma = mk[0], la = lk[0], aa = ak[0];
-      const float me = mk[1], le = lk[1], ae = ak[1];
-      const float mr = mk[2], lr = lk[2], ar = ak[2];
-      // remainder = approximate total minus the removed top-k terms (m_a frame)
-      float lrest = la, arest = aa;
-      if (la > 0.f && lr > 0.f) {
-        const float f = exp2f(mr - ma);
-        lrest = la - lr * f;
-        arest = aa - ar * f;
-        if (lrest < 0.f) lrest = 0.f;
-      }
-      float mm = me, wl = 1.f, wa = 0.f;
-      if (la > 0.f) {
-        mm = fmaxf(me, ma);
-        wl = exp2f(me - mm);
-        wa = exp2f(ma - mm);
-      }
-      const int b = seg / p.hkv, h = seg % p.hkv;
-      p.out[((size_t)b * p.H + h * G + j) * kD + c] = (ae * wl + arest * wa) / (le * wl + lrest * wa);
+      p.out[((size_t)bb * p.H + hh * G + j) * kD + c] = acc / l;
     }
   }
   // keep this CTA's shared memory alive until every peer has read it
   cl.sync();
 }
 
-// Largest cluster size (<= 8) whose clusters all fit on the device at once
-// (so the whole grid runs in one wave), using up to about two CTAs per SM.
-template <int G>
+template <int G, bool SEL>
 static int pick_cluster(int n_seg, int num_sms) {
-  constexpr size_t smem = finish_smem_bytes<G>();
+  constexpr size_t smem = fin_smem_bytes<G>();
   int best = 1;
   for (int c = 2; c <= kFinMaxC; c *= 2) {
     if ((long long)n_seg * c > 2LL * num_sms) break;
@@ -540,7 +947,7 @@ static int pick_cluster(int n_seg, int num_sms) {
     cfg.attrs = at;
     cfg.numAttrs = 1;
     int n_active = 0;
-    if (cudaOccupancyMaxActiveClusters(&n_active, finish_kernel<G>, &cfg) != cudaSuccess) {
+    if (cudaOccupancyMaxActiveClusters(&n_active, finish_kernel<G, SEL>, &cfg) != cudaSuccess) {
       cudaGetLastError();
       break;
     }
@@ -550,15 +957,15 @@ static int pick_cluster(int n_seg, int num_sms) {
   return best;
 }
 
-template <int G>
+template <int G, bool SEL>
 static int launch_finish_t(FinishParams fp, int n_seg, cudaStream_t st) {
-  constexpr size_t smem = finish_smem_bytes<G>();
+  constexpr size_t smem = fin_smem_bytes<G>();
   static bool configured[64] = {false};
   static int memo_seg[64][8] = {{0}}, memo_c[64][8] = {{0}};  // cluster size per (device, n_seg)
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !configured[dev]) {
-    if (cudaFuncSetAttribute(finish_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(finish_kernel<G, SEL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem) != cudaSuccess)
       return JFA_ERR_CUDA;
     configured[dev] = true;
@@ -569,7 +976,7 @@ static int launch_finish_t(FinishParams fp, int n_seg, cudaStream_t st) {
       if (memo_seg[dev][i] == n_seg) C = memo_c[dev][i];
   }
   if (C == 0) {
-    C = pick_cluster<G>(n_seg, num_sms_current());
+    C = pick_cluster<G, SEL>(n_seg, num_sms_current());
     if (dev >= 0 && dev < 64) {
       for (int i = 0; i < 8; ++i)
         if (memo_seg[dev][i] == 0) {
@@ -579,7 +986,7 @@ static int launch_finish_t(FinishParams fp, int n_seg, cudaStream_t st) {
         }
     }
   }
-  const int nq = fp.m.nq;
+  const int nq = fp.nq;
   fp.slice = nq > 0 ? ((nq + C - 1) / C + 63) / 64 * 64 : 64;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(n_seg * C);
@@ -595,57 +1002,63 @@ static int launch_finish_t(FinishParams fp, int n_seg, cudaStream_t st) {
   at[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = at;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, finish_kernel<G>, fp) == cudaSuccess ? JFA_OK : JFA_ERR_CUDA;
+  return cudaLaunchKernelEx(&cfg, finish_kernel<G, SEL>, fp) == cudaSuccess ? JFA_OK : JFA_ERR_CUDA;
+}
+
+template <bool SEL>
+static int launch_finish_g(const FinishParams& fp, int G, int n_seg, cudaStream_t st) {
+  switch (G) {
+    case 1: return launch_finish_t<1, SEL>(fp, n_seg, st);
+    case 2: return launch_finish_t<2, SEL>(fp, n_seg, st);
+    case 3: return launch_finish_t<3, SEL>(fp, n_seg, st);
+    case 4: return launch_finish_t<4, SEL>(fp, n_seg, st);
+    case 5: return launch_finish_t<5, SEL>(fp, n_seg, st);
+    case 6: return launch_finish_t<6, SEL>(fp, n_seg, st);
+    case 7: return launch_finish_t<7, SEL>(fp, n_seg, st);
+    default: return launch_finish_t<8, SEL>(fp, n_seg, st);
+  }
 }
 
 int launch_finish(const jfa_geom& g, const jfa_cache& c, const uint16_t* q, float scale, int k,
-                  int32_t* idx, const uint16_t* k_exact, const uint16_t* v_exact, uint8_t* ws,
-                  const jfa_workspace_layout& L, float* out, cudaStream_t st) {
+                  int32_t* idx_out, const int32_t* idx_in, const uint16_t* k_exact,
+                  const uint16_t* v_exact, uint8_t* ws, const jfa_workspace_layout& L, float* out,
+                  cudaStream_t st) {
   const int n_seg = g.batch * g.num_kv_heads;
   const int nq = split_point(g.n_ctx);
   FinishParams fp;
-  MergeParams& p = fp.m;
-  p.groups = static_cast<const uint8_t*>(c.groups);
-  p.tail_k = c.tail_k;
-  p.tail_v = c.tail_v;
-  p.k_exact = k_exact;
-  p.v_exact = v_exact;
-  p.q = q;
-  p.idx = idx;
-  p.scan_part = reinterpret_cast<const float*>(ws + L.off_partials);
-  p.chunk_part = nullptr;
-  p.out = out;
-  p.flag = reinterpret_cast<uint32_t*>(ws + L.off_flag);
-  p.k = k;
-  p.tail = g.n_ctx - nq;
-  p.nq = nq;
-  p.capacity = g.capacity;
-  p.ng_cap = g.capacity / kKG;
-  p.hkv = g.num_kv_heads;
-  p.G = g.num_heads / g.num_kv_heads;
-  p.H = g.num_heads;
-  p.n_chunks = 0;
-  p.key_bits = g.key_bits;
-  p.val_bits = g.val_bits;
-  p.rec_bytes = record_bytes(g.key_bits, g.val_bits);
-  ScanPlan plan = scan_plan(g, num_sms_current());
-  p.scan_total = plan.total_groups;
-  p.scan_warps = plan.n_warps;
-  p.ng = plan.ng;
-  p.kappa = scale * 1.4426950408889634f;
+  fp.groups = static_cast<const uint8_t*>(c.groups);
+  fp.tail_k = c.tail_k;
+  fp.tail_v = c.tail_v;
+  fp.k_exact = k_exact;
+  fp.v_exact = v_exact;
+  fp.q = q;
   fp.scores = reinterpret_cast<const float*>(ws + L.off_scores);
-  fp.idx_out = idx;
-  fp.lists = reinterpret_cast<uint2*>(ws + L.off_cand);
-  switch (p.G) {
-    case 1: return launch_finish_t<1>(fp, n_seg, st);
-    case 2: return launch_finish_t<2>(fp, n_seg, st);
-    case 3: return launch_finish_t<3>(fp, n_seg, st);
-    case 4: return launch_finish_t<4>(fp, n_seg, st);
-    case 5: return launch_finish_t<5>(fp, n_seg, st);
-    case 6: return launch_finish_t<6>(fp, n_seg, st);
-    case 7: return launch_finish_t<7>(fp, n_seg, st);
-    default: return launch_finish_t<8>(fp, n_seg, st);
-  }
+  fp.scan_part = reinterpret_cast<const float*>(ws + L.off_partials);
+  fp.m_used = reinterpret_cast<const float*>(ws + L.off_mused);
+  fp.hist = reinterpret_cast<uint32_t*>(ws + L.off_scan_hist);
+  fp.glists = reinterpret_cast<uint32_t*>(ws + L.off_cand);
+  fp.idx_in = idx_in;
+  fp.idx_out = idx_out;
+  fp.out = out;
+  fp.flag = reinterpret_cast<uint32_t*>(ws + L.off_flag);
+  fp.k = k;
+  fp.nq = nq;
+  fp.tail = g.n_ctx - nq;
+  fp.capacity = g.capacity;
+  fp.ng_cap = g.capacity / kKG;
+  fp.hkv = g.num_kv_heads;
+  fp.H = g.num_heads;
+  fp.key_bits = g.key_bits;
+  fp.val_bits = g.val_bits;
+  fp.rec_bytes = record_bytes(g.key_bits, g.val_bits);
+  const ScanPlan plan = scan_plan(g, num_sms_current());
+  fp.scan_total = plan.total_groups;
+  fp.scan_warps = plan.n_warps;
+  fp.ng = plan.ng;
+  fp.kappa = scale * 1.4426950408889634f;
+  fp.slice = 64;
+  const int G = g.num_heads / g.num_kv_heads;
+  return idx_in ? launch_finish_g<false>(fp, G, n_seg, st) : launch_finish_g<true>(fp, G, n_seg, st);
 }
 
 }  // namespace jfa

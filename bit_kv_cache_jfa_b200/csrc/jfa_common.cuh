@@ -20,11 +20,11 @@ constexpr int kVG = JFA_VAL_GROUP;       // 32 channels per value group
 constexpr int kTail = JFA_TAIL_MAX;      // 64
 constexpr int kMaxG = JFA_MAX_GQA;       // 8
 constexpr int kPartStride = 132;         // floats per (slot, head): m, l, pad2, acc[128]
-constexpr int kScanWarps = 8;            // warps per scan CTA
-constexpr int kMaxScanWarps = 2048;      // cap on scan warps (partial slots)
+constexpr int kMaxScanWarps = 4096;      // cap on scan warps (partial slots)
+constexpr int kScanHistBits = 13;        // selection-score histogram of the scan: top 13 key bits
+constexpr int kScanHistBins = 1 << kScanHistBits;
 constexpr int kHistBins = 2048;          // top-k first-level histogram (11 key bits)
 constexpr int kCtrStride = 8;            // top-k counters per segment: [0] scan warps done, [2] b*, [3] keys above b*
-constexpr int kMergeChunk = 32;          // tokens per correct/merge CTA
 
 // ---------------------------------------------------------------------------
 // Packed group record: 64 tokens of one (sequence, KV head).
@@ -41,6 +41,14 @@ JFA_HD int off_kc() { return 512; }
 JFA_HD int off_vs(int kb) { return 512 + kc_bytes(kb); }
 JFA_HD int off_vc(int kb) { return 512 + kc_bytes(kb) + 1024; }
 JFA_HD int record_bytes(int kb, int vb) { return off_vc(kb) + vc_bytes(vb); }
+
+// Warps per scan CTA: each warp owns a two-record shared-memory ring and the
+// CTA takes a whole SM (227 KB of shared memory), at most 16 warps.
+constexpr int scan_cta_warps(int kb, int vb) {
+  return ((227 * 1024 - 1024) / (2 * (512 + 1024 * kb + 1024 + 1024 * vb))) > 16
+             ? 16
+             : ((227 * 1024 - 1024) / (2 * (512 + 1024 * kb + 1024 + 1024 * vb)));
+}
 
 struct BitLoc {
   int byte;  // byte offset of the 32-bit word inside its section

@@ -56,13 +56,12 @@ int launch_scores(const jfa_geom& g, const jfa_cache& c, const uint16_t* q, floa
                   uint8_t* ws, const jfa_workspace_layout& L, cudaStream_t st);
 int launch_topk(const jfa_geom& g, int k, uint8_t* ws, const jfa_workspace_layout& L,
                 int32_t* idx, cudaStream_t st);
-int launch_correct_merge(const jfa_geom& g, const jfa_cache& c, const uint16_t* q, float scale,
-                         const int32_t* idx, int k, const uint16_t* k_exact,
-                         const uint16_t* v_exact, int exact_on_host, uint8_t* ws,
-                         const jfa_workspace_layout& L, float* out, cudaStream_t st);
 int count_topk_launches(const jfa_geom& g, int k);
+// Selection (idx_in == nullptr: top-k written to idx_out) or a given index
+// set (idx_in), then correction and merge: one cluster per segment.
 int launch_finish(const jfa_geom& g, const jfa_cache& c, const uint16_t* q, float scale, int k,
-                  int32_t* idx, const uint16_t* k_exact, const uint16_t* v_exact, uint8_t* ws,
-                  const jfa_workspace_layout& L, float* out, cudaStream_t st);
+                  int32_t* idx_out, const int32_t* idx_in, const uint16_t* k_exact,
+                  const uint16_t* v_exact, uint8_t* ws, const jfa_workspace_layout& L, float* out,
+                  cudaStream_t st);
 
 }  // namespace jfa

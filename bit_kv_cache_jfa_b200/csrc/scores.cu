@@ -1,31 +1,32 @@
 // scores.cu — jfa_decode_scores: the approximate scan over packed keys and
 // values (Jet-QSparse abstract: a dense scan scores the full key history).
 //
-// Per 64-token group g of a (sequence, KV head) and query head h:
+// Per 64-token group g of a (sequence, KV head) and query head h the logit
 //   s_hat[h][t] = scale * ( sum_c (q[h][c]*s[g][c]) * k'[t][c] + sum_c q[h][c]*m[g][c] )
-// which is HACK's affine identity (HACK review, Eq. (4)) with an
-// unquantized query: integer codes times a scaled query, plus a per-group
-// bias.  The integer product runs on mma.sync.m16n8k16 (fp16 in, fp32 acc):
-// rows 0-7 of A hold fp16(q*s) ("hi") and rows 8-15 the rounding remainder
-// ("lo") of the G <= 8 query heads, so hi+lo carries q*s exactly; the codes
-// are exact small integers in fp16.  Columns are tokens.
+// is HACK's affine identity (HACK review, Eq. (4)) with an unquantized query;
+// jfa_approx.cuh holds that arithmetic (mma.sync with q*s as an exact fp16
+// pair, the bias as an MMA chain).
 //
 // The same pass accumulates, per query head, the online-softmax partial over
 // the dequantized values v_hat = s_v * v' + m_v (v' codes exact in fp16):
 //   sum_t p_t v_hat[t][c] = sum_t (p_t s_v[t][j]) v'[t][c] + sum_t p_t m_v[t][j]
 // as an MMA with A = value codes (rows = channels, columns = tokens) and
-// B = p * s_v (columns = heads), plus a small MMA whose A rows are the value
-// zeros of the four channel groups and a row of ones (giving sum p).  Both
-// B operands enter as an fp16 pair (rounded value, rounding remainder) in two
-// MMAs, so each token's weight carries ~22 bits: the correction step later
-// subtracts the top-k tokens' terms, and a plain fp16 weight would leave a
-// 2^-12 residue of the largest weights in the output.
+// B = fp16(p) * s_v (columns = heads), plus a small MMA whose A rows are the
+// value zeros of the four channel groups and a row of ones (giving sum p).
+// The running maximum each group's weights were taken against is stored
+// (m_used), so the correction step recomputes exactly these fp16 weights for
+// the top-k tokens and removes their terms without a rounding residue.
 //
-// Work split: W warps (8 per CTA, one CTA per SM) take balanced contiguous
+// Also written per token: the selection score S_t = max over the G heads
+// (natural-log units), and a per-segment histogram of its top 13 key bits
+// (the first radix level of the top-k selection).
+//
+// Work split: W warps (NW per CTA, one CTA per SM) take balanced contiguous
 // ranges of the flattened (segment, group) list.  Each warp streams its
-// records through a private two- or three-stage shared-memory ring filled by
+// records through a private two-stage shared-memory ring filled by
 // cp.async.bulk (one bulk copy per 6.5-9.5 KB record, completion on an
 // mbarrier) and writes one softmax partial per segment it touched.
+#include "jfa_approx.cuh"
 #include "jfa_internal.cuh"
 
 namespace jfa {
@@ -35,6 +36,8 @@ struct ScanParams {
   const uint16_t* q;
   float* scores;
   float* partials;
+  float* m_used;    // [n_seg][ng_cap][8]
+  uint32_t* hist;   // [n_seg][kScanHistBins]
   uint32_t* flag;
   long long total;  // n_seg * ng
   int ng, ng_cap, capacity;
@@ -56,15 +59,17 @@ constexpr unsigned kFull = 0xFFFFFFFFu;
 template <int KB, int VB>
 struct ScanCfg {
   static constexpr int REC = 512 + 1024 * KB + 1024 + 1024 * VB;
-  // three ring stages per warp when they fit in shared memory, else two
-  static constexpr int STAGES = (kScanWarps * 3 * REC + 1024 <= 227 * 1024) ? 3 : 2;
-  static constexpr int SMEM = kScanWarps * STAGES * REC + kScanWarps * STAGES * 8;
+  static constexpr int NW = scan_cta_warps(KB, VB);
+  static constexpr int STAGES = 2;
+  static constexpr int SMEM = NW * STAGES * REC + NW * STAGES * 8;
+  static_assert(SMEM <= 227 * 1024, "scan ring exceeds shared memory");
 };
 
 template <int KB, int VB>
-__global__ void __launch_bounds__(kScanWarps * 32, 1) scan_kernel(const ScanParams p) {
+__global__ void __launch_bounds__(ScanCfg<KB, VB>::NW * 32, 1) scan_kernel(const ScanParams p) {
   constexpr int REC = ScanCfg<KB, VB>::REC;
   constexpr int S = ScanCfg<KB, VB>::STAGES;
+  constexpr int NW = ScanCfg<KB, VB>::NW;
   constexpr int OFF_KC = 512;
   constexpr int OFF_VS = 512 + 1024 * KB;
   constexpr int OFF_VC = OFF_VS + 1024;
@@ -73,14 +78,14 @@ __global__ void __launch_bounds__(kScanWarps * 32, 1) scan_kernel(const ScanPara
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gid = lane >> 2, tig = lane & 3;
   pdl_wait();
-  const long long wg = (long long)blockIdx.x * kScanWarps + warp;
+  const long long wg = (long long)blockIdx.x * NW + warp;
   if (wg >= p.n_warps) return;
   const long long W = p.n_warps, T = p.total;
   const long long g0 = scan_range_begin(wg, W, T), g1 = scan_range_begin(wg + 1, W, T);
   if (g0 >= g1) return;
 
   uint8_t* ring = smem + (size_t)warp * S * REC;
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + (size_t)kScanWarps * S * REC) + warp * S;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + (size_t)NW * S * REC) + warp * S;
   const uint64_t pol = policy_evict_first();
   if (lane == 0) {
 #pragma unroll
@@ -111,7 +116,6 @@ __global__ void __launch_bounds__(kScanWarps * 32, 1) scan_kernel(const ScanPara
   float dz[4];
   float m_run = 0.f;
   uint32_t q2[16];
-  float qf[32];
   long long cur = -1;
 
   auto reset = [&](long long seg) {
@@ -120,16 +124,7 @@ __global__ void __launch_bounds__(kScanWarps * 32, 1) scan_kernel(const ScanPara
     dz[0] = dz[1] = dz[2] = dz[3] = 0.f;
     m_run = head_ok ? -INFINITY : 0.f;
     const int b = (int)(seg / p.hkv), h = (int)(seg % p.hkv);
-    const uint16_t* qrow = p.q + ((size_t)b * p.H + (size_t)h * p.G + (head_ok ? gid : 0)) * kD;
-#pragma unroll
-    for (int pp = 0; pp < 16; ++pp) {
-      const int c = 16 * (pp >> 1) + 2 * tig + 8 * (pp & 1);
-      uint32_t w = head_ok ? *reinterpret_cast<const uint32_t*>(qrow + c) : 0u;
-      float lo = __uint_as_float(w << 16), hi = __uint_as_float(w & 0xFFFF0000u);
-      qf[2 * pp] = lo;
-      qf[2 * pp + 1] = hi;
-      q2[pp] = pack_h2(lo, hi);
-    }
+    q_frag(p.q + ((size_t)b * p.H + (size_t)h * p.G + (head_ok ? gid : 0)) * kD, head_ok, tig, q2);
   };
 
   auto flush = [&](long long seg) {
@@ -190,45 +185,25 @@ __global__ void __launch_bounds__(kScanWarps * 32, 1) scan_kernel(const ScanPara
     }
     const uint8_t* r = ring + st * REC;
 
-    // ---- q * s (hi/lo) and the per-group bias sum_c q_c m_c ----
+    // ---- q * s (hi/lo) and the group bias ----
     uint32_t ahi[16], alo[16];
-    float beta = 0.f;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint4 sv = lds128(r + i * 64 + tig * 16);
-      const uint4 zv = lds128(r + (4 + i) * 64 + tig * 16);
-      const uint32_t s4[4] = {sv.x, sv.y, sv.z, sv.w};
-      const uint32_t z4[4] = {zv.x, zv.y, zv.z, zv.w};
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int pp = 4 * i + k;
-        ahi[pp] = h2_mul(q2[pp], s4[k]);
-        alo[pp] = h2_fma(q2[pp], s4[k], ahi[pp] ^ 0x80008000u);
-        const float2 z = unpack_h2(z4[k]);
-        beta = fmaf(qf[2 * pp], z.x, beta);
-        beta = fmaf(qf[2 * pp + 1], z.y, beta);
-      }
+    float bk;
+    {
+      uint32_t sk[16], zk[16];
+      key_sz(r, tig, sk, zk);
+      bk = q_tilde(q2, sk, zk, p.kappa, ahi, alo);
     }
-    beta += __shfl_xor_sync(kFull, beta, 1);
-    beta += __shfl_xor_sync(kFull, beta, 2);
-    const float bk = beta * p.kappa;
 
     // ---- approximate logits (log2 units) for head gid, 64 tokens ----
-    // two n-tiles at a time so two independent MMA chains interleave
     float u[8][2];
     auto qk_pair = [&](int nt, const uint32_t* b0, const uint32_t* b1) {
-      float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        mma16816(d0, ahi[2 * ks], alo[2 * ks], ahi[2 * ks + 1], alo[2 * ks + 1], b0[2 * ks],
-                 b0[2 * ks + 1]);
-        mma16816(d1, ahi[2 * ks], alo[2 * ks], ahi[2 * ks + 1], alo[2 * ks + 1], b1[2 * ks],
-                 b1[2 * ks + 1]);
-      }
-      u[nt][0] = head_ok ? fmaf(d0[0] + d0[2], p.kappa, bk) : -INFINITY;
-      u[nt][1] = head_ok ? fmaf(d0[1] + d0[3], p.kappa, bk) : -INFINITY;
-      u[nt + 1][0] = head_ok ? fmaf(d1[0] + d1[2], p.kappa, bk) : -INFINITY;
-      u[nt + 1][1] = head_ok ? fmaf(d1[1] + d1[3], p.kappa, bk) : -INFINITY;
+      float d0[4], d1[4];
+      qk_chain(ahi, alo, b0, d0);
+      qk_chain(ahi, alo, b1, d1);
+      u[nt][0] = head_ok ? approx_logit(d0, 0, p.kappa, bk) : -INFINITY;
+      u[nt][1] = head_ok ? approx_logit(d0, 1, p.kappa, bk) : -INFINITY;
+      u[nt + 1][0] = head_ok ? approx_logit(d1, 0, p.kappa, bk) : -INFINITY;
+      u[nt + 1][1] = head_ok ? approx_logit(d1, 1, p.kappa, bk) : -INFINITY;
     };
     if constexpr (KB == 4) {
 #pragma unroll
@@ -287,6 +262,8 @@ __global__ void __launch_bounds__(kScanWarps * 32, 1) scan_kernel(const ScanPara
       dz[3] *= a1;
       m_run = m_new;
     }
+    // the maximum this group's weights are taken against, for the correction
+    if (tig == 0 && head_ok) p.m_used[((size_t)seg * p.ng_cap + g) * kMaxG + gid] = m_run;
 
     // ---- selection score: max over the G heads (lanes differing in gid) ----
     {
@@ -319,34 +296,29 @@ __global__ void __launch_bounds__(kScanWarps * 32, 1) scan_kernel(const ScanPara
       o.y = s2[1] * kLn2;
       *reinterpret_cast<float2*>(p.scores + (size_t)seg * p.capacity + (size_t)g * kKG +
                                  8 * gid + 2 * tig) = o;
+      uint32_t* hs = p.hist + (size_t)seg * kScanHistBins;
+      atomicAdd(hs + (float_key(o.x) >> (32 - kScanHistBits)), 1u);
+      atomicAdd(hs + (float_key(o.y) >> (32 - kScanHistBits)), 1u);
     }
 
-    // ---- probabilities: fp16 pairs (tokens 8nt+2tig, +1) and their rounding
-    // remainders, so p and p*s_v enter the MMAs with ~22-bit precision ----
-    uint32_t ph[8], pl[8];
+    // ---- weights fp16(2^(u - m)) of tokens 8nt+2tig, +1 ----
+    uint32_t ph[8];
 #pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-      const float p0 = exp2f(u[nt][0] - m_run), p1 = exp2f(u[nt][1] - m_run);
-      ph[nt] = pack_h2(p0, p1);
-      const float2 hf = unpack_h2(ph[nt]);
-      pl[nt] = pack_h2(p0 - hf.x, p1 - hf.y);
-    }
+    for (int nt = 0; nt < 8; ++nt)
+      ph[nt] = pack_h2(approx_weight(u[nt][0], m_run), approx_weight(u[nt][1], m_run));
 
-    // ---- value aggregate: acc^T[c][h] += sum_t v'[t][c] * (p[t][h] s_v[t][j]) ----
+    // ---- value aggregate: acc^T[c][h] += sum_t v'[t][c] * fp16(p[t][h] s_v[t][j]) ----
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk) {
       const uint4 s0 = lds128(r + OFF_VS + kk * 128 + tig * 32);
       const uint4 s1 = lds128(r + OFF_VS + kk * 128 + tig * 32 + 16);
       const uint32_t sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
       const uint32_t pa = ph[2 * kk], pb = ph[2 * kk + 1];
-      const uint32_t la = pl[2 * kk], lb = pl[2 * kk + 1];
-      uint32_t bh[4][2], bl[4][2];
+      uint32_t bh[4][2];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         bh[j][0] = h2_mul(pa, sv[2 * j]);
         bh[j][1] = h2_mul(pb, sv[2 * j + 1]);
-        bl[j][0] = h2_fma(la, sv[2 * j], h2_fma(pa, sv[2 * j], bh[j][0] ^ 0x80008000u));
-        bl[j][1] = h2_fma(lb, sv[2 * j + 1], h2_fma(pb, sv[2 * j + 1], bh[j][1] ^ 0x80008000u));
       }
       uint32_t za0 = 0u, za2 = 0u;
       if (gid < 4) {
@@ -357,7 +329,6 @@ __global__ void __launch_bounds__(kScanWarps * 32, 1) scan_kernel(const ScanPara
         za0 = za2 = kOneH2;
       }
       mma16816(dz, za0, 0u, za2, 0u, pa, pb);
-      mma16816(dz, za0, 0u, za2, 0u, la, lb);
       if constexpr (VB == 4) {
         const uint4 v0 = lds128(r + OFF_VC + (2 * kk) * 512 + lane * 16);
         const uint4 v1 = lds128(r + OFF_VC + (2 * kk + 1) * 512 + lane * 16);
@@ -367,7 +338,6 @@ __global__ void __launch_bounds__(kScanWarps * 32, 1) scan_kernel(const ScanPara
           uint32_t a[4];
           unpack4(vw[mt], a);
           mma16816(acc[mt], a[0], a[1], a[2], a[3], bh[mt >> 1][0], bh[mt >> 1][1]);
-          mma16816(acc[mt], a[0], a[1], a[2], a[3], bl[mt >> 1][0], bl[mt >> 1][1]);
         }
       } else {
         const uint4 v = lds128(r + OFF_VC + kk * 512 + lane * 16);
@@ -378,8 +348,6 @@ __global__ void __launch_bounds__(kScanWarps * 32, 1) scan_kernel(const ScanPara
           unpack2(vw[mp], a);
           mma16816(acc[2 * mp], a[0], a[1], a[2], a[3], bh[mp][0], bh[mp][1]);
           mma16816(acc[2 * mp + 1], a[4], a[5], a[6], a[7], bh[mp][0], bh[mp][1]);
-          mma16816(acc[2 * mp], a[0], a[1], a[2], a[3], bl[mp][0], bl[mp][1]);
-          mma16816(acc[2 * mp + 1], a[4], a[5], a[6], a[7], bl[mp][0], bl[mp][1]);
         }
       }
     }
@@ -396,9 +364,8 @@ __global__ void __launch_bounds__(kScanWarps * 32, 1) scan_kernel(const ScanPara
     }
   }
   flush(cur);
-  // the next kernel may be scheduled once every scan CTA got here: launching it
-  // earlier would let its CTAs hold SMs the scan still needs
-  pdl_launch_dependents();
+  // No explicit launch_dependents: the dependent kernel is released as the
+  // scan's CTAs exit, so its thread-block clusters find whole SMs free.
 }
 
 template <int KB, int VB>
@@ -411,8 +378,8 @@ static int launch_scan_t(const ScanParams& sp, int n_ctas, cudaStream_t st) {
       return JFA_ERR_CUDA;
     configured = true;
   }
-  return launch_pdl(scan_kernel<KB, VB>, dim3(n_ctas), dim3(kScanWarps * 32), (size_t)smem, st,
-                    sp) == cudaSuccess
+  return launch_pdl(scan_kernel<KB, VB>, dim3(n_ctas), dim3(ScanCfg<KB, VB>::NW * 32), (size_t)smem,
+                    st, sp) == cudaSuccess
              ? JFA_OK
              : JFA_ERR_CUDA;
 }
@@ -426,6 +393,8 @@ int launch_scores(const jfa_geom& g, const jfa_cache& c, const uint16_t* q, floa
   sp.q = q;
   sp.scores = reinterpret_cast<float*>(ws + L.off_scores);
   sp.partials = reinterpret_cast<float*>(ws + L.off_partials);
+  sp.m_used = reinterpret_cast<float*>(ws + L.off_mused);
+  sp.hist = reinterpret_cast<uint32_t*>(ws + L.off_scan_hist);
   sp.flag = reinterpret_cast<uint32_t*>(ws + L.off_flag);
   sp.total = plan.total_groups;
   sp.ng = plan.ng;

@@ -99,22 +99,28 @@ typedef struct jfa_cache_layout {
 } jfa_cache_layout;
 
 /* Workspace layout: scratch of the decode step (selection scores, split
- * softmax partials, top-k histograms/candidates, merge partials, the error
- * flag).  Sized by jfa_workspace_layout_get for a geometry and a maximum k. */
+ * softmax partials, the running maxima and score histogram of the scan,
+ * top-k histograms/candidates, the error flag).  Sized by
+ * jfa_workspace_layout_get for a geometry and a maximum k. */
 typedef struct jfa_workspace_layout {
   size_t total_bytes;
   size_t off_flag;       /* uint32 device error flag                          */
   size_t off_scores;     /* fp32 [B][H_kv][capacity]: selection score S_t     */
   size_t off_partials;   /* fp32 split partials of the approximate scan       */
-  size_t off_hist;       /* top-k histograms                                  */
-  size_t off_counters;   /* top-k counters                                    */
-  size_t off_cand;       /* top-k per-chunk (key, index) lists                */
-  size_t off_sel;        /* top-k per-chunk list lengths                      */
-  size_t off_merge;      /* fp32 per-chunk exact / removal partials           */
+  size_t off_mused;      /* fp32 [B][H_kv][capacity/64][8]: per key group and
+                            query head, the running maximum the scan's
+                            weights were taken against                        */
+  size_t off_scan_hist;  /* uint32 [B][H_kv][8192]: histogram of the top 13
+                            bits of the selection keys, built by the scan and
+                            cleared by the finishing kernel                   */
+  size_t off_hist;       /* top-k histograms (jfa_topk)                       */
+  size_t off_counters;   /* top-k counters (jfa_topk)                         */
+  size_t off_cand;       /* top-k candidate lists                             */
+  size_t off_sel;        /* top-k per-chunk list lengths (jfa_topk)           */
   int32_t max_topk;
   int32_t partial_slots; /* slots of off_partials                             */
   int32_t cand_cap;      /* list entries per segment                          */
-  int32_t merge_chunks;  /* chunks of off_merge per segment                   */
+  int32_t reserved;
 } jfa_workspace_layout;
 
 /* Human-readable name of a status code (static string). */
@@ -212,7 +218,13 @@ int jfa_topk_noalloc(const float* scores, int32_t n_seg, int32_t stride,
  * minus the top-k tokens' approximate terms); merged as
  *   m = max(m_e, m_a), out = (acc_e e^(m_e-m) + acc_a e^(m_a-m)) /
  *                            (l_e e^(m_e-m) + l_a e^(m_a-m)).
- *   idx          : int32 [B][H_kv][k] from jfa_topk (entries -1 ignored).
+ *   idx          : int32 [B][H_kv][k] from jfa_topk (entries -1 ignored;
+ *                  the others distinct, in [0, N_q), else the device flag
+ *                  JFA_DEVERR_BAD_INDEX is set and the entry skipped).
+ * The approximate terms of the top-k tokens are taken out of the scan's
+ * partials by recomputing, from the packed records and the running maxima
+ * the scan stored, exactly the fp16 weights the scan used, so the removal
+ * leaves only fp32 rounding.
  *   k_exact,
  *   v_exact      : bf16 [B][H_kv][capacity][128], every cached token; device
  *                  memory, or pinned host memory the device can address

@@ -76,7 +76,9 @@ def scan_partials(run: GpuRun):
     n_seg = w.batch * w.kv_heads
     T = n_seg * ng
     sms = torch.cuda.get_device_properties(0).multi_processor_count
-    Wn = min(T, sms * 8, 2048)
+    rec = 512 + 1024 * w.key_bits + 1024 + 1024 * w.val_bits
+    nw = min(16, (227 * 1024 - 1024) // (2 * rec))   # warps per scan CTA
+    Wn = min(T, sms * nw, 4096)
     L = run.ws.layout
     G = w.group
     part = run.ws.buf[L.off_partials:L.off_partials + 4 * L.partial_slots * G * 132]
@@ -110,10 +112,14 @@ def test_scores_and_scan_partials(kb, vb, heads, kv):
     parts = scan_partials(run)
     for (b, hq), (m, l, acc) in parts.items():
         pa = ref.approx_all[b][hq]
-        # same normalised aggregate and consistent mass
-        assert np.allclose(acc / l, O.finish(pa), rtol=1e-4, atol=1e-4)
+        # The scan feeds each weight to the value MMAs as fp16(p) and fp16(p * s_v):
+        # two round-to-nearest steps of relative error <= 2^-11 each, so the
+        # aggregate and the mass are within 2^-10 relative of the fp64 values.
+        want = O.finish(pa)
+        tol = 2.0 ** -10 * 2 * max(1.0, np.abs(want).max())
+        assert np.abs(acc / l - want).max() <= tol
         assert abs(m / np.log2(np.e) - pa.m) < 1e-4
-        assert abs(l * 2.0 ** (m - pa.m * np.log2(np.e)) / pa.l - 1) < 1e-4
+        assert abs(l * 2.0 ** (m - pa.m * np.log2(np.e)) / pa.l - 1) < 2.0 ** -10
 
 
 # ---------------------------------------------------------------- top-k
