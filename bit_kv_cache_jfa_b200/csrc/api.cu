@@ -78,7 +78,7 @@ ScanPlan scan_plan(const jfa_geom& g, int num_sms) {
   const long long n_seg = (long long)g.batch * g.num_kv_heads;
   p.ng = split_point(g.n_ctx) / kKG;
   p.total_groups = n_seg * p.ng;
-  const int nw = scan_cta_warps(g.key_bits, g.val_bits);
+  const int nw = scan_cta_warps(g.key_bits, g.val_bits, g.num_heads / g.num_kv_heads > 4 ? 2 : 1);
   long long w = (long long)num_sms * nw;
   if (w > kMaxScanWarps) w = kMaxScanWarps;
   if (w > p.total_groups) w = p.total_groups;
@@ -264,13 +264,12 @@ int jfa_unpack_record(int32_t key_bits, int32_t val_bits, const void* record, ui
   if (k_codes) {
     for (int t = 0; t < kKG; ++t)
       for (int c = 0; c < kD; ++c) {
-        BitLoc L = kc_loc(key_bits, t, c);
-        uint32_t code;
-        if (key_bits == 3 && kc3_is_pair15(c)) {
-          code = 0;
-          for (int b = 0; b < 3; ++b) code |= ((word(off_kc() + L.byte + 4 * b) >> L.bit) & 1u) << b;
+        BitLoc L[3];
+        uint32_t code = 0;
+        if (kc_bits(key_bits, t, c, L) == 1) {
+          code = (word(off_kc() + L[0].byte) >> L[0].bit) & km;
         } else {
-          code = (word(off_kc() + L.byte) >> L.bit) & km;
+          for (int b = 0; b < 3; ++b) code |= ((word(off_kc() + L[b].byte) >> L[b].bit) & 1u) << b;
         }
         k_codes[t * kD + c] = (uint8_t)code;
       }

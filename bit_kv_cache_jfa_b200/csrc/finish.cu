@@ -87,7 +87,7 @@ struct FinSelect {
 // Record pieces of one quantized token, staged by cp.async.
 struct WStage {
   uint8_t ksz[512];    // key scales / zeros of its group
-  uint8_t kcode[512];  // key codes of its 8-token tile, in lane order
+  uint8_t kcode[1024]; // key codes of its 16-token m-tile, in lane order
   uint8_t vp[256];     // value-code pieces holding its column (8 or 16 x 16 B)
   uint8_t vsz[64];     // its value scales (32 B block) and zeros (32 B block)
   float mu[kMaxG];     // the scan's running maxima of its group
@@ -282,8 +282,8 @@ __device__ __forceinline__ T4 ld16(const void* p) {
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
 }
-__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+__device__ __forceinline__ void cp_async8(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
@@ -296,15 +296,17 @@ __device__ __forceinline__ void stage_issue(const FinishParams& p, int seg, int 
                                             int lane) {
   if (tok_quant(t)) {
     const uint8_t* rec = p.groups + ((size_t)seg * p.ng_cap + (size_t)(t / kKG)) * p.rec_bytes;
-    const int tt = t % kKG, nt = tt >> 3, kk = tt >> 4, tgt = (tt & 7) >> 1;
+    const int tt = t % kKG, kk = tt >> 4, tgt = (tt & 7) >> 1;
     cp_async16(S.ksz + lane * 16, rec + lane * 16);
     if (p.key_bits == 4) {
-      cp_async16(S.kcode + lane * 16, rec + off_kc() + nt * 512 + lane * 16);
+      const uint8_t* src = rec + off_kc() + kk * 1024 + lane * 32;
+      cp_async16(S.kcode + lane * 32, src);
+      cp_async16(S.kcode + lane * 32 + 16, src + 16);
     } else {
-      const uint8_t* src = rec + off_kc() + (nt >> 2) * 1536 + lane * 48 + (nt & 3) * 12;
-      cp_async4(S.kcode + lane * 12, src);
-      cp_async4(S.kcode + lane * 12 + 4, src + 4);
-      cp_async4(S.kcode + lane * 12 + 8, src + 8);
+      const uint8_t* src = rec + off_kc() + kk * 768 + lane * 24;
+      cp_async8(S.kcode + lane * 24, src);
+      cp_async8(S.kcode + lane * 24 + 8, src + 8);
+      cp_async8(S.kcode + lane * 24 + 16, src + 16);
     }
     const int vslots = p.val_bits == 4 ? 16 : 8;
     if (lane < vslots) {
@@ -333,51 +335,58 @@ __device__ __forceinline__ void row_load(const FinishParams& p, int seg, int t, 
 }
 
 // The scan's fp16 weights of quantized token t for every head, recomputed
-// from its staged group pieces with the scan's own arithmetic (q_frag,
-// key_sz/q_tilde, qk_chain, approx_logit, approx_weight, in the same order,
-// here fused per k-step); ph[j] = fp16 bits of head j's weight, on all lanes.
+// from its staged group pieces with the scan's own functions on the same
+// operands (key_sz, bias_mma, scale_pos, q_tilde_col, key_afrag, qk_chain,
+// approx_logit, approx_weight); ph[j] = fp16 bits of head j's weight, on all
+// lanes.  q2[n]: the lane's q of head (gid >> 1) + 4n, as the scan holds it.
+template <int KB, int G>
+__device__ __forceinline__ void replay_weights_t(const FinishParams& p, int t, const WStage& S,
+                                                 const uint32_t (&q2)[2][16], int lane,
+                                                 uint32_t ph[G]) {
+  constexpr int NT = G > 4 ? 2 : 1;
+  const int gid = lane >> 2, tig = lane & 3;
+  const int tt = t % kKG, row = tt & 7, rr = (tt >> 3) & 1;
+  uint32_t sk[16], zk[16], sf[16], qb[NT][16];
+  float bk[NT];
+  key_sz(S.ksz, tig, sk, zk);
+#pragma unroll
+  for (int n = 0; n < NT; ++n) bk[n] = bias_mma(q2[n], zk, p.kappa);
+  scale_pos<KB>(sk, sf);
+#pragma unroll
+  for (int n = 0; n < NT; ++n) q_tilde_col(q2[n], sf, (gid & 1) != 0, qb[n]);
+  uint32_t w[KeyPos<KB>::WORDS];
+  const uint32_t* kw = reinterpret_cast<const uint32_t*>(S.kcode + lane * 4 * KeyPos<KB>::WORDS);
+#pragma unroll
+  for (int i = 0; i < KeyPos<KB>::WORDS; ++i) w[i] = kw[i];
+  uint32_t a[16][2];
+  key_afrag<KB>(w, a);
+  const float kappa_u = p.kappa * KeyPos<KB>::unscale;
+  uint32_t mine[NT];
+#pragma unroll
+  for (int n = 0; n < NT; ++n) {
+    float d[4];
+    qk_chain(a, qb[n], d);
+    const int h = tig + 4 * n;
+    mine[n] = (gid == row && h < G)
+                  ? f2h_rn(approx_weight(approx_logit(d, rr, kappa_u, bk[n]), S.mu[h]))
+                  : 0u;
+  }
+#pragma unroll
+  for (int j = 0; j < G; ++j) ph[j] = __shfl_sync(kAll, mine[j >> 2], row * 4 + (j & 3));
+}
 template <int G>
 __device__ __forceinline__ void replay_weights(const FinishParams& p, int t, const WStage& S,
-                                               const uint32_t q2[16], int lane, uint32_t ph[G]) {
-  const int gid = lane >> 2, tig = lane & 3;
-  const int tt = t % kKG, tq = (tt & 7) >> 1, e = tt & 1;
-  uint32_t b[16];
-  if (p.key_bits == 4) {
-    const uint4 c = ld16<uint4>(S.kcode + lane * 16);
-    unpack4(c.x, b);
-    unpack4(c.y, b + 4);
-    unpack4(c.z, b + 8);
-    unpack4(c.w, b + 12);
-  } else {
-    const uint32_t* w = reinterpret_cast<const uint32_t*>(S.kcode + lane * 12);
-    unpack3(w[0], w[1], w[2], b);
-  }
-  float d[4] = {0.f, 0.f, 0.f, 0.f}, db[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-  for (int ks = 0; ks < 8; ++ks) {
-    const int p0 = 2 * ks, p1 = 2 * ks + 1;
-    const uint32_t s0 = *reinterpret_cast<const uint32_t*>(S.ksz + (p0 >> 2) * 64 + tig * 16 + (p0 & 3) * 4);
-    const uint32_t s1 = *reinterpret_cast<const uint32_t*>(S.ksz + (p1 >> 2) * 64 + tig * 16 + (p1 & 3) * 4);
-    const uint32_t z0 = *reinterpret_cast<const uint32_t*>(S.ksz + (4 + (p0 >> 2)) * 64 + tig * 16 + (p0 & 3) * 4);
-    const uint32_t z1 = *reinterpret_cast<const uint32_t*>(S.ksz + (4 + (p1 >> 2)) * 64 + tig * 16 + (p1 & 3) * 4);
-    const uint32_t h0 = h2_mul(q2[p0], s0), h1 = h2_mul(q2[p1], s1);
-    const uint32_t l0 = h2_fma(q2[p0], s0, h0 ^ 0x80008000u);
-    const uint32_t l1 = h2_fma(q2[p1], s1, h1 ^ 0x80008000u);
-    mma16816(db, q2[p0], 0u, q2[p1], 0u, z0, z1);
-    mma16816(d, h0, l0, h1, l1, b[p0], b[p1]);
-  }
-  const float bk = __fmul_rn(db[0], p.kappa);
-  uint32_t mine = 0u;
-  if (gid < G && tig == tq) mine = f2h_rn(approx_weight(approx_logit(d, e, p.kappa, bk), S.mu[gid]));
-#pragma unroll
-  for (int j = 0; j < G; ++j) ph[j] = __shfl_sync(kAll, mine, j * 4 + tq);
+                                               const uint32_t (&q2)[2][16], int lane,
+                                               uint32_t ph[G]) {
+  if (p.key_bits == 4) replay_weights_t<4, G>(p, t, S, q2, lane, ph);
+  else replay_weights_t<3, G>(p, t, S, q2, lane, ph);
 }
 
 // One token into the warp's combined partial (m, l, a): + its exact term,
 // and, for a quantized token, - the approximate term the scan added for it.
 template <int G>
 __device__ __forceinline__ void warp_token(const FinishParams& p, int t, const WStage& S, uint2 kr,
-                                           uint2 vr, const FinParts<G>& P, const uint32_t q2[16],
+                                           uint2 vr, const FinParts<G>& P, const uint32_t (&q2)[2][16],
                                            int lane, float (&m)[G], float (&l)[G],
                                            float (&a)[G][4]) {
   const float kf[4] = {__uint_as_float(kr.x << 16), __uint_as_float(kr.x & 0xFFFF0000u),
@@ -437,7 +446,7 @@ __device__ __forceinline__ void warp_token(const FinishParams& p, int t, const W
 // updated, stored back).
 template <int G, typename TokAt>
 __device__ __forceinline__ void warp_correct(const FinishParams& p, int seg, TokAt tok_at, int n,
-                                             WStage* ring, FinParts<G>& P, const uint32_t q2[16],
+                                             WStage* ring, FinParts<G>& P, const uint32_t (&q2)[2][16],
                                              int warp, int lane) {
   float m[G], l[G], a[G][4];
 #pragma unroll
@@ -508,8 +517,14 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
     P.qs[i / kD][i % kD] = bf16f(p.q[((size_t)bb * p.H + hh * G + i / kD) * kD + i % kD]);
   for (int i = tid; i < kFinWarps * G * kPartStride; i += kFinThreads)
     (&P.wp[0][0][0])[i] = (i % kPartStride) == 0 ? -INFINITY : 0.f;
-  uint32_t q2[16];
-  q_frag(p.q + ((size_t)bb * p.H + (size_t)hh * G + (gid < G ? gid : 0)) * kD, gid < G, tig, q2);
+  // the lane's q as the scan holds it: head (gid >> 1) + 4n of n-tile n
+  uint32_t q2[2][16];
+#pragma unroll
+  for (int n = 0; n < 2; ++n) {
+    const int hq = (gid >> 1) + 4 * n;
+    const bool ok = hq < G && (n == 0 || G > 4);
+    q_frag(p.q + ((size_t)bb * p.H + (size_t)hh * G + (ok ? hq : 0)) * kD, ok, tig, q2[n]);
+  }
   __syncthreads();
   const int warp = tid >> 5;
 
@@ -854,20 +869,23 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
         reinterpret_cast<float4*>(tile + row * kPartStride)[v] = ld16<float4>(src + 4 * v);
       }
       __syncthreads();
+#pragma unroll
+      for (int i = 0; i < kH2; ++i) {
+        const int j = half + 2 * i;
+        if (j < G) {
 #pragma unroll 1
-      for (int row = 0; row < nr; ++row) {
-        const int j = (r0 + row) % G;
-        if ((j & 1) != half) continue;
-        const float* tr = tile + row * kPartStride;
-        const float rl = tr[1];
-        if (rl > 0.f) {
-          const int i = j >> 1;
-          const float mn = fmaxf(mrun[i], tr[0]);
-          const float s0f = lrun[i] > 0.f ? exp2f(mrun[i] - mn) : 0.f;
-          const float s1f = exp2f(tr[0] - mn);
-          lrun[i] = lrun[i] * s0f + rl * s1f;
-          arun[i] = arun[i] * s0f + tr[4 + c] * s1f;
-          mrun[i] = mn;
+          for (int row = (j - r0 % G + G) % G; row < nr; row += G) {
+            const float* tr = tile + row * kPartStride;
+            const float rl = tr[1];
+            if (rl > 0.f) {
+              const float mn = fmaxf(mrun[i], tr[0]);
+              const float s0f = lrun[i] > 0.f ? exp2f(mrun[i] - mn) : 0.f;
+              const float s1f = exp2f(tr[0] - mn);
+              lrun[i] = lrun[i] * s0f + rl * s1f;
+              arun[i] = arun[i] * s0f + tr[4 + c] * s1f;
+              mrun[i] = mn;
+            }
+          }
         }
       }
       __syncthreads();

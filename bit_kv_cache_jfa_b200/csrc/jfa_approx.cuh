@@ -8,17 +8,42 @@
 // Arithmetic (HACK review, Eq. (4): the product with affinely quantized keys
 // is an integer product plus correction terms), per 64-token group g:
 //   u[h][t] = kappa * ( sum_c (q[h][c] s[g][c]) k'[t][c] + sum_c q[h][c] m[g][c] )
-// in log2 units (kappa = softmax scale * log2 e).  q*s enters mma.sync as an
-// exact fp16 pair (hi, lo): rows 0-7 of the A operand hold hi for the G <= 8
-// heads, rows 8-15 lo; the codes k' are exact small integers in fp16.
+// in log2 units (kappa = softmax scale * log2 e), on mma.sync.m16n8k16:
+//   A = key codes, rows = 16 tokens of an m-tile, columns = channels.  A code
+//       sits in the low mantissa bits of an fp16 half at bit position pos, so
+//       the half is the subnormal code * 2^(pos - 24) and one AND extracts it.
+//   B = q*s as an exact fp16 pair: column 2*h' + 0 holds hi = fp16(q s F),
+//       column 2*h' + 1 holds lo = q s F - hi, for the 4 heads h' of an
+//       n-tile; F = 2^(P - pos) per channel pair undoes the bit position, so
+//       every product is code * q*s * 2^(P - 24).
+//   The bias sum_c q_c m_c is an MMA chain with A = the zero points (every
+//   row) and B = q.
 #pragma once
 
 #include "jfa_common.cuh"
 
 namespace jfa {
 
-// q of query head `gid` as mma.sync A fragments: pair pp = 0..15 holds
-// channels c = 16*(pp>>1) + 2*tig + 8*(pp&1) and c+1 (bf16 -> fp16).
+// Key-code bit positions: largest position P and the position of slot s
+// (slot = channel pair of the B fragment, s = 2*k_step + (channels 8..15)).
+template <int KB>
+struct KeyPos {
+  static constexpr int P = KB == 4 ? 4 : 6;
+  static constexpr int WORDS = KB == 4 ? 8 : 6;  // 32-bit words per lane per m-tile
+  __host__ __device__ static constexpr int pos(int s) {
+    return KB == 4 ? (s < 8 ? 0 : 4) : (s < 6 ? 0 : (s < 12 ? 3 : (s < 15 ? 6 : 0)));
+  }
+  // fp16x2 of F = 2^(P - pos(s))
+  __host__ __device__ static constexpr uint32_t factor(int s) {
+    return KB == 4 ? (s < 8 ? 0x4C004C00u : 0x3C003C00u)
+                   : (s < 6 ? 0x54005400u : (s < 12 ? 0x48004800u : (s < 15 ? 0x3C003C00u : 0x54005400u)));
+  }
+  // kappa multiplier undoing the common 2^(P - 24)
+  static constexpr float unscale = KB == 4 ? 1048576.0f : 262144.0f;
+};
+
+// q of query head h as mma.sync B-fragment channel pairs of the lane:
+// pair pp = 0..15 holds channels c = 16*(pp>>1) + 2*tig + 8*(pp&1), c + 1.
 __device__ __forceinline__ void q_frag(const uint16_t* qrow, bool ok, int tig, uint32_t q2[16]) {
 #pragma unroll
   for (int pp = 0; pp < 16; ++pp) {
@@ -46,36 +71,81 @@ __device__ __forceinline__ void key_sz(const uint8_t* ks, int tig, uint32_t s[16
   }
 }
 
-// q~ = q*s as (hi, lo) fp16 pairs with hi + lo = q*s exactly, and the group
-// bias kappa * sum_c q_c m_c (an fp32 MMA chain: A = q rows, B = the zero
-// points broadcast over the 8 columns).
-__device__ __forceinline__ float q_tilde(const uint32_t q2[16], const uint32_t s[16],
-                                         const uint32_t z[16], float kappa, uint32_t hi[16],
-                                         uint32_t lo[16]) {
+// Key scales times the position factors F (exact powers of two).
+template <int KB>
+__device__ __forceinline__ void scale_pos(const uint32_t s[16], uint32_t sf[16]) {
+#pragma unroll
+  for (int pp = 0; pp < 16; ++pp) sf[pp] = h2_mul(s[pp], KeyPos<KB>::factor(pp));
+}
+
+// The lane's B column of q~ = q * s * F: limb 0 (hi) or 1 (lo), hi + lo exact.
+__device__ __forceinline__ void q_tilde_col(const uint32_t q2[16], const uint32_t sf[16], bool lo,
+                                            uint32_t b[16]) {
 #pragma unroll
   for (int pp = 0; pp < 16; ++pp) {
-    hi[pp] = h2_mul(q2[pp], s[pp]);
-    lo[pp] = h2_fma(q2[pp], s[pp], hi[pp] ^ 0x80008000u);
+    const uint32_t hi = h2_mul(q2[pp], sf[pp]);
+    b[pp] = h2_fma(q2[pp], sf[pp], lo ? (hi ^ 0x80008000u) : 0u);
   }
+}
+
+// kappa * sum_c q_c m_c for the head of the lane's n-tile column pair
+// (lane (gid, tig): head tig of the n-tile); rows all equal.
+__device__ __forceinline__ float bias_mma(const uint32_t q2[16], const uint32_t z[16], float kappa) {
   float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-  for (int ks = 0; ks < 8; ++ks) mma16816(d, q2[2 * ks], 0u, q2[2 * ks + 1], 0u, z[2 * ks], z[2 * ks + 1]);
+  for (int ks = 0; ks < 8; ++ks)
+    mma16816(d, z[2 * ks], z[2 * ks], z[2 * ks + 1], z[2 * ks + 1], q2[2 * ks], q2[2 * ks + 1]);
   return __fmul_rn(d[0], kappa);
 }
 
-// One n-tile (8 tokens): d[e] (hi rows) and d[2+e] (lo rows) for head gid,
-// token 8*nt + 2*tig + e.  b[] = the n-tile's codes as B fragments.
-__device__ __forceinline__ void qk_chain(const uint32_t hi[16], const uint32_t lo[16],
-                                         const uint32_t b[16], float d[4]) {
+// Key codes of one m-tile as A fragments: a[s][0] = slot s for token row gid,
+// a[s][1] = for row gid + 8, from the lane's WORDS words.
+template <int KB>
+__device__ __forceinline__ void key_afrag(const uint32_t* w, uint32_t a[16][2]) {
+  if constexpr (KB == 4) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint32_t ws = w[i] >> 8;
+      a[i][0] = w[i] & 0x000F000Fu;
+      a[i][1] = ws & 0x000F000Fu;
+      a[8 + i][0] = w[i] & 0x00F000F0u;
+      a[8 + i][1] = ws & 0x00F000F0u;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 6; ++i) {
+      const uint32_t ws = w[i] >> 9;
+      a[i][0] = w[i] & 0x00070007u;
+      a[i][1] = ws & 0x00070007u;
+      a[6 + i][0] = w[i] & 0x00380038u;
+      a[6 + i][1] = ws & 0x00380038u;
+    }
+#pragma unroll
+    for (int i = 0; i < 3; ++i) {
+      a[12 + i][0] = w[2 * i] & 0x01C001C0u;
+      a[12 + i][1] = w[2 * i + 1] & 0x01C001C0u;
+    }
+    // slot 15: bit b of the code in bit 15 (31) of word b (rows gid) or 3 + b
+    uint32_t t0 = (w[0] >> 15) & 0x00010001u, t1 = (w[3] >> 15) & 0x00010001u;
+    t0 = lop_and_or(w[1] >> 14, 0x00020002u, t0);
+    t1 = lop_and_or(w[4] >> 14, 0x00020002u, t1);
+    a[15][0] = lop_and_or(w[2] >> 13, 0x00040004u, t0);
+    a[15][1] = lop_and_or(w[5] >> 13, 0x00040004u, t1);
+  }
+}
+
+// One m-tile x one n-tile, 8 k-steps: d[0] (hi) + d[1] (lo) for token row
+// gid, d[2] + d[3] for row gid + 8, head tig of the n-tile.
+__device__ __forceinline__ void qk_chain(const uint32_t a[16][2], const uint32_t b[16], float d[4]) {
   d[0] = d[1] = d[2] = d[3] = 0.f;
 #pragma unroll
   for (int ks = 0; ks < 8; ++ks)
-    mma16816(d, hi[2 * ks], lo[2 * ks], hi[2 * ks + 1], lo[2 * ks + 1], b[2 * ks], b[2 * ks + 1]);
+    mma16816(d, a[2 * ks][0], a[2 * ks][1], a[2 * ks + 1][0], a[2 * ks + 1][1], b[2 * ks], b[2 * ks + 1]);
 }
 
-// Approximate logit (log2 units) of head gid, token 8*nt + 2*tig + e.
-__device__ __forceinline__ float approx_logit(const float d[4], int e, float kappa, float bk) {
-  return __fmaf_rn(__fadd_rn(d[e], d[2 + e]), kappa, bk);
+// Approximate logit (log2 units) of token row gid (r = 0) or gid + 8 (r = 1).
+__device__ __forceinline__ float approx_logit(const float d[4], int r, float kappa_u, float bk) {
+  return __fmaf_rn(__fadd_rn(d[2 * r], d[2 * r + 1]), kappa_u, bk);
 }
 
 // Softmax weight of a logit u against the running maximum m, as the scan
@@ -90,21 +160,5 @@ __device__ __forceinline__ uint16_t h_mul_rn(uint16_t a, uint16_t b) {
 }
 __device__ __forceinline__ uint16_t f2h_rn(float x) { return __half_as_ushort(__float2half_rn(x)); }
 __device__ __forceinline__ float h2f(uint16_t h) { return __half2float(__ushort_as_half(h)); }
-
-// Key codes of n-tile nt as B fragments of the lane, from the record's key
-// code section (shared or global memory).
-template <int KB>
-__device__ __forceinline__ void key_codes(const uint8_t* kc, int nt, int lane, uint32_t b[16]) {
-  if constexpr (KB == 4) {
-    const uint4 c = *reinterpret_cast<const uint4*>(kc + nt * 512 + lane * 16);
-    unpack4(c.x, b);
-    unpack4(c.y, b + 4);
-    unpack4(c.z, b + 8);
-    unpack4(c.w, b + 12);
-  } else {
-    const uint32_t* w = reinterpret_cast<const uint32_t*>(kc + (nt >> 2) * 1536 + lane * 48 + (nt & 3) * 12);
-    unpack3(w[0], w[1], w[2], b);
-  }
-}
 
 }  // namespace jfa

@@ -31,8 +31,8 @@ constexpr int kCtrStride = 8;            // top-k counters per segment: [0] scan
 //   [KS: key scales+zeros 512 B][KC: key codes 64*128*kb/8 B]
 //   [VS: value scales+zeros 1024 B][VC: value codes 64*128*vb/8 B]
 // The code order follows the register fragments of mma.sync.m16n8k16 so the
-// scan kernel turns one 128-bit shared-memory load into ready B (keys) or A
-// (values) operands; see kc_loc / vc_loc for the exact bit positions.
+// scan kernel turns 128-bit shared-memory loads into ready A operands (keys
+// and values); see kc_bits / vc_loc for the exact bit positions.
 // ---------------------------------------------------------------------------
 JFA_HD int kc_bytes(int kb) { return kKG * kD * kb / 8; }
 JFA_HD int vc_bytes(int vb) { return kKG * kD * vb / 8; }
@@ -43,10 +43,11 @@ JFA_HD int off_vc(int kb) { return 512 + kc_bytes(kb) + 1024; }
 JFA_HD int record_bytes(int kb, int vb) { return off_vc(kb) + vc_bytes(vb); }
 
 // Warps per scan CTA: each warp owns a two-record shared-memory ring and the
-// CTA takes a whole SM (227 KB of shared memory), at most 16 warps.
-constexpr int scan_cta_warps(int kb, int vb) {
-  return ((227 * 1024 - 1024) / (2 * (512 + 1024 * kb + 1024 + 1024 * vb))) > 16
-             ? 16
+// CTA takes a whole SM (227 KB of shared memory); at most 16 warps (12 when
+// the query heads of a KV head fill two n-tiles and need more registers).
+constexpr int scan_cta_warps(int kb, int vb, int nt) {
+  return ((227 * 1024 - 1024) / (2 * (512 + 1024 * kb + 1024 + 1024 * vb))) > (nt == 2 ? 12 : 16)
+             ? (nt == 2 ? 12 : 16)
              : ((227 * 1024 - 1024) / (2 * (512 + 1024 * kb + 1024 + 1024 * vb)));
 }
 
@@ -55,7 +56,7 @@ struct BitLoc {
   int bit;   // bit of the code's least significant bit inside that word
 };
 
-// Fragment coordinates of key channel c for the QK product (B operand rows):
+// Fragment coordinates of key channel c as a q-pair index of the lane:
 // k-step ks = c/16; inside it the thread tig = (c%8)/2 holds channels
 // {2tig, 2tig+1} (half hf=0) and {2tig+8, 2tig+9} (hf=1); e picks the fp16
 // half of the register.  Pair index p = 2*ks + hf runs over 16 pairs.
@@ -67,38 +68,47 @@ JFA_HD void key_channel_frag(int c, int& tig, int& pair, int& e) {
   pair = 2 * ks + hf;
 }
 
-// Key code of (token t, channel c); for 3-bit keys pair 15 is split over the
-// spare top bit of each half of the thread's three words (bit-th code bit in
-// word bit_word); the function reports the word of code bit 0 and the caller
-// asks kc3_pair15 for the other bits.
-JFA_HD BitLoc kc_loc(int kb, int t, int c) {
-  int tig, p, e;
-  key_channel_frag(c, tig, p, e);
-  int nt = t >> 3, gid = t & 7;
-  int lane = gid * 4 + tig;
-  BitLoc L;
+// Key code of (token t, channel c) for the QK product with tokens as the
+// A-operand rows of mma.sync.m16n8k16: m-tile mt = t/16 holds 32 lanes x W
+// 32-bit words (W = 6 for 3-bit, 8 for 4-bit codes); lane = (t%8)*4 + tig,
+// pair slot s = key_channel_frag's pair, row r = (t%16)/8 (token gid or
+// gid + 8), half e (+16 bits).  Inside a 16-bit half a code sits at bit
+// position 0, 3 or 6 (3-bit) or 0 or 4 (4-bit), so the half read as fp16 is
+// the subnormal code * 2^(pos-24) after one AND; rows gid + 8 sit 9 (3-bit)
+// or 8 (4-bit) bits higher, or in the next word.  3-bit slot 15 spreads its
+// three code bits over bit 15 of three words.  Returns the number of pieces:
+// 1 (code bits contiguous from L[0]) or 3 (code bit b at L[b]).
+JFA_HD int kc_bits(int kb, int t, int c, BitLoc L[3]) {
+  int tig, s, e;
+  key_channel_frag(c, tig, s, e);
+  const int mt = t >> 4, row = t & 15, gid = row & 7, r = row >> 3;
+  const int W = kb == 4 ? 8 : 6;
+  const int base = mt * 32 * 4 * W + (gid * 4 + tig) * 4 * W;
   if (kb == 4) {
-    int w = p >> 2;
-    L.byte = nt * 512 + lane * 16 + w * 4;
-    L.bit = 4 * (p & 3) + 16 * e;
-  } else {  // 3-bit
-    int nt4 = nt >> 2, rr = nt & 3;
-    int base = nt4 * 1536 + lane * 48 + rr * 12;
-    if (p < 15) {
-      int w = p / 5;
-      L.byte = base + w * 4;
-      L.bit = 3 * (p % 5) + 16 * e;
-    } else {
-      L.byte = base;  // bit b of the code lives in word b at bit 15 + 16e
-      L.bit = 15 + 16 * e;
-    }
+    L[0].byte = base + 4 * (s & 7);
+    L[0].bit = 4 * (s >> 3) + 8 * r + 16 * e;
+    return 1;
   }
-  return L;
-}
-JFA_HD bool kc3_is_pair15(int c) {
-  int tig, p, e;
-  key_channel_frag(c, tig, p, e);
-  return p == 15;
+  if (s < 6) {
+    L[0].byte = base + 4 * s;
+    L[0].bit = 9 * r + 16 * e;
+    return 1;
+  }
+  if (s < 12) {
+    L[0].byte = base + 4 * (s - 6);
+    L[0].bit = 3 + 9 * r + 16 * e;
+    return 1;
+  }
+  if (s < 15) {
+    L[0].byte = base + 4 * (2 * (s - 12) + r);
+    L[0].bit = 6 + 16 * e;
+    return 1;
+  }
+  for (int b = 0; b < 3; ++b) {
+    L[b].byte = base + 4 * (3 * r + b);
+    L[b].bit = 15 + 16 * e;
+  }
+  return 3;
 }
 
 // Key scale/zero of channel c: chunk i (16 B per tig) holds 4 pairs; chunks

@@ -90,16 +90,16 @@ __global__ void __launch_bounds__(256) pack_groups_kernel(PackParams p) {
     bad |= !finite_h(zb) || !finite_h(sb);
     *reinterpret_cast<uint16_t*>(rb + off_ks() + ks_scale_off(c)) = sb;
     *reinterpret_cast<uint16_t*>(rb + off_ks() + ks_zero_off(c)) = zb;
-    const bool split15 = (p.key_bits == 3) && kc3_is_pair15(c);
     for (int t = 0; t < kKG; ++t) {
       uint32_t code = quant_code((double)bf(xk[t][c]), z, s, p.key_bits);
-      BitLoc L = kc_loc(p.key_bits, t, c);
-      uint32_t* base = reinterpret_cast<uint32_t*>(rb + off_kc() + L.byte);
-      if (!split15) {
-        if (code) atomicOr(base, code << L.bit);
+      BitLoc L[3];
+      const int n = kc_bits(p.key_bits, t, c, L);
+      if (n == 1) {
+        if (code) atomicOr(reinterpret_cast<uint32_t*>(rb + off_kc() + L[0].byte), code << L[0].bit);
       } else {
         for (int b = 0; b < 3; ++b)
-          if ((code >> b) & 1u) atomicOr(base + b, 1u << L.bit);
+          if ((code >> b) & 1u)
+            atomicOr(reinterpret_cast<uint32_t*>(rb + off_kc() + L[b].byte), 1u << L[b].bit);
       }
     }
   } else {

@@ -4,18 +4,21 @@
 // Per 64-token group g of a (sequence, KV head) and query head h the logit
 //   s_hat[h][t] = scale * ( sum_c (q[h][c]*s[g][c]) * k'[t][c] + sum_c q[h][c]*m[g][c] )
 // is HACK's affine identity (HACK review, Eq. (4)) with an unquantized query;
-// jfa_approx.cuh holds that arithmetic (mma.sync with q*s as an exact fp16
-// pair, the bias as an MMA chain).
+// jfa_approx.cuh holds that arithmetic: mma.sync with the 16 tokens of an
+// m-tile as A rows (codes extracted by one AND as fp16 subnormals), q*s as an
+// exact (hi, lo) fp16 column pair per head as B, the bias as an MMA chain.
 //
 // The same pass accumulates, per query head, the online-softmax partial over
 // the dequantized values v_hat = s_v * v' + m_v (v' codes exact in fp16):
 //   sum_t p_t v_hat[t][c] = sum_t (p_t s_v[t][j]) v'[t][c] + sum_t p_t m_v[t][j]
 // as an MMA with A = value codes (rows = channels, columns = tokens) and
-// B = fp16(p) * s_v (columns = heads), plus a small MMA whose A rows are the
-// value zeros of the four channel groups and a row of ones (giving sum p).
-// The running maximum each group's weights were taken against is stored
-// (m_used), so the correction step recomputes exactly these fp16 weights for
-// the top-k tokens and removes their terms without a rounding residue.
+// B = fp16(p) * s_v (columns = heads; the weights move from the QK output
+// layout to this operand layout by two shuffles per 16 tokens), plus a small
+// MMA whose A rows are the value zeros of the four channel groups and a row
+// of ones (giving sum p).  The running maximum each group's weights were
+// taken against is stored (m_used), so the correction step recomputes
+// exactly these fp16 weights for the top-k tokens and removes their terms
+// without a rounding residue.
 //
 // Also written per token: the selection score S_t = max over the G heads
 // (natural-log units), and a per-segment histogram of its top 13 key bits
@@ -56,23 +59,25 @@ __device__ __forceinline__ uint2 lds64(const uint8_t* p) {
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr unsigned kFull = 0xFFFFFFFFu;
 
-template <int KB, int VB>
+template <int KB, int VB, int NT>
 struct ScanCfg {
   static constexpr int REC = 512 + 1024 * KB + 1024 + 1024 * VB;
-  static constexpr int NW = scan_cta_warps(KB, VB);
+  static constexpr int NW = scan_cta_warps(KB, VB, NT);
   static constexpr int STAGES = 2;
   static constexpr int SMEM = NW * STAGES * REC + NW * STAGES * 8;
   static_assert(SMEM <= 227 * 1024, "scan ring exceeds shared memory");
 };
 
-template <int KB, int VB>
-__global__ void __launch_bounds__(ScanCfg<KB, VB>::NW * 32, 1) scan_kernel(const ScanParams p) {
-  constexpr int REC = ScanCfg<KB, VB>::REC;
-  constexpr int S = ScanCfg<KB, VB>::STAGES;
-  constexpr int NW = ScanCfg<KB, VB>::NW;
+template <int KB, int VB, int NT>
+__global__ void __launch_bounds__(ScanCfg<KB, VB, NT>::NW * 32, 1) scan_kernel(const ScanParams p) {
+  using Cfg = ScanCfg<KB, VB, NT>;
+  constexpr int REC = Cfg::REC;
+  constexpr int S = Cfg::STAGES;
+  constexpr int NW = Cfg::NW;
   constexpr int OFF_KC = 512;
   constexpr int OFF_VS = 512 + 1024 * KB;
   constexpr int OFF_VC = OFF_VS + 1024;
+  constexpr int KW = KeyPos<KB>::WORDS;
   extern __shared__ __align__(128) uint8_t smem[];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -111,20 +116,39 @@ __global__ void __launch_bounds__(ScanCfg<KB, VB>::NW * 32, 1) scan_kernel(const
       if (g0 + i < g1) issue_next(i);
   }
 
-  const bool head_ok = gid < p.G;
+  // lane roles: B column gid of n-tile n = (head (gid >> 1) + 4n, limb gid & 1);
+  // logits of head tig + 4n; value columns (heads) 2 tig, 2 tig + 1
+  const bool lo_lane = (gid & 1) != 0;
+  bool hv[NT];  // head tig + 4n exists
+#pragma unroll
+  for (int n = 0; n < NT; ++n) hv[n] = tig + 4 * n < p.G;
+  const float kappa_u = p.kappa * KeyPos<KB>::unscale;
   float acc[8][4];
   float dz[4];
-  float m_run = 0.f;
-  uint32_t q2[16];
+  float m_run[NT];
+  uint32_t q2[NT][16];
   long long cur = -1;
 
   auto reset = [&](long long seg) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
     dz[0] = dz[1] = dz[2] = dz[3] = 0.f;
-    m_run = head_ok ? -INFINITY : 0.f;
     const int b = (int)(seg / p.hkv), h = (int)(seg % p.hkv);
-    q_frag(p.q + ((size_t)b * p.H + (size_t)h * p.G + (head_ok ? gid : 0)) * kD, head_ok, tig, q2);
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+      m_run[n] = hv[n] ? -INFINITY : 0.f;
+      const int hq = (gid >> 1) + 4 * n;
+      const bool ok = hq < p.G;
+      q_frag(p.q + ((size_t)b * p.H + (size_t)h * p.G + (ok ? hq : 0)) * kD, ok, tig, q2[n]);
+    }
+  };
+
+  // running maximum of head hh (held by lanes with tig = hh & 3)
+  auto head_m = [&](int hh) {
+    float v[NT];
+#pragma unroll
+    for (int n = 0; n < NT; ++n) v[n] = __shfl_sync(kFull, m_run[n], hh & 3);
+    return NT == 2 && (hh >> 2) ? v[NT - 1] : v[0];
   };
 
   auto flush = [&](long long seg) {
@@ -137,8 +161,7 @@ __global__ void __launch_bounds__(ScanCfg<KB, VB>::NW * 32, 1) scan_kernel(const
     }
     const float l0 = __shfl_sync(kFull, dz[0], 16 + tig);
     const float l1 = __shfl_sync(kFull, dz[1], 16 + tig);
-    const float mh0 = __shfl_sync(kFull, m_run, (2 * tig) * 4);
-    const float mh1 = __shfl_sync(kFull, m_run, (2 * tig + 1) * 4);
+    const float mh0 = head_m(2 * tig), mh1 = head_m(2 * tig + 1);
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
       const int h = 2 * tig + e;
@@ -185,70 +208,72 @@ __global__ void __launch_bounds__(ScanCfg<KB, VB>::NW * 32, 1) scan_kernel(const
     }
     const uint8_t* r = ring + st * REC;
 
-    // ---- q * s (hi/lo) and the group bias ----
-    uint32_t ahi[16], alo[16];
-    float bk;
+    // ---- B operands: q~ = q * s * F (hi or lo per lane) and the group bias
+    uint32_t qb[NT][16];
+    float bk[NT];
     {
-      uint32_t sk[16], zk[16];
+      uint32_t sk[16], zk[16], sf[16];
       key_sz(r, tig, sk, zk);
-      bk = q_tilde(q2, sk, zk, p.kappa, ahi, alo);
+#pragma unroll
+      for (int n = 0; n < NT; ++n) bk[n] = bias_mma(q2[n], zk, p.kappa);
+      scale_pos<KB>(sk, sf);
+#pragma unroll
+      for (int n = 0; n < NT; ++n) q_tilde_col(q2[n], sf, lo_lane, qb[n]);
     }
 
-    // ---- approximate logits (log2 units) for head gid, 64 tokens ----
-    float u[8][2];
-    auto qk_pair = [&](int nt, const uint32_t* b0, const uint32_t* b1) {
-      float d0[4], d1[4];
-      qk_chain(ahi, alo, b0, d0);
-      qk_chain(ahi, alo, b1, d1);
-      u[nt][0] = head_ok ? approx_logit(d0, 0, p.kappa, bk) : -INFINITY;
-      u[nt][1] = head_ok ? approx_logit(d0, 1, p.kappa, bk) : -INFINITY;
-      u[nt + 1][0] = head_ok ? approx_logit(d1, 0, p.kappa, bk) : -INFINITY;
-      u[nt + 1][1] = head_ok ? approx_logit(d1, 1, p.kappa, bk) : -INFINITY;
-    };
-    if constexpr (KB == 4) {
+    // ---- approximate logits (log2 units): u[mt][n][r] of head tig + 4n,
+    // token 16 mt + gid + 8 r
+    float u[4][NT][2];
 #pragma unroll
-      for (int nt = 0; nt < 8; nt += 2) {
-        const uint4 ca = lds128(r + OFF_KC + nt * 512 + lane * 16);
-        const uint4 cb = lds128(r + OFF_KC + (nt + 1) * 512 + lane * 16);
-        uint32_t b0[16], b1[16];
-        unpack4(ca.x, b0);
-        unpack4(ca.y, b0 + 4);
-        unpack4(ca.z, b0 + 8);
-        unpack4(ca.w, b0 + 12);
-        unpack4(cb.x, b1);
-        unpack4(cb.y, b1 + 4);
-        unpack4(cb.z, b1 + 8);
-        unpack4(cb.w, b1 + 12);
-        qk_pair(nt, b0, b1);
+    for (int mt = 0; mt < 4; ++mt) {
+      uint32_t w[KW];
+      const uint8_t* kp = r + OFF_KC + mt * (32 * 4 * KW) + lane * 4 * KW;
+      if constexpr (KB == 4) {
+        const uint4 c0 = lds128(kp), c1 = lds128(kp + 16);
+        w[0] = c0.x; w[1] = c0.y; w[2] = c0.z; w[3] = c0.w;
+        w[4] = c1.x; w[5] = c1.y; w[6] = c1.z; w[7] = c1.w;
+      } else {
+        const uint2 c0 = lds64(kp), c1 = lds64(kp + 8), c2 = lds64(kp + 16);
+        w[0] = c0.x; w[1] = c0.y; w[2] = c1.x; w[3] = c1.y; w[4] = c2.x; w[5] = c2.y;
       }
-    } else {
+      uint32_t a[16][2];
+      key_afrag<KB>(w, a);
 #pragma unroll
-      for (int nt4 = 0; nt4 < 2; ++nt4) {
-        const uint8_t* cp = r + OFF_KC + nt4 * 1536 + lane * 48;
-        const uint4 c0 = lds128(cp), c1 = lds128(cp + 16), c2 = lds128(cp + 32);
-        const uint32_t w[12] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y,
-                                c1.z, c1.w, c2.x, c2.y, c2.z, c2.w};
-#pragma unroll
-        for (int rr = 0; rr < 4; rr += 2) {
-          uint32_t b0[16], b1[16];
-          unpack3(w[3 * rr], w[3 * rr + 1], w[3 * rr + 2], b0);
-          unpack3(w[3 * rr + 3], w[3 * rr + 4], w[3 * rr + 5], b1);
-          qk_pair(nt4 * 4 + rr, b0, b1);
-        }
+      for (int n = 0; n < NT; ++n) {
+        float d[4];
+        qk_chain(a, qb[n], d);
+        u[mt][n][0] = hv[n] ? approx_logit(d, 0, kappa_u, bk[n]) : -INFINITY;
+        u[mt][n][1] = hv[n] ? approx_logit(d, 1, kappa_u, bk[n]) : -INFINITY;
       }
     }
 
-    // ---- online softmax bookkeeping for head gid ----
-    float mx = u[0][0];
+    // ---- online softmax bookkeeping, head tig + 4n (reduce over gid)
+    bool grow = false;
+    float m_new[NT];
 #pragma unroll
-    for (int nt = 0; nt < 8; ++nt) mx = fmaxf(mx, fmaxf(u[nt][0], u[nt][1]));
-    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
-    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
-    const float m_new = fmaxf(m_run, mx);
-    if (__any_sync(kFull, m_new > m_run)) {
-      const float alpha = exp2f(m_run - m_new);
-      const float a0 = __shfl_sync(kFull, alpha, (2 * tig) * 4);
-      const float a1 = __shfl_sync(kFull, alpha, (2 * tig + 1) * 4);
+    for (int n = 0; n < NT; ++n) {
+      float mx = u[0][n][0];
+#pragma unroll
+      for (int mt = 0; mt < 4; ++mt) mx = fmaxf(mx, fmaxf(u[mt][n][0], u[mt][n][1]));
+      mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 4));
+      mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 8));
+      mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
+      m_new[n] = fmaxf(m_run[n], mx);
+      grow |= m_new[n] > m_run[n];
+    }
+    if (__any_sync(kFull, grow)) {
+      float al[NT];
+#pragma unroll
+      for (int n = 0; n < NT; ++n) al[n] = exp2f(m_run[n] - m_new[n]);
+      // value columns are heads 2 tig, 2 tig + 1: their factors from lanes tig' = h & 3
+      float a0v[NT], a1v[NT];
+#pragma unroll
+      for (int n = 0; n < NT; ++n) {
+        a0v[n] = __shfl_sync(kFull, al[n], (2 * tig) & 3);
+        a1v[n] = __shfl_sync(kFull, al[n], (2 * tig + 1) & 3);
+      }
+      const float a0 = (NT == 2 && tig >= 2) ? a0v[NT - 1] : a0v[0];
+      const float a1 = (NT == 2 && tig >= 2) ? a1v[NT - 1] : a1v[0];
 #pragma unroll
       for (int mt = 0; mt < 8; ++mt) {
         acc[mt][0] *= a0;
@@ -260,60 +285,80 @@ __global__ void __launch_bounds__(ScanCfg<KB, VB>::NW * 32, 1) scan_kernel(const
       dz[1] *= a1;
       dz[2] *= a0;
       dz[3] *= a1;
-      m_run = m_new;
+#pragma unroll
+      for (int n = 0; n < NT; ++n) m_run[n] = m_new[n];
     }
     // the maximum this group's weights are taken against, for the correction
-    if (tig == 0 && head_ok) p.m_used[((size_t)seg * p.ng_cap + g) * kMaxG + gid] = m_run;
+    if (gid == 0) {
+#pragma unroll
+      for (int n = 0; n < NT; ++n)
+        if (hv[n]) p.m_used[((size_t)seg * p.ng_cap + g) * kMaxG + tig + 4 * n] = m_run[n];
+    }
 
-    // ---- selection score: max over the G heads (lanes differing in gid) ----
+    // ---- selection score S = max over heads; lane ends with m-tile tig,
+    // tokens 16 tig + gid and + 8
     {
-      float v8[4][2], v4[2][2], s2[2];
-      const bool b2 = (gid & 4) != 0, b1 = (gid & 2) != 0, b0 = (gid & 1) != 0;
+      float v[4][2];
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
+      for (int mt = 0; mt < 4; ++mt)
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const float keep = b2 ? u[i + 4][e] : u[i][e];
-          const float send = b2 ? u[i][e] : u[i + 4][e];
-          v8[i][e] = fmaxf(keep, __shfl_xor_sync(kFull, send, 16));
+        for (int rr = 0; rr < 2; ++rr) {
+          float x = u[mt][0][rr];
+#pragma unroll
+          for (int n = 1; n < NT; ++n) x = fmaxf(x, u[mt][n][rr]);
+          v[mt][rr] = x;
         }
+      const bool b1 = (tig & 2) != 0, b0 = (tig & 1) != 0;
+      float w2[2][2];
 #pragma unroll
       for (int i = 0; i < 2; ++i)
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const float keep = b1 ? v8[i + 2][e] : v8[i][e];
-          const float send = b1 ? v8[i][e] : v8[i + 2][e];
-          v4[i][e] = fmaxf(keep, __shfl_xor_sync(kFull, send, 8));
+        for (int rr = 0; rr < 2; ++rr) {
+          const float keep = b1 ? v[2 + i][rr] : v[i][rr];
+          const float send = b1 ? v[i][rr] : v[2 + i][rr];
+          w2[i][rr] = fmaxf(keep, __shfl_xor_sync(kFull, send, 2));
         }
+      float sc[2];
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const float keep = b0 ? v4[1][e] : v4[0][e];
-        const float send = b0 ? v4[0][e] : v4[1][e];
-        s2[e] = fmaxf(keep, __shfl_xor_sync(kFull, send, 4));
+      for (int rr = 0; rr < 2; ++rr) {
+        const float keep = b0 ? w2[1][rr] : w2[0][rr];
+        const float send = b0 ? w2[0][rr] : w2[1][rr];
+        sc[rr] = fmaxf(keep, __shfl_xor_sync(kFull, send, 1)) * kLn2;
       }
-      float2 o;
-      o.x = s2[0] * kLn2;
-      o.y = s2[1] * kLn2;
-      *reinterpret_cast<float2*>(p.scores + (size_t)seg * p.capacity + (size_t)g * kKG +
-                                 8 * gid + 2 * tig) = o;
+      float* srow = p.scores + (size_t)seg * p.capacity + (size_t)g * kKG + 16 * tig + gid;
+      srow[0] = sc[0];
+      srow[8] = sc[1];
       uint32_t* hs = p.hist + (size_t)seg * kScanHistBins;
-      atomicAdd(hs + (float_key(o.x) >> (32 - kScanHistBits)), 1u);
-      atomicAdd(hs + (float_key(o.y) >> (32 - kScanHistBits)), 1u);
+      atomicAdd(hs + (float_key(sc[0]) >> (32 - kScanHistBits)), 1u);
+      atomicAdd(hs + (float_key(sc[1]) >> (32 - kScanHistBits)), 1u);
     }
 
-    // ---- weights fp16(2^(u - m)) of tokens 8nt+2tig, +1 ----
-    uint32_t ph[8];
+    // ---- weights fp16(2^(u - m)) packed per m-tile: (token gid, token gid + 8)
+    uint32_t X[4][NT];
 #pragma unroll
-    for (int nt = 0; nt < 8; ++nt)
-      ph[nt] = pack_h2(approx_weight(u[nt][0], m_run), approx_weight(u[nt][1], m_run));
+    for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+      for (int n = 0; n < NT; ++n)
+        X[mt][n] = pack_h2(approx_weight(u[mt][n][0], m_run[n]), approx_weight(u[mt][n][1], m_run[n]));
 
     // ---- value aggregate: acc^T[c][h] += sum_t v'[t][c] * fp16(p[t][h] s_v[t][j]) ----
+    const int src0 = (2 * tig) * 4 + (gid & 3), src1 = (2 * tig + 1) * 4 + (gid & 3);
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk) {
+      // weights of head gid, tokens 16kk + 2tig, +1 (pa) and + 8, + 9 (pb)
+      uint32_t y0 = __shfl_sync(kFull, X[kk][0], src0), y1 = __shfl_sync(kFull, X[kk][0], src1);
+      if constexpr (NT == 2) {
+        const uint32_t z0 = __shfl_sync(kFull, X[kk][NT - 1], src0);
+        const uint32_t z1 = __shfl_sync(kFull, X[kk][NT - 1], src1);
+        if (gid >= 4) {
+          y0 = z0;
+          y1 = z1;
+        }
+      }
+      const uint32_t pa = __byte_perm(y0, y1, 0x5410), pb = __byte_perm(y0, y1, 0x7632);
       const uint4 s0 = lds128(r + OFF_VS + kk * 128 + tig * 32);
       const uint4 s1 = lds128(r + OFF_VS + kk * 128 + tig * 32 + 16);
       const uint32_t sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-      const uint32_t pa = ph[2 * kk], pb = ph[2 * kk + 1];
       uint32_t bh[4][2];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
@@ -368,20 +413,25 @@ __global__ void __launch_bounds__(ScanCfg<KB, VB>::NW * 32, 1) scan_kernel(const
   // scan's CTAs exit, so its thread-block clusters find whole SMs free.
 }
 
-template <int KB, int VB>
+template <int KB, int VB, int NT>
 static int launch_scan_t(const ScanParams& sp, int n_ctas, cudaStream_t st) {
-  const int smem = ScanCfg<KB, VB>::SMEM;
+  using Cfg = ScanCfg<KB, VB, NT>;
   static bool configured = false;
   if (!configured) {
-    if (cudaFuncSetAttribute(scan_kernel<KB, VB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             smem) != cudaSuccess)
+    if (cudaFuncSetAttribute(scan_kernel<KB, VB, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Cfg::SMEM) != cudaSuccess)
       return JFA_ERR_CUDA;
     configured = true;
   }
-  return launch_pdl(scan_kernel<KB, VB>, dim3(n_ctas), dim3(ScanCfg<KB, VB>::NW * 32), (size_t)smem,
+  return launch_pdl(scan_kernel<KB, VB, NT>, dim3(n_ctas), dim3(Cfg::NW * 32), (size_t)Cfg::SMEM,
                     st, sp) == cudaSuccess
              ? JFA_OK
              : JFA_ERR_CUDA;
+}
+
+template <int KB, int VB>
+static int launch_scan_g(const ScanParams& sp, int n_ctas, cudaStream_t st) {
+  return sp.G > 4 ? launch_scan_t<KB, VB, 2>(sp, n_ctas, st) : launch_scan_t<KB, VB, 1>(sp, n_ctas, st);
 }
 
 int launch_scores(const jfa_geom& g, const jfa_cache& c, const uint16_t* q, float scale,
@@ -405,10 +455,10 @@ int launch_scores(const jfa_geom& g, const jfa_cache& c, const uint16_t* q, floa
   sp.H = g.num_heads;
   sp.n_warps = plan.n_warps;
   sp.kappa = scale * 1.4426950408889634f;
-  if (g.key_bits == 3 && g.val_bits == 2) return launch_scan_t<3, 2>(sp, plan.n_ctas, st);
-  if (g.key_bits == 4 && g.val_bits == 4) return launch_scan_t<4, 4>(sp, plan.n_ctas, st);
-  if (g.key_bits == 3 && g.val_bits == 4) return launch_scan_t<3, 4>(sp, plan.n_ctas, st);
-  if (g.key_bits == 4 && g.val_bits == 2) return launch_scan_t<4, 2>(sp, plan.n_ctas, st);
+  if (g.key_bits == 3 && g.val_bits == 2) return launch_scan_g<3, 2>(sp, plan.n_ctas, st);
+  if (g.key_bits == 4 && g.val_bits == 4) return launch_scan_g<4, 4>(sp, plan.n_ctas, st);
+  if (g.key_bits == 3 && g.val_bits == 4) return launch_scan_g<3, 4>(sp, plan.n_ctas, st);
+  if (g.key_bits == 4 && g.val_bits == 2) return launch_scan_g<4, 2>(sp, plan.n_ctas, st);
   return JFA_ERR_UNSUPPORTED;
 }
 

@@ -77,7 +77,7 @@ def scan_partials(run: GpuRun):
     T = n_seg * ng
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     rec = 512 + 1024 * w.key_bits + 1024 + 1024 * w.val_bits
-    nw = min(16, (227 * 1024 - 1024) // (2 * rec))   # warps per scan CTA
+    nw = min(12 if w.group > 4 else 16, (227 * 1024 - 1024) // (2 * rec))   # warps per scan CTA
     Wn = min(T, sms * nw, 4096)
     L = run.ws.layout
     G = w.group
