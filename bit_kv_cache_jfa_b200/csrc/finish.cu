@@ -411,13 +411,17 @@ __device__ __forceinline__ void warp_token(const FinishParams& p, int t, const W
     zv = h2f(*reinterpret_cast<const uint16_t*>(S.vsz + 32 + jg * 8 + hi8 * 4 + 2 * e));
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const int c = 4 * lane + i, mt = c >> 4, rc = c & 15, gd = rc & 7, r = (rc >> 3) + 2 * hi8;
+      // the staged pieces are the token column's lanes (gd*4 + tig) of the
+      // k-step's chunks; word and bit as in vc_loc
+      const int c = 4 * lane + i, mt = c >> 4, rc = c & 15, gd = rc & 7, chi = rc >> 3;
+      const int bit = vc_pos(p.val_bits, mt) + 8 * chi + 16 * e;
       if (p.val_bits == 4) {
-        const uint32_t w = *reinterpret_cast<const uint32_t*>(S.vp + ((mt >> 2) * 8 + gd) * 16 + (mt & 3) * 4);
-        code[i] = (float)((w >> (4 * r + 16 * e)) & 15u);
+        const int w8 = 2 * (mt & 3) + hi8;
+        const uint32_t w = *reinterpret_cast<const uint32_t*>(S.vp + ((w8 >> 2) * 8 + gd) * 16 + (w8 & 3) * 4);
+        code[i] = (float)((w >> bit) & 15u);
       } else {
-        const uint32_t w = *reinterpret_cast<const uint32_t*>(S.vp + gd * 16 + (mt >> 1) * 4);
-        code[i] = (float)((w >> (2 * (4 * (mt & 1) + r) + 16 * e)) & 3u);
+        const uint32_t w = *reinterpret_cast<const uint32_t*>(S.vp + gd * 16 + (2 * (mt & 1) + hi8) * 4);
+        code[i] = (float)((w >> bit) & 3u);
       }
     }
   }

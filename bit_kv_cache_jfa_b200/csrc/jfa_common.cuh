@@ -126,24 +126,28 @@ JFA_HD int ks_zero_off(int c) {
 
 // Value code of (token t, channel c) for the PV product (A operand: rows =
 // channels, columns = tokens).  k-step kk = t/16; thread tig holds tokens
-// {2tig, 2tig+1} (+8 for the second half); m-tile mt = c/16, row gid = c%8,
-// +8 rows for channels 8..15.  Register r = chi + 2*hi8 as in the A fragment.
+// {2tig, 2tig+1} (hi8 = 0) and {2tig+8, 2tig+9} (hi8 = 1); m-tile mt = c/16,
+// row gid = c%8, chi = 1 for channels 8..15 of the tile.  Every code of
+// m-tile mt sits at bit position p(mt) inside its 16-bit half (2-bit codes:
+// 2*(mt/2), 4-bit: 4*(mt/4)), rows chi = 1 eight bits higher, so one AND
+// (after a shift by 8) gives the fp16 subnormal code * 2^(p - 24) and the
+// tile's accumulator is scaled back once.  Per lane and k-step: 4 words
+// (2-bit, one 512-byte chunk) or 8 words (4-bit, chunks 2kk and 2kk+1); word
+// 2*(mt%2) + hi8 (2-bit) or 2*(mt%4) + hi8 (4-bit).
+JFA_HD int vc_pos(int vb, int mt) { return vb == 4 ? 4 * (mt >> 2) : 2 * (mt >> 1); }
 JFA_HD BitLoc vc_loc(int vb, int t, int c) {
   int kk = t >> 4, rt = t & 15;
   int hi8 = rt >> 3, tig = (rt & 7) >> 1, e = rt & 1;
   int mt = c >> 4, rc = c & 15;
   int gid = rc & 7, chi = rc >> 3;
-  int r = chi + 2 * hi8;
   int lane = gid * 4 + tig;
   BitLoc L;
+  L.bit = vc_pos(vb, mt) + 8 * chi + 16 * e;
   if (vb == 4) {
-    int wi = kk * 8 + mt;
-    L.byte = (wi >> 2) * 512 + lane * 16 + (wi & 3) * 4;
-    L.bit = 4 * r + 16 * e;
+    int w8 = 2 * (mt & 3) + hi8;  // word among the k-step's 8
+    L.byte = (2 * kk + (w8 >> 2)) * 512 + lane * 16 + (w8 & 3) * 4;
   } else {  // 2-bit
-    int mp = mt >> 1, em = mt & 1;
-    L.byte = kk * 512 + lane * 16 + mp * 4;
-    L.bit = 2 * (4 * em + r) + 16 * e;
+    L.byte = kk * 512 + lane * 16 + (2 * (mt & 1) + hi8) * 4;
   }
   return L;
 }

@@ -169,8 +169,11 @@ __global__ void __launch_bounds__(ScanCfg<KB, VB, NT>::NW * 32, 1) scan_kernel(c
         float* row = base + h * kPartStride;
 #pragma unroll
         for (int mt = 0; mt < 8; ++mt) {
-          row[4 + 16 * mt + gid] = acc[mt][e] + zj[mt >> 1][e];
-          row[4 + 16 * mt + gid + 8] = acc[mt][2 + e] + zj[mt >> 1][e];
+          // undo the code position 2^(p - 24) of the tile's value codes
+          const float us = VB == 4 ? ((mt >> 2) ? 1048576.0f : 16777216.0f)
+                                   : (float)(1 << (24 - 2 * (mt >> 1)));
+          row[4 + 16 * mt + gid] = fmaf(acc[mt][e], us, zj[mt >> 1][e]);
+          row[4 + 16 * mt + gid + 8] = fmaf(acc[mt][2 + e], us, zj[mt >> 1][e]);
         }
         if (gid == 0) {
           row[0] = e ? mh1 : mh0;
@@ -374,25 +377,33 @@ __global__ void __launch_bounds__(ScanCfg<KB, VB, NT>::NW * 32, 1) scan_kernel(c
         za0 = za2 = kOneH2;
       }
       mma16816(dz, za0, 0u, za2, 0u, pa, pb);
+      // value codes: one AND per register (fp16 subnormals, position p(mt))
       if constexpr (VB == 4) {
         const uint4 v0 = lds128(r + OFF_VC + (2 * kk) * 512 + lane * 16);
         const uint4 v1 = lds128(r + OFF_VC + (2 * kk + 1) * 512 + lane * 16);
         const uint32_t vw[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+        uint32_t vs[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) vs[i] = vw[i] >> 8;
 #pragma unroll
         for (int mt = 0; mt < 8; ++mt) {
-          uint32_t a[4];
-          unpack4(vw[mt], a);
-          mma16816(acc[mt], a[0], a[1], a[2], a[3], bh[mt >> 1][0], bh[mt >> 1][1]);
+          const int q = mt & 3;
+          const uint32_t mask = 0x000F000Fu << (4 * (mt >> 2));
+          mma16816(acc[mt], vw[2 * q] & mask, vs[2 * q] & mask, vw[2 * q + 1] & mask,
+                   vs[2 * q + 1] & mask, bh[mt >> 1][0], bh[mt >> 1][1]);
         }
       } else {
         const uint4 v = lds128(r + OFF_VC + kk * 512 + lane * 16);
         const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
+        uint32_t vs[4];
 #pragma unroll
-        for (int mp = 0; mp < 4; ++mp) {
-          uint32_t a[8];
-          unpack2(vw[mp], a);
-          mma16816(acc[2 * mp], a[0], a[1], a[2], a[3], bh[mp][0], bh[mp][1]);
-          mma16816(acc[2 * mp + 1], a[4], a[5], a[6], a[7], bh[mp][0], bh[mp][1]);
+        for (int i = 0; i < 4; ++i) vs[i] = vw[i] >> 8;
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+          const int q = mt & 1;
+          const uint32_t mask = 0x00030003u << (2 * (mt >> 1));
+          mma16816(acc[mt], vw[2 * q] & mask, vs[2 * q] & mask, vw[2 * q + 1] & mask,
+                   vs[2 * q + 1] & mask, bh[mt >> 1][0], bh[mt >> 1][1]);
         }
       }
     }
