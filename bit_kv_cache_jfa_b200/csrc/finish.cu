@@ -334,6 +334,37 @@ __device__ __forceinline__ void row_load(const FinishParams& p, int seg, int t, 
   vr = *reinterpret_cast<const uint2*>(vb + off + 4 * lane);
 }
 
+// L2 prefetch of one of the 27 128-byte pieces token t's correction
+// reads: its bf16 K and V rows, and for a quantized token its group's key
+// scales/zeros, its m-tile's key codes, the value-code chunk(s) of its column,
+// its value scales/zeros and the stored running maxima.
+__device__ __forceinline__ void prefetch_part(const FinishParams& p, int seg, int t, int part) {
+  const bool tail = (t & (1 << 30)) != 0;
+  if (part < 4) {
+    const size_t off = tail ? ((size_t)seg * kTail + (t & 0xFFFF)) * kD : ((size_t)seg * p.capacity + t) * kD;
+    const uint16_t* base = (part & 2) ? (tail ? p.tail_v : p.v_exact) : (tail ? p.tail_k : p.k_exact);
+    prefetch_l2(base + off + 64 * (part & 1));
+    return;
+  }
+  if (tail) return;
+  const uint8_t* rec = p.groups + ((size_t)seg * p.ng_cap + (size_t)(t / kKG)) * p.rec_bytes;
+  const int tt = t % kKG, kk = tt >> 4, tgt = (tt & 7) >> 1;
+  if (part < 8) {
+    prefetch_l2(rec + 128 * (part - 4));
+  } else if (part < 16) {
+    const int i = part - 8, mbytes = p.key_bits == 4 ? 1024 : 768;
+    if (128 * i < mbytes) prefetch_l2(rec + off_kc() + kk * mbytes + 128 * i);
+  } else if (part < 24) {
+    const int i = part - 16;
+    if (p.val_bits == 4 || i < 4)
+      prefetch_l2(rec + off_vc(p.key_bits) + (p.val_bits == 4 ? 2 * kk : kk) * 512 + 128 * i);
+  } else if (part < 26) {
+    prefetch_l2(rec + off_vs(p.key_bits) + kk * 128 + tgt * 32 + 512 * (part - 24));
+  } else {
+    prefetch_l2(p.m_used + ((size_t)seg * p.ng_cap + (size_t)(t / kKG)) * kMaxG);
+  }
+}
+
 // The scan's fp16 weights of quantized token t for every head, recomputed
 // from its staged group pieces with the scan's own functions on the same
 // operands (key_sz, bias_mma, scale_pos, q_tilde_col, key_afrag, qk_chain,
@@ -465,20 +496,24 @@ __device__ __forceinline__ void warp_correct(const FinishParams& p, int seg, Tok
   }
 #pragma unroll
   for (int i = 0; i < kWD - 1; ++i) stage_issue(p, seg, i < n ? tok_at(i) : -1, ring[i], lane);
-  uint2 kr = make_uint2(0u, 0u), vr = kr;
+  // exact rows two tokens ahead in registers
+  uint2 kr = make_uint2(0u, 0u), vr = kr, kr1 = kr, vr1 = kr;
   if (n > 0) row_load(p, seg, tok_at(0), lane, kr, vr);
+  if (n > 1) row_load(p, seg, tok_at(1), lane, kr1, vr1);
 #pragma unroll 1
   for (int i = 0; i < n; ++i) {
     const int t = tok_at(i);
     stage_issue(p, seg, i + kWD - 1 < n ? tok_at(i + kWD - 1) : -1, ring[(i + kWD - 1) % kWD], lane);
-    uint2 kn = kr, vn = vr;
-    if (i + 1 < n) row_load(p, seg, tok_at(i + 1), lane, kn, vn);
+    uint2 kr2 = kr1, vr2 = vr1;
+    if (i + 2 < n) row_load(p, seg, tok_at(i + 2), lane, kr2, vr2);
     cp_async_wait<kWD - 1>();
     __syncwarp();
     warp_token<G>(p, t, ring[i % kWD], kr, vr, P, q2, lane, m, l, a);
     __syncwarp();
-    kr = kn;
-    vr = vn;
+    kr = kr1;
+    vr = vr1;
+    kr1 = kr2;
+    vr1 = vr2;
   }
   cp_async_wait<0>();
   __syncwarp();
@@ -517,6 +552,11 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
   const int bb = seg / p.hkv, hh = seg % p.hkv;
 
   // ---- set-up: nothing here is written by the scan
+  {  // this CTA's tail rows into L2 while the set-up runs
+    const int n_mine = p.tail > r ? (p.tail - r + C - 1) / C : 0;
+    for (int i = tid; i < n_mine * 4; i += kFinThreads)
+      prefetch_part(p, seg, (1 << 30) | (r + C * (i >> 2)), i & 3);
+  }
   for (int i = tid; i < G * kD; i += kFinThreads)
     P.qs[i / kD][i % kD] = bf16f(p.q[((size_t)bb * p.H + hh * G + i / kD) * kD + i % kD]);
   for (int i = tid; i < kFinWarps * G * kPartStride; i += kFinThreads)
@@ -549,6 +589,15 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
   bool hist_ok = false;
   // ---- P1 + P2: bin b* from the scan's histogram, then this slice's lists
   if (select) {
+    // the slice's first 16 scores of this thread, loaded together with the
+    // histogram so both round trips overlap
+    const float* S = p.scores + (size_t)seg * p.capacity;
+    float4 v0[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int b0 = lo + 16 * tid + 4 * u;
+      v0[u] = b0 < hi ? ld16<float4>(S + b0) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
     // thread t owns bins [32t, 32t + 32): loaded straight into registers
     const uint32_t* hg = p.hist + (size_t)seg * kScanHistBins + 32 * tid;
     uint32_t hb[32];
@@ -584,13 +633,13 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
     const uint32_t bstar = (uint32_t)s_bin;
     uint32_t base_s = 0, base_t = 0;
     if (hist_ok) {
-      const float* S = p.scores + (size_t)seg * p.capacity;
       for (int t0 = lo; t0 < hi; t0 += 16 * kFinThreads) {
         const int b0 = t0 + 16 * tid;
         float4 v[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u)
-          v[u] = b0 + 4 * u < hi ? ld16<float4>(S + b0 + 4 * u) : make_float4(0.f, 0.f, 0.f, 0.f);
+          v[u] = t0 == lo ? v0[u]
+                          : (b0 + 4 * u < hi ? ld16<float4>(S + b0 + 4 * u) : make_float4(0.f, 0.f, 0.f, 0.f));
         uint32_t keys[16];
         uint32_t ms = 0, mt = 0, ns = 0, nt = 0;
 #pragma unroll
@@ -673,32 +722,36 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
     }
     __syncthreads();
     if (s_mode == 0) {
-      for (int q = 0; q < C; ++q) {
+      // every CTA's ties in one pass (all remote loads in flight together)
+      for (uint32_t i = tid; i < s_tpre[C]; i += kFinThreads) {
+        int q = 0;
+        while (q + 1 < C && s_tpre[q + 1] <= i) ++q;
         const FinPersist* o = cl.map_shared_rank(&PS, q);
-        const uint32_t n = s_tpre[q + 1] - s_tpre[q];
-        for (uint32_t i = tid; i < n; i += kFinThreads) {
-          SS.akey[s_tpre[q] + i] = o->tkey[i];
-          SS.aidx[s_tpre[q] + i] = o->tidx[i];
-        }
+        SS.akey[i] = o->tkey[i - s_tpre[q]];
+        SS.aidx[i] = o->tidx[i - s_tpre[q]];
       }
       __syncthreads();
       n_ch = (uint32_t)k - s_pre[C];
       const uint32_t T = s_tpre[C];
-      if (T <= (uint32_t)kFinThreads) {
+      if (T <= (uint32_t)kFinThreads / 2) {
         // direct ranking: entry i is chosen iff fewer than n_ch entries come
-        // before it in (key descending, index ascending) order
-        uint32_t chosen = 0, my_idx = 0;
-        if ((uint32_t)tid < T) {
-          const uint32_t key = SS.akey[tid];
-          my_idx = SS.aidx[tid];
-          uint32_t rank = 0;
+        // before it in (key descending, index ascending) order; tpe threads
+        // (a power of two) share an entry's comparisons
+        uint32_t tpe = 2;
+        while (tpe < 32 && tpe * 2 * T <= (uint32_t)kFinThreads) tpe *= 2;
+        const uint32_t e = tid / tpe, part = tid % tpe;
+        uint32_t rank = 0, my_idx = 0;
+        if (e < T) {
+          const uint32_t key = SS.akey[e];
+          my_idx = SS.aidx[e];
 #pragma unroll 4
-          for (uint32_t j = 0; j < T; ++j) {
+          for (uint32_t j = part; j < T; j += tpe) {
             const uint32_t k2 = SS.akey[j];
             rank += (k2 > key || (k2 == key && SS.aidx[j] < my_idx)) ? 1u : 0u;
           }
-          chosen = rank < n_ch ? 1u : 0u;
         }
+        for (uint32_t o = 1; o < tpe; o <<= 1) rank += __shfl_xor_sync(kAll, rank, o);
+        const uint32_t chosen = (e < T && part == 0 && rank < n_ch) ? 1u : 0u;
         uint32_t tot;
         const uint32_t pos = block_prefix_excl(chosen, scratch, &tot);
         if (chosen) PS.chtie[pos] = my_idx;  // entries are in index order
@@ -807,6 +860,8 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
     }
     __syncthreads();
     const int n = (int)base;
+    for (int i = tid; i < n * 4; i += kFinThreads)  // the exact rows into L2
+      prefetch_part(p, seg, FC.tok[i >> 2], i & 3);
     const int n_w = n > warp ? (n - warp + kFinWarps - 1) / kFinWarps : 0;
     const int32_t* tl = FC.tok;
     auto chosen_at = [&](int i) { return tl[warp + kFinWarps * i]; };
@@ -845,7 +900,7 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
       w0 = scan_warp_of(x0, W, T);
       w1 = scan_warp_of(x1, W, T);
     }
-    const int ns = (int)(w1 - w0 + 1);
+    const int ns = (int)(w1 - w0 + 1);  // one partial slot per scan warp of the segment
     const int s0 = (int)((long long)ns * r / C), s1 = (int)((long long)ns * (r + 1) / C);
     // rows (slot, head) staged in shared memory a tile at a time, every load
     // of a tile in flight together; thread (channel, half) merges the heads
@@ -865,7 +920,7 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
     const int nrows = (s1 - s0) * G;
     for (int r0 = 0; r0 < nrows; r0 += kTR) {
       const int nr = min(kTR, nrows - r0);
-#pragma unroll 4
+#pragma unroll 8
       for (int i = tid; i < nr * kV; i += kFinThreads) {
         const int row = i / kV, v = i % kV;
         const int gr = r0 + row;

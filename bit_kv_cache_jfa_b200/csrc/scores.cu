@@ -84,15 +84,15 @@ __global__ void __launch_bounds__(ScanCfg<KB, VB, NT>::NW * 32, 1) scan_kernel(c
   const int gid = lane >> 2, tig = lane & 3;
   pdl_wait();
   const long long wg = (long long)blockIdx.x * NW + warp;
-  if (wg >= p.n_warps) return;
   const long long W = p.n_warps, T = p.total;
-  const long long g0 = scan_range_begin(wg, W, T), g1 = scan_range_begin(wg + 1, W, T);
-  if (g0 >= g1) return;
+  const long long g0 = wg < W ? scan_range_begin(wg, W, T) : 0;
+  const long long g1 = wg < W ? scan_range_begin(wg + 1, W, T) : 0;
+  const bool has_work = g0 < g1;  // warp-uniform
 
   uint8_t* ring = smem + (size_t)warp * S * REC;
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + (size_t)NW * S * REC) + warp * S;
   const uint64_t pol = policy_evict_first();
-  if (lane == 0) {
+  if (lane == 0 && has_work) {
 #pragma unroll
     for (int i = 0; i < S; ++i) mbar_init(&bar[i], 1);
     fence_mbar_init();
@@ -110,7 +110,7 @@ __global__ void __launch_bounds__(ScanCfg<KB, VB, NT>::NW * 32, 1) scan_kernel(c
       ++pf_seg;
     }
   };
-  if (lane == 0) {
+  if (lane == 0 && has_work) {
 #pragma unroll
     for (int i = 0; i < S; ++i)
       if (g0 + i < g1) issue_next(i);
@@ -187,6 +187,7 @@ __global__ void __launch_bounds__(ScanCfg<KB, VB, NT>::NW * 32, 1) scan_kernel(c
   int g = (int)(g0 - seg * p.ng);
   int st = 0;
   uint32_t par = 0;
+  bool failed = false;
   for (long long gi = g0; gi < g1; ++gi) {
     if (seg != cur) {
       if (cur >= 0) flush(cur);
@@ -207,7 +208,8 @@ __global__ void __launch_bounds__(ScanCfg<KB, VB, NT>::NW * 32, 1) scan_kernel(c
         }
       }
       __syncwarp();
-      return;
+      failed = true;
+      break;
     }
     const uint8_t* r = ring + st * REC;
 
@@ -419,7 +421,8 @@ __global__ void __launch_bounds__(ScanCfg<KB, VB, NT>::NW * 32, 1) scan_kernel(c
       ++seg;
     }
   }
-  flush(cur);
+  if (has_work && !failed) flush(cur);
+
   // No explicit launch_dependents: the dependent kernel is released as the
   // scan's CTAs exit, so its thread-block clusters find whole SMs free.
 }
