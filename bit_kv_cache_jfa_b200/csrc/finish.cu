@@ -584,6 +584,33 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
   pdl_wait();
   pdl_launch_dependents();
 
+  // ---- P5a (loads): this CTA's share of the scan's split partials, every
+  // head: when the rows fit beside the selection buffers they are copied now
+  // (cp.async) and merged after the selection, so their latency hides
+  // behind it; else they are staged tile by tile then.
+    long long w0 = 0, w1 = -1;
+    if (p.ng > 0) {
+      const long long T = p.scan_total, W = p.scan_warps;
+      const long long x0 = (long long)seg * p.ng, x1 = x0 + p.ng - 1;
+      w0 = scan_warp_of(x0, W, T);
+      w1 = scan_warp_of(x1, W, T);
+    }
+    const int ns = (int)(w1 - w0 + 1);  // one partial slot per scan warp of the segment
+    const int s0 = (int)((long long)ns * r / C), s1 = (int)((long long)ns * (r + 1) / C);
+    constexpr int kV = kPartStride / 4;  // float4 per row
+    const int nrows = (s1 - s0) * G;
+    float* early = reinterpret_cast<float*>(U + sizeof(FinSelect));
+    constexpr int kEarlyRows = (int)((sizeof(FinCorr) - sizeof(FinSelect)) / (kPartStride * sizeof(float)));
+    const bool early_ok = nrows <= kEarlyRows;
+    if (early_ok) {
+      for (int i = tid; i < nrows * kV; i += kFinThreads) {
+        const int row = i / kV, v = i % kV;
+        cp_async16(early + row * kPartStride + 4 * v,
+                   p.scan_part + ((size_t)(w0 + s0 + row / G + seg) * G + row % G) * kPartStride + 4 * v);
+      }
+    }
+    cp_async_commit();
+
   const bool select = SELECT && k < nq;
   const int lo = min(nq, r * p.slice), hi = min(nq, lo + p.slice);
   bool hist_ok = false;
@@ -820,6 +847,70 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
       *reinterpret_cast<uint4*>(hg + i) = make_uint4(0u, 0u, 0u, 0u);
   }
 
+  // ---- P5a (merge)
+  {
+    // rows (slot, head) staged in shared memory a tile at a time, every load
+    // of a tile in flight together; thread (channel, half) merges the heads
+    // j = half, half + 2, ... online
+    const int c = tid & (kD - 1), half = tid >> 7;
+    constexpr int kH2 = (G + 1) / 2;
+    float mrun[kH2], lrun[kH2], arun[kH2];
+#pragma unroll
+    for (int i = 0; i < kH2; ++i) {
+      mrun[i] = -INFINITY;
+      lrun[i] = 0.f;
+      arun[i] = 0.f;
+    }
+    float* tile = reinterpret_cast<float*>(U);
+    constexpr int kTR = (int)(sizeof(FinCorr) / (kPartStride * sizeof(float)));
+    if (early_ok) {
+      cp_async_wait<0>();
+      __syncthreads();
+    }
+    for (int r0 = 0; r0 < nrows; r0 += (early_ok ? nrows : kTR)) {
+      const int nr = early_ok ? nrows : min(kTR, nrows - r0);
+      if (early_ok) tile = early;
+#pragma unroll 8
+      for (int i = tid; i < (early_ok ? 0 : nr * kV); i += kFinThreads) {
+        const int row = i / kV, v = i % kV;
+        const int gr = r0 + row;
+        const float* src = p.scan_part + ((size_t)(w0 + s0 + gr / G + seg) * G + gr % G) * kPartStride;
+        reinterpret_cast<float4*>(tile + row * kPartStride)[v] = ld16<float4>(src + 4 * v);
+      }
+      __syncthreads();
+#pragma unroll
+      for (int i = 0; i < kH2; ++i) {
+        const int j = half + 2 * i;
+        if (j < G) {
+#pragma unroll 1
+          for (int row = (j - r0 % G + G) % G; row < nr; row += G) {
+            const float* tr = tile + row * kPartStride;
+            const float rl = tr[1];
+            if (rl > 0.f) {
+              const float mn = fmaxf(mrun[i], tr[0]);
+              const float s0f = lrun[i] > 0.f ? exp2f(mrun[i] - mn) : 0.f;
+              const float s1f = exp2f(tr[0] - mn);
+              lrun[i] = lrun[i] * s0f + rl * s1f;
+              arun[i] = arun[i] * s0f + tr[4 + c] * s1f;
+              mrun[i] = mn;
+            }
+          }
+        }
+      }
+      __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < kH2; ++i) {
+      const int j = half + 2 * i;
+      if (j < G) {
+        P.sp[j][4 + c] = arun[i];
+        if (c == 0) {
+          P.sp[j][0] = lrun[i] > 0.f ? mrun[i] : -INFINITY;
+          P.sp[j][1] = lrun[i];
+        }
+      }
+    }
+  }
   // ---- P4: correction of an even share of the chosen set: the token list
   // first (compacted, in shared memory), then a warp per token
   {
@@ -891,76 +982,6 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
     }
   }
 
-  // ---- P5a: this CTA's share of the scan's split partials, every head
-  {
-    long long w0 = 0, w1 = -1;
-    if (p.ng > 0) {
-      const long long T = p.scan_total, W = p.scan_warps;
-      const long long x0 = (long long)seg * p.ng, x1 = x0 + p.ng - 1;
-      w0 = scan_warp_of(x0, W, T);
-      w1 = scan_warp_of(x1, W, T);
-    }
-    const int ns = (int)(w1 - w0 + 1);  // one partial slot per scan warp of the segment
-    const int s0 = (int)((long long)ns * r / C), s1 = (int)((long long)ns * (r + 1) / C);
-    // rows (slot, head) staged in shared memory a tile at a time, every load
-    // of a tile in flight together; thread (channel, half) merges the heads
-    // j = half, half + 2, ... online
-    const int c = tid & (kD - 1), half = tid >> 7;
-    constexpr int kH2 = (G + 1) / 2;
-    float mrun[kH2], lrun[kH2], arun[kH2];
-#pragma unroll
-    for (int i = 0; i < kH2; ++i) {
-      mrun[i] = -INFINITY;
-      lrun[i] = 0.f;
-      arun[i] = 0.f;
-    }
-    float* tile = reinterpret_cast<float*>(U);
-    constexpr int kTR = (int)(sizeof(FinCorr) / (kPartStride * sizeof(float)));
-    constexpr int kV = kPartStride / 4;  // float4 per row
-    const int nrows = (s1 - s0) * G;
-    for (int r0 = 0; r0 < nrows; r0 += kTR) {
-      const int nr = min(kTR, nrows - r0);
-#pragma unroll 8
-      for (int i = tid; i < nr * kV; i += kFinThreads) {
-        const int row = i / kV, v = i % kV;
-        const int gr = r0 + row;
-        const float* src = p.scan_part + ((size_t)(w0 + s0 + gr / G + seg) * G + gr % G) * kPartStride;
-        reinterpret_cast<float4*>(tile + row * kPartStride)[v] = ld16<float4>(src + 4 * v);
-      }
-      __syncthreads();
-#pragma unroll
-      for (int i = 0; i < kH2; ++i) {
-        const int j = half + 2 * i;
-        if (j < G) {
-#pragma unroll 1
-          for (int row = (j - r0 % G + G) % G; row < nr; row += G) {
-            const float* tr = tile + row * kPartStride;
-            const float rl = tr[1];
-            if (rl > 0.f) {
-              const float mn = fmaxf(mrun[i], tr[0]);
-              const float s0f = lrun[i] > 0.f ? exp2f(mrun[i] - mn) : 0.f;
-              const float s1f = exp2f(tr[0] - mn);
-              lrun[i] = lrun[i] * s0f + rl * s1f;
-              arun[i] = arun[i] * s0f + tr[4 + c] * s1f;
-              mrun[i] = mn;
-            }
-          }
-        }
-      }
-      __syncthreads();
-    }
-#pragma unroll
-    for (int i = 0; i < kH2; ++i) {
-      const int j = half + 2 * i;
-      if (j < G) {
-        P.sp[j][4 + c] = arun[i];
-        if (c == 0) {
-          P.sp[j][0] = lrun[i] > 0.f ? mrun[i] : -INFINITY;
-          P.sp[j][1] = lrun[i];
-        }
-      }
-    }
-  }
   cl.sync();
 
   // ---- P5b: CTA r owns heads j = r, r + C, ...: merge the C CTAs' scan
