@@ -424,11 +424,41 @@ __device__ __forceinline__ void warp_token(const FinishParams& p, int t, const W
                        __uint_as_float(kr.y << 16), __uint_as_float(kr.y & 0xFFFF0000u)};
   const float vf[4] = {__uint_as_float(vr.x << 16), __uint_as_float(vr.x & 0xFFFF0000u),
                        __uint_as_float(vr.y << 16), __uint_as_float(vr.y & 0xFFFF0000u)};
+  // exact logits: per-lane partial dots, a reduce-scatter over the lanes
+  // (each level halves the values a lane carries), then every head's total
+  // gathered from the lane that holds it
+  constexpr int GP = G <= 1 ? 1 : (G <= 2 ? 2 : (G <= 4 ? 4 : 8));
+  constexpr int LG = GP == 1 ? 0 : (GP == 2 ? 1 : (GP == 4 ? 2 : 3));
+  float v[GP];
+#pragma unroll
+  for (int j = 0; j < GP; ++j) {
+    if (j < G) {
+      const float4 qv = *reinterpret_cast<const float4*>(&P.qs[j][4 * lane]);
+      v[j] = fmaf(qv.x, kf[0], fmaf(qv.y, kf[1], fmaf(qv.z, kf[2], qv.w * kf[3])));
+    } else {
+      v[j] = 0.f;
+    }
+  }
+#pragma unroll
+  for (int L = 0; L < LG; ++L) {
+    const int o = 16 >> L, half = GP >> (L + 1);
+    const bool up = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < half; ++i) {
+      const float keep = up ? v[half + i] : v[i];
+      const float send = up ? v[i] : v[half + i];
+      v[i] = keep + __shfl_xor_sync(kAll, send, o);
+    }
+  }
+#pragma unroll
+  for (int o = 16 >> LG; o > 0; o >>= 1) v[0] += __shfl_xor_sync(kAll, v[0], o);
   float se[G];
 #pragma unroll
   for (int j = 0; j < G; ++j) {
-    const float4 qv = *reinterpret_cast<const float4*>(&P.qs[j][4 * lane]);
-    se[j] = warp_sum(fmaf(qv.x, kf[0], fmaf(qv.y, kf[1], fmaf(qv.z, kf[2], qv.w * kf[3])))) * p.kappa;
+    int src = 0;
+#pragma unroll
+    for (int L = 0; L < LG; ++L) src += ((j >> (LG - 1 - L)) & 1) * (16 >> L);
+    se[j] = __shfl_sync(kAll, v[0], src) * p.kappa;
   }
   const bool qt = tok_quant(t);
   uint32_t ph[G];
@@ -456,24 +486,32 @@ __device__ __forceinline__ void warp_token(const FinishParams& p, int t, const W
       }
     }
   }
+  // the partial's frame m moves only when a new term would exceed it by more
+  // than 2^8 (warp-uniform test), so most tokens need no rescale
 #pragma unroll
   for (int j = 0; j < G; ++j) {
     const float mu = qt ? S.mu[j] : -INFINITY;
-    const float mn = fmaxf(fmaxf(m[j], se[j]), mu);
-    const float al = exp2f(m[j] - mn);  // 0 while the partial is empty (m = -inf)
-    const float pe = exp2f(se[j] - mn);
-    l[j] = fmaf(l[j], al, pe);
+    const float cand = fmaxf(se[j], mu);
+    if (cand > m[j] + 8.f) {
+      const float al = exp2f(m[j] - cand);  // 0 while the partial is empty (m = -inf)
+      l[j] *= al;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) a[j][i] = fmaf(a[j][i], al, pe * vf[i]);
-    if (qt) {
-      const float f = exp2f(mu - mn);
-      const uint16_t phj = (uint16_t)ph[j];
-      const float pf = h2f(phj), w = h2f(h_mul_rn(phj, svb));
-      l[j] -= pf * f;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) a[j][i] -= f * fmaf(w, code[i], pf * zv);
+      for (int i = 0; i < 4; ++i) a[j][i] *= al;
+      m[j] = cand;
     }
-    m[j] = mn;
+    const float pe = exp2f(se[j] - m[j]);
+    l[j] += pe;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) a[j][i] = fmaf(pe, vf[i], a[j][i]);
+    if (qt) {
+      const float f = exp2f(mu - m[j]);
+      const uint16_t phj = (uint16_t)ph[j];
+      const float pf = h2f(phj) * f, w = h2f(h_mul_rn(phj, svb)) * f;
+      const float zt = pf * zv;
+      l[j] -= pf;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[j][i] -= fmaf(w, code[i], zt);
+    }
   }
 }
 
