@@ -31,7 +31,7 @@ METRIC = "decode attn: cached KV tokens/s on 1 B200 and % of HBM roofline (K3V2,
 FLUSH_BYTES = 256 << 20   # > 126 MB L2
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
@@ -43,7 +43,12 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-clocks", action="store_true")
-    return ap.parse_args()
+    return ap.parse_args(argv)
+
+
+def workload_of(args):
+    import workloads as W
+    return W.WORKLOADS[args.workload or W.DEFAULT_WORKLOAD]
 
 
 # ---------------------------------------------------------------------------
@@ -426,8 +431,7 @@ def run_jfa(args, w):
 
 def main():
     args = parse()
-    import workloads as W
-    w = W.WORKLOADS[args.workload or W.DEFAULT_WORKLOAD]
+    w = workload_of(args)
     if args.impl == "reference":
         return run_reference(args, w)
     return run_jfa(args, w)
