@@ -145,11 +145,40 @@ def recorded_traffic(workload: str):
 # clocks during the timed region
 # ---------------------------------------------------------------------------
 class Clocks:
+    """SM clock and clock-event reasons sampled during the timed region: NVML
+    polled from a thread every ~2 ms (read-only queries), else nvidia-smi."""
+
+    # NVML clock-event reason bits
+    REASONS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+               "hw_thermal_slowdown": 0x40}
+
     def __init__(self, index: int, enabled: bool):
-        self.proc = None
-        self.path = None
+        self.samples, self.max_mhz, self.reasons = [], 0.0, set()
+        self.thread = self.proc = self.path = None
+        self.stop_flag = False
         if not enabled:
             return
+        try:
+            import threading
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+
+            def poll():
+                while not self.stop_flag:
+                    self.samples.append(float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)))
+                    bits = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                    for n, v in self.REASONS.items():
+                        if bits & v:
+                            self.reasons.add(n)
+                    time.sleep(0.002)
+
+            self.thread = threading.Thread(target=poll, daemon=True)
+            self.thread.start()
+            return
+        except Exception:
+            self.thread = None
         fd, self.path = tempfile.mkstemp(prefix="jfa_clocks_", suffix=".csv")
         os.close(fd)
         q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -158,12 +187,20 @@ class Clocks:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={index}", f"--query-gpu={q}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
 
     def stop(self):
+        if self.thread is not None:
+            self.stop_flag = True
+            self.thread.join(timeout=5)
+            if not self.samples:
+                return None
+            return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                    "reasons": sorted(self.reasons), "samples": len(self.samples),
+                    "source": "nvml"}
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -190,7 +227,7 @@ class Clocks:
         if not sm:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "source": "nvidia-smi"}
 
 
 # ---------------------------------------------------------------------------
@@ -345,19 +382,19 @@ def run_jfa(args, w):
     ms = statistics.mean(step_ms)
     ms_max = max_over_ranks(ms, world, dev)
 
-    # the scan kernel alone (roofline): its own launches, L2 flushed before each
+    # the scan kernel alone (roofline): its own launches, L2 flushed before each,
+    # on a workspace of its own (scan-only launches leave the selection
+    # histogram for a finishing kernel to consume)
+    ws_scan = jfa.Workspace(cache, w.topk, device=dev)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     for i in range(args.steps):
         flush.zero_()
         evs[i][0].record(stream)
-        _lib.check(_lib.jfa_decode_scores(geom, cst, q, scale, ws.buf, sp), "scores")
+        _lib.check(_lib.jfa_decode_scores(geom, cst, q, scale, ws_scan.buf, sp), "scores")
         evs[i][1].record(stream)
     torch.cuda.synchronize()
     scan_avg = statistics.mean(evs[i][0].elapsed_time(evs[i][1]) for i in range(args.steps))
-    # scan-only launches leave the selection histogram uncleared; one full step
-    # consumes and clears it before the end-to-end loop
-    step()
-    torch.cuda.synchronize()
+    del ws_scan
 
     # end to end through the public API: q from pinned host in, out back to pinned host
     q_host = q.cpu().pin_memory()
