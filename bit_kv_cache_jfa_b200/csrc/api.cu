@@ -38,7 +38,7 @@ int workspace_layout(const jfa_geom& g, int max_topk, jfa_workspace_layout* out)
   L.off_partials = off;
   off = align_up(off + (size_t)L.partial_slots * G * kPartStride * sizeof(float), 256);
   L.off_mused = off;
-  off = align_up(off + n_seg * (size_t)(g.capacity / kKG) * kMaxG * sizeof(float), 256);
+  off = align_up(off + n_seg * (size_t)(g.capacity / kKG) * 2 * kMaxG * sizeof(float), 256);
   L.off_scan_hist = off;
   off = align_up(off + n_seg * kScanHistBins * sizeof(uint32_t), 256);
   L.off_hist = off;

@@ -44,7 +44,7 @@ struct FinishParams {
   const uint16_t* q;
   const float* scores;     // [n_seg][capacity]
   const float* scan_part;  // per scan warp and segment: [slot][G][kPartStride]
-  const float* m_used;     // [n_seg][ng_cap][8]
+  const float* m_used;     // [n_seg][ng_cap][16]: the scan's running maxima and biases
   uint32_t* hist;          // [n_seg][kScanHistBins], zeroed here after use
   uint32_t* glists;        // [n_seg][C][slice] chosen lists of the fallback
   const int32_t* idx_in;   // given index sets (no selection), [n_seg][k]
@@ -90,7 +90,7 @@ struct WStage {
   uint8_t kcode[1024]; // key codes of its 16-token m-tile, in lane order
   uint8_t vp[256];     // value-code pieces holding its column (8 or 16 x 16 B)
   uint8_t vsz[64];     // its value scales (32 B block) and zeros (32 B block)
-  float mu[kMaxG];     // the scan's running maxima of its group
+  float mu[2 * kMaxG]; // the scan's running maxima (8) and biases (8) of its group
 };
 constexpr int kTokCap = 1024;  // tokens listed per correction round
 struct FinCorr {
@@ -316,9 +316,9 @@ __device__ __forceinline__ void stage_issue(const FinishParams& p, int seg, int 
     if (lane < 4)
       cp_async16(S.vsz + lane * 16,
                  rec + off_vs(p.key_bits) + kk * 128 + tgt * 32 + (lane & 1) * 16 + (lane >> 1) * 512);
-    if (lane < 2)
+    if (lane < 4)
       cp_async16(reinterpret_cast<uint8_t*>(S.mu) + lane * 16,
-                 p.m_used + ((size_t)seg * p.ng_cap + (size_t)(t / kKG)) * kMaxG + lane * 4);
+                 p.m_used + ((size_t)seg * p.ng_cap + (size_t)(t / kKG)) * (2 * kMaxG) + lane * 4);
   }
   cp_async_commit();
 }
@@ -361,15 +361,15 @@ __device__ __forceinline__ void prefetch_part(const FinishParams& p, int seg, in
   } else if (part < 26) {
     prefetch_l2(rec + off_vs(p.key_bits) + kk * 128 + tgt * 32 + 512 * (part - 24));
   } else {
-    prefetch_l2(p.m_used + ((size_t)seg * p.ng_cap + (size_t)(t / kKG)) * kMaxG);
+    prefetch_l2(p.m_used + ((size_t)seg * p.ng_cap + (size_t)(t / kKG)) * (2 * kMaxG));
   }
 }
 
 // The scan's fp16 weights of quantized token t for every head, recomputed
 // from its staged group pieces with the scan's own functions on the same
-// operands (key_sz, bias_mma, scale_pos, q_tilde_col, key_afrag, qk_chain,
-// approx_logit, approx_weight); ph[j] = fp16 bits of head j's weight, on all
-// lanes.  q2[n]: the lane's q of head (gid >> 1) + 4n, as the scan holds it.
+// operands (key_sz, scale_pos, q_tilde_col, key_afrag, qk_chain, approx_logit,
+// approx_weight; the group bias as the scan stored it); ph[j] = fp16 bits of
+// head j's weight, on all lanes.  q2[n]: the lane's q of head (gid >> 1) + 4n, as the scan holds it.
 template <int KB, int G>
 __device__ __forceinline__ void replay_weights_t(const FinishParams& p, int t, const WStage& S,
                                                  const uint32_t (&q2)[2][16], int lane,
@@ -380,8 +380,9 @@ __device__ __forceinline__ void replay_weights_t(const FinishParams& p, int t, c
   uint32_t sk[16], zk[16], sf[16], qb[NT][16];
   float bk[NT];
   key_sz(S.ksz, tig, sk, zk);
+  // the group bias of head tig + 4n exactly as the scan computed and stored it
 #pragma unroll
-  for (int n = 0; n < NT; ++n) bk[n] = bias_mma(q2[n], zk, p.kappa);
+  for (int n = 0; n < NT; ++n) bk[n] = S.mu[kMaxG + (tig + 4 * n < G ? tig + 4 * n : 0)];
   scale_pos<KB>(sk, sf);
 #pragma unroll
   for (int n = 0; n < NT; ++n) q_tilde_col(q2[n], sf, (gid & 1) != 0, qb[n]);

@@ -39,7 +39,7 @@ struct ScanParams {
   const uint16_t* q;
   float* scores;
   float* partials;
-  float* m_used;    // [n_seg][ng_cap][8]
+  float* m_used;    // [n_seg][ng_cap][16]: running maxima (8) and biases (8) per head
   uint32_t* hist;   // [n_seg][kScanHistBins]
   uint32_t* flag;
   long long total;  // n_seg * ng
@@ -293,11 +293,16 @@ __global__ void __launch_bounds__(ScanCfg<KB, VB, NT>::NW * 32, 1) scan_kernel(c
 #pragma unroll
       for (int n = 0; n < NT; ++n) m_run[n] = m_new[n];
     }
-    // the maximum this group's weights are taken against, for the correction
+    // the maximum this group's weights are taken against, and the group's bias
+    // (kappa * q . m), for the correction's replay
     if (gid == 0) {
 #pragma unroll
       for (int n = 0; n < NT; ++n)
-        if (hv[n]) p.m_used[((size_t)seg * p.ng_cap + g) * kMaxG + tig + 4 * n] = m_run[n];
+        if (hv[n]) {
+          float* mrec = p.m_used + ((size_t)seg * p.ng_cap + g) * (2 * kMaxG);
+          mrec[tig + 4 * n] = m_run[n];
+          mrec[kMaxG + tig + 4 * n] = bk[n];
+        }
     }
 
     // ---- selection score S = max over heads; lane ends with m-tile tig,
