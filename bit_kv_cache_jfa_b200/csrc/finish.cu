@@ -32,8 +32,6 @@ constexpr int kFinMaxC = 8;
 constexpr int kLCap = 1024;   // sure / tie list entries per CTA
 constexpr int kTCap = 1024;   // gathered tie entries
 constexpr int kRefBins = 2048;
-constexpr int kWD = 3;        // cp.async stages per warp (tokens in flight)
-constexpr int kFinWarps = kFinThreads / 32;
 
 struct FinishParams {
   const uint8_t* groups;
@@ -72,10 +70,8 @@ struct FinPersist {
 // so l may be negative.
 template <int G>
 struct FinParts {
-  float qs[G][kD];
-  float run[G][kPartStride];   // this CTA's exact-minus-removed partial
+  float run[G][kPartStride];   // this CTA's exact-minus-removed partial (frame, mass, acc)
   float sp[G][kPartStride];    // this CTA's share of the scan partials
-  float wp[kFinWarps][G][kPartStride];  // per-warp partials
 };
 // Shared-memory histograms store bin b at hpad(b) = b + b/32, so threads
 // that each read a contiguous run of bins hit distinct banks.
@@ -84,18 +80,39 @@ struct FinSelect {
   uint32_t hist[kRefBins + kRefBins / 32];
   uint32_t akey[kTCap], aidx[kTCap];
 };
-// Record pieces of one quantized token, staged by cp.async.
-struct WStage {
-  uint8_t ksz[512];    // key scales / zeros of its group
-  uint8_t kcode[1024]; // key codes of its 16-token m-tile, in lane order
-  uint8_t vp[256];     // value-code pieces holding its column (8 or 16 x 16 B)
-  uint8_t vsz[64];     // its value scales (32 B block) and zeros (32 B block)
-  float mu[2 * kMaxG]; // the scan's running maxima (8) and biases (8) of its group
+// One token of a correction batch: its record pieces (cp.async) and its
+// exact bf16 K and V rows.  The 16-byte pad puts the rows of consecutive
+// tokens 4 banks apart, so the tensor-core operand loads are conflict-free.
+struct TokStage {
+  uint8_t ksz[512];      // key scales / zeros of its group
+  uint8_t kcode[128];    // key-code words of the 4 lanes holding its m-tile row
+  uint8_t vp[256];       // value-code pieces holding its column (8 or 16 x 16 B)
+  uint8_t vsz[64];       // its value scales (32 B block) and zeros (32 B block)
+  float mu[2 * kMaxG];   // the scan's running maxima (8) and biases (8) of its group
+  uint16_t krow[kD];     // bf16 K row
+  uint16_t vrow[kD];     // bf16 V row
+  uint8_t pad[16];
 };
+static_assert(sizeof(TokStage) == 1552, "token stage layout");
 constexpr int kTokCap = 1024;  // tokens listed per correction round
+constexpr int kBT = 16;        // tokens per correction batch (one mma k-step)
+// Correction batches, double-buffered: batch b + 1 is staged while batch b
+// is computed.  The weights are bf16 triples (hi, mid, lo: 24 significant
+// bits), head-major (the B operands of the value MMAs).
+struct FinBatchT {
+  TokStage st[2][kBT];
+  int tok[2][kBT];
+  uint16_t bex[3][kMaxG][kBT];      // exact weights
+  uint16_t brem[3][4][kMaxG][kBT];  // minus the removed weights per 32-channel group
+  uint16_t bpf[2][kMaxG][kBT];      // removed masses 2^(m_used - m) p as fp16 (hi, lo)
+  float se[kBT][kMaxG];             // exact logits (log2 units)
+  uint16_t ph[kBT][kMaxG];          // replayed fp16 weights of the scan
+  float alpha[kMaxG];               // frame move of this batch per head
+  float zsum[kMaxG][4];             // removed zero-point terms per head and channel group (final)
+};
 struct FinCorr {
-  WStage st[kFinWarps][kWD];
-  int32_t tok[kTokCap];
+  FinBatchT b;
+  int32_t tok[kTokCap + kTail];
 };
 template <int G>
 constexpr size_t fin_smem_bytes() {
@@ -291,47 +308,39 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-// Stage the record pieces of token t (one commit group per lane, possibly empty).
-__device__ __forceinline__ void stage_issue(const FinishParams& p, int seg, int t, WStage& S,
-                                            int lane) {
-  if (tok_quant(t)) {
-    const uint8_t* rec = p.groups + ((size_t)seg * p.ng_cap + (size_t)(t / kKG)) * p.rec_bytes;
-    const int tt = t % kKG, kk = tt >> 4, tgt = (tt & 7) >> 1;
-    cp_async16(S.ksz + lane * 16, rec + lane * 16);
-    if (p.key_bits == 4) {
-      const uint8_t* src = rec + off_kc() + kk * 1024 + lane * 32;
-      cp_async16(S.kcode + lane * 32, src);
-      cp_async16(S.kcode + lane * 32 + 16, src + 16);
-    } else {
-      const uint8_t* src = rec + off_kc() + kk * 768 + lane * 24;
-      cp_async8(S.kcode + lane * 24, src);
-      cp_async8(S.kcode + lane * 24 + 8, src + 8);
-      cp_async8(S.kcode + lane * 24 + 16, src + 16);
+// Record pieces of quantized token t into S: piece i (0..63) of the token
+// is one 16-byte cp.async; the caller commits.
+__device__ __forceinline__ void stage_piece(const FinishParams& p, int seg, int t, TokStage& S, int i) {
+  const uint8_t* rec = p.groups + ((size_t)seg * p.ng_cap + (size_t)(t / kKG)) * p.rec_bytes;
+  const int tt = t % kKG, kk = tt >> 4, row = tt & 7, tgt = (tt & 7) >> 1;
+  if (i < 32) {
+    cp_async16(S.ksz + 16 * i, rec + 16 * i);
+  } else if (i < 40) {
+    const int j = i - 32;
+    if (p.key_bits == 4) cp_async16(S.kcode + 16 * j, rec + off_kc() + kk * 1024 + row * 128 + 16 * j);
+    else if (j < 6) cp_async16(S.kcode + 16 * j, rec + off_kc() + kk * 768 + row * 96 + 16 * j);
+  } else if (i < 56) {
+    const int j = i - 40;
+    if (p.val_bits == 4 || j < 8) {
+      const int chunk = p.val_bits == 4 ? 2 * kk + (j >> 3) : kk;
+      cp_async16(S.vp + 16 * j, rec + off_vc(p.key_bits) + chunk * 512 + ((j & 7) * 4 + tgt) * 16);
     }
-    const int vslots = p.val_bits == 4 ? 16 : 8;
-    if (lane < vslots) {
-      const int chunk = p.val_bits == 4 ? 2 * kk + (lane >> 3) : kk;
-      cp_async16(S.vp + lane * 16, rec + off_vc(p.key_bits) + chunk * 512 + ((lane & 7) * 4 + tgt) * 16);
-    }
-    if (lane < 4)
-      cp_async16(S.vsz + lane * 16,
-                 rec + off_vs(p.key_bits) + kk * 128 + tgt * 32 + (lane & 1) * 16 + (lane >> 1) * 512);
-    if (lane < 4)
-      cp_async16(reinterpret_cast<uint8_t*>(S.mu) + lane * 16,
-                 p.m_used + ((size_t)seg * p.ng_cap + (size_t)(t / kKG)) * (2 * kMaxG) + lane * 4);
+  } else if (i < 60) {
+    const int j = i - 56;
+    cp_async16(S.vsz + 16 * j, rec + off_vs(p.key_bits) + kk * 128 + tgt * 32 + (j & 1) * 16 + (j >> 1) * 512);
+  } else {
+    const int j = i - 60;
+    cp_async16(reinterpret_cast<uint8_t*>(S.mu) + 16 * j,
+               p.m_used + ((size_t)seg * p.ng_cap + (size_t)(t / kKG)) * (2 * kMaxG) + 4 * j);
   }
-  cp_async_commit();
 }
 
-// Exact bf16 row pieces of token t for lane l: channels 4l..4l+3 of K and V.
-__device__ __forceinline__ void row_load(const FinishParams& p, int seg, int t, int lane, uint2& kr,
-                                         uint2& vr) {
-  const size_t off = (t & (1 << 30)) ? ((size_t)seg * kTail + (t & 0xFFFF)) * kD
-                                     : ((size_t)seg * p.capacity + t) * kD;
-  const uint16_t* kb = (t & (1 << 30)) ? p.tail_k : p.k_exact;
-  const uint16_t* vb = (t & (1 << 30)) ? p.tail_v : p.v_exact;
-  kr = *reinterpret_cast<const uint2*>(kb + off + 4 * lane);
-  vr = *reinterpret_cast<const uint2*>(vb + off + 4 * lane);
+// 16-byte piece `piece` (0..15) of token t's exact K (v = false) or V row.
+__device__ __forceinline__ uint4 row_piece(const FinishParams& p, int seg, int t, bool v, int piece) {
+  const bool tail = (t & (1 << 30)) != 0;
+  const size_t off = tail ? ((size_t)seg * kTail + (t & 0xFFFF)) * kD : ((size_t)seg * p.capacity + t) * kD;
+  const uint16_t* base = v ? (tail ? p.tail_v : p.v_exact) : (tail ? p.tail_k : p.k_exact);
+  return ld16<uint4>(base + off + 8 * piece);
 }
 
 // L2 prefetch of one of the 27 128-byte pieces token t's correction
@@ -369,11 +378,12 @@ __device__ __forceinline__ void prefetch_part(const FinishParams& p, int seg, in
 // from its staged group pieces with the scan's own functions on the same
 // operands (key_sz, scale_pos, q_tilde_col, key_afrag, qk_chain, approx_logit,
 // approx_weight; the group bias as the scan stored it); ph[j] = fp16 bits of
-// head j's weight, on all lanes.  q2[n]: the lane's q of head (gid >> 1) + 4n, as the scan holds it.
+// head j's weight, written by the lane whose MMA row and column hold it.
+// q2[n]: the lane's q of head (gid >> 1) + 4n, as the scan holds it.
 template <int KB, int G>
-__device__ __forceinline__ void replay_weights_t(const FinishParams& p, int t, const WStage& S,
+__device__ __forceinline__ void replay_weights_t(const FinishParams& p, int t, const TokStage& S,
                                                  const uint32_t (&q2)[2][16], int lane,
-                                                 uint32_t ph[G]) {
+                                                 uint16_t* ph) {
   constexpr int NT = G > 4 ? 2 : 1;
   const int gid = lane >> 2, tig = lane & 3;
   const int tt = t % kKG, row = tt & 7, rr = (tt >> 3) & 1;
@@ -386,185 +396,319 @@ __device__ __forceinline__ void replay_weights_t(const FinishParams& p, int t, c
   scale_pos<KB>(sk, sf);
 #pragma unroll
   for (int n = 0; n < NT; ++n) q_tilde_col(q2[n], sf, (gid & 1) != 0, qb[n]);
+  // only row `row` of the m-tile is staged; the other rows' codes are zero
+  // (an MMA output row depends on its own A row alone)
   uint32_t w[KeyPos<KB>::WORDS];
-  const uint32_t* kw = reinterpret_cast<const uint32_t*>(S.kcode + lane * 4 * KeyPos<KB>::WORDS);
+  const uint32_t* kw = reinterpret_cast<const uint32_t*>(S.kcode + tig * 4 * KeyPos<KB>::WORDS);
 #pragma unroll
-  for (int i = 0; i < KeyPos<KB>::WORDS; ++i) w[i] = kw[i];
+  for (int i = 0; i < KeyPos<KB>::WORDS; ++i) w[i] = gid == row ? kw[i] : 0u;
   uint32_t a[16][2];
   key_afrag<KB>(w, a);
   const float kappa_u = p.kappa * KeyPos<KB>::unscale;
-  uint32_t mine[NT];
 #pragma unroll
   for (int n = 0; n < NT; ++n) {
     float d[4];
     qk_chain(a, qb[n], d);
     const int h = tig + 4 * n;
-    mine[n] = (gid == row && h < G)
-                  ? f2h_rn(approx_weight(approx_logit(d, rr, kappa_u, bk[n]), S.mu[h]))
-                  : 0u;
+    if (gid == row && h < G) ph[h] = f2h_rn(approx_weight(approx_logit(d, rr, kappa_u, bk[n]), S.mu[h]));
   }
-#pragma unroll
-  for (int j = 0; j < G; ++j) ph[j] = __shfl_sync(kAll, mine[j >> 2], row * 4 + (j & 3));
 }
 template <int G>
-__device__ __forceinline__ void replay_weights(const FinishParams& p, int t, const WStage& S,
+__device__ __forceinline__ void replay_weights(const FinishParams& p, int t, const TokStage& S,
                                                const uint32_t (&q2)[2][16], int lane,
-                                               uint32_t ph[G]) {
+                                               uint16_t* ph) {
   if (p.key_bits == 4) replay_weights_t<4, G>(p, t, S, q2, lane, ph);
   else replay_weights_t<3, G>(p, t, S, q2, lane, ph);
 }
 
-// One token into the warp's combined partial (m, l, a): + its exact term,
-// and, for a quantized token, - the approximate term the scan added for it.
-template <int G>
-__device__ __forceinline__ void warp_token(const FinishParams& p, int t, const WStage& S, uint2 kr,
-                                           uint2 vr, const FinParts<G>& P, const uint32_t (&q2)[2][16],
-                                           int lane, float (&m)[G], float (&l)[G],
-                                           float (&a)[G][4]) {
-  const float kf[4] = {__uint_as_float(kr.x << 16), __uint_as_float(kr.x & 0xFFFF0000u),
-                       __uint_as_float(kr.y << 16), __uint_as_float(kr.y & 0xFFFF0000u)};
-  const float vf[4] = {__uint_as_float(vr.x << 16), __uint_as_float(vr.x & 0xFFFF0000u),
-                       __uint_as_float(vr.y << 16), __uint_as_float(vr.y & 0xFFFF0000u)};
-  // exact logits: per-lane partial dots, a reduce-scatter over the lanes
-  // (each level halves the values a lane carries), then every head's total
-  // gathered from the lane that holds it
-  constexpr int GP = G <= 1 ? 1 : (G <= 2 ? 2 : (G <= 4 ? 4 : 8));
-  constexpr int LG = GP == 1 ? 0 : (GP == 2 ? 1 : (GP == 4 ? 2 : 3));
-  float v[GP];
+__device__ __forceinline__ void mma_bf16_16816(float* d, uint32_t a0, uint32_t a1, uint32_t a2,
+                                               uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+// fp32 x as a bf16 triple hi + mid + lo (each the bf16 rounding of what the
+// previous limbs leave; the remainder is below 2^-24 |x|).
+__device__ __forceinline__ uint16_t bf16_bits(float x) {
+  return __bfloat16_as_ushort(__float2bfloat16_rn(x));
+}
+__device__ __forceinline__ float bf16_val(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
+__device__ __forceinline__ void split3(float x, uint16_t& hi, uint16_t& mid, uint16_t& lo) {
+  hi = bf16_bits(x);
+  const float r1 = x - bf16_val(hi);
+  mid = bf16_bits(r1);
+  lo = bf16_bits(r1 - bf16_val(mid));
+}
+// Correction of the tokens tok_at(0..n), 16 at a time, into this CTA's
+// combined partial P.run (frame m, mass l, acc; all 256 threads).  Batch
+// b + 1 is staged (record pieces by cp.async, exact rows through registers)
+// while batch b is computed:
+//   replay the scan's fp16 weights of each quantized token (warp w: tokens
+//          2w, 2w + 1); warp 0 also computes the 16 x 8 exact logits (bf16
+//          MMA) and moves the frame of a head when one of the batch's terms
+//          exceeds it by more than 2^8;
+//   weights thread (head, token): exact weight 2^(s - m), removed mass
+//          2^(m_used - m) p and removed value weights 2^(m_used - m) fp16(p s_v),
+//          split into bf16 triples / fp16 pairs (B operands);
+//   values warp w = channels 16w..16w+15: acc += V^T exact + codes^T removed;
+//          the last warp also sums the masses (ones x exact, ones x removed)
+//          and the zero-point terms (zeros x removed) on tensor cores; fp32
+//          accumulators stay in registers across batches.
+template <int G, typename TokAt>
+__device__ __forceinline__ void batch_correct(const FinishParams& p, int seg, TokAt tok_at, int n,
+                                              FinBatchT& B, FinParts<G>& P,
+                                              const uint32_t (&q2)[2][16],
+                                              const uint32_t (&qb)[8][2]) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int gid = lane >> 2, tig = lane & 3;
+  constexpr int kSumWarp = kFinThreads / 32 - 1;
+  const int c0 = 16 * warp + gid;
+  const bool h0ok = 2 * tig < G, h1ok = 2 * tig + 1 < G;
+  float acc[4];
+  acc[0] = h0ok ? P.run[2 * tig][4 + c0] : 0.f;
+  acc[1] = h1ok ? P.run[2 * tig + 1][4 + c0] : 0.f;
+  acc[2] = h0ok ? P.run[2 * tig][4 + c0 + 8] : 0.f;
+  acc[3] = h1ok ? P.run[2 * tig + 1][4 + c0 + 8] : 0.f;
+  // sums (last warp): dE = exact mass (every row), dF row 0 = removed mass,
+  // rows 1..4 = removed zero-point terms of channel groups 0..3
+  float dE[4], dF[4] = {0.f, 0.f, 0.f, 0.f};
+  dE[0] = dE[2] = h0ok ? P.run[2 * tig][1] : 0.f;
+  dE[1] = dE[3] = h1ok ? P.run[2 * tig + 1][1] : 0.f;
+  const int nbatch = (n + kBT - 1) / kBT;
+  // staging of batch bi into buffer buf: this warp's tokens 2w, 2w + 1;
+  // the lane's row pieces: token 2w + (lane >> 4), piece lane & 15
+  int rt = -1;
+  uint4 kx = make_uint4(0u, 0u, 0u, 0u), vx = kx;
+  auto issue = [&](int bi, int buf) {
 #pragma unroll
-  for (int j = 0; j < GP; ++j) {
-    if (j < G) {
-      const float4 qv = *reinterpret_cast<const float4*>(&P.qs[j][4 * lane]);
-      v[j] = fmaf(qv.x, kf[0], fmaf(qv.y, kf[1], fmaf(qv.z, kf[2], qv.w * kf[3])));
-    } else {
-      v[j] = 0.f;
+    for (int k2 = 0; k2 < 2; ++k2) {
+      const int j = bi * kBT + 2 * warp + k2;
+      const int t = j < n ? tok_at(j) : -1;
+      if (tok_quant(t)) {
+        TokStage& S = B.st[buf][2 * warp + k2];
+#pragma unroll
+        for (int i = lane; i < 64; i += 32) stage_piece(p, seg, t, S, i);
+      }
+      if ((lane >> 4) == k2) rt = t;
     }
-  }
-#pragma unroll
-  for (int L = 0; L < LG; ++L) {
-    const int o = 16 >> L, half = GP >> (L + 1);
-    const bool up = (lane & o) != 0;
-#pragma unroll
-    for (int i = 0; i < half; ++i) {
-      const float keep = up ? v[half + i] : v[i];
-      const float send = up ? v[i] : v[half + i];
-      v[i] = keep + __shfl_xor_sync(kAll, send, o);
+    cp_async_commit();
+    kx = make_uint4(0u, 0u, 0u, 0u);
+    vx = kx;
+    if (rt != -1) {
+      kx = row_piece(p, seg, rt, false, lane & 15);
+      vx = row_piece(p, seg, rt, true, lane & 15);
     }
+  };
+  auto store_rows = [&](int buf) {
+    TokStage& S = B.st[buf][2 * warp + (lane >> 4)];
+    *reinterpret_cast<uint4*>(&S.krow[8 * (lane & 15)]) = kx;
+    *reinterpret_cast<uint4*>(&S.vrow[8 * (lane & 15)]) = vx;
+    if ((lane & 15) == 0) B.tok[buf][2 * warp + (lane >> 4)] = rt;
+  };
+  if (nbatch > 0) {
+    issue(0, 0);
+    store_rows(0);
   }
+#pragma unroll 1
+  for (int bi = 0; bi < nbatch; ++bi) {
+    const int buf = bi & 1;
+    cp_async_wait<0>();
+    __syncthreads();
+    if (bi + 1 < nbatch) issue(bi + 1, buf ^ 1);
+    // ---- exact logits and frames (warp 0), replay (warp w: tokens 2w, 2w + 1)
+    if (warp == 0) {
+      float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-  for (int o = 16 >> LG; o > 0; o >>= 1) v[0] += __shfl_xor_sync(kAll, v[0], o);
-  float se[G];
+      for (int ks = 0; ks < 8; ++ks) {
+        const uint16_t* r0 = B.st[buf][gid].krow + 16 * ks + 2 * tig;
+        const uint16_t* r1 = B.st[buf][gid + 8].krow + 16 * ks + 2 * tig;
+        mma_bf16_16816(d, *reinterpret_cast<const uint32_t*>(r0), *reinterpret_cast<const uint32_t*>(r1),
+                       *reinterpret_cast<const uint32_t*>(r0 + 8), *reinterpret_cast<const uint32_t*>(r1 + 8),
+                       qb[ks][0], qb[ks][1]);
+      }
 #pragma unroll
-  for (int j = 0; j < G; ++j) {
-    int src = 0;
+      for (int i = 0; i < 4; ++i) d[i] *= p.kappa;
+      B.se[gid][2 * tig] = d[0];
+      B.se[gid][2 * tig + 1] = d[1];
+      B.se[gid + 8][2 * tig] = d[2];
+      B.se[gid + 8][2 * tig + 1] = d[3];
+      // the batch's largest term per head (exact logits, the scan maxima of
+      // the removed tokens' groups), over the 16 token rows
+      const int ta = B.tok[buf][gid], tb = B.tok[buf][gid + 8];
+      const float* mua = B.st[buf][gid].mu;
+      const float* mub = B.st[buf][gid + 8].mu;
 #pragma unroll
-    for (int L = 0; L < LG; ++L) src += ((j >> (LG - 1 - L)) & 1) * (16 >> L);
-    se[j] = __shfl_sync(kAll, v[0], src) * p.kappa;
-  }
-  const bool qt = tok_quant(t);
-  uint32_t ph[G];
-  float code[4] = {0.f, 0.f, 0.f, 0.f};
-  uint16_t svb = 0;
-  float zv = 0.f;
-  if (qt) {
-    replay_weights<G>(p, t, S, q2, lane, ph);
-    const int tt = t % kKG, rt = tt & 15, hi8 = rt >> 3, e = rt & 1, jg = lane >> 3;
-    svb = *reinterpret_cast<const uint16_t*>(S.vsz + jg * 8 + hi8 * 4 + 2 * e);
-    zv = h2f(*reinterpret_cast<const uint16_t*>(S.vsz + 32 + jg * 8 + hi8 * 4 + 2 * e));
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      // the staged pieces are the token column's lanes (gd*4 + tig) of the
-      // k-step's chunks; word and bit as in vc_loc
-      const int c = 4 * lane + i, mt = c >> 4, rc = c & 15, gd = rc & 7, chi = rc >> 3;
-      const int bit = vc_pos(p.val_bits, mt) + 8 * chi + 16 * e;
-      if (p.val_bits == 4) {
-        const int w8 = 2 * (mt & 3) + hi8;
-        const uint32_t w = *reinterpret_cast<const uint32_t*>(S.vp + ((w8 >> 2) * 8 + gd) * 16 + (w8 & 3) * 4);
-        code[i] = (float)((w >> bit) & 15u);
-      } else {
-        const uint32_t w = *reinterpret_cast<const uint32_t*>(S.vp + gd * 16 + (2 * (mt & 1) + hi8) * 4);
-        code[i] = (float)((w >> bit) & 3u);
+      for (int c = 0; c < 2; ++c) {
+        const int h = 2 * tig + c;
+        float v = -INFINITY;
+        if (ta != -1) v = fmaxf(v, d[c]);
+        if (tb != -1) v = fmaxf(v, d[2 + c]);
+        if (tok_quant(ta)) v = fmaxf(v, mua[h]);
+        if (tok_quant(tb)) v = fmaxf(v, mub[h]);
+        v = fmaxf(v, __shfl_xor_sync(kAll, v, 4));
+        v = fmaxf(v, __shfl_xor_sync(kAll, v, 8));
+        v = fmaxf(v, __shfl_xor_sync(kAll, v, 16));
+        if (gid == 0 && h < G) {
+          const float m = P.run[h][0];
+          float al = 1.f;
+          if (v > m + 8.f) {
+            al = exp2f(m - v);  // 0 while the partial is empty (m = -inf)
+            P.run[h][0] = v;
+          }
+          B.alpha[h] = al;
+        }
       }
     }
-  }
-  // the partial's frame m moves only when a new term would exceed it by more
-  // than 2^8 (warp-uniform test), so most tokens need no rescale
-#pragma unroll
-  for (int j = 0; j < G; ++j) {
-    const float mu = qt ? S.mu[j] : -INFINITY;
-    const float cand = fmaxf(se[j], mu);
-    if (cand > m[j] + 8.f) {
-      const float al = exp2f(m[j] - cand);  // 0 while the partial is empty (m = -inf)
-      l[j] *= al;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) a[j][i] *= al;
-      m[j] = cand;
-    }
-    const float pe = exp2f(se[j] - m[j]);
-    l[j] += pe;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) a[j][i] = fmaf(pe, vf[i], a[j][i]);
-    if (qt) {
-      const float f = exp2f(mu - m[j]);
-      const uint16_t phj = (uint16_t)ph[j];
-      const float pf = h2f(phj) * f, w = h2f(h_mul_rn(phj, svb)) * f;
-      const float zt = pf * zv;
-      l[j] -= pf;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) a[j][i] -= fmaf(w, code[i], zt);
-    }
-  }
-}
-
-// The warp's tokens tok_at(0..n) into its partial P.wp[warp] (loaded,
-// updated, stored back).
-template <int G, typename TokAt>
-__device__ __forceinline__ void warp_correct(const FinishParams& p, int seg, TokAt tok_at, int n,
-                                             WStage* ring, FinParts<G>& P, const uint32_t (&q2)[2][16],
-                                             int warp, int lane) {
-  float m[G], l[G], a[G][4];
-#pragma unroll
-  for (int j = 0; j < G; ++j) {
-    m[j] = P.wp[warp][j][0];
-    l[j] = P.wp[warp][j][1];
-    const float4 v = *reinterpret_cast<const float4*>(&P.wp[warp][j][4 + 4 * lane]);
-    a[j][0] = v.x;
-    a[j][1] = v.y;
-    a[j][2] = v.z;
-    a[j][3] = v.w;
-  }
-#pragma unroll
-  for (int i = 0; i < kWD - 1; ++i) stage_issue(p, seg, i < n ? tok_at(i) : -1, ring[i], lane);
-  // exact rows two tokens ahead in registers
-  uint2 kr = make_uint2(0u, 0u), vr = kr, kr1 = kr, vr1 = kr;
-  if (n > 0) row_load(p, seg, tok_at(0), lane, kr, vr);
-  if (n > 1) row_load(p, seg, tok_at(1), lane, kr1, vr1);
 #pragma unroll 1
-  for (int i = 0; i < n; ++i) {
-    const int t = tok_at(i);
-    stage_issue(p, seg, i + kWD - 1 < n ? tok_at(i + kWD - 1) : -1, ring[(i + kWD - 1) % kWD], lane);
-    uint2 kr2 = kr1, vr2 = vr1;
-    if (i + 2 < n) row_load(p, seg, tok_at(i + 2), lane, kr2, vr2);
-    cp_async_wait<kWD - 1>();
-    __syncwarp();
-    warp_token<G>(p, t, ring[i % kWD], kr, vr, P, q2, lane, m, l, a);
-    __syncwarp();
-    kr = kr1;
-    vr = vr1;
-    kr1 = kr2;
-    vr1 = vr2;
-  }
-  cp_async_wait<0>();
-  __syncwarp();
-#pragma unroll
-  for (int j = 0; j < G; ++j) {
-    if (lane == 0) {
-      P.wp[warp][j][0] = m[j];
-      P.wp[warp][j][1] = l[j];
+    for (int k2 = 0; k2 < 2; ++k2) {
+      const int tl = 2 * warp + k2, t = B.tok[buf][tl];
+      if (tok_quant(t)) replay_weights<G>(p, t, B.st[buf][tl], q2, lane, B.ph[tl]);
     }
-    *reinterpret_cast<float4*>(&P.wp[warp][j][4 + 4 * lane]) = make_float4(a[j][0], a[j][1], a[j][2], a[j][3]);
+    __syncthreads();
+    // ---- weights: thread (head h, token slot tl)
+    if (tid < kBT * G) {
+      const int h = tid >> 4, tl = tid & 15;
+      const int t = B.tok[buf][tl];
+      const bool valid = t != -1, qt = tok_quant(t);
+      const TokStage& S = B.st[buf][tl];
+      const float m = P.run[h][0];
+      const float pe = valid ? exp2f(B.se[tl][h] - m) : 0.f;
+      split3(pe, B.bex[0][h][tl], B.bex[1][h][tl], B.bex[2][h][tl]);
+      const float f = qt ? exp2f(S.mu[h] - m) : 0.f;
+      const uint16_t phb = qt ? B.ph[tl][h] : (uint16_t)0;
+      const float pf = h2f(phb) * f;
+      const uint16_t pfh = f2h_rn(pf);
+      B.bpf[0][h][tl] = pfh;
+      B.bpf[1][h][tl] = f2h_rn(pf - h2f(pfh));
+      const int tt = qt ? t % kKG : 0, hi8 = (tt & 15) >> 3, e = tt & 1;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint16_t vsc = *reinterpret_cast<const uint16_t*>(S.vsz + j * 8 + hi8 * 4 + 2 * e);
+        const float wv = qt ? h2f(h_mul_rn(phb, vsc)) * f : 0.f;
+        split3(-wv, B.brem[0][j][h][tl], B.brem[1][j][h][tl], B.brem[2][j][h][tl]);
+      }
+    }
+    __syncthreads();
+    // ---- values: warp w = channels 16w .. 16w + 15
+    {
+      const float a0s = h0ok ? B.alpha[2 * tig] : 1.f;
+      const float a1s = h1ok ? B.alpha[2 * tig + 1] : 1.f;
+      acc[0] *= a0s;
+      acc[1] *= a1s;
+      acc[2] *= a0s;
+      acc[3] *= a1s;
+      // A operands: rows = channels c0, c0 + 8; columns = token slots
+      // 2tig, 2tig + 1 (a0, a1) and 2tig + 8, 2tig + 9 (a2, a3)
+      uint32_t va[4], ca[4];
+#pragma unroll
+      for (int hs = 0; hs < 2; ++hs) {
+        const int s0 = 2 * tig + 8 * hs;
+        const TokStage& S0 = B.st[buf][s0];
+        const TokStage& S1 = B.st[buf][s0 + 1];
+        va[2 * hs] = (uint32_t)S0.vrow[c0] | ((uint32_t)S1.vrow[c0] << 16);
+        va[2 * hs + 1] = (uint32_t)S0.vrow[c0 + 8] | ((uint32_t)S1.vrow[c0 + 8] << 16);
+        uint32_t cb[2][2];  // [token][row half]: bf16 bits of the code
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int t = B.tok[buf][s0 + u];
+          const TokStage& S = u ? S1 : S0;
+          uint32_t c_lo = 0u, c_hi = 0u;
+          if (tok_quant(t)) {
+            const int tt = t % kKG, hi8 = (tt & 15) >> 3, e = tt & 1;
+            const int bit = vc_pos(p.val_bits, warp) + 16 * e;
+            if (p.val_bits == 4) {
+              const int w8 = 2 * (warp & 3) + hi8;
+              const uint32_t wd = *reinterpret_cast<const uint32_t*>(S.vp + ((w8 >> 2) * 8 + gid) * 16 + (w8 & 3) * 4);
+              c_lo = (wd >> bit) & 15u;
+              c_hi = (wd >> (bit + 8)) & 15u;
+            } else {
+              const uint32_t wd = *reinterpret_cast<const uint32_t*>(S.vp + gid * 16 + (2 * (warp & 1) + hi8) * 4);
+              c_lo = (wd >> bit) & 3u;
+              c_hi = (wd >> (bit + 8)) & 3u;
+            }
+          }
+          cb[u][0] = __float_as_uint((float)c_lo) >> 16;
+          cb[u][1] = __float_as_uint((float)c_hi) >> 16;
+        }
+        ca[2 * hs] = cb[0][0] | (cb[1][0] << 16);
+        ca[2 * hs + 1] = cb[0][1] | (cb[1][1] << 16);
+      }
+      const int j = warp >> 1;
+#pragma unroll
+      for (int l = 0; l < 3; ++l)
+        mma_bf16_16816(acc, va[0], va[1], va[2], va[3], *reinterpret_cast<const uint32_t*>(&B.bex[l][gid][2 * tig]),
+                       *reinterpret_cast<const uint32_t*>(&B.bex[l][gid][2 * tig + 8]));
+#pragma unroll
+      for (int l = 0; l < 3; ++l)
+        mma_bf16_16816(acc, ca[0], ca[1], ca[2], ca[3], *reinterpret_cast<const uint32_t*>(&B.brem[l][j][gid][2 * tig]),
+                       *reinterpret_cast<const uint32_t*>(&B.brem[l][j][gid][2 * tig + 8]));
+      if (warp == kSumWarp) {
+        dE[0] *= a0s;
+        dE[1] *= a1s;
+        dE[2] *= a0s;
+        dE[3] *= a1s;
+        dF[0] *= a0s;
+        dF[1] *= a1s;
+        dF[2] *= a0s;
+        dF[3] *= a1s;
+        constexpr uint32_t kOnesBf = 0x3F803F80u;
+#pragma unroll
+        for (int l = 0; l < 3; ++l)
+          mma_bf16_16816(dE, kOnesBf, kOnesBf, kOnesBf, kOnesBf,
+                         *reinterpret_cast<const uint32_t*>(&B.bex[l][gid][2 * tig]),
+                         *reinterpret_cast<const uint32_t*>(&B.bex[l][gid][2 * tig + 8]));
+        // A rows: 0 = ones, 1..4 = the value zero points of channel group
+        // gid - 1 (fp16), others 0; columns = token slots
+        uint32_t za[2];
+#pragma unroll
+        for (int hs = 0; hs < 2; ++hs) {
+          uint32_t zz = 0u;
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int sl = 2 * tig + 8 * hs + u, t = B.tok[buf][sl];
+            uint32_t zh = 0u;
+            if (gid == 0) {
+              zh = 0x3C00u;
+            } else if (gid <= 4 && tok_quant(t)) {
+              const int tt = t % kKG, hi8 = (tt & 15) >> 3, e = tt & 1;
+              zh = *reinterpret_cast<const uint16_t*>(B.st[buf][sl].vsz + 32 + (gid - 1) * 8 + hi8 * 4 + 2 * e);
+            }
+            zz |= zh << (16 * u);
+          }
+          za[hs] = zz;
+        }
+#pragma unroll
+        for (int l = 0; l < 2; ++l)
+          mma16816(dF, za[0], 0u, za[1], 0u, *reinterpret_cast<const uint32_t*>(&B.bpf[l][gid][2 * tig]),
+                   *reinterpret_cast<const uint32_t*>(&B.bpf[l][gid][2 * tig + 8]));
+      }
+    }
+    if (bi + 1 < nbatch) store_rows(buf ^ 1);
   }
-  __syncwarp();
+  if (warp == kSumWarp) {
+    if (gid == 0) {  // mass: exact minus removed
+      if (h0ok) P.run[2 * tig][1] = dE[0] - dF[0];
+      if (h1ok) P.run[2 * tig + 1][1] = dE[1] - dF[1];
+    } else if (gid <= 4) {
+      if (h0ok) B.zsum[2 * tig][gid - 1] = -dF[0];
+      if (h1ok) B.zsum[2 * tig + 1][gid - 1] = -dF[1];
+    }
+  }
+  __syncthreads();
+  {
+    const int j = warp >> 1;
+    if (h0ok) {
+      P.run[2 * tig][4 + c0] = acc[0] + B.zsum[2 * tig][j];
+      P.run[2 * tig][4 + c0 + 8] = acc[2] + B.zsum[2 * tig][j];
+    }
+    if (h1ok) {
+      P.run[2 * tig + 1][4 + c0] = acc[1] + B.zsum[2 * tig + 1][j];
+      P.run[2 * tig + 1][4 + c0 + 8] = acc[3] + B.zsum[2 * tig + 1][j];
+    }
+  }
+  __syncthreads();
 }
 
 template <int G, bool SELECT>
@@ -596,11 +740,10 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
     for (int i = tid; i < n_mine * 4; i += kFinThreads)
       prefetch_part(p, seg, (1 << 30) | (r + C * (i >> 2)), i & 3);
   }
-  for (int i = tid; i < G * kD; i += kFinThreads)
-    P.qs[i / kD][i % kD] = bf16f(p.q[((size_t)bb * p.H + hh * G + i / kD) * kD + i % kD]);
-  for (int i = tid; i < kFinWarps * G * kPartStride; i += kFinThreads)
-    (&P.wp[0][0][0])[i] = (i % kPartStride) == 0 ? -INFINITY : 0.f;
-  // the lane's q as the scan holds it: head (gid >> 1) + 4n of n-tile n
+  for (int i = tid; i < G * kPartStride; i += kFinThreads)
+    (&P.run[0][0])[i] = (i % kPartStride) == 0 ? -INFINITY : 0.f;
+  // the lane's q as the scan holds it (head (gid >> 1) + 4n of n-tile n), and
+  // as bf16 B fragments of the exact-logit MMA (head gid)
   uint32_t q2[2][16];
 #pragma unroll
   for (int n = 0; n < 2; ++n) {
@@ -608,17 +751,16 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
     const bool ok = hq < G && (n == 0 || G > 4);
     q_frag(p.q + ((size_t)bb * p.H + (size_t)hh * G + (ok ? hq : 0)) * kD, ok, tig, q2[n]);
   }
-  __syncthreads();
-  const int warp = tid >> 5;
-
-  // ---- T: this CTA's tail slots r, r + C, ... (exact rows only), warp w
-  // taking every kFinWarps-th of them
+  uint32_t qb[8][2];
   {
-    const int n_mine = p.tail > r ? (p.tail - r + C - 1) / C : 0;
-    const int n_w = n_mine > warp ? (n_mine - warp + kFinWarps - 1) / kFinWarps : 0;
-    auto tail_at = [&](int i) { return (1 << 30) | (r + C * (warp + kFinWarps * i)); };
-    warp_correct<G>(p, seg, tail_at, n_w, FC.st[warp], P, q2, warp, lane);
+    const uint16_t* qrow = p.q + ((size_t)bb * p.H + (size_t)hh * G + (gid < G ? gid : 0)) * kD;
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      qb[ks][0] = gid < G ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * tig) : 0u;
+      qb[ks][1] = gid < G ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * tig + 8) : 0u;
+    }
   }
+  __syncthreads();
 
   pdl_wait();
   pdl_launch_dependents();
@@ -950,16 +1092,22 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
       }
     }
   }
-  // ---- P4: correction of an even share of the chosen set: the token list
-  // first (compacted, in shared memory), then a warp per token
+  // ---- P4: correction of this CTA's tail slots r, r + C, ... and an even
+  // share of the chosen set: the token list first (compacted, in shared
+  // memory), then batches of 16 tokens
   {
     const int n_x = select ? k : (SELECT ? nq : k);  // positions of the chosen sequence
     const int per = (n_x + C - 1) / C;
     const int x0 = min(n_x, r * per), x1 = min(n_x, x0 + per);
+    const int n_tail = p.tail > r ? (p.tail - r + C - 1) / C : 0;
 #pragma unroll 1
-    for (int xr = x0; xr < x1; xr += kTokCap) {
+    for (int xr = x0, first = 1; first || xr < x1; xr += kTokCap, first = 0) {
     const int xe = min(x1, xr + kTokCap);
     uint32_t base = 0;
+    if (first) {
+      for (int i = tid; i < n_tail; i += kFinThreads) FC.tok[i] = (1 << 30) | (r + C * i);
+      base = (uint32_t)n_tail;
+    }
 #pragma unroll 1
     for (int xb = xr; xb < xe; xb += kFinThreads) {
       const int j = xb + tid;
@@ -992,35 +1140,11 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
     const int n = (int)base;
     for (int i = tid; i < n * 4; i += kFinThreads)  // the exact rows into L2
       prefetch_part(p, seg, FC.tok[i >> 2], i & 3);
-    const int n_w = n > warp ? (n - warp + kFinWarps - 1) / kFinWarps : 0;
     const int32_t* tl = FC.tok;
-    auto chosen_at = [&](int i) { return tl[warp + kFinWarps * i]; };
-    warp_correct<G>(p, seg, chosen_at, n_w, FC.st[warp], P, q2, warp, lane);
-    __syncthreads();
-    }
-    // combine the warps' partials into P.run: thread (channel, half) merges
-    // heads half, half + 2, ...
-    const int c = tid & (kD - 1), half = tid >> 7;
-    for (int j = half; j < G; j += 2) {
-      float mx = -INFINITY;
-#pragma unroll
-      for (int w = 0; w < kFinWarps; ++w) mx = fmaxf(mx, P.wp[w][j][0]);
-      float l = 0.f, acc = 0.f;
-#pragma unroll
-      for (int w = 0; w < kFinWarps; ++w) {
-        const float mw = P.wp[w][j][0];
-        const float f = mw == -INFINITY ? 0.f : exp2f(mw - mx);  // empty partials add nothing
-        l = fmaf(P.wp[w][j][1], f, l);
-        acc = fmaf(P.wp[w][j][4 + c], f, acc);
-      }
-      P.run[j][4 + c] = acc;
-      if (c == 0) {
-        P.run[j][0] = mx;
-        P.run[j][1] = l;
-      }
+    auto chosen_at = [&](int i) { return tl[i]; };
+    batch_correct<G>(p, seg, chosen_at, n, FC.b, P, q2, qb);
     }
   }
-
   cl.sync();
 
   // ---- P5b: CTA r owns heads j = r, r + C, ...: merge the C CTAs' scan
