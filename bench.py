@@ -28,7 +28,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "decode attn: cached KV tokens/s on 1 B200 and % of HBM roofline (K3V2, K4V4)"
-FLUSH_BYTES = 256 << 20   # > 126 MB L2
+L2_BYTES = 126 << 20      # B200 L2
 
 
 def parse(argv=None):
@@ -305,11 +305,14 @@ def run_reference(args, w):
     return 0
 
 
-def config_of(w, args):
+def config_of(w, args, n_copies=0, packed_bytes=0):
     return {"workload": w.name, "batch": w.batch, "heads": w.heads, "kv_heads": w.kv_heads,
             "ctx": w.ctx, "format": w.fmt, "topk": w.topk,
             "exact_rows": "pinned_host" if args.host_resident else "hbm",
-            "l2": "flushed before every timed step (256 MB write)",
+            "l2": (f"not flushed: the timed steps rotate over {n_copies} copies of the packed "
+                   f"cache and of the exact rows ({n_copies} x {packed_bytes / 2**20:.0f} MiB "
+                   f"packed > 126 MB L2), so every step reads its inputs from HBM")
+                  if n_copies else "host run",
             "parallelism": f"replicas x{args.gpus}"}
 
 
@@ -331,88 +334,105 @@ def run_jfa(args, w):
 
     q = W.gen_q(w).to(dev)
     k_all, v_all = W.gen_kv_device(w, dev, W.gen_q(w))
-    cache = jfa.KVCache(w.batch, w.heads, w.kv_heads, w.ctx, w.key_bits, w.val_bits, device=dev)
-    ws = jfa.Workspace(cache, w.topk, device=dev)
-    cache.append(k_all, v_all, ws)
-    if args.host_resident:
-        k_exact = k_all.cpu().pin_memory()
-        v_exact = v_all.cpu().pin_memory()
-        del k_all, v_all
-    else:
-        k_exact, v_exact = k_all, v_all
+    # R copies of the cache (and of the exact rows the correction gathers),
+    # together larger than L2: the timed steps rotate over them, so every
+    # step reads its inputs from HBM without an L2 flush between steps
+    probe = jfa.KVCache(w.batch, w.heads, w.kv_heads, w.ctx, w.key_bits, w.val_bits, device=dev)
+    packed_bytes = probe.layout.groups_bytes
+    n_copies = 1 + -(-L2_BYTES // max(1, packed_bytes))
+    del probe
+    ws = None
+    copies = []
+    for c in range(n_copies):
+        cache = jfa.KVCache(w.batch, w.heads, w.kv_heads, w.ctx, w.key_bits, w.val_bits, device=dev)
+        if ws is None:
+            ws = jfa.Workspace(cache, w.topk, device=dev)
+        cache.append(k_all, v_all, ws)
+        if args.host_resident:
+            ke, ve = k_all.cpu().pin_memory(), v_all.cpu().pin_memory()
+        else:
+            ke, ve = (k_all, v_all) if c == 0 else (k_all.clone(), v_all.clone())
+        copies.append((cache, cache.geom(), cache.struct(), ke, ve))
+    del k_all, v_all
     torch.cuda.synchronize()
     out = torch.empty(w.batch, w.heads, 128, dtype=torch.float32, device=dev)
     idx = torch.empty(w.batch, w.kv_heads, w.topk, dtype=torch.int32, device=dev)
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
     sp = stream.cuda_stream
-    geom, cst = cache.geom(), cache.struct()
     scale = W.default_scale(w)
     host = 1 if args.host_resident else 0
+    geom = copies[0][1]
 
-    def step():
-        _lib.check(_lib.jfa_decode_scores(geom, cst, q, scale, ws.buf, sp), "scores")
-        _lib.check(_lib.jfa_decode_finish(geom, cst, q, scale, w.topk, idx, k_exact, v_exact,
+    def step(i, wsb=None):
+        _, g, cs, ke, ve = copies[i % n_copies]
+        _lib.check(_lib.jfa_decode_scores(g, cs, q, scale, ws.buf, sp), "scores")
+        _lib.check(_lib.jfa_decode_finish(g, cs, q, scale, w.topk, idx, ke, ve,
                                           host, ws.buf, out, sp), "finish")
 
-    for _ in range(max(3, args.warmup)):
-        flush.zero_()
-        step()
+    for i in range(max(3, args.warmup)):
+        step(i)
     torch.cuda.synchronize()
     st, flag = _lib.jfa_check_error(geom, ws.buf, sp)
     if flag:
         raise RuntimeError(f"device error flag {flag:#x}")
 
-    # timed steps: the call sequence of a decode step, nothing between the calls
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    # timed steps: K decode steps back to back (the call sequence of a step,
+    # nothing between the calls), one event pair around all of them
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = Clocks(local, not args.no_clocks)
     barrier(world)
     torch.cuda.synchronize()
     wall0 = time.perf_counter()
+    e0.record(stream)
     for i in range(args.steps):
-        flush.zero_()
-        ev[i][0].record(stream)
-        step()
-        ev[i][1].record(stream)
+        step(i)
+    e1.record(stream)
     torch.cuda.synchronize()
     barrier(world)
     wall = time.perf_counter() - wall0
     clk = clocks.stop()
-    step_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(args.steps)]
-    ms = statistics.mean(step_ms)
+    ms = e0.elapsed_time(e1) / args.steps
     ms_max = max_over_ranks(ms, world, dev)
 
-    # the scan kernel alone (roofline): its own launches, L2 flushed before each,
-    # on a workspace of its own (scan-only launches leave the selection
-    # histogram for a finishing kernel to consume)
-    ws_scan = jfa.Workspace(cache, w.topk, device=dev)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    # the scan kernel alone (roofline): its own launches back to back over the
+    # same rotation, on a workspace of its own (scan-only launches leave the
+    # selection histogram for a finishing kernel to consume)
+    ws_scan = jfa.Workspace(copies[0][0], w.topk, device=dev)
+    for i in range(3):
+        _, g, cs, _, _ = copies[i % n_copies]
+        _lib.check(_lib.jfa_decode_scores(g, cs, q, scale, ws_scan.buf, sp), "scores")
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s0.record(stream)
     for i in range(args.steps):
-        flush.zero_()
-        evs[i][0].record(stream)
-        _lib.check(_lib.jfa_decode_scores(geom, cst, q, scale, ws_scan.buf, sp), "scores")
-        evs[i][1].record(stream)
+        _, g, cs, _, _ = copies[i % n_copies]
+        _lib.check(_lib.jfa_decode_scores(g, cs, q, scale, ws_scan.buf, sp), "scores")
+    s1.record(stream)
     torch.cuda.synchronize()
-    scan_avg = statistics.mean(evs[i][0].elapsed_time(evs[i][1]) for i in range(args.steps))
+    scan_avg = s0.elapsed_time(s1) / args.steps
     del ws_scan
 
-    # end to end through the public API: q from pinned host in, out back to pinned host
+    # end to end through the public API: every step copies q in from pinned
+    # host memory and its output back to pinned host memory
     q_host = q.cpu().pin_memory()
     out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    e2e_ms = []
-    for i in range(args.warmup + args.steps):
-        flush.zero_()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
+
+    def e2e_step(i):
+        cache, _, _, ke, ve = copies[i % n_copies]
         q.copy_(q_host, non_blocking=True)
-        jfa.decode_step(cache, q, w.topk, k_exact, v_exact, ws, scale=scale, out=out, idx=idx,
+        jfa.decode_step(cache, q, w.topk, ke, ve, ws, scale=scale, out=out, idx=idx,
                         exact_on_host=bool(host), stream=stream)
         out_host.copy_(out, non_blocking=True)
-        e1.record(stream)
-        if i >= args.warmup:
-            e2e_ms.append((e0, e1))
+
+    for i in range(max(3, args.warmup)):
+        e2e_step(i)
+    x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
-    e2e_avg = statistics.mean(a.elapsed_time(b) for a, b in e2e_ms)
+    x0.record(stream)
+    for i in range(args.steps):
+        e2e_step(i)
+    x1.record(stream)
+    torch.cuda.synchronize()
+    e2e_avg = x0.elapsed_time(x1) / args.steps
     e2e_max = max_over_ranks(e2e_avg, world, dev)
 
     st, flag = _lib.jfa_check_error(geom, ws.buf, sp)
@@ -440,7 +460,7 @@ def run_jfa(args, w):
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "f32", "data": "synthetic", "config": config_of(w, args),
+            "dtype": "f32", "data": "synthetic", "config": config_of(w, args, n_copies, packed_bytes),
             "roofline": {"bound": "hbm", "kernel": "scan_kernel (jfa_decode_scores)",
                          "achieved": achieved, "peak": peak, "peak_kind": peak_kind,
                          "unit": "GB/s", "frac": achieved / peak,

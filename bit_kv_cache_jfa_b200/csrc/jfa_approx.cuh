@@ -149,8 +149,14 @@ __device__ __forceinline__ float approx_logit(const float d[4], int r, float kap
 }
 
 // Softmax weight of a logit u against the running maximum m, as the scan
-// feeds it to the value MMAs: fp16(2^(u - m)).
-__device__ __forceinline__ float approx_weight(float u, float m) { return exp2f(__fsub_rn(u, m)); }
+// feeds it to the value MMAs (rounded to fp16 there): 2^(u - m) from the
+// hardware base-2 exponential; results below 2^-126 flush to zero, far under
+// the fp16 range the weight is stored in.
+__device__ __forceinline__ float approx_weight(float u, float m) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(__fsub_rn(u, m)));
+  return r;
+}
 
 // fp16 multiply with round-to-nearest (the value weight p * s_v of one token).
 __device__ __forceinline__ uint16_t h_mul_rn(uint16_t a, uint16_t b) {
