@@ -87,6 +87,7 @@ SIGNATURES = {
                                     POINTER(c_uint16), POINTER(c_uint16), POINTER(c_uint8),
                                     POINTER(c_uint16), POINTER(c_uint16)]),
     "jfa_decode_step_launches": (c_int32, [POINTER(Geom), c_int32]),
+    "jfa_scan_warps": (c_int32, [POINTER(Geom)]),
 }
 
 _lib = None
@@ -226,3 +227,7 @@ def jfa_unpack_record(key_bits: int, val_bits: int, record: bytes):
 
 def jfa_decode_step_launches(geom: Geom, k: int) -> int:
     return load().jfa_decode_step_launches(ctypes.byref(geom), k)
+
+
+def jfa_scan_warps(geom: Geom) -> int:
+    return load().jfa_scan_warps(ctypes.byref(geom))

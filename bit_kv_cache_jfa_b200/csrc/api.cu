@@ -81,6 +81,9 @@ ScanPlan scan_plan(const jfa_geom& g, int num_sms) {
   const int nw = scan_cta_warps(g.key_bits, g.val_bits, g.num_heads / g.num_kv_heads > 4 ? 2 : 1);
   long long w = (long long)num_sms * nw;
   if (w > kMaxScanWarps) w = kMaxScanWarps;
+  const long long w_min_rec = (p.total_groups + kScanMinRecords - 1) / kScanMinRecords;
+  if (w > w_min_rec) w = w_min_rec;
+  if (w < 1) w = 1;
   if (w > p.total_groups) w = p.total_groups;
   p.n_warps = (int)w;
   p.n_ctas = (int)((w + nw - 1) / nw);
@@ -214,6 +217,12 @@ int jfa_decode_step_launches(const jfa_geom* geom, int32_t k) {
   if (!geom_ok(geom) || geom->n_ctx < 1 || k < 1 || k > JFA_MAX_TOPK) return 0;
   const int scan = split_point(geom->n_ctx) > 0 ? 1 : 0;
   return scan + 1;  // scan + fused finishing kernel
+}
+
+int jfa_scan_warps(const jfa_geom* geom) {
+  if (!geom_ok(geom) || geom->n_ctx < 1) return 0;
+  const ScanPlan plan = scan_plan(*geom, num_sms_current());
+  return plan.total_groups > 0 ? plan.n_warps : 0;
 }
 
 int jfa_clear_error(const jfa_geom* geom, void* ws, void* stream) {

@@ -725,6 +725,7 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
   __shared__ uint32_t s_cnt[kFinMaxC], s_pre[kFinMaxC + 1], s_tpre[kFinMaxC + 1];
   __shared__ uint32_t s_chq[kFinMaxC + 1];  // chosen ties before slice q
   __shared__ int s_mode;                     // 0 lists in shared memory, 1 fallback lists
+  __shared__ uint32_t s_hmax[kMaxG];          // per head: largest scan-partial maximum (key)
 
   cg::cluster_group cl = cg::this_cluster();
   const int C = (int)cl.num_blocks();
@@ -1028,57 +1029,68 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
       *reinterpret_cast<uint4*>(hg + i) = make_uint4(0u, 0u, 0u, 0u);
   }
 
-  // ---- P5a (merge)
+  // ---- P5a (merge): per head the largest partial maximum M first, then
+  // every row's terms scaled by 2^(m_row - M) and summed (no exponential on
+  // the accumulation chain); rows from the early copy, else staged a tile
+  // at a time; thread (channel, half) takes heads j = half, half + 2, ...
   {
-    // rows (slot, head) staged in shared memory a tile at a time, every load
-    // of a tile in flight together; thread (channel, half) merges the heads
-    // j = half, half + 2, ... online
     const int c = tid & (kD - 1), half = tid >> 7;
     constexpr int kH2 = (G + 1) / 2;
-    float mrun[kH2], lrun[kH2], arun[kH2];
+    if (tid < G) s_hmax[tid] = 0u;  // key of -inf and below
+    if (early_ok) cp_async_wait<0>();
+    __syncthreads();
+    for (int gr = tid; gr < nrows; gr += kFinThreads) {
+      float m, l;
+      if (early_ok) {
+        m = early[gr * kPartStride];
+        l = early[gr * kPartStride + 1];
+      } else {
+        const float* src = p.scan_part + ((size_t)(w0 + s0 + gr / G + seg) * G + gr % G) * kPartStride;
+        m = src[0];
+        l = src[1];
+      }
+      if (l > 0.f) atomicMax(&s_hmax[gr % G], float_key(m));
+    }
+    __syncthreads();
+    float mh[kH2], lrun[kH2], arun[kH2];
 #pragma unroll
     for (int i = 0; i < kH2; ++i) {
-      mrun[i] = -INFINITY;
+      const int j = half + 2 * i;
+      mh[i] = j < G && s_hmax[j] != 0u ? key_float(s_hmax[j]) : -INFINITY;
       lrun[i] = 0.f;
       arun[i] = 0.f;
     }
     float* tile = reinterpret_cast<float*>(U);
-    constexpr int kTR = (int)(sizeof(FinCorr) / (kPartStride * sizeof(float)));
-    if (early_ok) {
-      cp_async_wait<0>();
-      __syncthreads();
-    }
+    constexpr int kTR = (int)(sizeof(FinCorr) / (kPartStride * sizeof(float))) / kMaxG * kMaxG;
     for (int r0 = 0; r0 < nrows; r0 += (early_ok ? nrows : kTR)) {
       const int nr = early_ok ? nrows : min(kTR, nrows - r0);
-      if (early_ok) tile = early;
+      if (early_ok) {
+        tile = early;
+      } else {
 #pragma unroll 8
-      for (int i = tid; i < (early_ok ? 0 : nr * kV); i += kFinThreads) {
-        const int row = i / kV, v = i % kV;
-        const int gr = r0 + row;
-        const float* src = p.scan_part + ((size_t)(w0 + s0 + gr / G + seg) * G + gr % G) * kPartStride;
-        reinterpret_cast<float4*>(tile + row * kPartStride)[v] = ld16<float4>(src + 4 * v);
+        for (int i = tid; i < nr * kV; i += kFinThreads) {
+          const int row = i / kV, v = i % kV;
+          const int gr = r0 + row;
+          const float* src = p.scan_part + ((size_t)(w0 + s0 + gr / G + seg) * G + gr % G) * kPartStride;
+          reinterpret_cast<float4*>(tile + row * kPartStride)[v] = ld16<float4>(src + 4 * v);
+        }
+        __syncthreads();
       }
-      __syncthreads();
 #pragma unroll
       for (int i = 0; i < kH2; ++i) {
         const int j = half + 2 * i;
         if (j < G) {
-#pragma unroll 1
+#pragma unroll 4
           for (int row = (j - r0 % G + G) % G; row < nr; row += G) {
             const float* tr = tile + row * kPartStride;
             const float rl = tr[1];
-            if (rl > 0.f) {
-              const float mn = fmaxf(mrun[i], tr[0]);
-              const float s0f = lrun[i] > 0.f ? exp2f(mrun[i] - mn) : 0.f;
-              const float s1f = exp2f(tr[0] - mn);
-              lrun[i] = lrun[i] * s0f + rl * s1f;
-              arun[i] = arun[i] * s0f + tr[4 + c] * s1f;
-              mrun[i] = mn;
-            }
+            const float f = rl > 0.f ? exp2f(tr[0] - mh[i]) : 0.f;
+            lrun[i] = fmaf(rl, f, lrun[i]);
+            arun[i] = fmaf(tr[4 + c], f, arun[i]);
           }
         }
       }
-      __syncthreads();
+      if (!early_ok) __syncthreads();
     }
 #pragma unroll
     for (int i = 0; i < kH2; ++i) {
@@ -1086,7 +1098,7 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
       if (j < G) {
         P.sp[j][4 + c] = arun[i];
         if (c == 0) {
-          P.sp[j][0] = lrun[i] > 0.f ? mrun[i] : -INFINITY;
+          P.sp[j][0] = lrun[i] > 0.f ? mh[i] : -INFINITY;
           P.sp[j][1] = lrun[i];
         }
       }

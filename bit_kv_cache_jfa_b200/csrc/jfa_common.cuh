@@ -21,6 +21,8 @@ constexpr int kTail = JFA_TAIL_MAX;      // 64
 constexpr int kMaxG = JFA_MAX_GQA;       // 8
 constexpr int kPartStride = 132;         // floats per (slot, head): m, l, pad2, acc[128]
 constexpr int kMaxScanWarps = 4096;      // cap on scan warps (partial slots)
+constexpr int kScanMinRecords = 2;       // records per scan warp at least (when the
+                                         // work allows): fewer partials to merge
 constexpr int kScanHistBits = 13;        // selection-score histogram of the scan: top 13 key bits
 constexpr int kScanHistBins = 1 << kScanHistBits;
 constexpr int kHistBins = 2048;          // top-k first-level histogram (11 key bits)
@@ -365,6 +367,10 @@ __device__ __forceinline__ void set_flag(uint32_t* flag, uint32_t bits) {
 __device__ __forceinline__ uint32_t float_key(float f) {
   uint32_t u = __float_as_uint(f);
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+// Inverse of float_key.
+__device__ __forceinline__ float key_float(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
 }
 
 }  // namespace jfa

@@ -110,11 +110,10 @@ __global__ void __launch_bounds__(ScanCfg<KB, VB, NT>::NW * 32, 1) scan_kernel(c
       ++pf_seg;
     }
   };
-  if (lane == 0 && has_work) {
-#pragma unroll
-    for (int i = 0; i < S; ++i)
-      if (g0 + i < g1) issue_next(i);
-  }
+  // only the first stage now: every warp's first record is requested before
+  // any second one, so the first records arrive sooner; the other stages
+  // follow once the first has landed
+  if (lane == 0 && has_work) issue_next(0);
 
   // lane roles: B column gid of n-tile n = (head (gid >> 1) + 4n, limb gid & 1);
   // logits of head tig + 4n; value columns (heads) 2 tig, 2 tig + 1
@@ -201,7 +200,7 @@ __global__ void __launch_bounds__(ScanCfg<KB, VB, NT>::NW * 32, 1) scan_kernel(c
         // drain the copies still in flight before leaving (bounded)
         for (int i = 0; i < S; ++i) {
           const long long gj = gi + i;
-          if (gj >= g1) break;
+          if (gj >= g1 || (gi == g0 && i > 0)) break;  // later stages not yet requested
           const int sj = (st + i) % S;
           const uint32_t pj = par ^ (uint32_t)((st + i) / S);
           mbar_wait_bounded(&bar[sj], pj & 1u);
@@ -210,6 +209,11 @@ __global__ void __launch_bounds__(ScanCfg<KB, VB, NT>::NW * 32, 1) scan_kernel(c
       __syncwarp();
       failed = true;
       break;
+    }
+    if (gi == g0 && lane == 0) {
+#pragma unroll
+      for (int i = 1; i < S; ++i)
+        if (g0 + i < g1) issue_next(i);
     }
     const uint8_t* r = ring + st * REC;
 

@@ -277,6 +277,13 @@ int jfa_unpack_record(int32_t key_bits, int32_t val_bits, const void* record,
  * (for launch accounting); 0 on a bad geometry. */
 int jfa_decode_step_launches(const jfa_geom* geom, int32_t k);
 
+/* Number of warps jfa_decode_scores splits the quantized groups over on the
+ * current device (0 on a bad geometry or when no group is quantized).  Warp w
+ * takes a contiguous range of the flattened (segment, group) list and writes
+ * its softmax partial for segment s to slot w + s of the workspace's
+ * partials; exposed for inspection and tests. */
+int jfa_scan_warps(const jfa_geom* geom);
+
 #ifdef __cplusplus
 }
 #endif

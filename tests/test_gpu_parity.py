@@ -75,10 +75,8 @@ def scan_partials(run: GpuRun):
     ng = nq // 64
     n_seg = w.batch * w.kv_heads
     T = n_seg * ng
-    sms = torch.cuda.get_device_properties(0).multi_processor_count
-    rec = 512 + 1024 * w.key_bits + 1024 + 1024 * w.val_bits
-    nw = min(12 if w.group > 4 else 16, (227 * 1024 - 1024) // (2 * rec))   # warps per scan CTA
-    Wn = min(T, sms * nw, 4096)
+    Wn = _lib.jfa_scan_warps(g)  # warp w covers flattened groups [w T / Wn, (w + 1) T / Wn)
+    assert 1 <= Wn <= min(T, 4096)
     L = run.ws.layout
     G = w.group
     part = run.ws.buf[L.off_partials:L.off_partials + 4 * L.partial_slots * G * 132]
