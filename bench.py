@@ -119,7 +119,7 @@ def measured_peaks():
 
 def kernel_hash() -> str:
     h = hashlib.sha256()
-    for f in ("scores.cu", "jfa_common.cuh"):
+    for f in ("scores.cu", "jfa_common.cuh", "jfa_approx.cuh", "jfa_internal.cuh"):
         with open(os.path.join(ROOT, "bit_kv_cache_jfa_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
