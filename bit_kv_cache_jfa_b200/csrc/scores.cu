@@ -82,7 +82,6 @@ __global__ void __launch_bounds__(ScanCfg<KB, VB, NT>::NW * 32, 1) scan_kernel(c
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gid = lane >> 2, tig = lane & 3;
-  pdl_wait();
   const long long wg = (long long)blockIdx.x * NW + warp;
   const long long W = p.n_warps, T = p.total;
   const long long g0 = wg < W ? scan_range_begin(wg, W, T) : 0;
@@ -114,6 +113,11 @@ __global__ void __launch_bounds__(ScanCfg<KB, VB, NT>::NW * 32, 1) scan_kernel(c
   // any second one, so the first records arrive sooner; the other stages
   // follow once the first has landed
   if (lane == 0 && has_work) issue_next(0);
+  // Only now wait for the previous kernel in the stream: the first record
+  // copy reads the packed cache, which no kernel that releases this one
+  // early writes; the scores, histogram, partials and running maxima this
+  // kernel writes are read or cleared by the previous step's finishing kernel.
+  pdl_wait();
 
   // lane roles: B column gid of n-tile n = (head (gid >> 1) + 4n, limb gid & 1);
   // logits of head tig + 4n; value columns (heads) 2 tig, 2 tig + 1

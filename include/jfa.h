@@ -172,7 +172,11 @@ int jfa_pack_kv(const jfa_geom* geom, const jfa_cache* cache,
  *   q     : bf16 [B][H][128] device pointer, 16-B aligned.
  *   scale : softmax scale (e.g. 1/sqrt(128)).
  *   ws    : workspace for at least this geometry.
- * Writes S (workspace off_scores) and the split partials. */
+ * Writes S (workspace off_scores) and the split partials.  Launched as a
+ * programmatic dependent of the previous kernel in the stream: each warp's
+ * first packed-record copy may start before that kernel has finished when it
+ * releases its dependents early, so the packed records must not be written
+ * by such a kernel (this library's own packing kernel releases none). */
 int jfa_decode_scores(const jfa_geom* geom, const jfa_cache* cache,
                       const uint16_t* q, float scale, void* ws, void* stream);
 
