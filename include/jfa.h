@@ -234,7 +234,9 @@ int jfa_topk_noalloc(const float* scores, int32_t n_seg, int32_t stride,
  *   v_exact      : bf16 [B][H_kv][capacity][128], every cached token; device
  *                  memory, or pinned host memory the device can address
  *                  (exact_on_host = 1: rows are read by zero-copy loads).
- *   out          : fp32 [B][H][128] device pointer.
+ *   out          : fp32 [B][H][128]; device memory, or pinned host memory
+ *                  the device can address (the kernel's stores then cross
+ *                  the host link directly; no separate copy is needed).
  * Must follow jfa_decode_scores with the same geometry, q and scale. */
 int jfa_correct_merge(const jfa_geom* geom, const jfa_cache* cache,
                       const uint16_t* q, float scale, const int32_t* idx,

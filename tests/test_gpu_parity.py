@@ -216,6 +216,21 @@ def test_host_resident_rows_match_device_rows():
     assert np.array_equal(oa, ob)
 
 
+def test_output_in_pinned_host_memory():
+    # the finishing kernel writes out straight into pinned host memory
+    w = small(3, 2, heads=32, kv=8, ctx=3000, batch=2, topk=128)
+    run = GpuRun(w)
+    od, idd = run.fused_step()
+    out_h = torch.full(tuple(run.out.shape), float("nan"), dtype=torch.float32).pin_memory()
+    idx = torch.empty_like(run.idx)
+    _lib.check(_lib.jfa_decode_step(run.cache.geom(), run.cache.struct(), run.q, run.scale, run.k,
+                                    idx, run.k_exact, run.v_exact, run.exact_on_host, run.ws.buf,
+                                    out_h), "decode_step")
+    torch.cuda.synchronize()
+    assert np.array_equal(idx.cpu().numpy(), idd)
+    assert np.array_equal(out_h.double().numpy(), od)
+
+
 # ---------------------------------------------------------------- edge cases
 @pytest.mark.parametrize("ctx", [1, 37, 64, 65, 127, 128, 129, 191])
 def test_short_contexts(ctx):
