@@ -33,7 +33,7 @@ def build(verbose: bool = False, force: bool = False) -> str:
         t = os.path.getmtime(OUT)
         if all(os.path.getmtime(d) <= t for d in deps):
             return OUT
-    cmd = [nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3",
+    cmd = [nvcc(), "--threads", "0", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3",
            "-std=c++17", "--expt-relaxed-constexpr", "-Xcompiler", "-fPIC,-O2", "-shared",
            "-I", os.path.join(ROOT, "include"), "-I", os.path.join(PKG, "csrc"),
            "-o", OUT + ".tmp", *srcs]

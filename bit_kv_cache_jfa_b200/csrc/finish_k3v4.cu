@@ -1,0 +1,11 @@
+// finish_k3v4.cu — the finishing kernel for 3-bit keys and 4-bit values.
+#include "finish_impl.cuh"
+
+namespace jfa {
+
+int launch_finish_k3v4(const FinishParams& fp, int G, int n_seg, bool select, cudaStream_t st) {
+  return select ? launch_finish_g<true, 3, 4>(fp, G, n_seg, st)
+                : launch_finish_g<false, 3, 4>(fp, G, n_seg, st);
+}
+
+}  // namespace jfa

@@ -1,0 +1,11 @@
+// finish_k4v2.cu — the finishing kernel for 4-bit keys and 2-bit values.
+#include "finish_impl.cuh"
+
+namespace jfa {
+
+int launch_finish_k4v2(const FinishParams& fp, int G, int n_seg, bool select, cudaStream_t st) {
+  return select ? launch_finish_g<true, 4, 2>(fp, G, n_seg, st)
+                : launch_finish_g<false, 4, 2>(fp, G, n_seg, st);
+}
+
+}  // namespace jfa
