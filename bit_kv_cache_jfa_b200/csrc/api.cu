@@ -46,9 +46,10 @@ int workspace_layout(const jfa_geom& g, int max_topk, jfa_workspace_layout* out)
   L.off_counters = off;
   off = align_up(off + n_seg * 8 * sizeof(uint32_t), 256);
   // top-k lists: per 4096-score chunk, up to 4096 (key, index) pairs; then counts
-  // (also holds the per-CTA lists of the fused finishing kernel: <= capacity + 512)
+  // (also holds the per-CTA lists of the fused finishing kernel: slices of
+  // the quantized tokens rounded up to 64, <= capacity + 64 per CTA)
   const size_t n_chunks_cap = ((size_t)g.capacity + 4095) / 4096;
-  const size_t cap_fused = (size_t)g.capacity + 512;
+  const size_t cap_fused = (size_t)g.capacity + 64 * kFinMaxCluster;
   L.cand_cap = (int32_t)(n_chunks_cap * 4096 > cap_fused ? n_chunks_cap * 4096 : cap_fused);
   L.off_cand = off;
   off = align_up(off + n_seg * (size_t)L.cand_cap * 2 * sizeof(uint32_t), 256);

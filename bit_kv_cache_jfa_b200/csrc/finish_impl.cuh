@@ -1,5 +1,5 @@
 // finish_impl.cuh — everything after the scan in one kernel.  A thread-block
-// cluster of C CTAs (C <= 8) per (sequence, KV head):
+// cluster of C CTAs (C <= 16) per (sequence, KV head):
 //   T   (before waiting for the scan) corrects its share of the bf16 tail;
 //   P1  reads the scan's 8192-bin histogram of the selection keys and finds
 //       the bin b* holding the k-th largest key (every CTA, redundantly);
@@ -31,7 +31,7 @@ namespace cg = cooperative_groups;
 namespace jfa {
 
 constexpr int kFinThreads = 256;
-constexpr int kFinMaxC = 8;
+constexpr int kFinMaxC = kFinMaxCluster;  // 16: non-portable cluster size, few segments only
 constexpr int kLCap = 1024;   // sure / tie list entries per CTA
 constexpr int kTCap = 1024;   // gathered tie entries
 constexpr int kRefBins = 2048;
@@ -1118,11 +1118,34 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
   //   out = (a_c 2^(m_c-m) + a_a 2^(m_a-m)) / (l_c 2^(m_c-m) + l_a 2^(m_a-m))
   for (int j = r; j < G; j += C) {
     const int c = tid;
-    if (c < kD) {
-      float2 hd[kFinMaxC][2];
-      float av[kFinMaxC][2];
+    if (c < kD && C > 8) {  // large clusters: frame first, then the sums (re-reading the frames)
+      float ma = -INFINITY, mc = -INFINITY;
+#pragma unroll 4
+      for (int q = 0; q < C; ++q) {
+        const FinParts<G>* o = cl.map_shared_rank(&P, q);
+        const float2 ha = *reinterpret_cast<const float2*>(&o->sp[j][0]);
+        const float2 hc = *reinterpret_cast<const float2*>(&o->run[j][0]);
+        if (ha.y > 0.f) ma = fmaxf(ma, ha.x);
+        mc = fmaxf(mc, hc.x);
+      }
+      const float m = fmaxf(ma, mc);
+      float l = 0.f, acc = 0.f;
+#pragma unroll 4
+      for (int q = 0; q < C; ++q) {
+        const FinParts<G>* o = cl.map_shared_rank(&P, q);
+        const float2 ha = *reinterpret_cast<const float2*>(&o->sp[j][0]);
+        const float2 hc = *reinterpret_cast<const float2*>(&o->run[j][0]);
+        const float fa = ha.y > 0.f ? exp2f(ha.x - m) : 0.f;
+        const float fc = hc.x == -INFINITY ? 0.f : exp2f(hc.x - m);
+        l = fmaf(ha.y, fa, fmaf(hc.y, fc, l));
+        acc = fmaf(o->sp[j][4 + c], fa, fmaf(o->run[j][4 + c], fc, acc));
+      }
+      p.out[((size_t)bb * p.H + hh * G + j) * kD + c] = acc / l;
+    } else if (c < kD) {
+      float2 hd[8][2];
+      float av[8][2];
 #pragma unroll
-      for (int q = 0; q < kFinMaxC; ++q) {
+      for (int q = 0; q < 8; ++q) {
         if (q < C) {
           FinParts<G>* o = cl.map_shared_rank(&P, q);
           hd[q][0] = *reinterpret_cast<const float2*>(&o->sp[j][0]);
@@ -1133,7 +1156,7 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
       }
       float ma = -INFINITY, mc = -INFINITY;
 #pragma unroll
-      for (int q = 0; q < kFinMaxC; ++q)
+      for (int q = 0; q < 8; ++q)
         if (q < C) {
           if (hd[q][0].y > 0.f) ma = fmaxf(ma, hd[q][0].x);
           mc = fmaxf(mc, hd[q][1].x);
@@ -1141,7 +1164,7 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
       const float m = fmaxf(ma, mc);
       float l = 0.f, acc = 0.f;
 #pragma unroll
-      for (int q = 0; q < kFinMaxC; ++q)
+      for (int q = 0; q < 8; ++q)
         if (q < C) {
           const float fa = hd[q][0].y > 0.f ? exp2f(hd[q][0].x - m) : 0.f;
           const float fc = hd[q][1].x == -INFINITY ? 0.f : exp2f(hd[q][1].x - m);
@@ -1156,10 +1179,10 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
 }
 
 template <int G, bool SEL, int KB, int VB>
-static int pick_cluster(int n_seg, int num_sms) {
+static int pick_cluster(int n_seg, int max_c, int num_sms) {
   constexpr size_t smem = fin_smem_bytes<G>();
   int best = 1;
-  for (int c = 2; c <= kFinMaxC; c *= 2) {
+  for (int c = 2; c <= max_c; c *= 2) {
     if ((long long)n_seg * c > 2LL * num_sms) break;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(n_seg * c);
@@ -1187,26 +1210,35 @@ template <int G, bool SEL, int KB, int VB>
 static int launch_finish_t(FinishParams fp, int n_seg, cudaStream_t st) {
   constexpr size_t smem = fin_smem_bytes<G>();
   static bool configured[64] = {false};
-  static int memo_seg[64][8] = {{0}}, memo_c[64][8] = {{0}};  // cluster size per (device, n_seg)
+  static int memo_seg[64][8] = {{0}}, memo_c[64][8] = {{0}};  // cluster size per (device, key)
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !configured[dev]) {
     if (cudaFuncSetAttribute(finish_kernel<G, SEL, KB, VB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem) != cudaSuccess)
       return JFA_ERR_CUDA;
+    // clusters of 16 (beyond the portable 8) for workloads with few segments;
+    // if the device refuses, the occupancy query below keeps clusters <= 8
+    if (cudaFuncSetAttribute(finish_kernel<G, SEL, KB, VB>, cudaFuncAttributeNonPortableClusterSizeAllowed,
+                             1) != cudaSuccess)
+      cudaGetLastError();
     configured[dev] = true;
   }
+  // clusters of 16 pay off once the slices are long (measured: 32K-token
+  // segments gain, 8K ones lose); memoized per (segments, cap)
+  const int max_c = fp.nq >= 16384 ? kFinMaxC : 8;
+  const int key = n_seg * 2 + (max_c > 8 ? 1 : 0);
   int C = 0;
   if (dev >= 0 && dev < 64) {
     for (int i = 0; i < 8; ++i)
-      if (memo_seg[dev][i] == n_seg) C = memo_c[dev][i];
+      if (memo_seg[dev][i] == key) C = memo_c[dev][i];
   }
   if (C == 0) {
-    C = pick_cluster<G, SEL, KB, VB>(n_seg, num_sms_current());
+    C = pick_cluster<G, SEL, KB, VB>(n_seg, max_c, num_sms_current());
     if (dev >= 0 && dev < 64) {
       for (int i = 0; i < 8; ++i)
         if (memo_seg[dev][i] == 0) {
-          memo_seg[dev][i] = n_seg;
+          memo_seg[dev][i] = key;
           memo_c[dev][i] = C;
           break;
         }

@@ -21,6 +21,7 @@ constexpr int kTail = JFA_TAIL_MAX;      // 64
 constexpr int kMaxG = JFA_MAX_GQA;       // 8
 constexpr int kPartStride = 132;         // floats per (slot, head): m, l, pad2, acc[128]
 constexpr int kMaxScanWarps = 4096;      // cap on scan warps (partial slots)
+constexpr int kFinMaxCluster = 16;       // CTAs per (sequence, KV head) in the finishing kernel
 constexpr int kScanMinRecords = 2;       // records per scan warp at least (when the
                                          // work allows): fewer partials to merge
 constexpr int kScanHistBits = 13;        // selection-score histogram of the scan: top 13 key bits
