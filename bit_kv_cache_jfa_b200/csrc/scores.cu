@@ -233,6 +233,13 @@ __global__ void __launch_bounds__(ScanCfg<KB, VB, NT>::NW * 32, 1) scan_kernel(c
 #pragma unroll
       for (int n = 0; n < NT; ++n) q_tilde_col(q2[n], sf, lo_lane, qb[n]);
     }
+    // the bias of an absent head is -inf, so its logits are -inf without a
+    // select per logit (kept per logit for K4V4 with two n-tiles, where the
+    // register allocation measured slower the other way)
+    constexpr bool kInfBias = !(KB == 4 && VB == 4 && NT == 2);
+    float bku[NT];
+#pragma unroll
+    for (int n = 0; n < NT; ++n) bku[n] = (!kInfBias || hv[n]) ? bk[n] : -INFINITY;
 
     // ---- approximate logits (log2 units): u[mt][n][r] of head tig + 4n,
     // token 16 mt + gid + 8 r
@@ -255,8 +262,8 @@ __global__ void __launch_bounds__(ScanCfg<KB, VB, NT>::NW * 32, 1) scan_kernel(c
       for (int n = 0; n < NT; ++n) {
         float d[4];
         qk_chain(a, qb[n], d);
-        u[mt][n][0] = hv[n] ? approx_logit(d, 0, kappa_u, bk[n]) : -INFINITY;
-        u[mt][n][1] = hv[n] ? approx_logit(d, 1, kappa_u, bk[n]) : -INFINITY;
+        u[mt][n][0] = (kInfBias || hv[n]) ? approx_logit(d, 0, kappa_u, bku[n]) : -INFINITY;
+        u[mt][n][1] = (kInfBias || hv[n]) ? approx_logit(d, 1, kappa_u, bku[n]) : -INFINITY;
       }
     }
 

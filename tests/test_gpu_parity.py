@@ -291,6 +291,20 @@ def test_fused_step_matches_separate_calls(kb, vb, heads, kv, ctx, k, batch):
         assert_out_close(out1, run.oracle_step(idx=idx1).out)
 
 
+@pytest.mark.parametrize("kb,vb,heads,kv", [(3, 2, 8, 2), (4, 4, 32, 4)])
+def test_long_segments_sixteen_cta_clusters(kb, vb, heads, kv):
+    # few segments of >= 16K quantized tokens: the finishing kernel runs
+    # clusters of 16 CTAs; it must agree with the separate calls and the oracle
+    w = small(kb, vb, heads=heads, kv=kv, ctx=20000, batch=1, topk=384, planted=32)
+    run = GpuRun(w)
+    out3, idx3 = run.step()
+    out1, idx1 = run.fused_step()
+    assert np.array_equal(idx1, idx3)
+    assert np.allclose(out1, out3, rtol=1e-5, atol=1e-6)
+    assert_topk_valid(idx1, run.oracle_step().select, w.topk)
+    assert_out_close(out1, run.oracle_step(idx=idx1).out)
+
+
 def test_fused_step_tiny_workload_against_oracle():
     w = W.WORKLOADS["tiny_k4v4_4k"]
     run = GpuRun(w)
