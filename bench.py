@@ -450,6 +450,7 @@ def run_jfa(args, w):
     if rank == 0:
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
+            k_exact, v_exact = copies[0][3], copies[0][4]
             kv_cpu = lambda b, h: (k_exact[b, h].cpu(), v_exact[b, h].cpu())
             val, n, spent = time_oracle(w, args.cpu_seconds, kv_cpu)
             cpu = {"value": val, "unit": "tokens/s", "cores": oracle_cores(), "kind": "oracle",
