@@ -8,14 +8,6 @@ namespace jfa {
 
 constexpr unsigned kAll = 0xFFFFFFFFu;
 
-__device__ __forceinline__ float bf16f(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
-
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kAll, v, o);
-  return v;
-}
-
 // Block-wide exclusive sum over threads in DESCENDING thread order:
 // returns the sum of v over threads with a larger index.
 __device__ __forceinline__ uint32_t block_suffix_excl(uint32_t v, uint32_t* scratch) {

@@ -206,70 +206,13 @@ __device__ __forceinline__ uint32_t h2_fma(uint32_t a, uint32_t b, uint32_t c) {
   asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
   return r;
 }
-__device__ __forceinline__ uint32_t h2_sub(uint32_t a, uint32_t b) {
-  uint32_t r;
-  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
-  return r;
-}
 __device__ __forceinline__ uint32_t h2_mul(uint32_t a, uint32_t b) {
   uint32_t r;
   asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
   return r;
 }
 
-constexpr uint32_t kMagic = 0x64006400u;  // fp16x2 (1024, 1024)
-// fp16x2 constants (2^-pos, 2^-pos) and (-1024*2^-pos, ...)
-constexpr uint32_t kOneH2 = 0x3C003C00u;      // 1.0
-constexpr uint32_t kS4 = 0x34003400u;          // 1/4
-constexpr uint32_t kS8 = 0x30003000u;          // 1/8
-constexpr uint32_t kS16 = 0x2C002C00u;         // 1/16
-constexpr uint32_t kS64 = 0x24002400u;         // 1/64
-constexpr uint32_t kS256 = 0x1C001C00u;        // 1/256
-constexpr uint32_t kB0 = 0xE400E400u;          // -1024
-constexpr uint32_t kB2 = 0xDC00DC00u;          // -256
-constexpr uint32_t kB3 = 0xD800D800u;          // -128
-constexpr uint32_t kB4 = 0xD400D400u;          // -64
-constexpr uint32_t kB6 = 0xCC00CC00u;          // -16
-constexpr uint32_t kB8 = 0xC400C400u;          // -4
-
-// 4-bit word -> 4 fp16x2 code pairs (positions 0, 4, 8, 12)
-__device__ __forceinline__ void unpack4(uint32_t w, uint32_t* o) {
-  uint32_t w8 = w >> 8;
-  o[0] = h2_sub(lop_and_or(w, 0x000F000Fu, kMagic), kMagic);
-  o[1] = h2_fma(lop_and_or(w, 0x00F000F0u, kMagic), kS16, kB4);
-  o[2] = h2_sub(lop_and_or(w8, 0x000F000Fu, kMagic), kMagic);
-  o[3] = h2_fma(lop_and_or(w8, 0x00F000F0u, kMagic), kS16, kB4);
-}
-// 2-bit word -> 8 fp16x2 code pairs (positions 0, 2, ..., 14)
-__device__ __forceinline__ void unpack2(uint32_t w, uint32_t* o) {
-  uint32_t ws = w >> 10;
-  o[0] = h2_sub(lop_and_or(w, 0x00030003u, kMagic), kMagic);
-  o[1] = h2_fma(lop_and_or(w, 0x000C000Cu, kMagic), kS4, kB2);
-  o[2] = h2_fma(lop_and_or(w, 0x00300030u, kMagic), kS16, kB4);
-  o[3] = h2_fma(lop_and_or(w, 0x00C000C0u, kMagic), kS64, kB6);
-  o[4] = h2_fma(lop_and_or(w, 0x03000300u, kMagic), kS256, kB8);
-  o[5] = h2_sub(lop_and_or(ws, 0x00030003u, kMagic), kMagic);
-  o[6] = h2_fma(lop_and_or(ws, 0x000C000Cu, kMagic), kS4, kB2);
-  o[7] = h2_fma(lop_and_or(ws, 0x00300030u, kMagic), kS16, kB4);
-}
-// three 3-bit words -> 16 fp16x2 code pairs (five per word + one split pair)
-__device__ __forceinline__ void unpack3_word(uint32_t w, uint32_t* o) {
-  uint32_t ws = w >> 9;
-  o[0] = h2_sub(lop_and_or(w, 0x00070007u, kMagic), kMagic);
-  o[1] = h2_fma(lop_and_or(w, 0x00380038u, kMagic), kS8, kB3);
-  o[2] = h2_fma(lop_and_or(w, 0x01C001C0u, kMagic), kS64, kB6);
-  o[3] = h2_sub(lop_and_or(ws, 0x00070007u, kMagic), kMagic);
-  o[4] = h2_fma(lop_and_or(ws, 0x00380038u, kMagic), kS8, kB3);
-}
-__device__ __forceinline__ void unpack3(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t* o) {
-  unpack3_word(w0, o);
-  unpack3_word(w1, o + 5);
-  unpack3_word(w2, o + 10);
-  uint32_t t = lop_and_or(w0 >> 15, 0x00010001u, kMagic);
-  t = lop_and_or(w1 >> 14, 0x00020002u, t);
-  t = lop_and_or(w2 >> 13, 0x00040004u, t);
-  o[15] = h2_sub(t, kMagic);
-}
+constexpr uint32_t kOneH2 = 0x3C003C00u;  // fp16x2 (1.0, 1.0)
 
 // ---------------------------------------------------------------------------
 // mma.sync m16n8k16, fp16 inputs, fp32 accumulate (D += A * B)
@@ -286,9 +229,6 @@ __device__ __forceinline__ void mma16816(float* d, uint32_t a0, uint32_t a1, uin
 __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
   __half2 h = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
-}
-__device__ __forceinline__ float2 unpack_h2(uint32_t v) {
-  return __half22float2(*reinterpret_cast<__half2*>(&v));
 }
 
 // ---------------------------------------------------------------------------
