@@ -457,6 +457,14 @@ def run_jfa(args, w):
                    "sample": f"{n} of {w.batch * w.kv_heads} (sequence, KV head) segments "
                              f"({w.ctx} tokens each) in {spent:.1f} s, extrapolated to a "
                              f"full step"}
+            try:  # the same oracle on one core (numpy's BLAS pool limited to 1 thread)
+                from threadpoolctl import threadpool_limits
+                with threadpool_limits(limits=1):
+                    v1, n1, s1 = time_oracle(w, args.cpu_seconds / 2, kv_cpu)
+                cpu["one_core"] = {"value": v1, "cores": 1,
+                                   "sample": f"{n1} segments in {s1:.1f} s, extrapolated"}
+            except ImportError:
+                pass
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
