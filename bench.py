@@ -394,6 +394,26 @@ def run_jfa(args, w):
     ms = e0.elapsed_time(e1) / args.steps
     ms_max = max_over_ranks(ms, world, dev)
 
+    # the same steps as the three separate calls (scores, top-k, correct+merge)
+    # instead of the fused finishing kernel, for reference
+    def step3(i):
+        _, g, cs, ke, ve = copies[i % n_copies]
+        _lib.check(_lib.jfa_decode_scores(g, cs, q, scale, ws.buf, sp), "scores")
+        _lib.check(_lib.jfa_topk(g, w.topk, ws.buf, idx, sp), "topk")
+        _lib.check(_lib.jfa_correct_merge(g, cs, q, scale, idx, w.topk, ke, ve, host, ws.buf, out,
+                                          sp), "correct_merge")
+
+    for i in range(3):
+        step3(i)
+    u0, u1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    u0.record(stream)
+    for i in range(args.steps):
+        step3(i)
+    u1.record(stream)
+    torch.cuda.synchronize()
+    unfused_ms = u0.elapsed_time(u1) / args.steps
+
     # the scan kernel alone (roofline): its own launches back to back over the
     # same rotation, on a workspace of its own (scan-only launches leave the
     # selection histogram for a finishing kernel to consume)
@@ -483,6 +503,8 @@ def run_jfa(args, w):
                     "ms_per_step": e2e_max,
                     "h2d_bytes_per_step": q.numel() * q.element_size(),
                     "d2h_bytes_per_step": out.numel() * out.element_size()},
+            "unfused": {"ms_per_step": unfused_ms,
+                        "calls": "jfa_decode_scores + jfa_topk + jfa_correct_merge"},
             "gpu_launches": launches * args.steps,
             "clocks": clk,
             "wall_s_timed_region": wall,
