@@ -253,10 +253,8 @@ __device__ __forceinline__ uint32_t lower_bound_u32(const uint32_t* a, uint32_t 
 }
 
 // ---------------------------------------------------------------------------
-// Correction, a warp per token.  Token encoding: t in [0, nq) a quantized
-// token, (1 << 30) | s the tail slot s.  Lane l owns channels 4l..4l+3 of
-// every head.  The quantized token's record pieces are staged by cp.async
-// kWD tokens ahead; its exact bf16 row is loaded one token ahead.
+// Correction helpers.  Token encoding: t in [0, nq) a quantized token,
+// (1 << 30) | s the tail slot s (exact rows only); -1 an empty batch slot.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ bool tok_quant(int t) { return t >= 0 && !(t & (1 << 30)); }
 
