@@ -87,6 +87,7 @@ SIGNATURES = {
                                     POINTER(c_uint16), POINTER(c_uint16), POINTER(c_uint8),
                                     POINTER(c_uint16), POINTER(c_uint16)]),
     "jfa_decode_step_launches": (c_int32, [POINTER(Geom), c_int32]),
+    "jfa_selftest_bounded_wait": (c_int32, [POINTER(Geom), c_void_p, c_void_p]),
     "jfa_scan_warps": (c_int32, [POINTER(Geom)]),
 }
 
@@ -194,6 +195,10 @@ def jfa_decode_finish(geom, cache, q, scale, k, idx, k_exact, v_exact, exact_on_
     return load().jfa_decode_finish(ctypes.byref(geom), ctypes.byref(cache), _ptr(q), scale, k,
                                     _ptr(idx), _ptr(k_exact), _ptr(v_exact), int(exact_on_host),
                                     _ptr(ws), _ptr(out), _stream(stream))
+
+
+def jfa_selftest_bounded_wait(geom, ws, stream=None) -> int:
+    return load().jfa_selftest_bounded_wait(ctypes.byref(geom), _ptr(ws), _stream(stream))
 
 
 def jfa_clear_error(geom, ws, stream=None) -> int:

@@ -95,6 +95,12 @@ ScanPlan scan_plan(const jfa_geom& g, int num_sms) {
 
 using namespace jfa;
 
+// selftest.cu: one warp waits on an mbarrier that never completes; the
+// bounded wait sets JFA_DEVERR_TIMEOUT in *flag.
+namespace jfa {
+int launch_bounded_wait_selftest(uint32_t* flag, cudaStream_t st);
+}
+
 extern "C" {
 
 const char* jfa_status_string(int status) {
@@ -224,6 +230,14 @@ int jfa_scan_warps(const jfa_geom* geom) {
   if (!geom_ok(geom) || geom->n_ctx < 1) return 0;
   const ScanPlan plan = scan_plan(*geom, num_sms_current());
   return plan.total_groups > 0 ? plan.n_warps : 0;
+}
+
+int jfa_selftest_bounded_wait(const jfa_geom* geom, void* ws, void* stream) {
+  if (!geom_ok(geom) || !ws) return JFA_ERR_INVALID_ARG;
+  jfa_workspace_layout L;
+  workspace_layout(*geom, 1, &L);
+  return launch_bounded_wait_selftest(reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + L.off_flag),
+                                      static_cast<cudaStream_t>(stream));
 }
 
 int jfa_clear_error(const jfa_geom* geom, void* ws, void* stream) {

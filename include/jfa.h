@@ -262,6 +262,14 @@ int jfa_decode_finish(const jfa_geom* geom, const jfa_cache* cache,
                       const uint16_t* k_exact, const uint16_t* v_exact,
                       int32_t exact_on_host, void* ws, float* out, void* stream);
 
+/* Failure-detection self test: launches one warp that waits, with the same
+ * bounded wait the scan uses for its record copies, on an mbarrier whose
+ * phase cannot complete.  After about one second the wait gives up and the
+ * kernel sets JFA_DEVERR_TIMEOUT in the workspace flag; nothing faults and the
+ * context stays usable (read the flag with jfa_check_error, then clear it).
+ * Stream-ordered; JFA_ERR_INVALID_ARG on a bad geometry or null workspace. */
+int jfa_selftest_bounded_wait(const jfa_geom* geom, void* ws, void* stream);
+
 /* Clear the workspace error flag (stream-ordered). */
 int jfa_clear_error(const jfa_geom* geom, void* ws, void* stream);
 

@@ -231,6 +231,20 @@ def test_output_in_pinned_host_memory():
     assert np.array_equal(out_h.double().numpy(), od)
 
 
+def test_bounded_wait_gives_up_and_the_context_stays_usable():
+    # a wait that nothing completes ends after ~1 s with the timeout flag set
+    w = small(3, 2, heads=8, kv=2, ctx=3000, batch=1, topk=64)
+    run = GpuRun(w)
+    g = run.cache.geom()
+    _lib.check(_lib.jfa_clear_error(g, run.ws.buf), "clear")
+    _lib.check(_lib.jfa_selftest_bounded_wait(g, run.ws.buf), "selftest")
+    st, flag = _lib.jfa_check_error(g, run.ws.buf)
+    assert flag == _lib.DEVERR_TIMEOUT and st == _lib.JFA_ERR_DEVICE
+    _lib.check(_lib.jfa_clear_error(g, run.ws.buf), "clear")
+    out, idx = run.fused_step()  # asserts a clear flag itself
+    assert_out_close(out, run.oracle_step(idx=idx).out)
+
+
 # ---------------------------------------------------------------- edge cases
 @pytest.mark.parametrize("ctx", [1, 37, 64, 65, 127, 128, 129, 191])
 def test_short_contexts(ctx):
