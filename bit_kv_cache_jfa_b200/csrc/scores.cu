@@ -450,12 +450,14 @@ __global__ void __launch_bounds__(ScanCfg<KB, VB, NT>::NW * 32, 1) scan_kernel(c
 template <int KB, int VB, int NT>
 static int launch_scan_t(const ScanParams& sp, int n_ctas, cudaStream_t st) {
   using Cfg = ScanCfg<KB, VB, NT>;
-  static bool configured = false;
-  if (!configured) {
+  static bool configured[64] = {false};  // per device: the attribute is set on each
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64 || !configured[dev]) {
     if (cudaFuncSetAttribute(scan_kernel<KB, VB, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              Cfg::SMEM) != cudaSuccess)
       return JFA_ERR_CUDA;
-    configured = true;
+    if (dev >= 0 && dev < 64) configured[dev] = true;
   }
   return launch_pdl(scan_kernel<KB, VB, NT>, dim3(n_ctas), dim3(Cfg::NW * 32), (size_t)Cfg::SMEM,
                     st, sp) == cudaSuccess
