@@ -21,7 +21,7 @@ from ._lib import (  # noqa: F401  (re-exported C ABI names)
     jfa_decode_step_launches, jfa_pack_kv, jfa_topk, jfa_unpack_record,
     jfa_workspace_layout_get, load)
 
-__all__ = ["KVCache", "Workspace", "decode_step", "JfaError", "load"]
+__all__ = ["KVCache", "Workspace", "decode_step", "DecodeGraph", "JfaError", "load"]
 
 
 def _torch():
@@ -114,3 +114,39 @@ def decode_step(cache: KVCache, q, k: int, k_exact, v_exact, ws: Workspace, scal
     check(jfa_decode_step(cache.geom(), cache.struct(), q, float(scale), k, idx, k_exact,
                           v_exact, exact_on_host, ws.buf, out, stream), "jfa_decode_step")
     return out, idx
+
+
+class DecodeGraph:
+    """decode_step captured once in a CUDA graph and replayed.
+
+    The graph holds the step's two kernel launches with their arguments as
+    they were at capture: the cache length, every buffer address (q, the
+    exact rows, the workspace, out, idx) and k.  Write the next query into
+    the same q tensor and call replay(); after appending to the cache,
+    capture a new graph (the length is part of the launch arguments)."""
+
+    def __init__(self, cache: KVCache, q, k: int, k_exact, v_exact, ws: Workspace, scale=None,
+                 out=None, idx=None, exact_on_host: bool = False):
+        torch = _torch()
+        dev = cache.groups.device
+        if out is None:
+            out = torch.empty(cache.batch, cache.num_heads, cache.head_dim, dtype=torch.float32,
+                              device=dev)
+        if idx is None:
+            idx = torch.empty(cache.batch, cache.num_kv_heads, k, dtype=torch.int32, device=dev)
+        self.out, self.idx = out, idx
+        args = (cache, q, k, k_exact, v_exact, ws)
+        kw = dict(scale=scale, out=out, idx=idx, exact_on_host=exact_on_host)
+        side = torch.cuda.Stream(device=dev)
+        side.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(side):  # one eager step: one-time kernel set-up stays out of the graph
+            decode_step(*args, stream=side, **kw)
+        torch.cuda.current_stream(dev).wait_stream(side)
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            decode_step(*args, stream=torch.cuda.current_stream(dev), **kw)
+
+    def replay(self):
+        """Run the captured step on the current stream; returns (out, idx)."""
+        self.graph.replay()
+        return self.out, self.idx

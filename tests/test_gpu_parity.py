@@ -7,6 +7,7 @@ import torch
 
 import oracle.jfa_oracle as O
 import workloads as W
+import bit_kv_cache_jfa_b200 as jfa
 from bit_kv_cache_jfa_b200 import _lib
 
 from jfa_testutil import (GpuRun, SCORE_ABS, assert_out_close, assert_topk_valid)
@@ -229,6 +230,29 @@ def test_output_in_pinned_host_memory():
     torch.cuda.synchronize()
     assert np.array_equal(idx.cpu().numpy(), idd)
     assert np.array_equal(out_h.double().numpy(), od)
+
+
+def test_decode_graph_replay_equals_eager_step():
+    w = small(3, 2, heads=32, kv=8, ctx=5000, batch=2, topk=128)
+    run = GpuRun(w)
+    od, idd = run.fused_step()
+    q = run.q.clone()
+    graph = jfa.DecodeGraph(run.cache, q, run.k, run.k_exact, run.v_exact, run.ws,
+                            scale=run.scale, exact_on_host=bool(run.exact_on_host))
+    for _ in range(3):
+        out, idx = graph.replay()
+    torch.cuda.synchronize()
+    assert np.array_equal(idx.cpu().numpy(), idd)
+    assert np.array_equal(out.cpu().double().numpy(), od)
+    # a new query written into the captured q buffer is picked up by the next replay
+    q.copy_(torch.flip(run.q, dims=[1]))
+    out, idx = graph.replay()
+    torch.cuda.synchronize()
+    ref = jfa.decode_step(run.cache, q, run.k, run.k_exact, run.v_exact, run.ws, scale=run.scale,
+                          exact_on_host=bool(run.exact_on_host))
+    torch.cuda.synchronize()
+    assert np.array_equal(idx.cpu().numpy(), ref[1].cpu().numpy())
+    assert np.array_equal(out.cpu().numpy(), ref[0].cpu().numpy())
 
 
 def test_bounded_wait_gives_up_and_the_context_stays_usable():
