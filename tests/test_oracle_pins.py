@@ -118,6 +118,79 @@ def test_grid_data_reconstructs_exactly():
         assert np.array_equal(O.dequantize_keys(kc, ks, kz)[0, 0], k)
 
 
+def test_value_round_trip_through_pack_cache():
+    # values are quantized per (token, 32-channel group): the dequantized
+    # cache the step aggregates stays within half a step of the bf16 input
+    for kb, vb, lognormal in ((3, 2, False), (4, 4, True)):
+        w = W.Workload("vrt", batch=2, heads=4, kv_heads=2, ctx=321, key_bits=kb,
+                       val_bits=vb, topk=8, planted=4, seed=23, value_lognormal=lognormal)
+        q = W.gen_q(w)
+        k, v = W.gen_kv(w, q)
+        v = v.double().numpy()
+        cache = O.pack_cache(k.double().numpy(), v, w.ctx, kb, vb)
+        nq = cache.n_quant
+        vh = cache.v_hat()
+        assert vh.shape == (2, 2, nq, 128)
+        step = np.repeat(cache.v_scale.astype(np.float64), 32, axis=-1)   # [B,H,N_q,128]
+        assert np.all(np.abs(v[:, :, :nq] - vh) <= step / 2 * (1 + 1e-12))
+        # the bound is tight somewhere (not a vacuous huge scale)
+        assert np.max(np.abs(v[:, :, :nq] - vh) / step) > 0.4
+        grp = v[:, :, :nq].reshape(2, 2, nq, 4, 32)
+        assert np.all(cache.v_zero.astype(np.float64) <= grp.min(-1))
+
+
+def test_value_grid_data_reconstructs_exactly():
+    # value rows on a grid zero + scale * code (per token and channel group)
+    # come back bit for bit, with the codes, scales and zeros that built them
+    rng = np.random.default_rng(9)
+    for bits in (2, 4):
+        lv = (1 << bits) - 1
+        n = 128
+        codes = rng.integers(0, lv + 1, (n, 4, 32))
+        codes[:, :, 0], codes[:, :, 1] = 0, lv
+        zero = rng.choice([-2.0, -0.5, 0.25, 1.0], (n, 4))
+        scale = rng.choice([0.0625, 0.25, 1.0], (n, 4))
+        v = (zero[..., None] + scale[..., None] * codes).reshape(n, 128)
+        vc, vs, vz = O.quantize_values(v[None, None], bits)
+        assert np.array_equal(vc[0, 0].reshape(n, 4, 32), codes)
+        assert np.array_equal(vs[0, 0].astype(np.float64), scale)
+        assert np.array_equal(vz[0, 0].astype(np.float64), zero)
+        assert np.array_equal(O.dequantize_values(vc, vs, vz)[0, 0], v)
+
+
+@pytest.mark.parametrize("kb,vb", [(3, 2), (4, 4)])
+def test_affine_identity_on_the_value_side(kb, vb):
+    # HACK review, Eq. (4) applied to P V: sum_t p_t (s_v v' + m_v) is the
+    # integer-code product weighted by p_t s_v plus the zero-point term
+    # sum_t p_t m_v, computed here from the raw codes, scales and zeros
+    w, q, k, v, cache = _small(kb=kb, vb=vb, lognormal=True)
+    rng = np.random.default_rng(4)
+    nq = cache.n_quant
+    p = rng.random(nq)
+    codes = cache.v_codes[1, 0].astype(np.float64).reshape(nq, 4, 32)
+    s = cache.v_scale[1, 0].astype(np.float64)          # [N_q, 4]
+    z = cache.v_zero[1, 0].astype(np.float64)
+    integer_part = np.einsum("tj,tjc->jc", p[:, None] * s, codes)
+    zero_part = (p[:, None] * z).sum(0)[:, None]
+    direct = (integer_part + zero_part).reshape(128)
+    assert np.allclose(p @ cache.v_hat()[1, 0], direct, rtol=1e-12, atol=1e-12)
+
+
+def test_exact_attention_is_torch_softmax_attention():
+    w, q, k, v, cache = _small(heads=8, kv=2)
+    scale = 0.083
+    got = O.exact_attention(q, k, v, w.ctx, scale)
+    for b in range(2):
+        for hq in range(8):
+            h = hq // 4
+            ref = _torch_attention(q[b, hq], k[b, h, :w.ctx], v[b, h, :w.ctx], scale)
+            assert np.allclose(got[b, hq], ref, rtol=1e-12, atol=1e-13)
+    # a shorter context ignores the later tokens
+    got2 = O.exact_attention(q, k, v, 100, scale)
+    ref2 = _torch_attention(q[1, 3], k[1, 0, :100], v[1, 0, :100], scale)
+    assert np.allclose(got2[1, 3], ref2, rtol=1e-12, atol=1e-13)
+
+
 def test_split_point_closed_form():
     assert [O.split_point(n) for n in (0, 1, 63, 64, 65, 128, 129, 4096)] == \
         [0, 0, 0, 0, 64, 64, 128, 4032]
@@ -326,3 +399,42 @@ def test_topk_empty_rows_pad_with_minus_one():
     # N_q = 0 (context within the tail): no quantized token can be chosen
     out = O.topk_indices(np.zeros((2, 3, 0)), 4)
     assert out.shape == (2, 3, 4) and np.all(out == -1)
+
+
+def test_pins_reject_swapped_value_scale_and_zero(monkeypatch):
+    monkeypatch.setattr(O.PackedCache, "v_hat",
+                        lambda self: O.dequantize_values(self.v_codes, self.v_zero, self.v_scale))
+    with pytest.raises(AssertionError):
+        test_value_round_trip_through_pack_cache()
+
+
+def test_pins_reject_value_groups_along_tokens(monkeypatch):
+    # a value dequantizer that broadcasts the per-token scales along the wrong
+    # axis (group index taken from the token instead of the channel)
+    def bad(codes, scale, zero):
+        *lead, nq, d = codes.shape
+        s = np.repeat(scale.astype(np.float64), 32, axis=-1)
+        z = np.repeat(zero.astype(np.float64), 32, axis=-1)
+        return np.swapaxes(s, -1, -2).reshape(s.shape) * codes + z
+    monkeypatch.setattr(O, "dequantize_values", bad)
+    with pytest.raises(AssertionError):
+        test_value_grid_data_reconstructs_exactly()
+
+
+def test_pins_reject_unscaled_exact_attention(monkeypatch):
+    real = O.softmax_partial
+    monkeypatch.setattr(O, "exact_attention",
+                        lambda q, k, v, n, scale: O.__dict__["_exact_attention_unscaled"](q, k, v, n))
+    def unscaled(q, k, v, n):
+        q = np.asarray(q, dtype=np.float64)
+        b, h, d = q.shape
+        g = h // np.asarray(k).shape[1]
+        out = np.zeros((b, h, d))
+        for bi in range(b):
+            for hq in range(h):
+                out[bi, hq] = O.finish(real(np.asarray(k)[bi, hq // g, :n] @ q[bi, hq],
+                                            np.asarray(v)[bi, hq // g, :n]))
+        return out
+    monkeypatch.setitem(O.__dict__, "_exact_attention_unscaled", unscaled)
+    with pytest.raises(AssertionError):
+        test_exact_attention_is_torch_softmax_attention()
