@@ -41,7 +41,10 @@ def parse(argv=None):
                     help="exact bf16 rows in pinned host memory (zero-copy gather)")
     ap.add_argument("--impl", default="jfa", choices=["jfa", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--cpu-rounds", type=int, default=3,
+                    help="rounds of the oracle baseline (one segment per host process each)")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the K4V4 128K (HBM, host rows) and Qwen GQA-8 lines")
     ap.add_argument("--no-clocks", action="store_true")
     return ap.parse_args(argv)
 
@@ -231,45 +234,94 @@ class Clocks:
 
 
 # ---------------------------------------------------------------------------
-# CPU oracle timing (baseline leg only)
+# CPU oracle timing (baseline legs only): the oracle as it stands, one
+# (sequence, KV head) segment per process, processes started with `spawn`
 # ---------------------------------------------------------------------------
-def oracle_cores() -> int:
-    try:
-        from threadpoolctl import threadpool_info
-        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
-        if n:
-            return int(max(n))
-    except Exception:
-        pass
-    return os.cpu_count() or 1
+def _bf16_bits(t) -> "object":
+    """bf16 tensor -> its raw 16-bit patterns as a numpy int16 array (cheap to pickle)."""
+    import torch
+    return t.contiguous().view(torch.int16).numpy()
 
 
-def time_oracle(w, seconds: float, kv_fn, segs=None):
-    """Time the oracle's decode step on whole (sequence, KV head) segments of
-    the workload (packing untimed) until about `seconds` of CPU work or the
-    end of `segs`; returns (tokens/s in the metric's unit, segments, seconds)."""
+def _oracle_worker(jobs, barrier, results, n_rounds: int):
+    """One host core: per round, pack its segment (untimed), wait for the
+    other workers, then time the oracle's decode step on it."""
+    for var in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS"):
+        os.environ[var] = "1"
+    sys.path.insert(0, ROOT)
+    import numpy as np
     import oracle.jfa_oracle as O
+
+    def f64(bits):
+        return (bits.astype(np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+    for r in range(n_rounds):
+        job = jobs.get()
+        t0 = t1 = 0.0
+        if job is not None:
+            q, k, v, ctx, kb, vb, topk, scale = job
+            kk, vv = f64(k)[None, None], f64(v)[None, None]
+            cache = O.pack_cache(kk, vv, ctx, kb, vb)
+            qq = f64(q)[None]
+        barrier.wait()
+        if job is not None:
+            t0 = time.time()
+            O.decode_step(qq, kk, vv, cache, topk, scale)
+            t1 = time.time()
+        results.put((r, t0, t1, job is not None))
+        barrier.wait()
+
+
+def time_oracle_pool(w, n_rounds: int, kv_fn, workers: int | None = None):
+    """Time the oracle's decode step on `workers` host processes at once, one
+    segment each per round (packing untimed), for n_rounds rounds.  Returns
+    (tokens/s of a full step, segments timed, seconds in the timed windows,
+    workers, per-round windows).  A round's window runs from the first
+    worker's start to the last worker's end; a full step (batch * kv_heads
+    segments) is extrapolated from the segments per second in the windows."""
+    import multiprocessing as mp
+
     import workloads as W
+    n_seg = w.batch * w.kv_heads
+    if workers is None:
+        workers = max(1, min(os.cpu_count() or 1, n_seg, 32))
+    ctx = mp.get_context("spawn")
+    jobs, results = ctx.Queue(), ctx.Queue()
+    barrier = ctx.Barrier(workers)
+    procs = [ctx.Process(target=_oracle_worker, args=(jobs, barrier, results, n_rounds),
+                         daemon=True) for _ in range(workers)]
+    for pr in procs:
+        pr.start()
     q = W.gen_q(w)
-    if segs is None:
-        segs = W.sample_segments(w, w.batch * w.kv_heads, seed=1)
     g = w.group
-    done, spent = 0, 0.0
-    for (b, h) in segs:
-        k, v = kv_fn(b, h)
-        kk = k.double().numpy()[None, None]
-        vv = v.double().numpy()[None, None]
-        qq = q[b:b + 1, h * g:(h + 1) * g].double().numpy()
-        cache = O.pack_cache(kk, vv, w.ctx, w.key_bits, w.val_bits)
-        t0 = time.perf_counter()
-        O.decode_step(qq, kk, vv, cache, w.topk, W.default_scale(w))
-        spent += time.perf_counter() - t0
-        done += 1
-        if spent >= seconds:
-            break
-    # one full step covers batch * kv_heads segments of ctx tokens each
-    step_s = spent / done * (w.batch * w.kv_heads)
-    return w.batch * w.ctx / step_s, done, spent
+    order = W.sample_segments(w, n_seg, seed=1)
+    memo, memo_bytes = {}, 0
+    i = 0
+    for r in range(n_rounds):
+        for _ in range(workers):
+            b, h = order[i % n_seg]
+            i += 1
+            job = memo.get((b, h))
+            if job is None:
+                k, v = kv_fn(b, h)
+                job = (_bf16_bits(q[b, h * g:(h + 1) * g]), _bf16_bits(k), _bf16_bits(v), w.ctx,
+                       w.key_bits, w.val_bits, w.topk, W.default_scale(w))
+                if memo_bytes < (2 << 30):   # segments recur across rounds: keep them
+                    memo[(b, h)] = job
+                    memo_bytes += job[1].nbytes + job[2].nbytes
+            jobs.put(job)
+    windows, done = [], 0
+    for r in range(n_rounds):
+        rs = [results.get(timeout=600) for _ in range(workers)]
+        t0 = min(x[1] for x in rs if x[3])
+        t1 = max(x[2] for x in rs if x[3])
+        windows.append(t1 - t0)
+        done += sum(1 for x in rs if x[3])
+    for pr in procs:
+        pr.join(timeout=60)
+    spent = sum(windows)
+    step_s = spent / done * n_seg
+    return w.batch * w.ctx / step_s, done, spent, workers, windows
 
 
 # ---------------------------------------------------------------------------
@@ -280,24 +332,24 @@ def run_reference(args, w):
     if rank != 0:
         return 0
     import workloads as W
-    times = []
+    rounds = args.warmup + args.steps
+    _, _, _, workers, windows = time_oracle_pool(
+        w, rounds, lambda bb, hh: W.gen_segment(w, bb, hh))
     n_seg = w.batch * w.kv_heads
-    for i in range(args.warmup + args.steps):
-        seg = divmod(i % n_seg, w.kv_heads)
-        val, n, s = time_oracle(w, 0.0, lambda bb, hh: W.gen_segment(w, bb, hh), segs=[seg])
-        if i >= args.warmup:
-            times.append(w.batch * w.ctx / val)     # seconds per full step (extrapolated)
+    per_round = min(workers, n_seg)
+    # each step: one round of `workers` segments in parallel, extrapolated to
+    # the n_seg segments of a full step
+    times = [win / per_round * n_seg for win in windows[args.warmup:]]
     step_s = statistics.mean(times)
     value = w.batch * w.ctx / step_s
-    cores = oracle_cores()
-    sample = (f"one (sequence, KV head) segment of {w.ctx} tokens per step, extrapolated to "
-              f"the {w.batch * w.kv_heads} segments of a full step")
+    sample = (f"per step, {per_round} of the {n_seg} (sequence, KV head) segments of "
+              f"{w.ctx} tokens, one per host process in parallel, extrapolated to a full step")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": config_of(w, args),
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores,
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": workers,
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
@@ -305,26 +357,155 @@ def run_reference(args, w):
     return 0
 
 
-def config_of(w, args, n_copies=0, packed_bytes=0):
+def config_of(w, args, host_resident=None):
+    host = args.host_resident if host_resident is None else host_resident
     return {"workload": w.name, "batch": w.batch, "heads": w.heads, "kv_heads": w.kv_heads,
             "ctx": w.ctx, "format": w.fmt, "topk": w.topk,
-            "exact_rows": "pinned_host" if args.host_resident else "hbm",
-            "l2": (f"not flushed: the timed steps rotate over {n_copies} copies of the packed "
-                   f"cache and of the exact rows ({n_copies} x {packed_bytes / 2**20:.0f} MiB "
-                   f"packed > 126 MB L2), so every step reads its inputs from HBM")
-                  if n_copies else "host run",
+            "exact_rows": "pinned_host" if host else "hbm",
             "parallelism": f"replicas x{args.gpus}"}
 
 
 # ---------------------------------------------------------------------------
 # the CUDA path
 # ---------------------------------------------------------------------------
+class Setup:
+    """A workload resident on the device: R copies of the packed cache (and of
+    the exact rows the correction gathers), together larger than L2, so steps
+    that rotate over them read their inputs from HBM without an L2 flush."""
+
+    def __init__(self, w, dev, host_resident: bool):
+        import torch
+
+        import bit_kv_cache_jfa_b200 as jfa
+        import workloads as W
+        self.w, self.dev, self.host = w, dev, host_resident
+        self.q = W.gen_q(w).to(dev)
+        k_all, v_all = W.gen_kv_device(w, dev, W.gen_q(w))
+        probe = jfa.KVCache(w.batch, w.heads, w.kv_heads, w.ctx, w.key_bits, w.val_bits, device=dev)
+        self.packed_bytes = probe.layout.groups_bytes
+        self.n_copies = 1 + -(-L2_BYTES // max(1, self.packed_bytes))
+        del probe
+        self.ws = None
+        self.copies = []
+        for c in range(self.n_copies):
+            cache = jfa.KVCache(w.batch, w.heads, w.kv_heads, w.ctx, w.key_bits, w.val_bits,
+                                device=dev)
+            if self.ws is None:
+                self.ws = jfa.Workspace(cache, w.topk, device=dev)
+            cache.append(k_all, v_all, self.ws)
+            if host_resident:
+                ke, ve = k_all.cpu().pin_memory(), v_all.cpu().pin_memory()
+            else:
+                ke, ve = (k_all, v_all) if c == 0 else (k_all.clone(), v_all.clone())
+            self.copies.append((cache, cache.geom(), cache.struct(), ke, ve))
+        del k_all, v_all
+        torch.cuda.synchronize()
+        self.out = torch.empty(w.batch, w.heads, 128, dtype=torch.float32, device=dev)
+        self.idx = torch.empty(w.batch, w.kv_heads, w.topk, dtype=torch.int32, device=dev)
+        self.stream = torch.cuda.current_stream(dev)
+        self.sp = self.stream.cuda_stream
+        self.scale = W.default_scale(w)
+        self.geom = self.copies[0][1]
+
+    def l2_note(self) -> str:
+        return (f"not flushed: the timed steps rotate over {self.n_copies} copies of the packed "
+                f"cache and of the exact rows ({self.n_copies} x "
+                f"{self.packed_bytes / 2**20:.0f} MiB packed > 126 MB L2), so every step reads "
+                f"its inputs from HBM")
+
+    def step(self, i):
+        from bit_kv_cache_jfa_b200 import _lib
+        _, g, cs, ke, ve = self.copies[i % self.n_copies]
+        _lib.check(_lib.jfa_decode_scores(g, cs, self.q, self.scale, self.ws.buf, self.sp),
+                   "scores")
+        _lib.check(_lib.jfa_decode_finish(g, cs, self.q, self.scale, self.w.topk, self.idx, ke,
+                                          ve, int(self.host), self.ws.buf, self.out, self.sp),
+                   "finish")
+
+    def step3(self, i):
+        from bit_kv_cache_jfa_b200 import _lib
+        _, g, cs, ke, ve = self.copies[i % self.n_copies]
+        _lib.check(_lib.jfa_decode_scores(g, cs, self.q, self.scale, self.ws.buf, self.sp),
+                   "scores")
+        _lib.check(_lib.jfa_topk(g, self.w.topk, self.ws.buf, self.idx, self.sp), "topk")
+        _lib.check(_lib.jfa_correct_merge(g, cs, self.q, self.scale, self.idx, self.w.topk, ke, ve,
+                                          int(self.host), self.ws.buf, self.out, self.sp),
+                   "correct_merge")
+
+    def check_flag(self):
+        from bit_kv_cache_jfa_b200 import _lib
+        st, flag = _lib.jfa_check_error(self.geom, self.ws.buf, self.sp)
+        if flag:
+            raise RuntimeError(f"device error flag {flag:#x}")
+
+    def timed(self, fn, steps: int, warmup: int) -> float:
+        """ms per call of fn(i): warm-up calls, then `steps` calls back to back
+        between one pair of CUDA events on the launching stream."""
+        import torch
+        for i in range(warmup):
+            fn(i)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(self.stream)
+        for i in range(steps):
+            fn(i)
+        e1.record(self.stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / steps
+
+    def scan_ms(self, steps: int) -> float:
+        """The scan kernel alone, over the same rotation, on a workspace of its
+        own (scan-only launches leave the selection histogram for a finishing
+        kernel to consume)."""
+        import bit_kv_cache_jfa_b200 as jfa
+        from bit_kv_cache_jfa_b200 import _lib
+        ws_scan = jfa.Workspace(self.copies[0][0], self.w.topk, device=self.dev)
+
+        def scan(i):
+            _, g, cs, _, _ = self.copies[i % self.n_copies]
+            _lib.check(_lib.jfa_decode_scores(g, cs, self.q, self.scale, ws_scan.buf, self.sp),
+                       "scores")
+        ms = self.timed(scan, steps, 3)
+        del ws_scan
+        return ms
+
+    def summary(self, step_ms: float, scan_ms: float) -> dict:
+        w = self.w
+        peak, _ = measured_peaks()
+        scan_gbs = scan_alg_bytes(w) / (scan_ms / 1e3) / 1e9
+        step_gbs = step_alg_bytes(w) / (step_ms / 1e3) / 1e9
+        return {"us_per_step": step_ms * 1e3, "tokens_per_s": w.batch * w.ctx / (step_ms / 1e3),
+                "scan_us": scan_ms * 1e3, "scan_frac": scan_gbs / peak,
+                "step_frac": step_gbs / peak, "step_alg_bytes": step_alg_bytes(w)}
+
+
+def per_config_line(args, dev, name: str, host: bool) -> dict:
+    import torch
+
+    import workloads as W
+    w = W.WORKLOADS[name]
+    st = Setup(w, dev, host)
+    steps = max(20, min(args.steps, 200))
+    step_ms = st.timed(st.step, steps, max(3, args.warmup))
+    st.check_flag()
+    d = {"workload": name, "exact_rows": "pinned_host" if host else "hbm", "steps": steps,
+         **st.summary(step_ms, st.scan_ms(steps))}
+    if host:
+        # bytes the step gathers across the host link: the top-k rows of every
+        # segment (the tail rows sit in the cache's device tail buffer)
+        keff = min(w.topk, w.n_quant)
+        link = w.batch * w.kv_heads * keff * 512
+        d["host_link_bytes_per_step"] = link
+    del st
+    torch.cuda.empty_cache()
+    return d
+
+
 def run_jfa(args, w):
     import torch
 
     import bit_kv_cache_jfa_b200 as jfa
     from bit_kv_cache_jfa_b200 import _lib
-    import workloads as W
 
     rank, world, local = dist_env()
     torch.cuda.set_device(local)
@@ -332,49 +513,11 @@ def run_jfa(args, w):
     dist_init(world, "nccl")
     jfa.load()
 
-    q = W.gen_q(w).to(dev)
-    k_all, v_all = W.gen_kv_device(w, dev, W.gen_q(w))
-    # R copies of the cache (and of the exact rows the correction gathers),
-    # together larger than L2: the timed steps rotate over them, so every
-    # step reads its inputs from HBM without an L2 flush between steps
-    probe = jfa.KVCache(w.batch, w.heads, w.kv_heads, w.ctx, w.key_bits, w.val_bits, device=dev)
-    packed_bytes = probe.layout.groups_bytes
-    n_copies = 1 + -(-L2_BYTES // max(1, packed_bytes))
-    del probe
-    ws = None
-    copies = []
-    for c in range(n_copies):
-        cache = jfa.KVCache(w.batch, w.heads, w.kv_heads, w.ctx, w.key_bits, w.val_bits, device=dev)
-        if ws is None:
-            ws = jfa.Workspace(cache, w.topk, device=dev)
-        cache.append(k_all, v_all, ws)
-        if args.host_resident:
-            ke, ve = k_all.cpu().pin_memory(), v_all.cpu().pin_memory()
-        else:
-            ke, ve = (k_all, v_all) if c == 0 else (k_all.clone(), v_all.clone())
-        copies.append((cache, cache.geom(), cache.struct(), ke, ve))
-    del k_all, v_all
-    torch.cuda.synchronize()
-    out = torch.empty(w.batch, w.heads, 128, dtype=torch.float32, device=dev)
-    idx = torch.empty(w.batch, w.kv_heads, w.topk, dtype=torch.int32, device=dev)
-    stream = torch.cuda.current_stream(dev)
-    sp = stream.cuda_stream
-    scale = W.default_scale(w)
-    host = 1 if args.host_resident else 0
-    geom = copies[0][1]
-
-    def step(i, wsb=None):
-        _, g, cs, ke, ve = copies[i % n_copies]
-        _lib.check(_lib.jfa_decode_scores(g, cs, q, scale, ws.buf, sp), "scores")
-        _lib.check(_lib.jfa_decode_finish(g, cs, q, scale, w.topk, idx, ke, ve,
-                                          host, ws.buf, out, sp), "finish")
-
+    st = Setup(w, dev, args.host_resident)
     for i in range(max(3, args.warmup)):
-        step(i)
+        st.step(i)
     torch.cuda.synchronize()
-    st, flag = _lib.jfa_check_error(geom, ws.buf, sp)
-    if flag:
-        raise RuntimeError(f"device error flag {flag:#x}")
+    st.check_flag()
 
     # timed steps: K decode steps back to back (the call sequence of a step,
     # nothing between the calls), one event pair around all of them
@@ -383,10 +526,10 @@ def run_jfa(args, w):
     barrier(world)
     torch.cuda.synchronize()
     wall0 = time.perf_counter()
-    e0.record(stream)
+    e0.record(st.stream)
     for i in range(args.steps):
-        step(i)
-    e1.record(stream)
+        st.step(i)
+    e1.record(st.stream)
     torch.cuda.synchronize()
     barrier(world)
     wall = time.perf_counter() - wall0
@@ -395,119 +538,89 @@ def run_jfa(args, w):
     ms_max = max_over_ranks(ms, world, dev)
 
     # the same steps as the three separate calls (scores, top-k, correct+merge)
-    # instead of the fused finishing kernel, for reference
-    def step3(i):
-        _, g, cs, ke, ve = copies[i % n_copies]
-        _lib.check(_lib.jfa_decode_scores(g, cs, q, scale, ws.buf, sp), "scores")
-        _lib.check(_lib.jfa_topk(g, w.topk, ws.buf, idx, sp), "topk")
-        _lib.check(_lib.jfa_correct_merge(g, cs, q, scale, idx, w.topk, ke, ve, host, ws.buf, out,
-                                          sp), "correct_merge")
+    unfused_ms = st.timed(st.step3, args.steps, 3)
+    scan_avg = st.scan_ms(args.steps)
 
-    for i in range(3):
-        step3(i)
-    u0, u1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    torch.cuda.synchronize()
-    u0.record(stream)
-    for i in range(args.steps):
-        step3(i)
-    u1.record(stream)
-    torch.cuda.synchronize()
-    unfused_ms = u0.elapsed_time(u1) / args.steps
+    # end to end through the public API, two ways; every step copies q in from
+    # pinned host memory and the finishing kernel writes out straight into
+    # pinned host memory (out may be host-resident):
+    #  - eager: one jfa_decode_step C-ABI call per step (decode_step);
+    #  - graph: the step captured once per cache copy (DecodeGraph) and replayed
+    q_host = st.q.cpu().pin_memory()
+    out_host = torch.empty(st.out.shape, dtype=st.out.dtype).pin_memory()
 
-    # the scan kernel alone (roofline): its own launches back to back over the
-    # same rotation, on a workspace of its own (scan-only launches leave the
-    # selection histogram for a finishing kernel to consume)
-    ws_scan = jfa.Workspace(copies[0][0], w.topk, device=dev)
-    for i in range(3):
-        _, g, cs, _, _ = copies[i % n_copies]
-        _lib.check(_lib.jfa_decode_scores(g, cs, q, scale, ws_scan.buf, sp), "scores")
-    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s0.record(stream)
-    for i in range(args.steps):
-        _, g, cs, _, _ = copies[i % n_copies]
-        _lib.check(_lib.jfa_decode_scores(g, cs, q, scale, ws_scan.buf, sp), "scores")
-    s1.record(stream)
-    torch.cuda.synchronize()
-    scan_avg = s0.elapsed_time(s1) / args.steps
-    del ws_scan
+    def eager_step(i):
+        cache, _, _, ke, ve = st.copies[i % st.n_copies]
+        st.q.copy_(q_host, non_blocking=True)
+        jfa.decode_step(cache, st.q, w.topk, ke, ve, st.ws, scale=st.scale, out=out_host,
+                        idx=st.idx, exact_on_host=bool(st.host), stream=st.sp)
 
-    # end to end through the public API: every step copies q in from pinned
-    # host memory and replays the step captured in a CUDA graph (one per
-    # cache copy, captured before the timed region), whose finishing kernel
-    # writes its output straight into pinned host memory (out may be
-    # host-resident)
-    q_host = q.cpu().pin_memory()
-    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    graphs = [jfa.DecodeGraph(cache, q, w.topk, ke, ve, ws, scale=scale, out=out_host, idx=idx,
-                              exact_on_host=bool(host))
-              for cache, _, _, ke, ve in copies]
+    eager_ms = st.timed(eager_step, args.steps, max(3, args.warmup))
+    graphs = [jfa.DecodeGraph(cache, st.q, w.topk, ke, ve, st.ws, scale=st.scale, out=out_host,
+                              idx=st.idx, exact_on_host=bool(st.host))
+              for cache, _, _, ke, ve in st.copies]
 
-    def e2e_step(i):
-        q.copy_(q_host, non_blocking=True)
-        graphs[i % n_copies].replay()
+    def graph_step(i):
+        st.q.copy_(q_host, non_blocking=True)
+        graphs[i % st.n_copies].replay()
 
-    for i in range(max(3, args.warmup)):
-        e2e_step(i)
-    x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    torch.cuda.synchronize()
-    x0.record(stream)
-    for i in range(args.steps):
-        e2e_step(i)
-    x1.record(stream)
-    torch.cuda.synchronize()
-    e2e_avg = x0.elapsed_time(x1) / args.steps
-    e2e_max = max_over_ranks(e2e_avg, world, dev)
+    graph_ms = st.timed(graph_step, args.steps, max(3, args.warmup))
+    e2e_max = max_over_ranks(min(eager_ms, graph_ms), world, dev)
+    e2e_api = "graph replay (DecodeGraph.replay)" if graph_ms <= eager_ms else \
+        "eager C-ABI call per step (jfa_decode_step)"
+    st.check_flag()
+    del graphs
 
-    st, flag = _lib.jfa_check_error(geom, ws.buf, sp)
-    if flag:
-        raise RuntimeError(f"device error flag {flag:#x}")
+    per_config = []
+    if not args.no_per_config and world == 1:
+        for name, host in (("llama8b_k4v4_128k", False), ("llama8b_k4v4_128k", True),
+                           ("qwen30b_k3v2_32k", False)):
+            if name == w.name and host == args.host_resident:
+                continue
+            per_config.append(per_config_line(args, dev, name, host))
 
     tokens = w.batch * w.ctx
     value = world * tokens / (ms_max / 1e3)
     peak, peak_kind = measured_peaks()
-    achieved = scan_alg_bytes(w) / (scan_avg / 1e3) / 1e9
-    step_gbs = step_alg_bytes(w) / (ms / 1e3) / 1e9
-    launches = jfa.jfa_decode_step_launches(geom, w.topk)
+    summ = st.summary(ms, scan_avg)
+    launches = jfa.jfa_decode_step_launches(st.geom, w.topk)
 
     line = None
     if rank == 0:
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
-            k_exact, v_exact = copies[0][3], copies[0][4]
-            kv_cpu = lambda b, h: (k_exact[b, h].cpu(), v_exact[b, h].cpu())
-            val, n, spent = time_oracle(w, args.cpu_seconds, kv_cpu)
-            cpu = {"value": val, "unit": "tokens/s", "cores": oracle_cores(), "kind": "oracle",
-                   "sample": f"{n} of {w.batch * w.kv_heads} (sequence, KV head) segments "
-                             f"({w.ctx} tokens each) in {spent:.1f} s, extrapolated to a "
-                             f"full step"}
-            try:  # the same oracle on one core (numpy's BLAS pool limited to 1 thread)
-                from threadpoolctl import threadpool_limits
-                with threadpool_limits(limits=1):
-                    v1, n1, s1 = time_oracle(w, args.cpu_seconds / 2, kv_cpu)
-                cpu["one_core"] = {"value": v1, "cores": 1,
-                                   "sample": f"{n1} segments in {s1:.1f} s, extrapolated"}
-            except ImportError:
-                pass
+            k0, v0 = st.copies[0][3], st.copies[0][4]
+            kv_cpu = lambda b, h: (k0[b, h].cpu(), v0[b, h].cpu())
+            rounds = max(1, args.cpu_rounds)
+            val, n, spent, workers, _ = time_oracle_pool(w, rounds, kv_cpu)
+            cpu = {"value": val, "unit": "tokens/s", "cores": workers, "kind": "oracle",
+                   "sample": f"{n} (sequence, KV head) segments of {w.ctx} tokens, {workers} "
+                             f"at a time on {workers} host processes ({rounds} rounds, "
+                             f"{spent:.2f} s in the timed windows), extrapolated to the "
+                             f"{w.batch * w.kv_heads} segments of a full step"}
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "f32", "data": "synthetic", "config": config_of(w, args, n_copies, packed_bytes),
+            "dtype": "f32", "data": "synthetic", "config": config_of(w, args),
+            "l2": st.l2_note(),
             "roofline": {"bound": "hbm", "kernel": "scan_kernel (jfa_decode_scores)",
-                         "achieved": achieved, "peak": peak, "peak_kind": peak_kind,
-                         "unit": "GB/s", "frac": achieved / peak,
+                         "achieved": summ["scan_frac"] * peak, "peak": peak,
+                         "peak_kind": peak_kind, "unit": "GB/s", "frac": summ["scan_frac"],
                          "traffic": recorded_traffic(w.name),
                          "alg_bytes_per_launch": scan_alg_bytes(w),
                          "us_per_launch": scan_avg * 1e3},
-            "step_roofline": {"achieved": step_gbs, "peak": peak, "unit": "GB/s",
-                              "frac": step_gbs / peak, "alg_bytes_per_step": step_alg_bytes(w)},
+            "step_roofline": {"achieved": summ["step_frac"] * peak, "peak": peak, "unit": "GB/s",
+                              "frac": summ["step_frac"], "alg_bytes_per_step": step_alg_bytes(w)},
             "cpu_baseline": cpu,
             "e2e": {"value": world * tokens / (e2e_max / 1e3), "unit": "tokens/s",
-                    "ms_per_step": e2e_max,
-                    "h2d_bytes_per_step": q.numel() * q.element_size(),
-                    "d2h_bytes_per_step": out.numel() * out.element_size()},
+                    "ms_per_step": e2e_max, "api": e2e_api,
+                    "eager_ms_per_step": eager_ms, "graph_ms_per_step": graph_ms,
+                    "h2d_bytes_per_step": st.q.numel() * st.q.element_size(),
+                    "d2h_bytes_per_step": st.out.numel() * st.out.element_size()},
             "unfused": {"ms_per_step": unfused_ms,
                         "calls": "jfa_decode_scores + jfa_topk + jfa_correct_merge"},
+            "per_config": per_config,
             "gpu_launches": launches * args.steps,
             "clocks": clk,
             "wall_s_timed_region": wall,

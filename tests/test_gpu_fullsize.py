@@ -16,7 +16,7 @@ import bit_kv_cache_jfa_b200 as jfa
 from bit_kv_cache_jfa_b200 import _lib
 import oracle.jfa_oracle as O
 import workloads as W
-from jfa_testutil import assert_out_close, assert_topk_valid
+from jfa_testutil import SCORE_ABS, assert_out_close, assert_topk_valid
 
 pytestmark = pytest.mark.gpu
 
@@ -27,6 +27,10 @@ CASES = [
     ("qwen30b_k3v2_32k", False, 3),
     ("llama70b_k3v2_32k_b8", False, 2),
     ("llama70b_k4v4_32k_b8", False, 2),
+    ("llama70b_k3v2_8k_b1", False, 2),
+    ("llama70b_k3v2_128k_b32", False, 2),
+    ("llama70b_k3v2_256k_b1", False, 2),
+    ("llama70b_k4v4_256k_b1", False, 2),
 ]
 
 
@@ -58,6 +62,8 @@ def test_fullsize_sampled_segments(name, host_rows, n_seg):
     out_h, idx_h = out.cpu().double().numpy(), idx.cpu().numpy()
     g = w.group
     nq = cache.n_quant
+    scores = ws.scores(cache)
+    worst = 0.0
     for (b, h) in W.sample_segments(w, n_seg, seed=7):
         kk = k_all[b, h].cpu().double().numpy()[None, None]
         vv = v_all[b, h].cpu().double().numpy()[None, None]
@@ -74,8 +80,13 @@ def test_fullsize_sampled_segments(name, host_rows, n_seg):
             assert np.array_equal(vs, oc.v_scale[0, 0, sl].view(np.uint16)), (b, h, gi)
             assert np.array_equal(vz, oc.v_zero[0, 0, sl].view(np.uint16)), (b, h, gi)
         ref = O.decode_step(qq, kk, vv, oc, w.topk, scale)
+        s_gpu = scores[b, h, :nq].cpu().double().numpy()
+        err = float(np.abs(s_gpu - ref.select[0, 0]).max())
+        worst = max(worst, err)
+        assert err <= SCORE_ABS, (b, h, err)
         assert_topk_valid(idx_h[b:b + 1, h:h + 1], ref.select, w.topk)
         # the output with the device's own index set (a tie-window swap changes
         # which tokens are exact, so the oracle follows the same choice)
         ref_same = O.decode_step(qq, kk, vv, oc, w.topk, scale, idx=idx_h[b:b + 1, h:h + 1])
         assert_out_close(out_h[b:b + 1, h * g:(h + 1) * g], ref_same.out)
+    print(f"{name}: max selection-score error {worst:.2e} (bound {SCORE_ABS:.0e})")

@@ -325,8 +325,9 @@ def test_fused_step_matches_separate_calls(kb, vb, heads, kv, ctx, k, batch):
     out1, idx1 = run.fused_step()
     assert np.array_equal(idx1, idx3)
     assert np.allclose(out1, out3, rtol=1e-5, atol=1e-6)
-    if ctx <= 9000:
-        assert_out_close(out1, run.oracle_step(idx=idx1).out)
+    ref = run.oracle_step()
+    assert_topk_valid(idx1, ref.select, k)
+    assert_out_close(out1, run.oracle_step(idx=idx1).out)
 
 
 @pytest.mark.parametrize("kb,vb,heads,kv", [(3, 2, 8, 2), (4, 4, 32, 4)])
@@ -349,4 +350,50 @@ def test_fused_step_tiny_workload_against_oracle():
     out, idx = run.fused_step()
     ref = run.oracle_step()
     assert_topk_valid(idx, ref.select, w.topk)
+    assert_out_close(out, ref.out)
+
+
+def test_whole_segment_fallback_selection():
+    # scan once, then run the finishing kernel twice: the first consumes and
+    # clears the scan's score histogram, so the second must select over the
+    # whole segment from the stored scores (the fallback path); both choices
+    # equal the bit-exact top-k of those scores
+    w = small(3, 2, heads=32, kv=8, ctx=9000, batch=2, topk=256, lognormal=True)
+    run = GpuRun(w)
+    run.scores()
+    g, cs = run.cache.geom(), run.cache.struct()
+    outs = []
+    for _ in range(2):
+        out = torch.empty_like(run.out)
+        idx = torch.empty_like(run.idx)
+        _lib.check(_lib.jfa_decode_finish(g, cs, run.q, run.scale, run.k, idx, run.k_exact,
+                                          run.v_exact, 0, run.ws.buf, out), "finish")
+        torch.cuda.synchronize()
+        outs.append((out.cpu().double().numpy(), idx.cpu().numpy()))
+    assert run.ws.error_flag(run.cache) == 0
+    s_gpu = run.selection_scores()
+    want = O.topk_indices(s_gpu, run.k)
+    for out, idx in outs:
+        assert np.array_equal(idx, want)
+        assert_out_close(out, run.oracle_step(idx=idx).out)
+    assert np.allclose(outs[0][0], outs[1][0], rtol=1e-6, atol=1e-7)
+
+
+@pytest.mark.parametrize("ctx,k", [(20000, 4096), (6000, 1000)])
+def test_all_scores_tied_picks_lowest_indices(ctx, k):
+    # constant keys: every selection score is equal, so the chosen set is the
+    # k lowest indices; the tie bin overflows every shared-memory list
+    w = small(4, 4, heads=32, kv=8, ctx=ctx, batch=1, topk=k, planted=0)
+    q = W.gen_q(w)
+    kc = torch.full((1, 8, ctx, 128), 0.375, dtype=torch.bfloat16)
+    vc = W.gen_kv(w, q, ctx)[1]
+    run = GpuRun(w, q=q, kv=(kc, vc))
+    out, idx = run.fused_step()
+    nq = run.cache.n_quant
+    s_gpu = run.selection_scores()
+    assert np.all(s_gpu == s_gpu[0, 0, 0])
+    want = np.broadcast_to(np.arange(k, dtype=np.int32), idx.shape)
+    assert np.array_equal(idx, want)
+    ref = run.oracle_step()
+    assert np.array_equal(ref.idx, want)
     assert_out_close(out, ref.out)

@@ -6,6 +6,7 @@ import pytest
 import torch
 
 import bit_kv_cache_jfa_b200 as jfa
+import oracle.jfa_oracle as O
 from bit_kv_cache_jfa_b200 import _lib
 
 
@@ -34,10 +35,12 @@ def test_noalloc_topk_matches_topk_twice():
     s1 = (rng.standard_normal((8, 32704)) * 2).astype(np.float32)
     ref1, new1 = _reference_and_noalloc(8, 32704, 256, s1)
     assert np.array_equal(ref1, new1)
+    assert np.array_equal(new1, O.topk_indices(s1.astype(np.float64), 256))
     # second call on the shared scratch: other shape, many ties
     s2 = (np.round(rng.standard_normal((4, 8192)) * 4) / 4).astype(np.float32)
     ref2, new2 = _reference_and_noalloc(4, 8192, 300, s2)
     assert np.array_equal(ref2, new2)
+    assert np.array_equal(new2, O.topk_indices(s2.astype(np.float64), 300))
 
 
 @pytest.mark.gpu
