@@ -376,7 +376,9 @@ def test_whole_segment_fallback_selection():
     for out, idx in outs:
         assert np.array_equal(idx, want)
         assert_out_close(out, run.oracle_step(idx=idx).out)
-    assert np.allclose(outs[0][0], outs[1][0], rtol=1e-6, atol=1e-7)
+    # the two paths spread the correction differently over the cluster: fp32
+    # sums in another order
+    assert np.allclose(outs[0][0], outs[1][0], rtol=1e-5, atol=1e-6)
 
 
 @pytest.mark.parametrize("ctx,k", [(20000, 4096), (6000, 1000)])
