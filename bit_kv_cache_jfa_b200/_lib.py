@@ -53,7 +53,8 @@ class CacheLayout(ctypes.Structure):
 
 class WorkspaceLayout(ctypes.Structure):
     _fields_ = [("total_bytes", c_size_t), ("off_flag", c_size_t), ("off_scores", c_size_t),
-                ("off_partials", c_size_t), ("off_mused", c_size_t), ("off_scan_hist", c_size_t),
+                ("off_partials", c_size_t), ("off_mused", c_size_t), ("off_wts", c_size_t),
+                ("off_scan_hist", c_size_t),
                 ("off_hist", c_size_t), ("off_counters", c_size_t),
                 ("off_cand", c_size_t), ("off_sel", c_size_t),
                 ("max_topk", c_int32), ("partial_slots", c_int32), ("cand_cap", c_int32),

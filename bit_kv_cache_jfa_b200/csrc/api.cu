@@ -38,9 +38,11 @@ int workspace_layout(const jfa_geom& g, int max_topk, jfa_workspace_layout* out)
   L.off_partials = off;
   off = align_up(off + (size_t)L.partial_slots * G * kPartStride * sizeof(float), 256);
   L.off_mused = off;
-  off = align_up(off + n_seg * (size_t)(g.capacity / kKG) * 2 * kMaxG * sizeof(float), 256);
+  off = align_up(off + n_seg * (size_t)(g.capacity / kKG) * kMaxG * sizeof(float), 256);
+  L.off_wts = off;
+  off = align_up(off + n_seg * (size_t)(g.capacity / kKG) * 4 * (G > 4 ? 2 : 1) * 32 * sizeof(uint32_t), 256);
   L.off_scan_hist = off;
-  off = align_up(off + n_seg * kScanHistBins * sizeof(uint32_t), 256);
+  off = align_up(off + n_seg * kScanHistStride * sizeof(uint32_t), 256);
   L.off_hist = off;
   off += n_seg * kHistBins * sizeof(uint32_t);
   L.off_counters = off;

@@ -21,6 +21,7 @@ int launch_finish(const jfa_geom& g, const jfa_cache& c, const uint16_t* q, floa
   fp.scores = reinterpret_cast<const float*>(ws + L.off_scores);
   fp.scan_part = reinterpret_cast<const float*>(ws + L.off_partials);
   fp.m_used = reinterpret_cast<const float*>(ws + L.off_mused);
+  fp.wts = reinterpret_cast<const uint32_t*>(ws + L.off_wts);
   fp.hist = reinterpret_cast<uint32_t*>(ws + L.off_scan_hist);
   fp.glists = reinterpret_cast<uint32_t*>(ws + L.off_cand);
   fp.idx_in = idx_in;

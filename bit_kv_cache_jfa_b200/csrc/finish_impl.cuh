@@ -1,23 +1,30 @@
 // finish_impl.cuh — everything after the scan in one kernel.  A thread-block
-// cluster of C CTAs (C <= 16) per (sequence, KV head):
-//   T   (before waiting for the scan) corrects its share of the bf16 tail;
-//   P1  reads the scan's 8192-bin histogram of the selection keys and finds
+// cluster of C CTAs (C <= 16) per (sequence, KV head); CTA r owns slice r of
+// the quantized tokens and the tail slots r, r + C, ...
+//
+//   S1  reads the scan's 8192-bin histogram of the selection keys and finds
 //       the bin b* holding the k-th largest key (every CTA, redundantly);
-//   P2  lists its slice's keys above b* ("sure") and in b* ("ties"), in
-//       index order, in its shared memory;
-//   P3  after a cluster barrier, gathers every CTA's ties and resolves the
-//       k-th key inside b* by two more radix levels (ties to lower indices),
-//       writes its own chosen indices to idx in ascending order and takes
-//       an even share of the chosen set for the correction;
-//   P4  corrects that share: exact bf16 logits and values, and the scan's
-//       approximate terms of each chosen token recomputed bit for bit
-//       (jfa_approx.cuh, with the stored running maxima) for removal;
-//   P5  merges a share of the scan's split partials, then the CTAs owning a
-//       query head combine scan, exact and removal partials of all C CTAs
-//       (distributed shared memory) in log-sum-exp form.
-// With a given index set (jfa_correct_merge) P1-P3 are skipped.  If the
-// histogram is stale or the candidates overflow shared memory, every CTA
-// selects over the whole segment instead (slower, same result).
+//   S2  lists its slice's keys above b* ("sure": chosen whatever the ties
+//       decide) and in b* ("ties"), in index order, and arrives on a
+//       cluster barrier;
+//   A   corrects its tail slots and its sure tokens while the other CTAs
+//       reach the barrier: every warp takes its own tokens, stages their
+//       record pieces and exact rows, and folds them into a running fp32
+//       softmax partial per query head (exact bf16 term in, the scan's
+//       approximate term out: the fp16 weights the scan stored, against the
+//       running maximum it stored, times the dequantized value);
+//   S3  waits on the barrier, gathers every CTA's ties and ranks them (larger
+//       key first, equal keys to the lower index);
+//   B   corrects the chosen ties of its slice into the same partials and
+//       writes its chosen indices, ascending, at its offset of idx;
+//   M   merges its warps' partials and its share of the scan's split
+//       partials; the CTAs owning a query head combine the C CTAs' partials
+//       (distributed shared memory) in log-sum-exp form and write out.
+// With a given index set (jfa_correct_merge) or k >= N_q there is no
+// selection: A corrects the CTA's even share of the set.  If the histogram is
+// stale or a list overflows, every CTA selects over the whole segment from
+// the stored scores instead and the correction restarts on that set (slower,
+// same result).
 #pragma once
 
 #include <cooperative_groups.h>
@@ -31,82 +38,71 @@ namespace cg = cooperative_groups;
 namespace jfa {
 
 constexpr int kFinThreads = 256;
+constexpr int kFinWarps = kFinThreads / 32;
 constexpr int kFinMaxC = kFinMaxCluster;  // 16: non-portable cluster size, few segments only
 constexpr int kLCap = 1024;   // sure / tie list entries per CTA
 constexpr int kTCap = 1024;   // gathered tie entries
 constexpr int kRefBins = 2048;
+constexpr int kTokCap = 1024;  // tokens listed per correction round (plus the tail slots)
+constexpr int kChunk = 4;      // tokens a warp stages at once
 
-
-// Shared memory.  The persistent part is read by other CTAs of the cluster
-// (lists, counts, partials) and lives until the last barrier; the union part
-// is private and reused: selection buffers, then the correction's token list
-// and per-warp staging rings.
+// Shared memory.  The persistent part is read by the other CTAs of the
+// cluster (lists, counts, partials) and lives until the last barrier.
 struct FinPersist {
   uint32_t sure[kLCap];               // chosen-for-sure indices of the slice, ascending
   uint32_t tkey[kLCap], tidx[kLCap];  // ties of the slice (key, index), ascending index
   uint32_t chtie[kTCap];              // chosen ties of the whole segment, ascending
   uint32_t n_sure, n_tie, overflow, n_gl;
 };
-// A correction partial (m, l, pad, pad, acc[128]) per query head; in the
-// combined form the top-k tokens' approximate terms enter with a minus sign,
-// so l may be negative.
+// A partial (m, l, pad, pad, acc[128]) per query head: `run` holds this CTA's
+// exact-minus-removed terms (l may be negative), `sp` its share of the scan's
+// split partials.
 template <int G>
 struct FinParts {
-  float run[G][kPartStride];   // this CTA's exact-minus-removed partial (frame, mass, acc)
-  float sp[G][kPartStride];    // this CTA's share of the scan partials
+  float run[G][kPartStride];
+  float sp[G][kPartStride];
 };
 // Shared-memory histograms store bin b at hpad(b) = b + b/32, so threads
 // that each read a contiguous run of bins hit distinct banks.
 __device__ __forceinline__ int hpad(int b) { return b + (b >> 5); }
-struct FinSelect {
+
+// Pieces of one quantized token, staged by its warp (16-byte copies).
+struct TokPieces {
+  uint8_t vp[256];     // value-code pieces holding its column (8 or 16 x 16 B)
+  uint8_t vsz[64];     // its value scales (32 B block) and zeros (32 B block)
+  uint32_t w[8];       // the scan's fp16 weights: word 4n + j = head 4n + j, tokens
+                       // (t mod 8) (low half) and (t mod 8) + 8 of its m-tile
+  float mu[kMaxG];     // the scan's running maxima of its group, per head
+};
+static_assert(sizeof(TokPieces) == 384, "token pieces layout");
+constexpr int kTokPieces16 = 24;  // 16-byte copies per token
+
+struct FinWork {                 // correction working set (phases A and B)
+  TokPieces ring[kFinWarps][kChunk];
+  uint32_t akey[kTCap], aidx[kTCap];      // gathered ties
   uint32_t hist[kRefBins + kRefBins / 32];
-  uint32_t akey[kTCap], aidx[kTCap];
-};
-// One token of a correction batch: its record pieces (cp.async) and its
-// exact bf16 K and V rows.  The 16-byte pad puts the rows of consecutive
-// tokens 4 banks apart, so the tensor-core operand loads are conflict-free.
-struct TokStage {
-  uint8_t ksz[512];      // key scales / zeros of its group
-  uint8_t kcode[128];    // key-code words of the 4 lanes holding its m-tile row
-  uint8_t vp[256];       // value-code pieces holding its column (8 or 16 x 16 B)
-  uint8_t vsz[64];       // its value scales (32 B block) and zeros (32 B block)
-  float mu[2 * kMaxG];   // the scan's running maxima (8) and biases (8) of its group
-  uint16_t krow[kD];     // bf16 K row
-  uint16_t vrow[kD];     // bf16 V row
-  uint8_t pad[16];
-};
-static_assert(sizeof(TokStage) == 1552, "token stage layout");
-constexpr int kTokCap = 1024;  // tokens listed per correction round
-constexpr int kBT = 16;        // tokens per correction batch (one mma k-step)
-// Correction batches, double-buffered: batch b + 1 is staged while batch b
-// is computed.  The weights are bf16 triples (hi, mid, lo: 24 significant
-// bits), head-major (the B operands of the value MMAs).
-struct FinBatchT {
-  TokStage st[2][kBT];
-  int tok[2][kBT];
-  uint16_t bex[3][kMaxG][kBT];      // exact weights
-  uint16_t brem[3][4][kMaxG][kBT];  // minus the removed weights per 32-channel group
-  uint16_t bpf[2][kMaxG][kBT];      // removed masses 2^(m_used - m) p as fp16 (hi, lo)
-  float se[kBT][kMaxG];             // exact logits (log2 units)
-  uint16_t ph[kBT][kMaxG];          // replayed fp16 weights of the scan
-  float alpha[kMaxG];               // frame move of this batch per head
-  float zsum[kMaxG][4];             // removed zero-point terms per head and channel group (final)
-};
-struct FinCorr {
-  FinBatchT b;
-  int32_t tok[kTokCap + kTail];
 };
 template <int G>
+struct FinMerge {                // warps' partials, after the correction
+  float w[kFinWarps][G][kPartStride];
+};
+template <int G>
+constexpr size_t fin_union_bytes() {
+  return sizeof(FinWork) > sizeof(FinMerge<G>) ? sizeof(FinWork) : sizeof(FinMerge<G>);
+}
+constexpr size_t kEarlyBytes = 24 * 1024;  // early copy of the scan partials' share
+template <int G>
 constexpr size_t fin_smem_bytes() {
-  return sizeof(FinPersist) + sizeof(FinParts<G>) +
-         (sizeof(FinSelect) > sizeof(FinCorr) ? sizeof(FinSelect) : sizeof(FinCorr));
+  return sizeof(FinPersist) + sizeof(FinParts<G>) + (size_t)G * kD * sizeof(float) +
+         (kTokCap + kTail) * sizeof(int32_t) + fin_union_bytes<G>() + kEarlyBytes;
 }
 
 // From bin counts h[hpad(0..nbins)) (nbins a multiple of blockDim) find the
 // bin where the count taken from the top reaches r (1 <= r); *bin = -1 if
 // the total < r.
-static __device__ __noinline__ void find_bin_from_top(const uint32_t* h, int nbins, uint32_t r, uint32_t* scratch,
-                                  int* bin, uint32_t* above, uint32_t* total) {
+static __device__ __noinline__ void find_bin_from_top(const uint32_t* h, int nbins, uint32_t r,
+                                                      uint32_t* scratch, int* bin, uint32_t* above,
+                                                      uint32_t* total) {
   const int per = nbins / blockDim.x;
   const int b0 = threadIdx.x * per;
   uint32_t local = 0;
@@ -128,32 +124,38 @@ static __device__ __noinline__ void find_bin_from_top(const uint32_t* h, int nbi
   __syncthreads();
 }
 
-// Selection inside the histogram bin b* (keys share their top 13 bits):
-// the r largest of the T ties akey/aidx (index order), larger key first and
-// equal keys to the lower index, two radix levels (11 + 8 bits) and one
-// ordered pass.  Writes the chosen indices ascending to chosen[] (r of them).
-static __device__ __noinline__ void refine_ties(const uint32_t* akey, const uint32_t* aidx, uint32_t T, uint32_t r,
-                            uint32_t* h, uint32_t* chosen, uint32_t* scratch, int* s_bin,
-                            uint32_t* s_above, uint32_t* s_tot) {
+// Selection inside the histogram bin b* (keys share their top 15 bits): the
+// r largest of the T ties akey/aidx (index order), larger key first and equal
+// keys to the lower index, two radix levels over the other 17 bits (8 + 9)
+// and one ordered pass.  Writes the chosen indices ascending to chosen[] (r
+// of them).
+constexpr int kRef2Shift = 32 - kScanHistBits - 8;  // level 2: the next 8 bits
+constexpr int kRef3Bits = kRef2Shift;              // level 3: the rest (9 bits)
+static_assert(kRef3Bits == 9, "refinement levels cover the key");
+static __device__ __noinline__ void refine_ties(const uint32_t* akey, const uint32_t* aidx, uint32_t T,
+                                                uint32_t r, uint32_t* h, uint32_t* chosen,
+                                                uint32_t* scratch, int* s_bin, uint32_t* s_above,
+                                                uint32_t* s_tot) {
   const int tid = threadIdx.x;
-  // level 2: key bits 18..8
-  for (int i = tid; i < hpad(kRefBins); i += blockDim.x) h[i] = 0u;
+  constexpr uint32_t m2 = 255u, m3 = (1u << kRef3Bits) - 1u;
+  // level 2: the 8 key bits below the shared ones
+  for (int i = tid; i < hpad(256); i += blockDim.x) h[i] = 0u;
   __syncthreads();
-  for (uint32_t i = tid; i < T; i += blockDim.x) atomicAdd(&h[hpad((akey[i] >> 8) & 2047u)], 1u);
+  for (uint32_t i = tid; i < T; i += blockDim.x) atomicAdd(&h[hpad((akey[i] >> kRef2Shift) & m2)], 1u);
   __syncthreads();
-  find_bin_from_top(h, kRefBins, r, scratch, s_bin, s_above, s_tot);
+  find_bin_from_top(h, 256, r, scratch, s_bin, s_above, s_tot);
   const uint32_t d2 = (uint32_t)*s_bin;
   const uint32_t r2 = r - *s_above;
   __syncthreads();
-  // level 3: key bits 7..0 among keys whose bits 18..8 are d2
-  for (int i = tid; i < hpad(256); i += blockDim.x) h[i] = 0u;
+  // level 3: the low bits among keys whose level-2 digit is d2
+  for (int i = tid; i < hpad(1 << kRef3Bits); i += blockDim.x) h[i] = 0u;
   __syncthreads();
   for (uint32_t i = tid; i < T; i += blockDim.x)
-    if (((akey[i] >> 8) & 2047u) == d2) atomicAdd(&h[hpad(akey[i] & 255u)], 1u);
+    if (((akey[i] >> kRef2Shift) & m2) == d2) atomicAdd(&h[hpad(akey[i] & m3)], 1u);
   __syncthreads();
-  find_bin_from_top(h, 256, r2, scratch, s_bin, s_above, s_tot);
-  const uint32_t low = (akey[0] >> 19) << 19;  // the shared top bits
-  const uint32_t kstar = low | (d2 << 8) | (uint32_t)*s_bin;
+  find_bin_from_top(h, 1 << kRef3Bits, r2, scratch, s_bin, s_above, s_tot);
+  const uint32_t low = (akey[0] >> (32 - kScanHistBits)) << (32 - kScanHistBits);  // the shared top bits
+  const uint32_t kstar = low | (d2 << kRef2Shift) | (uint32_t)*s_bin;
   const uint32_t r3 = r2 - *s_above;
   __syncthreads();
   // ordered pass: thread t owns entries [t*per, (t+1)*per)
@@ -184,9 +186,9 @@ static __device__ __noinline__ void refine_ties(const uint32_t* akey, const uint
 // Fallback selection over the whole segment (stale histogram or too many
 // candidates): three radix levels (11 + 11 + 10 bits) over all nq scores, then this CTA's slice
 // [lo, hi) of chosen indices, ascending, into out[]; returns their count.
-static __device__ __noinline__ uint32_t select_full(const float* S, int nq, int k, int lo, int hi, uint32_t* h,
-                                uint32_t* out, uint32_t* scratch, int* s_bin, uint32_t* s_above,
-                                uint32_t* s_tot) {
+static __device__ __noinline__ uint32_t select_full(const float* S, int nq, int k, int lo, int hi,
+                                                    uint32_t* h, uint32_t* out, uint32_t* scratch,
+                                                    int* s_bin, uint32_t* s_above, uint32_t* s_tot) {
   const int tid = threadIdx.x;
   uint32_t prefix = 0, r = (uint32_t)k;
   const int shifts[3] = {21, 10, 0};
@@ -252,16 +254,21 @@ __device__ __forceinline__ uint32_t lower_bound_u32(const uint32_t* a, uint32_t 
   return lo;
 }
 
+// Split cluster barrier: arrive (release: this CTA's shared-memory writes
+// become visible to the cluster) and wait (acquire).
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
 // ---------------------------------------------------------------------------
-// Correction helpers.  Token encoding: t in [0, nq) a quantized token,
-// (1 << 30) | s the tail slot s (exact rows only); -1 an empty batch slot.
+// Correction.  Token encoding: t in [0, nq) a quantized token,
+// (1 << 30) | s the tail slot s (exact rows only); -1 none.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ bool tok_quant(int t) { return t >= 0 && !(t & (1 << 30)); }
 
-template <typename T4>
-__device__ __forceinline__ T4 ld16(const void* p) {
-  return *reinterpret_cast<const T4*>(p);
-}
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
 }
@@ -271,44 +278,41 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-// Record pieces of quantized token t into S: piece i (0..63) of the token
-// is one 16-byte cp.async; the caller commits.
-template <int KB, int VB>
-__device__ __forceinline__ void stage_piece(const FinishParams& p, int seg, int t, TokStage& S, int i) {
-  const uint8_t* rec = p.groups + ((size_t)seg * p.ng_cap + (size_t)(t / kKG)) * p.rec_bytes;
+// 16-byte piece i (0..23) of quantized token t's pieces into S: value codes,
+// value scales/zeros, the scan's weights (NT n-tiles) and running maxima.
+template <int KB, int VB, int NT>
+__device__ __forceinline__ void stage_piece(const FinishParams& p, int seg, int t, TokPieces& S, int i) {
+  const int g = t / kKG;
+  const size_t rg = (size_t)seg * p.ng_cap + (size_t)g;
+  const uint8_t* rec = p.groups + rg * p.rec_bytes;
   const int tt = t % kKG, kk = tt >> 4, row = tt & 7, tgt = (tt & 7) >> 1;
-  if (i < 32) {
-    cp_async16(S.ksz + 16 * i, rec + 16 * i);
-  } else if (i < 40) {
-    const int j = i - 32;
-    if (KB == 4) cp_async16(S.kcode + 16 * j, rec + off_kc() + kk * 1024 + row * 128 + 16 * j);
-    else if (j < 6) cp_async16(S.kcode + 16 * j, rec + off_kc() + kk * 768 + row * 96 + 16 * j);
-  } else if (i < 56) {
-    const int j = i - 40;
-    if (VB == 4 || j < 8) {
-      const int chunk = VB == 4 ? 2 * kk + (j >> 3) : kk;
-      cp_async16(S.vp + 16 * j, rec + off_vc(KB) + chunk * 512 + ((j & 7) * 4 + tgt) * 16);
+  if (i < 16) {
+    if (VB == 4 || i < 8) {
+      const int chunk = VB == 4 ? 2 * kk + (i >> 3) : kk;
+      cp_async16(S.vp + 16 * i, rec + off_vc(KB) + chunk * 512 + ((i & 7) * 4 + tgt) * 16);
     }
-  } else if (i < 60) {
-    const int j = i - 56;
+  } else if (i < 20) {
+    const int j = i - 16;
     cp_async16(S.vsz + 16 * j, rec + off_vs(KB) + kk * 128 + tgt * 32 + (j & 1) * 16 + (j >> 1) * 512);
+  } else if (i < 22) {
+    const int n = i - 20;
+    if (n < NT) cp_async16(S.w + 4 * n, p.wts + (rg * 4 * NT + (size_t)(kk * NT + n)) * 32 + row * 4);
   } else {
-    const int j = i - 60;
-    cp_async16(reinterpret_cast<uint8_t*>(S.mu) + 16 * j,
-               p.m_used + ((size_t)seg * p.ng_cap + (size_t)(t / kKG)) * (2 * kMaxG) + 4 * j);
+    const int j = i - 22;
+    cp_async16(S.mu + 4 * j, p.m_used + rg * kMaxG + 4 * j);
   }
 }
 
-// 16-byte piece `piece` (0..15) of token t's exact K (v = false) or V row.
-__device__ __forceinline__ uint4 row_piece(const FinishParams& p, int seg, int t, bool v, int piece) {
+// The lane's 4 channels (4 lane .. 4 lane + 3) of token t's exact K (v =
+// false) or V row, as raw bf16 pairs.
+__device__ __forceinline__ uint2 row4(const FinishParams& p, int seg, int t, bool v, int lane) {
   const bool tail = (t & (1 << 30)) != 0;
   const size_t off = tail ? ((size_t)seg * kTail + (t & 0xFFFF)) * kD : ((size_t)seg * p.capacity + t) * kD;
   const uint16_t* base = v ? (tail ? p.tail_v : p.v_exact) : (tail ? p.tail_k : p.k_exact);
-  return ld16<uint4>(base + off + 8 * piece);
+  return *reinterpret_cast<const uint2*>(base + off + 4 * lane);
 }
 
-// L2 prefetch of one of the four 128-byte halves of token t's exact K and V
-// rows.
+// L2 prefetch of one of the four 128-byte halves of token t's exact K and V rows.
 __device__ __forceinline__ void prefetch_part(const FinishParams& p, int seg, int t, int part) {
   const bool tail = (t & (1 << 30)) != 0;
   const size_t off = tail ? ((size_t)seg * kTail + (t & 0xFFFF)) * kD : ((size_t)seg * p.capacity + t) * kD;
@@ -316,333 +320,211 @@ __device__ __forceinline__ void prefetch_part(const FinishParams& p, int seg, in
   prefetch_l2(base + off + 64 * (part & 1));
 }
 
-// The scan's fp16 weights of quantized token t for every head, recomputed
-// from its staged group pieces with the scan's own functions on the same
-// operands (key_sz, scale_pos, q_tilde_col, key_afrag, qk_chain, approx_logit,
-// approx_weight; the group bias as the scan stored it); ph[j] = fp16 bits of
-// head j's weight, written by the lane whose MMA row and column hold it.
-// q2[n]: the lane's q of head (gid >> 1) + 4n, as the scan holds it.
-template <int KB, int G>
-__device__ __forceinline__ void replay_weights_t(const FinishParams& p, int t, const TokStage& S,
-                                                 const uint32_t (&q2)[2][16], int lane,
-                                                 uint16_t* ph) {
-  constexpr int NT = G > 4 ? 2 : 1;
-  const int gid = lane >> 2, tig = lane & 3;
-  const int tt = t % kKG, row = tt & 7, rr = (tt >> 3) & 1;
-  uint32_t sk[16], zk[16], sf[16], qb[NT][16];
-  float bk[NT];
-  key_sz(S.ksz, tig, sk, zk);
-  // the group bias of head tig + 4n exactly as the scan computed and stored it
+// L2 prefetch of everything the correction reads for quantized token t: its
+// exact K and V rows and its pieces (see stage_piece).
+template <int KB, int VB, int NT>
+__device__ __forceinline__ void prefetch_token(const FinishParams& p, int seg, int t) {
+  for (int part = 0; part < 4; ++part) prefetch_part(p, seg, t, part);
+  const int g = t / kKG;
+  const size_t rg = (size_t)seg * p.ng_cap + (size_t)g;
+  const uint8_t* rec = p.groups + rg * p.rec_bytes;
+  const int tt = t % kKG, kk = tt >> 4, row = tt & 7, tgt = (tt & 7) >> 1;
+  const uint8_t* vc = rec + off_vc(KB) + (VB == 4 ? 2 * kk : kk) * 512 + tgt * 16;
+  for (int i = 0; i < (VB == 4 ? 8 : 4); ++i) prefetch_l2(vc + 128 * i);
+  prefetch_l2(rec + off_vs(KB) + kk * 128 + tgt * 32);
+  prefetch_l2(rec + off_vs(KB) + 512 + kk * 128 + tgt * 32);
+  for (int n = 0; n < NT; ++n) prefetch_l2(p.wts + (rg * 4 * NT + (size_t)(kk * NT + n)) * 32 + row * 4);
+  prefetch_l2(p.m_used + rg * kMaxG);
+}
+
+// A warp's running softmax partial per query head over the tokens it
+// corrected: frame m (log2 units, uniform over the lanes), mass l and the
+// lane's 4 channels of acc; exact terms enter with +, the scan's
+// approximate terms of the same tokens with -.
+template <int G>
+struct WarpPart {
+  float m[G], l[G], acc[G][4];
+  __device__ __forceinline__ void init() {
 #pragma unroll
-  for (int n = 0; n < NT; ++n) bk[n] = S.mu[kMaxG + (tig + 4 * n < G ? tig + 4 * n : 0)];
-  scale_pos<KB>(sk, sf);
+    for (int h = 0; h < G; ++h) {
+      m[h] = -INFINITY;
+      l[h] = 0.f;
+      acc[h][0] = acc[h][1] = acc[h][2] = acc[h][3] = 0.f;
+    }
+  }
+};
+
+// Warp sum of V values per lane (V a power of two <= 32) by halving
+// exchanges: afterwards x[0] of lane L holds the sum of value
+// (L >> (5 - log2 V)) & (V - 1); 2V - 1 shuffles instead of 5V.
+template <int V>
+__device__ __forceinline__ void warp_sum_scatter(float (&x)[V], int lane) {
+  int n = V;
 #pragma unroll
-  for (int n = 0; n < NT; ++n) q_tilde_col(q2[n], sf, (gid & 1) != 0, qb[n]);
-  // only row `row` of the m-tile is staged; the other rows' codes are zero
-  // (an MMA output row depends on its own A row alone)
-  uint32_t w[KeyPos<KB>::WORDS];
-  const uint32_t* kw = reinterpret_cast<const uint32_t*>(S.kcode + tig * 4 * KeyPos<KB>::WORDS);
+  for (int o = 16; o >= 1; o >>= 1) {
+    if (n > 1) {
+      const bool up = (lane & o) != 0;
 #pragma unroll
-  for (int i = 0; i < KeyPos<KB>::WORDS; ++i) w[i] = gid == row ? kw[i] : 0u;
-  uint32_t a[16][2];
-  key_afrag<KB>(w, a);
-  const float kappa_u = p.kappa * KeyPos<KB>::unscale;
-#pragma unroll
-  for (int n = 0; n < NT; ++n) {
-    float d[4];
-    qk_chain(a, qb[n], d);
-    const int h = tig + 4 * n;
-    if (gid == row && h < G) ph[h] = f2h_rn(approx_weight(approx_logit(d, rr, kappa_u, bk[n]), S.mu[h]));
+      for (int i = 0; i < V / 2; ++i) {
+        if (i < n / 2) {
+          const float keep = up ? x[i + n / 2] : x[i];
+          const float send = up ? x[i] : x[i + n / 2];
+          x[i] = keep + __shfl_xor_sync(kAll, send, o);
+        }
+      }
+      n >>= 1;
+    } else {
+      x[0] += __shfl_xor_sync(kAll, x[0], o);
+    }
   }
 }
-__device__ __forceinline__ void mma_bf16_16816(float* d, uint32_t a0, uint32_t a1, uint32_t a2,
-                                               uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
-      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-// fp32 x as a bf16 triple hi + mid + lo (each the bf16 rounding of what the
-// previous limbs leave; the remainder is below 2^-24 |x|).
-__device__ __forceinline__ uint16_t bf16_bits(float x) {
-  return __bfloat16_as_ushort(__float2bfloat16_rn(x));
-}
-__device__ __forceinline__ float bf16_val(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
-__device__ __forceinline__ void split3(float x, uint16_t& hi, uint16_t& mid, uint16_t& lo) {
-  hi = bf16_bits(x);
-  const float r1 = x - bf16_val(hi);
-  mid = bf16_bits(r1);
-  lo = bf16_bits(r1 - bf16_val(mid));
-}
-// Correction of the tokens tok_at(0..n), 16 at a time, into this CTA's
-// combined partial P.run (frame m, mass l, acc; all 256 threads).  Batch
-// b + 1 is staged (record pieces by cp.async, exact rows through registers)
-// while batch b is computed:
-//   replay the scan's fp16 weights of each quantized token (warp w: tokens
-//          2w, 2w + 1); warp 0 also computes the 16 x 8 exact logits (bf16
-//          MMA) and moves the frame of a head when one of the batch's terms
-//          exceeds it by more than 2^8;
-//   weights thread (head, token): exact weight 2^(s - m), removed mass
-//          2^(m_used - m) p and removed value weights 2^(m_used - m) fp16(p s_v),
-//          split into bf16 triples / fp16 pairs (B operands);
-//   values warp w = channels 16w..16w+15: acc += V^T exact + codes^T removed;
-//          the last warp also sums the masses (ones x exact, ones x removed)
-//          and the zero-point terms (zeros x removed) on tensor cores; fp32
-//          accumulators stay in registers across batches.
-template <int G, int KB, int VB, typename TokAt>
-__device__ __forceinline__ void batch_correct(const FinishParams& p, int seg, TokAt tok_at, int n,
-                                              FinBatchT& B, FinParts<G>& P,
-                                              const uint32_t (&q2)[2][16],
-                                              const uint32_t (&qb)[8][2]) {
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int gid = lane >> 2, tig = lane & 3;
-  constexpr int kSumWarp = kFinThreads / 32 - 1;
-  const int c0 = 16 * warp + gid;
-  const bool h0ok = 2 * tig < G, h1ok = 2 * tig + 1 < G;
-  float acc[4];
-  acc[0] = h0ok ? P.run[2 * tig][4 + c0] : 0.f;
-  acc[1] = h1ok ? P.run[2 * tig + 1][4 + c0] : 0.f;
-  acc[2] = h0ok ? P.run[2 * tig][4 + c0 + 8] : 0.f;
-  acc[3] = h1ok ? P.run[2 * tig + 1][4 + c0 + 8] : 0.f;
-  // sums (last warp): dE = exact mass (every row), dF row 0 = removed mass,
-  // rows 1..4 = removed zero-point terms of channel groups 0..3
-  float dE[4], dF[4] = {0.f, 0.f, 0.f, 0.f};
-  dE[0] = dE[2] = h0ok ? P.run[2 * tig][1] : 0.f;
-  dE[1] = dE[3] = h1ok ? P.run[2 * tig + 1][1] : 0.f;
-  const int nbatch = (n + kBT - 1) / kBT;
-  // staging of batch bi into buffer buf: this warp's tokens 2w, 2w + 1;
-  // the lane's row pieces: token 2w + (lane >> 4), piece lane & 15
-  int rt = -1;
-  uint4 kx = make_uint4(0u, 0u, 0u, 0u), vx = kx;
-  auto issue = [&](int bi, int buf) {
+template <int V>
+constexpr int log2c() { return V <= 1 ? 0 : 1 + log2c<V / 2>(); }
+
+// Correct tokens list[warp + kFinWarps * j], j = 0, 1, ... (n entries in
+// the list) into the warp's partial WP, NC tokens at a time: record pieces
+// by cp.async into the warp's ring and the lane's row channels into
+// registers, all issued before the first is used; then (pass 1) every
+// token's exact logits, (pass 2) one frame move per head for the chunk and the
+// tokens' terms.
+template <int G, int KB, int VB>
+__device__ __forceinline__ void warp_correct(const FinishParams& p, int seg, const int32_t* list, int n,
+                                             FinWork& FW, const float* qf, WarpPart<G>& WP) {
+  constexpr int GP = G <= 1 ? 1 : G <= 2 ? 2 : G <= 4 ? 4 : 8;  // heads padded to a power of two
+  constexpr int NC = G > 4 ? 2 : kChunk;                        // tokens per chunk
+  constexpr int V = NC * GP;                                    // logits reduced together
+  constexpr int VSH = 5 - log2c<V>();
+  constexpr int NT = G > 4 ? 2 : 1;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nj = n > warp ? (n - warp + kFinWarps - 1) / kFinWarps : 0;
+  // the lane's channels: c = 4 lane + i, value group j = lane / 8; value-code
+  // word of channel c in the staged pieces (see vc_loc): row gid_c, high
+  // half chi of the channel m-tile mt
+  const int mt = lane >> 2, chi = (lane & 3) >> 1, gbase = 4 * (lane & 1), vj = lane >> 3;
+#pragma unroll 1
+  for (int j0 = 0; j0 < nj; j0 += NC) {
+    int tk[NC];
+    uint2 kr[NC], vr[NC];
 #pragma unroll
-    for (int k2 = 0; k2 < 2; ++k2) {
-      const int j = bi * kBT + 2 * warp + k2;
-      const int t = j < n ? tok_at(j) : -1;
-      if (tok_quant(t)) {
-        TokStage& S = B.st[buf][2 * warp + k2];
-#pragma unroll
-        for (int i = lane; i < 64; i += 32) stage_piece<KB, VB>(p, seg, t, S, i);
+    for (int u = 0; u < NC; ++u) {
+      const int j = j0 + u;
+      tk[u] = j < nj ? list[warp + kFinWarps * j] : -1;
+      if (tok_quant(tk[u])) {
+        if (lane < kTokPieces16) stage_piece<KB, VB, NT>(p, seg, tk[u], FW.ring[warp][u], lane);
       }
-      if ((lane >> 4) == k2) rt = t;
+      if (tk[u] != -1) {
+        kr[u] = row4(p, seg, tk[u], false, lane);
+        vr[u] = row4(p, seg, tk[u], true, lane);
+      } else {
+        kr[u] = vr[u] = make_uint2(0u, 0u);
+      }
     }
     cp_async_commit();
-    kx = make_uint4(0u, 0u, 0u, 0u);
-    vx = kx;
-    if (rt != -1) {
-      kx = row_piece(p, seg, rt, false, lane & 15);
-      vx = row_piece(p, seg, rt, true, lane & 15);
-    }
-  };
-  auto store_rows = [&](int buf) {
-    TokStage& S = B.st[buf][2 * warp + (lane >> 4)];
-    *reinterpret_cast<uint4*>(&S.krow[8 * (lane & 15)]) = kx;
-    *reinterpret_cast<uint4*>(&S.vrow[8 * (lane & 15)]) = vx;
-    if ((lane & 15) == 0) B.tok[buf][2 * warp + (lane >> 4)] = rt;
-  };
-  if (nbatch > 0) {
-    issue(0, 0);
-    store_rows(0);
-  }
-#pragma unroll 1
-  for (int bi = 0; bi < nbatch; ++bi) {
-    const int buf = bi & 1;
     cp_async_wait<0>();
-    __syncthreads();
-    if (bi + 1 < nbatch) issue(bi + 1, buf ^ 1);
-    // ---- exact logits and frames (warp 0), replay (warp w: tokens 2w, 2w + 1)
-    if (warp == 0) {
-      float d[4] = {0.f, 0.f, 0.f, 0.f};
+    __syncwarp();
+    // ---- pass 1: exact logits
+    float x[V];
 #pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        const uint16_t* r0 = B.st[buf][gid].krow + 16 * ks + 2 * tig;
-        const uint16_t* r1 = B.st[buf][gid + 8].krow + 16 * ks + 2 * tig;
-        mma_bf16_16816(d, *reinterpret_cast<const uint32_t*>(r0), *reinterpret_cast<const uint32_t*>(r1),
-                       *reinterpret_cast<const uint32_t*>(r0 + 8), *reinterpret_cast<const uint32_t*>(r1 + 8),
-                       qb[ks][0], qb[ks][1]);
-      }
+    for (int u = 0; u < NC; ++u) {
+      const float k0 = __uint_as_float(kr[u].x << 16), k1 = __uint_as_float(kr[u].x & 0xFFFF0000u);
+      const float k2 = __uint_as_float(kr[u].y << 16), k3 = __uint_as_float(kr[u].y & 0xFFFF0000u);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) d[i] *= p.kappa;
-      B.se[gid][2 * tig] = d[0];
-      B.se[gid][2 * tig + 1] = d[1];
-      B.se[gid + 8][2 * tig] = d[2];
-      B.se[gid + 8][2 * tig + 1] = d[3];
-      // the batch's largest term per head (exact logits, the scan maxima of
-      // the removed tokens' groups), over the 16 token rows
-      const int ta = B.tok[buf][gid], tb = B.tok[buf][gid + 8];
-      const float* mua = B.st[buf][gid].mu;
-      const float* mub = B.st[buf][gid + 8].mu;
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        const int h = 2 * tig + c;
-        float v = -INFINITY;
-        if (ta != -1) v = fmaxf(v, d[c]);
-        if (tb != -1) v = fmaxf(v, d[2 + c]);
-        if (tok_quant(ta)) v = fmaxf(v, mua[h]);
-        if (tok_quant(tb)) v = fmaxf(v, mub[h]);
-        v = fmaxf(v, __shfl_xor_sync(kAll, v, 4));
-        v = fmaxf(v, __shfl_xor_sync(kAll, v, 8));
-        v = fmaxf(v, __shfl_xor_sync(kAll, v, 16));
-        if (gid == 0 && h < G) {
-          const float m = P.run[h][0];
-          float al = 1.f;
-          if (v > m + 8.f) {
-            al = exp2f(m - v);  // 0 while the partial is empty (m = -inf)
-            P.run[h][0] = v;
-          }
-          B.alpha[h] = al;
+      for (int h = 0; h < GP; ++h) {
+        if (h < G) {
+          const float4 qv = *reinterpret_cast<const float4*>(qf + h * kD + 4 * lane);
+          x[u * GP + h] = fmaf(qv.w, k3, fmaf(qv.z, k2, fmaf(qv.y, k1, qv.x * k0)));
+        } else {
+          x[u * GP + h] = 0.f;
         }
       }
     }
-#pragma unroll 1
-    for (int k2 = 0; k2 < 2; ++k2) {
-      const int tl = 2 * warp + k2, t = B.tok[buf][tl];
-      if (tok_quant(t)) replay_weights_t<KB, G>(p, t, B.st[buf][tl], q2, lane, B.ph[tl]);
-    }
-    __syncthreads();
-    // ---- weights: thread (head h, token slot tl)
-    if (tid < kBT * G) {
-      const int h = tid >> 4, tl = tid & 15;
-      const int t = B.tok[buf][tl];
-      const bool valid = t != -1, qt = tok_quant(t);
-      const TokStage& S = B.st[buf][tl];
-      const float m = P.run[h][0];
-      const float pe = valid ? exp2f(B.se[tl][h] - m) : 0.f;
-      split3(pe, B.bex[0][h][tl], B.bex[1][h][tl], B.bex[2][h][tl]);
-      const float f = qt ? exp2f(S.mu[h] - m) : 0.f;
-      const uint16_t phb = qt ? B.ph[tl][h] : (uint16_t)0;
-      const float pf = h2f(phb) * f;
-      const uint16_t pfh = f2h_rn(pf);
-      B.bpf[0][h][tl] = pfh;
-      B.bpf[1][h][tl] = f2h_rn(pf - h2f(pfh));
-      const int tt = qt ? t % kKG : 0, hi8 = (tt & 15) >> 3, e = tt & 1;
+    warp_sum_scatter<V>(x, lane);
+    // exact logit (log2 units) of value v = u * GP + h: lanes with v(L) = v
+    auto se_of = [&](int u, int h) {
+      return __shfl_sync(kAll, x[0], ((u * GP + h) << VSH)) * p.kappa;
+    };
+    float se[NC][G];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const uint16_t vsc = *reinterpret_cast<const uint16_t*>(S.vsz + j * 8 + hi8 * 4 + 2 * e);
-        const float wv = qt ? h2f(h_mul_rn(phb, vsc)) * f : 0.f;
-        split3(-wv, B.brem[0][j][h][tl], B.brem[1][j][h][tl], B.brem[2][j][h][tl]);
+    for (int u = 0; u < NC; ++u)
+#pragma unroll
+      for (int h = 0; h < G; ++h) se[u][h] = se_of(u, h);
+    // ---- pass 2: frame moves (the chunk's largest term per head), then terms
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      float top = -INFINITY;
+#pragma unroll
+      for (int u = 0; u < NC; ++u) {
+        if (tk[u] != -1) top = fmaxf(top, se[u][h]);
+        if (tok_quant(tk[u])) top = fmaxf(top, FW.ring[warp][u].mu[h]);
+      }
+      if (top > WP.m[h] + 8.f) {  // move the frame (0 while the partial is empty)
+        const float al = exp2f(WP.m[h] - top);
+        WP.l[h] *= al;
+        WP.acc[h][0] *= al;
+        WP.acc[h][1] *= al;
+        WP.acc[h][2] *= al;
+        WP.acc[h][3] *= al;
+        WP.m[h] = top;
       }
     }
-    __syncthreads();
-    // ---- values: warp w = channels 16w .. 16w + 15
-    {
-      const float a0s = h0ok ? B.alpha[2 * tig] : 1.f;
-      const float a1s = h1ok ? B.alpha[2 * tig + 1] : 1.f;
-      acc[0] *= a0s;
-      acc[1] *= a1s;
-      acc[2] *= a0s;
-      acc[3] *= a1s;
-      // A operands: rows = channels c0, c0 + 8; columns = token slots
-      // 2tig, 2tig + 1 (a0, a1) and 2tig + 8, 2tig + 9 (a2, a3)
-      uint32_t va[4], ca[4];
 #pragma unroll
-      for (int hs = 0; hs < 2; ++hs) {
-        const int s0 = 2 * tig + 8 * hs;
-        const TokStage& S0 = B.st[buf][s0];
-        const TokStage& S1 = B.st[buf][s0 + 1];
-        va[2 * hs] = (uint32_t)S0.vrow[c0] | ((uint32_t)S1.vrow[c0] << 16);
-        va[2 * hs + 1] = (uint32_t)S0.vrow[c0 + 8] | ((uint32_t)S1.vrow[c0 + 8] << 16);
-        uint32_t cb[2][2];  // [token][row half]: bf16 bits of the code
+    for (int u = 0; u < NC; ++u) {
+      const int t = tk[u];
+      if (t == -1) continue;  // warp-uniform
+      const bool quant = tok_quant(t);
+      const TokPieces& S = FW.ring[warp][u];
+      const float v0 = __uint_as_float(vr[u].x << 16), v1 = __uint_as_float(vr[u].x & 0xFFFF0000u);
+      const float v2 = __uint_as_float(vr[u].y << 16), v3 = __uint_as_float(vr[u].y & 0xFFFF0000u);
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int t = B.tok[buf][s0 + u];
-          const TokStage& S = u ? S1 : S0;
-          uint32_t c_lo = 0u, c_hi = 0u;
-          if (tok_quant(t)) {
-            const int tt = t % kKG, hi8 = (tt & 15) >> 3, e = tt & 1;
-            const int bit = vc_pos(VB, warp) + 16 * e;
-            if (VB == 4) {
-              const int w8 = 2 * (warp & 3) + hi8;
-              const uint32_t wd = *reinterpret_cast<const uint32_t*>(S.vp + ((w8 >> 2) * 8 + gid) * 16 + (w8 & 3) * 4);
-              c_lo = (wd >> bit) & 15u;
-              c_hi = (wd >> (bit + 8)) & 15u;
-            } else {
-              const uint32_t wd = *reinterpret_cast<const uint32_t*>(S.vp + gid * 16 + (2 * (warp & 1) + hi8) * 4);
-              c_lo = (wd >> bit) & 3u;
-              c_hi = (wd >> (bit + 8)) & 3u;
-            }
+      for (int h = 0; h < G; ++h) {
+        const float pe = exp2f(se[u][h] - WP.m[h]);
+        WP.l[h] += pe;
+        WP.acc[h][0] = fmaf(pe, v0, WP.acc[h][0]);
+        WP.acc[h][1] = fmaf(pe, v1, WP.acc[h][1]);
+        WP.acc[h][2] = fmaf(pe, v2, WP.acc[h][2]);
+        WP.acc[h][3] = fmaf(pe, v3, WP.acc[h][3]);
+      }
+      if (quant) {
+        // removal operands: the value codes of the lane's channels, the
+        // value scale and zero of its channel group
+        const int tt = t % kKG, hi8 = (tt & 15) >> 3, e = tt & 1;
+        float code[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int gc = gbase + i;
+          uint32_t wd, c;
+          if (VB == 4) {
+            const int w8 = 2 * (mt & 3) + hi8;
+            wd = *reinterpret_cast<const uint32_t*>(S.vp + ((w8 >> 2) * 8 + gc) * 16 + (w8 & 3) * 4);
+            c = (wd >> (vc_pos(4, mt) + 8 * chi + 16 * e)) & 15u;
+          } else {
+            wd = *reinterpret_cast<const uint32_t*>(S.vp + gc * 16 + (2 * (mt & 1) + hi8) * 4);
+            c = (wd >> (vc_pos(2, mt) + 8 * chi + 16 * e)) & 3u;
           }
-          cb[u][0] = __float_as_uint((float)c_lo) >> 16;
-          cb[u][1] = __float_as_uint((float)c_hi) >> 16;
+          code[i] = (float)c;
         }
-        ca[2 * hs] = cb[0][0] | (cb[1][0] << 16);
-        ca[2 * hs + 1] = cb[0][1] | (cb[1][1] << 16);
-      }
-      const int j = warp >> 1;
+        const uint16_t vsc = *reinterpret_cast<const uint16_t*>(S.vsz + vj * 8 + hi8 * 4 + 2 * e);
+        const float vz = h2f(*reinterpret_cast<const uint16_t*>(S.vsz + 32 + vj * 8 + hi8 * 4 + 2 * e));
 #pragma unroll
-      for (int l = 0; l < 3; ++l)
-        mma_bf16_16816(acc, va[0], va[1], va[2], va[3], *reinterpret_cast<const uint32_t*>(&B.bex[l][gid][2 * tig]),
-                       *reinterpret_cast<const uint32_t*>(&B.bex[l][gid][2 * tig + 8]));
-#pragma unroll
-      for (int l = 0; l < 3; ++l)
-        mma_bf16_16816(acc, ca[0], ca[1], ca[2], ca[3], *reinterpret_cast<const uint32_t*>(&B.brem[l][j][gid][2 * tig]),
-                       *reinterpret_cast<const uint32_t*>(&B.brem[l][j][gid][2 * tig + 8]));
-      if (warp == kSumWarp) {
-        dE[0] *= a0s;
-        dE[1] *= a1s;
-        dE[2] *= a0s;
-        dE[3] *= a1s;
-        dF[0] *= a0s;
-        dF[1] *= a1s;
-        dF[2] *= a0s;
-        dF[3] *= a1s;
-        constexpr uint32_t kOnesBf = 0x3F803F80u;
-#pragma unroll
-        for (int l = 0; l < 3; ++l)
-          mma_bf16_16816(dE, kOnesBf, kOnesBf, kOnesBf, kOnesBf,
-                         *reinterpret_cast<const uint32_t*>(&B.bex[l][gid][2 * tig]),
-                         *reinterpret_cast<const uint32_t*>(&B.bex[l][gid][2 * tig + 8]));
-        // A rows: 0 = ones, 1..4 = the value zero points of channel group
-        // gid - 1 (fp16), others 0; columns = token slots
-        uint32_t za[2];
-#pragma unroll
-        for (int hs = 0; hs < 2; ++hs) {
-          uint32_t zz = 0u;
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int sl = 2 * tig + 8 * hs + u, t = B.tok[buf][sl];
-            uint32_t zh = 0u;
-            if (gid == 0) {
-              zh = 0x3C00u;
-            } else if (gid <= 4 && tok_quant(t)) {
-              const int tt = t % kKG, hi8 = (tt & 15) >> 3, e = tt & 1;
-              zh = *reinterpret_cast<const uint16_t*>(B.st[buf][sl].vsz + 32 + (gid - 1) * 8 + hi8 * 4 + 2 * e);
-            }
-            zz |= zh << (16 * u);
-          }
-          za[hs] = zz;
+        for (int h = 0; h < G; ++h) {
+          // the scan added fp16(p) to the mass, fp16(p) * m_v and
+          // fp16(fp16(p) * s_v) * code to the channels, against m_used
+          const uint16_t phb =
+              reinterpret_cast<const uint16_t*>(S.w)[2 * (4 * (h >> 2) + (h & 3)) + ((tt & 15) >> 3)];
+          const float f = exp2f(S.mu[h] - WP.m[h]);
+          const float pw = h2f(phb);
+          const float wv = h2f(h_mul_rn(phb, vsc));
+          const float pz = pw * vz;
+          WP.l[h] = fmaf(-f, pw, WP.l[h]);
+          WP.acc[h][0] = fmaf(-f, fmaf(wv, code[0], pz), WP.acc[h][0]);
+          WP.acc[h][1] = fmaf(-f, fmaf(wv, code[1], pz), WP.acc[h][1]);
+          WP.acc[h][2] = fmaf(-f, fmaf(wv, code[2], pz), WP.acc[h][2]);
+          WP.acc[h][3] = fmaf(-f, fmaf(wv, code[3], pz), WP.acc[h][3]);
         }
-#pragma unroll
-        for (int l = 0; l < 2; ++l)
-          mma16816(dF, za[0], 0u, za[1], 0u, *reinterpret_cast<const uint32_t*>(&B.bpf[l][gid][2 * tig]),
-                   *reinterpret_cast<const uint32_t*>(&B.bpf[l][gid][2 * tig + 8]));
       }
     }
-    if (bi + 1 < nbatch) store_rows(buf ^ 1);
+    __syncwarp();  // the ring is reused by the next chunk
   }
-  if (warp == kSumWarp) {
-    if (gid == 0) {  // mass: exact minus removed
-      if (h0ok) P.run[2 * tig][1] = dE[0] - dF[0];
-      if (h1ok) P.run[2 * tig + 1][1] = dE[1] - dF[1];
-    } else if (gid <= 4) {
-      if (h0ok) B.zsum[2 * tig][gid - 1] = -dF[0];
-      if (h1ok) B.zsum[2 * tig + 1][gid - 1] = -dF[1];
-    }
-  }
-  __syncthreads();
-  {
-    const int j = warp >> 1;
-    if (h0ok) {
-      P.run[2 * tig][4 + c0] = acc[0] + B.zsum[2 * tig][j];
-      P.run[2 * tig][4 + c0 + 8] = acc[2] + B.zsum[2 * tig][j];
-    }
-    if (h1ok) {
-      P.run[2 * tig + 1][4 + c0] = acc[1] + B.zsum[2 * tig + 1][j];
-      P.run[2 * tig + 1][4 + c0 + 8] = acc[3] + B.zsum[2 * tig + 1][j];
-    }
-  }
-  __syncthreads();
 }
 
 template <int G, bool SELECT, int KB, int VB>
@@ -650,9 +532,12 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
   extern __shared__ __align__(16) uint8_t fsm[];
   FinPersist& PS = *reinterpret_cast<FinPersist*>(fsm);
   FinParts<G>& P = *reinterpret_cast<FinParts<G>*>(fsm + sizeof(FinPersist));
-  uint8_t* U = fsm + sizeof(FinPersist) + sizeof(FinParts<G>);
-  FinSelect& SS = *reinterpret_cast<FinSelect*>(U);
-  FinCorr& FC = *reinterpret_cast<FinCorr*>(U);
+  float* qf = reinterpret_cast<float*>(fsm + sizeof(FinPersist) + sizeof(FinParts<G>));
+  int32_t* tok = reinterpret_cast<int32_t*>(qf + G * kD);
+  uint8_t* U = reinterpret_cast<uint8_t*>(tok + kTokCap + kTail);
+  FinWork& FW = *reinterpret_cast<FinWork*>(U);
+  FinMerge<G>& FM = *reinterpret_cast<FinMerge<G>*>(U);
+  float* early = reinterpret_cast<float*>(U + fin_union_bytes<G>());
   __shared__ uint32_t scratch[32];
   __shared__ int s_bin;
   __shared__ uint32_t s_above, s_tot;
@@ -660,12 +545,13 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
   __shared__ uint32_t s_chq[kFinMaxC + 1];  // chosen ties before slice q
   __shared__ int s_mode;                     // 0 lists in shared memory, 1 fallback lists
   __shared__ uint32_t s_hmax[kMaxG];          // per head: largest scan-partial maximum (key)
+  __shared__ uint32_t s_tie[kFinMaxC], s_ovf[kFinMaxC];
 
   cg::cluster_group cl = cg::this_cluster();
   const int C = (int)cl.num_blocks();
   const int r = (int)cl.block_rank();
   const int seg = blockIdx.x / C;
-  const int tid = threadIdx.x, lane = tid & 31, gid = lane >> 2, tig = lane & 3;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gid = lane >> 2, tig = lane & 3;
   const int nq = p.nq, k = p.k;
   const int bb = seg / p.hkv, hh = seg % p.hkv;
 
@@ -675,62 +561,44 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
     for (int i = tid; i < n_mine * 4; i += kFinThreads)
       prefetch_part(p, seg, (1 << 30) | (r + C * (i >> 2)), i & 3);
   }
-  for (int i = tid; i < G * kPartStride; i += kFinThreads)
-    (&P.run[0][0])[i] = (i % kPartStride) == 0 ? -INFINITY : 0.f;
-  // the lane's q as the scan holds it (head (gid >> 1) + 4n of n-tile n), and
-  // as bf16 B fragments of the exact-logit MMA (head gid)
-  uint32_t q2[2][16];
-#pragma unroll
-  for (int n = 0; n < 2; ++n) {
-    const int hq = (gid >> 1) + 4 * n;
-    const bool ok = hq < G && (n == 0 || G > 4);
-    q_frag(p.q + ((size_t)bb * p.H + (size_t)hh * G + (ok ? hq : 0)) * kD, ok, tig, q2[n]);
-  }
-  uint32_t qb[8][2];
-  {
-    const uint16_t* qrow = p.q + ((size_t)bb * p.H + (size_t)hh * G + (gid < G ? gid : 0)) * kD;
-#pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-      qb[ks][0] = gid < G ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * tig) : 0u;
-      qb[ks][1] = gid < G ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * tig + 8) : 0u;
-    }
+  for (int i = tid; i < G * kD; i += kFinThreads) {
+    const uint16_t b = p.q[((size_t)bb * p.H + (size_t)hh * G) * kD + i];
+    qf[i] = __uint_as_float((uint32_t)b << 16);
   }
   __syncthreads();
 
   pdl_wait();
   pdl_launch_dependents();
 
-  // ---- P5a (loads): this CTA's share of the scan's split partials, every
-  // head: when the rows fit beside the selection buffers they are copied now
-  // (cp.async) and merged after the selection, so their latency hides
-  // behind it; else they are staged tile by tile then.
-    long long w0 = 0, w1 = -1;
-    if (p.ng > 0) {
-      const long long T = p.scan_total, W = p.scan_warps;
-      const long long x0 = (long long)seg * p.ng, x1 = x0 + p.ng - 1;
-      w0 = scan_warp_of(x0, W, T);
-      w1 = scan_warp_of(x1, W, T);
+  // ---- early copy of this CTA's share of the scan's split partials, every
+  // head: when the rows fit they are copied now (cp.async) and merged at the
+  // end, so their latency hides behind the selection and the correction
+  long long w0 = 0, w1 = -1;
+  if (p.ng > 0) {
+    const long long T = p.scan_total, W = p.scan_warps;
+    const long long x0 = (long long)seg * p.ng, x1 = x0 + p.ng - 1;
+    w0 = scan_warp_of(x0, W, T);
+    w1 = scan_warp_of(x1, W, T);
+  }
+  const int ns = (int)(w1 - w0 + 1);  // one partial slot per scan warp of the segment
+  const int s0 = (int)((long long)ns * r / C), s1 = (int)((long long)ns * (r + 1) / C);
+  constexpr int kV = kPartStride / 4;  // float4 per row
+  const int nrows = (s1 - s0) * G;
+  constexpr int kEarlyRows = (int)(kEarlyBytes / (kPartStride * sizeof(float)));
+  const bool early_ok = nrows <= kEarlyRows;
+  if (early_ok) {
+    for (int i = tid; i < nrows * kV; i += kFinThreads) {
+      const int row = i / kV, v = i % kV;
+      cp_async16(early + row * kPartStride + 4 * v,
+                 p.scan_part + ((size_t)(w0 + s0 + row / G + seg) * G + row % G) * kPartStride + 4 * v);
     }
-    const int ns = (int)(w1 - w0 + 1);  // one partial slot per scan warp of the segment
-    const int s0 = (int)((long long)ns * r / C), s1 = (int)((long long)ns * (r + 1) / C);
-    constexpr int kV = kPartStride / 4;  // float4 per row
-    const int nrows = (s1 - s0) * G;
-    float* early = reinterpret_cast<float*>(U + sizeof(FinSelect));
-    constexpr int kEarlyRows = (int)((sizeof(FinCorr) - sizeof(FinSelect)) / (kPartStride * sizeof(float)));
-    const bool early_ok = nrows <= kEarlyRows;
-    if (early_ok) {
-      for (int i = tid; i < nrows * kV; i += kFinThreads) {
-        const int row = i / kV, v = i % kV;
-        cp_async16(early + row * kPartStride + 4 * v,
-                   p.scan_part + ((size_t)(w0 + s0 + row / G + seg) * G + row % G) * kPartStride + 4 * v);
-      }
-    }
-    cp_async_commit();
+  }
+  cp_async_commit();
 
   const bool select = SELECT && k < nq;
   const int lo = min(nq, r * p.slice), hi = min(nq, lo + p.slice);
   bool hist_ok = false;
-  // ---- P1 + P2: bin b* from the scan's histogram, then this slice's lists
+  // ---- S1 + S2: bin b* from the scan's histogram, then this slice's lists
   if (select) {
     // the slice's first 16 scores of this thread, loaded together with the
     // histogram so both round trips overlap
@@ -739,40 +607,41 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int b0 = lo + 16 * tid + 4 * u;
-      v0[u] = b0 < hi ? ld16<float4>(S + b0) : make_float4(0.f, 0.f, 0.f, 0.f);
+      v0[u] = b0 < hi ? *reinterpret_cast<const float4*>(S + b0) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    // thread t owns bins [32t, 32t + 32): loaded straight into registers
-    const uint32_t* hg = p.hist + (size_t)seg * kScanHistBins + 32 * tid;
-    uint32_t hb[32];
+    // the bin holding the k-th largest key: a window of 1024 bins below the
+    // segment's largest key (thread t owns 4 bins), then further windows
+    // down while the keys counted so far are fewer than k
+    const uint32_t* hg = p.hist + (size_t)seg * kScanHistStride;
+    const int top = (int)(hg[kScanHistBins] >> (32 - kScanHistBits));
+    int whi = min(kScanHistBins, (top | 3) + 1);
+    uint32_t above = 0;  // keys in the bins above the current window
+#pragma unroll 1
+    for (;;) {
+      const int wlo = max(0, whi - 4 * kFinThreads);
+      const int b0 = wlo + 4 * tid;
+      const uint4 hv = b0 < whi ? *reinterpret_cast<const uint4*>(hg + b0) : make_uint4(0u, 0u, 0u, 0u);
+      if (tid == 0) s_bin = -1;
+      uint32_t cum = above + block_suffix_excl(hv.x + hv.y + hv.z + hv.w, scratch);
+      const uint32_t hb[4] = {hv.x, hv.y, hv.z, hv.w};
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const uint4 v = ld16<uint4>(hg + 4 * u);
-      hb[4 * u] = v.x;
-      hb[4 * u + 1] = v.y;
-      hb[4 * u + 2] = v.z;
-      hb[4 * u + 3] = v.w;
-    }
-    uint32_t local = 0;
-#pragma unroll
-    for (int i = 0; i < 32; ++i) local += hb[i];
-    uint32_t tot_all;
-    block_prefix_excl(local, scratch, &tot_all);
-    uint32_t cum = block_suffix_excl(local, scratch);  // keys in bins above this thread's
-    if (tid == 0) {
-      s_bin = -1;
-      s_tot = tot_all;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int i = 31; i >= 0; --i) {
-      if (cum < (uint32_t)k && cum + hb[i] >= (uint32_t)k) {
-        s_bin = 32 * tid + i;
-        s_above = cum;
+      for (int i = 3; i >= 0; --i) {
+        if (cum < (uint32_t)k && cum + hb[i] >= (uint32_t)k) {
+          s_bin = b0 + i;
+          s_above = cum;
+        }
+        cum += hb[i];
       }
-      cum += hb[i];
+      if (tid == 0) s_tot = cum;  // every key in the bins from wlo up
+      __syncthreads();
+      if (s_bin >= 0 || wlo == 0) break;
+      above = s_tot;
+      whi = wlo;
+      __syncthreads();
     }
-    __syncthreads();
-    hist_ok = s_tot == (uint32_t)nq && s_bin >= 0;
+    // the lists below are checked against the counts the histogram promised,
+    // so a histogram that does not match these scores only costs the fallback
+    hist_ok = s_bin >= 0;
     const uint32_t bstar = (uint32_t)s_bin;
     uint32_t base_s = 0, base_t = 0;
     if (hist_ok) {
@@ -782,9 +651,10 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
 #pragma unroll
         for (int u = 0; u < 4; ++u)
           v[u] = t0 == lo ? v0[u]
-                          : (b0 + 4 * u < hi ? ld16<float4>(S + b0 + 4 * u) : make_float4(0.f, 0.f, 0.f, 0.f));
+                          : (b0 + 4 * u < hi ? *reinterpret_cast<const float4*>(S + b0 + 4 * u)
+                                             : make_float4(0.f, 0.f, 0.f, 0.f));
         uint32_t keys[16];
-        uint32_t ms = 0, mt = 0, ns = 0, nt = 0;
+        uint32_t ms = 0, mtie = 0, nsu = 0, nti = 0;
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           const float vals[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
@@ -795,14 +665,15 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
             const bool in = b0 + i < hi;
             const uint32_t bin = keys[i] >> (32 - kScanHistBits);
             const bool su = in && bin > bstar, ti = in && bin == bstar;
+            if (su) prefetch_token<KB, VB, (G > 4 ? 2 : 1)>(p, seg, b0 + i);
             ms |= (su ? 1u : 0u) << i;
-            mt |= (ti ? 1u : 0u) << i;
-            ns += su;
-            nt += ti;
+            mtie |= (ti ? 1u : 0u) << i;
+            nsu += su;
+            nti += ti;
           }
         }
         uint32_t tot;
-        const uint32_t pos = block_prefix_excl((ns << 16) | nt, scratch, &tot);
+        const uint32_t pos = block_prefix_excl((nsu << 16) | nti, scratch, &tot);
         uint32_t ps = base_s + (pos >> 16), pt = base_t + (pos & 0xFFFFu);
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
@@ -810,7 +681,7 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
             if (ps < (uint32_t)kLCap) PS.sure[ps] = (uint32_t)(b0 + i);
             ++ps;
           }
-          if (mt & (1u << i)) {
+          if (mtie & (1u << i)) {
             if (pt < (uint32_t)kLCap) {
               PS.tkey[pt] = keys[i];
               PS.tidx[pt] = (uint32_t)(b0 + i);
@@ -827,20 +698,78 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
       PS.n_tie = base_t;
       PS.overflow = (base_s > (uint32_t)kLCap || base_t > (uint32_t)kLCap) ? 1u : 0u;
     }
+    __syncthreads();
+    cluster_arrive();  // lists and counts are visible to the cluster
   }
-  cl.sync();
 
-  // ---- P3: resolve the selection; every CTA knows the whole chosen set:
-  // list q (CTA q's sure list, or its fallback list) and the chosen ties.
+  // ---- A: correct the tail slots and, when the lists hold, the sure tokens
+  // of the slice (or the CTA's share of a given / complete index set)
+  WarpPart<G> WP;
+  WP.init();
+  const int n_tail = p.tail > r ? (p.tail - r + C - 1) / C : 0;
+  if (select) {
+    const uint32_t ns_me = hist_ok && PS.overflow == 0u ? PS.n_sure : 0u;
+    for (int i = tid; i < n_tail; i += kFinThreads) tok[i] = (1 << 30) | (r + C * i);
+    // the sure list in chunks of kTokCap (beside the tail slots)
+#pragma unroll 1
+    for (uint32_t c0 = 0, first = 1; first || c0 < ns_me; c0 += kTokCap, first = 0) {
+      const int base = first ? n_tail : 0;
+      const uint32_t cn = min((uint32_t)kTokCap, ns_me - min(ns_me, c0));
+      for (uint32_t i = tid; i < cn; i += kFinThreads) tok[base + i] = (int32_t)PS.sure[c0 + i];
+      __syncthreads();
+      warp_correct<G, KB, VB>(p, seg, tok, base + (int)cn, FW, qf, WP);
+      __syncthreads();
+    }
+  } else {
+    // positions [x0, x1) of the set: idx_in entries, or every quantized token
+    const int n_x = SELECT ? nq : k;
+    const int per = (n_x + C - 1) / C;
+    const int x0 = min(n_x, r * per), x1 = min(n_x, x0 + per);
+#pragma unroll 1
+    for (int xr = x0, first = 1; first || xr < x1; xr += kTokCap, first = 0) {
+      const int xe = min(x1, xr + kTokCap);
+      uint32_t base = 0;
+      if (first) {
+        for (int i = tid; i < n_tail; i += kFinThreads) tok[i] = (1 << 30) | (r + C * i);
+        base = (uint32_t)n_tail;
+      }
+#pragma unroll 1
+      for (int xb = xr; xb < xe; xb += kFinThreads) {
+        const int j = xb + tid;
+        int t = -1;
+        if (j < xe) {
+          if (SELECT) {
+            t = j;
+          } else {
+            t = p.idx_in[(size_t)seg * k + j];
+            if (t < -1 || t >= nq) {
+              set_flag(p.flag, JFA_DEVERR_BAD_INDEX);
+              t = -1;
+            }
+          }
+        }
+        uint32_t tot;
+        const uint32_t pos = base + block_prefix_excl(t >= 0 ? 1u : 0u, scratch, &tot);
+        if (t >= 0) tok[pos] = t;
+        base += tot;
+      }
+      __syncthreads();
+      warp_correct<G, KB, VB>(p, seg, tok, (int)base, FW, qf, WP);
+      __syncthreads();
+    }
+  }
+
+  // ---- S3 + B: resolve the selection, correct the chosen ties of the slice
   uint32_t n_ch = 0;  // chosen ties (ascending in PS.chtie)
   const uint32_t* glist_base = p.glists + (size_t)seg * C * p.slice;
+  int mode = 0;
   if (select) {
-    if (r == 0) {  // the scan's histogram is consumed: clear it for the next scan
-      uint32_t* hg = p.hist + (size_t)seg * kScanHistBins;
-      for (int i = 4 * tid; i < kScanHistBins; i += 4 * kFinThreads)
+    cluster_wait();
+    {  // the scan's histogram is consumed: clear it for the next scan
+      uint32_t* hg = p.hist + (size_t)seg * kScanHistStride;
+      for (int i = 4 * (r * kFinThreads + tid); i < kScanHistStride; i += 4 * C * kFinThreads)
         *reinterpret_cast<uint4*>(hg + i) = make_uint4(0u, 0u, 0u, 0u);
     }
-    __shared__ uint32_t s_tie[kFinMaxC], s_ovf[kFinMaxC];
     if (tid < C) {
       const FinPersist* o = cl.map_shared_rank(&PS, tid);
       s_cnt[tid] = o->n_sure;
@@ -864,33 +793,34 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
       s_mode = (!hist_ok || ovf || pt > (uint32_t)kTCap || !consistent) ? 1 : 0;
     }
     __syncthreads();
-    if (s_mode == 0) {
+    mode = s_mode;
+    if (mode == 0) {
       // every CTA's ties in one pass (all remote loads in flight together)
       for (uint32_t i = tid; i < s_tpre[C]; i += kFinThreads) {
         int q = 0;
         while (q + 1 < C && s_tpre[q + 1] <= i) ++q;
         const FinPersist* o = cl.map_shared_rank(&PS, q);
-        SS.akey[i] = o->tkey[i - s_tpre[q]];
-        SS.aidx[i] = o->tidx[i - s_tpre[q]];
+        FW.akey[i] = o->tkey[i - s_tpre[q]];
+        FW.aidx[i] = o->tidx[i - s_tpre[q]];
       }
       __syncthreads();
       n_ch = (uint32_t)k - s_pre[C];
       const uint32_t T = s_tpre[C];
-      if (T <= (uint32_t)kFinThreads / 2) {
+      if (T <= (uint32_t)kFinThreads) {
         // direct ranking: entry i is chosen iff fewer than n_ch entries come
         // before it in (key descending, index ascending) order; tpe threads
         // (a power of two) share an entry's comparisons
-        uint32_t tpe = 2;
+        uint32_t tpe = 1;
         while (tpe < 32 && tpe * 2 * T <= (uint32_t)kFinThreads) tpe *= 2;
         const uint32_t e = tid / tpe, part = tid % tpe;
         uint32_t rank = 0, my_idx = 0;
         if (e < T) {
-          const uint32_t key = SS.akey[e];
-          my_idx = SS.aidx[e];
+          const uint32_t key = FW.akey[e];
+          my_idx = FW.aidx[e];
 #pragma unroll 4
           for (uint32_t j = part; j < T; j += tpe) {
-            const uint32_t k2 = SS.akey[j];
-            rank += (k2 > key || (k2 == key && SS.aidx[j] < my_idx)) ? 1u : 0u;
+            const uint32_t k2 = FW.akey[j];
+            rank += (k2 > key || (k2 == key && FW.aidx[j] < my_idx)) ? 1u : 0u;
           }
         }
         for (uint32_t o = 1; o < tpe; o <<= 1) rank += __shfl_xor_sync(kAll, rank, o);
@@ -900,47 +830,64 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
         if (chosen) PS.chtie[pos] = my_idx;  // entries are in index order
         __syncthreads();
       } else {
-        refine_ties(SS.akey, SS.aidx, T, n_ch, SS.hist, PS.chtie, scratch, &s_bin, &s_above,
+        refine_ties(FW.akey, FW.aidx, T, n_ch, FW.hist, PS.chtie, scratch, &s_bin, &s_above,
                     &s_tot);
       }
+      if (tid <= C) {
+        const uint32_t b0 = (uint32_t)min(nq, tid * p.slice);
+        s_chq[tid] = lower_bound_u32(PS.chtie, n_ch, b0);
+      }
+      __syncthreads();
+      // B: the chosen ties of this slice
+      const uint32_t c0 = s_chq[r], c1 = s_chq[r + 1];
+#pragma unroll 1
+      for (uint32_t cb = c0; cb < c1; cb += kTokCap) {
+        const uint32_t cn = min((uint32_t)kTokCap, c1 - cb);
+        for (uint32_t i = tid; i < cn; i += kFinThreads) tok[i] = (int32_t)PS.chtie[cb + i];
+        __syncthreads();
+        warp_correct<G, KB, VB>(p, seg, tok, (int)cn, FW, qf, WP);
+        __syncthreads();
+      }
     } else {
-      const uint32_t n =
-          select_full(p.scores + (size_t)seg * p.capacity, nq, k, lo, hi, SS.hist,
-                      const_cast<uint32_t*>(glist_base) + (size_t)r * p.slice, scratch, &s_bin,
-                      &s_above, &s_tot);
+      // fallback: select over the whole segment; the correction restarts on
+      // the tail slots and this slice's chosen tokens
+      uint32_t* gl = const_cast<uint32_t*>(glist_base) + (size_t)r * p.slice;
+      const uint32_t n = select_full(p.scores + (size_t)seg * p.capacity, nq, k, lo, hi, FW.hist, gl,
+                                     scratch, &s_bin, &s_above, &s_tot);
       if (tid == 0) PS.n_gl = n;
       __threadfence();
-    }
-  }
-  const int mode = select ? s_mode : 0;
-  if (select && mode == 1) {
-    cl.sync();  // the fallback lists and counts are complete
-    if (tid < C) s_cnt[tid] = cl.map_shared_rank(&PS, tid)->n_gl;
-    __syncthreads();
-    if (tid == 0) {
-      uint32_t ps = 0;
-      for (int q = 0; q < C; ++q) {
-        s_pre[q] = ps;
-        ps += s_cnt[q];
+      WP.init();
+#pragma unroll 1
+      for (uint32_t c0 = 0, first = 1; first || c0 < n; c0 += kTokCap, first = 0) {
+        const int base = first ? n_tail : 0;
+        if (first)
+          for (int i = tid; i < n_tail; i += kFinThreads) tok[i] = (1 << 30) | (r + C * i);
+        const uint32_t cn = min((uint32_t)kTokCap, n - min(n, c0));
+        for (uint32_t i = tid; i < cn; i += kFinThreads) tok[base + i] = (int32_t)gl[c0 + i];
+        __syncthreads();
+        warp_correct<G, KB, VB>(p, seg, tok, base + (int)cn, FW, qf, WP);
+        __syncthreads();
       }
-      s_pre[C] = ps;
+      cl.sync();  // the fallback lists and counts are complete
+      if (tid < C) s_cnt[tid] = cl.map_shared_rank(&PS, tid)->n_gl;
+      __syncthreads();
+      if (tid == 0) {
+        uint32_t ps = 0;
+        for (int q = 0; q < C; ++q) {
+          s_pre[q] = ps;
+          ps += s_cnt[q];
+        }
+        s_pre[C] = ps;
+      }
+      __syncthreads();
     }
-    __syncthreads();
   }
-  auto list_of = [&](int q) -> const uint32_t* {
-    return mode == 1 ? glist_base + (size_t)q * p.slice : cl.map_shared_rank(PS.sure, q);
-  };
 
   // ---- idx output: this CTA's chosen indices, ascending, at its offset
   if (select) {
-    if (tid <= C) {
-      const uint32_t b0 = (uint32_t)min(nq, tid * p.slice);
-      s_chq[tid] = lower_bound_u32(PS.chtie, n_ch, b0);
-    }
-    __syncthreads();
-    const uint32_t c0 = s_chq[r], c1 = s_chq[r + 1];
+    const uint32_t c0 = mode == 0 ? s_chq[r] : 0u, c1 = mode == 0 ? s_chq[r + 1] : 0u;
     const uint32_t off = s_pre[r] + c0;  // earlier slices: their lists and chosen ties
-    const uint32_t* Lr = list_of(r);
+    const uint32_t* Lr = mode == 1 ? glist_base + (size_t)r * p.slice : PS.sure;
     const uint32_t nr = s_cnt[r];
     int32_t* out = p.idx_out + (size_t)seg * k;
     for (uint32_t i = tid; i < nr; i += kFinThreads) {
@@ -957,21 +904,56 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
     int32_t* out = p.idx_out + (size_t)seg * k;
     for (int i = tid; i < k; i += kFinThreads) out[i] = i < nq ? i : -1;
   }
-  if (!SELECT && r == 0) {  // nothing reads the scan's histogram here: clear it
-    uint32_t* hg = p.hist + (size_t)seg * kScanHistBins;
-    for (int i = 4 * tid; i < kScanHistBins; i += 4 * kFinThreads)
+  if (!select) {  // nothing reads the scan's histogram here: clear it
+    uint32_t* hg = p.hist + (size_t)seg * kScanHistStride;
+    for (int i = 4 * (r * kFinThreads + tid); i < kScanHistStride; i += 4 * C * kFinThreads)
       *reinterpret_cast<uint4*>(hg + i) = make_uint4(0u, 0u, 0u, 0u);
   }
 
-  // ---- P5a (merge): per head the largest partial maximum M first, then
-  // every row's terms scaled by 2^(m_row - M) and summed (no exponential on
-  // the accumulation chain); rows from the early copy, else staged a tile
+  // ---- M1: the warps' partials into this CTA's partial P.run (per head the
+  // largest frame first, then every warp's terms scaled to it)
+  __syncthreads();  // the correction's shared memory is free
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    float* wrow = FM.w[warp][h];
+    if (lane == 0) {
+      wrow[0] = WP.m[h];
+      wrow[1] = WP.l[h];
+    }
+    *reinterpret_cast<float4*>(wrow + 4 + 4 * lane) =
+        make_float4(WP.acc[h][0], WP.acc[h][1], WP.acc[h][2], WP.acc[h][3]);
+  }
+  __syncthreads();
+  {
+    const int c = tid & (kD - 1), half = tid >> 7;
+    for (int h = half; h < G; h += 2) {
+      float m = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < kFinWarps; ++w) m = fmaxf(m, FM.w[w][h][0]);
+      float l = 0.f, a = 0.f;
+#pragma unroll
+      for (int w = 0; w < kFinWarps; ++w) {
+        const float f = FM.w[w][h][0] == -INFINITY ? 0.f : exp2f(FM.w[w][h][0] - m);
+        l = fmaf(FM.w[w][h][1], f, l);
+        a = fmaf(FM.w[w][h][4 + c], f, a);
+      }
+      P.run[h][4 + c] = a;
+      if (c == 0) {
+        P.run[h][0] = m;
+        P.run[h][1] = l;
+      }
+    }
+  }
+
+  // ---- M2: this CTA's share of the scan's split partials: per head the
+  // largest partial maximum M first, then every row's terms scaled by
+  // 2^(m_row - M) and summed; rows from the early copy, else staged a tile
   // at a time; thread (channel, half) takes heads j = half, half + 2, ...
   {
     const int c = tid & (kD - 1), half = tid >> 7;
     constexpr int kH2 = (G + 1) / 2;
     if (tid < G) s_hmax[tid] = 0u;  // key of -inf and below
-    if (early_ok) cp_async_wait<0>();
+    cp_async_wait<0>();
     __syncthreads();
     for (int gr = tid; gr < nrows; gr += kFinThreads) {
       float m, l;
@@ -994,8 +976,9 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
       lrun[i] = 0.f;
       arun[i] = 0.f;
     }
-    float* tile = reinterpret_cast<float*>(U);
-    constexpr int kTR = (int)(sizeof(FinCorr) / (kPartStride * sizeof(float))) / kMaxG * kMaxG;
+    float* tile = reinterpret_cast<float*>(U);  // the merge scratch is read: reuse it
+    constexpr int kTR = (int)(fin_union_bytes<G>() / (kPartStride * sizeof(float))) / kMaxG * kMaxG;
+    __syncthreads();
     for (int r0 = 0; r0 < nrows; r0 += (early_ok ? nrows : kTR)) {
       const int nr = early_ok ? nrows : min(kTR, nrows - r0);
       if (early_ok) {
@@ -1006,7 +989,7 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
           const int row = i / kV, v = i % kV;
           const int gr = r0 + row;
           const float* src = p.scan_part + ((size_t)(w0 + s0 + gr / G + seg) * G + gr % G) * kPartStride;
-          reinterpret_cast<float4*>(tile + row * kPartStride)[v] = ld16<float4>(src + 4 * v);
+          reinterpret_cast<float4*>(tile + row * kPartStride)[v] = *reinterpret_cast<const float4*>(src + 4 * v);
         }
         __syncthreads();
       }
@@ -1038,62 +1021,9 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
       }
     }
   }
-  // ---- P4: correction of this CTA's tail slots r, r + C, ... and an even
-  // share of the chosen set: the token list first (compacted, in shared
-  // memory), then batches of 16 tokens
-  {
-    const int n_x = select ? k : (SELECT ? nq : k);  // positions of the chosen sequence
-    const int per = (n_x + C - 1) / C;
-    const int x0 = min(n_x, r * per), x1 = min(n_x, x0 + per);
-    const int n_tail = p.tail > r ? (p.tail - r + C - 1) / C : 0;
-#pragma unroll 1
-    for (int xr = x0, first = 1; first || xr < x1; xr += kTokCap, first = 0) {
-    const int xe = min(x1, xr + kTokCap);
-    uint32_t base = 0;
-    if (first) {
-      for (int i = tid; i < n_tail; i += kFinThreads) FC.tok[i] = (1 << 30) | (r + C * i);
-      base = (uint32_t)n_tail;
-    }
-#pragma unroll 1
-    for (int xb = xr; xb < xe; xb += kFinThreads) {
-      const int j = xb + tid;
-      int t = -1;
-      if (j < xe) {
-        if (select) {
-          if ((uint32_t)j < s_pre[C]) {
-            int q = 0;
-            while (q + 1 < C && s_pre[q + 1] <= (uint32_t)j) ++q;
-            t = (int)list_of(q)[j - s_pre[q]];
-          } else {
-            t = (int)PS.chtie[j - s_pre[C]];
-          }
-        } else if (SELECT) {
-          t = j;
-        } else {
-          t = p.idx_in[(size_t)seg * k + j];
-          if (t < -1 || t >= nq) {
-            set_flag(p.flag, JFA_DEVERR_BAD_INDEX);
-            t = -1;
-          }
-        }
-      }
-      uint32_t tot;
-      const uint32_t pos = base + block_prefix_excl(t >= 0 ? 1u : 0u, scratch, &tot);
-      if (t >= 0) FC.tok[pos] = t;
-      base += tot;
-    }
-    __syncthreads();
-    const int n = (int)base;
-    for (int i = tid; i < n * 4; i += kFinThreads)  // the exact rows into L2
-      prefetch_part(p, seg, FC.tok[i >> 2], i & 3);
-    const int32_t* tl = FC.tok;
-    auto chosen_at = [&](int i) { return tl[i]; };
-    batch_correct<G, KB, VB>(p, seg, chosen_at, n, FC.b, P, q2, qb);
-    }
-  }
   cl.sync();
 
-  // ---- P5b: CTA r owns heads j = r, r + C, ...: merge the C CTAs' scan
+  // ---- M3: CTA r owns heads j = r, r + C, ...: merge the C CTAs' scan
   // partials (m_a, l_a, a_a) and exact-minus-removed partials (m_c, l_c, a_c),
   // remote loads issued together, and write
   //   out = (a_c 2^(m_c-m) + a_a 2^(m_a-m)) / (l_c 2^(m_c-m) + l_a 2^(m_a-m))

@@ -15,8 +15,9 @@ struct FinishParams {
   const uint16_t* q;
   const float* scores;     // [n_seg][capacity]
   const float* scan_part;  // per scan warp and segment: [slot][G][kPartStride]
-  const float* m_used;     // [n_seg][ng_cap][16]: the scan's running maxima and biases
-  uint32_t* hist;          // [n_seg][kScanHistBins], zeroed here after use
+  const float* m_used;     // [n_seg][ng_cap][8]: the scan's running maxima
+  const uint32_t* wts;     // the scan's fp16 weights, [n_seg][ng_cap][4][NT][32] words
+  uint32_t* hist;          // [n_seg][kScanHistStride] (bins, largest key), zeroed here after use
   uint32_t* glists;        // [n_seg][C][slice] chosen lists of the fallback
   const int32_t* idx_in;   // given index sets (no selection), [n_seg][k]
   int32_t* idx_out;        // [n_seg][k] (selection)

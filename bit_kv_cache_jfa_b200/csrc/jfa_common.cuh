@@ -24,8 +24,9 @@ constexpr int kMaxScanWarps = 4096;      // cap on scan warps (partial slots)
 constexpr int kFinMaxCluster = 16;       // CTAs per (sequence, KV head) in the finishing kernel
 constexpr int kScanMinRecords = 2;       // records per scan warp at least (when the
                                          // work allows): fewer partials to merge
-constexpr int kScanHistBits = 13;        // selection-score histogram of the scan: top 13 key bits
+constexpr int kScanHistBits = 15;        // selection-score histogram of the scan: top 15 key bits
 constexpr int kScanHistBins = 1 << kScanHistBits;
+constexpr int kScanHistStride = kScanHistBins + 32;  // per segment: the bins, then the largest key
 constexpr int kHistBins = 2048;          // top-k first-level histogram (11 key bits)
 constexpr int kCtrStride = 8;            // top-k counters per segment: [0] scan warps done, [2] b*, [3] keys above b*
 

@@ -15,10 +15,11 @@
 // B = fp16(p) * s_v (columns = heads; the weights move from the QK output
 // layout to this operand layout by two shuffles per 16 tokens), plus a small
 // MMA whose A rows are the value zeros of the four channel groups and a row
-// of ones (giving sum p).  The running maximum each group's weights were
-// taken against is stored (m_used), so the correction step recomputes
-// exactly these fp16 weights for the top-k tokens and removes their terms
-// without a rounding residue.
+// of ones (giving sum p).  The fp16 weights p themselves (one coalesced
+// 32-bit store per lane and m-tile) and the running maximum each group's
+// weights were taken against (m_used) are stored, so the correction step
+// removes exactly these terms for the top-k tokens, without a rounding
+// residue.
 //
 // Also written per token: the selection score S_t = max over the G heads
 // (natural-log units), and a per-segment histogram of its top 13 key bits
@@ -39,8 +40,9 @@ struct ScanParams {
   const uint16_t* q;
   float* scores;
   float* partials;
-  float* m_used;    // [n_seg][ng_cap][16]: running maxima (8) and biases (8) per head
-  uint32_t* hist;   // [n_seg][kScanHistBins]
+  float* m_used;    // [n_seg][ng_cap][8]: running maxima per head
+  uint32_t* wts;    // [n_seg][ng_cap][4][NT][32]: the fp16 weights, lane order
+  uint32_t* hist;   // [n_seg][kScanHistStride]: bins, then the largest key
   uint32_t* flag;
   long long total;  // n_seg * ng
   int ng, ng_cap, capacity;
@@ -308,16 +310,11 @@ __global__ void __launch_bounds__(ScanCfg<KB, VB, NT>::NW * 32, 1) scan_kernel(c
 #pragma unroll
       for (int n = 0; n < NT; ++n) m_run[n] = m_new[n];
     }
-    // the maximum this group's weights are taken against, and the group's bias
-    // (kappa * q . m), for the correction's replay
+    // the maximum this group's weights are taken against, for the correction
     if (gid == 0) {
 #pragma unroll
       for (int n = 0; n < NT; ++n)
-        if (hv[n]) {
-          float* mrec = p.m_used + ((size_t)seg * p.ng_cap + g) * (2 * kMaxG);
-          mrec[tig + 4 * n] = m_run[n];
-          mrec[kMaxG + tig + 4 * n] = bk[n];
-        }
+        if (hv[n]) p.m_used[((size_t)seg * p.ng_cap + g) * kMaxG + tig + 4 * n] = m_run[n];
     }
 
     // ---- selection score S = max over heads; lane ends with m-tile tig,
@@ -353,18 +350,27 @@ __global__ void __launch_bounds__(ScanCfg<KB, VB, NT>::NW * 32, 1) scan_kernel(c
       float* srow = p.scores + (size_t)seg * p.capacity + (size_t)g * kKG + 16 * tig + gid;
       srow[0] = sc[0];
       srow[8] = sc[1];
-      uint32_t* hs = p.hist + (size_t)seg * kScanHistBins;
-      atomicAdd(hs + (float_key(sc[0]) >> (32 - kScanHistBits)), 1u);
-      atomicAdd(hs + (float_key(sc[1]) >> (32 - kScanHistBits)), 1u);
+      uint32_t* hs = p.hist + (size_t)seg * kScanHistStride;
+      const uint32_t k0 = float_key(sc[0]), k1 = float_key(sc[1]);
+      atomicAdd(hs + (k0 >> (32 - kScanHistBits)), 1u);
+      atomicAdd(hs + (k1 >> (32 - kScanHistBits)), 1u);
+      // the segment's largest key: where the finishing kernel starts its
+      // search for the k-th largest
+      const uint32_t kmax = __reduce_max_sync(kFull, max(k0, k1));
+      if (lane == 0) atomicMax(hs + kScanHistBins, kmax);
     }
 
-    // ---- weights fp16(2^(u - m)) packed per m-tile: (token gid, token gid + 8)
+    // ---- weights fp16(2^(u - m)) packed per m-tile: (token gid, token gid + 8),
+    // stored as they are (word (mt, n) of the lane) for the correction
     uint32_t X[4][NT];
+    uint32_t* wrec = p.wts + ((size_t)seg * p.ng_cap + g) * (4 * NT * 32) + lane;
 #pragma unroll
     for (int mt = 0; mt < 4; ++mt)
 #pragma unroll
-      for (int n = 0; n < NT; ++n)
+      for (int n = 0; n < NT; ++n) {
         X[mt][n] = pack_h2(approx_weight(u[mt][n][0], m_run[n]), approx_weight(u[mt][n][1], m_run[n]));
+        wrec[(mt * NT + n) * 32] = X[mt][n];
+      }
 
     // ---- value aggregate: acc^T[c][h] += sum_t v'[t][c] * fp16(p[t][h] s_v[t][j]) ----
     const int src0 = (2 * tig) * 4 + (gid & 3), src1 = (2 * tig + 1) * 4 + (gid & 3);
@@ -444,7 +450,10 @@ __global__ void __launch_bounds__(ScanCfg<KB, VB, NT>::NW * 32, 1) scan_kernel(c
   if (has_work && !failed) flush(cur);
 
   // No explicit launch_dependents: the dependent kernel is released as the
-  // scan's CTAs exit, so its thread-block clusters find whole SMs free.
+  // scan's CTAs exit, so its thread-block clusters find whole SMs free (an
+  // early release measured slower: clusters placed beside the last scan CTAs
+  // left some of them a second wave).
+
 }
 
 template <int KB, int VB, int NT>
@@ -480,6 +489,7 @@ int launch_scores(const jfa_geom& g, const jfa_cache& c, const uint16_t* q, floa
   sp.scores = reinterpret_cast<float*>(ws + L.off_scores);
   sp.partials = reinterpret_cast<float*>(ws + L.off_partials);
   sp.m_used = reinterpret_cast<float*>(ws + L.off_mused);
+  sp.wts = reinterpret_cast<uint32_t*>(ws + L.off_wts);
   sp.hist = reinterpret_cast<uint32_t*>(ws + L.off_scan_hist);
   sp.flag = reinterpret_cast<uint32_t*>(ws + L.off_flag);
   sp.total = plan.total_groups;

@@ -107,13 +107,16 @@ typedef struct jfa_workspace_layout {
   size_t off_flag;       /* uint32 device error flag                          */
   size_t off_scores;     /* fp32 [B][H_kv][capacity]: selection score S_t     */
   size_t off_partials;   /* fp32 split partials of the approximate scan       */
-  size_t off_mused;      /* fp32 [B][H_kv][capacity/64][16]: per key group,
-                            for each query head the running maximum the
-                            scan's weights were taken against (8) and the
-                            group's bias scale*q.m (8)                       */
-  size_t off_scan_hist;  /* uint32 [B][H_kv][8192]: histogram of the top 13
-                            bits of the selection keys, built by the scan and
-                            cleared by the finishing kernel                   */
+  size_t off_mused;      /* fp32 [B][H_kv][capacity/64][8]: per key group, for
+                            each query head the running maximum the scan's
+                            weights were taken against                       */
+  size_t off_wts;        /* the scan's fp16 softmax weights of every quantized
+                            token and query head, in a layout private to
+                            this library (read by the correction)            */
+  size_t off_scan_hist;  /* uint32 [B][H_kv][32768 + 32]: histogram of the top
+                            15 bits of the selection keys, then the largest
+                            key, built by the scan and cleared by the
+                            finishing kernel                                  */
   size_t off_hist;       /* top-k histograms (jfa_topk)                       */
   size_t off_counters;   /* top-k counters (jfa_topk)                         */
   size_t off_cand;       /* top-k candidate lists                             */

@@ -62,8 +62,8 @@ def test_workspace_layout(lib):
     b = lib.jfa_workspace_layout_get(G(), 4096)
     assert b.total_bytes >= a.total_bytes and b.max_topk == 4096
     for L in (a, b):
-        offs = [L.off_flag, L.off_scores, L.off_partials, L.off_mused, L.off_scan_hist,
-                L.off_hist, L.off_cand, L.off_sel]
+        offs = [L.off_flag, L.off_scores, L.off_partials, L.off_mused, L.off_wts,
+                L.off_scan_hist, L.off_hist, L.off_cand, L.off_sel]
         assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
         assert L.off_counters == L.off_hist + 4 * 4 * 2048
         assert L.off_scores + 4 * 4 * 4096 <= L.off_partials
