@@ -2,29 +2,29 @@
 // cluster of C CTAs (C <= 16) per (sequence, KV head); CTA r owns slice r of
 // the quantized tokens and the tail slots r, r + C, ...
 //
-//   S1  reads the scan's 8192-bin histogram of the selection keys and finds
-//       the bin b* holding the k-th largest key (every CTA, redundantly);
-//   S2  lists its slice's keys above b* ("sure": chosen whatever the ties
-//       decide) and in b* ("ties"), in index order, and arrives on a
-//       cluster barrier;
-//   A   corrects its tail slots and its sure tokens while the other CTAs
-//       reach the barrier: every warp takes its own tokens, stages their
-//       record pieces and exact rows, and folds them into a running fp32
-//       softmax partial per query head (exact bf16 term in, the scan's
-//       approximate term out: the fp16 weights the scan stored, against the
+//   T   corrects its tail slots while the histogram's first load is in
+//       flight.  A correction folds a token into the warp's running fp32
+//       softmax partial per query head: its exact bf16 term in, the scan's
+//       approximate term out (the fp16 weights the scan stored, against the
 //       running maximum it stored, times the dequantized value);
-//   S3  waits on the barrier, gathers every CTA's ties and ranks them (larger
-//       key first, equal keys to the lower index);
-//   B   corrects the chosen ties of its slice into the same partials and
-//       writes its chosen indices, ascending, at its offset of idx;
+//   S1  reads a window of the scan's 32768-bin histogram of the selection
+//       keys below the segment's largest key and finds the bin b* holding
+//       the k-th largest key (every CTA, redundantly);
+//   S2  lists its slice's keys above b* ("sure": chosen whatever the ties
+//       decide) and in b* ("ties"), in index order;
+//   S3  after a cluster barrier, gathers every CTA's ties and ranks them
+//       (larger key first, equal keys to the lower index);
+//   C   corrects an even share of the chosen set (the CTAs' sure lists read
+//       through distributed shared memory, then the chosen ties) and writes
+//       its slice's chosen indices, ascending, at its offset of idx;
 //   M   merges its warps' partials and its share of the scan's split
 //       partials; the CTAs owning a query head combine the C CTAs' partials
 //       (distributed shared memory) in log-sum-exp form and write out.
 // With a given index set (jfa_correct_merge) or k >= N_q there is no
-// selection: A corrects the CTA's even share of the set.  If the histogram is
-// stale or a list overflows, every CTA selects over the whole segment from
-// the stored scores instead and the correction restarts on that set (slower,
-// same result).
+// selection: C corrects the CTA's even share of the set.  If the histogram
+// does not hold the k-th key where the stored scores put it, or a list
+// overflows, every CTA selects over the whole segment from the stored scores
+// instead (slower, same result).
 #pragma once
 
 #include <cooperative_groups.h>
@@ -254,15 +254,6 @@ __device__ __forceinline__ uint32_t lower_bound_u32(const uint32_t* a, uint32_t 
   return lo;
 }
 
-// Split cluster barrier: arrive (release: this CTA's shared-memory writes
-// become visible to the cluster) and wait (acquire).
-__device__ __forceinline__ void cluster_arrive() {
-  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_wait() {
-  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
 // ---------------------------------------------------------------------------
 // Correction.  Token encoding: t in [0, nq) a quantized token,
 // (1 << 30) | s the tail slot s (exact rows only); -1 none.
@@ -338,19 +329,23 @@ __device__ __forceinline__ void prefetch_token(const FinishParams& p, int seg, i
 }
 
 // A warp's running softmax partial per query head over the tokens it
-// corrected: frame m (log2 units, uniform over the lanes), mass l and the
-// lane's 4 channels of acc; exact terms enter with +, the scan's
-// approximate terms of the same tokens with -.
+// corrected: frame m (log2 units, uniform over the lanes) and the lane's 4
+// channels of acc; exact terms enter with +, the scan's approximate terms of
+// the same tokens with -.  The scalars of (head, value group) are spread over
+// the lanes: lane L keeps, for its pair (h, j) = ((L mod 4GP) / 4, L mod 4),
+// the mass l of head h (used from the lanes with j = 0) and the sum of the
+// removed zero-point terms of head h and group j (subtracted from the
+// channels of group j at the end).
 template <int G>
 struct WarpPart {
-  float m[G], l[G], acc[G][4];
+  float m[G], acc[G][4], lsum, zsum;
   __device__ __forceinline__ void init() {
 #pragma unroll
     for (int h = 0; h < G; ++h) {
       m[h] = -INFINITY;
-      l[h] = 0.f;
       acc[h][0] = acc[h][1] = acc[h][2] = acc[h][3] = 0.f;
     }
+    lsum = zsum = 0.f;
   }
 };
 
@@ -449,6 +444,7 @@ __device__ __forceinline__ void warp_correct(const FinishParams& p, int seg, con
 #pragma unroll
       for (int h = 0; h < G; ++h) se[u][h] = se_of(u, h);
     // ---- pass 2: frame moves (the chunk's largest term per head), then terms
+    const int pair = lane & (4 * GP - 1), ph = pair >> 2, pj = pair & 3;
 #pragma unroll
     for (int h = 0; h < G; ++h) {
       float top = -INFINITY;
@@ -459,36 +455,54 @@ __device__ __forceinline__ void warp_correct(const FinishParams& p, int seg, con
       }
       if (top > WP.m[h] + 8.f) {  // move the frame (0 while the partial is empty)
         const float al = exp2f(WP.m[h] - top);
-        WP.l[h] *= al;
         WP.acc[h][0] *= al;
         WP.acc[h][1] *= al;
         WP.acc[h][2] *= al;
         WP.acc[h][3] *= al;
+        if (ph == h) {
+          WP.lsum *= al;
+          WP.zsum *= al;
+        }
         WP.m[h] = top;
       }
     }
+    // the frame and logits of the lane's pair head ph
+    float mph = WP.m[0];
+#pragma unroll
+    for (int h = 1; h < G; ++h) mph = ph == h ? WP.m[h] : mph;
 #pragma unroll
     for (int u = 0; u < NC; ++u) {
       const int t = tk[u];
       if (t == -1) continue;  // warp-uniform
       const bool quant = tok_quant(t);
       const TokPieces& S = FW.ring[warp][u];
+      const int tt = quant ? t % kKG : 0, hi8 = (tt & 15) >> 3, e = tt & 1;
+      // pair scalars (head ph, value group pj): exact weight pe, and for a
+      // quantized token the removed value weight A = f fp16(p s_v) and
+      // zero-point term f p m_v, f = 2^(m_used - m) moving the scan's frame
+      float seh = se[u][0];
+#pragma unroll
+      for (int h = 1; h < G; ++h) seh = ph == h ? se[u][h] : seh;
+      float pe = 0.f, A = 0.f;
+      if (ph < G) {
+        pe = exp2f(seh - mph);
+        float dl = pe;
+        if (quant) {
+          const uint16_t pb = reinterpret_cast<const uint16_t*>(S.w)[2 * (4 * (ph >> 2) + (ph & 3)) + hi8];
+          const float f = exp2f(S.mu[ph] - mph);
+          const uint16_t vsc = *reinterpret_cast<const uint16_t*>(S.vsz + pj * 8 + hi8 * 4 + 2 * e);
+          const float vz = h2f(*reinterpret_cast<const uint16_t*>(S.vsz + 32 + pj * 8 + hi8 * 4 + 2 * e));
+          const float pw = h2f(pb);
+          A = f * h2f(h_mul_rn(pb, vsc));
+          WP.zsum = fmaf(f * pw, vz, WP.zsum);
+          dl = fmaf(-f, pw, dl);
+        }
+        WP.lsum += dl;
+      }
       const float v0 = __uint_as_float(vr[u].x << 16), v1 = __uint_as_float(vr[u].x & 0xFFFF0000u);
       const float v2 = __uint_as_float(vr[u].y << 16), v3 = __uint_as_float(vr[u].y & 0xFFFF0000u);
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const float pe = exp2f(se[u][h] - WP.m[h]);
-        WP.l[h] += pe;
-        WP.acc[h][0] = fmaf(pe, v0, WP.acc[h][0]);
-        WP.acc[h][1] = fmaf(pe, v1, WP.acc[h][1]);
-        WP.acc[h][2] = fmaf(pe, v2, WP.acc[h][2]);
-        WP.acc[h][3] = fmaf(pe, v3, WP.acc[h][3]);
-      }
-      if (quant) {
-        // removal operands: the value codes of the lane's channels, the
-        // value scale and zero of its channel group
-        const int tt = t % kKG, hi8 = (tt & 15) >> 3, e = tt & 1;
-        float code[4];
+      float code[4] = {0.f, 0.f, 0.f, 0.f};
+      if (quant) {  // the value codes of the lane's channels
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int gc = gbase + i;
@@ -503,24 +517,16 @@ __device__ __forceinline__ void warp_correct(const FinishParams& p, int seg, con
           }
           code[i] = (float)c;
         }
-        const uint16_t vsc = *reinterpret_cast<const uint16_t*>(S.vsz + vj * 8 + hi8 * 4 + 2 * e);
-        const float vz = h2f(*reinterpret_cast<const uint16_t*>(S.vsz + 32 + vj * 8 + hi8 * 4 + 2 * e));
+      }
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
-          // the scan added fp16(p) to the mass, fp16(p) * m_v and
-          // fp16(fp16(p) * s_v) * code to the channels, against m_used
-          const uint16_t phb =
-              reinterpret_cast<const uint16_t*>(S.w)[2 * (4 * (h >> 2) + (h & 3)) + ((tt & 15) >> 3)];
-          const float f = exp2f(S.mu[h] - WP.m[h]);
-          const float pw = h2f(phb);
-          const float wv = h2f(h_mul_rn(phb, vsc));
-          const float pz = pw * vz;
-          WP.l[h] = fmaf(-f, pw, WP.l[h]);
-          WP.acc[h][0] = fmaf(-f, fmaf(wv, code[0], pz), WP.acc[h][0]);
-          WP.acc[h][1] = fmaf(-f, fmaf(wv, code[1], pz), WP.acc[h][1]);
-          WP.acc[h][2] = fmaf(-f, fmaf(wv, code[2], pz), WP.acc[h][2]);
-          WP.acc[h][3] = fmaf(-f, fmaf(wv, code[3], pz), WP.acc[h][3]);
-        }
+      for (int h = 0; h < G; ++h) {
+        // head h's scalars for the lane's value group vj: lane 4h + vj
+        const float peh = __shfl_sync(kAll, pe, 4 * h + vj);
+        const float Ah = __shfl_sync(kAll, A, 4 * h + vj);
+        WP.acc[h][0] = fmaf(-Ah, code[0], fmaf(peh, v0, WP.acc[h][0]));
+        WP.acc[h][1] = fmaf(-Ah, code[1], fmaf(peh, v1, WP.acc[h][1]));
+        WP.acc[h][2] = fmaf(-Ah, code[2], fmaf(peh, v2, WP.acc[h][2]));
+        WP.acc[h][3] = fmaf(-Ah, code[3], fmaf(peh, v3, WP.acc[h][3]));
       }
     }
     __syncwarp();  // the ring is reused by the next chunk
@@ -546,12 +552,13 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
   __shared__ int s_mode;                     // 0 lists in shared memory, 1 fallback lists
   __shared__ uint32_t s_hmax[kMaxG];          // per head: largest scan-partial maximum (key)
   __shared__ uint32_t s_tie[kFinMaxC], s_ovf[kFinMaxC];
+  __shared__ __align__(8) uint64_t s_early_bar;  // completion of the early copy below
 
   cg::cluster_group cl = cg::this_cluster();
   const int C = (int)cl.num_blocks();
   const int r = (int)cl.block_rank();
   const int seg = blockIdx.x / C;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gid = lane >> 2, tig = lane & 3;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nq = p.nq, k = p.k;
   const int bb = seg / p.hkv, hh = seg % p.hkv;
 
@@ -565,14 +572,17 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
     const uint16_t b = p.q[((size_t)bb * p.H + (size_t)hh * G) * kD + i];
     qf[i] = __uint_as_float((uint32_t)b << 16);
   }
+  if (tid == 0) {  // initialised before any thread can wait on it
+    mbar_init(&s_early_bar, 1);
+    fence_mbar_init();
+  }
   __syncthreads();
 
   pdl_wait();
   pdl_launch_dependents();
 
   // ---- early copy of this CTA's share of the scan's split partials, every
-  // head: when the rows fit they are copied now (cp.async) and merged at the
-  // end, so their latency hides behind the selection and the correction
+  // head, when the rows fit (else they are staged a tile at a time below)
   long long w0 = 0, w1 = -1;
   if (p.ng > 0) {
     const long long T = p.scan_total, W = p.scan_warps;
@@ -586,22 +596,109 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
   const int nrows = (s1 - s0) * G;
   constexpr int kEarlyRows = (int)(kEarlyBytes / (kPartStride * sizeof(float)));
   const bool early_ok = nrows <= kEarlyRows;
-  if (early_ok) {
-    for (int i = tid; i < nrows * kV; i += kFinThreads) {
-      const int row = i / kV, v = i % kV;
-      cp_async16(early + row * kPartStride + 4 * v,
-                 p.scan_part + ((size_t)(w0 + s0 + row / G + seg) * G + row % G) * kPartStride + 4 * v);
-    }
+  // the rows (slot, head) are consecutive in the workspace: one bulk copy,
+  // completing on an mbarrier (independent of the warps' cp.async groups)
+  if (early_ok && nrows > 0 && tid == 0) {
+    const uint32_t bytes = (uint32_t)(nrows * kPartStride * sizeof(float));
+    mbar_expect_tx(&s_early_bar, bytes);
+    bulk_g2s_nohint(early, p.scan_part + ((size_t)(w0 + s0 + seg) * G) * kPartStride, bytes, &s_early_bar);
   }
-  cp_async_commit();
 
   const bool select = SELECT && k < nq;
   const int lo = min(nq, r * p.slice), hi = min(nq, lo + p.slice);
-  bool hist_ok = false;
+  const uint32_t* hg = p.hist + (size_t)seg * kScanHistStride;
+  // the segment's largest selection key: requested now, used after the merge
+  // of the scan partials below
+  const uint32_t top_key = select ? hg[kScanHistBins] : 0u;
+
+  WarpPart<G> WP;
+  WP.init();
+
+  // ---- M: this CTA's share of the scan's split partials: per head the
+  // largest partial maximum M first, then every row's terms scaled by
+  // 2^(m_row - M) and summed; rows from the early copy, else staged a tile
+  // at a time; thread (channel, half) takes heads j = half, half + 2, ...
+  {
+    const int c = tid & (kD - 1), half = tid >> 7;
+    constexpr int kH2 = (G + 1) / 2;
+    if (tid < G) s_hmax[tid] = 0u;  // key of -inf and below
+    if (early_ok && nrows > 0 && !mbar_wait_bounded(&s_early_bar, 0u)) {
+      if (tid == 0) set_flag(p.flag, JFA_DEVERR_TIMEOUT);
+      mbar_wait_bounded(&s_early_bar, 0u);  // the copy in flight, once more (bounded)
+    }
+    __syncthreads();
+    for (int gr = tid; gr < nrows; gr += kFinThreads) {
+      float m, l;
+      if (early_ok) {
+        m = early[gr * kPartStride];
+        l = early[gr * kPartStride + 1];
+      } else {
+        const float* src = p.scan_part + ((size_t)(w0 + s0 + gr / G + seg) * G + gr % G) * kPartStride;
+        m = src[0];
+        l = src[1];
+      }
+      if (l > 0.f) atomicMax(&s_hmax[gr % G], float_key(m));
+    }
+    __syncthreads();
+    float mh[kH2], lrun[kH2], arun[kH2];
+#pragma unroll
+    for (int i = 0; i < kH2; ++i) {
+      const int j = half + 2 * i;
+      mh[i] = j < G && s_hmax[j] != 0u ? key_float(s_hmax[j]) : -INFINITY;
+      lrun[i] = 0.f;
+      arun[i] = 0.f;
+    }
+    float* tile = reinterpret_cast<float*>(U);  // the correction's buffers are not in use yet
+    constexpr int kTR = (int)(fin_union_bytes<G>() / (kPartStride * sizeof(float))) / kMaxG * kMaxG;
+    __syncthreads();
+    for (int r0 = 0; r0 < nrows; r0 += (early_ok ? nrows : kTR)) {
+      const int nr = early_ok ? nrows : min(kTR, nrows - r0);
+      if (early_ok) {
+        tile = early;
+      } else {
+#pragma unroll 8
+        for (int i = tid; i < nr * kV; i += kFinThreads) {
+          const int row = i / kV, v = i % kV;
+          const int gr = r0 + row;
+          const float* src = p.scan_part + ((size_t)(w0 + s0 + gr / G + seg) * G + gr % G) * kPartStride;
+          reinterpret_cast<float4*>(tile + row * kPartStride)[v] = *reinterpret_cast<const float4*>(src + 4 * v);
+        }
+        __syncthreads();
+      }
+#pragma unroll
+      for (int i = 0; i < kH2; ++i) {
+        const int j = half + 2 * i;
+        if (j < G) {
+#pragma unroll 4
+          for (int row = (j - r0 % G + G) % G; row < nr; row += G) {
+            const float* tr = tile + row * kPartStride;
+            const float rl = tr[1];
+            const float f = rl > 0.f ? exp2f(tr[0] - mh[i]) : 0.f;
+            lrun[i] = fmaf(rl, f, lrun[i]);
+            arun[i] = fmaf(tr[4 + c], f, arun[i]);
+          }
+        }
+      }
+      if (!early_ok) __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < kH2; ++i) {
+      const int j = half + 2 * i;
+      if (j < G) {
+        P.sp[j][4 + c] = arun[i];
+        if (c == 0) {
+          P.sp[j][0] = lrun[i] > 0.f ? mh[i] : -INFINITY;
+          P.sp[j][1] = lrun[i];
+        }
+      }
+    }
+  }
+
   // ---- S1 + S2: bin b* from the scan's histogram, then this slice's lists
+  bool hist_ok = false;
   if (select) {
     // the slice's first 16 scores of this thread, loaded together with the
-    // histogram so both round trips overlap
+    // histogram window so both round trips overlap
     const float* S = p.scores + (size_t)seg * p.capacity;
     float4 v0[4];
 #pragma unroll
@@ -612,8 +709,7 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
     // the bin holding the k-th largest key: a window of 1024 bins below the
     // segment's largest key (thread t owns 4 bins), then further windows
     // down while the keys counted so far are fewer than k
-    const uint32_t* hg = p.hist + (size_t)seg * kScanHistStride;
-    const int top = (int)(hg[kScanHistBins] >> (32 - kScanHistBits));
+    const int top = (int)(top_key >> (32 - kScanHistBits));
     int whi = min(kScanHistBins, (top | 3) + 1);
     uint32_t above = 0;  // keys in the bins above the current window
 #pragma unroll 1
@@ -665,7 +761,6 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
             const bool in = b0 + i < hi;
             const uint32_t bin = keys[i] >> (32 - kScanHistBits);
             const bool su = in && bin > bstar, ti = in && bin == bstar;
-            if (su) prefetch_token<KB, VB, (G > 4 ? 2 : 1)>(p, seg, b0 + i);
             ms |= (su ? 1u : 0u) << i;
             mtie |= (ti ? 1u : 0u) << i;
             nsu += su;
@@ -698,77 +793,19 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
       PS.n_tie = base_t;
       PS.overflow = (base_s > (uint32_t)kLCap || base_t > (uint32_t)kLCap) ? 1u : 0u;
     }
-    __syncthreads();
-    cluster_arrive();  // lists and counts are visible to the cluster
+    cl.sync();  // every CTA's lists and counts are complete
   }
 
-  // ---- A: correct the tail slots and, when the lists hold, the sure tokens
-  // of the slice (or the CTA's share of a given / complete index set)
-  WarpPart<G> WP;
-  WP.init();
-  const int n_tail = p.tail > r ? (p.tail - r + C - 1) / C : 0;
-  if (select) {
-    const uint32_t ns_me = hist_ok && PS.overflow == 0u ? PS.n_sure : 0u;
-    for (int i = tid; i < n_tail; i += kFinThreads) tok[i] = (1 << 30) | (r + C * i);
-    // the sure list in chunks of kTokCap (beside the tail slots)
-#pragma unroll 1
-    for (uint32_t c0 = 0, first = 1; first || c0 < ns_me; c0 += kTokCap, first = 0) {
-      const int base = first ? n_tail : 0;
-      const uint32_t cn = min((uint32_t)kTokCap, ns_me - min(ns_me, c0));
-      for (uint32_t i = tid; i < cn; i += kFinThreads) tok[base + i] = (int32_t)PS.sure[c0 + i];
-      __syncthreads();
-      warp_correct<G, KB, VB>(p, seg, tok, base + (int)cn, FW, qf, WP);
-      __syncthreads();
-    }
-  } else {
-    // positions [x0, x1) of the set: idx_in entries, or every quantized token
-    const int n_x = SELECT ? nq : k;
-    const int per = (n_x + C - 1) / C;
-    const int x0 = min(n_x, r * per), x1 = min(n_x, x0 + per);
-#pragma unroll 1
-    for (int xr = x0, first = 1; first || xr < x1; xr += kTokCap, first = 0) {
-      const int xe = min(x1, xr + kTokCap);
-      uint32_t base = 0;
-      if (first) {
-        for (int i = tid; i < n_tail; i += kFinThreads) tok[i] = (1 << 30) | (r + C * i);
-        base = (uint32_t)n_tail;
-      }
-#pragma unroll 1
-      for (int xb = xr; xb < xe; xb += kFinThreads) {
-        const int j = xb + tid;
-        int t = -1;
-        if (j < xe) {
-          if (SELECT) {
-            t = j;
-          } else {
-            t = p.idx_in[(size_t)seg * k + j];
-            if (t < -1 || t >= nq) {
-              set_flag(p.flag, JFA_DEVERR_BAD_INDEX);
-              t = -1;
-            }
-          }
-        }
-        uint32_t tot;
-        const uint32_t pos = base + block_prefix_excl(t >= 0 ? 1u : 0u, scratch, &tot);
-        if (t >= 0) tok[pos] = t;
-        base += tot;
-      }
-      __syncthreads();
-      warp_correct<G, KB, VB>(p, seg, tok, (int)base, FW, qf, WP);
-      __syncthreads();
-    }
-  }
-
-  // ---- S3 + B: resolve the selection, correct the chosen ties of the slice
-  uint32_t n_ch = 0;  // chosen ties (ascending in PS.chtie)
+  // ---- S3: resolve the selection; every CTA learns the whole chosen set:
+  // the CTAs' sure lists (in CTA order) and the chosen ties (ascending)
+  uint32_t n_ch = 0;
   const uint32_t* glist_base = p.glists + (size_t)seg * C * p.slice;
   int mode = 0;
   if (select) {
-    cluster_wait();
     {  // the scan's histogram is consumed: clear it for the next scan
-      uint32_t* hg = p.hist + (size_t)seg * kScanHistStride;
+      uint32_t* hc = p.hist + (size_t)seg * kScanHistStride;
       for (int i = 4 * (r * kFinThreads + tid); i < kScanHistStride; i += 4 * C * kFinThreads)
-        *reinterpret_cast<uint4*>(hg + i) = make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4*>(hc + i) = make_uint4(0u, 0u, 0u, 0u);
     }
     if (tid < C) {
       const FinPersist* o = cl.map_shared_rank(&PS, tid);
@@ -838,36 +875,14 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
         s_chq[tid] = lower_bound_u32(PS.chtie, n_ch, b0);
       }
       __syncthreads();
-      // B: the chosen ties of this slice
-      const uint32_t c0 = s_chq[r], c1 = s_chq[r + 1];
-#pragma unroll 1
-      for (uint32_t cb = c0; cb < c1; cb += kTokCap) {
-        const uint32_t cn = min((uint32_t)kTokCap, c1 - cb);
-        for (uint32_t i = tid; i < cn; i += kFinThreads) tok[i] = (int32_t)PS.chtie[cb + i];
-        __syncthreads();
-        warp_correct<G, KB, VB>(p, seg, tok, (int)cn, FW, qf, WP);
-        __syncthreads();
-      }
     } else {
-      // fallback: select over the whole segment; the correction restarts on
-      // the tail slots and this slice's chosen tokens
+      // fallback: select over the whole segment; each CTA lists its slice's
+      // chosen indices in global memory
       uint32_t* gl = const_cast<uint32_t*>(glist_base) + (size_t)r * p.slice;
       const uint32_t n = select_full(p.scores + (size_t)seg * p.capacity, nq, k, lo, hi, FW.hist, gl,
                                      scratch, &s_bin, &s_above, &s_tot);
       if (tid == 0) PS.n_gl = n;
       __threadfence();
-      WP.init();
-#pragma unroll 1
-      for (uint32_t c0 = 0, first = 1; first || c0 < n; c0 += kTokCap, first = 0) {
-        const int base = first ? n_tail : 0;
-        if (first)
-          for (int i = tid; i < n_tail; i += kFinThreads) tok[i] = (1 << 30) | (r + C * i);
-        const uint32_t cn = min((uint32_t)kTokCap, n - min(n, c0));
-        for (uint32_t i = tid; i < cn; i += kFinThreads) tok[base + i] = (int32_t)gl[c0 + i];
-        __syncthreads();
-        warp_correct<G, KB, VB>(p, seg, tok, base + (int)cn, FW, qf, WP);
-        __syncthreads();
-      }
       cl.sync();  // the fallback lists and counts are complete
       if (tid < C) s_cnt[tid] = cl.map_shared_rank(&PS, tid)->n_gl;
       __syncthreads();
@@ -879,6 +894,66 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
         }
         s_pre[C] = ps;
       }
+      __syncthreads();
+    }
+  }
+
+  // ---- C: the tail slots r, r + C, ... and an even share of the chosen set
+  // (positions [x0, x1) of: the CTAs' lists in CTA order, then the chosen
+  // ties), or of a given index set, or of every quantized token when
+  // k >= N_q; every listed token's rows and pieces are prefetched into L2 as
+  // the list is built
+  {
+    const int n_x = select ? k : (SELECT ? nq : k);
+    const int per = (n_x + C - 1) / C;
+    const int x0 = min(n_x, r * per), x1 = min(n_x, x0 + per);
+    const int n_tail = p.tail > r ? (p.tail - r + C - 1) / C : 0;
+#pragma unroll 1
+    for (int xr = x0, first = 1; first || xr < x1; xr += kTokCap, first = 0) {
+      const int xe = min(x1, xr + kTokCap);
+      uint32_t base = 0;
+      if (first) {
+        for (int i = tid; i < n_tail; i += kFinThreads) {
+          const int t = (1 << 30) | (r + C * i);
+          tok[i] = t;
+          for (int part = 0; part < 4; ++part) prefetch_part(p, seg, t, part);
+        }
+        base = (uint32_t)n_tail;
+      }
+#pragma unroll 1
+      for (int xb = xr; xb < xe; xb += kFinThreads) {
+        const int j = xb + tid;
+        int t = -1;
+        if (j < xe) {
+          if (select) {
+            if ((uint32_t)j < s_pre[C]) {
+              int q = 0;
+              while (q + 1 < C && s_pre[q + 1] <= (uint32_t)j) ++q;
+              t = (int)(mode == 1 ? glist_base[(size_t)q * p.slice + (j - s_pre[q])]
+                                  : cl.map_shared_rank(PS.sure, q)[j - s_pre[q]]);
+            } else {
+              t = (int)PS.chtie[j - s_pre[C]];
+            }
+          } else if (SELECT) {
+            t = j;
+          } else {
+            t = p.idx_in[(size_t)seg * k + j];
+            if (t < -1 || t >= nq) {
+              set_flag(p.flag, JFA_DEVERR_BAD_INDEX);
+              t = -1;
+            }
+          }
+        }
+        uint32_t tot;
+        const uint32_t pos = base + block_prefix_excl(t >= 0 ? 1u : 0u, scratch, &tot);
+        if (t >= 0) {
+          tok[pos] = t;
+          prefetch_token<KB, VB, (G > 4 ? 2 : 1)>(p, seg, t);
+        }
+        base += tot;
+      }
+      __syncthreads();
+      warp_correct<G, KB, VB>(p, seg, tok, (int)base, FW, qf, WP);
       __syncthreads();
     }
   }
@@ -915,13 +990,16 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
   __syncthreads();  // the correction's shared memory is free
 #pragma unroll
   for (int h = 0; h < G; ++h) {
+    // head h's mass from lane 4h, its zero-point sum of group j from lane 4h + j
+    const float lh = __shfl_sync(kAll, WP.lsum, 4 * h);
+    const float zh = __shfl_sync(kAll, WP.zsum, 4 * h + (lane >> 3));
     float* wrow = FM.w[warp][h];
     if (lane == 0) {
       wrow[0] = WP.m[h];
-      wrow[1] = WP.l[h];
+      wrow[1] = lh;
     }
     *reinterpret_cast<float4*>(wrow + 4 + 4 * lane) =
-        make_float4(WP.acc[h][0], WP.acc[h][1], WP.acc[h][2], WP.acc[h][3]);
+        make_float4(WP.acc[h][0] - zh, WP.acc[h][1] - zh, WP.acc[h][2] - zh, WP.acc[h][3] - zh);
   }
   __syncthreads();
   {
@@ -945,82 +1023,6 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
     }
   }
 
-  // ---- M2: this CTA's share of the scan's split partials: per head the
-  // largest partial maximum M first, then every row's terms scaled by
-  // 2^(m_row - M) and summed; rows from the early copy, else staged a tile
-  // at a time; thread (channel, half) takes heads j = half, half + 2, ...
-  {
-    const int c = tid & (kD - 1), half = tid >> 7;
-    constexpr int kH2 = (G + 1) / 2;
-    if (tid < G) s_hmax[tid] = 0u;  // key of -inf and below
-    cp_async_wait<0>();
-    __syncthreads();
-    for (int gr = tid; gr < nrows; gr += kFinThreads) {
-      float m, l;
-      if (early_ok) {
-        m = early[gr * kPartStride];
-        l = early[gr * kPartStride + 1];
-      } else {
-        const float* src = p.scan_part + ((size_t)(w0 + s0 + gr / G + seg) * G + gr % G) * kPartStride;
-        m = src[0];
-        l = src[1];
-      }
-      if (l > 0.f) atomicMax(&s_hmax[gr % G], float_key(m));
-    }
-    __syncthreads();
-    float mh[kH2], lrun[kH2], arun[kH2];
-#pragma unroll
-    for (int i = 0; i < kH2; ++i) {
-      const int j = half + 2 * i;
-      mh[i] = j < G && s_hmax[j] != 0u ? key_float(s_hmax[j]) : -INFINITY;
-      lrun[i] = 0.f;
-      arun[i] = 0.f;
-    }
-    float* tile = reinterpret_cast<float*>(U);  // the merge scratch is read: reuse it
-    constexpr int kTR = (int)(fin_union_bytes<G>() / (kPartStride * sizeof(float))) / kMaxG * kMaxG;
-    __syncthreads();
-    for (int r0 = 0; r0 < nrows; r0 += (early_ok ? nrows : kTR)) {
-      const int nr = early_ok ? nrows : min(kTR, nrows - r0);
-      if (early_ok) {
-        tile = early;
-      } else {
-#pragma unroll 8
-        for (int i = tid; i < nr * kV; i += kFinThreads) {
-          const int row = i / kV, v = i % kV;
-          const int gr = r0 + row;
-          const float* src = p.scan_part + ((size_t)(w0 + s0 + gr / G + seg) * G + gr % G) * kPartStride;
-          reinterpret_cast<float4*>(tile + row * kPartStride)[v] = *reinterpret_cast<const float4*>(src + 4 * v);
-        }
-        __syncthreads();
-      }
-#pragma unroll
-      for (int i = 0; i < kH2; ++i) {
-        const int j = half + 2 * i;
-        if (j < G) {
-#pragma unroll 4
-          for (int row = (j - r0 % G + G) % G; row < nr; row += G) {
-            const float* tr = tile + row * kPartStride;
-            const float rl = tr[1];
-            const float f = rl > 0.f ? exp2f(tr[0] - mh[i]) : 0.f;
-            lrun[i] = fmaf(rl, f, lrun[i]);
-            arun[i] = fmaf(tr[4 + c], f, arun[i]);
-          }
-        }
-      }
-      if (!early_ok) __syncthreads();
-    }
-#pragma unroll
-    for (int i = 0; i < kH2; ++i) {
-      const int j = half + 2 * i;
-      if (j < G) {
-        P.sp[j][4 + c] = arun[i];
-        if (c == 0) {
-          P.sp[j][0] = lrun[i] > 0.f ? mh[i] : -INFINITY;
-          P.sp[j][1] = lrun[i];
-        }
-      }
-    }
-  }
   cl.sync();
 
   // ---- M3: CTA r owns heads j = r, r + C, ...: merge the C CTAs' scan
