@@ -77,7 +77,7 @@ struct TokPieces {
 static_assert(sizeof(TokPieces) == 384, "token pieces layout");
 constexpr int kTokPieces16 = 24;  // 16-byte copies per token
 
-struct FinWork {                 // correction working set (phases A and B)
+struct FinWork {                 // correction working set
   TokPieces ring[kFinWarps][kChunk];
   uint32_t akey[kTCap], aidx[kTCap];      // gathered ties
   uint32_t hist[kRefBins + kRefBins / 32];
@@ -311,23 +311,6 @@ __device__ __forceinline__ void prefetch_part(const FinishParams& p, int seg, in
   prefetch_l2(base + off + 64 * (part & 1));
 }
 
-// L2 prefetch of everything the correction reads for quantized token t: its
-// exact K and V rows and its pieces (see stage_piece).
-template <int KB, int VB, int NT>
-__device__ __forceinline__ void prefetch_token(const FinishParams& p, int seg, int t) {
-  for (int part = 0; part < 4; ++part) prefetch_part(p, seg, t, part);
-  const int g = t / kKG;
-  const size_t rg = (size_t)seg * p.ng_cap + (size_t)g;
-  const uint8_t* rec = p.groups + rg * p.rec_bytes;
-  const int tt = t % kKG, kk = tt >> 4, row = tt & 7, tgt = (tt & 7) >> 1;
-  const uint8_t* vc = rec + off_vc(KB) + (VB == 4 ? 2 * kk : kk) * 512 + tgt * 16;
-  for (int i = 0; i < (VB == 4 ? 8 : 4); ++i) prefetch_l2(vc + 128 * i);
-  prefetch_l2(rec + off_vs(KB) + kk * 128 + tgt * 32);
-  prefetch_l2(rec + off_vs(KB) + 512 + kk * 128 + tgt * 32);
-  for (int n = 0; n < NT; ++n) prefetch_l2(p.wts + (rg * 4 * NT + (size_t)(kk * NT + n)) * 32 + row * 4);
-  prefetch_l2(p.m_used + rg * kMaxG);
-}
-
 // A warp's running softmax partial per query head over the tokens it
 // corrected: frame m (log2 units, uniform over the lanes) and the lane's 4
 // channels of acc; exact terms enter with +, the scan's approximate terms of
@@ -470,11 +453,12 @@ __device__ __forceinline__ void warp_correct(const FinishParams& p, int seg, con
     float mph = WP.m[0];
 #pragma unroll
     for (int h = 1; h < G; ++h) mph = ph == h ? WP.m[h] : mph;
+    // every token of the chunk in straight-line code (an empty slot or a
+    // tail token carries zero weights), so the tokens' chains interleave
 #pragma unroll
     for (int u = 0; u < NC; ++u) {
       const int t = tk[u];
-      if (t == -1) continue;  // warp-uniform
-      const bool quant = tok_quant(t);
+      const bool valid = t != -1, quant = tok_quant(t);
       const TokPieces& S = FW.ring[warp][u];
       const int tt = quant ? t % kKG : 0, hi8 = (tt & 15) >> 3, e = tt & 1;
       // pair scalars (head ph, value group pj): exact weight pe, and for a
@@ -483,40 +467,34 @@ __device__ __forceinline__ void warp_correct(const FinishParams& p, int seg, con
       float seh = se[u][0];
 #pragma unroll
       for (int h = 1; h < G; ++h) seh = ph == h ? se[u][h] : seh;
-      float pe = 0.f, A = 0.f;
-      if (ph < G) {
-        pe = exp2f(seh - mph);
-        float dl = pe;
-        if (quant) {
-          const uint16_t pb = reinterpret_cast<const uint16_t*>(S.w)[2 * (4 * (ph >> 2) + (ph & 3)) + hi8];
-          const float f = exp2f(S.mu[ph] - mph);
-          const uint16_t vsc = *reinterpret_cast<const uint16_t*>(S.vsz + pj * 8 + hi8 * 4 + 2 * e);
-          const float vz = h2f(*reinterpret_cast<const uint16_t*>(S.vsz + 32 + pj * 8 + hi8 * 4 + 2 * e));
-          const float pw = h2f(pb);
-          A = f * h2f(h_mul_rn(pb, vsc));
-          WP.zsum = fmaf(f * pw, vz, WP.zsum);
-          dl = fmaf(-f, pw, dl);
-        }
-        WP.lsum += dl;
-      }
+      const bool live = valid && ph < G, qlive = quant && ph < G;
+      const float pe = live ? exp2f(seh - mph) : 0.f;
+      const uint16_t pb = reinterpret_cast<const uint16_t*>(S.w)[2 * (4 * (ph >> 2) + (ph & 3)) + hi8];
+      const float f = qlive ? exp2f(S.mu[ph < G ? ph : 0] - mph) : 0.f;
+      const uint16_t vsc = *reinterpret_cast<const uint16_t*>(S.vsz + pj * 8 + hi8 * 4 + 2 * e);
+      const float vz = h2f(*reinterpret_cast<const uint16_t*>(S.vsz + 32 + pj * 8 + hi8 * 4 + 2 * e));
+      const float pw = qlive ? h2f(pb) : 0.f;
+      const float A = qlive ? f * h2f(h_mul_rn(pb, vsc)) : 0.f;
+      WP.zsum = qlive ? fmaf(f * pw, vz, WP.zsum) : WP.zsum;
+      WP.lsum += fmaf(-f, pw, pe);
       const float v0 = __uint_as_float(vr[u].x << 16), v1 = __uint_as_float(vr[u].x & 0xFFFF0000u);
       const float v2 = __uint_as_float(vr[u].y << 16), v3 = __uint_as_float(vr[u].y & 0xFFFF0000u);
-      float code[4] = {0.f, 0.f, 0.f, 0.f};
-      if (quant) {  // the value codes of the lane's channels
+      // the value codes of the lane's channels (meaningless, and multiplied
+      // by A = 0, unless the token is quantized)
+      float code[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int gc = gbase + i;
-          uint32_t wd, c;
-          if (VB == 4) {
-            const int w8 = 2 * (mt & 3) + hi8;
-            wd = *reinterpret_cast<const uint32_t*>(S.vp + ((w8 >> 2) * 8 + gc) * 16 + (w8 & 3) * 4);
-            c = (wd >> (vc_pos(4, mt) + 8 * chi + 16 * e)) & 15u;
-          } else {
-            wd = *reinterpret_cast<const uint32_t*>(S.vp + gc * 16 + (2 * (mt & 1) + hi8) * 4);
-            c = (wd >> (vc_pos(2, mt) + 8 * chi + 16 * e)) & 3u;
-          }
-          code[i] = (float)c;
+      for (int i = 0; i < 4; ++i) {
+        const int gc = gbase + i;
+        uint32_t wd, c;
+        if (VB == 4) {
+          const int w8 = 2 * (mt & 3) + hi8;
+          wd = *reinterpret_cast<const uint32_t*>(S.vp + ((w8 >> 2) * 8 + gc) * 16 + (w8 & 3) * 4);
+          c = (wd >> (vc_pos(4, mt) + 8 * chi + 16 * e)) & 15u;
+        } else {
+          wd = *reinterpret_cast<const uint32_t*>(S.vp + gc * 16 + (2 * (mt & 1) + hi8) * 4);
+          c = (wd >> (vc_pos(2, mt) + 8 * chi + 16 * e)) & 3u;
         }
+        code[i] = (float)c;
       }
 #pragma unroll
       for (int h = 0; h < G; ++h) {
@@ -607,92 +585,11 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
   const bool select = SELECT && k < nq;
   const int lo = min(nq, r * p.slice), hi = min(nq, lo + p.slice);
   const uint32_t* hg = p.hist + (size_t)seg * kScanHistStride;
-  // the segment's largest selection key: requested now, used after the merge
-  // of the scan partials below
+  // the segment's largest selection key
   const uint32_t top_key = select ? hg[kScanHistBins] : 0u;
 
   WarpPart<G> WP;
   WP.init();
-
-  // ---- M: this CTA's share of the scan's split partials: per head the
-  // largest partial maximum M first, then every row's terms scaled by
-  // 2^(m_row - M) and summed; rows from the early copy, else staged a tile
-  // at a time; thread (channel, half) takes heads j = half, half + 2, ...
-  {
-    const int c = tid & (kD - 1), half = tid >> 7;
-    constexpr int kH2 = (G + 1) / 2;
-    if (tid < G) s_hmax[tid] = 0u;  // key of -inf and below
-    if (early_ok && nrows > 0 && !mbar_wait_bounded(&s_early_bar, 0u)) {
-      if (tid == 0) set_flag(p.flag, JFA_DEVERR_TIMEOUT);
-      mbar_wait_bounded(&s_early_bar, 0u);  // the copy in flight, once more (bounded)
-    }
-    __syncthreads();
-    for (int gr = tid; gr < nrows; gr += kFinThreads) {
-      float m, l;
-      if (early_ok) {
-        m = early[gr * kPartStride];
-        l = early[gr * kPartStride + 1];
-      } else {
-        const float* src = p.scan_part + ((size_t)(w0 + s0 + gr / G + seg) * G + gr % G) * kPartStride;
-        m = src[0];
-        l = src[1];
-      }
-      if (l > 0.f) atomicMax(&s_hmax[gr % G], float_key(m));
-    }
-    __syncthreads();
-    float mh[kH2], lrun[kH2], arun[kH2];
-#pragma unroll
-    for (int i = 0; i < kH2; ++i) {
-      const int j = half + 2 * i;
-      mh[i] = j < G && s_hmax[j] != 0u ? key_float(s_hmax[j]) : -INFINITY;
-      lrun[i] = 0.f;
-      arun[i] = 0.f;
-    }
-    float* tile = reinterpret_cast<float*>(U);  // the correction's buffers are not in use yet
-    constexpr int kTR = (int)(fin_union_bytes<G>() / (kPartStride * sizeof(float))) / kMaxG * kMaxG;
-    __syncthreads();
-    for (int r0 = 0; r0 < nrows; r0 += (early_ok ? nrows : kTR)) {
-      const int nr = early_ok ? nrows : min(kTR, nrows - r0);
-      if (early_ok) {
-        tile = early;
-      } else {
-#pragma unroll 8
-        for (int i = tid; i < nr * kV; i += kFinThreads) {
-          const int row = i / kV, v = i % kV;
-          const int gr = r0 + row;
-          const float* src = p.scan_part + ((size_t)(w0 + s0 + gr / G + seg) * G + gr % G) * kPartStride;
-          reinterpret_cast<float4*>(tile + row * kPartStride)[v] = *reinterpret_cast<const float4*>(src + 4 * v);
-        }
-        __syncthreads();
-      }
-#pragma unroll
-      for (int i = 0; i < kH2; ++i) {
-        const int j = half + 2 * i;
-        if (j < G) {
-#pragma unroll 4
-          for (int row = (j - r0 % G + G) % G; row < nr; row += G) {
-            const float* tr = tile + row * kPartStride;
-            const float rl = tr[1];
-            const float f = rl > 0.f ? exp2f(tr[0] - mh[i]) : 0.f;
-            lrun[i] = fmaf(rl, f, lrun[i]);
-            arun[i] = fmaf(tr[4 + c], f, arun[i]);
-          }
-        }
-      }
-      if (!early_ok) __syncthreads();
-    }
-#pragma unroll
-    for (int i = 0; i < kH2; ++i) {
-      const int j = half + 2 * i;
-      if (j < G) {
-        P.sp[j][4 + c] = arun[i];
-        if (c == 0) {
-          P.sp[j][0] = lrun[i] > 0.f ? mh[i] : -INFINITY;
-          P.sp[j][1] = lrun[i];
-        }
-      }
-    }
-  }
 
   // ---- S1 + S2: bin b* from the scan's histogram, then this slice's lists
   bool hist_ok = false;
@@ -793,8 +690,89 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
       PS.n_tie = base_t;
       PS.overflow = (base_s > (uint32_t)kLCap || base_t > (uint32_t)kLCap) ? 1u : 0u;
     }
-    cl.sync();  // every CTA's lists and counts are complete
   }
+
+  // ---- M: this CTA's share of the scan's split partials: per head the
+  // largest partial maximum M first, then every row's terms scaled by
+  // 2^(m_row - M) and summed; rows from the early copy, else staged a tile
+  // at a time; thread (channel, half) takes heads j = half, half + 2, ...
+  {
+    const int c = tid & (kD - 1), half = tid >> 7;
+    constexpr int kH2 = (G + 1) / 2;
+    if (tid < G) s_hmax[tid] = 0u;  // key of -inf and below
+    if (early_ok && nrows > 0 && !mbar_wait_bounded(&s_early_bar, 0u)) {
+      if (tid == 0) set_flag(p.flag, JFA_DEVERR_TIMEOUT);
+      mbar_wait_bounded(&s_early_bar, 0u);  // the copy in flight, once more (bounded)
+    }
+    __syncthreads();
+    for (int gr = tid; gr < nrows; gr += kFinThreads) {
+      float m, l;
+      if (early_ok) {
+        m = early[gr * kPartStride];
+        l = early[gr * kPartStride + 1];
+      } else {
+        const float* src = p.scan_part + ((size_t)(w0 + s0 + gr / G + seg) * G + gr % G) * kPartStride;
+        m = src[0];
+        l = src[1];
+      }
+      if (l > 0.f) atomicMax(&s_hmax[gr % G], float_key(m));
+    }
+    __syncthreads();
+    float mh[kH2], lrun[kH2], arun[kH2];
+#pragma unroll
+    for (int i = 0; i < kH2; ++i) {
+      const int j = half + 2 * i;
+      mh[i] = j < G && s_hmax[j] != 0u ? key_float(s_hmax[j]) : -INFINITY;
+      lrun[i] = 0.f;
+      arun[i] = 0.f;
+    }
+    float* tile = reinterpret_cast<float*>(U);  // the correction's buffers are not in use yet
+    constexpr int kTR = (int)(fin_union_bytes<G>() / (kPartStride * sizeof(float))) / kMaxG * kMaxG;
+    __syncthreads();
+    for (int r0 = 0; r0 < nrows; r0 += (early_ok ? nrows : kTR)) {
+      const int nr = early_ok ? nrows : min(kTR, nrows - r0);
+      if (early_ok) {
+        tile = early;
+      } else {
+#pragma unroll 8
+        for (int i = tid; i < nr * kV; i += kFinThreads) {
+          const int row = i / kV, v = i % kV;
+          const int gr = r0 + row;
+          const float* src = p.scan_part + ((size_t)(w0 + s0 + gr / G + seg) * G + gr % G) * kPartStride;
+          reinterpret_cast<float4*>(tile + row * kPartStride)[v] = *reinterpret_cast<const float4*>(src + 4 * v);
+        }
+        __syncthreads();
+      }
+#pragma unroll
+      for (int i = 0; i < kH2; ++i) {
+        const int j = half + 2 * i;
+        if (j < G) {
+#pragma unroll 4
+          for (int row = (j - r0 % G + G) % G; row < nr; row += G) {
+            const float* tr = tile + row * kPartStride;
+            const float rl = tr[1];
+            const float f = rl > 0.f ? exp2f(tr[0] - mh[i]) : 0.f;
+            lrun[i] = fmaf(rl, f, lrun[i]);
+            arun[i] = fmaf(tr[4 + c], f, arun[i]);
+          }
+        }
+      }
+      if (!early_ok) __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < kH2; ++i) {
+      const int j = half + 2 * i;
+      if (j < G) {
+        P.sp[j][4 + c] = arun[i];
+        if (c == 0) {
+          P.sp[j][0] = lrun[i] > 0.f ? mh[i] : -INFINITY;
+          P.sp[j][1] = lrun[i];
+        }
+      }
+    }
+  }
+
+  if (select) cl.sync();  // every CTA's lists and counts are complete
 
   // ---- S3: resolve the selection; every CTA learns the whole chosen set:
   // the CTAs' sure lists (in CTA order) and the chosen ties (ascending)
@@ -901,8 +879,7 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
   // ---- C: the tail slots r, r + C, ... and an even share of the chosen set
   // (positions [x0, x1) of: the CTAs' lists in CTA order, then the chosen
   // ties), or of a given index set, or of every quantized token when
-  // k >= N_q; every listed token's rows and pieces are prefetched into L2 as
-  // the list is built
+  // k >= N_q
   {
     const int n_x = select ? k : (SELECT ? nq : k);
     const int per = (n_x + C - 1) / C;
@@ -916,25 +893,30 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
         for (int i = tid; i < n_tail; i += kFinThreads) {
           const int t = (1 << 30) | (r + C * i);
           tok[i] = t;
-          for (int part = 0; part < 4; ++part) prefetch_part(p, seg, t, part);
         }
         base = (uint32_t)n_tail;
       }
+      if (select) {  // every position holds a chosen token: no compaction
+        for (int j = xr + tid; j < xe; j += kFinThreads) {
+          int t;
+          if ((uint32_t)j < s_pre[C]) {
+            int q = 0;
+            while (q + 1 < C && s_pre[q + 1] <= (uint32_t)j) ++q;
+            t = (int)(mode == 1 ? glist_base[(size_t)q * p.slice + (j - s_pre[q])]
+                                : cl.map_shared_rank(PS.sure, q)[j - s_pre[q]]);
+          } else {
+            t = (int)PS.chtie[j - s_pre[C]];
+          }
+          tok[base + (j - xr)] = t;
+        }
+        base += (uint32_t)(xe - xr);
+      }
 #pragma unroll 1
-      for (int xb = xr; xb < xe; xb += kFinThreads) {
+      for (int xb = xr; !select && xb < xe; xb += kFinThreads) {
         const int j = xb + tid;
         int t = -1;
         if (j < xe) {
-          if (select) {
-            if ((uint32_t)j < s_pre[C]) {
-              int q = 0;
-              while (q + 1 < C && s_pre[q + 1] <= (uint32_t)j) ++q;
-              t = (int)(mode == 1 ? glist_base[(size_t)q * p.slice + (j - s_pre[q])]
-                                  : cl.map_shared_rank(PS.sure, q)[j - s_pre[q]]);
-            } else {
-              t = (int)PS.chtie[j - s_pre[C]];
-            }
-          } else if (SELECT) {
+          if (SELECT) {
             t = j;
           } else {
             t = p.idx_in[(size_t)seg * k + j];
@@ -946,10 +928,7 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
         }
         uint32_t tot;
         const uint32_t pos = base + block_prefix_excl(t >= 0 ? 1u : 0u, scratch, &tot);
-        if (t >= 0) {
-          tok[pos] = t;
-          prefetch_token<KB, VB, (G > 4 ? 2 : 1)>(p, seg, t);
-        }
+        if (t >= 0) tok[pos] = t;
         base += tot;
       }
       __syncthreads();
