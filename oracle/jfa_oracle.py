@@ -268,6 +268,43 @@ def topk_indices(scores, k: int) -> np.ndarray:
 
 
 # ---------------------------------------------------------------------------
+# Block selection (Jet-QSparse abstract: 128-token blocks are selected for the
+# sparse high-precision value aggregation, so the exact rows are contiguous)
+# ---------------------------------------------------------------------------
+BLOCK = 128
+
+
+def block_scores(scores, block: int = BLOCK) -> np.ndarray:
+    """Score of every block of ``block`` consecutive quantized tokens: the
+    largest selection score inside it (the last block may be partial).
+    scores [..., N] -> [..., ceil(N / block)]."""
+    scores = np.asarray(scores, dtype=np.float64)
+    *lead, n = scores.shape
+    nb = -(-n // block)
+    pad = np.full((*lead, nb * block - n), -np.inf)
+    return np.concatenate([scores, pad], axis=-1).reshape(*lead, nb, block).max(axis=-1)
+
+
+def topk_blocks(scores, n_blocks: int, block: int = BLOCK) -> np.ndarray:
+    """The n_blocks blocks with the largest block score, order (score
+    descending, block index ascending), expanded to their token indices:
+    every token of a chosen block, ascending, then -1 padding up to
+    n_blocks * block entries (tokens past N in a partial last block are
+    -1).  scores [..., N] -> int32 [..., n_blocks * block]."""
+    scores = np.asarray(scores, dtype=np.float64)
+    *lead, n = scores.shape
+    bs = block_scores(scores, block)
+    rows = int(np.prod(lead)) if lead else 1
+    flat = bs.reshape(rows, -1)
+    out = np.full((rows, n_blocks * block), -1, dtype=np.int32)
+    for r in range(rows):
+        chosen = topk_indices(flat[r][None], n_blocks)[0]
+        toks = [t for b in chosen if b >= 0 for t in range(b * block, (b + 1) * block) if t < n]
+        out[r, :len(toks)] = toks
+    return out.reshape(*lead, n_blocks * block)
+
+
+# ---------------------------------------------------------------------------
 # Softmax partials and log-sum-exp merge
 # ---------------------------------------------------------------------------
 @dataclasses.dataclass

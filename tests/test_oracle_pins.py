@@ -438,3 +438,83 @@ def test_pins_reject_unscaled_exact_attention(monkeypatch):
     monkeypatch.setitem(O.__dict__, "_exact_attention_unscaled", unscaled)
     with pytest.raises(AssertionError):
         test_exact_attention_is_torch_softmax_attention()
+
+
+# --------------------------------------------------------------------------
+# block selection (Jet-QSparse abstract: 128-token blocks)
+# --------------------------------------------------------------------------
+def test_block_scores_are_block_maxima_by_brute_force():
+    rng = np.random.default_rng(21)
+    for n in (1, 64, 127, 128, 129, 320, 1000):
+        s = rng.standard_normal(n)
+        got = O.block_scores(s[None], 128)[0]
+        want = [max(s[i:i + 128]) for i in range(0, n, 128)]
+        assert got.tolist() == want
+
+
+def test_block_selection_with_unit_blocks_is_token_topk():
+    rng = np.random.default_rng(22)
+    s = np.round(rng.standard_normal((3, 300)) * 3) / 3       # ties included
+    for k in (1, 7, 64, 300, 310):
+        assert np.array_equal(O.topk_blocks(s, k, block=1), O.topk_indices(s, k))
+
+
+def test_block_selection_brute_force():
+    rng = np.random.default_rng(23)
+    for trial in range(30):
+        n = int(rng.integers(64, 1500))
+        nb = -(-n // 128)
+        k = int(rng.integers(1, nb + 3))
+        s = rng.integers(-3, 3, n).astype(np.float64)          # many equal block maxima
+        bmax = [max(s[i:i + 128]) for i in range(0, n, 128)]
+        order = sorted(range(nb), key=lambda b: (-bmax[b], b))[:k]
+        toks = [t for b in sorted(order) for t in range(128 * b, min(n, 128 * b + 128))]
+        want = toks + [-1] * (128 * k - len(toks))
+        assert O.topk_blocks(s[None], k)[0].tolist() == want
+
+
+def test_block_selection_hand_case():
+    # 300 tokens: blocks [0,128), [128,256), [256,300); the best token sits in
+    # block 2 (partial), the second best in block 0
+    s = np.zeros(300)
+    s[290], s[5], s[200] = 9.0, 7.0, 1.0
+    got = O.topk_blocks(s[None], 2)[0]
+    assert got[:128].tolist() == list(range(128))
+    assert got[128:172].tolist() == list(range(256, 300))
+    assert np.all(got[172:] == -1)
+
+
+def test_block_selection_step_matches_hand_mixture():
+    # the decode step with the chosen blocks' tokens as the exact set equals
+    # softmax attention over the mixed key/value matrix (exact rows for the
+    # chosen blocks, dequantized for the rest, exact tail)
+    w, q, k, v, cache = _small(ctx=700, kb=3, vb=2)
+    scale = 0.09
+    s_hat = O.approx_logits(q, cache, scale)
+    sel = O.selection_scores(s_hat, 2)
+    idx = O.topk_blocks(sel, 2)
+    res = O.decode_step(q, k, v, cache, 256, scale, idx=idx)
+    kh, vh = cache.k_hat(), cache.v_hat()
+    nq = cache.n_quant
+    for b in range(2):
+        for hq in range(4):
+            h = hq // 2
+            keys, vals = kh[b, h].copy(), vh[b, h].copy()
+            chosen = idx[b, h][idx[b, h] >= 0]
+            assert len(chosen) == 256 and np.all(np.diff(chosen) > 0)
+            keys[chosen], vals[chosen] = k[b, h, chosen], v[b, h, chosen]
+            keys = np.concatenate([keys, k[b, h, nq:]])
+            vals = np.concatenate([vals, v[b, h, nq:]])
+            ref = _torch_attention(q[b, hq], keys, vals, scale)
+            assert np.allclose(res.out[b, hq], ref, rtol=1e-11, atol=1e-12)
+
+
+def test_pins_reject_block_mean_instead_of_max(monkeypatch):
+    def mean_blocks(scores, block=128):
+        scores = np.asarray(scores, dtype=np.float64)
+        *lead, n = scores.shape
+        nb = -(-n // block)
+        return np.stack([scores[..., i * block:(i + 1) * block].mean(-1) for i in range(nb)], -1)
+    monkeypatch.setattr(O, "block_scores", mean_blocks)
+    with pytest.raises(AssertionError):
+        test_block_scores_are_block_maxima_by_brute_force()
