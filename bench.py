@@ -432,6 +432,20 @@ class Setup:
                                           int(self.host), self.ws.buf, self.out, self.sp),
                    "correct_merge")
 
+    def step_blocks(self, i, n_blocks):
+        """A step with 128-token block selection: scores, jfa_topk_blocks,
+        jfa_correct_merge on the chosen blocks' tokens."""
+        from bit_kv_cache_jfa_b200 import _lib
+        _, g, cs, ke, ve = self.copies[i % self.n_copies]
+        k = n_blocks * 128
+        _lib.check(_lib.jfa_decode_scores(g, cs, self.q, self.scale, self.ws.buf, self.sp),
+                   "scores")
+        _lib.check(_lib.jfa_topk_blocks(g, n_blocks, self.ws.buf, self.idx_blocks, self.sp),
+                   "topk_blocks")
+        _lib.check(_lib.jfa_correct_merge(g, cs, self.q, self.scale, self.idx_blocks, k, ke, ve,
+                                          int(self.host), self.ws.buf, self.out, self.sp),
+                   "correct_merge")
+
     def check_flag(self):
         from bit_kv_cache_jfa_b200 import _lib
         st, flag = _lib.jfa_check_error(self.geom, self.ws.buf, self.sp)
@@ -479,13 +493,38 @@ class Setup:
                 "step_frac": step_gbs / peak, "step_alg_bytes": step_alg_bytes(w)}
 
 
-def per_config_line(args, dev, name: str, host: bool) -> dict:
+def block_alg_bytes(w, n_blocks: int) -> int:
+    """Step bytes with block selection: codes + scales, the chosen blocks'
+    exact rows, tail rows, q and out."""
+    n_seg = w.batch * w.kv_heads
+    tail = w.ctx - w.n_quant
+    rows = min(n_blocks * 128, w.n_quant)
+    return (n_seg * (w.n_quant * bytes_per_token(w) + (rows + tail) * 512)
+            + w.batch * w.heads * 128 * (2 + 4))
+
+
+def per_config_line(args, dev, name: str, host: bool, n_blocks: int = 0) -> dict:
     import torch
 
     import workloads as W
     w = W.WORKLOADS[name]
     st = Setup(w, dev, host)
     steps = max(20, min(args.steps, 200))
+    if n_blocks:
+        st.idx_blocks = torch.empty(w.batch, w.kv_heads, n_blocks * 128, dtype=torch.int32,
+                                    device=dev)
+        step_ms = st.timed(lambda i: st.step_blocks(i, n_blocks), steps, max(3, args.warmup))
+        st.check_flag()
+        peak, _ = measured_peaks()
+        alg = block_alg_bytes(w, n_blocks)
+        d = {"workload": name, "selection": f"{n_blocks} blocks of 128 tokens",
+             "exact_rows": "pinned_host" if host else "hbm", "steps": steps,
+             "us_per_step": step_ms * 1e3, "tokens_per_s": w.batch * w.ctx / (step_ms / 1e3),
+             "step_frac": alg / (step_ms / 1e3) / 1e9 / peak, "step_alg_bytes": alg,
+             "calls": "jfa_decode_scores + jfa_topk_blocks + jfa_correct_merge"}
+        del st
+        torch.cuda.empty_cache()
+        return d
     step_ms = st.timed(st.step, steps, max(3, args.warmup))
     st.check_flag()
     d = {"workload": name, "exact_rows": "pinned_host" if host else "hbm", "steps": steps,
@@ -578,6 +617,7 @@ def run_jfa(args, w):
             if name == w.name and host == args.host_resident:
                 continue
             per_config.append(per_config_line(args, dev, name, host))
+        per_config.append(per_config_line(args, dev, "llama8b_k4v4_128k", False, n_blocks=64))
 
     tokens = w.batch * w.ctx
     value = world * tokens / (ms_max / 1e3)

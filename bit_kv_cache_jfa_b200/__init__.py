@@ -18,10 +18,11 @@ from ._lib import (  # noqa: F401  (re-exported C ABI names)
     Cache, CacheLayout, Geom, JfaError, WorkspaceLayout, check, jfa_cache_layout_get,
     jfa_check_error, jfa_clear_error, jfa_correct_merge, jfa_decode_finish, jfa_decode_scores,
     jfa_decode_step,
-    jfa_decode_step_launches, jfa_pack_kv, jfa_topk, jfa_unpack_record,
+    jfa_decode_step_launches, jfa_pack_kv, jfa_topk, jfa_topk_blocks, jfa_unpack_record,
     jfa_workspace_layout_get, load)
 
-__all__ = ["KVCache", "Workspace", "decode_step", "DecodeGraph", "JfaError", "load"]
+__all__ = ["KVCache", "Workspace", "decode_step", "decode_step_blocks", "DecodeGraph", "JfaError",
+           "load"]
 
 
 def _torch():
@@ -113,6 +114,30 @@ def decode_step(cache: KVCache, q, k: int, k_exact, v_exact, ws: Workspace, scal
         idx = torch.empty(cache.batch, cache.num_kv_heads, k, dtype=torch.int32, device=dev)
     check(jfa_decode_step(cache.geom(), cache.struct(), q, float(scale), k, idx, k_exact,
                           v_exact, exact_on_host, ws.buf, out, stream), "jfa_decode_step")
+    return out, idx
+
+
+def decode_step_blocks(cache: KVCache, q, n_blocks: int, k_exact, v_exact, ws: Workspace,
+                       scale=None, out=None, idx=None, exact_on_host: bool = False, stream=None):
+    """One decode step with 128-token block selection: jfa_decode_scores,
+    jfa_topk_blocks (the n_blocks best blocks per sequence and KV head), then
+    jfa_correct_merge on their tokens.  Returns (out fp32 [B, H, 128], idx
+    int32 [B, H_kv, n_blocks * 128])."""
+    torch = _torch()
+    if scale is None:
+        scale = default_scale(cache.head_dim)
+    dev = q.device
+    k = n_blocks * _lib.BLOCK_TOKENS
+    if out is None:
+        out = torch.empty(cache.batch, cache.num_heads, cache.head_dim, dtype=torch.float32,
+                          device=dev)
+    if idx is None:
+        idx = torch.empty(cache.batch, cache.num_kv_heads, k, dtype=torch.int32, device=dev)
+    g, cs = cache.geom(), cache.struct()
+    check(jfa_decode_scores(g, cs, q, float(scale), ws.buf, stream), "jfa_decode_scores")
+    check(jfa_topk_blocks(g, n_blocks, ws.buf, idx, stream), "jfa_topk_blocks")
+    check(jfa_correct_merge(g, cs, q, float(scale), idx, k, k_exact, v_exact, exact_on_host,
+                            ws.buf, out, stream), "jfa_correct_merge")
     return out, idx
 
 

@@ -27,6 +27,9 @@ VAL_GROUP = 32
 TAIL_MAX = 64
 MAX_GQA = 8
 MAX_TOPK = 4096
+MAX_EXACT = 8192
+BLOCK_TOKENS = 128
+MAX_BLOCKS = MAX_EXACT // BLOCK_TOKENS
 
 
 class JfaError(RuntimeError):
@@ -71,6 +74,7 @@ SIGNATURES = {
     "jfa_decode_scores": (c_int32, [POINTER(Geom), POINTER(Cache), c_void_p, c_float, c_void_p,
                                     c_void_p]),
     "jfa_topk": (c_int32, [POINTER(Geom), c_int32, c_void_p, c_void_p, c_void_p]),
+    "jfa_topk_blocks": (c_int32, [POINTER(Geom), c_int32, c_void_p, c_void_p, c_void_p]),
     "jfa_topk_noalloc": (c_int32, [c_void_p, c_int32, c_int32, c_int32, c_int32, c_void_p,
                                    c_void_p]),
     "jfa_correct_merge": (c_int32, [POINTER(Geom), POINTER(Cache), c_void_p, c_float, c_void_p,
@@ -168,6 +172,11 @@ def jfa_decode_scores(geom, cache, q, scale, ws, stream=None) -> int:
 
 def jfa_topk(geom, k, ws, idx, stream=None) -> int:
     return load().jfa_topk(ctypes.byref(geom), k, _ptr(ws), _ptr(idx), _stream(stream))
+
+
+def jfa_topk_blocks(geom, n_blocks, ws, idx, stream=None) -> int:
+    return load().jfa_topk_blocks(ctypes.byref(geom), n_blocks, _ptr(ws), _ptr(idx),
+                                  _stream(stream))
 
 
 def jfa_topk_noalloc(scores, n_seg, stride, n_scores, k, idx, stream=None) -> int:

@@ -174,17 +174,29 @@ int jfa_topk(const jfa_geom* geom, int32_t k, void* ws, int32_t* idx, void* stre
                      static_cast<cudaStream_t>(stream));
 }
 
+int jfa_topk_blocks(const jfa_geom* geom, int32_t n_blocks, void* ws, int32_t* idx, void* stream) {
+  if (!geom_ok(geom) || !ws || !aligned(ws, 256) || !idx || !aligned(idx, 4))
+    return JFA_ERR_INVALID_ARG;
+  if (geom->n_ctx < 1 || n_blocks < 1 || n_blocks > JFA_MAX_BLOCKS) return JFA_ERR_INVALID_ARG;
+  if ((split_point(geom->n_ctx) + JFA_BLOCK_TOKENS - 1) / JFA_BLOCK_TOKENS > kMaxSelBlocks)
+    return JFA_ERR_UNSUPPORTED;
+  jfa_workspace_layout L;
+  workspace_layout(*geom, 1, &L);
+  return launch_topk_blocks(*geom, n_blocks, static_cast<uint8_t*>(ws), L, idx,
+                            static_cast<cudaStream_t>(stream));
+}
+
 int jfa_correct_merge(const jfa_geom* geom, const jfa_cache* cache, const uint16_t* q,
                       float scale, const int32_t* idx, int32_t k, const uint16_t* k_exact,
                       const uint16_t* v_exact, int32_t exact_on_host, void* ws, float* out,
                       void* stream) {
   if (!geom_ok(geom) || !cache_ok(cache) || !ws || !aligned(ws, 256)) return JFA_ERR_INVALID_ARG;
   if (geom->n_ctx < 1 || !q || !aligned(q, 16) || !(scale > 0.f)) return JFA_ERR_INVALID_ARG;
-  if (k < 1 || k > JFA_MAX_TOPK || !idx || !out || !aligned(out, 16)) return JFA_ERR_INVALID_ARG;
+  if (k < 1 || k > JFA_MAX_EXACT || !idx || !out || !aligned(out, 16)) return JFA_ERR_INVALID_ARG;
   if (!k_exact || !v_exact || !aligned(k_exact, 16) || !aligned(v_exact, 16))
     return JFA_ERR_INVALID_ARG;
   jfa_workspace_layout L;
-  workspace_layout(*geom, k, &L);
+  workspace_layout(*geom, 1, &L);
   (void)exact_on_host;  // same loads either way; the rows are device-addressable
   return launch_finish(*geom, *cache, q, scale, k, nullptr, idx, k_exact, v_exact,
                        static_cast<uint8_t*>(ws), L, out, static_cast<cudaStream_t>(stream));

@@ -57,6 +57,11 @@ int launch_scores(const jfa_geom& g, const jfa_cache& c, const uint16_t* q, floa
 int launch_topk(const jfa_geom& g, int k, uint8_t* ws, const jfa_workspace_layout& L,
                 int32_t* idx, cudaStream_t st);
 int count_topk_launches(const jfa_geom& g, int k);
+// Block selection: at most kMaxSelBlocks blocks of 128 quantized tokens per
+// segment (N_q <= 1M tokens).
+constexpr int kMaxSelBlocks = 8192;
+int launch_topk_blocks(const jfa_geom& g, int n_blocks, uint8_t* ws, const jfa_workspace_layout& L,
+                       int32_t* idx, cudaStream_t st);
 // Selection (idx_in == nullptr: top-k written to idx_out) or a given index
 // set (idx_in), then correction and merge: one cluster per segment.
 int launch_finish(const jfa_geom& g, const jfa_cache& c, const uint16_t* q, float scale, int k,

@@ -52,6 +52,9 @@ extern "C" {
 #define JFA_TAIL_MAX 64
 #define JFA_MAX_GQA 8
 #define JFA_MAX_TOPK 4096
+#define JFA_MAX_EXACT 8192    /* exact tokens per segment jfa_correct_merge takes */
+#define JFA_BLOCK_TOKENS 128  /* tokens per block of jfa_topk_blocks             */
+#define JFA_MAX_BLOCKS (JFA_MAX_EXACT / JFA_BLOCK_TOKENS)
 
 typedef enum jfa_status {
   JFA_OK = 0,
@@ -194,6 +197,23 @@ int jfa_decode_scores(const jfa_geom* geom, const jfa_cache* cache,
 int jfa_topk(const jfa_geom* geom, int32_t k, void* ws, int32_t* idx,
              void* stream);
 
+/* jfa_topk_blocks — selection of whole 128-token blocks instead of single
+ * tokens (Jet-QSparse abstract: 128-token blocks are selected for the sparse
+ * high-precision value aggregation, so the exact rows are read as contiguous
+ * tiles).  Per (sequence, KV head) the score of block j is the largest
+ * selection score S_t of its quantized tokens t in [128 j, 128 j + 128)
+ * (the last block holds 64 when N_q is an odd multiple of 64); the n_blocks
+ * blocks with the largest scores, order (score descending, block index
+ * ascending), are chosen and their token indices written ascending to
+ * idx[B][H_kv][n_blocks * 128] (int32 device pointer); tokens at or past N_q
+ * of a partial block and the entries of unchosen blocks are -1.  The result
+ * is a given index set for jfa_correct_merge with k = n_blocks * 128.
+ *   1 <= n_blocks <= JFA_MAX_BLOCKS; N_q <= 1048576 (else
+ *   JFA_ERR_UNSUPPORTED).  Reads the scores jfa_decode_scores leaves in the
+ *   workspace; allocates nothing. */
+int jfa_topk_blocks(const jfa_geom* geom, int32_t n_blocks, void* ws, int32_t* idx,
+                    void* stream);
+
 /* jfa_topk_noalloc — the selection of jfa_topk for callers that cannot
  * allocate device memory: an inference-engine plugin whose execute callback
  * must not allocate, code between cudaStreamBeginCapture and EndCapture
@@ -226,8 +246,9 @@ int jfa_topk_noalloc(const float* scores, int32_t n_seg, int32_t stride,
  * minus the top-k tokens' approximate terms); merged as
  *   m = max(m_e, m_a), out = (acc_e e^(m_e-m) + acc_a e^(m_a-m)) /
  *                            (l_e e^(m_e-m) + l_a e^(m_a-m)).
- *   idx          : int32 [B][H_kv][k] from jfa_topk (entries -1 ignored;
- *                  the others distinct, in [0, N_q), else the device flag
+ *   idx          : int32 [B][H_kv][k] from jfa_topk or jfa_topk_blocks
+ *                  (1 <= k <= JFA_MAX_EXACT; entries -1 ignored; the others
+ *                  distinct, in [0, N_q), else the device flag
  *                  JFA_DEVERR_BAD_INDEX is set and the entry skipped).
  * The approximate terms of the top-k tokens are taken out of the scan's
  * partials by recomputing, from the packed records and the running maxima

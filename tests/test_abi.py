@@ -139,3 +139,14 @@ def test_record_decoder_is_a_bijection_on_bits(lib, kb, vb):
         key = (i, pos, val)
         assert key not in seen, (bit, seen.get(key))
         seen[key] = bit
+
+
+def test_topk_blocks_rejects_bad_block_counts(lib):
+    g = G()
+    buf = ctypes.create_string_buffer(1024 + 256)
+    ws = (ctypes.addressof(buf) + 255) // 256 * 256
+    idx = ws
+    for n in (0, -1, lib.MAX_BLOCKS + 1):
+        assert lib.jfa_topk_blocks(g, n, ws, idx) == lib.JFA_ERR_INVALID_ARG
+    assert lib.jfa_topk_blocks(g, 4, 0, idx) == lib.JFA_ERR_INVALID_ARG
+    assert lib.jfa_topk_blocks(g, 4, ws, 0) == lib.JFA_ERR_INVALID_ARG
