@@ -540,6 +540,77 @@ def per_config_line(args, dev, name: str, host: bool, n_blocks: int = 0) -> dict
     return d
 
 
+def per_config_append(args, dev, name: str) -> dict:
+    """A decode loop with the append inside the step: every step appends one
+    token per sequence at its own position (jfa_append_decode_step: the
+    append kernel, flushing full tails into groups, then the scan and the
+    finishing kernel).  Two copies of the cache (together larger than L2)
+    alternate, each growing by one token per step it runs."""
+    import numpy as np
+    import torch
+
+    import bit_kv_cache_jfa_b200 as jfa
+    from bit_kv_cache_jfa_b200 import _lib
+    import workloads as W
+    w = W.WORKLOADS[name]
+    steps = max(20, min(args.steps, 200))
+    warm = max(3, args.warmup)
+    grow = (steps + warm) // 2 + 2
+    cap = 64 * -(-(w.ctx + grow) // 64)
+    k_all, v_all = W.gen_kv_device(w, dev, W.gen_q(w))
+    copies = []
+    ws = None
+    for c in range(2):
+        cache = jfa.KVCache(w.batch, w.heads, w.kv_heads, cap, w.key_bits, w.val_bits, device=dev)
+        if ws is None:
+            ws = jfa.Workspace(cache, w.topk, device=dev)
+        cache.append(k_all, v_all, ws)
+        ke = torch.zeros(w.batch, w.kv_heads, cap, 128, dtype=torch.bfloat16, device=dev)
+        ve = torch.zeros_like(ke)
+        ke[:, :, :w.ctx], ve[:, :, :w.ctx] = k_all, v_all
+        copies.append([cache, ke, ve, np.full(w.batch, w.ctx, dtype=np.int32)])
+    del k_all, v_all
+    q = W.gen_q(w).to(dev)
+    kn = torch.randn(w.batch, w.kv_heads, 128, device=dev).to(torch.bfloat16)
+    vn = torch.randn(w.batch, w.kv_heads, 128, device=dev).to(torch.bfloat16)
+    out = torch.empty(w.batch, w.heads, 128, dtype=torch.float32, device=dev)
+    idx = torch.empty(w.batch, w.kv_heads, w.topk, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    scale = W.default_scale(w)
+
+    def step(i):
+        cache, ke, ve, lens = copies[i % 2]
+        _lib.check(_lib.jfa_append_decode_step(cache.geom(), lens, cache.struct(), kn, vn, ke, ve,
+                                               q, scale, w.topk, idx, 0, ws.buf, out,
+                                               stream.cuda_stream), "append_decode_step")
+        lens += 1
+
+    for i in range(warm):
+        step(i)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for i in range(steps):
+        step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    st, flag = _lib.jfa_check_error(copies[0][0].geom(), ws.buf, stream.cuda_stream)
+    if flag:
+        raise RuntimeError(f"device error flag {flag:#x}")
+    ms = e0.elapsed_time(e1) / steps
+    peak, _ = measured_peaks()
+    alg = step_alg_bytes(w)
+    d = {"workload": name, "selection": "top-k tokens, one token appended per sequence per step",
+         "exact_rows": "hbm", "steps": steps, "us_per_step": ms * 1e3,
+         "tokens_per_s": w.batch * w.ctx / (ms / 1e3), "step_frac": alg / (ms / 1e3) / 1e9 / peak,
+         "calls": "jfa_append_decode_step (append kernel, scan, finishing kernel)",
+         "lengths": f"{w.ctx} .. {int(copies[0][3][0])} tokens per sequence (64-token "
+                    f"boundaries crossed: tails flushed into groups inside the step)"}
+    del copies, ws
+    torch.cuda.empty_cache()
+    return d
+
+
 def run_jfa(args, w):
     import torch
 
@@ -618,6 +689,7 @@ def run_jfa(args, w):
                 continue
             per_config.append(per_config_line(args, dev, name, host))
         per_config.append(per_config_line(args, dev, "llama8b_k4v4_128k", False, n_blocks=64))
+        per_config.append(per_config_append(args, dev, w.name))
 
     tokens = w.batch * w.ctx
     value = world * tokens / (ms_max / 1e3)

@@ -17,12 +17,12 @@ from . import _lib
 from ._lib import (  # noqa: F401  (re-exported C ABI names)
     Cache, CacheLayout, Geom, JfaError, WorkspaceLayout, check, jfa_cache_layout_get,
     jfa_check_error, jfa_clear_error, jfa_correct_merge, jfa_decode_finish, jfa_decode_scores,
-    jfa_decode_step,
+    jfa_append_decode_step, jfa_decode_step, jfa_decode_step_ragged,
     jfa_decode_step_launches, jfa_pack_kv, jfa_topk, jfa_topk_blocks, jfa_unpack_record,
     jfa_workspace_layout_get, load)
 
-__all__ = ["KVCache", "Workspace", "decode_step", "decode_step_blocks", "DecodeGraph", "JfaError",
-           "load"]
+__all__ = ["KVCache", "Workspace", "decode_step", "decode_step_blocks", "decode_step_ragged",
+           "append_decode_step", "DecodeGraph", "JfaError", "load"]
 
 
 def _torch():
@@ -138,6 +138,47 @@ def decode_step_blocks(cache: KVCache, q, n_blocks: int, k_exact, v_exact, ws: W
     check(jfa_topk_blocks(g, n_blocks, ws.buf, idx, stream), "jfa_topk_blocks")
     check(jfa_correct_merge(g, cs, q, float(scale), idx, k, k_exact, v_exact, exact_on_host,
                             ws.buf, out, stream), "jfa_correct_merge")
+    return out, idx
+
+
+def decode_step_ragged(cache: KVCache, seq_lens, q, k: int, k_exact, v_exact, ws: Workspace,
+                       scale=None, out=None, idx=None, exact_on_host: bool = False, stream=None):
+    """decode_step for sequences of different lengths: seq_lens (host ints,
+    one per sequence) gives each sequence's cached tokens."""
+    torch = _torch()
+    if scale is None:
+        scale = default_scale(cache.head_dim)
+    dev = q.device
+    if out is None:
+        out = torch.empty(cache.batch, cache.num_heads, cache.head_dim, dtype=torch.float32,
+                          device=dev)
+    if idx is None:
+        idx = torch.empty(cache.batch, cache.num_kv_heads, k, dtype=torch.int32, device=dev)
+    check(jfa_decode_step_ragged(cache.geom(), seq_lens, cache.struct(), q, float(scale), k, idx,
+                                 k_exact, v_exact, exact_on_host, ws.buf, out, stream),
+          "jfa_decode_step_ragged")
+    return out, idx
+
+
+def append_decode_step(cache: KVCache, seq_lens, k_new, v_new, q, k: int, k_exact, v_exact,
+                       ws: Workspace, scale=None, out=None, idx=None, exact_on_host: bool = False,
+                       stream=None):
+    """Append one token per sequence (bf16 [B, H_kv, 128] k_new / v_new, at
+    position seq_lens[b]; also written into the exact copy) and run the
+    decode step over the grown cache.  The caller adds one to every length
+    afterwards."""
+    torch = _torch()
+    if scale is None:
+        scale = default_scale(cache.head_dim)
+    dev = q.device
+    if out is None:
+        out = torch.empty(cache.batch, cache.num_heads, cache.head_dim, dtype=torch.float32,
+                          device=dev)
+    if idx is None:
+        idx = torch.empty(cache.batch, cache.num_kv_heads, k, dtype=torch.int32, device=dev)
+    check(jfa_append_decode_step(cache.geom(), seq_lens, cache.struct(), k_new, v_new, k_exact,
+                                 v_exact, q, float(scale), k, idx, exact_on_host, ws.buf, out,
+                                 stream), "jfa_append_decode_step")
     return out, idx
 
 

@@ -83,6 +83,12 @@ SIGNATURES = {
     "jfa_decode_step": (c_int32, [POINTER(Geom), POINTER(Cache), c_void_p, c_float, c_int32,
                                   c_void_p, c_void_p, c_void_p, c_int32, c_void_p, c_void_p,
                                   c_void_p]),
+    "jfa_decode_step_ragged": (c_int32, [POINTER(Geom), c_void_p, POINTER(Cache), c_void_p, c_float,
+                                         c_int32, c_void_p, c_void_p, c_void_p, c_int32, c_void_p,
+                                         c_void_p, c_void_p]),
+    "jfa_append_decode_step": (c_int32, [POINTER(Geom), c_void_p, POINTER(Cache), c_void_p,
+                                         c_void_p, c_void_p, c_void_p, c_void_p, c_float, c_int32,
+                                         c_void_p, c_int32, c_void_p, c_void_p, c_void_p]),
     "jfa_decode_finish": (c_int32, [POINTER(Geom), POINTER(Cache), c_void_p, c_float, c_int32,
                                     c_void_p, c_void_p, c_void_p, c_int32, c_void_p, c_void_p,
                                     c_void_p]),
@@ -198,6 +204,31 @@ def jfa_decode_step(geom, cache, q, scale, k, idx, k_exact, v_exact, exact_on_ho
     return load().jfa_decode_step(ctypes.byref(geom), ctypes.byref(cache), _ptr(q), scale, k,
                                   _ptr(idx), _ptr(k_exact), _ptr(v_exact), int(exact_on_host),
                                   _ptr(ws), _ptr(out), _stream(stream))
+
+
+def _lens(seq_lens):
+    """Host int32 array of per-sequence lengths (kept alive by the caller's
+    reference for the duration of the call)."""
+    import numpy as np
+    a = np.ascontiguousarray(np.asarray(seq_lens, dtype=np.int32))
+    return a, a.ctypes.data
+
+
+def jfa_decode_step_ragged(geom, seq_lens, cache, q, scale, k, idx, k_exact, v_exact,
+                           exact_on_host, ws, out, stream=None) -> int:
+    a, p = _lens(seq_lens)
+    return load().jfa_decode_step_ragged(ctypes.byref(geom), p, ctypes.byref(cache), _ptr(q),
+                                         scale, k, _ptr(idx), _ptr(k_exact), _ptr(v_exact),
+                                         int(exact_on_host), _ptr(ws), _ptr(out), _stream(stream))
+
+
+def jfa_append_decode_step(geom, seq_lens, cache, k_new, v_new, k_exact, v_exact, q, scale, k,
+                           idx, exact_on_host, ws, out, stream=None) -> int:
+    a, p = _lens(seq_lens)
+    return load().jfa_append_decode_step(ctypes.byref(geom), p, ctypes.byref(cache), _ptr(k_new),
+                                         _ptr(v_new), _ptr(k_exact), _ptr(v_exact), _ptr(q),
+                                         scale, k, _ptr(idx), int(exact_on_host), _ptr(ws),
+                                         _ptr(out), _stream(stream))
 
 
 def jfa_decode_finish(geom, cache, q, scale, k, idx, k_exact, v_exact, exact_on_host, ws, out,

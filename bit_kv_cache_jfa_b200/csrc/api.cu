@@ -76,11 +76,30 @@ int num_sms_current() {
   return cache[dev];
 }
 
-ScanPlan scan_plan(const jfa_geom& g, int num_sms) {
+bool fill_seq_table(const jfa_geom& g, const int32_t* lens, SeqTable* t) {
+  if (g.batch < 1 || g.batch > kMaxBatch) return false;
+  memset(t, 0, sizeof(*t));
+  int32_t acc = 0;
+  for (int b = 0; b < g.batch; ++b) {
+    const int32_t n = lens ? lens[b] : g.n_ctx;
+    if (n < 1 || n > g.capacity) return false;
+    t->n_ctx[b] = n;
+    t->gpre[b] = acc;
+    acc += g.num_kv_heads * seq_groups(*t, b);
+  }
+  t->gpre[g.batch] = acc;
+  return true;
+}
+
+int max_nq(const jfa_geom& g, const SeqTable& t) {
+  int m = 0;
+  for (int b = 0; b < g.batch; ++b) m = t.n_ctx[b] > m ? t.n_ctx[b] : m;
+  return split_point(m);
+}
+
+ScanPlan scan_plan(const jfa_geom& g, const SeqTable& t, int num_sms) {
   ScanPlan p;
-  const long long n_seg = (long long)g.batch * g.num_kv_heads;
-  p.ng = split_point(g.n_ctx) / kKG;
-  p.total_groups = n_seg * p.ng;
+  p.total_groups = t.gpre[g.batch];
   const int nw = scan_cta_warps(g.key_bits, g.val_bits, g.num_heads / g.num_kv_heads > 4 ? 2 : 1);
   long long w = (long long)num_sms * nw;
   if (w > kMaxScanWarps) w = kMaxScanWarps;
@@ -160,7 +179,9 @@ int jfa_decode_scores(const jfa_geom* geom, const jfa_cache* cache, const uint16
     return JFA_ERR_INVALID_ARG;
   jfa_workspace_layout L;
   workspace_layout(*geom, 1, &L);
-  return launch_scores(*geom, *cache, q, scale, static_cast<uint8_t*>(ws), L,
+  SeqTable t;
+  if (!fill_seq_table(*geom, nullptr, &t)) return JFA_ERR_INVALID_ARG;
+  return launch_scores(*geom, t, *cache, q, scale, static_cast<uint8_t*>(ws), L,
                        static_cast<cudaStream_t>(stream));
 }
 
@@ -198,7 +219,9 @@ int jfa_correct_merge(const jfa_geom* geom, const jfa_cache* cache, const uint16
   jfa_workspace_layout L;
   workspace_layout(*geom, 1, &L);
   (void)exact_on_host;  // same loads either way; the rows are device-addressable
-  return launch_finish(*geom, *cache, q, scale, k, nullptr, idx, k_exact, v_exact,
+  SeqTable t;
+  if (!fill_seq_table(*geom, nullptr, &t)) return JFA_ERR_INVALID_ARG;
+  return launch_finish(*geom, t, *cache, q, scale, k, nullptr, idx, k_exact, v_exact,
                        static_cast<uint8_t*>(ws), L, out, static_cast<cudaStream_t>(stream));
 }
 
@@ -230,8 +253,76 @@ int jfa_decode_finish(const jfa_geom* geom, const jfa_cache* cache, const uint16
   (void)exact_on_host;  // same loads either way; the rows are device-addressable
   jfa_workspace_layout L;
   workspace_layout(*geom, k, &L);
-  return launch_finish(*geom, *cache, q, scale, k, idx, nullptr, k_exact, v_exact,
+  SeqTable t;
+  if (!fill_seq_table(*geom, nullptr, &t)) return JFA_ERR_INVALID_ARG;
+  return launch_finish(*geom, t, *cache, q, scale, k, idx, nullptr, k_exact, v_exact,
                        static_cast<uint8_t*>(ws), L, out, static_cast<cudaStream_t>(stream));
+}
+
+// The step for per-sequence lengths: scan over every sequence's own groups,
+// then the finishing kernel with each cluster's own N_q and tail.
+static int ragged_step(const jfa_geom* geom, const SeqTable& t, const jfa_cache* cache,
+                       const uint16_t* q, float scale, int32_t k, int32_t* idx,
+                       const uint16_t* k_exact, const uint16_t* v_exact, void* ws, float* out,
+                       cudaStream_t st, bool pdl_scan) {
+  jfa_workspace_layout L;
+  workspace_layout(*geom, k, &L);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  const int s = launch_scores(*geom, t, *cache, q, scale, w, L, st, pdl_scan);
+  if (s != JFA_OK) return s;
+  return launch_finish(*geom, t, *cache, q, scale, k, idx, nullptr, k_exact, v_exact, w, L, out, st);
+}
+
+static bool step_args_ok(const jfa_geom* geom, const jfa_cache* cache, const uint16_t* q,
+                         float scale, int32_t k, const int32_t* idx, const uint16_t* k_exact,
+                         const uint16_t* v_exact, const void* ws, const float* out) {
+  if (!geom_ok(geom) || !cache_ok(cache) || !ws || !aligned(ws, 256)) return false;
+  if (!q || !aligned(q, 16) || !(scale > 0.f)) return false;
+  if (k < 1 || k > JFA_MAX_TOPK || !idx || !aligned(idx, 4) || !out || !aligned(out, 16))
+    return false;
+  if (!k_exact || !v_exact || !aligned(k_exact, 16) || !aligned(v_exact, 16)) return false;
+  return true;
+}
+
+int jfa_decode_step_ragged(const jfa_geom* geom, const int32_t* seq_lens, const jfa_cache* cache,
+                           const uint16_t* q, float scale, int32_t k, int32_t* idx,
+                           const uint16_t* k_exact, const uint16_t* v_exact, int32_t exact_on_host,
+                           void* ws, float* out, void* stream) {
+  if (!seq_lens || !step_args_ok(geom, cache, q, scale, k, idx, k_exact, v_exact, ws, out))
+    return JFA_ERR_INVALID_ARG;
+  (void)exact_on_host;  // same loads either way; the rows are device-addressable
+  SeqTable t;
+  if (!fill_seq_table(*geom, seq_lens, &t)) return JFA_ERR_INVALID_ARG;
+  return ragged_step(geom, t, cache, q, scale, k, idx, k_exact, v_exact, ws, out,
+                     static_cast<cudaStream_t>(stream), true);
+}
+
+int jfa_append_decode_step(const jfa_geom* geom, const int32_t* seq_lens, const jfa_cache* cache,
+                           const uint16_t* k_new, const uint16_t* v_new, uint16_t* k_exact,
+                           uint16_t* v_exact, const uint16_t* q, float scale, int32_t k,
+                           int32_t* idx, int32_t exact_on_host, void* ws, float* out,
+                           void* stream) {
+  if (!seq_lens || !step_args_ok(geom, cache, q, scale, k, idx, k_exact, v_exact, ws, out))
+    return JFA_ERR_INVALID_ARG;
+  if (!k_new || !v_new || !aligned(k_new, 16) || !aligned(v_new, 16)) return JFA_ERR_INVALID_ARG;
+  (void)exact_on_host;  // the new rows are stored the same way either way
+  if (!geom_ok(geom) || geom->batch > kMaxBatch) return JFA_ERR_INVALID_ARG;
+  int32_t after[kMaxBatch];
+  for (int b = 0; b < geom->batch; ++b) {
+    if (seq_lens[b] < 0 || seq_lens[b] >= geom->capacity) return JFA_ERR_INVALID_ARG;
+    after[b] = seq_lens[b] + 1;
+  }
+  SeqTable t;
+  if (!fill_seq_table(*geom, after, &t)) return JFA_ERR_INVALID_ARG;
+  jfa_workspace_layout L;
+  workspace_layout(*geom, k, &L);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int s = launch_append1(*geom, t, *cache, k_new, v_new, k_exact, v_exact,
+                               reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + L.off_flag), st);
+  if (s != JFA_OK) return s;
+  // the scan follows the kernel that may have written a record: plain stream
+  // order, so its first record copies start after that kernel has finished
+  return ragged_step(geom, t, cache, q, scale, k, idx, k_exact, v_exact, ws, out, st, false);
 }
 
 int jfa_decode_step_launches(const jfa_geom* geom, int32_t k) {
@@ -242,7 +333,9 @@ int jfa_decode_step_launches(const jfa_geom* geom, int32_t k) {
 
 int jfa_scan_warps(const jfa_geom* geom) {
   if (!geom_ok(geom) || geom->n_ctx < 1) return 0;
-  const ScanPlan plan = scan_plan(*geom, num_sms_current());
+  SeqTable t;
+  if (!fill_seq_table(*geom, nullptr, &t)) return 0;
+  const ScanPlan plan = scan_plan(*geom, t, num_sms_current());
   return plan.total_groups > 0 ? plan.n_warps : 0;
 }
 

@@ -5,12 +5,11 @@
 
 namespace jfa {
 
-int launch_finish(const jfa_geom& g, const jfa_cache& c, const uint16_t* q, float scale, int k,
-                  int32_t* idx_out, const int32_t* idx_in, const uint16_t* k_exact,
-                  const uint16_t* v_exact, uint8_t* ws, const jfa_workspace_layout& L, float* out,
-                  cudaStream_t st) {
+int launch_finish(const jfa_geom& g, const SeqTable& t, const jfa_cache& c, const uint16_t* q,
+                  float scale, int k, int32_t* idx_out, const int32_t* idx_in,
+                  const uint16_t* k_exact, const uint16_t* v_exact, uint8_t* ws,
+                  const jfa_workspace_layout& L, float* out, cudaStream_t st) {
   const int n_seg = g.batch * g.num_kv_heads;
-  const int nq = split_point(g.n_ctx);
   FinishParams fp;
   fp.groups = static_cast<const uint8_t*>(c.groups);
   fp.tail_k = c.tail_k;
@@ -29,8 +28,6 @@ int launch_finish(const jfa_geom& g, const jfa_cache& c, const uint16_t* q, floa
   fp.out = out;
   fp.flag = reinterpret_cast<uint32_t*>(ws + L.off_flag);
   fp.k = k;
-  fp.nq = nq;
-  fp.tail = g.n_ctx - nq;
   fp.capacity = g.capacity;
   fp.ng_cap = g.capacity / kKG;
   fp.hkv = g.num_kv_heads;
@@ -38,19 +35,20 @@ int launch_finish(const jfa_geom& g, const jfa_cache& c, const uint16_t* q, floa
   fp.key_bits = g.key_bits;
   fp.val_bits = g.val_bits;
   fp.rec_bytes = record_bytes(g.key_bits, g.val_bits);
-  const ScanPlan plan = scan_plan(g, num_sms_current());
+  const ScanPlan plan = scan_plan(g, t, num_sms_current());
   fp.scan_total = plan.total_groups;
   fp.scan_warps = plan.n_warps;
-  fp.ng = plan.ng;
   fp.kappa = scale * 1.4426950408889634f;
-  fp.slice = 64;
+  fp.gl_stride = 2 * L.cand_cap;
+  fp.seq = t;
   const int G = g.num_heads / g.num_kv_heads;
   const bool select = idx_in == nullptr;
+  const int nq_max = max_nq(g, t);
   if (g.key_bits == 3)
-    return g.val_bits == 2 ? launch_finish_k3v2(fp, G, n_seg, select, st)
-                           : launch_finish_k3v4(fp, G, n_seg, select, st);
-  return g.val_bits == 2 ? launch_finish_k4v2(fp, G, n_seg, select, st)
-                         : launch_finish_k4v4(fp, G, n_seg, select, st);
+    return g.val_bits == 2 ? launch_finish_k3v2(fp, G, n_seg, nq_max, select, st)
+                           : launch_finish_k3v4(fp, G, n_seg, nq_max, select, st);
+  return g.val_bits == 2 ? launch_finish_k4v2(fp, G, n_seg, nq_max, select, st)
+                         : launch_finish_k4v4(fp, G, n_seg, nq_max, select, st);
 }
 
 }  // namespace jfa

@@ -512,7 +512,7 @@ __device__ __forceinline__ void warp_correct(const FinishParams& p, int seg, con
 }
 
 template <int G, bool SELECT, int KB, int VB>
-__global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishParams p) {
+__global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const __grid_constant__ FinishParams p) {
   extern __shared__ __align__(16) uint8_t fsm[];
   FinPersist& PS = *reinterpret_cast<FinPersist*>(fsm);
   FinParts<G>& P = *reinterpret_cast<FinParts<G>*>(fsm + sizeof(FinPersist));
@@ -537,12 +537,16 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
   const int r = (int)cl.block_rank();
   const int seg = blockIdx.x / C;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int nq = p.nq, k = p.k;
+  const int k = p.k;
   const int bb = seg / p.hkv, hh = seg % p.hkv;
+  // this sequence's quantized tokens, tail and groups, and this CTA's slice
+  const int n_ctx = p.seq.n_ctx[bb];
+  const int nq = split_point(n_ctx), tail = n_ctx - nq, ng = nq / kKG;
+  const int slice = nq > 0 ? ((nq + C - 1) / C + 63) / 64 * 64 : 64;
 
   // ---- set-up: nothing here is written by the scan
   {  // this CTA's tail rows into L2 while the set-up runs
-    const int n_mine = p.tail > r ? (p.tail - r + C - 1) / C : 0;
+    const int n_mine = tail > r ? (tail - r + C - 1) / C : 0;
     for (int i = tid; i < n_mine * 4; i += kFinThreads)
       prefetch_part(p, seg, (1 << 30) | (r + C * (i >> 2)), i & 3);
   }
@@ -562,9 +566,9 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
   // ---- early copy of this CTA's share of the scan's split partials, every
   // head, when the rows fit (else they are staged a tile at a time below)
   long long w0 = 0, w1 = -1;
-  if (p.ng > 0) {
+  if (ng > 0) {
     const long long T = p.scan_total, W = p.scan_warps;
-    const long long x0 = (long long)seg * p.ng, x1 = x0 + p.ng - 1;
+    const long long x0 = (long long)p.seq.gpre[bb] + (long long)hh * ng, x1 = x0 + ng - 1;
     w0 = scan_warp_of(x0, W, T);
     w1 = scan_warp_of(x1, W, T);
   }
@@ -583,7 +587,7 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
   }
 
   const bool select = SELECT && k < nq;
-  const int lo = min(nq, r * p.slice), hi = min(nq, lo + p.slice);
+  const int lo = min(nq, r * slice), hi = min(nq, lo + slice);
   const uint32_t* hg = p.hist + (size_t)seg * kScanHistStride;
   // the segment's largest selection key
   const uint32_t top_key = select ? hg[kScanHistBins] : 0u;
@@ -777,7 +781,7 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
   // ---- S3: resolve the selection; every CTA learns the whole chosen set:
   // the CTAs' sure lists (in CTA order) and the chosen ties (ascending)
   uint32_t n_ch = 0;
-  const uint32_t* glist_base = p.glists + (size_t)seg * C * p.slice;
+  const uint32_t* glist_base = p.glists + (size_t)seg * p.gl_stride;
   int mode = 0;
   if (select) {
     {  // the scan's histogram is consumed: clear it for the next scan
@@ -849,14 +853,14 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
                     &s_tot);
       }
       if (tid <= C) {
-        const uint32_t b0 = (uint32_t)min(nq, tid * p.slice);
+        const uint32_t b0 = (uint32_t)min(nq, tid * slice);
         s_chq[tid] = lower_bound_u32(PS.chtie, n_ch, b0);
       }
       __syncthreads();
     } else {
       // fallback: select over the whole segment; each CTA lists its slice's
       // chosen indices in global memory
-      uint32_t* gl = const_cast<uint32_t*>(glist_base) + (size_t)r * p.slice;
+      uint32_t* gl = const_cast<uint32_t*>(glist_base) + (size_t)r * slice;
       const uint32_t n = select_full(p.scores + (size_t)seg * p.capacity, nq, k, lo, hi, FW.hist, gl,
                                      scratch, &s_bin, &s_above, &s_tot);
       if (tid == 0) PS.n_gl = n;
@@ -884,7 +888,7 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
     const int n_x = select ? k : (SELECT ? nq : k);
     const int per = (n_x + C - 1) / C;
     const int x0 = min(n_x, r * per), x1 = min(n_x, x0 + per);
-    const int n_tail = p.tail > r ? (p.tail - r + C - 1) / C : 0;
+    const int n_tail = tail > r ? (tail - r + C - 1) / C : 0;
 #pragma unroll 1
     for (int xr = x0, first = 1; first || xr < x1; xr += kTokCap, first = 0) {
       const int xe = min(x1, xr + kTokCap);
@@ -902,7 +906,7 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
           if ((uint32_t)j < s_pre[C]) {
             int q = 0;
             while (q + 1 < C && s_pre[q + 1] <= (uint32_t)j) ++q;
-            t = (int)(mode == 1 ? glist_base[(size_t)q * p.slice + (j - s_pre[q])]
+            t = (int)(mode == 1 ? glist_base[(size_t)q * slice + (j - s_pre[q])]
                                 : cl.map_shared_rank(PS.sure, q)[j - s_pre[q]]);
           } else {
             t = (int)PS.chtie[j - s_pre[C]];
@@ -941,7 +945,7 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const FinishPara
   if (select) {
     const uint32_t c0 = mode == 0 ? s_chq[r] : 0u, c1 = mode == 0 ? s_chq[r + 1] : 0u;
     const uint32_t off = s_pre[r] + c0;  // earlier slices: their lists and chosen ties
-    const uint32_t* Lr = mode == 1 ? glist_base + (size_t)r * p.slice : PS.sure;
+    const uint32_t* Lr = mode == 1 ? glist_base + (size_t)r * slice : PS.sure;
     const uint32_t nr = s_cnt[r];
     int32_t* out = p.idx_out + (size_t)seg * k;
     for (uint32_t i = tid; i < nr; i += kFinThreads) {
@@ -1099,7 +1103,7 @@ static int pick_cluster(int n_seg, int max_c, int num_sms) {
 }
 
 template <int G, bool SEL, int KB, int VB>
-static int launch_finish_t(FinishParams fp, int n_seg, cudaStream_t st) {
+static int launch_finish_t(const FinishParams& fp, int n_seg, int nq_max, cudaStream_t st) {
   constexpr size_t smem = fin_smem_bytes<G>();
   static bool configured[64] = {false};
   static int memo_seg[64][8] = {{0}}, memo_c[64][8] = {{0}};  // cluster size per (device, key)
@@ -1118,7 +1122,7 @@ static int launch_finish_t(FinishParams fp, int n_seg, cudaStream_t st) {
   }
   // clusters of 16 pay off once the slices are long (measured: 32K-token
   // segments gain, 8K ones lose); memoized per (segments, cap)
-  const int max_c = fp.nq >= 16384 ? kFinMaxC : 8;
+  const int max_c = nq_max >= 16384 ? kFinMaxC : 8;
   const int key = n_seg * 2 + (max_c > 8 ? 1 : 0);
   int C = 0;
   if (dev >= 0 && dev < 64) {
@@ -1136,8 +1140,6 @@ static int launch_finish_t(FinishParams fp, int n_seg, cudaStream_t st) {
         }
     }
   }
-  const int nq = fp.nq;
-  fp.slice = nq > 0 ? ((nq + C - 1) / C + 63) / 64 * 64 : 64;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(n_seg * C);
   cfg.blockDim = dim3(kFinThreads);
@@ -1156,16 +1158,16 @@ static int launch_finish_t(FinishParams fp, int n_seg, cudaStream_t st) {
 }
 
 template <bool SEL, int KB, int VB>
-static int launch_finish_g(const FinishParams& fp, int G, int n_seg, cudaStream_t st) {
+static int launch_finish_g(const FinishParams& fp, int G, int n_seg, int nq_max, cudaStream_t st) {
   switch (G) {
-    case 1: return launch_finish_t<1, SEL, KB, VB>(fp, n_seg, st);
-    case 2: return launch_finish_t<2, SEL, KB, VB>(fp, n_seg, st);
-    case 3: return launch_finish_t<3, SEL, KB, VB>(fp, n_seg, st);
-    case 4: return launch_finish_t<4, SEL, KB, VB>(fp, n_seg, st);
-    case 5: return launch_finish_t<5, SEL, KB, VB>(fp, n_seg, st);
-    case 6: return launch_finish_t<6, SEL, KB, VB>(fp, n_seg, st);
-    case 7: return launch_finish_t<7, SEL, KB, VB>(fp, n_seg, st);
-    default: return launch_finish_t<8, SEL, KB, VB>(fp, n_seg, st);
+    case 1: return launch_finish_t<1, SEL, KB, VB>(fp, n_seg, nq_max, st);
+    case 2: return launch_finish_t<2, SEL, KB, VB>(fp, n_seg, nq_max, st);
+    case 3: return launch_finish_t<3, SEL, KB, VB>(fp, n_seg, nq_max, st);
+    case 4: return launch_finish_t<4, SEL, KB, VB>(fp, n_seg, nq_max, st);
+    case 5: return launch_finish_t<5, SEL, KB, VB>(fp, n_seg, nq_max, st);
+    case 6: return launch_finish_t<6, SEL, KB, VB>(fp, n_seg, nq_max, st);
+    case 7: return launch_finish_t<7, SEL, KB, VB>(fp, n_seg, nq_max, st);
+    default: return launch_finish_t<8, SEL, KB, VB>(fp, n_seg, nq_max, st);
   }
 }
 

@@ -23,18 +23,21 @@ struct FinishParams {
   int32_t* idx_out;        // [n_seg][k] (selection)
   float* out;
   uint32_t* flag;
-  int k, nq, tail, capacity, ng_cap, hkv, H, key_bits, val_bits, rec_bytes, ng, slice;
+  int k, capacity, ng_cap, hkv, H, key_bits, val_bits, rec_bytes;
+  int gl_stride;           // uint32 entries of glists per segment
   long long scan_total;
   int scan_warps;
   float kappa;
+  SeqTable seq;            // per-sequence lengths and the scan's group offsets
 };
 
 // Launch the finishing kernel for G = num_heads / num_kv_heads query heads per
 // KV head over n_seg (sequence, KV head) segments; select = run the top-k
 // selection (else fp.idx_in holds the index sets).  One per key/value width.
-int launch_finish_k3v2(const FinishParams& fp, int G, int n_seg, bool select, cudaStream_t st);
-int launch_finish_k3v4(const FinishParams& fp, int G, int n_seg, bool select, cudaStream_t st);
-int launch_finish_k4v2(const FinishParams& fp, int G, int n_seg, bool select, cudaStream_t st);
-int launch_finish_k4v4(const FinishParams& fp, int G, int n_seg, bool select, cudaStream_t st);
+// nq_max: the largest N_q of the batch (picks the cluster size).
+int launch_finish_k3v2(const FinishParams& fp, int G, int n_seg, int nq_max, bool select, cudaStream_t st);
+int launch_finish_k3v4(const FinishParams& fp, int G, int n_seg, int nq_max, bool select, cudaStream_t st);
+int launch_finish_k4v2(const FinishParams& fp, int G, int n_seg, int nq_max, bool select, cudaStream_t st);
+int launch_finish_k4v4(const FinishParams& fp, int G, int n_seg, int nq_max, bool select, cudaStream_t st);
 
 }  // namespace jfa

@@ -29,16 +29,35 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
 // Workspace layout for (geometry, max_topk); host and device agree on it.
 int workspace_layout(const jfa_geom& g, int max_topk, jfa_workspace_layout* out);
 
+// Per-sequence lengths of one call (the same for every KV head of a
+// sequence) and the offset of each sequence's first group in the flattened
+// (segment, group) list the scan splits: sequence b, KV head h, group g is
+// entry gpre[b] + h * ng(b) + g, ng(b) = N_q(b) / 64.  Passed by value in
+// the launch parameters (2 KB).
+constexpr int kMaxBatch = JFA_MAX_BATCH;
+struct SeqTable {
+  int32_t n_ctx[kMaxBatch];
+  int32_t gpre[kMaxBatch + 1];
+};
+// Fill the table for a geometry: lens[b] (host array) or, when lens is null,
+// geom.n_ctx for every sequence.  Returns false when a length is outside
+// [1, capacity] or the batch exceeds kMaxBatch.
+bool fill_seq_table(const jfa_geom& g, const int32_t* lens, SeqTable* t);
+__host__ __device__ __forceinline__ int seq_groups(const SeqTable& t, int b) {
+  return split_point(t.n_ctx[b]) / kKG;
+}
+// Largest quantized-token count over the batch.
+int max_nq(const jfa_geom& g, const SeqTable& t);
+
 // Scan decomposition: W warps each take a balanced contiguous range of the
 // flattened (segment, group) list; warp w writes one partial per segment it
 // touches into slot (w + segment).
 struct ScanPlan {
-  long long total_groups;  // n_seg * NG
-  int ng;                  // groups per segment in this call (N_q / 64)
+  long long total_groups;  // entries of the flattened list
   int n_warps;             // warps with work
   int n_ctas;
 };
-ScanPlan scan_plan(const jfa_geom& g, int num_sms);
+ScanPlan scan_plan(const jfa_geom& g, const SeqTable& t, int num_sms);
 int num_sms_current();
 
 // First warp whose range contains flattened group x (W warps, T groups).
@@ -52,8 +71,18 @@ __host__ __device__ __forceinline__ long long scan_range_begin(long long w, long
 
 int launch_pack(const jfa_geom& g, const jfa_cache& c, const uint16_t* k_new,
                 const uint16_t* v_new, int n_new, uint32_t* flag, cudaStream_t st);
-int launch_scores(const jfa_geom& g, const jfa_cache& c, const uint16_t* q, float scale,
-                  uint8_t* ws, const jfa_workspace_layout& L, cudaStream_t st);
+// One new token per sequence at position t.n_ctx[b] - 1 (t holds the lengths
+// after the append; a full tail is first flushed as one group); the new rows
+// also go to the exact copy when it is given.
+int launch_append1(const jfa_geom& g, const SeqTable& t, const jfa_cache& c, const uint16_t* k_new,
+                   const uint16_t* v_new, uint16_t* k_exact, uint16_t* v_exact, uint32_t* flag,
+                   cudaStream_t st);
+// pdl: launch as a programmatic dependent of the previous kernel (its first
+// record copies may then start before that kernel has finished); false for a
+// scan right after a kernel that writes the packed records.
+int launch_scores(const jfa_geom& g, const SeqTable& t, const jfa_cache& c, const uint16_t* q,
+                  float scale, uint8_t* ws, const jfa_workspace_layout& L, cudaStream_t st,
+                  bool pdl = true);
 int launch_topk(const jfa_geom& g, int k, uint8_t* ws, const jfa_workspace_layout& L,
                 int32_t* idx, cudaStream_t st);
 int count_topk_launches(const jfa_geom& g, int k);
@@ -64,7 +93,8 @@ int launch_topk_blocks(const jfa_geom& g, int n_blocks, uint8_t* ws, const jfa_w
                        int32_t* idx, cudaStream_t st);
 // Selection (idx_in == nullptr: top-k written to idx_out) or a given index
 // set (idx_in), then correction and merge: one cluster per segment.
-int launch_finish(const jfa_geom& g, const jfa_cache& c, const uint16_t* q, float scale, int k,
+int launch_finish(const jfa_geom& g, const SeqTable& t, const jfa_cache& c, const uint16_t* q,
+                  float scale, int k,
                   int32_t* idx_out, const int32_t* idx_in, const uint16_t* k_exact,
                   const uint16_t* v_exact, uint8_t* ws, const jfa_workspace_layout& L, float* out,
                   cudaStream_t st);

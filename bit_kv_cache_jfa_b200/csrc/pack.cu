@@ -51,6 +51,64 @@ __device__ __forceinline__ uint32_t quant_code(double x, double z, double s, int
 __device__ __forceinline__ bool finite_h(uint16_t b) { return (b & 0x7C00u) != 0x7C00u; }
 __device__ __forceinline__ float bf(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
 
+// Quantize one 64-token group staged in shared memory (bf16 bits, token
+// rows) into a zeroed record image rb; all 256 threads take part.
+__device__ __forceinline__ void quantize_tile(const uint16_t (*xk)[kD + 2], const uint16_t (*xv)[kD + 2],
+                                              uint8_t* rb, int key_bits, int val_bits, uint32_t* flag) {
+  const int tid = threadIdx.x;
+  bool bad = false;
+  // keys: thread c < 128 owns channel c
+  if (tid < kD) {
+    const int c = tid;
+    float mn = bf(xk[0][c]), mx = mn;
+    for (int t = 1; t < kKG; ++t) {
+      mn = fminf(mn, bf(xk[t][c]));
+      mx = fmaxf(mx, bf(xk[t][c]));
+    }
+    uint16_t zb, sb;
+    double z, s;
+    quant_params((double)mn, (double)mx, key_bits, zb, sb, z, s);
+    bad |= !finite_h(zb) || !finite_h(sb);
+    *reinterpret_cast<uint16_t*>(rb + off_ks() + ks_scale_off(c)) = sb;
+    *reinterpret_cast<uint16_t*>(rb + off_ks() + ks_zero_off(c)) = zb;
+    for (int t = 0; t < kKG; ++t) {
+      uint32_t code = quant_code((double)bf(xk[t][c]), z, s, key_bits);
+      BitLoc L[3];
+      const int n = kc_bits(key_bits, t, c, L);
+      if (n == 1) {
+        if (code) atomicOr(reinterpret_cast<uint32_t*>(rb + off_kc() + L[0].byte), code << L[0].bit);
+      } else {
+        for (int b = 0; b < 3; ++b)
+          if ((code >> b) & 1u)
+            atomicOr(reinterpret_cast<uint32_t*>(rb + off_kc() + L[b].byte), 1u << L[b].bit);
+      }
+    }
+  } else {
+    // values: threads 128..255 own (token, group) pairs 2 each
+    for (int u = tid - kD; u < kKG * (kD / kVG); u += 128) {
+      const int t = u >> 2, j = u & 3;
+      float mn = bf(xv[t][j * kVG]), mx = mn;
+      for (int c = 1; c < kVG; ++c) {
+        mn = fminf(mn, bf(xv[t][j * kVG + c]));
+        mx = fmaxf(mx, bf(xv[t][j * kVG + c]));
+      }
+      uint16_t zb, sb;
+      double z, s;
+      quant_params((double)mn, (double)mx, val_bits, zb, sb, z, s);
+      bad |= !finite_h(zb) || !finite_h(sb);
+      *reinterpret_cast<uint16_t*>(rb + off_vs(key_bits) + vs_scale_off(t, j)) = sb;
+      *reinterpret_cast<uint16_t*>(rb + off_vs(key_bits) + vs_zero_off(t, j)) = zb;
+      for (int cc = 0; cc < kVG; ++cc) {
+        const int c = j * kVG + cc;
+        uint32_t code = quant_code((double)bf(xv[t][c]), z, s, val_bits);
+        BitLoc L = vc_loc(val_bits, t, c);
+        if (code) atomicOr(reinterpret_cast<uint32_t*>(rb + off_vc(key_bits) + L.byte), code << L.bit);
+      }
+    }
+  }
+  if (bad) set_flag(flag, JFA_DEVERR_NONFINITE_QUANT);
+}
+
 // One CTA (256 threads) quantizes one 64-token group of one segment.
 __global__ void __launch_bounds__(256) pack_groups_kernel(PackParams p) {
   __shared__ uint16_t xk[kKG][kD + 2];  // bf16 bits
@@ -73,63 +131,92 @@ __global__ void __launch_bounds__(256) pack_groups_kernel(PackParams p) {
     xv[t][c2 + 1] = (uint16_t)(wv >> 16);
   }
   __syncthreads();
-
-  uint8_t* rb = reinterpret_cast<uint8_t*>(rec);
-  bool bad = false;
-  // keys: thread c < 128 owns channel c
-  if (tid < kD) {
-    const int c = tid;
-    float mn = bf(xk[0][c]), mx = mn;
-    for (int t = 1; t < kKG; ++t) {
-      mn = fminf(mn, bf(xk[t][c]));
-      mx = fmaxf(mx, bf(xk[t][c]));
-    }
-    uint16_t zb, sb;
-    double z, s;
-    quant_params((double)mn, (double)mx, p.key_bits, zb, sb, z, s);
-    bad |= !finite_h(zb) || !finite_h(sb);
-    *reinterpret_cast<uint16_t*>(rb + off_ks() + ks_scale_off(c)) = sb;
-    *reinterpret_cast<uint16_t*>(rb + off_ks() + ks_zero_off(c)) = zb;
-    for (int t = 0; t < kKG; ++t) {
-      uint32_t code = quant_code((double)bf(xk[t][c]), z, s, p.key_bits);
-      BitLoc L[3];
-      const int n = kc_bits(p.key_bits, t, c, L);
-      if (n == 1) {
-        if (code) atomicOr(reinterpret_cast<uint32_t*>(rb + off_kc() + L[0].byte), code << L[0].bit);
-      } else {
-        for (int b = 0; b < 3; ++b)
-          if ((code >> b) & 1u)
-            atomicOr(reinterpret_cast<uint32_t*>(rb + off_kc() + L[b].byte), 1u << L[b].bit);
-      }
-    }
-  } else {
-    // values: threads 128..255 own (token, group) pairs 2 each
-    for (int u = tid - kD; u < kKG * (kD / kVG); u += 128) {
-      const int t = u >> 2, j = u & 3;
-      float mn = bf(xv[t][j * kVG]), mx = mn;
-      for (int c = 1; c < kVG; ++c) {
-        mn = fminf(mn, bf(xv[t][j * kVG + c]));
-        mx = fmaxf(mx, bf(xv[t][j * kVG + c]));
-      }
-      uint16_t zb, sb;
-      double z, s;
-      quant_params((double)mn, (double)mx, p.val_bits, zb, sb, z, s);
-      bad |= !finite_h(zb) || !finite_h(sb);
-      *reinterpret_cast<uint16_t*>(rb + off_vs(p.key_bits) + vs_scale_off(t, j)) = sb;
-      *reinterpret_cast<uint16_t*>(rb + off_vs(p.key_bits) + vs_zero_off(t, j)) = zb;
-      for (int cc = 0; cc < kVG; ++cc) {
-        const int c = j * kVG + cc;
-        uint32_t code = quant_code((double)bf(xv[t][c]), z, s, p.val_bits);
-        BitLoc L = vc_loc(p.val_bits, t, c);
-        if (code) atomicOr(reinterpret_cast<uint32_t*>(rb + off_vc(p.key_bits) + L.byte), code << L.bit);
-      }
-    }
-  }
-  if (bad) set_flag(p.flag, JFA_DEVERR_NONFINITE_QUANT);
+  quantize_tile(xk, xv, reinterpret_cast<uint8_t*>(rec), p.key_bits, p.val_bits, p.flag);
   __syncthreads();
   uint4* dst = reinterpret_cast<uint4*>(p.groups + ((size_t)seg * p.ng_cap + g) * p.rec_bytes);
   const uint4* src = reinterpret_cast<const uint4*>(rec);
   for (int i = tid; i < p.rec_bytes / 16; i += 256) dst[i] = src[i];
+}
+
+// One new token per sequence, each at its own position n0 = n_ctx[b] (one
+// CTA per (sequence, KV head)).  A full tail (n0 a positive multiple of 64)
+// is first quantized as group n0/64 - 1 and the token starts a new tail;
+// else it joins the tail.  The token's rows also go to the exact copy at
+// position n0 when one is given.
+struct AppendParams {
+  uint8_t* groups;
+  uint16_t* tail_k;
+  uint16_t* tail_v;
+  const uint16_t* k_new;  // [n_seg][128]
+  const uint16_t* v_new;
+  uint16_t* k_exact;      // [n_seg][capacity][128] or null
+  uint16_t* v_exact;
+  uint32_t* flag;
+  int hkv, ng_cap, capacity, key_bits, val_bits, rec_bytes;
+  SeqTable seq;           // lengths after the append
+};
+
+__global__ void __launch_bounds__(256) append1_kernel(const __grid_constant__ AppendParams p) {
+  __shared__ uint16_t xk[kKG][kD + 2];
+  __shared__ uint16_t xv[kKG][kD + 2];
+  __shared__ __align__(16) uint32_t rec[9728 / 4];
+  const int seg = blockIdx.x, tid = threadIdx.x;
+  const int n0 = p.seq.n_ctx[seg / p.hkv] - 1;  // the table holds the lengths after
+  const int tl = n0 - split_point(n0);  // tail tokens before the append
+  const bool flush = tl == kTail;        // n0 a positive multiple of 64
+  if (flush) {
+    const int g = n0 / kKG - 1;
+    for (int i = tid; i < p.rec_bytes / 4; i += 256) rec[i] = 0u;
+    for (int i = tid; i < kKG * kD / 2; i += 256) {
+      const int t = i / (kD / 2), c2 = (i % (kD / 2)) * 2;
+      const uint32_t wk = reinterpret_cast<const uint32_t*>(p.tail_k + ((size_t)seg * kTail + t) * kD)[c2 / 2];
+      const uint32_t wv = reinterpret_cast<const uint32_t*>(p.tail_v + ((size_t)seg * kTail + t) * kD)[c2 / 2];
+      xk[t][c2] = (uint16_t)(wk & 0xFFFFu);
+      xk[t][c2 + 1] = (uint16_t)(wk >> 16);
+      xv[t][c2] = (uint16_t)(wv & 0xFFFFu);
+      xv[t][c2 + 1] = (uint16_t)(wv >> 16);
+    }
+    __syncthreads();
+    quantize_tile(xk, xv, reinterpret_cast<uint8_t*>(rec), p.key_bits, p.val_bits, p.flag);
+    __syncthreads();
+    uint4* dst = reinterpret_cast<uint4*>(p.groups + ((size_t)seg * p.ng_cap + g) * p.rec_bytes);
+    const uint4* src = reinterpret_cast<const uint4*>(rec);
+    for (int i = tid; i < p.rec_bytes / 16; i += 256) dst[i] = src[i];
+  }
+  // the token: tail slot (0 after a flush), then the exact copy
+  const int slot = flush ? 0 : tl;
+  if (tid < 16) {
+    const uint4 kv = reinterpret_cast<const uint4*>(p.k_new + (size_t)seg * kD)[tid];
+    reinterpret_cast<uint4*>(p.tail_k + ((size_t)seg * kTail + slot) * kD)[tid] = kv;
+    if (p.k_exact) reinterpret_cast<uint4*>(p.k_exact + ((size_t)seg * p.capacity + n0) * kD)[tid] = kv;
+  } else if (tid < 32) {
+    const uint4 vv = reinterpret_cast<const uint4*>(p.v_new + (size_t)seg * kD)[tid - 16];
+    reinterpret_cast<uint4*>(p.tail_v + ((size_t)seg * kTail + slot) * kD)[tid - 16] = vv;
+    if (p.v_exact) reinterpret_cast<uint4*>(p.v_exact + ((size_t)seg * p.capacity + n0) * kD)[tid - 16] = vv;
+  }
+}
+
+int launch_append1(const jfa_geom& g, const SeqTable& t, const jfa_cache& c, const uint16_t* k_new,
+                   const uint16_t* v_new, uint16_t* k_exact, uint16_t* v_exact, uint32_t* flag,
+                   cudaStream_t st) {
+  AppendParams p;
+  p.groups = static_cast<uint8_t*>(c.groups);
+  p.tail_k = c.tail_k;
+  p.tail_v = c.tail_v;
+  p.k_new = k_new;
+  p.v_new = v_new;
+  p.k_exact = k_exact;
+  p.v_exact = v_exact;
+  p.flag = flag;
+  p.hkv = g.num_kv_heads;
+  p.ng_cap = g.capacity / kKG;
+  p.capacity = g.capacity;
+  p.key_bits = g.key_bits;
+  p.val_bits = g.val_bits;
+  p.rec_bytes = record_bytes(g.key_bits, g.val_bits);
+  p.seq = t;
+  append1_kernel<<<dim3(g.batch * g.num_kv_heads), 256, 0, st>>>(p);
+  return cudaGetLastError() == cudaSuccess ? JFA_OK : JFA_ERR_CUDA;
 }
 
 // Tail update: copy new tokens [src0, n_new) to tail slots [dst0, ...).

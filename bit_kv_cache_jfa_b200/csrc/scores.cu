@@ -44,12 +44,35 @@ struct ScanParams {
   uint32_t* wts;    // [n_seg][ng_cap][4][NT][32]: the fp16 weights, lane order
   uint32_t* hist;   // [n_seg][kScanHistStride]: bins, then the largest key
   uint32_t* flag;
-  long long total;  // n_seg * ng
-  int ng, ng_cap, capacity;
-  int hkv, G, H;
+  long long total;  // entries of the flattened (segment, group) list
+  int ng_cap, capacity;
+  int hkv, G, H, n_seg;
   int n_warps;
   float kappa;      // scale * log2(e): logits are kept in log2 units
+  SeqTable seq;     // per-sequence lengths and group offsets
 };
+
+// (segment, group) of flattened entry x: the sequence by binary search over
+// the group offsets (a sequence without groups has an empty range), then the
+// KV head and group inside it.
+__device__ __forceinline__ void locate_group(const ScanParams& p, long long x, int& seg, int& g) {
+  int lo = 0, hi = p.n_seg / p.hkv;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (p.seq.gpre[mid] <= x) lo = mid;
+    else hi = mid;
+  }
+  const int ngb = seq_groups(p.seq, lo);
+  const int r = (int)(x - p.seq.gpre[lo]);
+  seg = lo * p.hkv + r / ngb;
+  g = r % ngb;
+}
+// The entry after the last group of segment seg: the next segment with groups.
+__device__ __forceinline__ int next_segment(const ScanParams& p, int seg) {
+  ++seg;
+  while (seg < p.n_seg && seq_groups(p.seq, seg / p.hkv) == 0) seg += p.hkv;
+  return seg;
+}
 
 __device__ __forceinline__ uint4 lds128(const uint8_t* p) {
   return *reinterpret_cast<const uint4*>(p);
@@ -71,7 +94,8 @@ struct ScanCfg {
 };
 
 template <int KB, int VB, int NT>
-__global__ void __launch_bounds__(ScanCfg<KB, VB, NT>::NW * 32, 1) scan_kernel(const ScanParams p) {
+__global__ void __launch_bounds__(ScanCfg<KB, VB, NT>::NW * 32, 1)
+    scan_kernel(const __grid_constant__ ScanParams p) {
   using Cfg = ScanCfg<KB, VB, NT>;
   constexpr int REC = Cfg::REC;
   constexpr int S = Cfg::STAGES;
@@ -100,15 +124,17 @@ __global__ void __launch_bounds__(ScanCfg<KB, VB, NT>::NW * 32, 1) scan_kernel(c
   }
   __syncwarp();
   // prefetch cursor (segment, group) of the next record to request
-  long long pf_seg = g0 / p.ng;
-  int pf_g = (int)(g0 - pf_seg * p.ng);
+  int pf_seg = 0, pf_g = 0;
+  if (has_work) locate_group(p, g0, pf_seg, pf_g);
+  int pf_ng = has_work ? seq_groups(p.seq, pf_seg / p.hkv) : 0;
   auto issue_next = [&](int stage) {
     mbar_expect_tx(&bar[stage], REC);
     bulk_g2s(ring + stage * REC, p.groups + ((size_t)pf_seg * p.ng_cap + (size_t)pf_g) * REC,
              REC, &bar[stage], pol);
-    if (++pf_g == p.ng) {
+    if (++pf_g == pf_ng) {
       pf_g = 0;
-      ++pf_seg;
+      pf_seg = next_segment(p, pf_seg);
+      pf_ng = pf_seg < p.n_seg ? seq_groups(p.seq, pf_seg / p.hkv) : 0;
     }
   };
   // only the first stage now: every warp's first record is requested before
@@ -188,8 +214,9 @@ __global__ void __launch_bounds__(ScanCfg<KB, VB, NT>::NW * 32, 1) scan_kernel(c
     }
   };
 
-  long long seg = g0 / p.ng;
-  int g = (int)(g0 - seg * p.ng);
+  int seg = 0, g = 0;
+  if (has_work) locate_group(p, g0, seg, g);
+  int ng_cur = has_work ? seq_groups(p.seq, seg / p.hkv) : 0;
   int st = 0;
   uint32_t par = 0;
   bool failed = false;
@@ -442,9 +469,10 @@ __global__ void __launch_bounds__(ScanCfg<KB, VB, NT>::NW * 32, 1) scan_kernel(c
       st = 0;
       par ^= 1u;
     }
-    if (++g == p.ng) {
+    if (++g == ng_cur) {
       g = 0;
-      ++seg;
+      seg = next_segment(p, seg);
+      ng_cur = seg < p.n_seg ? seq_groups(p.seq, seg / p.hkv) : 0;
     }
   }
   if (has_work && !failed) flush(cur);
@@ -457,7 +485,7 @@ __global__ void __launch_bounds__(ScanCfg<KB, VB, NT>::NW * 32, 1) scan_kernel(c
 }
 
 template <int KB, int VB, int NT>
-static int launch_scan_t(const ScanParams& sp, int n_ctas, cudaStream_t st) {
+static int launch_scan_t(const ScanParams& sp, int n_ctas, bool pdl, cudaStream_t st) {
   using Cfg = ScanCfg<KB, VB, NT>;
   static bool configured[64] = {false};  // per device: the attribute is set on each
   int dev = 0;
@@ -468,6 +496,10 @@ static int launch_scan_t(const ScanParams& sp, int n_ctas, cudaStream_t st) {
       return JFA_ERR_CUDA;
     if (dev >= 0 && dev < 64) configured[dev] = true;
   }
+  if (!pdl) {
+    scan_kernel<KB, VB, NT><<<dim3(n_ctas), dim3(Cfg::NW * 32), (size_t)Cfg::SMEM, st>>>(sp);
+    return cudaGetLastError() == cudaSuccess ? JFA_OK : JFA_ERR_CUDA;
+  }
   return launch_pdl(scan_kernel<KB, VB, NT>, dim3(n_ctas), dim3(Cfg::NW * 32), (size_t)Cfg::SMEM,
                     st, sp) == cudaSuccess
              ? JFA_OK
@@ -475,13 +507,15 @@ static int launch_scan_t(const ScanParams& sp, int n_ctas, cudaStream_t st) {
 }
 
 template <int KB, int VB>
-static int launch_scan_g(const ScanParams& sp, int n_ctas, cudaStream_t st) {
-  return sp.G > 4 ? launch_scan_t<KB, VB, 2>(sp, n_ctas, st) : launch_scan_t<KB, VB, 1>(sp, n_ctas, st);
+static int launch_scan_g(const ScanParams& sp, int n_ctas, bool pdl, cudaStream_t st) {
+  return sp.G > 4 ? launch_scan_t<KB, VB, 2>(sp, n_ctas, pdl, st)
+                  : launch_scan_t<KB, VB, 1>(sp, n_ctas, pdl, st);
 }
 
-int launch_scores(const jfa_geom& g, const jfa_cache& c, const uint16_t* q, float scale,
-                  uint8_t* ws, const jfa_workspace_layout& L, cudaStream_t st) {
-  ScanPlan plan = scan_plan(g, num_sms_current());
+int launch_scores(const jfa_geom& g, const SeqTable& t, const jfa_cache& c, const uint16_t* q,
+                  float scale, uint8_t* ws, const jfa_workspace_layout& L, cudaStream_t st,
+                  bool pdl) {
+  ScanPlan plan = scan_plan(g, t, num_sms_current());
   if (plan.total_groups == 0) return JFA_OK;
   ScanParams sp;
   sp.groups = static_cast<const uint8_t*>(c.groups);
@@ -493,18 +527,19 @@ int launch_scores(const jfa_geom& g, const jfa_cache& c, const uint16_t* q, floa
   sp.hist = reinterpret_cast<uint32_t*>(ws + L.off_scan_hist);
   sp.flag = reinterpret_cast<uint32_t*>(ws + L.off_flag);
   sp.total = plan.total_groups;
-  sp.ng = plan.ng;
   sp.ng_cap = g.capacity / kKG;
+  sp.n_seg = g.batch * g.num_kv_heads;
+  sp.seq = t;
   sp.capacity = g.capacity;
   sp.hkv = g.num_kv_heads;
   sp.G = g.num_heads / g.num_kv_heads;
   sp.H = g.num_heads;
   sp.n_warps = plan.n_warps;
   sp.kappa = scale * 1.4426950408889634f;
-  if (g.key_bits == 3 && g.val_bits == 2) return launch_scan_g<3, 2>(sp, plan.n_ctas, st);
-  if (g.key_bits == 4 && g.val_bits == 4) return launch_scan_g<4, 4>(sp, plan.n_ctas, st);
-  if (g.key_bits == 3 && g.val_bits == 4) return launch_scan_g<3, 4>(sp, plan.n_ctas, st);
-  if (g.key_bits == 4 && g.val_bits == 2) return launch_scan_g<4, 2>(sp, plan.n_ctas, st);
+  if (g.key_bits == 3 && g.val_bits == 2) return launch_scan_g<3, 2>(sp, plan.n_ctas, pdl, st);
+  if (g.key_bits == 4 && g.val_bits == 4) return launch_scan_g<4, 4>(sp, plan.n_ctas, pdl, st);
+  if (g.key_bits == 3 && g.val_bits == 4) return launch_scan_g<3, 4>(sp, plan.n_ctas, pdl, st);
+  if (g.key_bits == 4 && g.val_bits == 2) return launch_scan_g<4, 2>(sp, plan.n_ctas, pdl, st);
   return JFA_ERR_UNSUPPORTED;
 }
 

@@ -26,7 +26,9 @@
  *    out-of-range index handed to jfa_correct_merge, an exhausted bounded
  *    wait) set a flag word in the workspace; jfa_check_error reads it.
  *  - head_dim is 128; query heads per KV head G = H / H_kv must be 1..8.
- *  - All sequences of a batch hold the same number of tokens (n_ctx).
+ *  - The sequences of a batch hold geom->n_ctx tokens each, except in
+ *    jfa_decode_step_ragged and jfa_append_decode_step, which take a length
+ *    per sequence (at most JFA_MAX_BATCH sequences per call).
  */
 #ifndef JFA_H_
 #define JFA_H_
@@ -51,6 +53,7 @@ extern "C" {
 #define JFA_VAL_GROUP 32
 #define JFA_TAIL_MAX 64
 #define JFA_MAX_GQA 8
+#define JFA_MAX_BATCH 256     /* sequences per call                              */
 #define JFA_MAX_TOPK 4096
 #define JFA_MAX_EXACT 8192    /* exact tokens per segment jfa_correct_merge takes */
 #define JFA_BLOCK_TOKENS 128  /* tokens per block of jfa_topk_blocks             */
@@ -276,6 +279,42 @@ int jfa_decode_step(const jfa_geom* geom, const jfa_cache* cache,
                     const uint16_t* q, float scale, int32_t k, int32_t* idx,
                     const uint16_t* k_exact, const uint16_t* v_exact,
                     int32_t exact_on_host, void* ws, float* out, void* stream);
+
+/* jfa_decode_step_ragged — jfa_decode_step for a batch whose sequences hold
+ * different numbers of tokens (the decode steps on either side of the path:
+ * each sequence keeps its own quantized groups and bf16 tail; Jet-QSparse
+ * abstract: at most two BF16 pages per sequence and layer).
+ *   seq_lens : host int32[B], tokens cached per sequence, each in
+ *              [1, capacity]; geom->n_ctx is not used.  Sequence b splits into
+ *              N_q(b) = 64*floor((seq_lens[b]-1)/64) quantized tokens and a
+ *              tail of seq_lens[b] - N_q(b), and its top-k takes
+ *              min(k, N_q(b)) tokens.
+ * Other arguments as jfa_decode_step.  The lengths are read on the host when
+ * the call is made (they become launch arguments). */
+int jfa_decode_step_ragged(const jfa_geom* geom, const int32_t* seq_lens,
+                           const jfa_cache* cache, const uint16_t* q, float scale,
+                           int32_t k, int32_t* idx, const uint16_t* k_exact,
+                           const uint16_t* v_exact, int32_t exact_on_host, void* ws,
+                           float* out, void* stream);
+
+/* jfa_append_decode_step — one new token per sequence, then the decode step
+ * over the grown cache, in one call.  The new token of sequence b goes to
+ * position seq_lens[b]: into the bf16 tail, after the tail is first
+ * quantized as one 64-token group if it is full (HACK review, Figure 8: the
+ * last partial block stays in FP16, so an append never requantizes written
+ * codes), and into the exact copy.
+ *   seq_lens        : host int32[B], tokens cached before the append, each in
+ *                     [0, capacity - 1]; the caller adds one after the call.
+ *   k_new, v_new    : bf16 [B][H_kv][128] device pointers, 16-B aligned.
+ *   k_exact, v_exact: the exact copy (device or pinned host memory the device
+ *                     can address); row seq_lens[b] of every (sequence, KV
+ *                     head) is written here, then read like the others.
+ * Other arguments as jfa_decode_step (idx, out for the grown cache). */
+int jfa_append_decode_step(const jfa_geom* geom, const int32_t* seq_lens,
+                           const jfa_cache* cache, const uint16_t* k_new,
+                           const uint16_t* v_new, uint16_t* k_exact, uint16_t* v_exact,
+                           const uint16_t* q, float scale, int32_t k, int32_t* idx,
+                           int32_t exact_on_host, void* ws, float* out, void* stream);
 
 /* jfa_decode_finish — the rest of the step after jfa_decode_scores: top-k
  * selection, exact correction and merge in one kernel (a thread-block
