@@ -305,6 +305,157 @@ def topk_blocks(scores, n_blocks: int, block: int = BLOCK) -> np.ndarray:
 
 
 # ---------------------------------------------------------------------------
+# NVFP4 keys and FP4 scores (Jet-QSparse abstract: compact NVFP4 cache storage,
+# native FP4 query-key computation, then block selection and sparse FP16
+# value aggregation with FP32 accumulation)
+# ---------------------------------------------------------------------------
+FP4_BLOCK = 16                    # elements per UE4M3 block scale
+E2M1_MAX = 6.0
+E4M3_MAX = 448.0
+# the non-negative E2M1 values, by code 0..7 (sign bit 8)
+E2M1_GRID = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+
+
+def e2m1_round(v) -> np.ndarray:
+    """Codes (0..15, bit 3 = sign) of the E2M1 values nearest to v, ties to
+    the even code (the one whose mantissa bit is 0); |v| > 6 saturates."""
+    v = np.asarray(v, dtype=np.float64)
+    a = np.minimum(np.abs(v), E2M1_MAX)
+    d = np.abs(a[..., None] - E2M1_GRID)                  # distance to every grid value
+    best = d.min(axis=-1, keepdims=True)
+    cand = d == best
+    # among equally near values prefer an even code (mantissa bit 0)
+    even = cand & (np.arange(8) % 2 == 0)
+    code = np.where(even.any(axis=-1), np.argmax(even, axis=-1), np.argmax(cand, axis=-1))
+    sign = (v < 0) & (code > 0)
+    return (code + 8 * sign).astype(np.uint8)
+
+
+def e2m1_value(codes) -> np.ndarray:
+    codes = np.asarray(codes).astype(np.int64)
+    mag = E2M1_GRID[codes & 7]
+    return np.where(codes & 8, -mag, mag)
+
+
+def e4m3_values() -> np.ndarray:
+    """Every finite non-negative E4M3 value, ascending (bias 7, 3 mantissa
+    bits, subnormals below 2^-6; the largest finite value is 448)."""
+    vals = [m / 8 * 2.0 ** -6 for m in range(8)]
+    for e in range(1, 16):
+        for m in range(8):
+            if e == 15 and m == 7:       # the NaN encoding
+                continue
+            vals.append((1 + m / 8) * 2.0 ** (e - 7))
+    return np.array(vals)
+
+
+_E4M3 = e4m3_values()
+
+
+def e4m3_round_positive(v) -> np.ndarray:
+    """Nearest non-negative E4M3 value to v >= 0, ties to the even mantissa,
+    saturating at 448."""
+    v = np.minimum(np.asarray(v, dtype=np.float64), E4M3_MAX)
+    d = np.abs(v[..., None] - _E4M3)
+    best = d.min(axis=-1, keepdims=True)
+    cand = d == best
+    even = cand & (np.arange(_E4M3.size) % 2 == 0)      # code parity = mantissa parity
+    i = np.where(even.any(axis=-1), np.argmax(even, axis=-1), np.argmax(cand, axis=-1))
+    return _E4M3[i]
+
+
+def nvfp4_quantize(x, tensor_amax=None):
+    """NVFP4 of the rows of x [..., n] (n a multiple of 16): one fp32 scale
+    over the whole array, amax / (6 * 448) (stored as fp32; 1 when amax is
+    0), one UE4M3 scale per 16 consecutive elements of a row, the nearest
+    E4M3 to amax_block / (6 * s), and E2M1 codes of x / (block scale * s),
+    all quotients in fp64.  Returns (codes uint8 [..., n], block scales
+    fp64 [..., n/16], s float).  x_hat = e2m1 * block scale * s."""
+    x = np.asarray(x, dtype=np.float64)
+    amax = float(np.abs(x).max()) if tensor_amax is None else float(tensor_amax)
+    s = float(np.float32(amax / (E2M1_MAX * E4M3_MAX))) if amax > 0 else 1.0
+    *lead, n = x.shape
+    blocks = x.reshape(*lead, n // FP4_BLOCK, FP4_BLOCK)
+    bs = e4m3_round_positive(np.abs(blocks).max(axis=-1) / (E2M1_MAX * s))
+    with np.errstate(divide="ignore", invalid="ignore"):
+        q = blocks / (bs[..., None] * s)
+    q = np.where(bs[..., None] == 0, 0.0, q)
+    codes = e2m1_round(q).reshape(*lead, n)
+    return codes, bs, s
+
+
+def nvfp4_dequantize(codes, bs, s) -> np.ndarray:
+    codes = np.asarray(codes)
+    *lead, n = codes.shape
+    v = e2m1_value(codes).reshape(*lead, n // FP4_BLOCK, FP4_BLOCK)
+    return (v * np.asarray(bs, dtype=np.float64)[..., None] * s).reshape(*lead, n)
+
+
+def nvfp4_keys(k, n_quant: int):
+    """Keys [..., N, d] of one (sequence, KV head) list: every 64-token group
+    of the first n_quant tokens quantized with its own fp32 scale.  Returns
+    the dequantized keys [..., n_quant, d]."""
+    k = np.asarray(k, dtype=np.float64)[..., :n_quant, :]
+    out = np.zeros_like(k)
+    for g in range(n_quant // KEY_GROUP):
+        sl = slice(KEY_GROUP * g, KEY_GROUP * (g + 1))
+        blk = k[..., sl, :]
+        c, bs, s = nvfp4_quantize(blk)
+        out[..., sl, :] = nvfp4_dequantize(c, bs, s)
+    return out
+
+
+def nvfp4_scores(q, k, n_ctx: int, scale: float) -> np.ndarray:
+    """FP4 scores of every quantized token: scale * q_hat . k_hat with the
+    keys in NVFP4 per 64-token group and every query head in NVFP4 with its
+    own fp32 scale.  q [B, H, d], k [B, H_kv, >=N, d] -> [B, H, N_q]."""
+    q = np.asarray(q, dtype=np.float64)
+    b, h, d = q.shape
+    hkv = np.asarray(k).shape[1]
+    g = h // hkv
+    nq = split_point(n_ctx)
+    out = np.zeros((b, h, nq))
+    for bi in range(b):
+        for kv in range(hkv):
+            kh = nvfp4_keys(np.asarray(k)[bi, kv], nq)
+            for j in range(g):
+                hq = kv * g + j
+                cq, bq, sq = nvfp4_quantize(q[bi, hq][None])
+                qh = nvfp4_dequantize(cq, bq, sq)[0]
+                out[bi, hq] = scale * (kh @ qh)
+    return out
+
+
+def sparse_block_step(q, k_exact, v_exact, n_ctx: int, n_blocks: int, scale: float,
+                      idx=None):
+    """The Jet-QSparse step: FP4 scores, the n_blocks best 128-token blocks
+    per (sequence, KV head) by the largest score over the KV head's query
+    heads, and exact softmax attention over the chosen blocks' tokens plus
+    the bf16 tail (the other tokens are left out).  Returns (out [B, H, d],
+    idx [B, H_kv, n_blocks * 128], selection scores [B, H_kv, N_q])."""
+    q = np.asarray(q, dtype=np.float64)
+    ke = np.asarray(k_exact, dtype=np.float64)
+    ve = np.asarray(v_exact, dtype=np.float64)
+    b, h, d = q.shape
+    hkv = ke.shape[1]
+    g = h // hkv
+    nq = split_point(n_ctx)
+    sel = selection_scores(nvfp4_scores(q, ke, n_ctx, scale), hkv)
+    if idx is None:
+        idx = topk_blocks(sel, n_blocks)
+    out = np.zeros((b, h, d))
+    for bi in range(b):
+        for kv in range(hkv):
+            chosen = idx[bi, kv][idx[bi, kv] >= 0]
+            ex = np.concatenate([chosen, np.arange(nq, n_ctx)]).astype(np.int64)
+            for j in range(g):
+                hq = kv * g + j
+                out[bi, hq] = finish(softmax_partial(scale * (ke[bi, kv, ex] @ q[bi, hq]),
+                                                     ve[bi, kv, ex]))
+    return out, idx, sel
+
+
+# ---------------------------------------------------------------------------
 # Softmax partials and log-sum-exp merge
 # ---------------------------------------------------------------------------
 @dataclasses.dataclass

@@ -518,3 +518,168 @@ def test_pins_reject_block_mean_instead_of_max(monkeypatch):
     monkeypatch.setattr(O, "block_scores", mean_blocks)
     with pytest.raises(AssertionError):
         test_block_scores_are_block_maxima_by_brute_force()
+
+
+# --------------------------------------------------------------------------
+# NVFP4 keys and FP4 scores (Jet-QSparse abstract)
+# --------------------------------------------------------------------------
+import ml_dtypes  # noqa: E402  (independent library casts for the two minifloat formats)
+
+
+def _e2m1_library(x):
+    return np.asarray(x, dtype=np.float32).astype(ml_dtypes.float4_e2m1fn).astype(np.float64)
+
+
+def test_e2m1_rounding_matches_library_cast():
+    grid = O.E2M1_GRID
+    mids = (grid[1:] + grid[:-1]) / 2
+    x = np.concatenate([grid, mids, mids + 1e-6, mids - 1e-6, [6.5, 7.0, 100.0],
+                        np.linspace(0, 8, 4001)])
+    x = np.concatenate([x, -x])
+    assert np.array_equal(O.e2m1_value(O.e2m1_round(x)), _e2m1_library(x))
+
+
+def test_e4m3_values_and_rounding_match_library():
+    lib = np.arange(0x7F, dtype=np.uint8).view(ml_dtypes.float8_e4m3fn).astype(np.float64)
+    assert np.array_equal(O.e4m3_values(), lib)           # 0x00..0x7E, 0x7F is NaN
+    mids = (lib[1:] + lib[:-1]) / 2
+    x = np.concatenate([lib, mids, mids * (1 + 1e-6), mids * (1 - 1e-6),
+                        np.geomspace(1e-4, 448, 3000)])
+    want = x.astype(np.float32).astype(ml_dtypes.float8_e4m3fn).astype(np.float64)
+    assert np.array_equal(O.e4m3_round_positive(x), want)
+    assert O.e4m3_round_positive(1e4) == 448.0             # saturates
+
+
+def test_nvfp4_hand_case():
+    # one 16-element block with tensor amax 12: s = 12 / 2688 (as fp32), the
+    # block scale is the E4M3 nearest to 12 / (6 s) = 448, and x / (448 s) is
+    # x / 2 up to fp32 rounding of s: [6, -1.5, 0.35, 2.4, 0.6] -> E2M1
+    # [6, -1.5, 0.5, 2, 0.5], so x_hat = [12, -3, 1, 4, 1] up to that rounding
+    x = np.zeros(16)
+    x[:5] = [12.0, -3.0, 0.7, 4.8, 1.2]
+    codes, bs, s = O.nvfp4_quantize(x[None])
+    assert s == float(np.float32(12.0 / 2688.0))
+    assert bs.tolist() == [[448.0]]
+    assert O.e2m1_value(codes[0]).tolist()[:5] == [6.0, -1.5, 0.5, 2.0, 0.5]
+    xh = O.nvfp4_dequantize(codes, bs, s)[0]
+    assert np.allclose(xh[:5], [12.0, -3.0, 1.0, 4.0, 1.0], rtol=1e-6)
+    assert np.all(xh[5:] == 0)
+
+
+def _grid_block(rng, shape, unit):
+    """Values on the E2M1 grid times unit, every 16-block holding a +-6."""
+    v = rng.choice(np.concatenate([O.E2M1_GRID, -O.E2M1_GRID]), size=shape)
+    v[..., ::16] = 6.0 * rng.choice([-1.0, 1.0], size=v[..., ::16].shape)
+    return v * unit
+
+
+def test_nvfp4_grid_data_round_trips_exactly():
+    rng = np.random.default_rng(31)
+    # tensor amax 6 * 448 * 2^-10 gives s = 2^-10 and block scale 448 for
+    # blocks reaching the amax; a block reaching 6 * 28 * 2^-10 gets 28
+    x = _grid_block(rng, (64, 128), 448 * 2.0 ** -10)
+    x[3, 16:32] = _grid_block(rng, (16,), 28 * 2.0 ** -10)
+    codes, bs, s = O.nvfp4_quantize(x)
+    assert s == 2.0 ** -10
+    assert bs[3, 1] == 28.0 and bs[0, 0] == 448.0
+    assert np.array_equal(O.nvfp4_dequantize(codes, bs, s), x)
+
+
+def test_nvfp4_dequant_error_is_below_one_block_unit():
+    # |q - e2m1(q)| <= 1 for |q| <= 6 (the widest grid gap is 2), and the
+    # block scale is rounded so that |q| <= 6 (1 + 2^-4) / (1 - 2^-4) < 7:
+    # the error of every element is at most one unit bs * s of its block
+    rng = np.random.default_rng(32)
+    x = rng.standard_normal((64, 128))
+    x[:, [3, 77]] *= 30.0
+    x[5] *= 1e-3
+    codes, bs, s = O.nvfp4_quantize(x)
+    err = np.abs(x - O.nvfp4_dequantize(codes, bs, s))
+    unit = np.repeat(bs * s, 16, axis=-1)
+    assert np.all(err <= unit * (1 + 1e-12))
+    assert np.all(bs > 0) and np.all(bs <= 448)
+    # and the representable range is used: every block's largest |x_hat| is
+    # within an eighth of its largest |x|
+    xb = np.abs(x).reshape(64, 8, 16).max(-1)
+    xhb = np.abs(O.nvfp4_dequantize(codes, bs, s)).reshape(64, 8, 16).max(-1)
+    assert np.all(np.abs(xhb - xb) <= xb / 8)
+
+
+def test_nvfp4_scores_are_exact_on_grid_data():
+    # keys (per 64-token group) and queries (per head) exactly representable:
+    # the FP4 scores equal scale * q . k for every query head of the KV group
+    rng = np.random.default_rng(33)
+    b, h, hkv, n = 2, 6, 2, 200
+    unit = 448 * 2.0 ** -10
+    k = _grid_block(rng, (b, hkv, n, 128), unit)
+    q = _grid_block(rng, (b, h, 128), unit)
+    scale = 0.125
+    got = O.nvfp4_scores(q, k, n, scale)
+    nq = O.split_point(n)
+    for bi in range(b):
+        for hq in range(h):
+            want = scale * (k[bi, hq // 3, :nq] @ q[bi, hq])
+            assert np.array_equal(got[bi, hq], want)
+
+
+def _attend(q, keys, vals, scale):
+    t = torch.softmax(torch.as_tensor(keys) @ torch.as_tensor(q) * scale, 0)
+    return (t[:, None] * torch.as_tensor(vals)).sum(0).numpy()
+
+
+def _sparse_inputs(n=700, seed=34):
+    rng = np.random.default_rng(seed)
+    q = _bf16(rng.standard_normal((2, 4, 128)))
+    k = _bf16(rng.standard_normal((2, 2, n, 128)))
+    v = _bf16(rng.standard_normal((2, 2, n, 128)))
+    return q, k, v
+
+
+def test_sparse_step_with_every_block_is_exact_attention():
+    q, k, v = _sparse_inputs()
+    out, idx, _ = O.sparse_block_step(q, k, v, 700, 8, 0.09)
+    assert np.allclose(out, O.exact_attention(q, k, v, 700, 0.09), rtol=1e-12, atol=1e-13)
+    assert np.all(idx[..., :O.split_point(700)] >= 0)
+
+
+def test_sparse_step_with_no_block_is_attention_over_the_tail():
+    q, k, v = _sparse_inputs()
+    nq = O.split_point(700)
+    out, idx, _ = O.sparse_block_step(q, k, v, 700, 0, 0.09)
+    for bi in range(2):
+        for hq in range(4):
+            ref = _attend(q[bi, hq], k[bi, hq // 2, nq:700], v[bi, hq // 2, nq:700], 0.09)
+            assert np.allclose(out[bi, hq], ref, rtol=1e-12, atol=1e-13)
+
+
+def test_sparse_step_is_attention_over_chosen_blocks_and_tail():
+    q, k, v = _sparse_inputs()
+    nq = O.split_point(700)
+    out, idx, sel = O.sparse_block_step(q, k, v, 700, 2, 0.09)
+    assert np.array_equal(idx, O.topk_blocks(sel, 2))
+    for bi in range(2):
+        for hq in range(4):
+            h = hq // 2
+            toks = [t for t in idx[bi, h] if t >= 0] + list(range(nq, 700))
+            assert len(toks) == len(set(toks))
+            ref = _attend(q[bi, hq], k[bi, h, toks], v[bi, h, toks], 0.09)
+            assert np.allclose(out[bi, hq], ref, rtol=1e-12, atol=1e-13)
+
+
+def test_pins_reject_e2m1_ties_away_from_zero(monkeypatch):
+    def away(v):
+        v = np.asarray(v, dtype=np.float64)
+        a = np.minimum(np.abs(v), 6.0)
+        d = np.abs(a[..., None] - O.E2M1_GRID)
+        code = np.argmax(np.isclose(d, d.min(-1, keepdims=True)) * np.arange(8), axis=-1)
+        return (code + 8 * ((v < 0) & (code > 0))).astype(np.uint8)
+    monkeypatch.setattr(O, "e2m1_round", away)
+    with pytest.raises(AssertionError):
+        test_e2m1_rounding_matches_library_cast()
+
+
+def test_pins_reject_unscaled_fp4_scores(monkeypatch):
+    real = O.nvfp4_dequantize
+    monkeypatch.setattr(O, "nvfp4_dequantize", lambda c, bs, s: real(c, bs, 1.0))
+    with pytest.raises(AssertionError):
+        test_nvfp4_scores_are_exact_on_grid_data()
