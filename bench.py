@@ -46,6 +46,8 @@ def parse(argv=None):
     ap.add_argument("--no-per-config", action="store_true",
                     help="skip the K4V4 128K (HBM, host rows) and Qwen GQA-8 lines")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--only-fp4", action="store_true",
+                    help="print only the NVFP4 step lines (one JSON line per workload)")
     return ap.parse_args(argv)
 
 
@@ -611,6 +613,104 @@ def per_config_append(args, dev, name: str) -> dict:
     return d
 
 
+FP4_RECORD_BYTES = 9232    # NVFP4 keys of 128 tokens: codes, block scales, group scales
+
+
+def fp4_scan_bytes(w) -> int:
+    """Bytes the FP4 scan must read: every record of the N_q quantized
+    tokens (codes 64 B, block scales 8 B, group scales 1/16 B per token) and
+    the selection score it writes per token."""
+    n_seg = w.batch * w.kv_heads
+    return n_seg * (-(-w.n_quant // 128) * FP4_RECORD_BYTES + w.n_quant * 4)
+
+
+def fp4_step_bytes(w, n_blocks: int) -> int:
+    """FP4 step: the scan's bytes, the chosen blocks' exact K and V rows, the
+    tail rows, q and out."""
+    n_seg = w.batch * w.kv_heads
+    tail = w.ctx - w.n_quant
+    rows = min(n_blocks * 128, w.n_quant)
+    return fp4_scan_bytes(w) + n_seg * (rows + tail) * 512 + w.batch * w.heads * 128 * (2 + 4)
+
+
+def per_config_fp4(args, dev, name: str, n_blocks: int) -> dict:
+    """The NVFP4 step (Jet-QSparse abstract): jfa_fp4_decode_step = query
+    quantization, the tcgen05 FP4 scan, 128-token block selection and the
+    exact attention over the chosen blocks and the tail.  Copies of the key
+    pool (together larger than L2) and of the exact rows rotate."""
+    import torch
+
+    import bit_kv_cache_jfa_b200 as jfa
+    from bit_kv_cache_jfa_b200 import _lib
+    import workloads as W
+    w = W.WORKLOADS[name]
+    cap = 128 * -(-w.ctx // 128)
+    k_all, v_all = W.gen_kv_device(w, dev, W.gen_q(w))
+    q = W.gen_q(w).to(dev)
+    probe = jfa.FP4KeyPool(w.batch, w.heads, w.kv_heads, cap, device=dev)
+    n_copies = 1 + -(-L2_BYTES // probe.pool.numel())
+    ws = jfa.Workspace(probe, 64, device=dev)
+    del probe
+    copies = []
+    for c in range(n_copies):
+        pool = jfa.FP4KeyPool(w.batch, w.heads, w.kv_heads, cap, device=dev)
+        ke = torch.zeros(w.batch, w.kv_heads, cap, 128, dtype=torch.bfloat16, device=dev)
+        ve = torch.zeros_like(ke)
+        ke[:, :, :w.ctx], ve[:, :, :w.ctx] = k_all, v_all
+        pool.sync(ke, w.ctx, ws)
+        copies.append((pool, pool.geom(w.ctx), ke, ve))
+    del k_all, v_all
+    out = torch.empty(w.batch, w.heads, 128, dtype=torch.float32, device=dev)
+    idx = torch.empty(w.batch, w.kv_heads, n_blocks * 128, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sp = stream.cuda_stream
+    scale = W.default_scale(w)
+
+    def step(i):
+        pool, g, ke, ve = copies[i % n_copies]
+        _lib.check(_lib.jfa_fp4_decode_step(g, pool.pool, q, scale, n_blocks, idx, ke, ve, 0,
+                                            ws.buf, out, sp), "fp4_decode_step")
+
+    def scan(i):
+        pool, g, _, _ = copies[i % n_copies]
+        _lib.check(_lib.jfa_fp4_scores(g, pool.pool, q, scale, ws.buf, sp), "fp4_scores")
+
+    def timed(fn, steps, warm):
+        for i in range(warm):
+            fn(i)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for i in range(steps):
+            fn(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / steps
+
+    steps = max(20, min(args.steps, 200))
+    warm = max(3, args.warmup)
+    ms = timed(step, steps, warm)
+    scan_ms = timed(scan, steps, warm)
+    st, flag = _lib.jfa_check_error(copies[0][1], ws.buf, sp)
+    if flag:
+        raise RuntimeError(f"device error flag {flag:#x}")
+    peak, _ = measured_peaks()
+    alg = fp4_step_bytes(w, n_blocks)
+    d = {"workload": name, "format": "NVFP4 keys, exact bf16 rows",
+         "selection": f"{n_blocks} blocks of 128 tokens", "exact_rows": "hbm", "steps": steps,
+         "us_per_step": ms * 1e3, "tokens_per_s": w.batch * w.ctx / (ms / 1e3),
+         "step_frac": alg / (ms / 1e3) / 1e9 / peak, "step_alg_bytes": alg,
+         "scan_us": scan_ms * 1e3,
+         "scan_frac": fp4_scan_bytes(w) / (scan_ms / 1e3) / 1e9 / peak,
+         "scan_note": "jfa_fp4_scores: query records + the tcgen05 scan (two launches)",
+         "copies": n_copies,
+         "calls": "jfa_fp4_decode_step (query records, FP4 scan, block selection, sparse "
+                  "exact attention)"}
+    del copies, ws
+    torch.cuda.empty_cache()
+    return d
+
+
 def run_jfa(args, w):
     import torch
 
@@ -690,6 +790,8 @@ def run_jfa(args, w):
             per_config.append(per_config_line(args, dev, name, host))
         per_config.append(per_config_line(args, dev, "llama8b_k4v4_128k", False, n_blocks=64))
         per_config.append(per_config_append(args, dev, w.name))
+        for name in ("qwen30b_k3v2_32k", "llama8b_k4v4_128k"):
+            per_config.append(per_config_fp4(args, dev, name, 64))
 
     tokens = w.batch * w.ctx
     value = world * tokens / (ms_max / 1e3)
@@ -750,6 +852,14 @@ def main():
     w = workload_of(args)
     if args.impl == "reference":
         return run_reference(args, w)
+    if args.only_fp4:
+        import torch
+        dev = torch.device("cuda", dist_env()[2])
+        torch.cuda.set_device(dev)
+        names = [args.workload] if args.workload else ["qwen30b_k3v2_32k", "llama8b_k4v4_128k"]
+        for name in names:
+            print(json.dumps(per_config_fp4(args, dev, name, 64)), flush=True)
+        return 0
     return run_jfa(args, w)
 
 

@@ -18,11 +18,13 @@ from ._lib import (  # noqa: F401  (re-exported C ABI names)
     Cache, CacheLayout, Geom, JfaError, WorkspaceLayout, check, jfa_cache_layout_get,
     jfa_check_error, jfa_clear_error, jfa_correct_merge, jfa_decode_finish, jfa_decode_scores,
     jfa_append_decode_step, jfa_decode_step, jfa_decode_step_ragged,
-    jfa_decode_step_launches, jfa_pack_kv, jfa_topk, jfa_topk_blocks, jfa_unpack_record,
-    jfa_workspace_layout_get, load)
+    jfa_decode_step_launches, jfa_fp4_decode_step, jfa_fp4_pack_keys, jfa_fp4_pool_bytes,
+    jfa_fp4_scores, jfa_pack_kv, jfa_sparse_attend, jfa_topk, jfa_topk_blocks,
+    jfa_unpack_record, jfa_workspace_layout_get, load)
 
 __all__ = ["KVCache", "Workspace", "decode_step", "decode_step_blocks", "decode_step_ragged",
-           "append_decode_step", "DecodeGraph", "JfaError", "load"]
+           "append_decode_step", "FP4KeyPool", "fp4_decode_step", "sparse_attend", "DecodeGraph",
+           "JfaError", "load"]
 
 
 def _torch():
@@ -180,6 +182,77 @@ def append_decode_step(cache: KVCache, seq_lens, k_new, v_new, q, k: int, k_exac
                                  v_exact, q, float(scale), k, idx, exact_on_host, ws.buf, out,
                                  stream), "jfa_append_decode_step")
     return out, idx
+
+
+class FP4KeyPool:
+    """NVFP4 keys of one layer, one record per (sequence, KV head, 128-token
+    block), packed from the exact bf16 keys (device buffer owned by torch).
+    The geometry's key_bits / val_bits are not used by the FP4 calls."""
+
+    def __init__(self, batch: int, num_heads: int, num_kv_heads: int, capacity: int,
+                 device="cuda", head_dim: int = 128):
+        torch = _torch()
+        self.batch, self.num_heads, self.num_kv_heads = batch, num_heads, num_kv_heads
+        self.capacity, self.head_dim = capacity, head_dim
+        self.n_packed = 0
+        rc, nbytes = _lib.jfa_fp4_pool_bytes(self.geom(0))
+        check(rc, "jfa_fp4_pool_bytes")
+        self.pool = torch.zeros(nbytes, dtype=torch.uint8, device=device)
+
+    def geom(self, n_ctx: int = 0) -> Geom:
+        return Geom(self.batch, self.num_heads, self.num_kv_heads, self.head_dim, self.capacity,
+                    4, 4, n_ctx)
+
+    def pack(self, k_exact, n_to: int, ws: "Workspace", stream=None) -> None:
+        """Quantize the key groups from the packed length up to n_to (a
+        multiple of 64) from k_exact bf16 [B, H_kv, capacity, 128]."""
+        check(_lib.jfa_fp4_pack_keys(self.geom(n_to), self.n_packed, n_to, k_exact, self.pool,
+                                     ws.buf, stream), "jfa_fp4_pack_keys")
+        self.n_packed = max(self.n_packed, n_to)
+
+    def sync(self, k_exact, n_ctx: int, ws: "Workspace", stream=None) -> None:
+        """Pack every group below N_q of a context of n_ctx tokens."""
+        nq = 0 if n_ctx <= 0 else 64 * ((n_ctx - 1) // 64)
+        if nq > self.n_packed:
+            self.pack(k_exact, nq, ws, stream)
+
+
+def fp4_decode_step(pool: FP4KeyPool, n_ctx: int, q, n_blocks: int, k_exact, v_exact,
+                    ws: Workspace, scale=None, out=None, idx=None, exact_on_host: bool = False,
+                    stream=None):
+    """One NVFP4 decode step over n_ctx cached tokens (groups below N_q must
+    be packed): FP4 scan, the n_blocks best 128-token blocks, exact
+    attention over them and the tail.  Returns (out fp32 [B, H, 128], idx
+    int32 [B, H_kv, n_blocks * 128])."""
+    torch = _torch()
+    if scale is None:
+        scale = default_scale(pool.head_dim)
+    dev = q.device
+    if out is None:
+        out = torch.empty(pool.batch, pool.num_heads, pool.head_dim, dtype=torch.float32,
+                          device=dev)
+    if idx is None:
+        idx = torch.empty(pool.batch, pool.num_kv_heads, n_blocks * _lib.BLOCK_TOKENS,
+                          dtype=torch.int32, device=dev)
+    check(_lib.jfa_fp4_decode_step(pool.geom(n_ctx), pool.pool, q, float(scale), n_blocks, idx,
+                                   k_exact, v_exact, exact_on_host, ws.buf, out, stream),
+          "jfa_fp4_decode_step")
+    return out, idx
+
+
+def sparse_attend(geom: Geom, q, idx, k_exact, v_exact, ws: Workspace, scale=None, out=None,
+                  exact_on_host: bool = False, stream=None):
+    """Exact attention over the tokens idx [B, H_kv, k] (-1 = none) and the
+    tail [N_q, n_ctx) of every sequence; returns out fp32 [B, H, 128]."""
+    torch = _torch()
+    if scale is None:
+        scale = default_scale(geom.head_dim)
+    if out is None:
+        out = torch.empty(geom.batch, geom.num_heads, geom.head_dim, dtype=torch.float32,
+                          device=q.device)
+    check(_lib.jfa_sparse_attend(geom, q, float(scale), idx, idx.shape[-1], k_exact, v_exact,
+                                 exact_on_host, ws.buf, out, stream), "jfa_sparse_attend")
+    return out
 
 
 class DecodeGraph:

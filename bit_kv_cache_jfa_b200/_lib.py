@@ -60,6 +60,7 @@ class WorkspaceLayout(ctypes.Structure):
                 ("off_scan_hist", c_size_t),
                 ("off_hist", c_size_t), ("off_counters", c_size_t),
                 ("off_cand", c_size_t), ("off_sel", c_size_t),
+                ("off_fp4q", c_size_t), ("off_sparse", c_size_t), ("off_ticket", c_size_t),
                 ("max_topk", c_int32), ("partial_slots", c_int32), ("cand_cap", c_int32),
                 ("reserved", c_int32)]
 
@@ -100,6 +101,15 @@ SIGNATURES = {
     "jfa_decode_step_launches": (c_int32, [POINTER(Geom), c_int32]),
     "jfa_selftest_bounded_wait": (c_int32, [POINTER(Geom), c_void_p, c_void_p]),
     "jfa_scan_warps": (c_int32, [POINTER(Geom)]),
+    "jfa_fp4_pool_bytes": (c_int32, [POINTER(Geom), POINTER(c_size_t)]),
+    "jfa_fp4_pack_keys": (c_int32, [POINTER(Geom), c_int32, c_int32, c_void_p, c_void_p, c_void_p,
+                                    c_void_p]),
+    "jfa_fp4_scores": (c_int32, [POINTER(Geom), c_void_p, c_void_p, c_float, c_void_p, c_void_p]),
+    "jfa_sparse_attend": (c_int32, [POINTER(Geom), c_void_p, c_float, c_void_p, c_int32, c_void_p,
+                                    c_void_p, c_int32, c_void_p, c_void_p, c_void_p]),
+    "jfa_fp4_decode_step": (c_int32, [POINTER(Geom), c_void_p, c_void_p, c_float, c_int32,
+                                      c_void_p, c_void_p, c_void_p, c_int32, c_void_p, c_void_p,
+                                      c_void_p]),
 }
 
 _lib = None
@@ -204,6 +214,36 @@ def jfa_decode_step(geom, cache, q, scale, k, idx, k_exact, v_exact, exact_on_ho
     return load().jfa_decode_step(ctypes.byref(geom), ctypes.byref(cache), _ptr(q), scale, k,
                                   _ptr(idx), _ptr(k_exact), _ptr(v_exact), int(exact_on_host),
                                   _ptr(ws), _ptr(out), _stream(stream))
+
+
+def jfa_fp4_pool_bytes(geom) -> tuple[int, int]:
+    n = c_size_t(0)
+    rc = load().jfa_fp4_pool_bytes(ctypes.byref(geom), ctypes.byref(n))
+    return rc, n.value
+
+
+def jfa_fp4_pack_keys(geom, n_from, n_to, k_src, pool, ws, stream=None) -> int:
+    return load().jfa_fp4_pack_keys(ctypes.byref(geom), n_from, n_to, _ptr(k_src), _ptr(pool),
+                                    _ptr(ws), _stream(stream))
+
+
+def jfa_fp4_scores(geom, pool, q, scale, ws, stream=None) -> int:
+    return load().jfa_fp4_scores(ctypes.byref(geom), _ptr(pool), _ptr(q), scale, _ptr(ws),
+                                 _stream(stream))
+
+
+def jfa_sparse_attend(geom, q, scale, idx, k, k_exact, v_exact, exact_on_host, ws, out,
+                      stream=None) -> int:
+    return load().jfa_sparse_attend(ctypes.byref(geom), _ptr(q), scale, _ptr(idx), k,
+                                    _ptr(k_exact), _ptr(v_exact), int(exact_on_host), _ptr(ws),
+                                    _ptr(out), _stream(stream))
+
+
+def jfa_fp4_decode_step(geom, pool, q, scale, n_blocks, idx, k_exact, v_exact, exact_on_host, ws,
+                        out, stream=None) -> int:
+    return load().jfa_fp4_decode_step(ctypes.byref(geom), _ptr(pool), _ptr(q), scale, n_blocks,
+                                      _ptr(idx), _ptr(k_exact), _ptr(v_exact), int(exact_on_host),
+                                      _ptr(ws), _ptr(out), _stream(stream))
 
 
 def _lens(seq_lens):

@@ -2,7 +2,7 @@
 // layouts, launch plans and the host-side record decoder.
 #include <string.h>
 
-#include "jfa_internal.cuh"
+#include "jfa_fp4.cuh"
 
 namespace jfa {
 
@@ -58,6 +58,12 @@ int workspace_layout(const jfa_geom& g, int max_topk, jfa_workspace_layout* out)
   L.max_topk = max_topk;
   L.off_sel = off;
   off = align_up(off + n_seg * n_chunks_cap * sizeof(uint32_t), 256);
+  L.off_fp4q = off;
+  off = align_up(off + n_seg * kF4QBytes, 256);
+  L.off_sparse = off;
+  off = align_up(off + (n_seg > (size_t)kSpSlots ? n_seg : (size_t)kSpSlots) * kMaxG * 132 * sizeof(float), 256);
+  L.off_ticket = off;
+  off = align_up(off + n_seg * sizeof(uint32_t), 256);
   L.total_bytes = off;
   *out = L;
   return JFA_OK;
@@ -205,6 +211,86 @@ int jfa_topk_blocks(const jfa_geom* geom, int32_t n_blocks, void* ws, int32_t* i
   workspace_layout(*geom, 1, &L);
   return launch_topk_blocks(*geom, n_blocks, static_cast<uint8_t*>(ws), L, idx,
                             static_cast<cudaStream_t>(stream));
+}
+
+// ---------------------------------------------------------------------------
+// NVFP4 keys and block-sparse exact attention
+// ---------------------------------------------------------------------------
+static bool fp4_geom_ok(const jfa_geom* g) { return geom_ok(g) && g->capacity % kF4Tok == 0; }
+
+int jfa_fp4_pool_bytes(const jfa_geom* geom, size_t* pool_bytes) {
+  if (!fp4_geom_ok(geom) || !pool_bytes) return JFA_ERR_INVALID_ARG;
+  *pool_bytes = (size_t)geom->batch * geom->num_kv_heads * (geom->capacity / kF4Tok) * kF4RecBytes;
+  return JFA_OK;
+}
+
+int jfa_fp4_pack_keys(const jfa_geom* geom, int32_t n_from, int32_t n_to, const uint16_t* k_src,
+                      void* pool, void* ws, void* stream) {
+  if (!fp4_geom_ok(geom) || !pool || !aligned(pool, 16) || !ws || !aligned(ws, 256))
+    return JFA_ERR_INVALID_ARG;
+  if (n_from < 0 || n_to < n_from || n_to > geom->capacity || n_from % kKG || n_to % kKG)
+    return JFA_ERR_INVALID_ARG;
+  if (n_to == n_from) return JFA_OK;
+  if (!k_src || !aligned(k_src, 16)) return JFA_ERR_INVALID_ARG;
+  jfa_workspace_layout L;
+  workspace_layout(*geom, 1, &L);
+  return launch_fp4_pack(*geom, n_from / kKG, n_to / kKG, k_src, static_cast<uint8_t*>(pool),
+                         reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + L.off_flag),
+                         static_cast<cudaStream_t>(stream));
+}
+
+static bool fp4_scan_args_ok(const jfa_geom* geom, const void* pool, const uint16_t* q, float scale,
+                             const void* ws) {
+  return fp4_geom_ok(geom) && geom->n_ctx >= 1 && pool && aligned(pool, 16) && q && aligned(q, 16) &&
+         scale > 0.f && ws && aligned(ws, 256);
+}
+
+int jfa_fp4_scores(const jfa_geom* geom, const void* pool, const uint16_t* q, float scale, void* ws,
+                   void* stream) {
+  if (!fp4_scan_args_ok(geom, pool, q, scale, ws)) return JFA_ERR_INVALID_ARG;
+  jfa_workspace_layout L;
+  workspace_layout(*geom, 1, &L);
+  return launch_fp4_scores(*geom, static_cast<const uint8_t*>(pool), q, scale, static_cast<uint8_t*>(ws),
+                           L, static_cast<cudaStream_t>(stream));
+}
+
+static bool sparse_args_ok(const jfa_geom* geom, const uint16_t* q, float scale, const int32_t* idx,
+                           int32_t k, const uint16_t* k_exact, const uint16_t* v_exact, const void* ws,
+                           const float* out) {
+  return geom_ok(geom) && geom->n_ctx >= 1 && q && aligned(q, 16) && scale > 0.f && idx &&
+         aligned(idx, 4) && k >= 1 && k <= JFA_MAX_EXACT && k_exact && v_exact && aligned(k_exact, 16) &&
+         aligned(v_exact, 16) && ws && aligned(ws, 256) && out && aligned(out, 16);
+}
+
+int jfa_sparse_attend(const jfa_geom* geom, const uint16_t* q, float scale, const int32_t* idx,
+                      int32_t k, const uint16_t* k_exact, const uint16_t* v_exact,
+                      int32_t exact_on_host, void* ws, float* out, void* stream) {
+  if (!sparse_args_ok(geom, q, scale, idx, k, k_exact, v_exact, ws, out)) return JFA_ERR_INVALID_ARG;
+  jfa_workspace_layout L;
+  workspace_layout(*geom, 1, &L);
+  return launch_sparse_attend(*geom, q, scale, idx, k, k_exact, v_exact, exact_on_host != 0,
+                              static_cast<uint8_t*>(ws), L, out, static_cast<cudaStream_t>(stream));
+}
+
+int jfa_fp4_decode_step(const jfa_geom* geom, const void* pool, const uint16_t* q, float scale,
+                        int32_t n_blocks, int32_t* idx, const uint16_t* k_exact,
+                        const uint16_t* v_exact, int32_t exact_on_host, void* ws, float* out,
+                        void* stream) {
+  if (!fp4_scan_args_ok(geom, pool, q, scale, ws)) return JFA_ERR_INVALID_ARG;
+  if (n_blocks < 1 || n_blocks > JFA_MAX_BLOCKS) return JFA_ERR_INVALID_ARG;
+  const int k = n_blocks * JFA_BLOCK_TOKENS;
+  if (!sparse_args_ok(geom, q, scale, idx, k, k_exact, v_exact, ws, out)) return JFA_ERR_INVALID_ARG;
+  if ((split_point(geom->n_ctx) + JFA_BLOCK_TOKENS - 1) / JFA_BLOCK_TOKENS > kMaxSelBlocks)
+    return JFA_ERR_UNSUPPORTED;
+  jfa_workspace_layout L;
+  workspace_layout(*geom, 1, &L);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int rc = launch_fp4_scores(*geom, static_cast<const uint8_t*>(pool), q, scale, w, L, st);
+  if (rc == JFA_OK) rc = launch_topk_blocks(*geom, n_blocks, w, L, idx, st);
+  if (rc == JFA_OK)
+    rc = launch_sparse_attend(*geom, q, scale, idx, k, k_exact, v_exact, exact_on_host != 0, w, L, out, st);
+  return rc;
 }
 
 int jfa_correct_merge(const jfa_geom* geom, const jfa_cache* cache, const uint16_t* q,

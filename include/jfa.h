@@ -127,6 +127,11 @@ typedef struct jfa_workspace_layout {
   size_t off_counters;   /* top-k counters (jfa_topk)                         */
   size_t off_cand;       /* top-k candidate lists                             */
   size_t off_sel;        /* top-k per-chunk list lengths (jfa_topk)           */
+  size_t off_fp4q;       /* NVFP4 query records of jfa_fp4_scores, one per
+                            (sequence, KV head)                               */
+  size_t off_sparse;     /* split partials of jfa_sparse_attend              */
+  size_t off_ticket;     /* uint32 [B][H_kv] split counters of
+                            jfa_sparse_attend (zero between calls)           */
   int32_t max_topk;
   int32_t partial_slots; /* slots of off_partials                             */
   int32_t cand_cap;      /* list entries per segment                          */
@@ -218,11 +223,10 @@ int jfa_topk_blocks(const jfa_geom* geom, int32_t n_blocks, void* ws, int32_t* i
                     void* stream);
 
 /* jfa_topk_noalloc — the selection of jfa_topk for callers that cannot
- * allocate device memory: an inference-engine plugin whose execute callback
- * must not allocate, code between cudaStreamBeginCapture and EndCapture
- * (where cudaMalloc is not a stream operation and cannot be recorded), or a
- * latency-bound loop where an allocation would stall the device.  The pages
- * have no counterpart; it is a deployment convenience.
+ * allocate device memory, such as an inference-engine plugin whose execute
+ * callback must not allocate, or a latency-bound loop where an allocation
+ * would stall the device.  The pages have no counterpart; it is a
+ * deployment convenience.
  *   scores   : fp32 [n_seg][stride] device pointer, 16-B aligned; the first
  *              n_scores entries of each row are scored (n_scores % 4 == 0,
  *              stride % 4 == 0, stride >= n_scores).
@@ -232,8 +236,8 @@ int jfa_topk_blocks(const jfa_geom* geom, int32_t n_blocks, void* ws, int32_t* i
  * n_seg * ceil(n_scores / 4096) <= 64 (e.g. 8 rows of 32768 scores, 2 of
  * 131072); larger requests return JFA_ERR_UNSUPPORTED before any work.
  * The call allocates nothing.  Its first call on a device looks up the
- * array's device address (cudaGetSymbolAddress); make that first call
- * before any stream capture.  Every call clears the parts of the array that
+ * array's device address (cudaGetSymbolAddress).  Every call clears the
+ * parts of the array that
  * must start at zero and otherwise reuses the previous call's contents, so
  * calls that overlap on the GPU (other streams, other threads) race: keep
  * them on one stream. */
@@ -353,6 +357,81 @@ int jfa_unpack_record(int32_t key_bits, int32_t val_bits, const void* record,
 /* Number of kernel launches one jfa_decode_step issues for a geometry
  * (for launch accounting); 0 on a bad geometry. */
 int jfa_decode_step_launches(const jfa_geom* geom, int32_t k);
+
+/* ---------------------------------------------------------------------------
+ * NVFP4 keys and block-sparse exact attention (Jet-QSparse abstract: compact
+ * NVFP4 cache storage, query-key products in FP4 on Blackwell tensor cores,
+ * a dense scan over the whole key history that selects 128-token blocks, and
+ * the value aggregation over those blocks in high precision with FP32
+ * accumulation).
+ *
+ * NVFP4 here: E2M1 elements (0, 0.5, 1, 1.5, 2, 3, 4, 6 and negatives), a
+ * UE4M3 scale per 16 consecutive channels of a row, and an fp32 tensor scale
+ * s = amax / (6 * 448) (1 when amax is 0) per 64-token key group, or per
+ * query head for the query.  Block scale = the UE4M3 value nearest to
+ * amax_16 / (6 s) (ties to even, at most 448); code = the E2M1 value nearest
+ * to x / (block scale * s) (ties to even, saturating at 6); both quotients in
+ * fp64.  The score of a token for a query head is
+ *   scale * s_k s_q * sum_c (e2m1_k bs_k)(e2m1_q bs_q),
+ * accumulated in fp32 by the tensor cores, and its selection score the
+ * largest over the KV head's query heads.
+ *
+ * Geometry: jfa_geom with capacity a multiple of 128; key_bits and val_bits
+ * are not used by these calls (any valid pair).  The workspace is the one
+ * jfa_workspace_layout_get sizes (zero-filled once).  Errors as above.
+ * ------------------------------------------------------------------------- */
+#define JFA_FP4_RECORD_BYTES 9232 /* bytes per (sequence, KV head, 128-token block) */
+
+/* NVFP4 key pool: B * H_kv * capacity/128 records of JFA_FP4_RECORD_BYTES,
+ * [B][H_kv][capacity/128][record], in a layout private to this library
+ * (E2M1 codes in the tensor core's operand order, the block scales as
+ * scale-factor atoms, the two group scales).  Caller-allocated, 16-byte
+ * aligned.  Returns the pool size in *pool_bytes. */
+int jfa_fp4_pool_bytes(const jfa_geom* geom, size_t* pool_bytes);
+
+/* Quantize the 64-token key groups covering tokens [n_from, n_to) of every
+ * (sequence, KV head) into the pool, from the exact bf16 keys
+ *   k_src : [B][H_kv][capacity][128] (device, or pinned host memory)
+ * (the persistent cache packed straight from the BF16 activations).
+ * n_from, n_to multiples of 64, 0 <= n_from <= n_to <= capacity.  Groups
+ * already written are never rewritten.  A non-finite key sets
+ * JFA_DEVERR_NONFINITE_QUANT.  Stream-ordered. */
+int jfa_fp4_pack_keys(const jfa_geom* geom, int32_t n_from, int32_t n_to, const uint16_t* k_src,
+                      void* pool, void* ws, void* stream);
+
+/* FP4 scan: quantize q (bf16 [B][H][128], device) to NVFP4 per head and
+ * compute the selection score of each of the N_q = 64 floor((n_ctx-1)/64)
+ * quantized tokens (every group below N_q must have been packed) into the
+ * workspace's score array, where jfa_topk / jfa_topk_blocks read it.  Two
+ * launches (query records, then the tcgen05 scan).  Stream-ordered. */
+int jfa_fp4_scores(const jfa_geom* geom, const void* pool, const uint16_t* q, float scale,
+                   void* ws, void* stream);
+
+/* Exact attention over an index set and the tail, nothing else:
+ *   out[b, h] = softmax over T of (scale q_h . k_t) applied to v_t,
+ *   T = {idx[b, h/G, j] >= 0, j < k} + {N_q, ..., n_ctx - 1},
+ * with k_t, v_t rows of the exact bf16 copy
+ *   k_exact, v_exact : [B][H_kv][capacity][128] (device, or pinned host with
+ *                      exact_on_host = 1; read by zero-copy loads)
+ *   idx              : int32 [B][H_kv][k] (device), -1 = no token; an entry
+ *                      outside [-1, N_q) sets JFA_DEVERR_BAD_INDEX and is
+ *                      skipped; indices must be distinct
+ *   out              : fp32 [B][H][128] (device)
+ * 1 <= k <= JFA_MAX_EXACT.  Logits in fp32 from bf16 products, softmax
+ * weights carried at about 16 bits into an fp32 accumulation.  One launch.
+ * Stream-ordered. */
+int jfa_sparse_attend(const jfa_geom* geom, const uint16_t* q, float scale, const int32_t* idx,
+                      int32_t k, const uint16_t* k_exact, const uint16_t* v_exact,
+                      int32_t exact_on_host, void* ws, float* out, void* stream);
+
+/* The NVFP4 decode step: jfa_fp4_scores, jfa_topk_blocks (the n_blocks best
+ * 128-token blocks per (sequence, KV head), written to idx int32
+ * [B][H_kv][n_blocks * 128]) and jfa_sparse_attend over them and the tail.
+ * Four launches.  Stream-ordered. */
+int jfa_fp4_decode_step(const jfa_geom* geom, const void* pool, const uint16_t* q, float scale,
+                        int32_t n_blocks, int32_t* idx, const uint16_t* k_exact,
+                        const uint16_t* v_exact, int32_t exact_on_host, void* ws, float* out,
+                        void* stream);
 
 /* Number of warps jfa_decode_scores splits the quantized groups over on the
  * current device (0 on a bad geometry or when no group is quantized).  Warp w

@@ -22,7 +22,7 @@ def lib():
 def header_symbols():
     text = open(os.path.join(ROOT, "include", "jfa.h")).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(jfa_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(jfa_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_exports_every_declared_symbol(lib):
@@ -63,7 +63,8 @@ def test_workspace_layout(lib):
     assert b.total_bytes >= a.total_bytes and b.max_topk == 4096
     for L in (a, b):
         offs = [L.off_flag, L.off_scores, L.off_partials, L.off_mused, L.off_wts,
-                L.off_scan_hist, L.off_hist, L.off_cand, L.off_sel]
+                L.off_scan_hist, L.off_hist, L.off_cand, L.off_sel, L.off_fp4q, L.off_sparse,
+                L.off_ticket, L.total_bytes]
         assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
         assert L.off_counters == L.off_hist + 4 * 4 * 2048
         assert L.off_scores + 4 * 4 * 4096 <= L.off_partials
@@ -150,3 +151,22 @@ def test_topk_blocks_rejects_bad_block_counts(lib):
         assert lib.jfa_topk_blocks(g, n, ws, idx) == lib.JFA_ERR_INVALID_ARG
     assert lib.jfa_topk_blocks(g, 4, 0, idx) == lib.JFA_ERR_INVALID_ARG
     assert lib.jfa_topk_blocks(g, 4, ws, 0) == lib.JFA_ERR_INVALID_ARG
+
+
+def test_fp4_pool_size_and_argument_checks(lib):
+    rc, n = lib.jfa_fp4_pool_bytes(G(capacity=4096))
+    assert rc == 0 and n == 2 * 2 * 32 * 9232
+    rc, _ = lib.jfa_fp4_pool_bytes(G(capacity=4096 + 64))   # not a multiple of 128
+    assert rc == lib.JFA_ERR_INVALID_ARG
+    g = G(capacity=4096, n_ctx=1000)
+    bad = lib.JFA_ERR_INVALID_ARG
+    assert lib.jfa_fp4_pack_keys(g, 0, 100, 256, 256, 256) == bad            # not a group edge
+    assert lib.jfa_fp4_pack_keys(g, 128, 64, 256, 256, 256) == bad           # n_to < n_from
+    assert lib.jfa_fp4_pack_keys(g, 0, 4160, 256, 256, 256) == bad           # past capacity
+    assert lib.jfa_fp4_pack_keys(g, 64, 64, 256, 256, 256) == 0              # nothing to do
+    assert lib.jfa_fp4_scores(g, 256, 256, 0.0, 256) == bad                  # scale
+    assert lib.jfa_fp4_scores(g, 8, 256, 0.1, 256) == bad                    # pool alignment
+    assert lib.jfa_sparse_attend(g, 256, 0.1, 256, 0, 256, 256, 0, 256, 256) == bad   # k = 0
+    assert lib.jfa_sparse_attend(g, 256, 0.1, 256, 8193, 256, 256, 0, 256, 256) == bad
+    assert lib.jfa_fp4_decode_step(g, 256, 256, 0.1, 0, 256, 256, 256, 0, 256, 256) == bad
+    assert lib.jfa_fp4_decode_step(g, 256, 256, 0.1, 65, 256, 256, 256, 0, 256, 256) == bad
