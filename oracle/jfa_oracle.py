@@ -456,6 +456,83 @@ def sparse_block_step(q, k_exact, v_exact, n_ctx: int, n_blocks: int, scale: flo
 
 
 # ---------------------------------------------------------------------------
+# Critical-channel scores (TailorKV review: a channel's importance is the
+# product of the query's magnitude in it and the largest key magnitude in it,
+# s_i = |q_i| * max|K_i|; approximate attention scores from the critical
+# channels pick the top-k tokens, which are then fetched and attended exactly)
+# ---------------------------------------------------------------------------
+def channel_importance(q, k, n_quant: int) -> np.ndarray:
+    """Per (sequence, KV head) and channel: the largest |q_i| over the KV
+    head's query heads times the largest |K_{t,i}| over the quantized tokens
+    t < n_quant.  q [B, H, d], k [B, H_kv, >=n_quant, d] -> [B, H_kv, d]."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    b, h, d = q.shape
+    hkv = k.shape[1]
+    qmax = np.abs(q).reshape(b, hkv, h // hkv, d).max(axis=2)
+    kmax = np.abs(k[:, :, :n_quant]).max(axis=2) if n_quant > 0 else np.zeros((b, hkv, d))
+    return qmax * kmax
+
+
+def critical_channels(importance, r: int) -> np.ndarray:
+    """The r most important channels per row (importance descending, channel
+    index ascending on ties), sorted ascending.  [..., d] -> int [..., r]."""
+    return topk_indices(importance, r)
+
+
+def channel_scores(q, k, n_ctx: int, r: int, scale: float) -> np.ndarray:
+    """Selection scores from the r critical channels of each KV head: for
+    every quantized token t < N_q the largest over the KV head's query heads
+    of scale * sum over the critical channels i of q_{h,i} K_{t,i}.
+    -> [B, H_kv, N_q]."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    b, h, d = q.shape
+    hkv = k.shape[1]
+    g = h // hkv
+    nq = split_point(n_ctx)
+    chans = critical_channels(channel_importance(q, k, nq), r)
+    out = np.zeros((b, hkv, nq))
+    for bi in range(b):
+        for kv in range(hkv):
+            c = chans[bi, kv]
+            keys = k[bi, kv, :nq][:, c]                       # [N_q, r]
+            per_head = [scale * (keys @ q[bi, kv * g + j, c]) for j in range(g)]
+            out[bi, kv] = np.max(per_head, axis=0) if nq else out[bi, kv]
+    return out
+
+
+def attend_set(q, k_exact, v_exact, n_ctx: int, idx, scale: float) -> np.ndarray:
+    """Exact softmax attention of every query head over the tokens idx[b,
+    h_kv] (entries >= 0) and the tail N_q .. n_ctx - 1, nothing else."""
+    q = np.asarray(q, dtype=np.float64)
+    ke = np.asarray(k_exact, dtype=np.float64)
+    ve = np.asarray(v_exact, dtype=np.float64)
+    b, h, d = q.shape
+    hkv = ke.shape[1]
+    g = h // hkv
+    nq = split_point(n_ctx)
+    out = np.zeros((b, h, d))
+    for bi in range(b):
+        for kv in range(hkv):
+            chosen = idx[bi, kv][idx[bi, kv] >= 0]
+            ex = np.concatenate([chosen, np.arange(nq, n_ctx)]).astype(np.int64)
+            for j in range(g):
+                hq = kv * g + j
+                out[bi, hq] = finish(softmax_partial(scale * (ke[bi, kv, ex] @ q[bi, hq]),
+                                                     ve[bi, kv, ex]))
+    return out
+
+
+def channel_step(q, k_exact, v_exact, n_ctx: int, r: int, k: int, scale: float):
+    """Critical-channel scores, the top-k tokens per (sequence, KV head), and
+    exact attention over them and the tail.  Returns (out, idx, scores)."""
+    sel = channel_scores(q, k_exact, n_ctx, r, scale)
+    idx = topk_indices(sel, k)
+    return attend_set(q, k_exact, v_exact, n_ctx, idx, scale), idx, sel
+
+
+# ---------------------------------------------------------------------------
 # Softmax partials and log-sum-exp merge
 # ---------------------------------------------------------------------------
 @dataclasses.dataclass

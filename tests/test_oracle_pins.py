@@ -683,3 +683,79 @@ def test_pins_reject_unscaled_fp4_scores(monkeypatch):
     monkeypatch.setattr(O, "nvfp4_dequantize", lambda c, bs, s: real(c, bs, 1.0))
     with pytest.raises(AssertionError):
         test_nvfp4_scores_are_exact_on_grid_data()
+
+
+# --------------------------------------------------------------------------
+# critical-channel scores (TailorKV review)
+# --------------------------------------------------------------------------
+def test_all_channels_give_the_exact_logits():
+    # r = d: the channel scores are the exact logits, max over the group's heads
+    q, k, v = _sparse_inputs(n=300, seed=41)
+    nq = O.split_point(300)
+    got = O.channel_scores(q, k, 300, 128, 0.07)
+    for bi in range(2):
+        for h in range(2):
+            t = torch.as_tensor(k[bi, h, :nq]) @ torch.as_tensor(q[bi, 2 * h:2 * h + 2]).T
+            assert np.allclose(got[bi, h], 0.07 * t.max(1).values.numpy(), rtol=1e-13, atol=1e-13)
+
+
+def test_critical_channels_brute_force_with_ties():
+    rng = np.random.default_rng(42)
+    for _ in range(20):
+        imp = rng.integers(0, 4, 128).astype(np.float64)
+        r = int(rng.integers(1, 129))
+        want = sorted(sorted(range(128), key=lambda c: (-imp[c], c))[:r])
+        assert O.critical_channels(imp[None], r)[0].tolist() == want
+
+
+def test_channel_scores_hand_case():
+    # one sequence, one KV head, two query heads; channel 3: |q| max 2,
+    # max|K| 1 -> 2; channel 7: |q| max 5 (a negative query), max|K| 0.5 ->
+    # 2.5; channel 9: |q| 1, max|K| 4 -> 4.  r = 2 keeps channels 7 and 9.
+    q = np.zeros((1, 2, 128))
+    q[0, 0, 3], q[0, 1, 3] = 2.0, 1.0
+    q[0, 0, 7], q[0, 1, 7] = -5.0, 1.0
+    q[0, 0, 9], q[0, 1, 9] = 1.0, 0.5
+    k = np.zeros((1, 1, 129, 128))
+    k[0, 0, 0, 3], k[0, 0, 1, 7], k[0, 0, 2, 9], k[0, 0, 5, 9] = 1.0, -0.5, 4.0, -2.0
+    imp = O.channel_importance(q, k, 128)[0, 0]
+    assert (imp[3], imp[7], imp[9]) == (2.0, 2.5, 4.0)
+    assert O.critical_channels(imp[None], 2)[0].tolist() == [7, 9]
+    s = O.channel_scores(q, k, 129, 2, 1.0)[0, 0]
+    # token 1: head 0 gives -5 * -0.5 = 2.5, head 1 gives -0.5; token 2:
+    # 1 * 4 = 4 and 0.5 * 4 = 2; token 5: -2 and -1; token 0 (channel 3 is
+    # not critical): 0
+    assert (s[0], s[1], s[2], s[5]) == (0.0, 2.5, 4.0, -1.0)
+
+
+def test_channel_step_with_every_token_is_exact_attention():
+    q, k, v = _sparse_inputs(n=300, seed=43)
+    out, idx, _ = O.channel_step(q, k, v, 300, 16, 256, 0.09)
+    assert np.all(idx >= 0)
+    assert np.allclose(out, O.exact_attention(q, k, v, 300, 0.09), rtol=1e-12, atol=1e-13)
+
+
+def test_attend_set_matches_torch_attention():
+    q, k, v = _sparse_inputs(n=300, seed=44)
+    nq = O.split_point(300)
+    rng = np.random.default_rng(45)
+    idx = np.full((2, 2, 40), -1, np.int32)
+    idx[..., :30] = rng.choice(nq, 30, replace=False)
+    out = O.attend_set(q, k, v, 300, idx, 0.09)
+    for bi in range(2):
+        for hq in range(4):
+            toks = list(idx[bi, hq // 2, :30]) + list(range(nq, 300))
+            ref = _attend(q[bi, hq], k[bi, hq // 2, toks], v[bi, hq // 2, toks], 0.09)
+            assert np.allclose(out[bi, hq], ref, rtol=1e-12, atol=1e-13)
+
+
+def test_pins_reject_signed_channel_importance(monkeypatch):
+    def signed(q, k, n_quant):
+        q = np.asarray(q, dtype=np.float64)
+        k = np.asarray(k, dtype=np.float64)
+        b, h, d = q.shape
+        hkv = k.shape[1]
+        return q.reshape(b, hkv, h // hkv, d).max(axis=2) * np.abs(k[:, :, :n_quant]).max(axis=2)
+    monkeypatch.setattr(O, "channel_importance", signed)
+    with pytest.raises(AssertionError):
+        test_channel_scores_hand_case()
