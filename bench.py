@@ -48,6 +48,8 @@ def parse(argv=None):
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--only-fp4", action="store_true",
                     help="print only the NVFP4 step lines (one JSON line per workload)")
+    ap.add_argument("--only-channel", action="store_true",
+                    help="print only the critical-channel step line of the workload")
     return ap.parse_args(argv)
 
 
@@ -711,6 +713,86 @@ def per_config_fp4(args, dev, name: str, n_blocks: int) -> dict:
     return d
 
 
+def per_config_channel(args, dev, name: str, r: int) -> dict:
+    """Critical-channel selection (TailorKV review): jfa_channel_decode_step =
+    scores over the r most important channels of a channel-major key copy,
+    top-k, exact attention over the chosen tokens and the tail.  Copies of
+    the channel-major keys and of the exact rows rotate (together > L2)."""
+    import torch
+
+    import bit_kv_cache_jfa_b200 as jfa
+    from bit_kv_cache_jfa_b200 import _lib
+    import workloads as W
+    w = W.WORKLOADS[name]
+    cap = 64 * -(-w.ctx // 64)
+    k_all, v_all = W.gen_kv_device(w, dev, W.gen_q(w))
+    q = W.gen_q(w).to(dev)
+    n_seg = w.batch * w.kv_heads
+    scan_bytes = n_seg * w.n_quant * 2 * r
+    n_copies = 1 + -(-L2_BYTES // max(1, n_seg * w.n_quant * 2 * 128))
+    copies = []
+    ws = None
+    for c in range(n_copies):
+        keys = jfa.ChannelKeys(w.batch, w.heads, w.kv_heads, cap, device=dev)
+        if ws is None:
+            ws = jfa.Workspace(keys, w.topk, device=dev)
+        ke = torch.zeros(w.batch, w.kv_heads, cap, 128, dtype=torch.bfloat16, device=dev)
+        ve = torch.zeros_like(ke)
+        ke[:, :, :w.ctx], ve[:, :, :w.ctx] = k_all, v_all
+        keys.sync(ke, w.ctx)
+        copies.append((keys, keys.geom(w.ctx), ke, ve))
+    del k_all, v_all
+    out = torch.empty(w.batch, w.heads, 128, dtype=torch.float32, device=dev)
+    idx = torch.empty(w.batch, w.kv_heads, w.topk, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sp = stream.cuda_stream
+    scale = W.default_scale(w)
+
+    def step(i):
+        keys, g, ke, ve = copies[i % n_copies]
+        _lib.check(_lib.jfa_channel_decode_step(g, keys.k_t, keys.k_max, q, scale, r, w.topk, idx,
+                                                ke, ve, 0, ws.buf, out, sp), "channel_step")
+
+    def scan(i):
+        keys, g, _, _ = copies[i % n_copies]
+        _lib.check(_lib.jfa_channel_scores(g, keys.k_t, keys.k_max, q, scale, r, ws.buf, sp),
+                   "channel_scores")
+
+    def timed(fn, steps, warm):
+        for i in range(warm):
+            fn(i)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for i in range(steps):
+            fn(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / steps
+
+    steps = max(20, min(args.steps, 200))
+    warm = max(3, args.warmup)
+    ms = timed(step, steps, warm)
+    scan_ms = timed(scan, steps, warm)
+    st, flag = _lib.jfa_check_error(copies[0][1], ws.buf, sp)
+    if flag:
+        raise RuntimeError(f"device error flag {flag:#x}")
+    peak, _ = measured_peaks()
+    tail = w.ctx - w.n_quant
+    alg = (scan_bytes + n_seg * (min(w.topk, w.n_quant) + tail) * 512
+           + w.batch * w.heads * 128 * (2 + 4))
+    d = {"workload": name, "format": f"bf16 channel-major keys, {r} critical channels",
+         "selection": f"top-{w.topk} tokens", "exact_rows": "hbm", "steps": steps,
+         "us_per_step": ms * 1e3, "tokens_per_s": w.batch * w.ctx / (ms / 1e3),
+         "step_frac": alg / (ms / 1e3) / 1e9 / peak, "step_alg_bytes": alg,
+         "scan_us": scan_ms * 1e3, "scan_frac": scan_bytes / (scan_ms / 1e3) / 1e9 / peak,
+         "copies": n_copies,
+         "calls": "jfa_channel_decode_step (channel scores, top-k, sparse exact attention)"}
+    del copies, ws
+    torch.cuda.empty_cache()
+    return d
+
+
 def run_jfa(args, w):
     import torch
 
@@ -792,6 +874,7 @@ def run_jfa(args, w):
         per_config.append(per_config_append(args, dev, w.name))
         for name in ("qwen30b_k3v2_32k", "llama8b_k4v4_128k"):
             per_config.append(per_config_fp4(args, dev, name, 64))
+        per_config.append(per_config_channel(args, dev, w.name, 16))
 
     tokens = w.batch * w.ctx
     value = world * tokens / (ms_max / 1e3)
@@ -852,6 +935,12 @@ def main():
     w = workload_of(args)
     if args.impl == "reference":
         return run_reference(args, w)
+    if args.only_channel:
+        import torch
+        dev = torch.device("cuda", dist_env()[2])
+        torch.cuda.set_device(dev)
+        print(json.dumps(per_config_channel(args, dev, w.name, 16)), flush=True)
+        return 0
     if args.only_fp4:
         import torch
         dev = torch.device("cuda", dist_env()[2])

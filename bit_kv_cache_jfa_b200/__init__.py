@@ -18,13 +18,14 @@ from ._lib import (  # noqa: F401  (re-exported C ABI names)
     Cache, CacheLayout, Geom, JfaError, WorkspaceLayout, check, jfa_cache_layout_get,
     jfa_check_error, jfa_clear_error, jfa_correct_merge, jfa_decode_finish, jfa_decode_scores,
     jfa_append_decode_step, jfa_decode_step, jfa_decode_step_ragged,
+    jfa_channel_decode_step, jfa_channel_pack, jfa_channel_scores,
     jfa_decode_step_launches, jfa_fp4_decode_step, jfa_fp4_pack_keys, jfa_fp4_pool_bytes,
     jfa_fp4_scores, jfa_pack_kv, jfa_sparse_attend, jfa_topk, jfa_topk_blocks,
     jfa_unpack_record, jfa_workspace_layout_get, load)
 
 __all__ = ["KVCache", "Workspace", "decode_step", "decode_step_blocks", "decode_step_ragged",
-           "append_decode_step", "FP4KeyPool", "fp4_decode_step", "sparse_attend", "DecodeGraph",
-           "JfaError", "load"]
+           "append_decode_step", "FP4KeyPool", "fp4_decode_step", "sparse_attend",
+           "ChannelKeys", "channel_decode_step", "DecodeGraph", "JfaError", "load"]
 
 
 def _torch():
@@ -253,6 +254,55 @@ def sparse_attend(geom: Geom, q, idx, k_exact, v_exact, ws: Workspace, scale=Non
     check(_lib.jfa_sparse_attend(geom, q, float(scale), idx, idx.shape[-1], k_exact, v_exact,
                                  exact_on_host, ws.buf, out, stream), "jfa_sparse_attend")
     return out
+
+
+class ChannelKeys:
+    """Channel-major bf16 copy of one layer's keys and the per-channel max|K|
+    (device buffers owned by torch), for the critical-channel selection."""
+
+    def __init__(self, batch: int, num_heads: int, num_kv_heads: int, capacity: int,
+                 device="cuda", head_dim: int = 128):
+        torch = _torch()
+        self.batch, self.num_heads, self.num_kv_heads = batch, num_heads, num_kv_heads
+        self.capacity, self.head_dim = capacity, head_dim
+        self.n_packed = 0
+        self.k_t = torch.zeros(batch, num_kv_heads, head_dim, capacity, dtype=torch.bfloat16,
+                               device=device)
+        self.k_max = torch.zeros(batch, num_kv_heads, head_dim, dtype=torch.float32,
+                                 device=device)
+
+    def geom(self, n_ctx: int = 0) -> Geom:
+        return Geom(self.batch, self.num_heads, self.num_kv_heads, self.head_dim, self.capacity,
+                    4, 4, n_ctx)
+
+    def sync(self, k_exact, n_ctx: int, stream=None) -> None:
+        """Copy every group below N_q of a context of n_ctx tokens."""
+        nq = 0 if n_ctx <= 0 else 64 * ((n_ctx - 1) // 64)
+        if nq > self.n_packed:
+            check(_lib.jfa_channel_pack(self.geom(nq), self.n_packed, nq, k_exact, self.k_t,
+                                        self.k_max, stream), "jfa_channel_pack")
+            self.n_packed = nq
+
+
+def channel_decode_step(keys: ChannelKeys, n_ctx: int, q, r: int, k: int, k_exact, v_exact,
+                        ws: Workspace, scale=None, out=None, idx=None, exact_on_host: bool = False,
+                        stream=None):
+    """One decode step with critical-channel selection: scores over the r
+    most important channels, the top-k tokens, exact attention over them and
+    the tail.  Returns (out fp32 [B, H, 128], idx int32 [B, H_kv, k])."""
+    torch = _torch()
+    if scale is None:
+        scale = default_scale(keys.head_dim)
+    dev = q.device
+    if out is None:
+        out = torch.empty(keys.batch, keys.num_heads, keys.head_dim, dtype=torch.float32,
+                          device=dev)
+    if idx is None:
+        idx = torch.empty(keys.batch, keys.num_kv_heads, k, dtype=torch.int32, device=dev)
+    check(_lib.jfa_channel_decode_step(keys.geom(n_ctx), keys.k_t, keys.k_max, q, float(scale), r,
+                                       k, idx, k_exact, v_exact, exact_on_host, ws.buf, out,
+                                       stream), "jfa_channel_decode_step")
+    return out, idx
 
 
 class DecodeGraph:

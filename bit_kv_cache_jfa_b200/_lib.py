@@ -61,6 +61,7 @@ class WorkspaceLayout(ctypes.Structure):
                 ("off_hist", c_size_t), ("off_counters", c_size_t),
                 ("off_cand", c_size_t), ("off_sel", c_size_t),
                 ("off_fp4q", c_size_t), ("off_sparse", c_size_t), ("off_ticket", c_size_t),
+                ("off_bkeys", c_size_t),
                 ("max_topk", c_int32), ("partial_slots", c_int32), ("cand_cap", c_int32),
                 ("reserved", c_int32)]
 
@@ -110,6 +111,13 @@ SIGNATURES = {
     "jfa_fp4_decode_step": (c_int32, [POINTER(Geom), c_void_p, c_void_p, c_float, c_int32,
                                       c_void_p, c_void_p, c_void_p, c_int32, c_void_p, c_void_p,
                                       c_void_p]),
+    "jfa_channel_pack": (c_int32, [POINTER(Geom), c_int32, c_int32, c_void_p, c_void_p, c_void_p,
+                                   c_void_p]),
+    "jfa_channel_scores": (c_int32, [POINTER(Geom), c_void_p, c_void_p, c_void_p, c_float,
+                                     c_int32, c_void_p, c_void_p]),
+    "jfa_channel_decode_step": (c_int32, [POINTER(Geom), c_void_p, c_void_p, c_void_p, c_float,
+                                          c_int32, c_int32, c_void_p, c_void_p, c_void_p, c_int32,
+                                          c_void_p, c_void_p, c_void_p]),
 }
 
 _lib = None
@@ -244,6 +252,24 @@ def jfa_fp4_decode_step(geom, pool, q, scale, n_blocks, idx, k_exact, v_exact, e
     return load().jfa_fp4_decode_step(ctypes.byref(geom), _ptr(pool), _ptr(q), scale, n_blocks,
                                       _ptr(idx), _ptr(k_exact), _ptr(v_exact), int(exact_on_host),
                                       _ptr(ws), _ptr(out), _stream(stream))
+
+
+def jfa_channel_pack(geom, n_from, n_to, k_src, k_t, k_max, stream=None) -> int:
+    return load().jfa_channel_pack(ctypes.byref(geom), n_from, n_to, _ptr(k_src), _ptr(k_t),
+                                   _ptr(k_max), _stream(stream))
+
+
+def jfa_channel_scores(geom, k_t, k_max, q, scale, r, ws, stream=None) -> int:
+    return load().jfa_channel_scores(ctypes.byref(geom), _ptr(k_t), _ptr(k_max), _ptr(q), scale,
+                                     r, _ptr(ws), _stream(stream))
+
+
+def jfa_channel_decode_step(geom, k_t, k_max, q, scale, r, k, idx, k_exact, v_exact,
+                            exact_on_host, ws, out, stream=None) -> int:
+    return load().jfa_channel_decode_step(ctypes.byref(geom), _ptr(k_t), _ptr(k_max), _ptr(q),
+                                          scale, r, k, _ptr(idx), _ptr(k_exact), _ptr(v_exact),
+                                          int(exact_on_host), _ptr(ws), _ptr(out),
+                                          _stream(stream))
 
 
 def _lens(seq_lens):

@@ -64,6 +64,8 @@ int workspace_layout(const jfa_geom& g, int max_topk, jfa_workspace_layout* out)
   off = align_up(off + (n_seg > (size_t)kSpSlots ? n_seg : (size_t)kSpSlots) * kMaxG * 132 * sizeof(float), 256);
   L.off_ticket = off;
   off = align_up(off + n_seg * sizeof(uint32_t), 256);
+  L.off_bkeys = off;
+  off = align_up(off + n_seg * (size_t)((g.capacity + kF4Tok - 1) / kF4Tok) * sizeof(uint32_t), 256);
   L.total_bytes = off;
   *out = L;
   return JFA_OK;
@@ -287,7 +289,58 @@ int jfa_fp4_decode_step(const jfa_geom* geom, const void* pool, const uint16_t* 
   uint8_t* w = static_cast<uint8_t*>(ws);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   int rc = launch_fp4_scores(*geom, static_cast<const uint8_t*>(pool), q, scale, w, L, st);
-  if (rc == JFA_OK) rc = launch_topk_blocks(*geom, n_blocks, w, L, idx, st);
+  // the scan leaves every block's largest score in the block keys
+  if (rc == JFA_OK)
+    rc = launch_topk_blocks(*geom, n_blocks, w, L, idx, st,
+                            reinterpret_cast<const uint32_t*>(w + L.off_bkeys));
+  if (rc == JFA_OK)
+    rc = launch_sparse_attend(*geom, q, scale, idx, k, k_exact, v_exact, exact_on_host != 0, w, L, out, st);
+  return rc;
+}
+
+// ---------------------------------------------------------------------------
+// critical-channel selection
+// ---------------------------------------------------------------------------
+int jfa_channel_pack(const jfa_geom* geom, int32_t n_from, int32_t n_to, const uint16_t* k_src,
+                     uint16_t* k_t, float* k_max, void* stream) {
+  if (!geom_ok(geom) || !k_t || !aligned(k_t, 16) || !k_max || !aligned(k_max, 4))
+    return JFA_ERR_INVALID_ARG;
+  if (n_from < 0 || n_to < n_from || n_to > geom->capacity || n_from % kKG || n_to % kKG)
+    return JFA_ERR_INVALID_ARG;
+  if (n_to == n_from) return JFA_OK;
+  if (!k_src || !aligned(k_src, 16)) return JFA_ERR_INVALID_ARG;
+  return launch_channel_pack(*geom, n_from / kKG, n_to / kKG, k_src, k_t, k_max,
+                             static_cast<cudaStream_t>(stream));
+}
+
+static bool channel_args_ok(const jfa_geom* geom, const uint16_t* k_t, const float* k_max,
+                            const uint16_t* q, float scale, int32_t r, const void* ws) {
+  return geom_ok(geom) && geom->n_ctx >= 1 && k_t && aligned(k_t, 16) && k_max && aligned(k_max, 4) &&
+         q && aligned(q, 16) && scale > 0.f && r >= 1 && r <= kD && ws && aligned(ws, 256);
+}
+
+int jfa_channel_scores(const jfa_geom* geom, const uint16_t* k_t, const float* k_max,
+                       const uint16_t* q, float scale, int32_t r, void* ws, void* stream) {
+  if (!channel_args_ok(geom, k_t, k_max, q, scale, r, ws)) return JFA_ERR_INVALID_ARG;
+  jfa_workspace_layout L;
+  workspace_layout(*geom, 1, &L);
+  return launch_channel_scores(*geom, k_t, k_max, q, scale, r, static_cast<uint8_t*>(ws), L,
+                               static_cast<cudaStream_t>(stream));
+}
+
+int jfa_channel_decode_step(const jfa_geom* geom, const uint16_t* k_t, const float* k_max,
+                            const uint16_t* q, float scale, int32_t r, int32_t k, int32_t* idx,
+                            const uint16_t* k_exact, const uint16_t* v_exact,
+                            int32_t exact_on_host, void* ws, float* out, void* stream) {
+  if (!channel_args_ok(geom, k_t, k_max, q, scale, r, ws)) return JFA_ERR_INVALID_ARG;
+  if (k < 1 || k > JFA_MAX_TOPK) return JFA_ERR_INVALID_ARG;
+  if (!sparse_args_ok(geom, q, scale, idx, k, k_exact, v_exact, ws, out)) return JFA_ERR_INVALID_ARG;
+  jfa_workspace_layout L;
+  workspace_layout(*geom, k, &L);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int rc = launch_channel_scores(*geom, k_t, k_max, q, scale, r, w, L, st);
+  if (rc == JFA_OK) rc = launch_topk(*geom, k, w, L, idx, st);
   if (rc == JFA_OK)
     rc = launch_sparse_attend(*geom, q, scale, idx, k, k_exact, v_exact, exact_on_host != 0, w, L, out, st);
   return rc;

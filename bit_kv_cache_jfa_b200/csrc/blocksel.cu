@@ -19,7 +19,8 @@ namespace jfa {
 constexpr int kSelBlock = JFA_BLOCK_TOKENS;
 constexpr int kBlkThreads = 256;
 
-__global__ void __launch_bounds__(kBlkThreads) block_select_kernel(const float* scores, int capacity,
+__global__ void __launch_bounds__(kBlkThreads) block_select_kernel(const float* scores,
+                                                                   const uint32_t* bkeys, int capacity,
                                                                    int nq, int n_sel, int out_len,
                                                                    int32_t* idx) {
   extern __shared__ uint32_t bsm[];
@@ -35,17 +36,30 @@ __global__ void __launch_bounds__(kBlkThreads) block_select_kernel(const float* 
   const int seg = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const float* S = scores + (size_t)seg * capacity;
 
-  // 1. block keys (nq is a multiple of 64, so a float4 never straddles nq)
-  for (int b = warp; b < nb; b += kBlkThreads / 32) {
-    const int t0 = kSelBlock * b + 4 * lane;
-    float m = -INFINITY;
-    if (t0 < nq) {
-      const float4 v = *reinterpret_cast<const float4*>(S + t0);
-      m = fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w));
-    }
+  // 1. block keys: given, or the largest stored score of every block (nq is
+  // a multiple of 64, so a float4 never straddles nq); a warp takes 4 blocks
+  // at a time so that 4 loads per lane are in flight
+  if (bkeys) {
+    const uint32_t* K = bkeys + (size_t)seg * ((capacity + kSelBlock - 1) / kSelBlock);
+    for (int b = tid; b < nb; b += kBlkThreads) keys[b] = K[b];
+  } else {
+    constexpr int kWarps = kBlkThreads / 32;
+    for (int b0 = 4 * warp; b0 < nb; b0 += 4 * kWarps) {
+      float4 v[4];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kAll, m, o));
-    if (lane == 0) keys[b] = float_key(m);
+      for (int u = 0; u < 4; ++u) {
+        const int t0 = kSelBlock * (b0 + u) + 4 * lane;
+        v[u] = (b0 + u < nb && t0 < nq) ? *reinterpret_cast<const float4*>(S + t0)
+                                        : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        float m = fmaxf(fmaxf(v[u].x, v[u].y), fmaxf(v[u].z, v[u].w));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kAll, m, o));
+        if (lane == 0 && b0 + u < nb) keys[b0 + u] = float_key(m);
+      }
+    }
   }
   __syncthreads();
 
@@ -122,14 +136,14 @@ size_t block_select_smem(int nq, int n_blocks) {
 }
 
 int launch_topk_blocks(const jfa_geom& g, int n_blocks, uint8_t* ws, const jfa_workspace_layout& L,
-                       int32_t* idx, cudaStream_t st) {
+                       int32_t* idx, cudaStream_t st, const uint32_t* bkeys) {
   const int n_seg = g.batch * g.num_kv_heads;
   const int nq = split_point(g.n_ctx);
   const int out_len = n_blocks * kSelBlock;
   // at most kMaxSelBlocks block keys: 40 KB, inside the default 48 KB
   const size_t smem = block_select_smem(nq, n_blocks);
   return launch_pdl(block_select_kernel, dim3(n_seg), dim3(kBlkThreads), smem, st,
-                    reinterpret_cast<const float*>(ws + L.off_scores), g.capacity, nq, n_blocks,
+                    reinterpret_cast<const float*>(ws + L.off_scores), bkeys, g.capacity, nq, n_blocks,
                     out_len, idx) == cudaSuccess
              ? JFA_OK
              : JFA_ERR_CUDA;

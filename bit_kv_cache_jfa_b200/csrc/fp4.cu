@@ -14,11 +14,13 @@
 //                     epilogue scales a token's 8 head logits by its group's
 //                     and each head's tensor scale and stores the largest over
 //                     the KV head's query heads as the selection score.
-// Scan roles per CTA (6 warps): warp 0 streams records (bulk copies into a
-// 6-stage ring), warp 1 owns the tensor memory and issues scale copies and
-// MMAs, warps 2-5 read the accumulators (one 32-lane quarter each).  Every
-// wait is bounded: on a timeout the kernel records JFA_DEVERR_TIMEOUT, lets
-// its copies and MMAs drain, frees its tensor memory and returns.
+// Scan roles per CTA (6 warps): warp 0 streams records (bulk copies into an
+// 8-stage ring), warp 1 owns the tensor memory, copies each record's scales
+// aside and issues scale copies and MMAs (a stage is free again once its
+// MMAs have read it), warps 2-5 read the accumulators (one 32-lane quarter
+// each).  Every wait is bounded: on a timeout the kernel records
+// JFA_DEVERR_TIMEOUT, lets its copies and MMAs drain, frees its tensor memory
+// and returns.
 #include "jfa_fp4.cuh"
 
 namespace jfa {
@@ -107,7 +109,8 @@ int launch_fp4_pack(const jfa_geom& g, int g_from, int g_to, const uint16_t* k_s
 // query records: thread t quantizes channels 8 (t mod 16) .. +7 of head t / 16
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(128) fp4_query_kernel(const uint16_t* __restrict__ q, int H,
-                                                        int Hkv, int G, uint8_t* __restrict__ qrec) {
+                                                        int Hkv, int G, uint8_t* __restrict__ qrec,
+                                                        uint32_t* __restrict__ bkeys, int nb_cap) {
   __shared__ __align__(16) uint8_t rec[kF4QBytes];
   const int seg = blockIdx.x, b = seg / Hkv, kvh = seg % Hkv, t = threadIdx.x;
   const int h = t >> 4, c0 = (t & 15) * 8;
@@ -139,12 +142,14 @@ __global__ void __launch_bounds__(128) fp4_query_kernel(const uint16_t* __restri
   __syncthreads();
   uint4* dst = reinterpret_cast<uint4*>(qrec + (size_t)seg * kF4QBytes);
   for (int i = t; i < kF4QBytes / 16; i += 128) dst[i] = reinterpret_cast<const uint4*>(rec)[i];
+  // the scan raises every block key of this segment from zero
+  for (int i = t; i < nb_cap; i += 128) bkeys[(size_t)seg * nb_cap + i] = 0u;
 }
 
 // ---------------------------------------------------------------------------
 // tcgen05 scan
 // ---------------------------------------------------------------------------
-constexpr int kF4Stages = 6;
+constexpr int kF4Stages = 8;
 constexpr int kF4StageStride = 11264;  // record, then the query record at +kF4QStageOff
 constexpr int kF4QStageOff = 9344;
 constexpr int kF4Acc = 4;              // accumulator buffers (8 columns each)
@@ -158,6 +163,7 @@ struct Fp4ScanParams {
   const uint8_t* pool;
   const uint8_t* qrec;
   float* scores;
+  uint32_t* bkeys;  // [seg][nb_cap]: largest selection key of each record
   uint32_t* flag;
   long long total_tiles;
   int tiles_per_cta;
@@ -214,6 +220,10 @@ __device__ __forceinline__ void tc_mma_fp4(uint32_t d_tmem, uint64_t a, uint64_t
 __global__ void __launch_bounds__(kF4Threads, 1) fp4_scan_kernel(const __grid_constant__ Fp4ScanParams p) {
   extern __shared__ uint8_t f4raw[];
   __shared__ __align__(8) uint64_t full[kF4Stages], empty[kF4Stages], tfull[kF4Acc], tempty[kF4Acc];
+  // per accumulator buffer: the record's two group scales (times the softmax
+  // scale) and the query heads' scales, copied out of the stage by the MMA
+  // thread so that the stage is free as soon as the MMAs have read it
+  __shared__ float s_scales[kF4Acc][2 + kMaxG];
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(f4raw) + 1023) & ~(uintptr_t)1023);
@@ -225,10 +235,10 @@ __global__ void __launch_bounds__(kF4Threads, 1) fp4_scan_kernel(const __grid_co
   if (threadIdx.x == 0) {
     for (int s = 0; s < kF4Stages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1 + 4);
+      mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < kF4Acc; ++b) {
-      mbar_init(&tfull[b], 1);
+      mbar_init(&tfull[b], 2);  // the MMA thread's scales, then the MMAs
       mbar_init(&tempty[b], 4);
     }
     s_abort = 0;
@@ -292,6 +302,16 @@ __global__ void __launch_bounds__(kF4Threads, 1) fp4_scan_kernel(const __grid_co
         }
         if (*(volatile int*)&s_abort) break;
         tc_fence_after();
+        {
+          const uint8_t* sp = base + s * kF4StageStride;
+          const float* gs = reinterpret_cast<const float*>(sp + kF4GsOff);
+          const float* qs = reinterpret_cast<const float*>(sp + kF4QStageOff + kF4QScaleOff);
+          s_scales[b][0] = gs[0] * p.scale;
+          s_scales[b][1] = gs[1] * p.scale;
+#pragma unroll
+          for (int h = 0; h < kMaxG; ++h) s_scales[b][2 + h] = qs[h];
+          mbar_arrive1(&tfull[b]);
+        }
         const uint32_t st = smem_u32(base + s * kF4StageStride);
         const uint32_t sfa = tmem + 32u + 8u * (uint32_t)(i & 1), sfb = tmem + 48u + 8u * (uint32_t)(i & 1);
 #pragma unroll
@@ -318,10 +338,9 @@ __global__ void __launch_bounds__(kF4Threads, 1) fp4_scan_kernel(const __grid_co
     // ---- epilogue: warp w reads lanes 32 (w mod 4) .. + 31 (its tokens)
     const int sub = warp & 3, row = 32 * sub + lane;
     for (int i = 0; i < n_my; ++i) {
-      const int s = i % kF4Stages, b = i % kF4Acc;
-      const uint32_t ph = (uint32_t)(i / kF4Stages) & 1u, bph = (uint32_t)(i / kF4Acc) & 1u;
-      bool ok = __all_sync(0xFFFFFFFFu, mbar_wait_bounded(&tfull[b], bph));
-      if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait_bounded(&full[s], ph));
+      const int b = i % kF4Acc;
+      const uint32_t bph = (uint32_t)(i / kF4Acc) & 1u;
+      const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait_bounded(&tfull[b], bph));
       if (!ok) {
         if (lane == 0) {
           set_flag(p.flag, JFA_DEVERR_TIMEOUT);
@@ -337,21 +356,23 @@ __global__ void __launch_bounds__(kF4Threads, 1) fp4_scan_kernel(const __grid_co
             "=r"(d[7])
           : "r"(tmem + ((uint32_t)(32 * sub) << 16) + 8u * b));
       asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+      const float sk = s_scales[b][row >> 6];
+      float sq[kMaxG];
+#pragma unroll
+      for (int h = 0; h < kMaxG; ++h) sq[h] = s_scales[b][2 + h];
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive1(&tempty[b]);
-      const uint8_t* st = base + s * kF4StageStride;
-      const float sk = reinterpret_cast<const float*>(st + kF4GsOff)[row >> 6] * p.scale;
-      const float* sq = reinterpret_cast<const float*>(st + kF4QStageOff + kF4QScaleOff);
+      if (lane == 0) mbar_arrive1(&tempty[b]);  // accumulator and scales free
       float sel = -INFINITY;
 #pragma unroll
       for (int h = 0; h < kMaxG; ++h)
         if (h < p.G) sel = fmaxf(sel, __uint_as_float(d[h]) * (sk * sq[h]));
-      __syncwarp();
-      if (lane == 0) mbar_arrive1(&empty[s]);
       const long long tile = t0 + i;
-      const int seg = (int)(tile / p.nts), tok = (int)(tile % p.nts) * kF4Tok + row;
+      const int seg = (int)(tile / p.nts), tb = (int)(tile % p.nts), tok = tb * kF4Tok + row;
       if (tok < p.nq) p.scores[(size_t)seg * p.capacity + tok] = sel;
+      // the block key: the largest selection score of the record's tokens
+      const uint32_t bk = __reduce_max_sync(0xFFFFFFFFu, tok < p.nq ? float_key(sel) : 0u);
+      if (lane == 0) atomicMax(p.bkeys + (size_t)seg * p.nb_cap + tb, bk);
     }
   }
   pdl_launch_dependents();
@@ -370,8 +391,9 @@ int launch_fp4_scores(const jfa_geom& g, const uint8_t* pool, const uint16_t* q,
   const int nq = split_point(g.n_ctx);
   uint8_t* qrec = ws + L.off_fp4q;
   uint32_t* flag = reinterpret_cast<uint32_t*>(ws + L.off_flag);
+  uint32_t* bkeys = reinterpret_cast<uint32_t*>(ws + L.off_bkeys);
   if (launch_pdl(fp4_query_kernel, dim3(n_seg), dim3(128), 0, st, q, g.num_heads, g.num_kv_heads, G,
-                 qrec) != cudaSuccess)
+                 qrec, bkeys, g.capacity / kF4Tok) != cudaSuccess)
     return JFA_ERR_CUDA;
   if (nq == 0) return JFA_OK;
   static bool attr_set = false;
@@ -385,6 +407,7 @@ int launch_fp4_scores(const jfa_geom& g, const uint8_t* pool, const uint16_t* q,
   p.pool = pool;
   p.qrec = qrec;
   p.scores = reinterpret_cast<float*>(ws + L.off_scores);
+  p.bkeys = bkeys;
   p.flag = flag;
   p.capacity = g.capacity;
   p.nb_cap = g.capacity / kF4Tok;

@@ -90,6 +90,13 @@ int launch_fp4_scores(const jfa_geom& g, const uint8_t* pool, const uint16_t* q,
 int launch_sparse_attend(const jfa_geom& g, const uint16_t* q, float scale, const int32_t* idx,
                          int k, const uint16_t* k_exact, const uint16_t* v_exact, bool on_host,
                          uint8_t* ws, const jfa_workspace_layout& L, float* out, cudaStream_t st);
+// Channel-major key copy and per-channel max|K| for tokens in groups
+// [g_from, g_to); critical-channel selection scores into the workspace.
+int launch_channel_pack(const jfa_geom& g, int g_from, int g_to, const uint16_t* k_src, uint16_t* k_t,
+                        float* k_max, cudaStream_t st);
+int launch_channel_scores(const jfa_geom& g, const uint16_t* k_t, const float* k_max, const uint16_t* q,
+                          float scale, int r, uint8_t* ws, const jfa_workspace_layout& L,
+                          cudaStream_t st);
 // Splits per segment of the sparse attention (host rule shared with the
 // workspace sizing): at most kSpMaxSplit, and n_seg * splits <= max(n_seg, 512).
 constexpr int kSpMaxSplit = 32;

@@ -89,8 +89,10 @@ int count_topk_launches(const jfa_geom& g, int k);
 // Block selection: at most kMaxSelBlocks blocks of 128 quantized tokens per
 // segment (N_q <= 1M tokens).
 constexpr int kMaxSelBlocks = 8192;
+// bkeys: the block keys already computed (the FP4 scan leaves them), else
+// null to take every block's largest stored score.
 int launch_topk_blocks(const jfa_geom& g, int n_blocks, uint8_t* ws, const jfa_workspace_layout& L,
-                       int32_t* idx, cudaStream_t st);
+                       int32_t* idx, cudaStream_t st, const uint32_t* bkeys = nullptr);
 // Selection (idx_in == nullptr: top-k written to idx_out) or a given index
 // set (idx_in), then correction and merge: one cluster per segment.
 int launch_finish(const jfa_geom& g, const SeqTable& t, const jfa_cache& c, const uint16_t* q,

@@ -122,12 +122,17 @@ __global__ void __launch_bounds__(kSpThreads, 2) sparse_attend_kernel(const __gr
   }
 
   // run j of this warp: entries 16 (r_lo + warp + 4 j) ..; lane < 16 holds
-  // the token of row = lane
+  // the token of row = lane.  The tokens of the next run are loaded one run
+  // ahead (their global load overlaps the current run's work) and every
+  // issued run's tokens stay in shared memory until it is computed.
+  __shared__ int tok_s[kSpWarps][kSpStages][kSpRun];
   auto run_token = [&](int j) -> int {
-    return lane < kSpRun ? entry_token(p, ix, E, kSpRun * (r_lo + warp + kSpWarps * j) + lane) : -1;
+    return (lane < kSpRun && j < n_mine)
+               ? entry_token(p, ix, E, kSpRun * (r_lo + warp + kSpWarps * j) + lane)
+               : -1;
   };
-  auto issue = [&](int j) {
-    const int mytok = run_token(j);
+  auto issue = [&](int j, int mytok) {
+    if (lane < kSpRun) tok_s[warp][j % kSpStages][lane] = mytok;
     const uint32_t st = ring_s + (uint32_t)((j % kSpStages) * kSpStageBytes);
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
@@ -152,17 +157,27 @@ __global__ void __launch_bounds__(kSpThreads, 2) sparse_attend_kernel(const __gr
   for (int n = 0; n < 16; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
   float m = -INFINITY, l = 0.f;
 
+  int next_tok = run_token(0);
 #pragma unroll
   for (int j = 0; j < kSpStages - 1; ++j) {
-    if (j < n_mine) issue(j);
+    if (j < n_mine) {
+      const int mytok = next_tok;
+      next_tok = run_token(j + 1);
+      issue(j, mytok);
+    }
     asm volatile("cp.async.commit_group;" ::: "memory");
   }
   for (int j = 0; j < n_mine; ++j) {
-    if (j + kSpStages - 1 < n_mine) issue(j + kSpStages - 1);
+    if (j + kSpStages - 1 < n_mine) {
+      const int mytok = next_tok;
+      next_tok = run_token(j + kSpStages);
+      issue(j + kSpStages - 1, mytok);
+    }
     asm volatile("cp.async.commit_group;" ::: "memory");
     asm volatile("cp.async.wait_group %0;" ::"n"(kSpStages - 1) : "memory");
     __syncwarp();
-    const unsigned valid = __ballot_sync(0xFFFFFFFFu, run_token(j) >= 0);
+    const unsigned valid =
+        __ballot_sync(0xFFFFFFFFu, lane < kSpRun && tok_s[warp][j % kSpStages][lane] >= 0);
     const uint32_t kb = ring_s + (uint32_t)((j % kSpStages) * kSpStageBytes);
     const uint32_t vb = kb + kSpRun * 256;
 

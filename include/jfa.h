@@ -132,6 +132,9 @@ typedef struct jfa_workspace_layout {
   size_t off_sparse;     /* split partials of jfa_sparse_attend              */
   size_t off_ticket;     /* uint32 [B][H_kv] split counters of
                             jfa_sparse_attend (zero between calls)           */
+  size_t off_bkeys;      /* uint32 [B][H_kv][capacity/128]: per 128-token
+                            block the largest selection score of the FP4
+                            scan, as an order-preserving key                 */
   int32_t max_topk;
   int32_t partial_slots; /* slots of off_partials                             */
   int32_t cand_cap;      /* list entries per segment                          */
@@ -432,6 +435,41 @@ int jfa_fp4_decode_step(const jfa_geom* geom, const void* pool, const uint16_t* 
                         int32_t n_blocks, int32_t* idx, const uint16_t* k_exact,
                         const uint16_t* v_exact, int32_t exact_on_host, void* ws, float* out,
                         void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Critical-channel selection (TailorKV review: the importance of channel i is
+ * s_i = |q_i| * max_t |K_{t,i}|; approximate attention scores over the most
+ * important channels pick the top-k tokens, which are attended exactly).
+ * Here, per (sequence, KV head): |q_i| is the largest over the KV head's
+ * query heads, max|K_i| runs over the tokens packed into the channel copy
+ * (pack the groups below N_q), the r most important channels are kept (ties
+ * to the lower channel), and the selection score of a quantized token t is
+ * the largest over the query heads of scale * sum over kept channels of
+ * q_{h,i} K_{t,i} (fp32).  Geometry as for the NVFP4 calls (key_bits and
+ * val_bits unused; capacity a multiple of 64).
+ * ------------------------------------------------------------------------- */
+
+/* Channel-major copy of the keys of tokens [n_from, n_to) (multiples of 64):
+ *   k_src : bf16 [B][H_kv][capacity][128] (device or pinned host)
+ *   k_t   : bf16 [B][H_kv][128][capacity] (device, 16-byte aligned)
+ *   k_max : fp32 [B][H_kv][128] (device), zero before the first call; raised
+ *           to the largest |K| of each channel.  Stream-ordered. */
+int jfa_channel_pack(const jfa_geom* geom, int32_t n_from, int32_t n_to, const uint16_t* k_src,
+                     uint16_t* k_t, float* k_max, void* stream);
+
+/* Selection scores of the N_q quantized tokens from the r critical channels
+ * (1 <= r <= 128) into the workspace's score array (read by jfa_topk).  One
+ * launch.  Stream-ordered. */
+int jfa_channel_scores(const jfa_geom* geom, const uint16_t* k_t, const float* k_max,
+                       const uint16_t* q, float scale, int32_t r, void* ws, void* stream);
+
+/* jfa_channel_scores, jfa_topk (k tokens per (sequence, KV head), written to
+ * idx int32 [B][H_kv][k]) and jfa_sparse_attend over them and the tail.
+ * 1 <= k <= JFA_MAX_TOPK.  Stream-ordered. */
+int jfa_channel_decode_step(const jfa_geom* geom, const uint16_t* k_t, const float* k_max,
+                            const uint16_t* q, float scale, int32_t r, int32_t k, int32_t* idx,
+                            const uint16_t* k_exact, const uint16_t* v_exact,
+                            int32_t exact_on_host, void* ws, float* out, void* stream);
 
 /* Number of warps jfa_decode_scores splits the quantized groups over on the
  * current device (0 on a bad geometry or when no group is quantized).  Warp w

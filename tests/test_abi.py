@@ -64,7 +64,7 @@ def test_workspace_layout(lib):
     for L in (a, b):
         offs = [L.off_flag, L.off_scores, L.off_partials, L.off_mused, L.off_wts,
                 L.off_scan_hist, L.off_hist, L.off_cand, L.off_sel, L.off_fp4q, L.off_sparse,
-                L.off_ticket, L.total_bytes]
+                L.off_ticket, L.off_bkeys, L.total_bytes]
         assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
         assert L.off_counters == L.off_hist + 4 * 4 * 2048
         assert L.off_scores + 4 * 4 * 4096 <= L.off_partials
@@ -170,3 +170,18 @@ def test_fp4_pool_size_and_argument_checks(lib):
     assert lib.jfa_sparse_attend(g, 256, 0.1, 256, 8193, 256, 256, 0, 256, 256) == bad
     assert lib.jfa_fp4_decode_step(g, 256, 256, 0.1, 0, 256, 256, 256, 0, 256, 256) == bad
     assert lib.jfa_fp4_decode_step(g, 256, 256, 0.1, 65, 256, 256, 256, 0, 256, 256) == bad
+
+
+def test_channel_argument_checks(lib):
+    g = G(capacity=4096, n_ctx=1000)
+    bad = lib.JFA_ERR_INVALID_ARG
+    assert lib.jfa_channel_pack(g, 0, 100, 256, 256, 256) == bad        # not a group edge
+    assert lib.jfa_channel_pack(g, 0, 4160, 256, 256, 256) == bad       # past capacity
+    assert lib.jfa_channel_pack(g, 64, 64, 256, 256, 256) == 0          # nothing to do
+    assert lib.jfa_channel_scores(g, 256, 256, 256, 0.1, 0, 256) == bad     # r = 0
+    assert lib.jfa_channel_scores(g, 256, 256, 256, 0.1, 129, 256) == bad   # r > 128
+    assert lib.jfa_channel_scores(g, 8, 256, 256, 0.1, 16, 256) == bad      # k_t alignment
+    assert lib.jfa_channel_decode_step(g, 256, 256, 256, 0.1, 16, 0, 256, 256, 256, 0, 256,
+                                       256) == bad                          # k = 0
+    assert lib.jfa_channel_decode_step(g, 256, 256, 256, 0.1, 16, 4097, 256, 256, 256, 0, 256,
+                                       256) == bad                          # k > JFA_MAX_TOPK
