@@ -66,6 +66,8 @@ int workspace_layout(const jfa_geom& g, int max_topk, jfa_workspace_layout* out)
   off = align_up(off + n_seg * sizeof(uint32_t), 256);
   L.off_bkeys = off;
   off = align_up(off + n_seg * (size_t)((g.capacity + kF4Tok - 1) / kF4Tok) * sizeof(uint32_t), 256);
+  L.off_chan = off;
+  off = align_up(off + n_seg * (size_t)kChanRecBytes, 256);
   L.total_bytes = off;
   *out = L;
   return JFA_OK;

@@ -6,12 +6,13 @@
 //   channel_pack_kernel    one CTA per (64-token group, segment): writes the
 //                          group's keys channel-major (k_t [seg][128][cap],
 //                          bf16) and raises the segment's per-channel max|K|;
-//   channel_scores_kernel  one CTA per (2048 tokens, segment): ranks the 128
-//                          channels by importance (largest |q_i| over the KV
-//                          head's query heads times max|K_i|, both bf16 values
-//                          so the fp32 product is exact), keeps the r best
-//                          (ties to the lower channel), and streams those r
-//                          channel rows of k_t, 8 tokens per thread: the
+//   channel_select_kernel  one CTA per segment: ranks the 128 channels by
+//                          importance (largest |q_i| over the KV head's query
+//                          heads times max|K_i|, both bf16 values so the fp32
+//                          product is exact) and keeps the r best (ties to the
+//                          lower channel), with the scaled query at them;
+//   channel_scores_kernel  one CTA per (1024 tokens, segment): streams the r
+//                          kept channel rows of k_t, 4 tokens per thread: the
 //                          selection score of a token is the largest over the
 //                          query heads of scale * sum_i q_{h,i} K_{t,i}.
 // HBM-bound: 2 r bytes read and 4 written per token and KV head.
@@ -19,7 +20,7 @@
 
 namespace jfa {
 
-constexpr int kChTok = 2048;  // tokens per CTA of the score kernel (256 threads x 8)
+constexpr int kChTok = 1024;  // tokens per CTA of the score kernel (256 threads x 4)
 
 __device__ __forceinline__ float bf16f(uint32_t bits16) { return __uint_as_float(bits16 << 16); }
 
@@ -62,100 +63,105 @@ struct ChanParams {
   const float* k_max;
   const uint16_t* q;
   float* scores;
+  uint8_t* chan;  // per-segment channel records
   int capacity, H, Hkv, G, nq, r;
   float scale;
 };
 
-__global__ void __launch_bounds__(256) channel_scores_kernel(const __grid_constant__ ChanParams p) {
+// One CTA per segment: the importance of every channel, its rank
+// (importance descending, index ascending) and the kept channels with the
+// scaled query at them, written to the segment's channel record.
+__global__ void __launch_bounds__(128) channel_select_kernel(const __grid_constant__ ChanParams p) {
   __shared__ float imp[kD];
-  __shared__ float qs[kMaxG][kD];
-  __shared__ int chans[kD];
   __shared__ int wcount[4];
-  const int seg = blockIdx.y, b = seg / p.Hkv, kvh = seg % p.Hkv, tid = threadIdx.x;
+  const int seg = blockIdx.x, b = seg / p.Hkv, kvh = seg % p.Hkv, tid = threadIdx.x;
+  pdl_launch_dependents();  // the score kernel's set-up may overlap; it waits for this grid
   pdl_wait();
-  if (tid < kD) {
-    float qm = 0.f;
-    for (int h = 0; h < p.G; ++h) {
-      const float v = bf16f(p.q[((size_t)b * p.H + kvh * p.G + h) * kD + tid]);
-      qs[h][tid] = v * p.scale;
-      qm = fmaxf(qm, fabsf(v));
-    }
-    imp[tid] = qm * p.k_max[(size_t)seg * kD + tid];
+  float qv[kMaxG];
+  float qm = 0.f;
+#pragma unroll
+  for (int h = 0; h < kMaxG; ++h) {
+    qv[h] = h < p.G ? bf16f(p.q[((size_t)b * p.H + kvh * p.G + h) * kD + tid]) : 0.f;
+    qm = fmaxf(qm, fabsf(qv[h]));
   }
+  const float mine = qm * p.k_max[(size_t)seg * kD + tid];
+  imp[tid] = mine;
   __syncthreads();
-  // rank of channel tid (importance descending, index ascending); the r best
-  // are listed in channel order
-  bool keep = false;
-  if (tid < kD) {
-    const float mine = imp[tid];
-    int rank = 0;
+  int rank = 0;
 #pragma unroll 16
-    for (int c = 0; c < kD; ++c) {
-      const float o = imp[c];
-      rank += (o > mine) || (o == mine && c < tid);
-    }
-    keep = rank < p.r;
+  for (int c = 0; c < kD; ++c) {
+    const float o = imp[c];
+    rank += (o > mine) || (o == mine && c < tid);
   }
+  const bool keep = rank < p.r;
   const unsigned bal = __ballot_sync(0xFFFFFFFFu, keep);
-  if ((tid & 31) == 0 && tid < kD) wcount[tid >> 5] = __popc(bal);
+  if ((tid & 31) == 0) wcount[tid >> 5] = __popc(bal);
   __syncthreads();
   if (keep) {
     int pos = __popc(bal & ((1u << (tid & 31)) - 1u));
     for (int w = 0; w < (tid >> 5); ++w) pos += wcount[w];
-    chans[pos] = tid;
+    uint8_t* rec = p.chan + (size_t)seg * kChanRecBytes;
+    reinterpret_cast<int*>(rec)[pos] = tid;
+    float* qs = reinterpret_cast<float*>(rec + 128 * 4);
+#pragma unroll
+    for (int h = 0; h < kMaxG; ++h) qs[h * kD + pos] = qv[h] * p.scale;
+  }
+}
+
+// One CTA per (1024 tokens, segment), 4 tokens per thread.
+__global__ void __launch_bounds__(256, 4) channel_scores_kernel(const __grid_constant__ ChanParams p) {
+  __shared__ float qs[kMaxG][kD];
+  __shared__ int chans[kD];
+  const int seg = blockIdx.y, tid = threadIdx.x;
+  pdl_wait();
+  const uint8_t* rec = p.chan + (size_t)seg * kChanRecBytes;
+  for (int i = tid; i < p.r; i += 256) chans[i] = reinterpret_cast<const int*>(rec)[i];
+  for (int i = tid; i < kMaxG * kD; i += 256) {
+    const int h = i / kD, j = i % kD;
+    if (h < p.G && j < p.r) qs[h][j] = reinterpret_cast<const float*>(rec + 128 * 4)[i];
   }
   __syncthreads();
 
-  const int t = blockIdx.x * kChTok + tid * 8;
+  const int t = blockIdx.x * kChTok + tid * 4;
   if (t >= p.nq) return;
-  float acc[kMaxG][8];
+  float acc[kMaxG][4];
 #pragma unroll
   for (int h = 0; h < kMaxG; ++h)
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[h][e] = 0.f;
+    for (int e = 0; e < 4; ++e) acc[h][e] = 0.f;
   const uint16_t* base = p.k_t + (size_t)seg * kD * p.capacity + t;
-  // 4 channel rows per round: their loads are in flight together
-  for (int j0 = 0; j0 < p.r; j0 += 4) {
-    uint4 v[4];
-    int cu[4];
+  // 8 channel rows per round: their loads are in flight together
+  for (int j0 = 0; j0 < p.r; j0 += 8) {
+    uint2 v[8];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      cu[u] = j0 + u < p.r ? chans[j0 + u] : -1;
-      v[u] = cu[u] >= 0 ? *reinterpret_cast<const uint4*>(base + (size_t)cu[u] * p.capacity)
-                        : make_uint4(0, 0, 0, 0);
-    }
+    for (int u = 0; u < 8; ++u)
+      v[u] = j0 + u < p.r ? *reinterpret_cast<const uint2*>(base + (size_t)chans[j0 + u] * p.capacity)
+                          : make_uint2(0, 0);
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      if (cu[u] < 0) continue;
-      const uint32_t wv[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-      float k8[8];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        k8[2 * e] = __uint_as_float(wv[e] << 16);
-        k8[2 * e + 1] = __uint_as_float(wv[e] & 0xFFFF0000u);
-      }
+    for (int u = 0; u < 8; ++u) {
+      if (j0 + u >= p.r) break;
+      const float k4[4] = {__uint_as_float(v[u].x << 16), __uint_as_float(v[u].x & 0xFFFF0000u),
+                           __uint_as_float(v[u].y << 16), __uint_as_float(v[u].y & 0xFFFF0000u)};
 #pragma unroll
       for (int h = 0; h < kMaxG; ++h) {
         if (h < p.G) {
-          const float qv = qs[h][cu[u]];
+          const float qv = qs[h][j0 + u];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) acc[h][e] = fmaf(qv, k8[e], acc[h][e]);
+          for (int e = 0; e < 4; ++e) acc[h][e] = fmaf(qv, k4[e], acc[h][e]);
         }
       }
     }
   }
-  float s[8];
+  float s[4];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) {
+  for (int e = 0; e < 4; ++e) {
     float m = acc[0][e];
 #pragma unroll
     for (int h = 1; h < kMaxG; ++h)
       if (h < p.G) m = fmaxf(m, acc[h][e]);
     s[e] = m;
   }
-  float4* out = reinterpret_cast<float4*>(p.scores + (size_t)seg * p.capacity + t);
-  out[0] = make_float4(s[0], s[1], s[2], s[3]);
-  out[1] = make_float4(s[4], s[5], s[6], s[7]);
+  *reinterpret_cast<float4*>(p.scores + (size_t)seg * p.capacity + t) = make_float4(s[0], s[1], s[2], s[3]);
   pdl_launch_dependents();
 }
 
@@ -176,6 +182,7 @@ int launch_channel_scores(const jfa_geom& g, const uint16_t* k_t, const float* k
   p.k_max = k_max;
   p.q = q;
   p.scores = reinterpret_cast<float*>(ws + L.off_scores);
+  p.chan = ws + L.off_chan;
   p.capacity = g.capacity;
   p.H = g.num_heads;
   p.Hkv = g.num_kv_heads;
@@ -184,6 +191,8 @@ int launch_channel_scores(const jfa_geom& g, const uint16_t* k_t, const float* k
   p.r = r;
   p.scale = scale;
   if (p.nq == 0) return JFA_OK;
+  if (launch_pdl(channel_select_kernel, dim3(n_seg), dim3(kD), 0, st, p) != cudaSuccess)
+    return JFA_ERR_CUDA;
   const int chunks = (p.nq + kChTok - 1) / kChTok;
   return launch_pdl(channel_scores_kernel, dim3(chunks, n_seg), dim3(256), 0, st, p) == cudaSuccess
              ? JFA_OK

@@ -14,8 +14,11 @@
 //                     epilogue scales a token's 8 head logits by its group's
 //                     and each head's tensor scale and stores the largest over
 //                     the KV head's query heads as the selection score.
-// Scan roles per CTA (6 warps): warp 0 streams records (bulk copies into an
-// 8-stage ring), warp 1 owns the tensor memory, copies each record's scales
+// Scan roles per CTA (6 warps, 6 CTAs per SM: a CTA's throughput is set by
+// its one-thread issue chains, so more small CTAs beat deeper rings — with 2
+// CTAs per SM the scan reached 0.52 of HBM bandwidth at any ring depth, with
+// 6 CTAs of 3 stages 0.88): warp 0 streams records (bulk copies into a
+// 3-stage ring), warp 1 owns the tensor memory, copies each record's scales
 // aside and issues scale copies and MMAs (a stage is free again once its
 // MMAs have read it), warps 2-5 read the accumulators (one 32-lane quarter
 // each).  Every wait is bounded: on a timeout the kernel records
@@ -49,6 +52,9 @@ __device__ __forceinline__ uint2 e2m1_block(const float* x, double unit) {
 }
 
 // Thread t: token row r = t / 2 of the group, channels 64 (t mod 2) .. +63.
+// The kernel never lets its dependents start early: the scan requests its
+// first records before its own dependency wait, which is safe only because
+// every kernel after this one starts after it has finished.
 __global__ void __launch_bounds__(128) fp4_pack_kernel(const uint16_t* __restrict__ k_src,
                                                        uint8_t* __restrict__ pool, int capacity,
                                                        int g_from, uint32_t* flag) {
@@ -149,7 +155,13 @@ __global__ void __launch_bounds__(128) fp4_query_kernel(const uint16_t* __restri
 // ---------------------------------------------------------------------------
 // tcgen05 scan
 // ---------------------------------------------------------------------------
-constexpr int kF4Stages = 8;
+#ifndef JFA_F4_STAGES
+#define JFA_F4_STAGES 3
+#endif
+#ifndef JFA_F4_CTAS_PER_SM
+#define JFA_F4_CTAS_PER_SM 6
+#endif
+constexpr int kF4Stages = JFA_F4_STAGES;
 constexpr int kF4StageStride = 11264;  // record, then the query record at +kF4QStageOff
 constexpr int kF4QStageOff = 9344;
 constexpr int kF4Acc = 4;              // accumulator buffers (8 columns each)
@@ -158,6 +170,7 @@ constexpr uint32_t kF4TmemCols = 64;   // [0,32) accumulators, [32,48) A scales,
 constexpr int kF4Smem = kF4Stages * kF4StageStride + 1024;
 static_assert(kF4QStageOff >= kF4RecBytes && kF4QStageOff % 128 == 0, "query record after the record");
 static_assert(kF4QStageOff + kF4QBytes <= kF4StageStride, "stage holds both records");
+static_assert(JFA_F4_CTAS_PER_SM * 64 <= 512, "tensor memory of the CTAs of one SM");
 
 struct Fp4ScanParams {
   const uint8_t* pool;
@@ -255,14 +268,30 @@ __global__ void __launch_bounds__(kF4Threads, 1) fp4_scan_kernel(const __grid_co
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s_tmem;
-  pdl_wait();
 
   if (warp == 0) {
-    // ---- producer: record + query record per tile into the ring
+    // ---- producer: record + query record per tile into the ring.  The
+    // records of the first stages are requested before the wait on the
+    // previous kernel (the query kernel, which writes no record; the pool's
+    // writer finished before that kernel began), their query records after.
     if (lane == 0) {
       const uint64_t pol = policy_evict_first();
-      int issued = 0;
-      for (int i = 0; i < n_my; ++i) {
+      const int n_first = n_my < kF4Stages ? n_my : kF4Stages;
+      for (int i = 0; i < n_first; ++i) {
+        const long long tile = t0 + i;
+        const int seg = (int)(tile / p.nts), tb = (int)(tile % p.nts);
+        mbar_expect_tx(&full[i], kF4RecBytes + kF4QBytes);
+        bulk_g2s(base + i * kF4StageStride, p.pool + ((size_t)seg * p.nb_cap + tb) * kF4RecBytes,
+                 kF4RecBytes, &full[i], pol);
+      }
+      pdl_wait();
+      for (int i = 0; i < n_first; ++i) {
+        const int seg = (int)((t0 + i) / p.nts);
+        bulk_g2s_nohint(base + i * kF4StageStride + kF4QStageOff, p.qrec + (size_t)seg * kF4QBytes,
+                        kF4QBytes, &full[i]);
+      }
+      int issued = n_first;
+      for (int i = n_first; i < n_my; ++i) {
         const int s = i % kF4Stages;
         const uint32_t ph = (uint32_t)(i / kF4Stages) & 1u;
         if (i >= kF4Stages && !mbar_wait_bounded(&empty[s], ph ^ 1u)) {
@@ -288,6 +317,7 @@ __global__ void __launch_bounds__(kF4Threads, 1) fp4_scan_kernel(const __grid_co
     }
   } else if (warp == 1) {
     // ---- MMA issuer
+    pdl_wait();
     if (lane == 0) {
       int issued = 0;
       for (int i = 0; i < n_my; ++i) {
@@ -336,6 +366,7 @@ __global__ void __launch_bounds__(kF4Threads, 1) fp4_scan_kernel(const __grid_co
     }
   } else {
     // ---- epilogue: warp w reads lanes 32 (w mod 4) .. + 31 (its tokens)
+    pdl_wait();
     const int sub = warp & 3, row = 32 * sub + lane;
     for (int i = 0; i < n_my; ++i) {
       const int b = i % kF4Acc;
@@ -396,12 +427,24 @@ int launch_fp4_scores(const jfa_geom& g, const uint8_t* pool, const uint16_t* q,
                  qrec, bkeys, g.capacity / kF4Tok) != cudaSuccess)
     return JFA_ERR_CUDA;
   if (nq == 0) return JFA_OK;
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(fp4_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kF4Smem) !=
+  // Dynamic shared memory: the ring, padded so that at most
+  // JFA_F4_CTAS_PER_SM CTAs share an SM (their tensor-memory allocations,
+  // 64 columns each, then always fit the SM's 512 columns).
+  static int smem_dev = -1;
+  static size_t smem = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return JFA_ERR_CUDA;
+  if (dev != smem_dev) {
+    int per_sm = 0;
+    if (cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess)
+      return JFA_ERR_CUDA;
+    const size_t floor_bytes = (size_t)per_sm / (JFA_F4_CTAS_PER_SM + 1) + 1;  // N + 1 do not fit
+    const size_t need = (size_t)kF4Smem + 1024;  // + the per-CTA reservation
+    smem = (need > floor_bytes ? need : floor_bytes) - 1024;
+    if (cudaFuncSetAttribute(fp4_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess)
       return JFA_ERR_CUDA;
-    attr_set = true;
+    smem_dev = dev;
   }
   Fp4ScanParams p;
   p.pool = pool;
@@ -416,11 +459,11 @@ int launch_fp4_scores(const jfa_geom& g, const uint8_t* pool, const uint16_t* q,
   p.G = G;
   p.scale = scale;
   p.total_tiles = (long long)n_seg * p.nts;
-  const long long slots = 2LL * num_sms_current();
+  const long long slots = (long long)JFA_F4_CTAS_PER_SM * num_sms_current();
   const long long n_ctas0 = p.total_tiles < slots ? p.total_tiles : slots;
   p.tiles_per_cta = (int)((p.total_tiles + n_ctas0 - 1) / n_ctas0);
   const int n_ctas = (int)((p.total_tiles + p.tiles_per_cta - 1) / p.tiles_per_cta);
-  return launch_pdl(fp4_scan_kernel, dim3(n_ctas), dim3(kF4Threads), (size_t)kF4Smem, st, p) ==
+  return launch_pdl(fp4_scan_kernel, dim3(n_ctas), dim3(kF4Threads), smem, st, p) ==
                  cudaSuccess
              ? JFA_OK
              : JFA_ERR_CUDA;

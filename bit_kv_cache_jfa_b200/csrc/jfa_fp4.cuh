@@ -90,6 +90,10 @@ int launch_fp4_scores(const jfa_geom& g, const uint8_t* pool, const uint16_t* q,
 int launch_sparse_attend(const jfa_geom& g, const uint16_t* q, float scale, const int32_t* idx,
                          int k, const uint16_t* k_exact, const uint16_t* v_exact, bool on_host,
                          uint8_t* ws, const jfa_workspace_layout& L, float* out, cudaStream_t st);
+// Per-segment record of the critical channels: int32 channel[128] (the kept
+// ones first, ascending), then fp32 q[8][128] (scale * q_h at the kept
+// channels, in the same order).
+constexpr int kChanRecBytes = 128 * 4 + 8 * 128 * 4;
 // Channel-major key copy and per-channel max|K| for tokens in groups
 // [g_from, g_to); critical-channel selection scores into the workspace.
 int launch_channel_pack(const jfa_geom& g, int g_from, int g_to, const uint16_t* k_src, uint16_t* k_t,

@@ -22,9 +22,18 @@
 
 namespace jfa {
 
-constexpr int kSpWarps = 4;
+#ifndef JFA_SP_WARPS
+#define JFA_SP_WARPS 4
+#endif
+#ifndef JFA_SP_STAGES
+#define JFA_SP_STAGES 3
+#endif
+#ifndef JFA_SP_CTAS_PER_SM
+#define JFA_SP_CTAS_PER_SM 2
+#endif
+constexpr int kSpWarps = JFA_SP_WARPS;
 constexpr int kSpThreads = 32 * kSpWarps;
-constexpr int kSpStages = 3;
+constexpr int kSpStages = JFA_SP_STAGES;
 constexpr int kSpRun = 16;                        // entries per run (one MMA k-step of P V)
 constexpr int kSpStageBytes = 2 * kSpRun * kD * 2;  // K rows, then V rows
 constexpr int kSpSmem = kSpWarps * kSpStages * kSpStageBytes;
@@ -92,7 +101,7 @@ __device__ __forceinline__ int entry_token(const SparseParams& p, const int32_t*
   return p.nq + (e - p.k);
 }
 
-__global__ void __launch_bounds__(kSpThreads, 2) sparse_attend_kernel(const __grid_constant__ SparseParams p) {
+__global__ void __launch_bounds__(kSpThreads, JFA_SP_CTAS_PER_SM) sparse_attend_kernel(const __grid_constant__ SparseParams p) {
   extern __shared__ __align__(128) uint8_t spm[];
   __shared__ int s_last;
   const int seg = blockIdx.x / p.n_split, split = blockIdx.x % p.n_split;
@@ -258,27 +267,28 @@ __global__ void __launch_bounds__(kSpThreads, 2) sparse_attend_kernel(const __gr
   __syncthreads();
 
   // CTA partial: thread c merges channel c of every head
-  const int c = threadIdx.x;
   float* gp = p.part + ((size_t)seg * p.n_split + split) * kMaxG * kSpPart;
-  for (int h = 0; h < p.G; ++h) {
-    float M = -INFINITY;
+  for (int c = threadIdx.x; c < kD; c += kSpThreads) {
+    for (int h = 0; h < p.G; ++h) {
+      float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < kSpWarps; ++w) M = fmaxf(M, wp[(w * kMaxG + h) * kSpPart]);
-    float L = 0.f, O = 0.f;
-    if (M != -INFINITY) {
+      for (int w = 0; w < kSpWarps; ++w) M = fmaxf(M, wp[(w * kMaxG + h) * kSpPart]);
+      float L = 0.f, O = 0.f;
+      if (M != -INFINITY) {
 #pragma unroll
-      for (int w = 0; w < kSpWarps; ++w) {
-        const float* d = wp + (w * kMaxG + h) * kSpPart;
-        const float f = exp2f(d[0] - M);
-        L += d[1] * f;
-        O += d[4 + c] * f;
+        for (int w = 0; w < kSpWarps; ++w) {
+          const float* d = wp + (w * kMaxG + h) * kSpPart;
+          const float f = exp2f(d[0] - M);
+          L += d[1] * f;
+          O += d[4 + c] * f;
+        }
       }
+      if (c == 0) {
+        gp[h * kSpPart] = M;
+        gp[h * kSpPart + 1] = L;
+      }
+      gp[h * kSpPart + 4 + c] = O;
     }
-    if (c == 0) {
-      gp[h * kSpPart] = M;
-      gp[h * kSpPart + 1] = L;
-    }
-    gp[h * kSpPart + 4 + c] = O;
   }
   __threadfence();
   __syncthreads();
@@ -286,27 +296,46 @@ __global__ void __launch_bounds__(kSpThreads, 2) sparse_attend_kernel(const __gr
   __syncthreads();
   if (!s_last) return;
   __threadfence();
+  // the last CTA of the segment merges the n_split partials: every (split,
+  // head) frame is read once into shared memory and turned into its factor
+  // 2^(m - M); then thread c sums channel c of every head, all loads
+  // independent of one another
+  __shared__ float s_f[kSpMaxSplit][kMaxG];
+  __shared__ float s_l[kSpMaxSplit][kMaxG];
+  __shared__ float s_L[kMaxG];
   const float* sp = p.part + (size_t)seg * p.n_split * kMaxG * kSpPart;
-  for (int h = 0; h < p.G; ++h) {
-    float M = -INFINITY;
-    for (int s = 0; s < p.n_split; ++s) M = fmaxf(M, __ldcg(sp + (s * kMaxG + h) * kSpPart));
-    float L = 0.f, O = 0.f;
-    for (int s = 0; s < p.n_split; ++s) {
-      const float* d = sp + (s * kMaxG + h) * kSpPart;
-      const float ms = __ldcg(d);
-      if (ms == -INFINITY) continue;
-      const float f = exp2f(ms - M);
-      L += __ldcg(d + 1) * f;
-      O += __ldcg(d + 4 + c) * f;
-    }
-    p.out[((size_t)b * p.H + kvh * p.G + h) * kD + c] = O / L;
+  for (int i = threadIdx.x; i < p.n_split * p.G; i += kSpThreads) {
+    const int s = i / p.G, h = i % p.G;
+    s_f[s][h] = __ldcg(sp + (s * kMaxG + h) * kSpPart);
+    s_l[s][h] = __ldcg(sp + (s * kMaxG + h) * kSpPart + 1);
   }
+  __syncthreads();
+  if (threadIdx.x < p.G) {
+    const int h = threadIdx.x;
+    float M = -INFINITY;
+    for (int s = 0; s < p.n_split; ++s) M = fmaxf(M, s_f[s][h]);
+    float L = 0.f;
+    for (int s = 0; s < p.n_split; ++s) {
+      const float f = s_f[s][h] == -INFINITY ? 0.f : exp2f(s_f[s][h] - M);
+      s_f[s][h] = f;
+      L += s_l[s][h] * f;
+    }
+    s_L[h] = L;
+  }
+  __syncthreads();
+  for (int c = threadIdx.x; c < kD; c += kSpThreads)
+    for (int h = 0; h < p.G; ++h) {
+      float O = 0.f;
+#pragma unroll 8
+      for (int s = 0; s < p.n_split; ++s) O += __ldcg(sp + (s * kMaxG + h) * kSpPart + 4 + c) * s_f[s][h];
+      p.out[((size_t)b * p.H + kvh * p.G + h) * kD + c] = O / s_L[h];
+    }
   if (threadIdx.x == 0) p.ticket[seg] = 0u;
 }
 
 int sparse_splits(int n_seg, int entries, int num_sms) {
   const int nrun = (entries + kSpRun - 1) / kSpRun;
-  int s = (2 * num_sms) / (n_seg > 0 ? n_seg : 1);
+  int s = (JFA_SP_CTAS_PER_SM * num_sms) / (n_seg > 0 ? n_seg : 1);
   const int by_work = (nrun + kSpWarps - 1) / kSpWarps;  // at least one run per warp
   if (s > by_work) s = by_work;
   if (s > kSpMaxSplit) s = kSpMaxSplit;

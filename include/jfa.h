@@ -135,6 +135,8 @@ typedef struct jfa_workspace_layout {
   size_t off_bkeys;      /* uint32 [B][H_kv][capacity/128]: per 128-token
                             block the largest selection score of the FP4
                             scan, as an order-preserving key                 */
+  size_t off_chan;       /* per (sequence, KV head) the critical channels of
+                            jfa_channel_scores and the query at them         */
   int32_t max_topk;
   int32_t partial_slots; /* slots of off_partials                             */
   int32_t cand_cap;      /* list entries per segment                          */
