@@ -28,6 +28,7 @@
 #pragma once
 
 #include <cooperative_groups.h>
+#include <mutex>
 
 #include "finish_params.cuh"
 #include "jfa_approx.cuh"
@@ -1107,6 +1108,8 @@ static int launch_finish_t(const FinishParams& fp, int n_seg, int nq_max, cudaSt
   constexpr size_t smem = fin_smem_bytes<G>();
   static bool configured[64] = {false};
   static int memo_seg[64][8] = {{0}}, memo_c[64][8] = {{0}};  // cluster size per (device, key)
+  static std::mutex mu;  // host threads launching on one device share the tables
+  std::lock_guard<std::mutex> lock(mu);
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !configured[dev]) {

@@ -6,8 +6,9 @@
 // Every (sequence, KV head) has E = k + (n_ctx - N_q) entries: idx[0..k)
 // (token indices, -1 = none) then the tail tokens N_q .. n_ctx - 1.  A CTA
 // takes an even share of the entries in runs of 16; each of its 4 warps
-// streams its runs' K and V rows (bf16, 256 B each) into a private 3-stage
-// ring (cp.async, XOR-swizzled 16-byte chunks) and runs, per run:
+// streams its runs' K and V rows (bf16, 256 B each) into a private 2-stage
+// ring (cp.async, XOR-swizzled 16-byte chunks; 3 CTAs per SM: more warps
+// beat deeper rings here, measured) and runs, per run:
 //   logits   S^T = q K^T on mma.sync m16n8k16 (bf16 in, fp32 accumulate),
 //            rows = the KV head's query heads, so each lane holds the
 //            logits of head lane/4 for 4 of the 16 tokens;
@@ -26,10 +27,10 @@ namespace jfa {
 #define JFA_SP_WARPS 4
 #endif
 #ifndef JFA_SP_STAGES
-#define JFA_SP_STAGES 3
+#define JFA_SP_STAGES 2
 #endif
 #ifndef JFA_SP_CTAS_PER_SM
-#define JFA_SP_CTAS_PER_SM 2
+#define JFA_SP_CTAS_PER_SM 3
 #endif
 constexpr int kSpWarps = JFA_SP_WARPS;
 constexpr int kSpThreads = 32 * kSpWarps;

@@ -17,6 +17,8 @@
 //      first in list order; one ordered pass writes the chosen indices,
 //      already ascending; it then clears the segment's histogram and counters
 //      for the next call (the workspace starts zero-filled).
+#include <mutex>
+
 #include "jfa_blocks.cuh"
 
 namespace jfa {
@@ -392,8 +394,10 @@ namespace jfa {
 // device; the host-side name is only a stand-in, never a device address).
 static uint32_t* noalloc_scratch() {
   static uint32_t* addr[64] = {nullptr};
+  static std::mutex mu;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
   if (addr[dev] == nullptr) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_topk_scratch) != cudaSuccess || p == nullptr) return nullptr;
@@ -423,8 +427,12 @@ extern "C" int jfa_topk_noalloc(const float* scores, int32_t n_seg, int32_t stri
   }
   uint32_t* scratch = noalloc_scratch();
   if (scratch == nullptr) return JFA_ERR_CUDA;
-  // histogram and counters must start at zero; the previous call's contents remain
-  if (cudaMemsetAsync(scratch, 0, kNoAllocCountOff * sizeof(uint32_t), st) != cudaSuccess)
+  // the histogram and counters of the rows this call uses must start at zero
+  // (the final kernel clears its row after use; an earlier call that stopped
+  // short may not have): only those rows are cleared
+  if (cudaMemsetAsync(scratch, 0, (size_t)n_seg * jfa::kHistBins * sizeof(uint32_t), st) != cudaSuccess ||
+      cudaMemsetAsync(scratch + kNoAllocHistWords, 0, (size_t)n_seg * jfa::kCtrStride * sizeof(uint32_t),
+                      st) != cudaSuccess)
     return JFA_ERR_CUDA;
   TopkBufs b;
   b.scores = scores;

@@ -245,7 +245,8 @@ int jfa_topk_blocks(const jfa_geom* geom, int32_t n_blocks, void* ws, int32_t* i
  * parts of the array that
  * must start at zero and otherwise reuses the previous call's contents, so
  * calls that overlap on the GPU (other streams, other threads) race: keep
- * them on one stream. */
+ * them on one stream, and the stream must belong to the current device (the
+ * array looked up is the current device's). */
 int jfa_topk_noalloc(const float* scores, int32_t n_seg, int32_t stride,
                      int32_t n_scores, int32_t k, int32_t* idx, void* stream);
 

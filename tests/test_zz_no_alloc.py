@@ -51,3 +51,16 @@ def test_noalloc_topk_rejects_sizes_beyond_its_scratch():
     big = torch.zeros(2, 262144, dtype=torch.float32, device="cuda")
     idx2 = torch.empty(2, 8, dtype=torch.int32, device="cuda")
     assert _lib.jfa_topk_noalloc(big, 2, 262144, 262144, 8, idx2) == _lib.JFA_ERR_UNSUPPORTED
+
+
+@pytest.mark.gpu
+def test_noalloc_topk_k_at_least_n_scores_pads():
+    # k >= n_scores: every index in order, then -1
+    n_seg, nq, k = 3, 100, 128
+    src = torch.randn(n_seg, nq, dtype=torch.float32, device="cuda")
+    idx = torch.full((n_seg, k), -7, dtype=torch.int32, device="cuda")
+    _lib.check(_lib.jfa_topk_noalloc(src, n_seg, nq, nq, k, idx), "jfa_topk_noalloc")
+    torch.cuda.synchronize()
+    got = idx.cpu().numpy()
+    assert np.array_equal(got, O.topk_indices(src.double().cpu().numpy(), k))
+    assert np.all(got[:, :nq] == np.arange(nq)) and np.all(got[:, nq:] == -1)
