@@ -7,8 +7,10 @@
 //   1. block keys: the largest selection score of every 128-token block of
 //      the N_q quantized tokens (the last block may hold 64), as an
 //      order-preserving key, one warp per block (a float4 per lane, warp max);
-//   2. the n-th largest key by three radix levels (11 + 11 + 10 bits) over
-//      the block keys in shared memory; equal keys go to the lower block;
+//   2. the chosen blocks: up to 512 blocks by counting each block's rank
+//      directly, else the n-th largest key by three radix levels (11 + 11 +
+//      10 bits) over the block keys in shared memory; equal keys go to the
+//      lower block;
 //   3. one ordered pass lists the chosen blocks ascending, and every chosen
 //      block writes its 128 token indices (t >= N_q of a partial block and
 //      the unused tail of idx are -1).
@@ -18,6 +20,7 @@ namespace jfa {
 
 constexpr int kSelBlock = JFA_BLOCK_TOKENS;
 constexpr int kBlkThreads = 256;
+constexpr int kBlkDirect = 512;  // direct ranking up to this many blocks
 
 __global__ void __launch_bounds__(kBlkThreads) block_select_kernel(const float* scores,
                                                                    const uint32_t* bkeys, int capacity,
@@ -63,10 +66,26 @@ __global__ void __launch_bounds__(kBlkThreads) block_select_kernel(const float* 
   }
   __syncthreads();
 
-  // 2. the n_eff-th largest block key (n_eff = min(n_sel, nb))
+  // 2. which blocks are chosen (n_eff = min(n_sel, nb) of them).  Up to
+  // kBlkDirect blocks every block's rank is counted directly (flags in
+  // hist[]): a radix histogram of a few hundred near-equal maxima would
+  // serialize its shared-memory atomics on a handful of bins.  Beyond that,
+  // the n_eff-th largest key by three radix levels.
   const int n_eff = min(n_sel, nb);
+  const bool direct = n_eff < nb && nb <= kBlkDirect;
   uint32_t kstar = 0, r = (uint32_t)n_eff;
-  if (n_eff < nb) {
+  if (direct) {
+    for (int i = tid; i < nb; i += kBlkThreads) {
+      const uint32_t mine = keys[i];
+      uint32_t rank = 0;
+      for (int c = 0; c < nb; ++c) {
+        const uint32_t o = keys[c];
+        rank += (o > mine) | ((o == mine) & (c < i));
+      }
+      hist[i] = rank < (uint32_t)n_eff ? 1u : 0u;
+    }
+    __syncthreads();
+  } else if (n_eff < nb) {
     const int shifts[3] = {21, 10, 0};
     const int bits[3] = {11, 11, 10};
     uint32_t prefix = 0;
@@ -93,25 +112,29 @@ __global__ void __launch_bounds__(kBlkThreads) block_select_kernel(const float* 
   // [t*per, (t+1)*per); the equal keys before a thread decide its ties
   const int per = (nb + kBlkThreads - 1) / kBlkThreads;
   const int i0 = min(nb, tid * per), i1 = min(nb, i0 + per);
+  const bool radix = n_eff < nb && !direct;
+  auto take_at = [&](int i, uint32_t e) -> bool {
+    if (n_eff >= nb) return true;
+    if (direct) return hist[i] != 0u;
+    return keys[i] > kstar || (keys[i] == kstar && e < r);
+  };
   uint32_t tot;
   uint32_t n_eq = 0;
-  if (n_eff < nb)
+  if (radix)
     for (int i = i0; i < i1; ++i) n_eq += keys[i] == kstar;
   uint32_t er = block_prefix_excl(n_eq, scratch, &tot);
   uint32_t nc = 0;
   {
     uint32_t e2 = er;
     for (int i = i0; i < i1; ++i) {
-      const bool take = n_eff >= nb || keys[i] > kstar || (keys[i] == kstar && e2 < r);
-      nc += take;
-      e2 += (n_eff < nb && keys[i] == kstar) ? 1u : 0u;
+      nc += take_at(i, e2);
+      e2 += (radix && keys[i] == kstar) ? 1u : 0u;
     }
   }
   uint32_t pos = block_prefix_excl(nc, scratch, &tot);
   for (int i = i0; i < i1; ++i) {
-    const bool take = n_eff >= nb || keys[i] > kstar || (keys[i] == kstar && er < r);
-    if (take) chosen[pos++] = (uint32_t)i;
-    er += (n_eff < nb && keys[i] == kstar) ? 1u : 0u;
+    if (take_at(i, er)) chosen[pos++] = (uint32_t)i;
+    er += (radix && keys[i] == kstar) ? 1u : 0u;
   }
   __syncthreads();
 
