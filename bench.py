@@ -50,6 +50,8 @@ def parse(argv=None):
                     help="print only the NVFP4 step lines (one JSON line per workload)")
     ap.add_argument("--only-channel", action="store_true",
                     help="print only the critical-channel step line of the workload")
+    ap.add_argument("--only-onebit", action="store_true",
+                    help="print only the 1-bit dense-attention line of the workload")
     return ap.parse_args(argv)
 
 
@@ -793,6 +795,70 @@ def per_config_channel(args, dev, name: str, r: int) -> dict:
     return d
 
 
+def per_config_onebit(args, dev, name: str) -> dict:
+    """1-bit KV cache with dense attention (TailorKV review): jfa_onebit_attend
+    over every quantized token and the exact tail.  Copies of the pool
+    (together larger than L2) rotate."""
+    import torch
+
+    import bit_kv_cache_jfa_b200 as jfa
+    from bit_kv_cache_jfa_b200 import _lib
+    import workloads as W
+    w = W.WORKLOADS[name]
+    cap = 64 * -(-w.ctx // 64)
+    k_all, v_all = W.gen_kv_device(w, dev, W.gen_q(w))
+    q = W.gen_q(w).to(dev)
+    n_seg = w.batch * w.kv_heads
+    rec_bytes = n_seg * (w.n_quant // 64) * 3584
+    n_copies = 1 + -(-L2_BYTES // max(1, rec_bytes))
+    ke = torch.zeros(w.batch, w.kv_heads, cap, 128, dtype=torch.bfloat16, device=dev)
+    ve = torch.zeros_like(ke)
+    ke[:, :, :w.ctx], ve[:, :, :w.ctx] = k_all, v_all
+    del k_all, v_all
+    copies = []
+    ws = None
+    for c in range(n_copies):
+        cache = jfa.OneBitCache(w.batch, w.heads, w.kv_heads, cap, device=dev)
+        if ws is None:
+            ws = jfa.Workspace(cache, 64, device=dev)
+        cache.sync(ke, ve, w.ctx, ws)
+        copies.append((cache, cache.geom(w.ctx)))
+    out = torch.empty(w.batch, w.heads, 128, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sp = stream.cuda_stream
+    scale = W.default_scale(w)
+
+    def step(i):
+        cache, g = copies[i % n_copies]
+        _lib.check(_lib.jfa_onebit_attend(g, cache.pool, q, scale, ke, ve, 0, ws.buf, out, sp),
+                   "onebit_attend")
+
+    steps = max(20, min(args.steps, 200))
+    for i in range(max(3, args.warmup)):
+        step(i)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for i in range(steps):
+        step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    st, flag = _lib.jfa_check_error(copies[0][1], ws.buf, sp)
+    if flag:
+        raise RuntimeError(f"device error flag {flag:#x}")
+    peak, _ = measured_peaks()
+    alg = rec_bytes + n_seg * (w.ctx - w.n_quant) * 512 + w.batch * w.heads * 128 * (2 + 4)
+    d = {"workload": name, "format": "1-bit keys and values (3584 B per 64 tokens), exact tail",
+         "selection": "none: dense attention over every token", "exact_rows": "hbm",
+         "steps": steps, "us_per_step": ms * 1e3, "tokens_per_s": w.batch * w.ctx / (ms / 1e3),
+         "step_frac": alg / (ms / 1e3) / 1e9 / peak, "step_alg_bytes": alg, "copies": n_copies,
+         "calls": "jfa_onebit_attend (one launch)"}
+    del copies, ws
+    torch.cuda.empty_cache()
+    return d
+
+
 def run_jfa(args, w):
     import torch
 
@@ -875,6 +941,7 @@ def run_jfa(args, w):
         for name in ("qwen30b_k3v2_32k", "llama8b_k4v4_128k"):
             per_config.append(per_config_fp4(args, dev, name, 64))
         per_config.append(per_config_channel(args, dev, w.name, 16))
+        per_config.append(per_config_onebit(args, dev, w.name))
 
     tokens = w.batch * w.ctx
     value = world * tokens / (ms_max / 1e3)
@@ -940,6 +1007,12 @@ def main():
         dev = torch.device("cuda", dist_env()[2])
         torch.cuda.set_device(dev)
         print(json.dumps(per_config_channel(args, dev, w.name, 16)), flush=True)
+        return 0
+    if args.only_onebit:
+        import torch
+        dev = torch.device("cuda", dist_env()[2])
+        torch.cuda.set_device(dev)
+        print(json.dumps(per_config_onebit(args, dev, w.name)), flush=True)
         return 0
     if args.only_fp4:
         import torch

@@ -20,12 +20,14 @@ from ._lib import (  # noqa: F401  (re-exported C ABI names)
     jfa_append_decode_step, jfa_decode_step, jfa_decode_step_ragged,
     jfa_channel_decode_step, jfa_channel_pack, jfa_channel_scores,
     jfa_decode_step_launches, jfa_fp4_decode_step, jfa_fp4_pack_keys, jfa_fp4_pool_bytes,
+    jfa_onebit_attend, jfa_onebit_pack, jfa_onebit_pool_bytes,
     jfa_fp4_scores, jfa_pack_kv, jfa_sparse_attend, jfa_topk, jfa_topk_blocks,
     jfa_unpack_record, jfa_workspace_layout_get, load)
 
 __all__ = ["KVCache", "Workspace", "decode_step", "decode_step_blocks", "decode_step_ragged",
            "append_decode_step", "FP4KeyPool", "fp4_decode_step", "sparse_attend",
-           "ChannelKeys", "channel_decode_step", "DecodeGraph", "JfaError", "load"]
+           "ChannelKeys", "channel_decode_step", "OneBitCache", "onebit_attend", "DecodeGraph",
+           "JfaError", "load"]
 
 
 def _torch():
@@ -303,6 +305,48 @@ def channel_decode_step(keys: ChannelKeys, n_ctx: int, q, r: int, k: int, k_exac
                                        k, idx, k_exact, v_exact, exact_on_host, ws.buf, out,
                                        stream), "jfa_channel_decode_step")
     return out, idx
+
+
+class OneBitCache:
+    """One layer's 1-bit KV cache (records of 64-token groups packed from the
+    exact bf16 rows; device buffer owned by torch)."""
+
+    def __init__(self, batch: int, num_heads: int, num_kv_heads: int, capacity: int,
+                 device="cuda", head_dim: int = 128):
+        torch = _torch()
+        self.batch, self.num_heads, self.num_kv_heads = batch, num_heads, num_kv_heads
+        self.capacity, self.head_dim = capacity, head_dim
+        self.n_packed = 0
+        rc, nbytes = _lib.jfa_onebit_pool_bytes(self.geom(0))
+        check(rc, "jfa_onebit_pool_bytes")
+        self.pool = torch.zeros(nbytes, dtype=torch.uint8, device=device)
+
+    def geom(self, n_ctx: int = 0) -> Geom:
+        return Geom(self.batch, self.num_heads, self.num_kv_heads, self.head_dim, self.capacity,
+                    4, 4, n_ctx)
+
+    def sync(self, k_exact, v_exact, n_ctx: int, ws: "Workspace", stream=None) -> None:
+        """Pack every group below N_q of a context of n_ctx tokens."""
+        nq = 0 if n_ctx <= 0 else 64 * ((n_ctx - 1) // 64)
+        if nq > self.n_packed:
+            check(_lib.jfa_onebit_pack(self.geom(nq), self.n_packed, nq, k_exact, v_exact,
+                                       self.pool, ws.buf, stream), "jfa_onebit_pack")
+            self.n_packed = nq
+
+
+def onebit_attend(cache: OneBitCache, n_ctx: int, q, k_exact, v_exact, ws: Workspace, scale=None,
+                  out=None, exact_on_host: bool = False, stream=None):
+    """Dense attention over the 1-bit tokens and the exact tail; returns out
+    fp32 [B, H, 128]."""
+    torch = _torch()
+    if scale is None:
+        scale = default_scale(cache.head_dim)
+    if out is None:
+        out = torch.empty(cache.batch, cache.num_heads, cache.head_dim, dtype=torch.float32,
+                          device=q.device)
+    check(_lib.jfa_onebit_attend(cache.geom(n_ctx), cache.pool, q, float(scale), k_exact, v_exact,
+                                 exact_on_host, ws.buf, out, stream), "jfa_onebit_attend")
+    return out
 
 
 class DecodeGraph:

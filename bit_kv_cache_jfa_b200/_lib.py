@@ -111,6 +111,11 @@ SIGNATURES = {
     "jfa_fp4_decode_step": (c_int32, [POINTER(Geom), c_void_p, c_void_p, c_float, c_int32,
                                       c_void_p, c_void_p, c_void_p, c_int32, c_void_p, c_void_p,
                                       c_void_p]),
+    "jfa_onebit_pool_bytes": (c_int32, [POINTER(Geom), POINTER(c_size_t)]),
+    "jfa_onebit_pack": (c_int32, [POINTER(Geom), c_int32, c_int32, c_void_p, c_void_p, c_void_p,
+                                  c_void_p, c_void_p]),
+    "jfa_onebit_attend": (c_int32, [POINTER(Geom), c_void_p, c_void_p, c_float, c_void_p, c_void_p,
+                                    c_int32, c_void_p, c_void_p, c_void_p]),
     "jfa_channel_pack": (c_int32, [POINTER(Geom), c_int32, c_int32, c_void_p, c_void_p, c_void_p,
                                    c_void_p]),
     "jfa_channel_scores": (c_int32, [POINTER(Geom), c_void_p, c_void_p, c_void_p, c_float,
@@ -252,6 +257,24 @@ def jfa_fp4_decode_step(geom, pool, q, scale, n_blocks, idx, k_exact, v_exact, e
     return load().jfa_fp4_decode_step(ctypes.byref(geom), _ptr(pool), _ptr(q), scale, n_blocks,
                                       _ptr(idx), _ptr(k_exact), _ptr(v_exact), int(exact_on_host),
                                       _ptr(ws), _ptr(out), _stream(stream))
+
+
+def jfa_onebit_pool_bytes(geom) -> tuple[int, int]:
+    n = c_size_t(0)
+    rc = load().jfa_onebit_pool_bytes(ctypes.byref(geom), ctypes.byref(n))
+    return rc, n.value
+
+
+def jfa_onebit_pack(geom, n_from, n_to, k_src, v_src, pool, ws, stream=None) -> int:
+    return load().jfa_onebit_pack(ctypes.byref(geom), n_from, n_to, _ptr(k_src), _ptr(v_src),
+                                  _ptr(pool), _ptr(ws), _stream(stream))
+
+
+def jfa_onebit_attend(geom, pool, q, scale, k_exact, v_exact, exact_on_host, ws, out,
+                      stream=None) -> int:
+    return load().jfa_onebit_attend(ctypes.byref(geom), _ptr(pool), _ptr(q), scale, _ptr(k_exact),
+                                    _ptr(v_exact), int(exact_on_host), _ptr(ws), _ptr(out),
+                                    _stream(stream))
 
 
 def jfa_channel_pack(geom, n_from, n_to, k_src, k_t, k_max, stream=None) -> int:

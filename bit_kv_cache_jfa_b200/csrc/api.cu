@@ -348,6 +348,44 @@ int jfa_channel_decode_step(const jfa_geom* geom, const uint16_t* k_t, const flo
   return rc;
 }
 
+// ---------------------------------------------------------------------------
+// 1-bit KV cache, dense attention
+// ---------------------------------------------------------------------------
+int jfa_onebit_pool_bytes(const jfa_geom* geom, size_t* pool_bytes) {
+  if (!geom_ok(geom) || !pool_bytes) return JFA_ERR_INVALID_ARG;
+  *pool_bytes = (size_t)geom->batch * geom->num_kv_heads * (geom->capacity / kKG) * kOneBitRecBytes;
+  return JFA_OK;
+}
+
+int jfa_onebit_pack(const jfa_geom* geom, int32_t n_from, int32_t n_to, const uint16_t* k_src,
+                    const uint16_t* v_src, void* pool, void* ws, void* stream) {
+  if (!geom_ok(geom) || !pool || !aligned(pool, 16) || !ws || !aligned(ws, 256))
+    return JFA_ERR_INVALID_ARG;
+  if (n_from < 0 || n_to < n_from || n_to > geom->capacity || n_from % kKG || n_to % kKG)
+    return JFA_ERR_INVALID_ARG;
+  if (n_to == n_from) return JFA_OK;
+  if (!k_src || !v_src || !aligned(k_src, 16) || !aligned(v_src, 16)) return JFA_ERR_INVALID_ARG;
+  jfa_workspace_layout L;
+  workspace_layout(*geom, 1, &L);
+  return launch_onebit_pack(*geom, n_from / kKG, n_to / kKG, k_src, v_src, static_cast<uint8_t*>(pool),
+                            reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + L.off_flag),
+                            static_cast<cudaStream_t>(stream));
+}
+
+int jfa_onebit_attend(const jfa_geom* geom, const void* pool, const uint16_t* q, float scale,
+                      const uint16_t* k_exact, const uint16_t* v_exact, int32_t exact_on_host,
+                      void* ws, float* out, void* stream) {
+  if (!geom_ok(geom) || geom->n_ctx < 1 || !pool || !aligned(pool, 16) || !q || !aligned(q, 16) ||
+      !(scale > 0.f) || !k_exact || !v_exact || !aligned(k_exact, 16) || !aligned(v_exact, 16) || !ws ||
+      !aligned(ws, 256) || !out || !aligned(out, 16))
+    return JFA_ERR_INVALID_ARG;
+  (void)exact_on_host;  // the tail rows are read with plain loads either way
+  jfa_workspace_layout L;
+  workspace_layout(*geom, 1, &L);
+  return launch_onebit_attend(*geom, static_cast<const uint8_t*>(pool), q, scale, k_exact, v_exact,
+                              static_cast<uint8_t*>(ws), L, out, static_cast<cudaStream_t>(stream));
+}
+
 int jfa_correct_merge(const jfa_geom* geom, const jfa_cache* cache, const uint16_t* q,
                       float scale, const int32_t* idx, int32_t k, const uint16_t* k_exact,
                       const uint16_t* v_exact, int32_t exact_on_host, void* ws, float* out,

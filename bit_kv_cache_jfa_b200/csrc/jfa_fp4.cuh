@@ -101,6 +101,14 @@ int launch_channel_pack(const jfa_geom& g, int g_from, int g_to, const uint16_t*
 int launch_channel_scores(const jfa_geom& g, const uint16_t* k_t, const float* k_max, const uint16_t* q,
                           float scale, int r, uint8_t* ws, const jfa_workspace_layout& L,
                           cudaStream_t st);
+// 1-bit KV pool: records of 64-token groups quantized at 1 bit from the exact
+// bf16 rows; dense attention over every quantized token and the exact tail.
+constexpr int kOneBitRecBytes = 3584;
+int launch_onebit_pack(const jfa_geom& g, int g_from, int g_to, const uint16_t* k_src,
+                       const uint16_t* v_src, uint8_t* pool, uint32_t* flag, cudaStream_t st);
+int launch_onebit_attend(const jfa_geom& g, const uint8_t* pool, const uint16_t* q, float scale,
+                         const uint16_t* k_exact, const uint16_t* v_exact, uint8_t* ws,
+                         const jfa_workspace_layout& L, float* out, cudaStream_t st);
 // Splits per segment of the sparse attention (host rule shared with the
 // workspace sizing): at most kSpMaxSplit, and n_seg * splits <= max(n_seg, 512).
 constexpr int kSpMaxSplit = 32;

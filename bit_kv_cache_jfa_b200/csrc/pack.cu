@@ -7,7 +7,7 @@
 //   code  = round-half-even((x - zero) / scale), clipped; both quotients fp64.
 // Keys: one (scale, zero) per (64-token group, channel); values: one per
 // (token, 32-channel group).
-#include "jfa_internal.cuh"
+#include "jfa_quant.cuh"
 
 namespace jfa {
 
@@ -31,25 +31,6 @@ __device__ __forceinline__ const uint16_t* token_row(const uint16_t* tail, const
   if (tau < p.n0) return tail + ((size_t)seg * kTail + (tau - p.nq0)) * kD;
   return fresh + ((size_t)seg * p.n_new + (tau - p.n0)) * kD;
 }
-
-__device__ __forceinline__ void quant_params(double mn, double mx, int bits, uint16_t& zbits,
-                                             uint16_t& sbits, double& z, double& s) {
-  zbits = fp16_bits_rd(mn);
-  z = (double)__half2float(__ushort_as_half(zbits));
-  sbits = fp16_bits_ru((mx - z) / (double)((1 << bits) - 1));
-  s = (double)__half2float(__ushort_as_half(sbits));
-}
-
-__device__ __forceinline__ uint32_t quant_code(double x, double z, double s, int bits) {
-  if (s == 0.0) return 0u;
-  double c = rint((x - z) / s);
-  double lv = (double)((1 << bits) - 1);
-  c = c < 0.0 ? 0.0 : (c > lv ? lv : c);
-  return (uint32_t)c;
-}
-
-__device__ __forceinline__ bool finite_h(uint16_t b) { return (b & 0x7C00u) != 0x7C00u; }
-__device__ __forceinline__ float bf(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
 
 // Quantize one 64-token group staged in shared memory (bf16 bits, token
 // rows) into a zeroed record image rb; all 256 threads take part.

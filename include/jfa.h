@@ -474,6 +474,40 @@ int jfa_channel_decode_step(const jfa_geom* geom, const uint16_t* k_t, const flo
                             const uint16_t* k_exact, const uint16_t* v_exact,
                             int32_t exact_on_host, void* ws, float* out, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * 1-bit KV cache with dense attention (TailorKV review: layers whose attention
+ * is spread over many tokens keep the whole cache at 1 bit per number and
+ * attend over all of it, an FP16 x INT1 product, with no tokens fetched back).
+ * The quantization is jfa_pack_kv's rule at b = 1 (keys per channel over
+ * 64-token groups, values per token over 32-channel groups, fp16 zero point
+ * = the minimum rounded down, fp16 scale = the range rounded up, code = the
+ * nearer end, ties to 0).  Geometry as for the NVFP4 calls (key_bits and
+ * val_bits unused; capacity a multiple of 64).
+ * ------------------------------------------------------------------------- */
+#define JFA_ONEBIT_RECORD_BYTES 3584 /* bytes per (sequence, KV head, 64-token group) */
+
+/* Pool of B * H_kv * capacity/64 records, [B][H_kv][capacity/64][record], in a
+ * layout private to this library (key bit-planes, value bit-rows and their
+ * fp16 scales and zeros).  Caller-allocated, 16-byte aligned. */
+int jfa_onebit_pool_bytes(const jfa_geom* geom, size_t* pool_bytes);
+
+/* Quantize the 64-token groups covering tokens [n_from, n_to) (multiples of
+ * 64) of every (sequence, KV head) from the exact bf16 rows
+ *   k_src, v_src : [B][H_kv][capacity][128] (device or pinned host).
+ * A non-finite scale or zero sets JFA_DEVERR_NONFINITE_QUANT.  Stream-ordered. */
+int jfa_onebit_pack(const jfa_geom* geom, int32_t n_from, int32_t n_to, const uint16_t* k_src,
+                    const uint16_t* v_src, void* pool, void* ws, void* stream);
+
+/* Dense attention: out[b, h] = softmax over every token t < n_ctx of
+ * (scale q_h . k_t) applied to v_t, where tokens t < N_q use the dequantized
+ * 1-bit keys and values of the pool (every group below N_q packed) and the
+ * tail N_q .. n_ctx - 1 the exact rows k_exact / v_exact [B][H_kv][capacity]
+ * [128] (device, or pinned host with exact_on_host = 1).  fp32 arithmetic.
+ * One launch.  Stream-ordered. */
+int jfa_onebit_attend(const jfa_geom* geom, const void* pool, const uint16_t* q, float scale,
+                      const uint16_t* k_exact, const uint16_t* v_exact, int32_t exact_on_host,
+                      void* ws, float* out, void* stream);
+
 /* Number of warps jfa_decode_scores splits the quantized groups over on the
  * current device (0 on a bad geometry or when no group is quantized).  Warp w
  * takes a contiguous range of the flattened (segment, group) list and writes

@@ -185,3 +185,17 @@ def test_channel_argument_checks(lib):
                                        256) == bad                          # k = 0
     assert lib.jfa_channel_decode_step(g, 256, 256, 256, 0.1, 16, 4097, 256, 256, 256, 0, 256,
                                        256) == bad                          # k > JFA_MAX_TOPK
+
+
+def test_onebit_argument_checks(lib):
+    rc, n = lib.jfa_onebit_pool_bytes(G(capacity=4096))
+    assert rc == 0 and n == 2 * 2 * 64 * 3584
+    g = G(capacity=4096, n_ctx=1000)
+    bad = lib.JFA_ERR_INVALID_ARG
+    assert lib.jfa_onebit_pack(g, 0, 100, 256, 256, 256, 256) == bad       # not a group edge
+    assert lib.jfa_onebit_pack(g, 0, 4160, 256, 256, 256, 256) == bad      # past capacity
+    assert lib.jfa_onebit_pack(g, 64, 64, 256, 256, 256, 256) == 0         # nothing to do
+    assert lib.jfa_onebit_attend(g, 256, 256, 0.0, 256, 256, 0, 256, 256) == bad   # scale
+    assert lib.jfa_onebit_attend(g, 8, 256, 0.1, 256, 256, 0, 256, 256) == bad     # pool alignment
+    assert lib.jfa_onebit_attend(G(capacity=4096, n_ctx=0), 256, 256, 0.1, 256, 256, 0, 256,
+                                 256) == bad                                     # empty context

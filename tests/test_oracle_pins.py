@@ -47,7 +47,7 @@ def test_quantization_golden(case):
     assert int(scale.view(np.uint16)[0]) == int(case["scale_bits"][0], 16)
 
 
-@pytest.mark.parametrize("bits", [2, 3, 4])
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
 def test_quantization_error_bound(bits):
     rng = np.random.default_rng(bits)
     x = _bf16(rng.standard_normal((500, 64)) * rng.choice([0.01, 1, 10, 300], (500, 1)))
@@ -292,7 +292,7 @@ def test_k_at_least_nq_is_exact_attention(kb, vb):
             assert np.allclose(res.out[b, h], ref, rtol=1e-11, atol=1e-12)
 
 
-@pytest.mark.parametrize("kb,vb", [(3, 2), (4, 4)])
+@pytest.mark.parametrize("kb,vb", [(3, 2), (4, 4), (1, 1)])
 def test_k_zero_is_attention_over_dequantized_plus_exact_tail(kb, vb):
     w, q, k, v, cache = _small(kb=kb, vb=vb, lognormal=True)
     scale = 0.07
@@ -759,3 +759,30 @@ def test_pins_reject_signed_channel_importance(monkeypatch):
     monkeypatch.setattr(O, "channel_importance", signed)
     with pytest.raises(AssertionError):
         test_channel_scores_hand_case()
+
+
+# --------------------------------------------------------------------------
+# 1-bit cache (TailorKV review: the whole cache at 1 bit, attended densely)
+# --------------------------------------------------------------------------
+def test_one_bit_two_level_data_reconstructs_exactly():
+    # every key channel group and value channel group takes two fp16-exact
+    # levels a < b with b - a fp16-exact: zero = a, scale = b - a, codes exact
+    rng = np.random.default_rng(51)
+    a = np.round(rng.standard_normal((1, 2, 1, 128)) * 4) / 4
+    d = rng.integers(1, 8, (1, 2, 1, 128)) / 4.0
+    bits = rng.integers(0, 2, (1, 2, 256, 128))
+    bits[:, :, 0], bits[:, :, 1] = 0, 1          # both levels in every group
+    bits[:, :, 64], bits[:, :, 65] = 0, 1
+    bits[:, :, 128], bits[:, :, 129] = 0, 1
+    bits[:, :, 192], bits[:, :, 193] = 0, 1
+    k = a + d * bits
+    lv = np.round(rng.standard_normal((1, 2, 256, 4, 1)) * 4) / 4
+    dv = rng.integers(1, 8, (1, 2, 256, 4, 1)) / 4.0
+    vb = rng.integers(0, 2, (1, 2, 256, 4, 32))
+    vb[..., 0], vb[..., 1] = 0, 1
+    v = (lv + dv * vb).reshape(1, 2, 256, 128)
+    k = np.concatenate([k, np.zeros((1, 2, 10, 128))], axis=2)
+    v = np.concatenate([v, np.zeros((1, 2, 10, 128))], axis=2)
+    c = O.pack_cache(k, v, 266, 1, 1)
+    assert np.array_equal(c.k_hat(), k[:, :, :256]) and np.array_equal(c.v_hat(), v[:, :, :256])
+    assert np.array_equal(c.k_codes, bits) and np.array_equal(c.v_codes, vb.reshape(1, 2, 256, 128))
