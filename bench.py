@@ -44,7 +44,7 @@ def parse(argv=None):
     ap.add_argument("--cpu-rounds", type=int, default=3,
                     help="rounds of the oracle baseline (one segment per host process each)")
     ap.add_argument("--no-per-config", action="store_true",
-                    help="skip the K4V4 128K (HBM, host rows) and Qwen GQA-8 lines")
+                    help="skip the other workloads and variants (the per_config lines)")
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--only-fp4", action="store_true",
                     help="print only the NVFP4 step lines (one JSON line per workload)")
@@ -932,7 +932,8 @@ def run_jfa(args, w):
     per_config = []
     if not args.no_per_config and world == 1:
         for name, host in (("llama8b_k4v4_128k", False), ("llama8b_k4v4_128k", True),
-                           ("qwen30b_k3v2_32k", False)):
+                           ("qwen30b_k3v2_32k", False), ("llama70b_k3v2_32k_b8", False),
+                           ("llama70b_k4v4_128k_b8", False), ("llama70b_k3v2_8k_b1", False)):
             if name == w.name and host == args.host_resident:
                 continue
             per_config.append(per_config_line(args, dev, name, host))
