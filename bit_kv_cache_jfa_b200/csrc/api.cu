@@ -42,7 +42,7 @@ int workspace_layout(const jfa_geom& g, int max_topk, jfa_workspace_layout* out)
   L.off_wts = off;
   off = align_up(off + n_seg * (size_t)(g.capacity / kKG) * 4 * (G > 4 ? 2 : 1) * 32 * sizeof(uint32_t), 256);
   L.off_scan_hist = off;
-  off = align_up(off + n_seg * kScanHistStride * sizeof(uint32_t), 256);
+  off = align_up(off + n_seg * (size_t)scan_hist_reps((long long)n_seg) * kScanHistStride * sizeof(uint32_t), 256);
   L.off_hist = off;
   off += n_seg * kHistBins * sizeof(uint32_t);
   L.off_counters = off;

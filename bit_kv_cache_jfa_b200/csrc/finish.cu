@@ -22,6 +22,7 @@ int launch_finish(const jfa_geom& g, const SeqTable& t, const jfa_cache& c, cons
   fp.m_used = reinterpret_cast<const float*>(ws + L.off_mused);
   fp.wts = reinterpret_cast<const uint32_t*>(ws + L.off_wts);
   fp.hist = reinterpret_cast<uint32_t*>(ws + L.off_scan_hist);
+  fp.hist_reps = scan_hist_reps((long long)g.batch * g.num_kv_heads);
   fp.glists = reinterpret_cast<uint32_t*>(ws + L.off_cand);
   fp.idx_in = idx_in;
   fp.idx_out = idx_out;

@@ -589,9 +589,12 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const __grid_con
 
   const bool select = SELECT && k < nq;
   const int lo = min(nq, r * slice), hi = min(nq, lo + slice);
-  const uint32_t* hg = p.hist + (size_t)seg * kScanHistStride;
-  // the segment's largest selection key
-  const uint32_t top_key = select ? hg[kScanHistBins] : 0u;
+  const int R = p.hist_reps;
+  const uint32_t* hg = p.hist + (size_t)seg * R * kScanHistStride;
+  // the segment's largest selection key (the largest over the copies)
+  uint32_t top_key = 0u;
+  if (select)
+    for (int c = 0; c < R; ++c) top_key = max(top_key, hg[(size_t)c * kScanHistStride + kScanHistBins]);
 
   WarpPart<G> WP;
   WP.init();
@@ -618,7 +621,17 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const __grid_con
     for (;;) {
       const int wlo = max(0, whi - 4 * kFinThreads);
       const int b0 = wlo + 4 * tid;
-      const uint4 hv = b0 < whi ? *reinterpret_cast<const uint4*>(hg + b0) : make_uint4(0u, 0u, 0u, 0u);
+      uint4 hv = make_uint4(0u, 0u, 0u, 0u);
+      if (b0 < whi) {
+#pragma unroll 4
+        for (int c = 0; c < R; ++c) {
+          const uint4 h = *reinterpret_cast<const uint4*>(hg + (size_t)c * kScanHistStride + b0);
+          hv.x += h.x;
+          hv.y += h.y;
+          hv.z += h.z;
+          hv.w += h.w;
+        }
+      }
       if (tid == 0) s_bin = -1;
       uint32_t cum = above + block_suffix_excl(hv.x + hv.y + hv.z + hv.w, scratch);
       const uint32_t hb[4] = {hv.x, hv.y, hv.z, hv.w};
@@ -786,8 +799,8 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const __grid_con
   int mode = 0;
   if (select) {
     {  // the scan's histogram is consumed: clear it for the next scan
-      uint32_t* hc = p.hist + (size_t)seg * kScanHistStride;
-      for (int i = 4 * (r * kFinThreads + tid); i < kScanHistStride; i += 4 * C * kFinThreads)
+      uint32_t* hc = p.hist + (size_t)seg * R * kScanHistStride;
+      for (int i = 4 * (r * kFinThreads + tid); i < R * kScanHistStride; i += 4 * C * kFinThreads)
         *reinterpret_cast<uint4*>(hc + i) = make_uint4(0u, 0u, 0u, 0u);
     }
     if (tid < C) {
@@ -964,9 +977,9 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const __grid_con
     for (int i = tid; i < k; i += kFinThreads) out[i] = i < nq ? i : -1;
   }
   if (!select) {  // nothing reads the scan's histogram here: clear it
-    uint32_t* hg = p.hist + (size_t)seg * kScanHistStride;
-    for (int i = 4 * (r * kFinThreads + tid); i < kScanHistStride; i += 4 * C * kFinThreads)
-      *reinterpret_cast<uint4*>(hg + i) = make_uint4(0u, 0u, 0u, 0u);
+    uint32_t* hz = p.hist + (size_t)seg * R * kScanHistStride;
+    for (int i = 4 * (r * kFinThreads + tid); i < R * kScanHistStride; i += 4 * C * kFinThreads)
+      *reinterpret_cast<uint4*>(hz + i) = make_uint4(0u, 0u, 0u, 0u);
   }
 
   // ---- M1: the warps' partials into this CTA's partial P.run (per head the

@@ -17,7 +17,7 @@ struct FinishParams {
   const float* scan_part;  // per scan warp and segment: [slot][G][kPartStride]
   const float* m_used;     // [n_seg][ng_cap][8]: the scan's running maxima
   const uint32_t* wts;     // the scan's fp16 weights, [n_seg][ng_cap][4][NT][32] words
-  uint32_t* hist;          // [n_seg][kScanHistStride] (bins, largest key), zeroed here after use
+  uint32_t* hist;          // [n_seg][hist_reps][kScanHistStride] (bins, largest key), zeroed here after use
   uint32_t* glists;        // [n_seg][C][slice] chosen lists of the fallback
   const int32_t* idx_in;   // given index sets (no selection), [n_seg][k]
   int32_t* idx_out;        // [n_seg][k] (selection)
@@ -27,6 +27,7 @@ struct FinishParams {
   int gl_stride;           // uint32 entries of glists per segment
   long long scan_total;
   int scan_warps;
+  int hist_reps;           // copies of each segment's histogram (scan_hist_reps)
   float kappa;
   SeqTable seq;            // per-sequence lengths and the scan's group offsets
 };

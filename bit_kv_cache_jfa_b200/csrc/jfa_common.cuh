@@ -27,6 +27,12 @@ constexpr int kScanMinRecords = 2;       // records per scan warp at least (when
 constexpr int kScanHistBits = 15;        // selection-score histogram of the scan: top 15 key bits
 constexpr int kScanHistBins = 1 << kScanHistBits;
 constexpr int kScanHistStride = kScanHistBins + 32;  // per segment: the bins, then the largest key
+// Copies of each segment's scan histogram.  With few segments every scan warp
+// adds into the same few hot bins, and atomics on one address serialise in
+// L2; scan warp w adds into copy w mod R, and the readers sum the copies.
+__host__ __device__ __forceinline__ int scan_hist_reps(long long n_seg) {
+  return n_seg >= 32 ? 1 : (n_seg <= 2 ? 16 : (int)(32 / n_seg));
+}
 constexpr int kHistBins = 2048;          // top-k first-level histogram (11 key bits)
 constexpr int kCtrStride = 8;            // top-k counters per segment: [0] scan warps done, [2] b*, [3] keys above b*
 

@@ -42,12 +42,13 @@ struct ScanParams {
   float* partials;
   float* m_used;    // [n_seg][ng_cap][8]: running maxima per head
   uint32_t* wts;    // [n_seg][ng_cap][4][NT][32]: the fp16 weights, lane order
-  uint32_t* hist;   // [n_seg][kScanHistStride]: bins, then the largest key
+  uint32_t* hist;   // [n_seg][hist_reps][kScanHistStride]: bins, then the largest key
   uint32_t* flag;
   long long total;  // entries of the flattened (segment, group) list
   int ng_cap, capacity;
   int hkv, G, H, n_seg;
   int n_warps;
+  int hist_reps;    // histogram copies per segment
   float kappa;      // scale * log2(e): logits are kept in log2 units
   SeqTable seq;     // per-sequence lengths and group offsets
 };
@@ -113,6 +114,7 @@ __global__ void __launch_bounds__(ScanCfg<KB, VB, NT>::NW * 32, 1)
   const long long g0 = wg < W ? scan_range_begin(wg, W, T) : 0;
   const long long g1 = wg < W ? scan_range_begin(wg + 1, W, T) : 0;
   const bool has_work = g0 < g1;  // warp-uniform
+  const int hrep = (int)(wg % p.hist_reps);  // this warp's histogram copy
 
   uint8_t* ring = smem + (size_t)warp * S * REC;
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + (size_t)NW * S * REC) + warp * S;
@@ -377,7 +379,7 @@ __global__ void __launch_bounds__(ScanCfg<KB, VB, NT>::NW * 32, 1)
       float* srow = p.scores + (size_t)seg * p.capacity + (size_t)g * kKG + 16 * tig + gid;
       srow[0] = sc[0];
       srow[8] = sc[1];
-      uint32_t* hs = p.hist + (size_t)seg * kScanHistStride;
+      uint32_t* hs = p.hist + ((size_t)seg * p.hist_reps + hrep) * kScanHistStride;
       const uint32_t k0 = float_key(sc[0]), k1 = float_key(sc[1]);
       atomicAdd(hs + (k0 >> (32 - kScanHistBits)), 1u);
       atomicAdd(hs + (k1 >> (32 - kScanHistBits)), 1u);
@@ -535,6 +537,7 @@ int launch_scores(const jfa_geom& g, const SeqTable& t, const jfa_cache& c, cons
   sp.G = g.num_heads / g.num_kv_heads;
   sp.H = g.num_heads;
   sp.n_warps = plan.n_warps;
+  sp.hist_reps = scan_hist_reps(sp.n_seg);
   sp.kappa = scale * 1.4426950408889634f;
   if (g.key_bits == 3 && g.val_bits == 2) return launch_scan_g<3, 2>(sp, plan.n_ctas, pdl, st);
   if (g.key_bits == 4 && g.val_bits == 4) return launch_scan_g<4, 4>(sp, plan.n_ctas, pdl, st);

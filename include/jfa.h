@@ -119,10 +119,11 @@ typedef struct jfa_workspace_layout {
   size_t off_wts;        /* the scan's fp16 softmax weights of every quantized
                             token and query head, in a layout private to
                             this library (read by the correction)            */
-  size_t off_scan_hist;  /* uint32 [B][H_kv][32768 + 32]: histogram of the top
-                            15 bits of the selection keys, then the largest
-                            key, built by the scan and cleared by the
-                            finishing kernel                                  */
+  size_t off_scan_hist;  /* uint32 [B][H_kv][R][32768 + 32]: histogram of the
+                            top 15 bits of the selection keys, then the
+                            largest key, in R copies (R = 1 from 32 segments
+                            B*H_kv up, else 32/(B*H_kv), at most 16), built
+                            by the scan and cleared by the finishing kernel */
   size_t off_hist;       /* top-k histograms (jfa_topk)                       */
   size_t off_counters;   /* top-k counters (jfa_topk)                         */
   size_t off_cand;       /* top-k candidate lists                             */
