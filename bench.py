@@ -899,9 +899,10 @@ def run_jfa(args, w):
     unfused_ms = st.timed(st.step3, args.steps, 3)
     scan_avg = st.scan_ms(args.steps)
 
-    # end to end through the public API, two ways; every step copies q in from
-    # pinned host memory and the finishing kernel writes out straight into
-    # pinned host memory (out may be host-resident):
+    # end to end through the public API, two ways; every step takes q from
+    # pinned host memory (the step's first kernel copies it across the host
+    # link into the workspace) and the finishing kernel writes out straight
+    # into pinned host memory:
     #  - eager: one jfa_decode_step C-ABI call per step (decode_step);
     #  - graph: the step captured once per cache copy (DecodeGraph) and replayed
     q_host = st.q.cpu().pin_memory()
@@ -909,17 +910,15 @@ def run_jfa(args, w):
 
     def eager_step(i):
         cache, _, _, ke, ve = st.copies[i % st.n_copies]
-        st.q.copy_(q_host, non_blocking=True)
-        jfa.decode_step(cache, st.q, w.topk, ke, ve, st.ws, scale=st.scale, out=out_host,
+        jfa.decode_step(cache, q_host, w.topk, ke, ve, st.ws, scale=st.scale, out=out_host,
                         idx=st.idx, exact_on_host=bool(st.host), stream=st.sp)
 
     eager_ms = st.timed(eager_step, args.steps, max(3, args.warmup))
-    graphs = [jfa.DecodeGraph(cache, st.q, w.topk, ke, ve, st.ws, scale=st.scale, out=out_host,
+    graphs = [jfa.DecodeGraph(cache, q_host, w.topk, ke, ve, st.ws, scale=st.scale, out=out_host,
                               idx=st.idx, exact_on_host=bool(st.host))
               for cache, _, _, ke, ve in st.copies]
 
     def graph_step(i):
-        st.q.copy_(q_host, non_blocking=True)
         graphs[i % st.n_copies].replay()
 
     graph_ms = st.timed(graph_step, args.steps, max(3, args.warmup))

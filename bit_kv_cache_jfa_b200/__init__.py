@@ -105,13 +105,15 @@ def decode_step(cache: KVCache, q, k: int, k_exact, v_exact, ws: Workspace, scal
                 out=None, idx=None, exact_on_host: bool = False, stream=None):
     """One decode step for every sequence and query head.
 
-    q: bf16 [B, H, 128]; k_exact/v_exact: bf16 [B, H_kv, capacity, 128]
-    (device, or pinned host with exact_on_host=True).  Returns (out fp32
-    [B, H, 128], idx int32 [B, H_kv, k])."""
+    q: bf16 [B, H, 128], device or pinned host memory (a host query is
+    copied into the workspace by the step's first kernel); k_exact/v_exact:
+    bf16 [B, H_kv, capacity, 128] (device, or pinned host with
+    exact_on_host=True).  Returns (out fp32 [B, H, 128], idx int32
+    [B, H_kv, k]), on the cache's device unless given."""
     torch = _torch()
     if scale is None:
         scale = default_scale(cache.head_dim)
-    dev = q.device
+    dev = cache.groups.device  # q may be in pinned host memory
     if out is None:
         out = torch.empty(cache.batch, cache.num_heads, cache.head_dim, dtype=torch.float32,
                           device=dev)
@@ -131,7 +133,7 @@ def decode_step_blocks(cache: KVCache, q, n_blocks: int, k_exact, v_exact, ws: W
     torch = _torch()
     if scale is None:
         scale = default_scale(cache.head_dim)
-    dev = q.device
+    dev = cache.groups.device  # q may be in pinned host memory
     k = n_blocks * _lib.BLOCK_TOKENS
     if out is None:
         out = torch.empty(cache.batch, cache.num_heads, cache.head_dim, dtype=torch.float32,
@@ -153,7 +155,7 @@ def decode_step_ragged(cache: KVCache, seq_lens, q, k: int, k_exact, v_exact, ws
     torch = _torch()
     if scale is None:
         scale = default_scale(cache.head_dim)
-    dev = q.device
+    dev = cache.groups.device  # q may be in pinned host memory
     if out is None:
         out = torch.empty(cache.batch, cache.num_heads, cache.head_dim, dtype=torch.float32,
                           device=dev)
@@ -175,7 +177,7 @@ def append_decode_step(cache: KVCache, seq_lens, k_new, v_new, q, k: int, k_exac
     torch = _torch()
     if scale is None:
         scale = default_scale(cache.head_dim)
-    dev = q.device
+    dev = cache.groups.device  # q may be in pinned host memory
     if out is None:
         out = torch.empty(cache.batch, cache.num_heads, cache.head_dim, dtype=torch.float32,
                           device=dev)

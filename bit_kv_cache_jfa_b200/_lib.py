@@ -61,7 +61,7 @@ class WorkspaceLayout(ctypes.Structure):
                 ("off_hist", c_size_t), ("off_counters", c_size_t),
                 ("off_cand", c_size_t), ("off_sel", c_size_t),
                 ("off_fp4q", c_size_t), ("off_sparse", c_size_t), ("off_ticket", c_size_t),
-                ("off_bkeys", c_size_t), ("off_chan", c_size_t),
+                ("off_bkeys", c_size_t), ("off_chan", c_size_t), ("off_qstage", c_size_t),
                 ("max_topk", c_int32), ("partial_slots", c_int32), ("cand_cap", c_int32),
                 ("reserved", c_int32)]
 

@@ -68,6 +68,8 @@ int workspace_layout(const jfa_geom& g, int max_topk, jfa_workspace_layout* out)
   off = align_up(off + n_seg * (size_t)((g.capacity + kF4Tok - 1) / kF4Tok) * sizeof(uint32_t), 256);
   L.off_chan = off;
   off = align_up(off + n_seg * (size_t)kChanRecBytes, 256);
+  L.off_qstage = off;
+  off = align_up(off + (size_t)g.batch * g.num_heads * kD * sizeof(uint16_t), 256);
   L.total_bytes = off;
   *out = L;
   return JFA_OK;
@@ -414,6 +416,10 @@ int jfa_decode_step(const jfa_geom* geom, const jfa_cache* cache, const uint16_t
     return JFA_ERR_INVALID_ARG;
   if (!k_exact || !v_exact || !aligned(k_exact, 16) || !aligned(v_exact, 16))
     return JFA_ERR_INVALID_ARG;
+  jfa_workspace_layout L;
+  workspace_layout(*geom, k, &L);
+  const int sq = stage_query(*geom, &q, static_cast<uint8_t*>(ws), L, static_cast<cudaStream_t>(stream));
+  if (sq != JFA_OK) return sq;
   const int s = jfa_decode_scores(geom, cache, q, scale, ws, stream);
   if (s != JFA_OK) return s;
   return jfa_decode_finish(geom, cache, q, scale, k, idx, k_exact, v_exact, exact_on_host, ws,
@@ -447,6 +453,8 @@ static int ragged_step(const jfa_geom* geom, const SeqTable& t, const jfa_cache*
   jfa_workspace_layout L;
   workspace_layout(*geom, k, &L);
   uint8_t* w = static_cast<uint8_t*>(ws);
+  const int sq = stage_query(*geom, &q, w, L, st);
+  if (sq != JFA_OK) return sq;
   const int s = launch_scores(*geom, t, *cache, q, scale, w, L, st, pdl_scan);
   if (s != JFA_OK) return s;
   return launch_finish(*geom, t, *cache, q, scale, k, idx, nullptr, k_exact, v_exact, w, L, out, st);

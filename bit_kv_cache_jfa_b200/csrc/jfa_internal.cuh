@@ -29,6 +29,13 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
 // Workspace layout for (geometry, max_topk); host and device agree on it.
 int workspace_layout(const jfa_geom& g, int max_topk, jfa_workspace_layout* out);
 
+// A decode step's query: device (or managed) memory is used as it is; pinned
+// host memory is copied into the workspace's staging region by one kernel
+// (launched here) and *q is pointed there.  JFA_ERR_INVALID_ARG for pageable
+// host memory.
+int stage_query(const jfa_geom& g, const uint16_t** q, uint8_t* ws, const jfa_workspace_layout& L,
+                cudaStream_t st);
+
 // Per-sequence lengths of one call (the same for every KV head of a
 // sequence) and the offset of each sequence's first group in the flattened
 // (segment, group) list the scan splits: sequence b, KV head h, group g is

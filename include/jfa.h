@@ -138,6 +138,8 @@ typedef struct jfa_workspace_layout {
                             scan, as an order-preserving key                 */
   size_t off_chan;       /* per (sequence, KV head) the critical channels of
                             jfa_channel_scores and the query at them         */
+  size_t off_qstage;     /* bf16 [B][H][128]: the query of a decode step
+                            given in pinned host memory, copied here first   */
   int32_t max_topk;
   int32_t partial_slots; /* slots of off_partials                             */
   int32_t cand_cap;      /* list entries per segment                          */
@@ -285,7 +287,13 @@ int jfa_correct_merge(const jfa_geom* geom, const jfa_cache* cache,
 /* The whole decode step (scores, top-k, correct+merge) in one call, with the
  * same results as the three calls in order (idx identical, out to rounding):
  * the scan, then one kernel in which a thread-block cluster per (sequence,
- * KV head) selects, corrects and merges.  idx is written as by jfa_topk. */
+ * KV head) selects, corrects and merges.  idx is written as by jfa_topk.
+ *   q : bf16 [B][H][128], 16-B aligned: device memory, or pinned host
+ *       memory (the step then first copies it into the workspace's
+ *       off_qstage region with one kernel, which reads it across the host
+ *       link while the previous kernel in the stream is still running;
+ *       pageable host memory: JFA_ERR_INVALID_ARG).  The same holds for
+ *       jfa_decode_step_ragged and jfa_append_decode_step. */
 int jfa_decode_step(const jfa_geom* geom, const jfa_cache* cache,
                     const uint16_t* q, float scale, int32_t k, int32_t* idx,
                     const uint16_t* k_exact, const uint16_t* v_exact,
@@ -361,8 +369,9 @@ int jfa_unpack_record(int32_t key_bits, int32_t val_bits, const void* record,
                       uint8_t* k_codes, uint16_t* k_scale, uint16_t* k_zero,
                       uint8_t* v_codes, uint16_t* v_scale, uint16_t* v_zero);
 
-/* Number of kernel launches one jfa_decode_step issues for a geometry
- * (for launch accounting); 0 on a bad geometry. */
+/* Number of kernel launches one jfa_decode_step issues for a geometry with
+ * q in device memory (for launch accounting; one more with q in pinned host
+ * memory); 0 on a bad geometry. */
 int jfa_decode_step_launches(const jfa_geom* geom, int32_t k);
 
 /* ---------------------------------------------------------------------------

@@ -64,7 +64,7 @@ def test_workspace_layout(lib):
     for L in (a, b):
         offs = [L.off_flag, L.off_scores, L.off_partials, L.off_mused, L.off_wts,
                 L.off_scan_hist, L.off_hist, L.off_cand, L.off_sel, L.off_fp4q, L.off_sparse,
-                L.off_ticket, L.off_bkeys, L.off_chan, L.total_bytes]
+                L.off_ticket, L.off_bkeys, L.off_chan, L.off_qstage, L.total_bytes]
         assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
         assert L.off_counters == L.off_hist + 4 * 4 * 2048
         assert L.off_scores + 4 * 4 * 4096 <= L.off_partials
