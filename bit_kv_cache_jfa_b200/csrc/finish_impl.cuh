@@ -55,13 +55,15 @@ struct FinPersist {
   uint32_t chtie[kTCap];              // chosen ties of the whole segment, ascending
   uint32_t n_sure, n_tie, overflow, n_gl;
 };
-// A partial (m, l, pad, pad, acc[128]) per query head: `run` holds this CTA's
-// exact-minus-removed terms (l may be negative), `sp` its share of the scan's
-// split partials.
+// Partials (m, l, pad, pad, acc[128]): `sp` per query head this CTA's share
+// of the scan's split partials; `recv` for the heads this CTA owns (j with
+// j mod C = rank) the C CTAs' partials of head j (their exact-minus-removed
+// terms together with their share of the scan's partials), slot
+// (j / C) C + source rank, written by the sources.
 template <int G>
 struct FinParts {
-  float run[G][kPartStride];
   float sp[G][kPartStride];
+  float recv[kFinMaxC > kMaxG ? kFinMaxC : kMaxG][kPartStride];
 };
 // Shared-memory histograms store bin b at hpad(b) = b + b/32, so threads
 // that each read a contiguous run of bins hit distinct banks.
@@ -534,6 +536,9 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const __grid_con
   __shared__ __align__(8) uint64_t s_early_bar;  // completion of the early copy below
 
   cg::cluster_group cl = cg::this_cluster();
+  // every CTA of the cluster has started once the matching wait returns:
+  // only then may a CTA store into another's shared memory
+  cluster_arrive_relaxed();
   const int C = (int)cl.num_blocks();
   const int r = (int)cl.block_rank();
   const int seg = blockIdx.x / C;
@@ -601,6 +606,7 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const __grid_con
 
   // ---- S1 + S2: bin b* from the scan's histogram, then this slice's lists
   bool hist_ok = false;
+  uint32_t base_s_out = 0, base_t_out = 0;  // the slice's sure and tie counts
   if (select) {
     // the slice's first 16 scores of this thread, loaded together with the
     // histogram window so both round trips overlap
@@ -703,10 +709,23 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const __grid_con
         base_t += tot & 0xFFFFu;
       }
     }
+    base_s_out = base_s;
+    base_t_out = base_t;
     if (tid == 0) {
       PS.n_sure = base_s;
       PS.n_tie = base_t;
       PS.overflow = (base_s > (uint32_t)kLCap || base_t > (uint32_t)kLCap) ? 1u : 0u;
+    }
+  }
+  cluster_wait();  // every CTA of the cluster has started
+  if (select && tid == 0) {
+    // this slice's counts into every CTA's shared memory (read after the
+    // barrier below)
+    const uint32_t ovf = (base_s_out > (uint32_t)kLCap || base_t_out > (uint32_t)kLCap) ? 1u : 0u;
+    for (int q = 0; q < C; ++q) {
+      cl.map_shared_rank(s_cnt, q)[r] = base_s_out;
+      cl.map_shared_rank(s_tie, q)[r] = base_t_out;
+      cl.map_shared_rank(s_ovf, q)[r] = ovf;
     }
   }
 
@@ -803,13 +822,6 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const __grid_con
       for (int i = 4 * (r * kFinThreads + tid); i < R * kScanHistStride; i += 4 * C * kFinThreads)
         *reinterpret_cast<uint4*>(hc + i) = make_uint4(0u, 0u, 0u, 0u);
     }
-    if (tid < C) {
-      const FinPersist* o = cl.map_shared_rank(&PS, tid);
-      s_cnt[tid] = o->n_sure;
-      s_tie[tid] = o->n_tie;
-      s_ovf[tid] = o->overflow;
-    }
-    __syncthreads();
     if (tid == 0) {
       uint32_t ps = 0, pt = 0, ovf = 0;
       for (int q = 0; q < C; ++q) {
@@ -982,8 +994,11 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const __grid_con
       *reinterpret_cast<uint4*>(hz + i) = make_uint4(0u, 0u, 0u, 0u);
   }
 
-  // ---- M1: the warps' partials into this CTA's partial P.run (per head the
-  // largest frame first, then every warp's terms scaled to it)
+  // ---- M1: this CTA's partial per head (the warps' exact-minus-removed
+  // terms, largest frame first, then every warp's terms scaled to it,
+  // together with the CTA's share of the scan's partials), stored straight
+  // into the shared memory of the head's owner, so that the merge after the
+  // barrier reads only local memory
   __syncthreads();  // the correction's shared memory is free
 #pragma unroll
   for (int h = 0; h < G; ++h) {
@@ -1012,80 +1027,45 @@ __global__ void __launch_bounds__(kFinThreads, 2) finish_kernel(const __grid_con
         l = fmaf(FM.w[w][h][1], f, l);
         a = fmaf(FM.w[w][h][4 + c], f, a);
       }
-      P.run[h][4 + c] = a;
+      // with the scan partials' share (m_a, l_a, a_a) in one frame; an empty
+      // part (no tokens, or l_a = 0) has weight 0
+      const float ma = P.sp[h][0], la = P.sp[h][1];
+      const float mt = la > 0.f ? fmaxf(m, ma) : m;
+      const float fc = m == -INFINITY ? 0.f : exp2f(m - mt);
+      const float fa = la > 0.f ? exp2f(ma - mt) : 0.f;
+      float* dst = cl.map_shared_rank(&P.recv[(h / C) * C + r][0], h % C);
+      dst[4 + c] = fmaf(a, fc, P.sp[h][4 + c] * fa);
       if (c == 0) {
-        P.run[h][0] = m;
-        P.run[h][1] = l;
+        dst[0] = mt;
+        dst[1] = fmaf(l, fc, la * fa);
       }
     }
   }
 
-  cl.sync();
+  cl.sync();  // every CTA's partials are in their owners' shared memory
 
-  // ---- M3: CTA r owns heads j = r, r + C, ...: merge the C CTAs' scan
-  // partials (m_a, l_a, a_a) and exact-minus-removed partials (m_c, l_c, a_c),
-  // remote loads issued together, and write
-  //   out = (a_c 2^(m_c-m) + a_a 2^(m_a-m)) / (l_c 2^(m_c-m) + l_a 2^(m_a-m))
+  // ---- M3: CTA r owns heads j = r, r + C, ...: merge the C partials (m_q,
+  // l_q, a_q) of head j and write out = sum a_q 2^(m_q-M) / sum l_q 2^(m_q-M),
+  // M the largest m_q.  Only local memory is read from here on, so no CTA
+  // waits for the others before it exits.
   for (int j = r; j < G; j += C) {
     const int c = tid;
-    if (c < kD && C > 8) {  // large clusters: frame first, then the sums (re-reading the frames)
-      float ma = -INFINITY, mc = -INFINITY;
+    if (c < kD) {
+      const float* base = &P.recv[(j / C) * C][0];
+      float M = -INFINITY;
 #pragma unroll 4
-      for (int q = 0; q < C; ++q) {
-        const FinParts<G>* o = cl.map_shared_rank(&P, q);
-        const float2 ha = *reinterpret_cast<const float2*>(&o->sp[j][0]);
-        const float2 hc = *reinterpret_cast<const float2*>(&o->run[j][0]);
-        if (ha.y > 0.f) ma = fmaxf(ma, ha.x);
-        mc = fmaxf(mc, hc.x);
-      }
-      const float m = fmaxf(ma, mc);
+      for (int q = 0; q < C; ++q) M = fmaxf(M, base[q * kPartStride]);
       float l = 0.f, acc = 0.f;
 #pragma unroll 4
       for (int q = 0; q < C; ++q) {
-        const FinParts<G>* o = cl.map_shared_rank(&P, q);
-        const float2 ha = *reinterpret_cast<const float2*>(&o->sp[j][0]);
-        const float2 hc = *reinterpret_cast<const float2*>(&o->run[j][0]);
-        const float fa = ha.y > 0.f ? exp2f(ha.x - m) : 0.f;
-        const float fc = hc.x == -INFINITY ? 0.f : exp2f(hc.x - m);
-        l = fmaf(ha.y, fa, fmaf(hc.y, fc, l));
-        acc = fmaf(o->sp[j][4 + c], fa, fmaf(o->run[j][4 + c], fc, acc));
+        const float mq = base[q * kPartStride];
+        const float f = mq == -INFINITY ? 0.f : exp2f(mq - M);
+        l = fmaf(base[q * kPartStride + 1], f, l);
+        acc = fmaf(base[q * kPartStride + 4 + c], f, acc);
       }
-      p.out[((size_t)bb * p.H + hh * G + j) * kD + c] = acc / l;
-    } else if (c < kD) {
-      float2 hd[8][2];
-      float av[8][2];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        if (q < C) {
-          FinParts<G>* o = cl.map_shared_rank(&P, q);
-          hd[q][0] = *reinterpret_cast<const float2*>(&o->sp[j][0]);
-          hd[q][1] = *reinterpret_cast<const float2*>(&o->run[j][0]);
-          av[q][0] = o->sp[j][4 + c];
-          av[q][1] = o->run[j][4 + c];
-        }
-      }
-      float ma = -INFINITY, mc = -INFINITY;
-#pragma unroll
-      for (int q = 0; q < 8; ++q)
-        if (q < C) {
-          if (hd[q][0].y > 0.f) ma = fmaxf(ma, hd[q][0].x);
-          mc = fmaxf(mc, hd[q][1].x);
-        }
-      const float m = fmaxf(ma, mc);
-      float l = 0.f, acc = 0.f;
-#pragma unroll
-      for (int q = 0; q < 8; ++q)
-        if (q < C) {
-          const float fa = hd[q][0].y > 0.f ? exp2f(hd[q][0].x - m) : 0.f;
-          const float fc = hd[q][1].x == -INFINITY ? 0.f : exp2f(hd[q][1].x - m);
-          l = fmaf(hd[q][0].y, fa, fmaf(hd[q][1].y, fc, l));
-          acc = fmaf(av[q][0], fa, fmaf(av[q][1], fc, acc));
-        }
       p.out[((size_t)bb * p.H + hh * G + j) * kD + c] = acc / l;
     }
   }
-  // keep this CTA's shared memory alive until every peer has read it
-  cl.sync();
 }
 
 template <int G, bool SEL, int KB, int VB>

@@ -306,6 +306,13 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
 // Programmatic dependent launch: wait for the preceding kernel of the stream
 // (its writes visible) / let the next kernel of the stream start launching.
 // Both are no-ops for a kernel launched without the PDL attribute.
+// Split cluster barrier: a relaxed arrive (orders no memory access) and the
+// wait for every thread of the cluster's arrive; between the two a thread
+// runs no other cluster barrier.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
