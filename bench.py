@@ -531,10 +531,11 @@ def per_config_line(args, dev, name: str, host: bool, n_blocks: int = 0) -> dict
         del st
         torch.cuda.empty_cache()
         return d
+    scan_ms = st.scan_ms(steps)
     step_ms = st.timed(st.step, steps, max(3, args.warmup))
     st.check_flag()
     d = {"workload": name, "exact_rows": "pinned_host" if host else "hbm", "steps": steps,
-         **st.summary(step_ms, st.scan_ms(steps))}
+         **st.summary(step_ms, scan_ms)}
     if host:
         # bytes the step gathers across the host link: the top-k rows of every
         # segment (the tail rows sit in the cache's device tail buffer)
@@ -872,6 +873,10 @@ def run_jfa(args, w):
     jfa.load()
 
     st = Setup(w, dev, args.host_resident)
+    # the scan kernel alone (the roofline object), before the step loop: in
+    # the same loop after the step loops some processes measured it ~35 %
+    # slower than inside the step, others not; that figure is reported too
+    scan_avg = st.scan_ms(args.steps)
     for i in range(max(3, args.warmup)):
         st.step(i)
     torch.cuda.synchronize()
@@ -897,7 +902,7 @@ def run_jfa(args, w):
 
     # the same steps as the three separate calls (scores, top-k, correct+merge)
     unfused_ms = st.timed(st.step3, args.steps, 3)
-    scan_avg = st.scan_ms(args.steps)
+    scan_after = st.scan_ms(args.steps)
 
     # end to end through the public API, two ways; every step takes q from
     # pinned host memory (the step's first kernel copies it across the host
@@ -973,7 +978,8 @@ def run_jfa(args, w):
                          "peak_kind": peak_kind, "unit": "GB/s", "frac": summ["scan_frac"],
                          "traffic": recorded_traffic(w.name),
                          "alg_bytes_per_launch": scan_alg_bytes(w),
-                         "us_per_launch": scan_avg * 1e3},
+                         "us_per_launch": scan_avg * 1e3,
+                         "us_per_launch_after_step_loops": scan_after * 1e3},
             "step_roofline": {"achieved": summ["step_frac"] * peak, "peak": peak, "unit": "GB/s",
                               "frac": summ["step_frac"], "alg_bytes_per_step": step_alg_bytes(w)},
             "cpu_baseline": cpu,

@@ -93,7 +93,10 @@ template <int G>
 constexpr size_t fin_union_bytes() {
   return sizeof(FinWork) > sizeof(FinMerge<G>) ? sizeof(FinWork) : sizeof(FinMerge<G>);
 }
-constexpr size_t kEarlyBytes = 24 * 1024;  // early copy of the scan partials' share
+// Early copy of the CTA's share of the scan partials: 77 (slot, head) rows,
+// enough for the shares of 32K-128K segments at G = 4 and G = 8 (larger
+// shares are staged a tile at a time); two CTAs per SM still fit at G = 8.
+constexpr size_t kEarlyBytes = 40 * 1024;
 template <int G>
 constexpr size_t fin_smem_bytes() {
   return sizeof(FinPersist) + sizeof(FinParts<G>) + (size_t)G * kD * sizeof(float) +
