@@ -449,13 +449,13 @@ int jfa_decode_finish(const jfa_geom* geom, const jfa_cache* cache, const uint16
 static int ragged_step(const jfa_geom* geom, const SeqTable& t, const jfa_cache* cache,
                        const uint16_t* q, float scale, int32_t k, int32_t* idx,
                        const uint16_t* k_exact, const uint16_t* v_exact, void* ws, float* out,
-                       cudaStream_t st, bool pdl_scan) {
+                       cudaStream_t st, bool defer_last) {
   jfa_workspace_layout L;
   workspace_layout(*geom, k, &L);
   uint8_t* w = static_cast<uint8_t*>(ws);
   const int sq = stage_query(*geom, &q, w, L, st);
   if (sq != JFA_OK) return sq;
-  const int s = launch_scores(*geom, t, *cache, q, scale, w, L, st, pdl_scan);
+  const int s = launch_scores(*geom, t, *cache, q, scale, w, L, st, true, defer_last);
   if (s != JFA_OK) return s;
   return launch_finish(*geom, t, *cache, q, scale, k, idx, nullptr, k_exact, v_exact, w, L, out, st);
 }
@@ -481,7 +481,7 @@ int jfa_decode_step_ragged(const jfa_geom* geom, const int32_t* seq_lens, const 
   SeqTable t;
   if (!fill_seq_table(*geom, seq_lens, &t)) return JFA_ERR_INVALID_ARG;
   return ragged_step(geom, t, cache, q, scale, k, idx, k_exact, v_exact, ws, out,
-                     static_cast<cudaStream_t>(stream), true);
+                     static_cast<cudaStream_t>(stream), false);
 }
 
 int jfa_append_decode_step(const jfa_geom* geom, const int32_t* seq_lens, const jfa_cache* cache,
@@ -507,9 +507,9 @@ int jfa_append_decode_step(const jfa_geom* geom, const int32_t* seq_lens, const 
   const int s = launch_append1(*geom, t, *cache, k_new, v_new, k_exact, v_exact,
                                reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + L.off_flag), st);
   if (s != JFA_OK) return s;
-  // the scan follows the kernel that may have written a record: plain stream
-  // order, so its first record copies start after that kernel has finished
-  return ragged_step(geom, t, cache, q, scale, k, idx, k_exact, v_exact, ws, out, st, false);
+  // the scan follows the kernel that may write each sequence's last group:
+  // that record is requested only after the scan's dependency wait
+  return ragged_step(geom, t, cache, q, scale, k, idx, k_exact, v_exact, ws, out, st, true);
 }
 
 int jfa_decode_step_launches(const jfa_geom* geom, int32_t k) {

@@ -85,11 +85,12 @@ int launch_append1(const jfa_geom& g, const SeqTable& t, const jfa_cache& c, con
                    const uint16_t* v_new, uint16_t* k_exact, uint16_t* v_exact, uint32_t* flag,
                    cudaStream_t st);
 // pdl: launch as a programmatic dependent of the previous kernel (its first
-// record copies may then start before that kernel has finished); false for a
-// scan right after a kernel that writes the packed records.
+// record copies may then start before that kernel has finished); defer_last:
+// the previous kernel may be writing each sequence's last group (the append
+// kernel), so that record is requested only after the dependency wait.
 int launch_scores(const jfa_geom& g, const SeqTable& t, const jfa_cache& c, const uint16_t* q,
                   float scale, uint8_t* ws, const jfa_workspace_layout& L, cudaStream_t st,
-                  bool pdl = true);
+                  bool pdl = true, bool defer_last = false);
 int launch_topk(const jfa_geom& g, int k, uint8_t* ws, const jfa_workspace_layout& L,
                 int32_t* idx, cudaStream_t st);
 int count_topk_launches(const jfa_geom& g, int k);

@@ -145,6 +145,14 @@ __global__ void __launch_bounds__(256) append1_kernel(const __grid_constant__ Ap
   const int n0 = p.seq.n_ctx[seg / p.hkv] - 1;  // the table holds the lengths after
   const int tl = n0 - split_point(n0);  // tail tokens before the append
   const bool flush = tl == kTail;        // n0 a positive multiple of 64
+  // Launched as a programmatic dependent: its CTAs are resident when the
+  // previous kernel ends, and everything below comes after the wait (the
+  // previous step's kernels read the tail slots and the exact copy; the new
+  // rows may come from the kernel just before).  The scan that follows may
+  // start at once: before its own wait it copies no record of a sequence's
+  // last group, the only record written here.
+  pdl_launch_dependents();
+  pdl_wait();
   if (flush) {
     const int g = n0 / kKG - 1;
     for (int i = tid; i < p.rec_bytes / 4; i += 256) rec[i] = 0u;
@@ -196,8 +204,9 @@ int launch_append1(const jfa_geom& g, const SeqTable& t, const jfa_cache& c, con
   p.val_bits = g.val_bits;
   p.rec_bytes = record_bytes(g.key_bits, g.val_bits);
   p.seq = t;
-  append1_kernel<<<dim3(g.batch * g.num_kv_heads), 256, 0, st>>>(p);
-  return cudaGetLastError() == cudaSuccess ? JFA_OK : JFA_ERR_CUDA;
+  return launch_pdl(append1_kernel, dim3(g.batch * g.num_kv_heads), dim3(256), 0, st, p) == cudaSuccess
+             ? JFA_OK
+             : JFA_ERR_CUDA;
 }
 
 // Tail update: copy new tokens [src0, n_new) to tail slots [dst0, ...).

@@ -49,6 +49,7 @@ struct ScanParams {
   int hkv, G, H, n_seg;
   int n_warps;
   int hist_reps;    // histogram copies per segment
+  int defer_last;   // request no record of a sequence's last group before the dependency wait
   float kappa;      // scale * log2(e): logits are kept in log2 units
   SeqTable seq;     // per-sequence lengths and group offsets
 };
@@ -142,12 +143,16 @@ __global__ void __launch_bounds__(ScanCfg<KB, VB, NT>::NW * 32, 1)
   // only the first stage now: every warp's first record is requested before
   // any second one, so the first records arrive sooner; the other stages
   // follow once the first has landed
-  if (lane == 0 && has_work) issue_next(0);
   // Only now wait for the previous kernel in the stream: the first record
   // copy reads the packed cache, which no kernel that releases this one
-  // early writes; the scores, histogram, partials and running maxima this
-  // kernel writes are read or cleared by the previous step's finishing kernel.
+  // early writes (the append kernel writes a sequence's last group: with
+  // defer_last that record is requested after the wait); the scores,
+  // histogram, partials and running maxima this kernel writes are read or
+  // cleared by the previous step's finishing kernel.
+  const bool early = has_work && !(p.defer_last && pf_g == pf_ng - 1);
+  if (lane == 0 && early) issue_next(0);
   pdl_wait();
+  if (lane == 0 && has_work && !early) issue_next(0);
 
   // lane roles: B column gid of n-tile n = (head (gid >> 1) + 4n, limb gid & 1);
   // logits of head tig + 4n; value columns (heads) 2 tig, 2 tig + 1
@@ -516,7 +521,7 @@ static int launch_scan_g(const ScanParams& sp, int n_ctas, bool pdl, cudaStream_
 
 int launch_scores(const jfa_geom& g, const SeqTable& t, const jfa_cache& c, const uint16_t* q,
                   float scale, uint8_t* ws, const jfa_workspace_layout& L, cudaStream_t st,
-                  bool pdl) {
+                  bool pdl, bool defer_last) {
   ScanPlan plan = scan_plan(g, t, num_sms_current());
   if (plan.total_groups == 0) return JFA_OK;
   ScanParams sp;
@@ -538,6 +543,7 @@ int launch_scores(const jfa_geom& g, const SeqTable& t, const jfa_cache& c, cons
   sp.H = g.num_heads;
   sp.n_warps = plan.n_warps;
   sp.hist_reps = scan_hist_reps(sp.n_seg);
+  sp.defer_last = defer_last ? 1 : 0;
   sp.kappa = scale * 1.4426950408889634f;
   if (g.key_bits == 3 && g.val_bits == 2) return launch_scan_g<3, 2>(sp, plan.n_ctas, pdl, st);
   if (g.key_bits == 4 && g.val_bits == 4) return launch_scan_g<4, 4>(sp, plan.n_ctas, pdl, st);
