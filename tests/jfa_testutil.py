@@ -28,7 +28,7 @@ def cap_for(ctx: int) -> int:
     return max(64, 64 * math.ceil(ctx / 64))
 
 
-class GpuRun:
+class DeviceRun:
     """One workload on the device: packed cache, exact copies, workspace."""
 
     def __init__(self, w: W.Workload, ctx: int | None = None, k: int | None = None,

@@ -11,7 +11,7 @@ import workloads as W
 from bit_kv_cache_jfa_b200 import _lib
 import bit_kv_cache_jfa_b200 as jfa
 
-from jfa_testutil import GpuRun, TIE_WINDOW, assert_out_close
+from jfa_testutil import DeviceRun, TIE_WINDOW, assert_out_close
 
 pytestmark = pytest.mark.gpu
 
@@ -29,7 +29,7 @@ def small(kb, vb, heads, kv, ctx, batch, k, planted=16, seed=0, lognormal=False)
 def test_topk_blocks_bit_exact_on_written_scores(ctx, n_blocks, mode):
     w = small(4, 4, 8, 4, ctx, 2, 64)
     zeros = torch.zeros(2, 4, ctx, 128, dtype=torch.bfloat16)
-    run = GpuRun(w, kv=(zeros, zeros))
+    run = DeviceRun(w, kv=(zeros, zeros))
     nq = run.cache.n_quant
     rng = np.random.default_rng(ctx + n_blocks)
     if mode == "normal":
@@ -68,7 +68,7 @@ def _block_sets_valid(idx, sel, n_blocks, window=TIE_WINDOW):
     (4, 2, 64, 8, 3000, 30, 2)])
 def test_block_step_against_oracle(kb, vb, heads, kv, ctx, n_blocks, batch):
     w = small(kb, vb, heads, kv, ctx, batch, 64, lognormal=True)
-    run = GpuRun(w)   # the block path takes its own idx; the workspace is sized for jfa_topk
+    run = DeviceRun(w)   # the block path takes its own idx; the workspace is sized for jfa_topk
     out, idx = jfa.decode_step_blocks(run.cache, run.q, n_blocks, run.k_exact, run.v_exact,
                                       run.ws, scale=run.scale)
     torch.cuda.synchronize()

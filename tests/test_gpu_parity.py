@@ -10,7 +10,7 @@ import workloads as W
 import bit_kv_cache_jfa_b200 as jfa
 from bit_kv_cache_jfa_b200 import _lib
 
-from jfa_testutil import (GpuRun, SCORE_ABS, assert_out_close, assert_topk_valid)
+from jfa_testutil import (DeviceRun, SCORE_ABS, assert_out_close, assert_topk_valid)
 
 pytestmark = pytest.mark.gpu
 
@@ -24,7 +24,7 @@ def small(kb=4, vb=4, heads=8, kv=2, ctx=4096, batch=1, topk=64, planted=16, see
                       value_lognormal=lognormal)
 
 
-def check_pack(run: GpuRun):
+def check_pack(run: DeviceRun):
     oc = run.oracle_cache()
     torch.cuda.synchronize()
     w = run.w
@@ -51,7 +51,7 @@ def check_pack(run: GpuRun):
 @pytest.mark.parametrize("kb,vb", [(4, 4), (3, 2), (3, 4), (4, 2)])
 def test_pack_bulk_bit_exact(kb, vb):
     w = small(kb, vb, ctx=1000, batch=2, lognormal=True)
-    check_pack(GpuRun(w))
+    check_pack(DeviceRun(w))
 
 
 def test_pack_appends_equal_bulk():
@@ -59,16 +59,16 @@ def test_pack_appends_equal_bulk():
     w = small(3, 2, ctx=777, batch=2)
     chunks = [1, 63, 1, 64, 65, 2, 1, 200, 127, 129, 64, 60]
     assert sum(chunks) == 777
-    check_pack(GpuRun(w, chunks=chunks))
+    check_pack(DeviceRun(w, chunks=chunks))
 
 
 def test_pack_single_token_appends():
     w = small(4, 4, ctx=200)
-    check_pack(GpuRun(w, chunks=[1] * 200))
+    check_pack(DeviceRun(w, chunks=[1] * 200))
 
 
 # ---------------------------------------------------------------- scores
-def scan_partials(run: GpuRun):
+def scan_partials(run: DeviceRun):
     """Merge the scan's split partials on the host (log2 units)."""
     g = run.cache.geom()
     w = run.w
@@ -102,7 +102,7 @@ def scan_partials(run: GpuRun):
                                             (4, 4, 32, 4), (3, 4, 8, 8), (4, 2, 4, 2)])
 def test_scores_and_scan_partials(kb, vb, heads, kv):
     w = small(kb, vb, heads=heads, kv=kv, ctx=2100, batch=2, lognormal=True)
-    run = GpuRun(w)
+    run = DeviceRun(w)
     run.scores()
     s_gpu = run.selection_scores()
     ref = run.oracle_step()
@@ -122,7 +122,7 @@ def test_scores_and_scan_partials(kb, vb, heads, kv):
 
 
 # ---------------------------------------------------------------- top-k
-def write_scores(run: GpuRun, s: np.ndarray):
+def write_scores(run: DeviceRun, s: np.ndarray):
     v = run.ws.scores(run.cache)
     v[:, :, :s.shape[2]] = torch.from_numpy(s.astype(np.float32)).cuda()
 
@@ -134,7 +134,7 @@ def write_scores(run: GpuRun, s: np.ndarray):
                                            (4096, 4031, "normal")])
 def test_topk_bit_exact_on_synthetic_scores(nq_ctx, k, mode):
     w = small(4, 4, ctx=nq_ctx, batch=2, heads=8, kv=4)
-    run = GpuRun(w, k=k, chunks=[nq_ctx], kv=(torch.zeros(2, 4, nq_ctx, 128, dtype=torch.bfloat16),
+    run = DeviceRun(w, k=k, chunks=[nq_ctx], kv=(torch.zeros(2, 4, nq_ctx, 128, dtype=torch.bfloat16),
                                               torch.zeros(2, 4, nq_ctx, 128, dtype=torch.bfloat16)))
     nq = run.cache.n_quant
     rng = np.random.default_rng(nq_ctx + k)
@@ -156,7 +156,7 @@ def test_topk_bit_exact_on_synthetic_scores(nq_ctx, k, mode):
 
 def test_topk_k_at_least_nq_fills():
     w = small(4, 4, ctx=300)
-    run = GpuRun(w, k=300)
+    run = DeviceRun(w, k=300)
     run.topk()
     got = run.idx.cpu().numpy()
     nq = run.cache.n_quant
@@ -169,7 +169,7 @@ def test_topk_k_at_least_nq_fills():
                                                   (4, 2, 4, 1, 777, 33)])
 def test_correct_merge_with_oracle_index_set(kb, vb, heads, kv, ctx, k):
     w = small(kb, vb, heads=heads, kv=kv, ctx=ctx, batch=2, topk=k, lognormal=True)
-    run = GpuRun(w)
+    run = DeviceRun(w)
     ref = run.oracle_step()
     run.scores()
     oidx = torch.from_numpy(ref.idx.astype(np.int32)).cuda()
@@ -181,7 +181,7 @@ def test_correct_merge_with_oracle_index_set(kb, vb, heads, kv, ctx, k):
 @pytest.mark.parametrize("wl", ["tiny_k4v4_4k"])
 def test_end_to_end_tiny_workload(wl):
     w = W.WORKLOADS[wl]
-    run = GpuRun(w)
+    run = DeviceRun(w)
     out, idx = run.step()
     ref = run.oracle_step()
     assert_topk_valid(idx, ref.select, w.topk)
@@ -199,7 +199,7 @@ def test_end_to_end_tiny_workload(wl):
 def test_end_to_end_no_planted(kb, vb, heads, kv, ctx, k, batch):
     # without planted tokens the bulk of the distribution carries the output
     w = small(kb, vb, heads=heads, kv=kv, ctx=ctx, batch=batch, topk=k, planted=0, seed=5)
-    run = GpuRun(w)
+    run = DeviceRun(w)
     out, idx = run.step()
     ref = run.oracle_step()
     assert_topk_valid(idx, ref.select, k)
@@ -209,8 +209,8 @@ def test_end_to_end_no_planted(kb, vb, heads, kv, ctx, k, batch):
 
 def test_host_resident_rows_match_device_rows():
     w = small(4, 4, heads=32, kv=8, ctx=3000, batch=2, topk=128)
-    a = GpuRun(w)
-    b = GpuRun(w, exact_on_host=True)
+    a = DeviceRun(w)
+    b = DeviceRun(w, exact_on_host=True)
     oa, ia = a.step()
     ob, ib = b.step()
     assert np.array_equal(ia, ib)
@@ -220,7 +220,7 @@ def test_host_resident_rows_match_device_rows():
 def test_output_in_pinned_host_memory():
     # the finishing kernel writes out straight into pinned host memory
     w = small(3, 2, heads=32, kv=8, ctx=3000, batch=2, topk=128)
-    run = GpuRun(w)
+    run = DeviceRun(w)
     od, idd = run.fused_step()
     out_h = torch.full(tuple(run.out.shape), float("nan"), dtype=torch.float32).pin_memory()
     idx = torch.empty_like(run.idx)
@@ -234,7 +234,7 @@ def test_output_in_pinned_host_memory():
 
 def test_decode_graph_replay_equals_eager_step():
     w = small(3, 2, heads=32, kv=8, ctx=5000, batch=2, topk=128)
-    run = GpuRun(w)
+    run = DeviceRun(w)
     od, idd = run.fused_step()
     q = run.q.clone()
     graph = jfa.DecodeGraph(run.cache, q, run.k, run.k_exact, run.v_exact, run.ws,
@@ -258,7 +258,7 @@ def test_decode_graph_replay_equals_eager_step():
 def test_bounded_wait_gives_up_and_the_context_stays_usable():
     # a wait that nothing completes ends after ~1 s with the timeout flag set
     w = small(3, 2, heads=8, kv=2, ctx=3000, batch=1, topk=64)
-    run = GpuRun(w)
+    run = DeviceRun(w)
     g = run.cache.geom()
     _lib.check(_lib.jfa_clear_error(g, run.ws.buf), "clear")
     _lib.check(_lib.jfa_selftest_bounded_wait(g, run.ws.buf), "selftest")
@@ -273,7 +273,7 @@ def test_bounded_wait_gives_up_and_the_context_stays_usable():
 @pytest.mark.parametrize("ctx", [1, 37, 64, 65, 127, 128, 129, 191])
 def test_short_contexts(ctx):
     w = small(3, 2, heads=8, kv=2, ctx=ctx, batch=2, topk=16, planted=0)
-    run = GpuRun(w)
+    run = DeviceRun(w)
     out, idx = run.step()
     ref = run.oracle_step()
     assert np.array_equal(idx, ref.idx)
@@ -282,7 +282,7 @@ def test_short_contexts(ctx):
 
 def test_k_at_least_nq_is_exact_attention():
     w = small(4, 4, heads=8, kv=2, ctx=700, batch=1, topk=700)
-    run = GpuRun(w)
+    run = DeviceRun(w)
     out, idx = run.step()
     ref = O.exact_attention(run.q_cpu.double().numpy(), run.k_cpu.double().numpy(),
                             run.v_cpu.double().numpy(), 700, run.scale)
@@ -291,7 +291,7 @@ def test_k_at_least_nq_is_exact_attention():
 
 def test_bad_index_sets_device_flag_without_fault():
     w = small(4, 4, ctx=600, topk=8)
-    run = GpuRun(w)
+    run = DeviceRun(w)
     run.scores()
     bad = torch.full((1, 2, 8), -1, dtype=torch.int32, device="cuda")
     bad[0, 0, 0] = 10_000_000
@@ -306,7 +306,7 @@ def test_bad_index_sets_device_flag_without_fault():
 
 def test_capacity_larger_than_context():
     w = small(3, 2, heads=32, kv=8, ctx=1500, batch=2, topk=100)
-    run = GpuRun(w, capacity=4096)
+    run = DeviceRun(w, capacity=4096)
     out, idx = run.step()
     ref = run.oracle_step()
     assert_topk_valid(idx, ref.select, 100)
@@ -320,7 +320,7 @@ def test_capacity_larger_than_context():
     (3, 2, 32, 8, 100, 16, 2), (4, 4, 8, 2, 64, 8, 1), (3, 2, 32, 8, 40000, 4096, 1)])
 def test_fused_step_matches_separate_calls(kb, vb, heads, kv, ctx, k, batch):
     w = small(kb, vb, heads=heads, kv=kv, ctx=ctx, batch=batch, topk=k, lognormal=True)
-    run = GpuRun(w)
+    run = DeviceRun(w)
     out3, idx3 = run.step()
     out1, idx1 = run.fused_step()
     assert np.array_equal(idx1, idx3)
@@ -335,7 +335,7 @@ def test_long_segments_sixteen_cta_clusters(kb, vb, heads, kv):
     # few segments of >= 16K quantized tokens: the finishing kernel runs
     # clusters of 16 CTAs; it must agree with the separate calls and the oracle
     w = small(kb, vb, heads=heads, kv=kv, ctx=20000, batch=1, topk=384, planted=32)
-    run = GpuRun(w)
+    run = DeviceRun(w)
     out3, idx3 = run.step()
     out1, idx1 = run.fused_step()
     assert np.array_equal(idx1, idx3)
@@ -346,7 +346,7 @@ def test_long_segments_sixteen_cta_clusters(kb, vb, heads, kv):
 
 def test_fused_step_tiny_workload_against_oracle():
     w = W.WORKLOADS["tiny_k4v4_4k"]
-    run = GpuRun(w)
+    run = DeviceRun(w)
     out, idx = run.fused_step()
     ref = run.oracle_step()
     assert_topk_valid(idx, ref.select, w.topk)
@@ -359,7 +359,7 @@ def test_whole_segment_fallback_selection():
     # whole segment from the stored scores (the fallback path); both choices
     # equal the bit-exact top-k of those scores
     w = small(3, 2, heads=32, kv=8, ctx=9000, batch=2, topk=256, lognormal=True)
-    run = GpuRun(w)
+    run = DeviceRun(w)
     run.scores()
     g, cs = run.cache.geom(), run.cache.struct()
     outs = []
@@ -389,7 +389,7 @@ def test_all_scores_tied_picks_lowest_indices(ctx, k):
     q = W.gen_q(w)
     kc = torch.full((1, 8, ctx, 128), 0.375, dtype=torch.bfloat16)
     vc = W.gen_kv(w, q, ctx)[1]
-    run = GpuRun(w, q=q, kv=(kc, vc))
+    run = DeviceRun(w, q=q, kv=(kc, vc))
     out, idx = run.fused_step()
     nq = run.cache.n_quant
     s_gpu = run.selection_scores()
