@@ -70,6 +70,21 @@ def test_workspace_layout(lib):
         assert L.off_scores + 4 * 4 * 4096 <= L.off_partials
 
 
+@pytest.mark.parametrize("batch,kv", [(1, 1), (1, 2), (1, 8), (2, 8), (3, 4), (4, 8), (8, 8),
+                                      (16, 4)])
+def test_workspace_histogram_copies_and_query_region(lib, batch, kv):
+    # the scan's histogram: 32768 bins + 32 words per copy, R copies per
+    # (sequence, KV head): 16 up to 2 segments, 32 / segments below 32, else 1
+    n_seg = batch * kv
+    reps = 1 if n_seg >= 32 else (16 if n_seg <= 2 else 32 // n_seg)
+    L = lib.jfa_workspace_layout_get(G(batch=batch, num_heads=4 * kv, num_kv_heads=kv), 64)
+    assert L.off_hist - L.off_scan_hist >= n_seg * reps * (32768 + 32) * 4
+    assert L.off_hist - L.off_scan_hist < n_seg * reps * (32768 + 32) * 4 + 256
+    # the staged query of a step given q in pinned host memory: bf16 [B][H][128]
+    assert L.total_bytes - L.off_qstage >= batch * 4 * kv * 128 * 2
+    assert L.off_qstage % 256 == 0
+
+
 @pytest.mark.parametrize("bad", [dict(head_dim=64), dict(num_heads=12, num_kv_heads=1),
                                  dict(num_heads=9), dict(capacity=100), dict(key_bits=2),
                                  dict(val_bits=3), dict(n_ctx=5000), dict(batch=0)])
