@@ -786,3 +786,58 @@ def test_one_bit_two_level_data_reconstructs_exactly():
     c = O.pack_cache(k, v, 266, 1, 1)
     assert np.array_equal(c.k_hat(), k[:, :, :256]) and np.array_equal(c.v_hat(), v[:, :, :256])
     assert np.array_equal(c.k_codes, bits) and np.array_equal(c.v_codes, vb.reshape(1, 2, 256, 128))
+
+
+# ---------------------------------------------------------------- directed fp16 rounding
+def _all_finite_fp16():
+    v = np.arange(65536, dtype=np.uint16).view(np.float16).astype(np.float64)
+    return np.unique(v[np.isfinite(v)])  # sorted, -0 and +0 merged
+
+
+@pytest.mark.filterwarnings("ignore:overflow encountered in nextafter")
+def test_fp16_directed_rounding_brackets_by_enumeration():
+    # the neighbours of x among all finite fp16 values, found by search in the
+    # enumerated table: round-down is the largest <= x, round-up the smallest >= x
+    table = _all_finite_fp16()
+    rng = np.random.default_rng(41)
+    x = np.concatenate([
+        rng.standard_normal(4000) * 10.0 ** rng.integers(-9, 5, 4000),  # subnormal .. 1e4
+        table[rng.integers(0, table.size, 500)],                          # exact fp16 values
+        (table[:-1] + np.diff(table) / 2)[rng.integers(0, table.size - 1, 500)],  # midpoints
+        [0.0, -0.0, 65504.0, -65504.0, 6.0e-8, -6.0e-8]])
+    down = O.fp16_round_down(x).astype(np.float64)
+    up = O.fp16_round_up(x).astype(np.float64)
+    i = np.searchsorted(table, x, side="right") - 1
+    j = np.searchsorted(table, x, side="left")
+    assert np.array_equal(down, table[i])
+    assert np.array_equal(up, table[j])
+    exact = np.isin(x, table)
+    assert np.array_equal(down[exact], x[exact]) and np.array_equal(up[exact], x[exact])
+
+
+def test_fp16_directed_rounding_rejects_nearest():
+    # nearest rounding is not a directed rounding: just above and just below
+    # an fp16 value the two differ from it
+    x = np.array([1.0 + 2.0 ** -12, 1.0 - 2.0 ** -13])
+    assert O.fp16_round_down(x)[0] == np.float16(1.0)
+    assert O.fp16_round_up(x)[0] == np.float16(1.0 + 2.0 ** -10)
+    assert O.fp16_round_down(x)[1] == np.float16(1.0 - 2.0 ** -11)
+    assert O.fp16_round_up(x)[1] == np.float16(1.0)
+
+
+# ---------------------------------------------------------------- NVFP4 keys per 64-token group
+def test_nvfp4_keys_quantize_each_64_token_group_on_its_own():
+    rng = np.random.default_rng(43)
+    # group g exactly representable with its own tensor scale 2^(-10 - g):
+    # the keys come back exactly only if each group gets its own fp32 scale
+    k = np.concatenate([_grid_block(rng, (64, 128), 448 * 2.0 ** (-10 - g)) for g in range(3)])
+    k = np.concatenate([k, rng.standard_normal((10, 128))])  # tokens past n_quant ignored
+    got = O.nvfp4_keys(k[None], 192)[0]
+    assert got.shape == (192, 128)
+    assert np.array_equal(got, k[:192])
+    # locality: a change inside group 1 leaves groups 0 and 2 unchanged
+    k2 = k.copy()
+    k2[70, 5] = 1e3
+    got2 = O.nvfp4_keys(k2[None], 192)[0]
+    assert np.array_equal(got2[:64], got[:64]) and np.array_equal(got2[128:], got[128:])
+    assert not np.array_equal(got2[64:128], got[64:128])
